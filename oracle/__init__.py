@@ -1,0 +1,177 @@
+"""CPU oracle for the routed 2-bit MoE FFN layer (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. The product path (the CUDA library and
+its binding) never touches it. The arithmetic lives in ``moeref.c``; this file
+only marshals numpy arrays into it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SO = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+F32, BF16 = 0, 1
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("hidden", "inter", "n_experts", "top_k", "shared_inter")]
+
+
+class Weights(ctypes.Structure):
+    _fields_ = [
+        (n, ctypes.c_void_p)
+        for n in (
+            "router_w", "router_bias", "gate_codes", "gate_d", "up_codes", "up_d",
+            "down_codes", "down_dd", "sh_gate", "sh_up", "sh_down",
+        )
+    ]
+
+
+def build(force: bool = False, openmp: bool = False) -> str:
+    """Compile the oracle: plain C99, -O2, no fast-math, no FMA contraction."""
+    src = os.path.join(_HERE, "moeref.c")
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(src):
+        cmd = ["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c99", "-fPIC", "-shared",
+               "-o", _SO, src, "-lm"]
+        subprocess.check_call(cmd)
+    return _SO
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_SO)
+        vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        L.moeref_f16_to_f64.restype = ctypes.c_double
+        L.moeref_f16_to_f64.argtypes = [ctypes.c_uint16]
+        L.moeref_bf16_to_f64.restype = ctypes.c_double
+        L.moeref_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        L.moeref_splitmix64_next.restype = ctypes.c_uint64
+        L.moeref_splitmix64_next.argtypes = [ctypes.POINTER(ctypes.c_uint64)]
+        L.moeref_grid.argtypes = [vp]
+        L.moeref_dequant_iq2.argtypes = [vp, vp, i64, vp]
+        L.moeref_dequant_q2k.argtypes = [vp, vp, i64, vp]
+        L.moeref_route.argtypes = [i32, i32, i32, vp, vp, vp, i32, i32, vp, vp, vp]
+        L.moeref_permute.argtypes = [i32, i32, i32, vp, vp, vp, vp]
+        L.moeref_expert_ffn.argtypes = [ctypes.POINTER(Desc), ctypes.POINTER(Weights), vp, i32, i32, vp, vp, vp, vp]
+        L.moeref_layer_forward.argtypes = [ctypes.POINTER(Desc), ctypes.POINTER(Weights), vp, i32, i32, vp, vp, vp, vp]
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    if a is None:
+        return None
+    assert isinstance(a, np.ndarray) and a.flags["C_CONTIGUOUS"], "arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dtype_code(x: np.ndarray) -> int:
+    if x.dtype == np.float32:
+        return F32
+    if x.dtype == np.uint16:
+        return BF16
+    raise TypeError("activations are fp32 or bf16 bit patterns (uint16)")
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise RuntimeError(f"oracle returned status {rc}")
+
+
+def splitmix64(state: int, n: int) -> list[int]:
+    s = ctypes.c_uint64(state)
+    return [int(lib().moeref_splitmix64_next(ctypes.byref(s))) for _ in range(n)]
+
+
+def grid() -> np.ndarray:
+    out = np.zeros((256, 8), np.uint8)
+    lib().moeref_grid(_p(out))
+    return out
+
+
+def f16_to_f64(h: int) -> float:
+    return float(lib().moeref_f16_to_f64(h))
+
+
+def dequant_iq2(codes: np.ndarray, d: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8).reshape(-1, 64)
+    d = np.ascontiguousarray(d, np.uint16).reshape(-1)
+    assert codes.shape[0] == d.shape[0]
+    out = np.zeros(codes.shape[0] * 256, np.float32)
+    lib().moeref_dequant_iq2(_p(codes), _p(d), codes.shape[0], _p(out))
+    return out
+
+
+def dequant_q2k(codes: np.ndarray, dd: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8).reshape(-1, 80)
+    dd = np.ascontiguousarray(dd, np.uint32).reshape(-1)
+    assert codes.shape[0] == dd.shape[0]
+    out = np.zeros(codes.shape[0] * 256, np.float32)
+    lib().moeref_dequant_q2k(_p(codes), _p(dd), codes.shape[0], _p(out))
+    return out
+
+
+def route(router_w, router_bias, x, k: int, want_logits: bool = False):
+    x = np.ascontiguousarray(x)
+    T, H = x.shape
+    E = router_w.shape[0]
+    idx = np.zeros((T, k), np.int32)
+    w = np.zeros((T, k), np.float32)
+    logits = np.zeros((T, E), np.float64) if want_logits else None
+    rb = None if router_bias is None else np.ascontiguousarray(router_bias, np.float32)
+    _check(lib().moeref_route(H, E, k, _p(np.ascontiguousarray(router_w)), _p(rb), _p(x), _dtype_code(x), T,
+                              _p(idx), _p(w), _p(logits)))
+    return (idx, w, logits) if want_logits else (idx, w)
+
+
+def permute(idx: np.ndarray, E: int):
+    idx = np.ascontiguousarray(idx, np.int32)
+    T, k = idx.shape
+    offsets = np.zeros(E + 1, np.int32)
+    perm = np.zeros(T * k, np.int32)
+    inv = np.zeros(T * k, np.int32)
+    _check(lib().moeref_permute(T, k, E, _p(idx), _p(offsets), _p(perm), _p(inv)))
+    return offsets, perm, inv
+
+
+def _structs(lw):
+    desc = Desc(lw.H, lw.I, lw.E, lw.k, lw.Is)
+    keep = [np.ascontiguousarray(a) if a is not None else None for a in (
+        lw.router_w, lw.router_bias, lw.gate_codes, lw.gate_d, lw.up_codes, lw.up_d,
+        lw.down_codes, lw.down_dd, lw.sh_gate, lw.sh_up, lw.sh_down)]
+    W = Weights(*[_p(a) for a in keep])
+    return desc, W, keep
+
+
+def expert_ffn(lw, x, idx, w, residual=None) -> np.ndarray:
+    x = np.ascontiguousarray(x)
+    T = x.shape[0]
+    desc, W, keep = _structs(lw)
+    y = np.zeros((T, lw.H), np.float32)
+    res = None if residual is None else np.ascontiguousarray(residual, np.float32)
+    _check(lib().moeref_expert_ffn(ctypes.byref(desc), ctypes.byref(W), _p(x), _dtype_code(x), T,
+                                   _p(np.ascontiguousarray(idx, np.int32)),
+                                   _p(np.ascontiguousarray(w, np.float32)), _p(res), _p(y)))
+    return y
+
+
+def layer_forward(lw, x, residual=None):
+    x = np.ascontiguousarray(x)
+    T = x.shape[0]
+    desc, W, keep = _structs(lw)
+    y = np.zeros((T, lw.H), np.float32)
+    idx = np.zeros((T, lw.k), np.int32)
+    w = np.zeros((T, lw.k), np.float32)
+    res = None if residual is None else np.ascontiguousarray(residual, np.float32)
+    _check(lib().moeref_layer_forward(ctypes.byref(desc), ctypes.byref(W), _p(x), _dtype_code(x), T,
+                                      _p(res), _p(y), _p(idx), _p(w)))
+    return y, idx, w
