@@ -1,0 +1,371 @@
+"""Benchmark of the routed 2-bit MoE FFN layer on B200.
+
+One step = one moe_layer_forward (router, top-k, permutation, routed expert
+FFNs, shared expert, combine) over one batch of synthetic tokens, with all
+inputs resident in HBM. Several layers with distinct weights are resident and
+used in rotation, so the bytes a step reads are not served from L2 (L2 is
+126 MB; one decode step touches ~190 MB and the rotation keeps >= 570 MB in
+flight between reuses).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode1|decode32|prefill|stack]
+                  [--impl ours|reference]
+
+Under torchrun each rank runs its own batches (weak scaling, no collective on
+the data path); the step time is the max over ranks. ``--impl reference``
+times the CPU oracle (the baseline arm) on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+HBM_FALLBACK_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="decode1", choices=["decode1", "decode32", "prefill", "stack"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=0, help="resident layers in rotation (0 = config default)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p.get("bf16_tflops", 0.0)), "measured"
+    except Exception:
+        return HBM_FALLBACK_GBS, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        self.path = None
+
+    def start(self):
+        try:
+            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------- bytes
+def expert_bytes(cfg) -> dict:
+    nb = cfg.I * cfg.H // 256
+    return {"gateup": 2 * nb * (64 + 2), "down": nb * (80 + 4), "shared": 3 * cfg.Is * cfg.H * 2,
+            "router": cfg.E * cfg.H * 2}
+
+
+def traffic_record(kernel: str):
+    """dram bytes per launch from a committed ncu summary, if its source hash
+    matches the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        rec = json.load(open(p)).get(kernel)
+        if not rec:
+            return None
+        src = os.path.join(ROOT, rec["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        return rec if h == rec["sha256"] else None
+    except Exception:
+        return None
+
+
+# --------------------------------------------------------------- reference
+def run_reference(args, cfg):
+    import oracle
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    oracle.build()
+    lw = synth.make_layer(cfg)
+    # per step: one token through the whole layer (router, k experts, shared)
+    x = synth.make_x_fast(cfg, max(args.steps + args.warmup, 1))
+    per_step_tokens = 1
+    for i in range(args.warmup):
+        oracle.layer_forward(lw, np.ascontiguousarray(x[i:i + 1]))
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        j = args.warmup + i
+        oracle.layer_forward(lw, np.ascontiguousarray(x[j:j + 1]))
+    dt = time.perf_counter() - t0
+    value = per_step_tokens * args.steps / dt
+    sample = f"{per_step_tokens} token per step through the full {cfg.name} layer (router, {cfg.k} experts, shared)"
+    line = {
+        "impl": "reference", "metric": "moe_layer_tokens_per_s", "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "tokens_per_step": per_step_tokens, "H": cfg.H, "I": cfg.I, "E": cfg.E,
+                   "k": cfg.k, "I_s": cfg.Is},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(cfg, budget_s=15.0):
+    import oracle
+
+    oracle.build()
+    lw = synth.make_layer(cfg)
+    x = synth.make_x_fast(cfg, 64)
+    n, t0 = 0, time.perf_counter()
+    while n < 64:
+        oracle.layer_forward(lw, np.ascontiguousarray(x[n:n + 1]))
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} tokens of the {cfg.name} layer one at a time, single-threaded C oracle ({dt:.1f} s)"}
+
+
+# -------------------------------------------------------------------- ours
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    from bit_quantized_routed_iq2_b200 import build as moebuild
+    from bit_quantized_routed_iq2_b200 import moe2bit
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    moebuild.build()
+    moe2bit.load()
+
+    n_layers = args.layers or {"decode1": 4, "decode32": 4, "prefill": 2, "stack": cfg.layers}[cfg.name]
+    T = cfg.T
+    layers = []
+    for l in range(n_layers):
+        lw = synth.make_layer(cfg, layer=l)
+        layers.append(moe2bit.to_device(lw))
+        del lw
+    n_slots = 4
+    xs_host = [synth.make_x_fast(cfg, T, layer=100 + s, cfg_seed=cfg.seed + 7919 * rank) for s in range(n_slots)]
+    xdt = torch.bfloat16 if cfg.x_dtype == "bf16" else torch.float32
+
+    def dev_x(a):
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
+        return t.view(torch.bfloat16) if a.dtype == np.uint16 else t
+
+    xs = [dev_x(a) for a in xs_host]
+    res = None
+    if cfg.name == "stack":
+        res = torch.from_numpy(synth.make_residual(cfg, T, cfg_seed=cfg.seed + rank)).cuda()
+    y = torch.empty((T, cfg.H), dtype=torch.float32, device="cuda")
+    ws = moe2bit.alloc_workspace(layers[0].desc, T)
+    stream = torch.cuda.current_stream()
+
+    if cfg.name == "stack":
+        # one step = 16-token decode through all resident layers chained by the residual stream
+        xa = torch.empty((T, cfg.H), dtype=torch.bfloat16, device="cuda")
+
+        def step(i):
+            cur = xs[i % n_slots]
+            for l, dl in enumerate(layers):
+                moe2bit.layer_forward(dl, cur, res if l == 0 else y, y, ws, stream)
+                xa.copy_(y)  # next layer input = bf16 of the residual stream
+                cur = xa
+        tokens_per_step = T
+    else:
+        def step(i):
+            moe2bit.layer_forward(layers[i % n_layers], xs[i % n_slots], None, y, ws, stream)
+        tokens_per_step = T
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+
+    # per-kernel durations (CUDA events around each library launch, same workload)
+    moe2bit.profile_enable(True)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    torch.cuda.synchronize()
+    prof = moe2bit.profile_read()
+    moe2bit.profile_enable(False)
+
+    # end to end through the public API with host buffers: pinned x -> device, layer, y -> pinned host
+    xh = [torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).pin_memory() for a in xs_host]
+    yh = torch.empty((T, cfg.H), dtype=torch.float32).pin_memory()
+    xd = torch.empty((T, cfg.H), dtype=torch.int16 if cfg.x_dtype == "bf16" else torch.float32, device="cuda")
+    xdv = xd.view(torch.bfloat16) if cfg.x_dtype == "bf16" else xd
+
+    def e2e_step(i):
+        xd.copy_(xh[i % n_slots], non_blocking=True)
+        if cfg.name == "stack":
+            cur = xdv
+            for l, dl in enumerate(layers):
+                moe2bit.layer_forward(dl, cur, res if l == 0 else y, y, ws, stream)
+                xa.copy_(y)
+                cur = xa
+        else:
+            moe2bit.layer_forward(layers[i % n_layers], xdv, None, y, ws, stream)
+        yh.copy_(y, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1) / args.steps
+    clocks = clk.stop()
+
+    mx = torch.tensor([ms, ms_e2e], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+    ms, ms_e2e = float(mx[0]), float(mx[1])
+
+    # realised active experts per step, from the library's own routing
+    act = []
+    for s in range(n_slots):
+        for l in range(min(n_layers, 4)):
+            dl = layers[l]
+            idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
+            w = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
+            off = torch.empty(cfg.E + 1, dtype=torch.int32, device="cuda")
+            perm = torch.empty(T * cfg.k, dtype=torch.int32, device="cuda")
+            inv = torch.empty(T * cfg.k, dtype=torch.int32, device="cuda")
+            moe2bit.route(dl.desc, dl.tensors["router_w"], dl.tensors["router_bias"], xs[s], idx, w, off, perm, inv, ws)
+            o = off.cpu().numpy()
+            act.append(int(np.count_nonzero(np.diff(o))))
+    n_active = float(np.mean(act))
+
+    hbm, bf16_tf, peak_kind = peaks()
+    eb = expert_bytes(cfg)
+    launches_per_step = {k: v[1] / args.steps for k, v in prof.items()}
+    avg_ms = {k: v[0] / max(v[1], 1) for k, v in prof.items()}
+    dom = max(prof, key=lambda k: prof[k][0])
+    if dom in ("gateup", "prefill_gateup"):
+        alg = n_active * eb["gateup"] + T * cfg.H * (2 if cfg.x_dtype == "bf16" else 4)
+    elif dom in ("down", "prefill_down"):
+        alg = n_active * eb["down"] + T * cfg.k * cfg.I * 4 + T * cfg.k * cfg.H * 4
+    elif dom in ("shared_gateup",):
+        alg = 2 * cfg.Is * cfg.H * 2
+    elif dom in ("shared_down",):
+        alg = cfg.Is * cfg.H * 2
+    else:
+        alg = 0
+    achieved = alg / (avg_ms[dom] * 1e-3) / 1e9 if alg else 0.0
+    tr = traffic_record(dom)
+    roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "peak_source": f"{peak_kind} hbm_gbs", "traffic": tr["bytes_per_launch"] if tr else None,
+            "algorithmic_bytes_per_launch": alg, "avg_launch_ms": avg_ms[dom]}
+    layer_bytes = n_active * (eb["gateup"] + eb["down"]) + eb["shared"] + eb["router"]
+    kernels_per_step = sum(launches_per_step.values()) * (n_layers if cfg.name == "stack" else 1) / (
+        n_layers if cfg.name == "stack" else 1)
+    bytes_x = T * cfg.H * (2 if cfg.x_dtype == "bf16" else 4)
+    line = {
+        "metric": "moe_layer_tokens_per_s", "value": tokens_per_step * world / (ms * 1e-3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8-codes/fp32-acc", "data": "synthetic",
+        "config": {"workload": cfg.name, "tokens_per_step": T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
+                   "I_s": cfg.Is, "x_dtype": cfg.x_dtype, "resident_layers": n_layers,
+                   "l2": f"inputs larger than L2: {n_layers} resident layers in rotation",
+                   "active_experts_per_layer": n_active, "layer_bytes_touched": layer_bytes},
+        "roofline": roof,
+        "layer_hbm_gbs": layer_bytes / (ms * 1e-3) / 1e9 if cfg.name != "stack" else None,
+        "kernels": {k: {"avg_ms": avg_ms[k], "launches_per_step": launches_per_step[k]} for k in prof},
+        "gpu_launches": int(round(sum(launches_per_step.values()) * args.steps)),
+        "clocks": clocks,
+        "e2e": {"value": tokens_per_step * world / (ms_e2e * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": bytes_x, "d2h_bytes_per_step": T * cfg.H * 4},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    cfg = synth.CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

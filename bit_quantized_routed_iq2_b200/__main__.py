@@ -1,0 +1,3 @@
+from .build import build
+
+print(build(force=True, verbose=False))

@@ -1,0 +1,49 @@
+// kernels.cuh - launchers shared between the translation units of the library.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+struct LayerShape {
+  int H, I, E, k, Is;
+};
+
+struct WeightPtrs {
+  const uint16_t* router_w;
+  const float* router_bias;
+  const uint8_t* gate_codes;
+  const uint16_t* gate_d;
+  const uint8_t* up_codes;
+  const uint16_t* up_d;
+  const uint8_t* down_codes;
+  const uint32_t* down_dd;
+  const uint16_t* sh_gate;
+  const uint16_t* sh_up;
+  const uint16_t* sh_down;
+};
+
+// Routing state produced by the router/permutation step (device pointers).
+struct Routing {
+  const float* topk_w;    // [T][k]
+  const int32_t* offsets; // [E+1]
+  const int32_t* perm;    // [T*k]
+  const int32_t* inv;     // [T*k]
+  const int32_t* active;  // [E+1]: compacted active experts, active[E] = count
+};
+
+int launch_route(const uint16_t* Wr, const float* bias, const void* x, int x_dtype, int T, int H, int E, int k,
+                 float* logits, int32_t* topk_idx, float* topk_w, int32_t* offsets, int32_t* perm, int32_t* inv,
+                 int32_t* active, cudaStream_t st);
+int launch_active_from_offsets(const int32_t* offsets, int E, int32_t* active, cudaStream_t st);
+
+// Workspace needed by the FFN stage for T tokens (bytes) and the launcher.
+size_t ffn_workspace_bytes(const LayerShape& s, int T);
+int launch_ffn(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
+               const float* residual, float* y, void* ws, cudaStream_t st);
+
+int launch_debug_dequant_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, float* out, cudaStream_t st);
+int launch_debug_dequant_q2k(const uint8_t* codes, const uint32_t* dd, int64_t nblocks, float* out,
+                             cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,227 @@
+/*
+ * moe2bit.h - C ABI of the routed 2-bit MoE FFN layer for NVIDIA B200 (sm_100a).
+ *
+ * One hot path: for each token, router logits -> top-k experts with
+ * renormalised weights -> per expert a SwiGLU FFN whose gate/up weights are in
+ * an IQ2_XXS-style 2-bit codebook format and whose down weights are in a
+ * Q2_K-style 2-bit format -> weighted combine plus an unquantized shared
+ * expert (plus an optional residual).
+ *
+ * Sources (the ds4 engine pages):
+ *   [Q] "ds4 : analyse pratique pour un usage documenté" (hysenlabs.com),
+ *       section « Support de modèles et choix de quantification »: only routed
+ *       MoE experts are quantized, up/gate in IQ2_XXS and down in Q2_K; shared
+ *       experts, projections and routing stay unquantized.
+ *   [W] "antirez/ds4 - Moteur local d'inférence DeepSeek V4 Flash pour Metal"
+ *       (news.hada.io), section « Poids du modèle »: the same split.
+ *   [R] "Un modèle de 284 milliards de paramètres tourne désormais sur un Mac
+ *       de 128 Go. Qui y perd ?" (tiblogics.com), section « Comment un modèle de
+ *       284 milliards de paramètres tient sur une seule machine »: a router picks
+ *       a few experts per token; routed experts hold most of the weights.
+ * The pages give no bit layout, no router function and no layer shapes; the
+ * layouts, the router function (softmax over the chosen top-k) and the
+ * numerics below are this library's specification.
+ *
+ * Conventions for every call:
+ *   - Pointers marked "device" must be device-accessible memory of the current
+ *     CUDA device; "host" pointers are ordinary host memory. All buffers are
+ *     owned by the caller. The library never allocates or frees device memory,
+ *     never synchronises, and only enqueues work on `stream`.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   - Argument and shape errors are detected on the host before anything is
+ *     enqueued and are returned as a status; nothing is launched in that case.
+ *     A failed launch returns MOE_ERR_CUDA (the CUDA error is left queryable by
+ *     cudaGetLastError). Faults in device code surface at the caller's next
+ *     synchronisation. No C++ exception crosses this interface.
+ *   - Supported shapes: hidden % 256 == 0; inter % 256 == 0 or 256 % inter == 0;
+ *     1 <= top_k <= min(n_experts, 16); 1 <= n_experts <= 1024;
+ *     shared_inter % 8 == 0 (0 = no shared expert); hidden <= 16384;
+ *     inter <= 16384; T >= 0 (T == 0 enqueues nothing and returns MOE_OK).
+ *     Anything else returns MOE_ERR_UNSUPPORTED_SHAPE.
+ *   - Device pointers must be 16-byte aligned (weights, activations, outputs,
+ *     workspace); otherwise MOE_ERR_INVALID_ARG.
+ */
+#ifndef MOE2BIT_H
+#define MOE2BIT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,         /* null pointer, misaligned pointer, bad dtype */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2,   /* shape outside the supported set above */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes < moe_workspace_size(...) */
+  MOE_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed */
+  MOE_ERR_TIMEOUT = 5              /* a bounded device-side wait gave up */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Layer shape. T (tokens) is passed per call. */
+typedef struct {
+  int32_t hidden;       /* H: model width, reduction length of gate/up */
+  int32_t inter;        /* I: routed expert intermediate width */
+  int32_t n_experts;    /* E: routed experts */
+  int32_t top_k;        /* k: experts per token */
+  int32_t shared_inter; /* I_s: shared expert intermediate width, 0 = none */
+} moe_layer_desc;
+
+/*
+ * Weights of one layer, all device pointers, read only.
+ *
+ * Routed expert planes (structure of arrays; blocks run along the reduction
+ * axis over the row-major flattened [rows][K] matrix of each expert, so for
+ * K < 256 one 256-weight block spans 256/K rows):
+ *
+ * IQ2-style (gate, up; matrix [I][H] per expert, K = H), per 256-weight block:
+ *   codes: 64 bytes. Sub-block s (weights 32s..32s+31) is bytes 8s..8s+7:
+ *          bytes 8s+j (j = 0..3) = codebook row of group j (weights 32s+8j..+7);
+ *          bytes 8s+4..8s+7 = little-endian u32 v with sign field sigma_j in
+ *          bits 7j..7j+6 (bit e set => element e negative, e = 0..6) and the
+ *          4-bit scale ls in bits 28..31; element 7 is negative iff
+ *          popcount(sigma_j) is odd.
+ *   d:     one IEEE fp16 per block.
+ *   value: w[32s + 8j + e] = d * (2*ls + 1) * grid[row][e] * sign_e / 8, where
+ *          grid is the library's 256 x 8 codebook over {8, 25, 43}: splitmix64
+ *          seeded 0x4951325F47524944, c = (next() >> 32) mod 6561, duplicates
+ *          rejected, 256 rows in acceptance order, element e = base-3 digit e of
+ *          c (least significant first) mapped 0->8, 1->25, 2->43.
+ *   plane shapes: codes [E][I*H/256][64] u8, d [E][I*H/256] u16.
+ *
+ * Q2K-style (down; matrix [H][I] per expert, K = I), per 256-weight block:
+ *   codes: 80 bytes. Byte s (0..15) = sub-block s (weights 16s..16s+15) scale
+ *          byte, sc = low nibble, m = high nibble. Byte 16+i holds weights
+ *          4i..4i+3, weight 4i+r in bits 2r..2r+1 (q = 0..3).
+ *   dd:    one u32 per block: fp16 d in bits 0..15, fp16 dmin in bits 16..31.
+ *   value: w = d * sc * q - dmin * m.
+ *   plane shapes: codes [E][H*I/256][80] u8, dd [E][H*I/256] u32.
+ *
+ * Router and shared expert (unquantized per [Q], [W]): bf16 bit patterns.
+ */
+typedef struct {
+  const uint16_t* router_w;    /* bf16 [E][H] */
+  const float* router_bias;    /* fp32 [E], or NULL; added to the logits */
+  const uint8_t* gate_codes;   /* IQ2-style codes [E][I*H/256][64] */
+  const uint16_t* gate_d;      /* fp16 [E][I*H/256] */
+  const uint8_t* up_codes;     /* IQ2-style codes [E][I*H/256][64] */
+  const uint16_t* up_d;        /* fp16 [E][I*H/256] */
+  const uint8_t* down_codes;   /* Q2K-style codes [E][H*I/256][80] */
+  const uint32_t* down_dd;     /* u32 [E][H*I/256] = fp16 d | fp16 dmin << 16 */
+  const uint16_t* sh_gate;     /* bf16 [I_s][H] (unused when I_s == 0) */
+  const uint16_t* sh_up;       /* bf16 [I_s][H] */
+  const uint16_t* sh_down;     /* bf16 [H][I_s] */
+} moe_layer_weights;
+
+/*
+ * Workspace bytes needed by moe_route / moe_expert_ffn / moe_layer_forward for
+ * any T <= max_tokens. Host only; touches no device. `bytes` is a host pointer.
+ */
+MOE_API moe_status moe_workspace_size(const moe_layer_desc* desc, int32_t max_tokens, size_t* bytes);
+
+/*
+ * Router and permutation ([R]: the router selects a few experts per token; [Q]:
+ * it is unquantized).
+ *   logits l[t][e] = sum_h x[t][h] * router_w[e][h] (+ router_bias[e]), fp32
+ *   accumulation of exact products;
+ *   topk_idx[t][j] = the k largest logits, j = 0 the largest, ties to the lower
+ *   expert index;
+ *   topk_w[t][j] = exp(l_j - l_0) / sum_i exp(l_i - l_0) over the chosen k
+ *   (softmax over all experts renormalised over the chosen ones);
+ *   assignment a = t*k + j; offsets[e] = number of assignments to experts < e
+ *   (offsets[E] = T*k); perm[offsets[e] + r] = the r-th smallest a routed to e;
+ *   inv[perm[p]] = p.
+ * x: device [T][H] in `x_dtype`. Outputs (device): topk_idx [T][k] i32,
+ * topk_w [T][k] f32, offsets [E+1] i32, perm [T*k] i32, inv [T*k] i32.
+ * ws: device workspace of ws_bytes >= moe_workspace_size(desc, T).
+ */
+MOE_API moe_status moe_route(const moe_layer_desc* desc, const uint16_t* router_w, const float* router_bias,
+                     const void* x, moe_dtype x_dtype, int32_t T, int32_t* topk_idx, float* topk_w,
+                     int32_t* offsets, int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Routed experts, shared expert and combine, given a routing (from moe_route
+ * or the caller's own; topk_w need not sum to one):
+ *   for each assignment a = t*k + j, with e the expert whose range
+ *   [offsets[e], offsets[e+1]) holds inv[a]:
+ *     g = Wg_e x_t, u = Wu_e x_t, h = silu(g) * u (silu(z) = z / (1 + e^-z)),
+ *     o_a = Wd_e h;
+ *   s_t = Wsd (silu(Wsg x_t) * (Wsu x_t))   (absent when I_s == 0);
+ *   y[t] = sum_{j ascending} topk_w[t][j] * o_{t*k+j} + s_t (+ residual[t]).
+ * Accumulation is fp32 (exact integer partial sums inside each 2-bit block);
+ * outputs are fp32 and are deterministic run to run.
+ * x: device [T][H]; residual: device fp32 [T][H] or NULL (may alias y);
+ * y: device fp32 [T][H].
+ */
+MOE_API moe_status moe_expert_ffn(const moe_layer_desc* desc, const moe_layer_weights* w, const void* x,
+                          moe_dtype x_dtype, int32_t T, const float* topk_w, const int32_t* offsets,
+                          const int32_t* perm, const int32_t* inv, const float* residual, float* y, void* ws,
+                          size_t ws_bytes, void* stream);
+
+/*
+ * The whole layer: moe_route then moe_expert_ffn, with the routing kept in the
+ * workspace. Same argument meanings as above.
+ */
+MOE_API moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights* w, const void* x,
+                             moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* Static, NUL-terminated name of a status code. */
+MOE_API const char* moe_status_string(moe_status s);
+
+/*
+ * Block-dequantisation unit exposed for testing: decodes `nblocks` consecutive
+ * 256-weight blocks to fp32 (device out [nblocks*256]). The result is exact:
+ * IQ2-style values have at most 22 significant bits and Q2K-style values are a
+ * single correctly rounded fp32 subtraction of two exact products.
+ */
+MOE_API moe_status moe_debug_dequant_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, float* out,
+                                 void* stream);
+MOE_API moe_status moe_debug_dequant_q2k(const uint8_t* codes, const uint32_t* dd, int64_t nblocks, float* out,
+                                 void* stream);
+
+/*
+ * Kernel timing, a profiling aid (off by default; not thread-safe). While
+ * enabled, every launch of the library records a pair of CUDA events on its
+ * stream around the kernel (ids below). moe_profile_read waits for the recorded
+ * events, writes per-kernel total milliseconds and launch counts into the host
+ * arrays (MOE_K_COUNT entries each) and clears the record. Enabling creates a
+ * fixed pool of events (no device memory); disabling destroys it.
+ */
+typedef enum {
+  MOE_K_ROUTER_LOGITS = 0,
+  MOE_K_TOPK = 1,
+  MOE_K_PERMUTE = 2,
+  MOE_K_ACTIVE = 3,
+  MOE_K_GATEUP = 4,
+  MOE_K_DOWN = 5,
+  MOE_K_SHARED_GATEUP = 6,
+  MOE_K_SHARED_DOWN = 7,
+  MOE_K_COMBINE = 8,
+  MOE_K_PREP = 9,
+  MOE_K_PREFILL_GATEUP = 10,
+  MOE_K_PREFILL_DOWN = 11,
+  MOE_K_COUNT = 16
+} moe_kernel_id;
+MOE_API moe_status moe_profile_enable(int32_t on);
+MOE_API moe_status moe_profile_read(float* total_ms, int32_t* launches);
+
+/* Host copy of the library's compiled-in 256 x 8 IQ2 codebook (row-major,
+ * values in {8, 25, 43}). `out` is a host pointer to 2048 bytes. */
+MOE_API void moe_debug_grid(uint8_t* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE2BIT_H */

@@ -1,0 +1,95 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+symbol the header declares, computes workspace sizes, rejects bad arguments
+before touching a device, and carries the same codebook as the oracle."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from bit_quantized_routed_iq2_b200 import build as moebuild
+from bit_quantized_routed_iq2_b200 import moe2bit
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    moebuild.build()
+    return moe2bit.load()
+
+
+def _header_symbols():
+    src = open(os.path.join(ROOT, "include", "moe2bit.h")).read()
+    return set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src))
+
+
+def test_header_declares_the_binding_exports():
+    assert _header_symbols() == set(moe2bit.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _header_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in moe2bit.STATUS.items():
+        assert moe2bit.status_string(code) == name
+
+
+def test_codebook_matches_oracle(lib):
+    # two independent implementations of the same generator definition
+    assert moe2bit.debug_grid() == oracle.grid().tobytes()
+
+
+DECODE = dict(H=7168, I=2048, E=256, k=8, Is=2048)
+
+
+def test_workspace_size_monotone(lib):
+    d = moe2bit.desc_of(**DECODE)
+    sizes = [moe2bit.workspace_size(d, T) for T in (0, 1, 2, 16, 32, 2048)]
+    assert all(a <= b for a, b in zip(sizes, sizes[1:]))
+    assert sizes[1] > 0
+
+
+@pytest.mark.parametrize(
+    "shape",
+    [dict(H=100, I=2048, E=256, k=8, Is=2048), dict(H=7168, I=300, E=256, k=8, Is=2048),
+     dict(H=7168, I=2048, E=4, k=8, Is=2048), dict(H=7168, I=2048, E=256, k=17, Is=2048),
+     dict(H=7168, I=2048, E=2048, k=8, Is=2048), dict(H=7168, I=2048, E=256, k=8, Is=4)],
+)
+def test_unsupported_shapes_rejected(lib, shape):
+    d = moe2bit.desc_of(**shape)
+    n = ctypes.c_size_t(0)
+    assert lib.moe_workspace_size(ctypes.byref(d), 4, ctypes.byref(n)) == 2
+
+
+def test_invalid_arguments_rejected_without_launch(lib):
+    d = moe2bit.desc_of(**DECODE)
+    w = moe2bit.Weights()
+    # null weights / activations: MOE_ERR_INVALID_ARG before any CUDA call
+    assert lib.moe_layer_forward(ctypes.byref(d), ctypes.byref(w), None, 1, 1, None, None, None, 0, None) == 1
+    assert lib.moe_layer_forward(ctypes.byref(d), None, None, 1, 1, None, None, None, 0, None) == 1
+    assert lib.moe_route(ctypes.byref(d), None, None, None, 1, 1, None, None, None, None, None, None, 0, None) == 1
+    # bad dtype
+    assert lib.moe_route(ctypes.byref(d), None, None, None, 7, 1, None, None, None, None, None, None, 0, None) == 1
+    # negative T
+    assert lib.moe_layer_forward(ctypes.byref(d), ctypes.byref(w), None, 1, -1, None, None, None, 0, None) == 1
+    # T == 0 is a no-op
+    assert lib.moe_layer_forward(ctypes.byref(d), ctypes.byref(w), None, 1, 0, None, None, None, 0, None) == 0
+    assert lib.moe_debug_dequant_iq2(None, None, 4, None, None) == 1
+    assert lib.moe_debug_dequant_q2k(None, None, -1, None, None) == 1
+
+
+def test_misaligned_and_small_workspace_rejected(lib):
+    d = moe2bit.desc_of(**DECODE)
+    fake = 1 << 40  # never dereferenced: validation fails first
+    w = moe2bit.Weights(*([fake] * 11))
+    need = moe2bit.workspace_size(d, 1)
+    # misaligned activation pointer
+    assert lib.moe_layer_forward(ctypes.byref(d), ctypes.byref(w), fake + 2, 1, 1, None, fake, fake, need, None) == 1
+    # workspace too small
+    assert lib.moe_layer_forward(ctypes.byref(d), ctypes.byref(w), fake, 1, 1, None, fake, fake, need - 1, None) == 3
