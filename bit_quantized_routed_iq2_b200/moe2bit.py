@@ -28,7 +28,9 @@ STATUS = {
 EXPORTS = (
     "moe_workspace_size", "moe_route", "moe_expert_ffn", "moe_layer_forward", "moe_status_string",
     "moe_debug_dequant_iq2", "moe_debug_dequant_q2k", "moe_debug_grid", "moe_profile_enable", "moe_profile_read",
+    "moe_layer_forward_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 32 << 20
 KERNEL_NAMES = ("router_logits", "topk", "permute", "active", "gateup", "down", "shared_gateup", "shared_down",
                 "combine", "prep", "prefill_gateup", "prefill_down")
 K_COUNT = 16
@@ -78,6 +80,7 @@ def load() -> ctypes.CDLL:
     L.moe_debug_dequant_q2k.argtypes = [vp, vp, i64, vp, vp]
     L.moe_debug_grid.argtypes = [vp]
     L.moe_debug_grid.restype = None
+    L.moe_layer_forward_noalloc.argtypes = [pd, pw, vp, i32, i32, vp, vp, vp]
     L.moe_profile_enable.argtypes = [i32]
     L.moe_profile_read.argtypes = [vp, vp]
     for name in EXPORTS:
@@ -220,6 +223,15 @@ def layer_forward(layer: DeviceLayer, x, residual, y, ws, stream=None):
     _check(load().moe_layer_forward(ctypes.byref(layer.desc), ctypes.byref(w), _ptr(x), _dtype_of(x), T,
                                     _ptr(residual), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
                                     _stream(stream)), "moe_layer_forward")
+
+
+def layer_forward_noalloc(layer: DeviceLayer, x, residual, y, stream=None):
+    """The whole layer with the library's own fixed scratch array (no workspace
+    argument); see moe_layer_forward_noalloc in include/moe2bit.h."""
+    T = x.shape[0]
+    w = layer.weights
+    _check(load().moe_layer_forward_noalloc(ctypes.byref(layer.desc), ctypes.byref(w), _ptr(x), _dtype_of(x), T,
+                                            _ptr(residual), _ptr(y), _stream(stream)), "moe_layer_forward_noalloc")
 
 
 def alloc_workspace(desc: Desc, max_tokens: int, device="cuda"):

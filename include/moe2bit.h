@@ -176,6 +176,31 @@ MOE_API moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer
                              moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws,
                              size_t ws_bytes, void* stream);
 
+/*
+ * The whole layer without any caller-provided scratch: same arguments and
+ * results as moe_layer_forward, minus `ws` / `ws_bytes`. (The ds4 pages have
+ * no counterpart of this call; it exists for callers of this library that
+ * cannot allocate device memory themselves, e.g. a plugin whose host engine
+ * hands out no workspace, or a serving loop that must not allocate after
+ * start-up because cudaMalloc may synchronise the device.)
+ *   - Scratch is a fixed device array of MOE_NOALLOC_SCRATCH_BYTES inside the
+ *     library, present on every GPU that loads the library until the process
+ *     exits. Calls whose workspace need (moe_workspace_size) exceeds it return
+ *     MOE_ERR_WORKSPACE_TOO_SMALL before anything is enqueued; the size covers
+ *     a 32-token decode batch at H=7168, I=2048, E=256, k=8, I_s=2048.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture. It allocates nothing, ever.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; the library clears whatever must start at zero itself. Calls
+ *     that overlap on the GPU (other streams, other host threads) race on the
+ *     array: serialise them.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+MOE_API moe_status moe_layer_forward_noalloc(const moe_layer_desc* desc, const moe_layer_weights* w,
+                                             const void* x, moe_dtype x_dtype, int32_t T, const float* residual,
+                                             float* y, void* stream);
+
 /* Static, NUL-terminated name of a status code. */
 MOE_API const char* moe_status_string(moe_status s);
 
