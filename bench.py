@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=0, help="resident layers in rotation (0 = config default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override the routed expert count (small cases for profiling; not a bench workload)")
     return ap.parse_args()
 
 
@@ -194,7 +196,7 @@ def run_ours(args, cfg):
     moebuild.build()
     moe2bit.load()
 
-    n_layers = args.layers or {"decode1": 4, "decode32": 4, "prefill": 2, "stack": cfg.layers}[cfg.name]
+    n_layers = args.layers or {"decode1": 4, "decode32": 4, "prefill": 2, "stack": cfg.layers}.get(cfg.name, 1)
     T = cfg.T
     layers = []
     for l in range(n_layers):
@@ -211,13 +213,13 @@ def run_ours(args, cfg):
 
     xs = [dev_x(a) for a in xs_host]
     res = None
-    if cfg.name == "stack":
+    if cfg.name.startswith("stack"):
         res = torch.from_numpy(synth.make_residual(cfg, T, cfg_seed=cfg.seed + rank)).cuda()
     y = torch.empty((T, cfg.H), dtype=torch.float32, device="cuda")
     ws = moe2bit.alloc_workspace(layers[0].desc, T)
     stream = torch.cuda.current_stream()
 
-    if cfg.name == "stack":
+    if cfg.name.startswith("stack"):
         # one step = 16-token decode through all resident layers chained by the residual stream
         xa = torch.empty((T, cfg.H), dtype=torch.bfloat16, device="cuda")
 
@@ -268,7 +270,7 @@ def run_ours(args, cfg):
 
     def e2e_step(i):
         xd.copy_(xh[i % n_slots], non_blocking=True)
-        if cfg.name == "stack":
+        if cfg.name.startswith("stack"):
             cur = xdv
             for l, dl in enumerate(layers):
                 moe2bit.layer_forward(dl, cur, res if l == 0 else y, y, ws, stream)
@@ -361,6 +363,8 @@ def run_ours(args, cfg):
 def main():
     args = parse()
     cfg = synth.CONFIGS[args.config]
+    if args.experts:
+        cfg = synth.Config(**{**cfg.__dict__, "E": args.experts, "name": f"{cfg.name}_E{args.experts}"})
     if args.impl == "reference":
         run_reference(args, cfg)
     else:

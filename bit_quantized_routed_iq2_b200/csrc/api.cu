@@ -35,6 +35,7 @@ LayerShape shape_of(const moe_layer_desc* d) {
 
 // Routing part of the workspace.
 struct RouteWs {
+  int* status;  // device status word (MOE_ERR_TIMEOUT from a bounded wait), cleared by each call
   float* logits;
   int32_t* topk_idx;
   float* topk_w;
@@ -56,6 +57,7 @@ RouteWs carve(const moe_layer_desc* d, int32_t T, void* base) {
     off += align_up(bytes > 0 ? bytes : 1, 256);
     return q;
   };
+  w.status = reinterpret_cast<int*>(take(16));
   w.logits = reinterpret_cast<float*>(take(static_cast<size_t>(T) * E * 4));
   w.topk_idx = reinterpret_cast<int32_t*>(take(nA * 4));
   w.topk_w = reinterpret_cast<float*>(take(nA * 4));
@@ -155,7 +157,8 @@ moe_status moe_expert_ffn(const moe_layer_desc* desc, const moe_layer_weights* w
   int rc = launch_active_from_offsets(offsets, desc->n_experts, w.active, s);
   if (rc != OK) return to_status(rc);
   Routing r{topk_w, offsets, perm, inv, w.active};
-  return to_status(launch_ffn(shape_of(desc), weights_of(weights), x, x_dtype, T, r, residual, y, w.ffn, s));
+  return to_status(
+      launch_ffn(shape_of(desc), weights_of(weights), x, x_dtype, T, r, residual, y, w.ffn, w.status, s));
 }
 
 moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights* weights, const void* x,
@@ -180,7 +183,8 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights
                         desc->top_k, w.logits, w.topk_idx, w.topk_w, w.offsets, w.perm, w.inv, w.active, s);
   if (rc != OK) return to_status(rc);
   Routing r{w.topk_w, w.offsets, w.perm, w.inv, w.active};
-  return to_status(launch_ffn(shape_of(desc), weights_of(weights), x, x_dtype, T, r, residual, y, w.ffn, s));
+  return to_status(
+      launch_ffn(shape_of(desc), weights_of(weights), x, x_dtype, T, r, residual, y, w.ffn, w.status, s));
 }
 
 moe_status moe_debug_dequant_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, float* out,

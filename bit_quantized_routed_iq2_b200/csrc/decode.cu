@@ -1,0 +1,386 @@
+// decode.cu - the routed-expert FFN path built on int8 warp MMAs: activation
+// digits, the gate/up and down dequant-GEMVs (gateup.cu, down.cu), the
+// unquantized shared expert and the weighted combine.
+//
+// Sources: "ds4 : analyse pratique pour un usage documenté", section « Support de
+// modèles et choix de quantification » (routed experts in 2-bit: up/gate IQ2_XXS,
+// down Q2_K; shared experts unquantized) and "Un modèle de 284 milliards de
+// paramètres tourne désormais sur un Mac de 128 Go. Qui y perd ?", section
+// « Comment un modèle de 284 milliards de paramètres tient sur une seule
+// machine » (the routed experts hold most of the bytes, so decode is bound by
+// HBM bandwidth).
+#include <algorithm>
+
+#include "decode.cuh"
+#include "kernels.cuh"
+#include "profile.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+// x [T][H] -> xd [T][2][H] int8 digits (plane 0 hi, plane 1 lo) and
+// xs [T][H/256] = 2^s / 8 per 256-element block (the 1/8 of the IQ2 scale is
+// folded in). One warp per 256-element block, 8 elements per lane. Block (0,0)
+// also clears the call's device status word.
+template <typename XT>
+__global__ void __launch_bounds__(256) x_digits_kernel(const XT* __restrict__ x, int T, int H,
+                                                       int8_t* __restrict__ xd, float* __restrict__ xs,
+                                                       int* __restrict__ err_word) {
+  if (err_word && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *err_word = 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x;
+  const int blk = blockIdx.y * 8 + warp;
+  if (t >= T || blk * 256 >= H) return;
+  const size_t base = static_cast<size_t>(t) * H + blk * 256 + lane * 8;
+  float v[8];
+  if constexpr (sizeof(XT) == 4) {
+    const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + base);
+    const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + base + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    const uint4 a = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(x) + base);
+    v[0] = __uint_as_float(a.x << 16); v[1] = __uint_as_float(a.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(a.y << 16); v[3] = __uint_as_float(a.y & 0xFFFF0000u);
+    v[4] = __uint_as_float(a.z << 16); v[5] = __uint_as_float(a.z & 0xFFFF0000u);
+    v[6] = __uint_as_float(a.w << 16); v[7] = __uint_as_float(a.w & 0xFFFF0000u);
+  }
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const int s = m > 0.f ? floor_log2_pos(m) - 11 : 0;
+  uint32_t hw[2] = {0, 0}, lw[2] = {0, 0};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int hi = 0, lo = 0;
+    if (m > 0.f) split_digits(v[i], s, hi, lo);
+    hw[i / 4] |= (static_cast<uint32_t>(hi) & 0xFFu) << (8 * (i % 4));
+    lw[i / 4] |= (static_cast<uint32_t>(lo) & 0xFFu) << (8 * (i % 4));
+  }
+  int8_t* row = xd + static_cast<size_t>(t) * 2 * H + blk * 256 + lane * 8;
+  *reinterpret_cast<uint2*>(row) = make_uint2(hw[0], hw[1]);
+  *reinterpret_cast<uint2*>(row + H) = make_uint2(lw[0], lw[1]);
+  if (lane == 0) xs[static_cast<size_t>(t) * (H / 256) + blk] = m > 0.f ? ldexpf(1.0f, s - 3) : 0.f;
+}
+
+// ------------------------------------------------------------ shared expert
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 w, float (&f)[8]) {
+  f[0] = __uint_as_float(w.x << 16); f[1] = __uint_as_float(w.x & 0xFFFF0000u);
+  f[2] = __uint_as_float(w.y << 16); f[3] = __uint_as_float(w.y & 0xFFFF0000u);
+  f[4] = __uint_as_float(w.z << 16); f[5] = __uint_as_float(w.z & 0xFFFF0000u);
+  f[6] = __uint_as_float(w.w << 16); f[7] = __uint_as_float(w.w & 0xFFFF0000u);
+}
+
+// hs[t][r] = silu(Wsg x_t)[r] * (Wsu x_t)[r] with bf16 weights: one warp per row
+// pair (gate r, up r); activations staged in shared memory (fp32) in chunks of
+// 2048; each lane keeps four 16-byte weight loads of each matrix in flight.
+template <typename XT, int TMAX>
+__global__ void __launch_bounds__(256) shared_gateup_kernel(int H, int Is, const uint16_t* __restrict__ sg,
+                                                            const uint16_t* __restrict__ su,
+                                                            const XT* __restrict__ x, int T,
+                                                            float* __restrict__ hs) {
+  constexpr int CH = 2048;
+  __shared__ __align__(16) float xs[TMAX][CH];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;
+  for (int t0 = 0; t0 < T; t0 += TMAX) {
+    const int nt = min(TMAX, T - t0);
+    float ag[TMAX], au[TMAX];
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) ag[t] = au[t] = 0.f;
+    for (int c0 = 0; c0 < H; c0 += CH) {
+      __syncthreads();
+      for (int i = threadIdx.x; i < TMAX * CH; i += 256) {
+        const int t = i / CH, c = i % CH;
+        float v = 0.f;
+        if (t < nt && c0 + c < H) {
+          const size_t idx = static_cast<size_t>(t0 + t) * H + c0 + c;
+          if constexpr (sizeof(XT) == 4) v = reinterpret_cast<const float*>(x)[idx];
+          else v = bf16_bits_to_float(reinterpret_cast<const uint16_t*>(x)[idx]);
+        }
+        xs[t][c] = v;
+      }
+      __syncthreads();
+      if (row < Is) {
+        const int lim = min(CH, H - c0);
+        for (int cb = lane * 8; cb < lim; cb += 4 * 256) {
+          uint4 wg[4], wu[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int c = cb + j * 256;
+            if (c < lim) {
+              wg[j] = *reinterpret_cast<const uint4*>(sg + static_cast<size_t>(row) * H + c0 + c);
+              wu[j] = *reinterpret_cast<const uint4*>(su + static_cast<size_t>(row) * H + c0 + c);
+            } else {
+              wg[j] = wu[j] = make_uint4(0u, 0u, 0u, 0u);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int c = cb + j * 256;
+            if (c >= lim) break;
+            float g8[8], u8[8];
+            bf16x8_to_f32(wg[j], g8);
+            bf16x8_to_f32(wu[j], u8);
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t) {
+              if (t >= nt) break;
+              const float4 xa = *reinterpret_cast<const float4*>(&xs[t][c]);
+              const float4 xb = *reinterpret_cast<const float4*>(&xs[t][c + 4]);
+              const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                ag[t] = fmaf(g8[i], xv[i], ag[t]);
+                au[t] = fmaf(u8[i], xv[i], au[t]);
+              }
+            }
+          }
+        }
+      }
+    }
+    if (row < Is) {
+#pragma unroll
+      for (int t = 0; t < TMAX; ++t) {
+        float gg = ag[t], uu = au[t];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          gg += __shfl_xor_sync(0xffffffffu, gg, o);
+          uu += __shfl_xor_sync(0xffffffffu, uu, o);
+        }
+        if (lane == 0 && t < nt) hs[static_cast<size_t>(t0 + t) * Is + row] = silu_mul(gg, uu);
+      }
+    }
+  }
+}
+
+// y[t][r] = sum_j w[t][j] o[inv[t*k+j]][r] (j ascending) + (Wsd hs_t)[r] + residual[t][r].
+// One warp per output row r, all tokens; the row's weights are loaded up front.
+template <int TMAX>
+__global__ void __launch_bounds__(256) shared_down_combine_kernel(int H, int Is, int k, const uint16_t* __restrict__ sd,
+                                                                  const float* __restrict__ hs, int T,
+                                                                  const float* __restrict__ topk_w,
+                                                                  const int32_t* __restrict__ inv,
+                                                                  const float* __restrict__ obuf,
+                                                                  const float* residual, float* y) {
+  constexpr int WMAX = 8;  // 16-byte weight loads per lane kept in registers (Is <= 2048)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= H) return;
+  const int nw = (Is + 255) / 256;
+  uint4 wv[WMAX];
+  const bool in_regs = nw <= WMAX;
+  if (in_regs) {
+#pragma unroll
+    for (int j = 0; j < WMAX; ++j) {
+      const int c = lane * 8 + j * 256;
+      wv[j] = (j < nw && c < Is) ? *reinterpret_cast<const uint4*>(sd + static_cast<size_t>(row) * Is + c)
+                                 : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  for (int t0 = 0; t0 < T; t0 += TMAX) {
+    const int nt = min(TMAX, T - t0);
+    float acc[TMAX];
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) acc[t] = 0.f;
+    auto dot8 = [&](const uint4 w, int c) {
+      float w8[8];
+      bf16x8_to_f32(w, w8);
+#pragma unroll
+      for (int t = 0; t < TMAX; ++t) {
+        if (t >= nt) break;
+        const float4 ha = *reinterpret_cast<const float4*>(hs + static_cast<size_t>(t0 + t) * Is + c);
+        const float4 hb = *reinterpret_cast<const float4*>(hs + static_cast<size_t>(t0 + t) * Is + c + 4);
+        float s = acc[t];
+        s = fmaf(w8[0], ha.x, s); s = fmaf(w8[1], ha.y, s); s = fmaf(w8[2], ha.z, s); s = fmaf(w8[3], ha.w, s);
+        s = fmaf(w8[4], hb.x, s); s = fmaf(w8[5], hb.y, s); s = fmaf(w8[6], hb.z, s); s = fmaf(w8[7], hb.w, s);
+        acc[t] = s;
+      }
+    };
+    if (in_regs) {
+#pragma unroll
+      for (int j = 0; j < WMAX; ++j) {
+        const int c = lane * 8 + j * 256;
+        if (j >= nw || c >= Is) break;
+        dot8(wv[j], c);
+      }
+    } else {
+      for (int c = lane * 8; c < Is; c += 256)
+        dot8(*reinterpret_cast<const uint4*>(sd + static_cast<size_t>(row) * Is + c), c);
+    }
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) {
+      float s = acc[t];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      acc[t] = s;
+    }
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) {
+      if (lane == t && t < nt) {
+        const int tt = t0 + t;
+        float v = 0.f;
+        for (int j = 0; j < k; ++j) {
+          const int aidx = tt * k + j;
+          v = fmaf(topk_w[aidx], obuf[static_cast<size_t>(inv[aidx]) * H + row], v);
+        }
+        v += acc[t];
+        if (residual) v += residual[static_cast<size_t>(tt) * H + row];
+        y[static_cast<size_t>(tt) * H + row] = v;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------ launcher
+namespace {
+int num_sms() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  return sms;
+}
+}  // namespace
+
+bool fast_path_supported(const LayerShape& s) { return s.I % 256 == 0 && s.H % 256 == 0; }
+
+namespace {
+int hsc_stride(int I) { return ((I / 256) + 3) & ~3; }
+}  // namespace
+
+// h = silu(g) * u for one assignment (blockIdx.x), split into int8 digits with
+// one power-of-two scale per 256-element block, stored in the order the down
+// MMA reads them: inside each 32-element block, element j of sub-block half
+// sub (0 for the first 16, 1 for the next) goes to byte 8*(j%4) + 4*sub + j/4.
+// Also writes, per 16-element sub-block, the exact integer sum of the digits'
+// values q = 128 hi + lo (the min term of the Q2K-style down projection).
+__global__ void __launch_bounds__(256) hquant_kernel(int I, const float* __restrict__ gu, int8_t* __restrict__ hd,
+                                                     float* __restrict__ hsc, int32_t* __restrict__ hq, int hss) {
+  const int p = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float* g = gu + static_cast<size_t>(p) * 2 * I;
+  const float* u = g + I;
+  for (int sb = warp; sb < I / 256; sb += 8) {
+    const int base = sb * 256 + lane * 8;
+    const float4 g0 = *reinterpret_cast<const float4*>(g + base), g1 = *reinterpret_cast<const float4*>(g + base + 4);
+    const float4 u0 = *reinterpret_cast<const float4*>(u + base), u1 = *reinterpret_cast<const float4*>(u + base + 4);
+    const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+    const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    float h[8], m = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      h[i] = silu_mul(gv[i], uv[i]);
+      m = fmaxf(m, fabsf(h[i]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const int e = m > 0.f ? floor_log2_pos(m) - 11 : 0;
+    int qs = 0;
+    int8_t* hi_row = hd + static_cast<size_t>(p) * 2 * I;
+    int8_t* lo_row = hi_row + I;
+    const int blk32 = base >> 5, jj0 = base & 31;  // this lane's 8 elements sit in one 32-block
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      int hi = 0, lo = 0;
+      if (m > 0.f) split_digits(h[i], e, hi, lo);
+      qs += hi * 128 + lo;
+      const int jj = jj0 + i, sub = jj >> 4, j = jj & 15;
+      const int pos = blk32 * 32 + 8 * (j & 3) + 4 * sub + (j >> 2);
+      hi_row[pos] = static_cast<int8_t>(hi);
+      lo_row[pos] = static_cast<int8_t>(lo);
+    }
+    qs += __shfl_xor_sync(0xffffffffu, qs, 1);  // lanes 2i, 2i+1 hold one 16-element sub-block
+    if ((lane & 1) == 0) hq[static_cast<size_t>(p) * (I / 16) + sb * 16 + (lane >> 1)] = qs;
+    if (lane == 0) hsc[static_cast<size_t>(p) * hss + sb] = m > 0.f ? ldexpf(1.0f, e) : 0.f;
+  }
+}
+
+size_t fast_ffn_workspace_bytes(const LayerShape& s, int T) {
+  const size_t nA = static_cast<size_t>(T) * s.k;
+  size_t b = 0;
+  b += align_up(static_cast<size_t>(T) * 2 * s.H, 256);           // xd
+  b += align_up(static_cast<size_t>(T) * (s.H / 256) * 4, 256);   // xs
+  b += align_up(nA * 2 * s.I * 4, 256);                           // gu
+  b += align_up(nA * 2 * s.I, 256);                               // hd
+  b += align_up(nA * hsc_stride(s.I) * 4, 256);                   // hsc
+  b += align_up(nA * (s.I / 16) * 4, 256);                        // hq
+  b += align_up(nA * s.H * 4, 256);                               // o
+  b += align_up(static_cast<size_t>(T) * (s.Is > 0 ? s.Is : 1) * 4, 256);  // shared h
+  return b;
+}
+
+int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
+                    const float* residual, float* y, void* ws, int* err, cudaStream_t st) {
+  const size_t nA = static_cast<size_t>(T) * s.k;
+  char* p = static_cast<char*>(ws);
+  auto take = [&](size_t bytes) {
+    char* q = p;
+    p += align_up(bytes, 256);
+    return q;
+  };
+  int8_t* xd = reinterpret_cast<int8_t*>(take(static_cast<size_t>(T) * 2 * s.H));
+  float* xs = reinterpret_cast<float*>(take(static_cast<size_t>(T) * (s.H / 256) * 4));
+  float* gu = reinterpret_cast<float*>(take(nA * 2 * s.I * 4));
+  int8_t* hd = reinterpret_cast<int8_t*>(take(nA * 2 * s.I));
+  float* hsc = reinterpret_cast<float*>(take(nA * hsc_stride(s.I) * 4));
+  int32_t* hq = reinterpret_cast<int32_t*>(take(nA * (s.I / 16) * 4));
+  float* obuf = reinterpret_cast<float*>(take(nA * s.H * 4));
+  float* hsh = reinterpret_cast<float*>(take(static_cast<size_t>(T) * (s.Is > 0 ? s.Is : 1) * 4));
+
+  const int sms = num_sms();
+  const int slots = static_cast<int>(std::min<size_t>(nA, static_cast<size_t>(s.E)));
+  int rc = OK;
+  {
+    ProfScope ps(MOE_K_PREP, st);
+    dim3 g(T, (s.H / 256 + 7) / 8);
+    if (x_dtype == 0)
+      x_digits_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(x), T, s.H, xd, xs, err);
+    else
+      x_digits_kernel<uint16_t><<<g, 256, 0, st>>>(static_cast<const uint16_t*>(x), T, s.H, xd, xs, err);
+  }
+  {
+    GateupArgs ga{};
+    ga.H = s.H; ga.I = s.I; ga.E = s.E; ga.k = s.k; ga.T = T;
+    ga.gate_codes = w.gate_codes; ga.gate_d = w.gate_d; ga.up_codes = w.up_codes; ga.up_d = w.up_d;
+    ga.xd = xd; ga.xs = xs; ga.offsets = r.offsets; ga.perm = r.perm; ga.active = r.active;
+    ga.gu = gu; ga.err = err;
+    ProfScope ps(MOE_K_GATEUP, st);
+    rc |= launch_gateup(ga, slots, sms, st);
+  }
+  if (s.Is > 0) {
+    ProfScope ps(MOE_K_SHARED_GATEUP, st);
+    const int grid = (s.Is + 7) / 8;
+    if (x_dtype == 0)
+      shared_gateup_kernel<float, 4><<<grid, 256, 0, st>>>(s.H, s.Is, w.sh_gate, w.sh_up,
+                                                           static_cast<const float*>(x), T, hsh);
+    else
+      shared_gateup_kernel<uint16_t, 4><<<grid, 256, 0, st>>>(s.H, s.Is, w.sh_gate, w.sh_up,
+                                                              static_cast<const uint16_t*>(x), T, hsh);
+  }
+  {
+    ProfScope ps(MOE_K_HQUANT, st);
+    hquant_kernel<<<static_cast<unsigned>(nA), 256, 0, st>>>(s.I, gu, hd, hsc, hq, hsc_stride(s.I));
+  }
+  {
+    DownArgs da{};
+    da.H = s.H; da.I = s.I; da.E = s.E; da.k = s.k;
+    da.codes = w.down_codes; da.dd = w.down_dd; da.hd = hd; da.hsc = hsc; da.hq = hq;
+    da.offsets = r.offsets; da.active = r.active; da.o = obuf; da.err = err;
+    ProfScope ps(MOE_K_DOWN, st);
+    rc |= launch_down(da, slots, T, sms, st);
+  }
+  {
+    ProfScope ps(MOE_K_COMBINE, st);
+    const int grid = (s.H + 7) / 8;
+    shared_down_combine_kernel<8><<<grid, 256, 0, st>>>(s.H, s.Is, s.k, s.Is > 0 ? w.sh_down : nullptr, hsh, T,
+                                                        r.topk_w, r.inv, obuf, residual, y);
+  }
+  if (rc != OK) return ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
+}
+
+}  // namespace moe

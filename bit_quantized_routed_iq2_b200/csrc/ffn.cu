@@ -222,8 +222,8 @@ __global__ void debug_dequant_q2k_kernel(const uint8_t* __restrict__ codes, cons
 
 }  // namespace
 
-// Workspace of the FFN stage: h [T*k][I], o [T*k][H], shared h [T][Is], s [T][H].
-size_t ffn_workspace_bytes(const LayerShape& s, int T) {
+// Workspace of the CUDA-core FFN stage: h [T*k][I], o [T*k][H], shared h [T][Is], s [T][H].
+static size_t simple_ffn_workspace_bytes(const LayerShape& s, int T) {
   const size_t nA = static_cast<size_t>(T) * s.k;
   size_t b = 0;
   b += align_up(nA * s.I * 4, 256);
@@ -233,8 +233,12 @@ size_t ffn_workspace_bytes(const LayerShape& s, int T) {
   return b;
 }
 
-int launch_ffn(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
-               const float* residual, float* y, void* ws, cudaStream_t st) {
+size_t ffn_workspace_bytes(const LayerShape& s, int T) {
+  return fast_path_supported(s) ? fast_ffn_workspace_bytes(s, T) : simple_ffn_workspace_bytes(s, T);
+}
+
+static int launch_ffn_simple(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T,
+                             const Routing& r, const float* residual, float* y, void* ws, cudaStream_t st) {
   const size_t nA = static_cast<size_t>(T) * s.k;
   char* p = static_cast<char*>(ws);
   float* hbuf = reinterpret_cast<float*>(p);
@@ -280,6 +284,12 @@ int launch_ffn(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dt
     combine_kernel<<<g3, 256, 0, st>>>(s, r, obuf, s.Is > 0 ? sbuf : nullptr, residual, y, T);
   }
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
+}
+
+int launch_ffn(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
+               const float* residual, float* y, void* ws, int* err, cudaStream_t st) {
+  if (fast_path_supported(s)) return launch_ffn_fast(s, w, x, x_dtype, T, r, residual, y, ws, err, st);
+  return launch_ffn_simple(s, w, x, x_dtype, T, r, residual, y, ws, st);
 }
 
 int launch_debug_dequant_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, float* out, cudaStream_t st) {

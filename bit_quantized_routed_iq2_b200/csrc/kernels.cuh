@@ -40,7 +40,13 @@ int launch_active_from_offsets(const int32_t* offsets, int E, int32_t* active, c
 // Workspace needed by the FFN stage for T tokens (bytes) and the launcher.
 size_t ffn_workspace_bytes(const LayerShape& s, int T);
 int launch_ffn(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
-               const float* residual, float* y, void* ws, cudaStream_t st);
+               const float* residual, float* y, void* ws, int* err, cudaStream_t st);
+
+// Tensor-core dequant-GEMV path (decode.cu): shapes with H % 256 == 0 and I % 256 == 0.
+bool fast_path_supported(const LayerShape& s);
+size_t fast_ffn_workspace_bytes(const LayerShape& s, int T);
+int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
+                    const float* residual, float* y, void* ws, int* err, cudaStream_t st);
 
 int launch_debug_dequant_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, float* out, cudaStream_t st);
 int launch_debug_dequant_q2k(const uint8_t* codes, const uint32_t* dd, int64_t nblocks, float* out,

@@ -14,18 +14,88 @@
 
 namespace moe {
 
+__device__ __forceinline__ void bf16x8(const uint4 w, float (&f)[8]) {
+  f[0] = __uint_as_float(w.x << 16); f[1] = __uint_as_float(w.x & 0xFFFF0000u);
+  f[2] = __uint_as_float(w.y << 16); f[3] = __uint_as_float(w.y & 0xFFFF0000u);
+  f[4] = __uint_as_float(w.z << 16); f[5] = __uint_as_float(w.z & 0xFFFF0000u);
+  f[6] = __uint_as_float(w.w << 16); f[7] = __uint_as_float(w.w & 0xFFFF0000u);
+}
+
+template <typename XT>
+__device__ __forceinline__ void load_x8(const XT* x, size_t i, float (&f)[8]) {
+  if constexpr (sizeof(XT) == 4) {
+    const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + i);
+    const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + i + 4);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  } else {
+    bf16x8(*reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(x) + i), f);
+  }
+}
+
 // ---------------------------------------------------------------------------
-// Logits: l[t][e] = sum_h x[t][h] * Wr[e][h] (+ b[e]), fp32 accumulation of the
-// exact bf16 x bf16 (or fp32 x bf16) products. One warp per expert, TT tokens
-// per CTA; lanes read 16-byte slices of the expert's row (coalesced) and the
-// tokens' activations from shared memory. The lane partial sums are combined by
-// a fixed shuffle tree, so results are deterministic.
+// Logits for few tokens: one CTA per (expert, group of TT tokens), 128 threads,
+// each thread holding all of its 16-byte slices of the expert's router row in
+// flight at once. Partial sums combine in a fixed order (deterministic).
+template <typename XT, int TT>
+__global__ void __launch_bounds__(128) router_logits_small_kernel(const uint16_t* __restrict__ Wr,
+                                                                  const float* __restrict__ bias,
+                                                                  const XT* __restrict__ x, int T, int H, int E,
+                                                                  float* __restrict__ logits) {
+  constexpr int MAXJ = 16;  // H <= 16 * 1024
+  __shared__ float part[4][TT];
+  const int e = blockIdx.y;
+  const int t0 = blockIdx.x * TT;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nj = H / 1024 + ((H % 1024) ? 1 : 0);
+  uint4 wv[MAXJ];
+#pragma unroll
+  for (int j = 0; j < MAXJ; ++j) {
+    const int c = tid * 8 + j * 1024;
+    wv[j] = (j < nj && c < H) ? *reinterpret_cast<const uint4*>(Wr + static_cast<size_t>(e) * H + c)
+                              : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float acc[TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) acc[t] = 0.f;
+#pragma unroll
+  for (int j = 0; j < MAXJ; ++j) {
+    const int c = tid * 8 + j * 1024;
+    if (j >= nj || c >= H) break;
+    float w8[8];
+    bf16x8(wv[j], w8);
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+      if (t0 + t >= T) break;
+      float x8[8];
+      load_x8(x, static_cast<size_t>(t0 + t) * H + c, x8);
+      float a = acc[t];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a = fmaf(w8[i], x8[i], a);
+      acc[t] = a;
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < TT; ++t) {
+    float a = acc[t];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (lane == 0) part[warp][t] = a;
+  }
+  __syncthreads();
+  if (tid < TT && t0 + tid < T) {
+    const float v = ((part[0][tid] + part[1][tid]) + (part[2][tid] + part[3][tid])) + (bias ? bias[e] : 0.f);
+    logits[static_cast<size_t>(t0 + tid) * E + e] = v;
+  }
+}
+
+// Logits for many tokens: one warp per expert, TT tokens per CTA, activations
+// staged in shared memory in chunks.
 template <typename XT, int TT>
 __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ Wr,
                                                             const float* __restrict__ bias,
                                                             const XT* __restrict__ x, int T, int H, int E,
                                                             float* __restrict__ logits) {
-  constexpr int CH = 1024;  // activation chunk (elements of H) staged in smem
+  constexpr int CH = 1024;
   __shared__ float xs[TT][CH];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * TT;
@@ -36,7 +106,7 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
   for (int h0 = 0; h0 < H; h0 += CH) {
     __syncthreads();
     for (int i = threadIdx.x; i < TT * CH; i += blockDim.x) {
-      int tt = i / CH, hh = i % CH;
+      const int tt = i / CH, hh = i % CH;
       float v = 0.f;
       if (t0 + tt < T && h0 + hh < H) {
         if constexpr (sizeof(XT) == 4) v = reinterpret_cast<const float*>(x)[(size_t)(t0 + tt) * H + h0 + hh];
@@ -48,12 +118,8 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
     if (e < E) {
       const int lim = min(CH, H - h0);
       for (int c = lane * 8; c < lim; c += 256) {
-        uint4 wv = *reinterpret_cast<const uint4*>(Wr + (size_t)e * H + h0 + c);
         float w8[8];
-        w8[0] = __uint_as_float(wv.x << 16); w8[1] = __uint_as_float(wv.x & 0xFFFF0000u);
-        w8[2] = __uint_as_float(wv.y << 16); w8[3] = __uint_as_float(wv.y & 0xFFFF0000u);
-        w8[4] = __uint_as_float(wv.z << 16); w8[5] = __uint_as_float(wv.z & 0xFFFF0000u);
-        w8[6] = __uint_as_float(wv.w << 16); w8[7] = __uint_as_float(wv.w & 0xFFFF0000u);
+        bf16x8(*reinterpret_cast<const uint4*>(Wr + (size_t)e * H + h0 + c), w8);
 #pragma unroll
         for (int tt = 0; tt < TT; ++tt) {
           const float4 xa = *reinterpret_cast<const float4*>(&xs[tt][c]);
@@ -77,47 +143,62 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
 }
 
 // ---------------------------------------------------------------------------
-// Top-k: one warp per token. k rounds of a warp argmax over the logits held in
-// shared memory (ties to the lower expert index); the winner is removed by
-// writing -inf. Weights: exp(l_j - l_0) / sum_i exp(l_i - l_0), summed in slot
-// order by lane 0.
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
-                                                   int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
-  extern __shared__ float sl[];  // [8 warps][E]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + warp;
-  if (t >= T) return;
-  float* l = sl + (size_t)warp * E;
-  for (int e = lane; e < E; e += 32) l[e] = logits[(size_t)t * E + e];
-  __syncwarp();
+// Top-k of one token by one warp: lane l holds the logits of experts l, l+32,
+// ... in registers (EPL per lane); k rounds of a warp argmax (ties to the lower
+// expert index) with a per-lane bitmask of taken entries. Weights:
+// exp(l_j - l_0) / sum_i exp(l_i - l_0), summed in slot order by lane 0.
+template <int EPL>
+__device__ __forceinline__ void topk_warp(const float* __restrict__ lrow, int E, int k, int32_t* idx_out,
+                                          float* w_out, int32_t* idx_smem) {
+  const int lane = threadIdx.x & 31;
+  float l[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    l[i] = e < E ? lrow[e] : -INFINITY;
+  }
+  uint32_t taken = 0;
   float chosen[16];
   int chosen_idx[16];
   for (int j = 0; j < k; ++j) {
     float bv = -INFINITY;
     int bi = 0x7fffffff;
-    for (int e = lane; e < E; e += 32) {
-      float v = l[e];
-      if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1u) && (l[i] > bv || (l[i] == bv && e < bi))) {
+        bv = l[i];
+        bi = e;
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
       if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
     }
     chosen[j] = bv;
     chosen_idx[j] = bi;
-    if (lane == 0) l[bi] = -INFINITY;
-    __syncwarp();
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
   }
   if (lane == 0) {
     float z = 0.f;
     for (int j = 0; j < k; ++j) z += expf(chosen[j] - chosen[0]);
     for (int j = 0; j < k; ++j) {
-      topk_idx[(size_t)t * k + j] = chosen_idx[j];
-      topk_w[(size_t)t * k + j] = expf(chosen[j] - chosen[0]) / z;
+      idx_out[j] = chosen_idx[j];
+      w_out[j] = expf(chosen[j] - chosen[0]) / z;
+      if (idx_smem) idx_smem[j] = chosen_idx[j];
     }
   }
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                   int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  topk_warp<EPL>(logits + static_cast<size_t>(t) * E, E, k, topk_idx + static_cast<size_t>(t) * k,
+                 topk_w + static_cast<size_t>(t) * k, nullptr);
 }
 
 // ---------------------------------------------------------------------------
@@ -127,38 +208,38 @@ __device__ __forceinline__ int block_exclusive_scan_1024(int v, int* warp_sums, 
   int s = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    int n = __shfl_up_sync(0xffffffffu, s, o);
+    const int n = __shfl_up_sync(0xffffffffu, s, o);
     if (lane >= o) s += n;
   }
   if (lane == 31) warp_sums[warp] = s;
   __syncthreads();
   if (warp == 0) {
-    int w = warp_sums[lane];
+    const int w = warp_sums[lane];
     int ws = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      int n = __shfl_up_sync(0xffffffffu, ws, o);
+      const int n = __shfl_up_sync(0xffffffffu, ws, o);
       if (lane >= o) ws += n;
     }
     warp_sums[lane] = ws - w;  // exclusive
     if (lane == 31) *total = ws;
   }
   __syncthreads();
-  int r = s - v + warp_sums[warp];
+  const int r = s - v + warp_sums[warp];
   __syncthreads();
   return r;
 }
 
-// Histogram + exclusive scan + stable scatter in one CTA of 1024 threads, plus
+// Histogram + exclusive scan + stable scatter by one CTA of 1024 threads, plus
 // the compacted list of experts that received at least one assignment.
 // Stability: assignments are consumed in rounds of 1024 consecutive ids; within
 // a round the rank of an assignment among those routed to the same expert is
 // (#earlier warps' matches, from a per-warp count table) + (#earlier lanes'
 // matches in its own warp, from __match_any_sync). All integer, deterministic.
-__global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict__ topk_idx, int n, int E,
-                                                       int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
-                                                       int32_t* __restrict__ inv, int32_t* __restrict__ active) {
-  extern __shared__ uint8_t smem_raw[];
+// smem: 32*E u16 + 3*E int.
+__device__ void permute_block(const int32_t* topk_idx, int n, int E, int32_t* __restrict__ offsets,
+                              int32_t* __restrict__ perm, int32_t* __restrict__ inv, int32_t* __restrict__ active,
+                              uint8_t* smem_raw) {
   uint16_t* cnt = reinterpret_cast<uint16_t*>(smem_raw);  // [32][E] per-round per-warp counts
   int* run = reinterpret_cast<int*>(cnt + 32 * E);        // [E] assignments placed so far
   int* off = run + E;                                     // [E] offsets
@@ -191,13 +272,13 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
     const int e = valid ? topk_idx[a] : E;  // E is a sentinel, never a real expert
     const unsigned m = __match_any_sync(0xffffffffu, e);
     const int rank_w = __popc(m & lt_mask);
-    if (valid && rank_w == 0) cnt[warp * E + e] = (uint16_t)__popc(m);
+    if (valid && rank_w == 0) cnt[warp * E + e] = static_cast<uint16_t>(__popc(m));
     __syncthreads();
     for (int ee = tid; ee < E; ee += 1024) {  // exclusive prefix over warps, in place
       int s = 0;
       for (int w = 0; w < 32; ++w) {
         const int c = cnt[w * E + ee];
-        cnt[w * E + ee] = (uint16_t)s;
+        cnt[w * E + ee] = static_cast<uint16_t>(s);
         s += c;
       }
       rt[ee] = s;
@@ -217,41 +298,96 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
   }
 }
 
+__global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict__ topk_idx, int n, int E,
+                                                       int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+                                                       int32_t* __restrict__ inv, int32_t* __restrict__ active) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  permute_block(topk_idx, n, E, offsets, perm, inv, active, smem_raw);
+}
+
+// Decode routing in one launch (T*k <= 1024, T <= 32): warp t takes the top-k
+// of token t, then the CTA builds the permutation from shared memory.
+template <int EPL>
+__global__ void __launch_bounds__(1024) topk_permute_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                            int32_t* __restrict__ topk_idx,
+                                                            float* __restrict__ topk_w,
+                                                            int32_t* __restrict__ offsets,
+                                                            int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                            int32_t* __restrict__ active) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  int32_t* idx_s = reinterpret_cast<int32_t*>(smem_raw);  // [T*k] <= 1024
+  uint8_t* pbuf = smem_raw + 1024 * sizeof(int32_t);
+  const int warp = threadIdx.x >> 5;
+  if (warp < T)
+    topk_warp<EPL>(logits + static_cast<size_t>(warp) * E, E, k, topk_idx + static_cast<size_t>(warp) * k,
+                   topk_w + static_cast<size_t>(warp) * k, idx_s + warp * k);
+  __syncthreads();
+  permute_block(idx_s, T * k, E, offsets, perm, inv, active, pbuf);
+}
+
 // Active-expert list from caller-provided offsets (used by moe_expert_ffn).
 __global__ void __launch_bounds__(1024) active_from_offsets_kernel(const int32_t* __restrict__ offsets, int E,
                                                                    int32_t* __restrict__ active) {
   __shared__ int warp_sums[32];
   __shared__ int total;
   const int tid = threadIdx.x;
-  int flag = (tid < E && offsets[tid + 1] > offsets[tid]) ? 1 : 0;
-  int pos = block_exclusive_scan_1024(flag, warp_sums, &total);
+  const int flag = (tid < E && offsets[tid + 1] > offsets[tid]) ? 1 : 0;
+  const int pos = block_exclusive_scan_1024(flag, warp_sums, &total);
   if (flag) active[pos] = tid;
   if (tid == 0) active[E] = total;
 }
 
 // ---------------------------------------------------------------------------
+template <typename K>
+static void set_smem(K kernel, size_t bytes) {
+  if (bytes > 48 * 1024) cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
 int launch_route(const uint16_t* Wr, const float* bias, const void* x, int x_dtype, int T, int H, int E, int k,
                  float* logits, int32_t* topk_idx, float* topk_w, int32_t* offsets, int32_t* perm, int32_t* inv,
                  int32_t* active, cudaStream_t st) {
-  constexpr int TT = 8;
-  dim3 g1((T + TT - 1) / TT, (E + 7) / 8);
   {
     ProfScope ps(MOE_K_ROUTER_LOGITS, st);
-    if (x_dtype == 0)
-      router_logits_kernel<float, TT><<<g1, 256, 0, st>>>(Wr, bias, static_cast<const float*>(x), T, H, E, logits);
-    else
-      router_logits_kernel<uint16_t, TT><<<g1, 256, 0, st>>>(Wr, bias, static_cast<const uint16_t*>(x), T, H, E,
-                                                             logits);
-  }
-  {
-    ProfScope ps(MOE_K_TOPK, st);
-    topk_kernel<<<(T + 7) / 8, 256, 8 * E * sizeof(float), st>>>(logits, T, E, k, topk_idx, topk_w);
+    if (T <= 64) {
+      constexpr int TT = 4;
+      dim3 g((T + TT - 1) / TT, E);
+      if (x_dtype == 0)
+        router_logits_small_kernel<float, TT><<<g, 128, 0, st>>>(Wr, bias, static_cast<const float*>(x), T, H, E,
+                                                                 logits);
+      else
+        router_logits_small_kernel<uint16_t, TT><<<g, 128, 0, st>>>(Wr, bias, static_cast<const uint16_t*>(x), T, H,
+                                                                    E, logits);
+    } else {
+      constexpr int TT = 8;
+      dim3 g((T + TT - 1) / TT, (E + 7) / 8);
+      if (x_dtype == 0)
+        router_logits_kernel<float, TT><<<g, 256, 0, st>>>(Wr, bias, static_cast<const float*>(x), T, H, E, logits);
+      else
+        router_logits_kernel<uint16_t, TT><<<g, 256, 0, st>>>(Wr, bias, static_cast<const uint16_t*>(x), T, H, E,
+                                                              logits);
+    }
   }
   const size_t psmem = 32 * E * sizeof(uint16_t) + 3 * E * sizeof(int);
-  if (psmem > 48 * 1024)
-    cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
-  {
+  if (T * k <= 1024 && T <= 32) {
     ProfScope ps(MOE_K_PERMUTE, st);
+    const size_t sm = 1024 * sizeof(int32_t) + psmem;
+    if (E <= 256) {
+      set_smem(topk_permute_kernel<8>, sm);
+      topk_permute_kernel<8><<<1, 1024, sm, st>>>(logits, T, E, k, topk_idx, topk_w, offsets, perm, inv, active);
+    } else {
+      set_smem(topk_permute_kernel<32>, sm);
+      topk_permute_kernel<32><<<1, 1024, sm, st>>>(logits, T, E, k, topk_idx, topk_w, offsets, perm, inv, active);
+    }
+  } else {
+    {
+      ProfScope ps(MOE_K_TOPK, st);
+      if (E <= 256)
+        topk_kernel<8><<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, topk_idx, topk_w);
+      else
+        topk_kernel<32><<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, topk_idx, topk_w);
+    }
+    ProfScope ps(MOE_K_PERMUTE, st);
+    set_smem(permute_kernel, psmem);
     permute_kernel<<<1, 1024, psmem, st>>>(topk_idx, T * k, E, offsets, perm, inv, active);
   }
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;

@@ -32,7 +32,7 @@ EXPORTS = (
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 KERNEL_NAMES = ("router_logits", "topk", "permute", "active", "gateup", "down", "shared_gateup", "shared_down",
-                "combine", "prep", "prefill_gateup", "prefill_down")
+                "combine", "prep", "prefill_gateup", "prefill_down", "hquant")
 K_COUNT = 16
 
 

@@ -236,6 +236,7 @@ typedef enum {
   MOE_K_PREP = 9,
   MOE_K_PREFILL_GATEUP = 10,
   MOE_K_PREFILL_DOWN = 11,
+  MOE_K_HQUANT = 12,
   MOE_K_COUNT = 16
 } moe_kernel_id;
 MOE_API moe_status moe_profile_enable(int32_t on);
