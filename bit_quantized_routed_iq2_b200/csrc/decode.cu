@@ -154,14 +154,77 @@ __global__ void __launch_bounds__(256) shared_gateup_kernel(int H, int Is, const
   }
 }
 
-// y[t][r] = sum_j w[t][j] o[inv[t*k+j]][r] (j ascending) + (Wsd hs_t)[r] + residual[t][r].
+// Same for few tokens (T <= TMAX): no shared-memory staging and no block-wide
+// barrier; activations come from global memory (L1-resident, the same for every
+// warp), four 16-byte weight loads of each matrix per lane are in flight.
+template <typename XT, int TMAX>
+__global__ void __launch_bounds__(256) shared_gateup_direct_kernel(int H, int Is, const uint16_t* __restrict__ sg,
+                                                                   const uint16_t* __restrict__ su,
+                                                                   const XT* __restrict__ x, int T,
+                                                                   float* __restrict__ hs) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= Is) return;
+  float ag[TMAX], au[TMAX];
+#pragma unroll
+  for (int t = 0; t < TMAX; ++t) ag[t] = au[t] = 0.f;
+  const uint16_t* gr = sg + static_cast<size_t>(row) * H;
+  const uint16_t* ur = su + static_cast<size_t>(row) * H;
+  for (int cb = lane * 8; cb < H; cb += 4 * 256) {
+    uint4 wg[4], wu[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = cb + j * 256;
+      wg[j] = c < H ? *reinterpret_cast<const uint4*>(gr + c) : make_uint4(0u, 0u, 0u, 0u);
+      wu[j] = c < H ? *reinterpret_cast<const uint4*>(ur + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = cb + j * 256;
+      if (c >= H) break;
+      float g8[8], u8[8];
+      bf16x8_to_f32(wg[j], g8);
+      bf16x8_to_f32(wu[j], u8);
+#pragma unroll
+      for (int t = 0; t < TMAX; ++t) {
+        if (t >= T) break;
+        float xv[8];
+        if constexpr (sizeof(XT) == 4) {
+          const float4 xa = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + static_cast<size_t>(t) * H + c);
+          const float4 xb = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + static_cast<size_t>(t) * H + c + 4);
+          xv[0] = xa.x; xv[1] = xa.y; xv[2] = xa.z; xv[3] = xa.w; xv[4] = xb.x; xv[5] = xb.y; xv[6] = xb.z; xv[7] = xb.w;
+        } else {
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(x) + static_cast<size_t>(t) * H + c), xv);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          ag[t] = fmaf(g8[i], xv[i], ag[t]);
+          au[t] = fmaf(u8[i], xv[i], au[t]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < TMAX; ++t) {
+    float gg = ag[t], uu = au[t];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      gg += __shfl_xor_sync(0xffffffffu, gg, o);
+      uu += __shfl_xor_sync(0xffffffffu, uu, o);
+    }
+    if (lane == 0 && t < T) hs[static_cast<size_t>(t) * Is + row] = silu_mul(gg, uu);
+  }
+}
+
+// y[t][r] = sum_j w[t][j] o[inv[t*k+j]][r] (j ascending) + (Wsd hs_t)[r] + residual[t][r],
+// where o of an assignment is the sum of its DP partial rows (parts in order).
 // One warp per output row r, all tokens; the row's weights are loaded up front.
 template <int TMAX>
 __global__ void __launch_bounds__(256) shared_down_combine_kernel(int H, int Is, int k, const uint16_t* __restrict__ sd,
                                                                   const float* __restrict__ hs, int T,
                                                                   const float* __restrict__ topk_w,
                                                                   const int32_t* __restrict__ inv,
-                                                                  const float* __restrict__ obuf,
+                                                                  const float* __restrict__ obuf, int DP,
                                                                   const float* residual, float* y) {
   constexpr int WMAX = 8;  // 16-byte weight loads per lane kept in registers (Is <= 2048)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -215,15 +278,19 @@ __global__ void __launch_bounds__(256) shared_down_combine_kernel(int H, int Is,
       for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
       acc[t] = s;
     }
+    // routed part: lane i takes (slot i / DP, part i % DP); fixed shuffle tree
 #pragma unroll
     for (int t = 0; t < TMAX; ++t) {
-      if (lane == t && t < nt) {
-        const int tt = t0 + t;
-        float v = 0.f;
-        for (int j = 0; j < k; ++j) {
-          const int aidx = tt * k + j;
-          v = fmaf(topk_w[aidx], obuf[static_cast<size_t>(inv[aidx]) * H + row], v);
-        }
+      if (t >= nt) break;
+      const int tt = t0 + t;
+      float v = 0.f;
+      for (int i = lane; i < k * DP; i += 32) {
+        const int aidx = tt * k + i / DP;
+        v = fmaf(topk_w[aidx], obuf[(static_cast<size_t>(inv[aidx]) * DP + i % DP) * H + row], v);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) {
         v += acc[t];
         if (residual) v += residual[static_cast<size_t>(tt) * H + row];
         y[static_cast<size_t>(tt) * H + row] = v;
@@ -258,18 +325,32 @@ int hsc_stride(int I) { return ((I / 256) + 3) & ~3; }
 // sub (0 for the first 16, 1 for the next) goes to byte 8*(j%4) + 4*sub + j/4.
 // Also writes, per 16-element sub-block, the exact integer sum of the digits'
 // values q = 128 hi + lo (the min term of the Q2K-style down projection).
-__global__ void __launch_bounds__(256) hquant_kernel(int I, const float* __restrict__ gu, int8_t* __restrict__ hd,
-                                                     float* __restrict__ hsc, int32_t* __restrict__ hq, int hss) {
+// g and u arrive as KP partial sums each ([p][2][KP][I]); they are added in
+// part order first.
+__global__ void __launch_bounds__(256) hquant_kernel(int I, int KP, const float* __restrict__ gu,
+                                                     int8_t* __restrict__ hd, float* __restrict__ hsc,
+                                                     int32_t* __restrict__ hq, int hss) {
   const int p = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float* g = gu + static_cast<size_t>(p) * 2 * I;
-  const float* u = g + I;
+  const float* g = gu + static_cast<size_t>(p) * 2 * KP * I;
+  const float* u = g + static_cast<size_t>(KP) * I;
   for (int sb = warp; sb < I / 256; sb += 8) {
     const int base = sb * 256 + lane * 8;
-    const float4 g0 = *reinterpret_cast<const float4*>(g + base), g1 = *reinterpret_cast<const float4*>(g + base + 4);
-    const float4 u0 = *reinterpret_cast<const float4*>(u + base), u1 = *reinterpret_cast<const float4*>(u + base + 4);
-    const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-    const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    float gv[8], uv[8];
+    {
+      const float4 g0 = *reinterpret_cast<const float4*>(g + base), g1 = *reinterpret_cast<const float4*>(g + base + 4);
+      const float4 u0 = *reinterpret_cast<const float4*>(u + base), u1 = *reinterpret_cast<const float4*>(u + base + 4);
+      gv[0] = g0.x; gv[1] = g0.y; gv[2] = g0.z; gv[3] = g0.w; gv[4] = g1.x; gv[5] = g1.y; gv[6] = g1.z; gv[7] = g1.w;
+      uv[0] = u0.x; uv[1] = u0.y; uv[2] = u0.z; uv[3] = u0.w; uv[4] = u1.x; uv[5] = u1.y; uv[6] = u1.z; uv[7] = u1.w;
+    }
+    for (int kp = 1; kp < KP; ++kp) {
+      const float* gp = g + static_cast<size_t>(kp) * I + base;
+      const float* up = u + static_cast<size_t>(kp) * I + base;
+      const float4 g0 = *reinterpret_cast<const float4*>(gp), g1 = *reinterpret_cast<const float4*>(gp + 4);
+      const float4 u0 = *reinterpret_cast<const float4*>(up), u1 = *reinterpret_cast<const float4*>(up + 4);
+      gv[0] += g0.x; gv[1] += g0.y; gv[2] += g0.z; gv[3] += g0.w; gv[4] += g1.x; gv[5] += g1.y; gv[6] += g1.z; gv[7] += g1.w;
+      uv[0] += u0.x; uv[1] += u0.y; uv[2] += u0.z; uv[3] += u0.w; uv[4] += u1.x; uv[5] += u1.y; uv[6] += u1.z; uv[7] += u1.w;
+    }
     float h[8], m = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -299,37 +380,70 @@ __global__ void __launch_bounds__(256) hquant_kernel(int I, const float* __restr
   }
 }
 
-size_t fast_ffn_workspace_bytes(const LayerShape& s, int T) {
+// The TMA-fed GEMVs (gemv_tma.cu) serve shapes with H % 1024 == 0 and
+// I % 512 == 0 for up to kTmaMaxT tokens; they write KP (gate/up) and DP
+// (down) partial sums per assignment.
+namespace {
+constexpr int kTmaMaxT = 16;
+bool tma_shape(const LayerShape& s, int T) { return s.H % 1024 == 0 && s.I % 512 == 0 && T <= kTmaMaxT; }
+
+struct FastWs {
+  int8_t* xd;
+  float* xs;
+  float* gu;
+  int8_t* hd;
+  float* hsc;
+  int32_t* hq;
+  float* obuf;
+  float* hsh;
+  size_t bytes;
+};
+
+FastWs carve_fast(const LayerShape& s, int T, int KP, int DP, char* base) {
   const size_t nA = static_cast<size_t>(T) * s.k;
-  size_t b = 0;
-  b += align_up(static_cast<size_t>(T) * 2 * s.H, 256);           // xd
-  b += align_up(static_cast<size_t>(T) * (s.H / 256) * 4, 256);   // xs
-  b += align_up(nA * 2 * s.I * 4, 256);                           // gu
-  b += align_up(nA * 2 * s.I, 256);                               // hd
-  b += align_up(nA * hsc_stride(s.I) * 4, 256);                   // hsc
-  b += align_up(nA * (s.I / 16) * 4, 256);                        // hq
-  b += align_up(nA * s.H * 4, 256);                               // o
-  b += align_up(static_cast<size_t>(T) * (s.Is > 0 ? s.Is : 1) * 4, 256);  // shared h
+  FastWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* q = base ? base + off : nullptr;
+    off += align_up(bytes > 0 ? bytes : 1, 256);
+    return q;
+  };
+  w.xd = reinterpret_cast<int8_t*>(take(static_cast<size_t>(T) * 2 * s.H));
+  w.xs = reinterpret_cast<float*>(take(static_cast<size_t>(T) * (s.H / 256) * 4));
+  w.gu = reinterpret_cast<float*>(take(nA * 2 * KP * s.I * 4));
+  w.hd = reinterpret_cast<int8_t*>(take(nA * 2 * s.I));
+  w.hsc = reinterpret_cast<float*>(take(nA * hsc_stride(s.I) * 4));
+  w.hq = reinterpret_cast<int32_t*>(take(nA * (s.I / 16) * 4));
+  w.obuf = reinterpret_cast<float*>(take(nA * DP * s.H * 4));
+  w.hsh = reinterpret_cast<float*>(take(static_cast<size_t>(T) * (s.Is > 0 ? s.Is : 1) * 4));
+  w.bytes = off;
+  return w;
+}
+}  // namespace
+
+size_t fast_ffn_workspace_bytes(const LayerShape& s, int T) {
+  size_t b = carve_fast(s, T, 1, 1, nullptr).bytes;
+  if (s.H % 1024 == 0 && s.I % 512 == 0) {
+    const int Tt = std::min(T, kTmaMaxT);  // keeps the size monotone in T
+    b = std::max(b, carve_fast(s, Tt, tma_gu_parts(s, Tt), tma_dn_parts(s, Tt), nullptr).bytes);
+  }
   return b;
 }
 
 int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
                     const float* residual, float* y, void* ws, int* err, cudaStream_t st) {
   const size_t nA = static_cast<size_t>(T) * s.k;
-  char* p = static_cast<char*>(ws);
-  auto take = [&](size_t bytes) {
-    char* q = p;
-    p += align_up(bytes, 256);
-    return q;
-  };
-  int8_t* xd = reinterpret_cast<int8_t*>(take(static_cast<size_t>(T) * 2 * s.H));
-  float* xs = reinterpret_cast<float*>(take(static_cast<size_t>(T) * (s.H / 256) * 4));
-  float* gu = reinterpret_cast<float*>(take(nA * 2 * s.I * 4));
-  int8_t* hd = reinterpret_cast<int8_t*>(take(nA * 2 * s.I));
-  float* hsc = reinterpret_cast<float*>(take(nA * hsc_stride(s.I) * 4));
-  int32_t* hq = reinterpret_cast<int32_t*>(take(nA * (s.I / 16) * 4));
-  float* obuf = reinterpret_cast<float*>(take(nA * s.H * 4));
-  float* hsh = reinterpret_cast<float*>(take(static_cast<size_t>(T) * (s.Is > 0 ? s.Is : 1) * 4));
+  const bool tma = tma_shape(s, T) && tma_path_supported(s, T);
+  const int KP = tma ? tma_gu_parts(s, T) : 1, DP = tma ? tma_dn_parts(s, T) : 1;
+  const FastWs fw = carve_fast(s, T, KP, DP, static_cast<char*>(ws));
+  int8_t* xd = fw.xd;
+  float* xs = fw.xs;
+  float* gu = fw.gu;
+  int8_t* hd = fw.hd;
+  float* hsc = fw.hsc;
+  int32_t* hq = fw.hq;
+  float* obuf = fw.obuf;
+  float* hsh = fw.hsh;
 
   const int sms = num_sms();
   const int slots = static_cast<int>(std::min<size_t>(nA, static_cast<size_t>(s.E)));
@@ -342,7 +456,10 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
     else
       x_digits_kernel<uint16_t><<<g, 256, 0, st>>>(static_cast<const uint16_t*>(x), T, s.H, xd, xs, err);
   }
-  {
+  if (tma) {
+    ProfScope ps(MOE_K_GATEUP, st);
+    rc |= launch_gateup_tma(s, w.gate_codes, w.gate_d, w.up_codes, w.up_d, xd, xs, T, r, gu, err, sms, st);
+  } else {
     GateupArgs ga{};
     ga.H = s.H; ga.I = s.I; ga.E = s.E; ga.k = s.k; ga.T = T;
     ga.gate_codes = w.gate_codes; ga.gate_d = w.gate_d; ga.up_codes = w.up_codes; ga.up_d = w.up_d;
@@ -354,18 +471,29 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
   if (s.Is > 0) {
     ProfScope ps(MOE_K_SHARED_GATEUP, st);
     const int grid = (s.Is + 7) / 8;
-    if (x_dtype == 0)
+    if (T <= 4) {
+      if (x_dtype == 0)
+        shared_gateup_direct_kernel<float, 4><<<grid, 256, 0, st>>>(s.H, s.Is, w.sh_gate, w.sh_up,
+                                                                    static_cast<const float*>(x), T, hsh);
+      else
+        shared_gateup_direct_kernel<uint16_t, 4><<<grid, 256, 0, st>>>(s.H, s.Is, w.sh_gate, w.sh_up,
+                                                                       static_cast<const uint16_t*>(x), T, hsh);
+    } else if (x_dtype == 0) {
       shared_gateup_kernel<float, 4><<<grid, 256, 0, st>>>(s.H, s.Is, w.sh_gate, w.sh_up,
                                                            static_cast<const float*>(x), T, hsh);
-    else
+    } else {
       shared_gateup_kernel<uint16_t, 4><<<grid, 256, 0, st>>>(s.H, s.Is, w.sh_gate, w.sh_up,
                                                               static_cast<const uint16_t*>(x), T, hsh);
+    }
   }
   {
     ProfScope ps(MOE_K_HQUANT, st);
-    hquant_kernel<<<static_cast<unsigned>(nA), 256, 0, st>>>(s.I, gu, hd, hsc, hq, hsc_stride(s.I));
+    hquant_kernel<<<static_cast<unsigned>(nA), 256, 0, st>>>(s.I, KP, gu, hd, hsc, hq, hsc_stride(s.I));
   }
-  {
+  if (tma) {
+    ProfScope ps(MOE_K_DOWN, st);
+    rc |= launch_down_tma(s, w.down_codes, w.down_dd, hd, hsc, hq, hsc_stride(s.I), T, r, obuf, err, sms, st);
+  } else {
     DownArgs da{};
     da.H = s.H; da.I = s.I; da.E = s.E; da.k = s.k;
     da.codes = w.down_codes; da.dd = w.down_dd; da.hd = hd; da.hsc = hsc; da.hq = hq;
@@ -377,7 +505,7 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
     ProfScope ps(MOE_K_COMBINE, st);
     const int grid = (s.H + 7) / 8;
     shared_down_combine_kernel<8><<<grid, 256, 0, st>>>(s.H, s.Is, s.k, s.Is > 0 ? w.sh_down : nullptr, hsh, T,
-                                                        r.topk_w, r.inv, obuf, residual, y);
+                                                        r.topk_w, r.inv, obuf, DP, residual, y);
   }
   if (rc != OK) return ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;

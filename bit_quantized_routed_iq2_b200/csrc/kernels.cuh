@@ -48,6 +48,17 @@ size_t fast_ffn_workspace_bytes(const LayerShape& s, int T);
 int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
                     const float* residual, float* y, void* ws, int* err, cudaStream_t st);
 
+// TMA-fed GEMVs (gemv_tma.cu).
+bool tma_path_supported(const LayerShape& s, int T);
+int tma_gu_parts(const LayerShape& s, int T);
+int tma_dn_parts(const LayerShape& s, int T);
+int launch_gateup_tma(const LayerShape& sh, const uint8_t* gate_codes, const uint16_t* gate_d,
+                      const uint8_t* up_codes, const uint16_t* up_d, const int8_t* xd, const float* xs, int T,
+                      const Routing& r, float* gpart, int* err, int sms, cudaStream_t st);
+int launch_down_tma(const LayerShape& sh, const uint8_t* down_codes, const uint32_t* down_dd, const int8_t* hd,
+                    const float* hsc, const int32_t* hq, int hss, int T, const Routing& r, float* opart, int* err,
+                    int sms, cudaStream_t st);
+
 int launch_debug_dequant_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, float* out, cudaStream_t st);
 int launch_debug_dequant_q2k(const uint8_t* codes, const uint32_t* dd, int64_t nblocks, float* out,
                              cudaStream_t st);

@@ -158,6 +158,11 @@ SMALL_CASES = {
     "flat_blocks_k1": _small(H=256, I=64, E=4, k=1, Is=32, T=9, seed=0x5A14),
     "single_expert": _small(E=1, k=1, Is=0, T=5, seed=0x5A15),
     "k_eq_E": _small(E=4, k=4, T=7, seed=0x5A16),
+    # shapes served by the TMA-fed GEMVs (H % 1024 == 0, I % 512 == 0, T <= 16)
+    "tma_t1": _small(H=1024, I=512, E=16, k=4, Is=64, T=1, seed=0x5A17),
+    "tma_t5": _small(H=2048, I=1024, E=8, k=4, Is=128, T=5, seed=0x5A18),
+    "tma_t16": _small(H=1024, I=512, E=8, k=4, Is=64, T=16, seed=0x5A19),
+    "tma_t16_zipf_f32": _small(H=1024, I=1024, E=12, k=3, Is=0, T=16, x_dtype="f32", zipf=True, seed=0x5A1A),
 }
 
 
