@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=0, help="resident layers in rotation (0 = config default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="launch every step directly instead of replaying CUDA graphs")
     ap.add_argument("--experts", type=int, default=0,
                     help="override the routed expert count (small cases for profiling; not a bench workload)")
     return ap.parse_args()
@@ -223,21 +225,48 @@ def run_ours(args, cfg):
         # one step = 16-token decode through all resident layers chained by the residual stream
         xa = torch.empty((T, cfg.H), dtype=torch.bfloat16, device="cuda")
 
-        def step(i):
+        def step_on(i, st):
             cur = xs[i % n_slots]
             for l, dl in enumerate(layers):
-                moe2bit.layer_forward(dl, cur, res if l == 0 else y, y, ws, stream)
+                moe2bit.layer_forward(dl, cur, res if l == 0 else y, y, ws, st)
                 xa.copy_(y)  # next layer input = bf16 of the residual stream
                 cur = xa
         tokens_per_step = T
     else:
-        def step(i):
-            moe2bit.layer_forward(layers[i % n_layers], xs[i % n_slots], None, y, ws, stream)
+        def step_on(i, st):
+            moe2bit.layer_forward(layers[i % n_layers], xs[i % n_slots], None, y, ws, st)
         tokens_per_step = T
+
+    def step(i):
+        step_on(i, stream)
 
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
+    # The timed steps replay CUDA graphs of the same library calls (the library
+    # launches nothing that a graph cannot hold); one graph per distinct
+    # (layer, input) slot of the rotation.
+    period = n_slots if cfg.name.startswith("stack") else int(np.lcm(n_layers, n_slots))
+    graphs = []
+    if args.graph:
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        for j in range(period):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                step_on(j, cap)
+            graphs.append(g)
+        torch.cuda.synchronize()
+        for j in range(period):
+            graphs[j].replay()
+        torch.cuda.synchronize()
+
+    def timed_step(i):
+        if graphs:
+            graphs[i % period].replay()
+        else:
+            step(i)
+
     if world > 1:
         dist.barrier()
     clk = ClockSampler(local)
@@ -247,7 +276,7 @@ def run_ours(args, cfg):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(args.steps):
-        step(args.warmup + i)
+        timed_step(args.warmup + i)
     e1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -338,11 +367,12 @@ def run_ours(args, cfg):
     line = {
         "metric": "moe_layer_tokens_per_s", "value": tokens_per_step * world / (ms * 1e-3), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8-codes/fp32-acc", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
         "config": {"workload": cfg.name, "tokens_per_step": T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
                    "I_s": cfg.Is, "x_dtype": cfg.x_dtype, "resident_layers": n_layers,
                    "l2": f"inputs larger than L2: {n_layers} resident layers in rotation",
-                   "active_experts_per_layer": n_active, "layer_bytes_touched": layer_bytes},
+                   "active_experts_per_layer": n_active, "layer_bytes_touched": layer_bytes,
+                   "launch": "cuda_graph" if graphs else "direct"},
         "roofline": roof,
         "layer_hbm_gbs": layer_bytes / (ms * 1e-3) / 1e9 if cfg.name != "stack" else None,
         "kernels": {k: {"avg_ms": avg_ms[k], "launches_per_step": launches_per_step[k]} for k in prof},

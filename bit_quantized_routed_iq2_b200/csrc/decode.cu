@@ -9,6 +9,8 @@
 // « Comment un modèle de 284 milliards de paramètres tient sur une seule
 // machine » (the routed experts hold most of the bytes, so decode is bound by
 // HBM bandwidth).
+#include <cuda_bf16.h>
+
 #include <algorithm>
 
 #include "decode.cuh"
@@ -22,10 +24,12 @@ namespace moe {
 // xs [T][H/256] = 2^s / 8 per 256-element block (the 1/8 of the IQ2 scale is
 // folded in). One warp per 256-element block, 8 elements per lane. Block (0,0)
 // also clears the call's device status word.
+// For fp32 x it also writes two bf16 parts xb[part][T][H] (hi = rn(v),
+// lo = rn(v - hi)) for the bf16 MMAs of the shared expert.
 template <typename XT>
 __global__ void __launch_bounds__(256) x_digits_kernel(const XT* __restrict__ x, int T, int H,
                                                        int8_t* __restrict__ xd, float* __restrict__ xs,
-                                                       int* __restrict__ err_word) {
+                                                       uint16_t* __restrict__ xb, int* __restrict__ err_word) {
   if (err_word && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *err_word = 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x;
@@ -62,6 +66,20 @@ __global__ void __launch_bounds__(256) x_digits_kernel(const XT* __restrict__ x,
   *reinterpret_cast<uint2*>(row) = make_uint2(hw[0], hw[1]);
   *reinterpret_cast<uint2*>(row + H) = make_uint2(lw[0], lw[1]);
   if (lane == 0) xs[static_cast<size_t>(t) * (H / 256) + blk] = m > 0.f ? ldexpf(1.0f, s - 3) : 0.f;
+  if (sizeof(XT) == 4 && xb) {
+    uint32_t hp[4], lp[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t h0 = __bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i]));
+      const uint32_t h1 = __bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i + 1]));
+      const uint32_t l0 = __bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i] - __uint_as_float(h0 << 16)));
+      const uint32_t l1 = __bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i + 1] - __uint_as_float(h1 << 16)));
+      hp[i] = h0 | (h1 << 16);
+      lp[i] = l0 | (l1 << 16);
+    }
+    *reinterpret_cast<uint4*>(xb + base) = make_uint4(hp[0], hp[1], hp[2], hp[3]);
+    *reinterpret_cast<uint4*>(xb + static_cast<size_t>(T) * H + base) = make_uint4(lp[0], lp[1], lp[2], lp[3]);
+  }
 }
 
 // ------------------------------------------------------------ shared expert
@@ -343,13 +361,29 @@ __global__ void __launch_bounds__(256) hquant_kernel(int I, int KP, const float*
       gv[0] = g0.x; gv[1] = g0.y; gv[2] = g0.z; gv[3] = g0.w; gv[4] = g1.x; gv[5] = g1.y; gv[6] = g1.z; gv[7] = g1.w;
       uv[0] = u0.x; uv[1] = u0.y; uv[2] = u0.z; uv[3] = u0.w; uv[4] = u1.x; uv[5] = u1.y; uv[6] = u1.z; uv[7] = u1.w;
     }
-    for (int kp = 1; kp < KP; ++kp) {
-      const float* gp = g + static_cast<size_t>(kp) * I + base;
-      const float* up = u + static_cast<size_t>(kp) * I + base;
-      const float4 g0 = *reinterpret_cast<const float4*>(gp), g1 = *reinterpret_cast<const float4*>(gp + 4);
-      const float4 u0 = *reinterpret_cast<const float4*>(up), u1 = *reinterpret_cast<const float4*>(up + 4);
-      gv[0] += g0.x; gv[1] += g0.y; gv[2] += g0.z; gv[3] += g0.w; gv[4] += g1.x; gv[5] += g1.y; gv[6] += g1.z; gv[7] += g1.w;
-      uv[0] += u0.x; uv[1] += u0.y; uv[2] += u0.z; uv[3] += u0.w; uv[4] += u1.x; uv[5] += u1.y; uv[6] += u1.z; uv[7] += u1.w;
+    // parts are added in order; loads of up to eight parts are in flight at once
+    for (int k0 = 1; k0 < KP; k0 += 8) {
+      float4 lg[8][2], lu[8][2];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (k0 + q < KP) {
+          const float* gp = g + static_cast<size_t>(k0 + q) * I + base;
+          const float* up = u + static_cast<size_t>(k0 + q) * I + base;
+          lg[q][0] = *reinterpret_cast<const float4*>(gp);
+          lg[q][1] = *reinterpret_cast<const float4*>(gp + 4);
+          lu[q][0] = *reinterpret_cast<const float4*>(up);
+          lu[q][1] = *reinterpret_cast<const float4*>(up + 4);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (k0 + q < KP) {
+          gv[0] += lg[q][0].x; gv[1] += lg[q][0].y; gv[2] += lg[q][0].z; gv[3] += lg[q][0].w;
+          gv[4] += lg[q][1].x; gv[5] += lg[q][1].y; gv[6] += lg[q][1].z; gv[7] += lg[q][1].w;
+          uv[0] += lu[q][0].x; uv[1] += lu[q][0].y; uv[2] += lu[q][0].z; uv[3] += lu[q][0].w;
+          uv[4] += lu[q][1].x; uv[5] += lu[q][1].y; uv[6] += lu[q][1].z; uv[7] += lu[q][1].w;
+        }
+      }
     }
     float h[8], m = 0.f;
 #pragma unroll
@@ -396,6 +430,8 @@ struct FastWs {
   int32_t* hq;
   float* obuf;
   float* hsh;
+  uint16_t* xb;  // bf16 parts of fp32 x [2][T][H]
+  uint16_t* hb;  // bf16 parts of the shared intermediate [2][T][Is]
   size_t bytes;
 };
 
@@ -416,6 +452,8 @@ FastWs carve_fast(const LayerShape& s, int T, int KP, int DP, char* base) {
   w.hq = reinterpret_cast<int32_t*>(take(nA * (s.I / 16) * 4));
   w.obuf = reinterpret_cast<float*>(take(nA * DP * s.H * 4));
   w.hsh = reinterpret_cast<float*>(take(static_cast<size_t>(T) * (s.Is > 0 ? s.Is : 1) * 4));
+  w.xb = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(T) * 2 * s.H * 2));
+  w.hb = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(T) * 2 * (s.Is > 0 ? s.Is : 1) * 2));
   w.bytes = off;
   return w;
 }
@@ -452,10 +490,14 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
     ProfScope ps(MOE_K_PREP, st);
     dim3 g(T, (s.H / 256 + 7) / 8);
     if (x_dtype == 0)
-      x_digits_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(x), T, s.H, xd, xs, err);
+      x_digits_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(x), T, s.H, xd, xs, fw.xb, err);
     else
-      x_digits_kernel<uint16_t><<<g, 256, 0, st>>>(static_cast<const uint16_t*>(x), T, s.H, xd, xs, err);
+      x_digits_kernel<uint16_t><<<g, 256, 0, st>>>(static_cast<const uint16_t*>(x), T, s.H, xd, xs, nullptr, err);
   }
+  // bf16 activations feed the shared expert's MMAs as one part, fp32 as two
+  const int xparts = x_dtype == 0 ? 2 : 1;
+  const uint16_t* xbp = x_dtype == 0 ? fw.xb : static_cast<const uint16_t*>(x);
+  const bool sh_mma = s.Is > 0 && shared_mma_supported(s.H, s.Is, T, xparts);
   if (tma) {
     ProfScope ps(MOE_K_GATEUP, st);
     rc |= launch_gateup_tma(s, w.gate_codes, w.gate_d, w.up_codes, w.up_d, xd, xs, T, r, gu, err, sms, st);
@@ -468,7 +510,10 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
     ProfScope ps(MOE_K_GATEUP, st);
     rc |= launch_gateup(ga, slots, sms, st);
   }
-  if (s.Is > 0) {
+  if (sh_mma) {
+    ProfScope ps(MOE_K_SHARED_GATEUP, st);
+    rc |= launch_shared_gateup_mma(s.H, s.Is, w.sh_gate, w.sh_up, xbp, xparts, T, fw.hb, st);
+  } else if (s.Is > 0) {
     ProfScope ps(MOE_K_SHARED_GATEUP, st);
     const int grid = (s.Is + 7) / 8;
     if (T <= 4) {
@@ -501,7 +546,11 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
     ProfScope ps(MOE_K_DOWN, st);
     rc |= launch_down(da, slots, T, sms, st);
   }
-  {
+  if (sh_mma) {
+    ProfScope ps(MOE_K_COMBINE, st);
+    rc |= launch_shared_down_combine_mma(s.H, s.Is, w.sh_down, fw.hb, T, s.k, r.topk_w, r.inv, obuf, DP, residual,
+                                         y, st);
+  } else {
     ProfScope ps(MOE_K_COMBINE, st);
     const int grid = (s.H + 7) / 8;
     shared_down_combine_kernel<8><<<grid, 256, 0, st>>>(s.H, s.Is, s.k, s.Is > 0 ? w.sh_down : nullptr, hsh, T,

@@ -1,22 +1,35 @@
 // gemv_tma.cu - decode dequant-GEMVs of the routed experts fed by 2-D TMA
 // tensor-map loads, with warp specialisation: one producer warp streams boxes
 // of code rows into a ring of shared-memory stages (full/empty mbarriers, all
-// waits bounded), eight consumer warps each own 16 rows and turn the codes into
-// int8 MMA operands. No block-wide barrier inside the main loop.
+// waits bounded), sixteen consumer warps each own 16 rows and turn the codes
+// into int8 MMA operands. No block-wide barrier inside the main loop.
 //
 // Sources: "ds4 : analyse pratique pour un usage documenté", section « Support
 // de modèles et choix de quantification » (up/gate IQ2_XXS, down Q2_K). The
 // operand construction and the integer accumulation are those of decode.cuh.
 //
-// Work is split into units small enough to balance over all SMs: a gate/up
-// unit is (expert, gate or up, 128 rows, 1024-wide part of H) and a down unit
-// is (expert, 128 rows of H, 512-wide part of I). Each unit writes partial
-// sums that the next kernel adds up in a fixed order.
+// Work is split into equal units so that every SM gets the same number: a
+// gate/up unit is (expert, gate or up, 256 rows, NB boxes of 512 of H) and a
+// down unit is (expert, 256 rows of H, NB blocks of 256 of I), NB = 1 for a
+// single token and 2 otherwise (fewer partial sums to keep). Each unit writes
+// partial sums that the next kernel adds up in a fixed order.
 //
-// gate/up boxes: 128 rows x 128 code bytes (16 sub-blocks), 128-byte swizzle,
-//   so the eight rows a warp reads together land in eight different 16-byte
-//   bank groups. down boxes: 128 rows x 160 code bytes (two blocks), dense; the
-//   160-byte pitch makes the eight-row reads two-way conflicted at most.
+// Routing metadata (offsets, active experts, token of each assignment) is
+// copied to shared memory once per CTA; units are walked with a mixed-radix
+// counter (no integer division in the loop), and the per-row fp16 scales of
+// the next unit are loaded one unit ahead, so no dependent global load sits
+// on the critical path of a unit.
+//
+// When the activations fit, they are staged in shared memory with rows padded
+// by 32 bytes, and the zero operand region is placed 64 bytes further, so the
+// hi-digit row, the lo-digit row and the zeros that one MMA's B operand reads
+// fall in different banks.
+//
+// gate/up boxes: 256 rows x 128 code bytes (16 sub-blocks), 128-byte swizzle,
+//   so the eight rows a quad column reads together land in eight different
+//   16-byte bank groups. down boxes: 256 rows x 80 code bytes (one block),
+//   dense; the 80-byte pitch maps eight consecutive rows to eight different
+//   16-byte bank groups as well.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -33,19 +46,105 @@ namespace {
 
 __device__ const Iq2SelTables d_sel_tables2 = make_sel_tables();
 
-constexpr int kCW = 8;                       // consumer warps (16 rows each)
+constexpr int kCW = 16;                      // consumer warps (16 rows each)
 constexpr int kThreadsT = (kCW + 1) * 32;    // + one producer warp
-constexpr int kBoxRows = 16 * kCW;           // 128 rows per box
-constexpr int kGuBox = kBoxRows * 128;       // bytes per gate/up box
-constexpr int kDnBox = kBoxRows * 160;       // bytes per down box
-constexpr uint32_t kLvlOff = 0;              // replicated level table (32 KB)
-constexpr uint32_t kSgnOff = 32768;          // replicated sign table (16 KB)
-constexpr uint32_t kXOff = 49152;            // activation digits when staged
+constexpr int kBoxRows = 16 * kCW;           // 256 rows per box
+constexpr int kGuW = 128;                    // code bytes per gate/up box row (512 weights)
+constexpr int kGuBox = kBoxRows * kGuW;      // 32 KB
+constexpr int kDnW = 80;                     // one Q2K-style block per down box row
+constexpr int kDnBox = kBoxRows * kDnW;      // 20 KB
+constexpr uint32_t kSgnOff = 32768;          // sign table after the level table (32 KB)
+constexpr int kTabWords = (256 + 128) * 32;  // both tables, each entry replicated for the 32 lanes
+constexpr int kZeroBytes = 1024;             // zero operand region for idle MMA columns
+constexpr int kRowPad = 32;                  // padding of a staged activation row
+constexpr int kMaxExpertsTma = 1024;
+constexpr int kMaxNB = 2;
+
+// Zero operand for the variants that read activations from global memory.
+__device__ __align__(128) const int8_t g_zero_operand[kZeroBytes] = {};
 
 __device__ __forceinline__ uint32_t rotr(uint32_t v, uint32_t n) { return __funnelshift_r(v, v, n); }
 
+__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+
+// Loads from shared memory at 32-bit shared-window addresses. They are volatile
+// so that they stay after the mbarrier wait that makes the data visible.
+__device__ __forceinline__ uint4 ld_s128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 ld_s64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_s32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_s8(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float ld_sf(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+
+__host__ __device__ inline size_t meta_bytes(int E, int nA, bool with_tok) {
+  return align_up(static_cast<size_t>(2 * (E + 1) + (with_tok ? nA : 0)) * 4, 128);
+}
+
+// Routing metadata in shared memory.
+struct MetaSmem {
+  int32_t* off;  // [E+1]
+  int32_t* act;  // [E+1], act[E] = number of active experts
+  int32_t* tok;  // [T*k] token of each expert-sorted assignment (gate/up only)
+};
+
+__device__ __forceinline__ void load_meta(const MetaSmem& m, const int32_t* offsets, const int32_t* active,
+                                          const int32_t* perm, int E, int nA, int k, int tid, int nthr) {
+  for (int i = tid; i <= E; i += nthr) {
+    m.off[i] = offsets[i];
+    m.act[i] = active[i];
+  }
+  if (m.tok)
+    for (int i = tid; i < nA; i += nthr) m.tok[i] = perm[i] / k;
+}
+
+// Copy rows of `row_bytes` (a multiple of 16) from global memory into shared
+// memory with a row pitch of row_bytes + kRowPad.
+__device__ __forceinline__ void stage_rows(int8_t* dst, const int8_t* src, int rows, int row_bytes, int tid,
+                                           int nthr) {
+  const int per = row_bytes / 16;
+  for (int i = tid; i < rows * per; i += nthr) {
+    const int r = i / per, cidx = i - r * per;
+    *reinterpret_cast<uint4*>(dst + static_cast<size_t>(r) * (row_bytes + kRowPad) + cidx * 16) =
+        reinterpret_cast<const uint4*>(src)[i];
+  }
+}
+
+// Ring position: stage index and phase parity.
+struct RingPos {
+  int s;
+  uint32_t ph;
+  __device__ __forceinline__ void next(int S) {
+    if (++s == S) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+};
+
+// ===========================================================================
+// gate/up
+// ===========================================================================
 struct GuTmaArgs {
-  int H, I, E, k, T, KP, S, x_in_smem;
+  int H, I, E, k, T, KP, NB, S;
   const uint16_t* gate_d;
   const uint16_t* up_d;
   const int8_t* xd;
@@ -57,123 +156,261 @@ struct GuTmaArgs {
   int* err;
 };
 
+// Unit u = ((slot * 2 + m) * rbs + rb) * KP + kp, walked in steps of gridDim.x.
+struct GuIter {
+  int kp, rb, m, slot, dkp, drb, dm, dslot;
+  __device__ __forceinline__ void init(int u0, int G, int KP, int rbs) {
+    kp = u0 % KP;
+    int r = u0 / KP;
+    rb = r % rbs;
+    r /= rbs;
+    m = r & 1;
+    slot = r >> 1;
+    dkp = G % KP;
+    r = G / KP;
+    drb = r % rbs;
+    r /= rbs;
+    dm = r & 1;
+    dslot = r >> 1;
+  }
+  __device__ __forceinline__ void next(int KP, int rbs) {
+    kp += dkp;
+    int c = kp >= KP ? 1 : 0;
+    kp -= c * KP;
+    rb += drb + c;
+    c = rb >= rbs ? 1 : 0;
+    rb -= c * rbs;
+    m += dm + c;
+    c = m >= 2 ? 1 : 0;
+    m -= 2 * c;
+    slot += dslot + c;
+  }
+};
+
+struct GuUnit {
+  int e, m, rb, kp, p0, ne;
+};
+
+__device__ __forceinline__ GuUnit gu_unit_of(const GuIter& t, const MetaSmem& ms) {
+  GuUnit w;
+  w.kp = t.kp;
+  w.rb = t.rb;
+  w.m = t.m;
+  w.e = ms.act[t.slot];
+  w.p0 = ms.off[w.e];
+  w.ne = ms.off[w.e + 1] - w.p0;
+  return w;
+}
+
 struct GuCtx {
+  const char* tab;      // level table, then sign table at +kSgnOff (static shared memory)
   const uint8_t* ring;
   uint64_t* full;
   uint64_t* empty;
-  const int8_t* xdig;
-  const float* xscl;
-  int warp, lane, g, tig, S;
+  const int8_t* xdig;   // rows (token, digit hi/lo) of H digits, pitch xpitch
+  const float* xscl;    // [T][H/256] 2^s / 8
+  const int8_t* zero;   // 128-byte aligned zero region
+  const int32_t* tok;
+  uint32_t ring_s, x_s, xs_s, zero_s;  // shared-window addresses (staged variant)
+  int xpitch, warp, lane, g, tig, S;
   uint32_t lane4, rot_idx, rot_sig;
 };
 
-// One unit (two boxes) for TPG tokens per MMA column group, up to MAXQ groups.
-// Returns false on a timed-out wait.
+// Selector word (level nibbles | sign bits) of grid group `tig` of one 8-byte
+// sub-block record -> two int8x4 A registers.
+__device__ __forceinline__ void iq2_operand(const GuCtx& c, uint2 rec, uint32_t& lo, uint32_t& hi) {
+  const uint32_t al = (rotr(rec.x, c.rot_idx) & 0x7F80u) | c.lane4;
+  const uint32_t as = (rotr(rec.y, c.rot_sig) & 0x3F80u) | c.lane4;
+  const uint32_t sel = *reinterpret_cast<const uint32_t*>(c.tab + al) |
+                       *reinterpret_cast<const uint32_t*>(c.tab + kSgnOff + as);
+  lo = prmt(kPosBytes, kNegBytes, sel);
+  hi = prmt(kPosBytes, kNegBytes, __umulhi(sel, 0x10000u));
+}
+
+// The eight records (four sub-blocks x rows g, g+8) of chunk pair cc.
+__device__ __forceinline__ void gu_records(const uint8_t* rg, int cc, int g, uint2 (&rec)[4][2]) {
+  const uint4 a0 = lds128(rg + (((2 * cc) ^ g) << 4));
+  const uint4 a1 = lds128(rg + (((2 * cc + 1) ^ g) << 4));
+  const uint4 b0 = lds128(rg + 1024 + (((2 * cc) ^ g) << 4));
+  const uint4 b1 = lds128(rg + 1024 + (((2 * cc + 1) ^ g) << 4));
+  rec[0][0] = make_uint2(a0.x, a0.y); rec[1][0] = make_uint2(a0.z, a0.w);
+  rec[2][0] = make_uint2(a1.x, a1.y); rec[3][0] = make_uint2(a1.z, a1.w);
+  rec[0][1] = make_uint2(b0.x, b0.y); rec[1][1] = make_uint2(b0.z, b0.w);
+  rec[2][1] = make_uint2(b1.x, b1.y); rec[3][1] = make_uint2(b1.z, b1.w);
+}
+
+// 2*ls+1 of sub-block sb (0..15) of the row at rg (swizzled 128-byte row).
+__device__ __forceinline__ int gu_odd(const uint8_t* rg, int sb, int g) {
+  const uint32_t b = rg[(((sb >> 1) ^ g) << 4) + (sb & 1) * 8 + 7];
+  return static_cast<int>((b >> 3) | 1u);
+}
+
+__device__ __forceinline__ float half_lo(uint32_t w) { return half_bits_to_float(static_cast<uint16_t>(w & 0xFFFFu)); }
+__device__ __forceinline__ float half_hi(uint32_t w) { return half_bits_to_float(static_cast<uint16_t>(w >> 16)); }
+
+// One unit whose expert holds a single assignment (every decode step with one
+// token), activations staged in shared memory. MMA columns: (sub-block slot
+// 0..3) x (digit hi, lo); the B operand of an idle column comes from the zero
+// region, so no select is needed. All shared-memory addresses are 32-bit and
+// the 128-byte swizzle is applied with one XOR per 16-byte chunk: with
+// rgg = row base + 16*g, logical chunk L of row g sits at rgg ^ (16*L).
+__device__ __forceinline__ bool gu_unit_one(const GuTmaArgs& a, const GuCtx& c, RingPos& rp, const GuUnit& w,
+                                            const uint32_t (&dp)[kMaxNB][2]) {
+  const int H = a.H, I = a.I, NB = a.NB;
+  const int g = c.g, tig = c.tig;
+  const int tok = c.tok[w.p0];
+  const int row_l = 16 * c.warp + g;
+  const uint32_t xrow = c.x_s + (tok * 2 + (g & 1)) * c.xpitch + w.kp * NB * 512 + 8 * tig;
+  const uint32_t zrow = c.zero_s + ((64 * (tok & 1) + 64) & 127) + 8 * tig;
+  const uint32_t xsc = c.xs_s + (tok * (H / 256) + 2 * NB * w.kp) * 4;
+  const uint32_t lsoff = ((((tig >> 1) ^ g)) << 4) + (tig & 1) * 8 + 7;
+  float f0 = 0.f, f1 = 0.f;
+#pragma unroll 1
+  for (int j = 0; j < NB; ++j) {
+    uint32_t bp[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) bp[u] = ((g >> 1) == u) ? xrow + j * 512 : zrow;
+    if (!mbar_wait_bounded(&c.full[rp.s], rp.ph, a.err, ERR_TIMEOUT)) return false;
+    const uint32_t rg = c.ring_s + rp.s * kGuBox + row_l * kGuW;
+    const int s = rp.s;
+    rp.next(c.S);
+    const uint32_t rgg = rg + 16 * g, lsa = rg + lsoff;
+    int i0 = 0, i1 = 0;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      const uint4 a0 = ld_s128(rgg ^ (32 * cc));
+      const uint4 a1 = ld_s128(rgg ^ (32 * cc + 16));
+      const uint4 b0 = ld_s128((rgg + 1024) ^ (32 * cc));
+      const uint4 b1 = ld_s128((rgg + 1024) ^ (32 * cc + 16));
+      uint2 bv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) bv[u] = ld_s64(bp[u] + (4 * cc + u) * 32);
+      const uint32_t l0 = ld_s8(lsa ^ (32 * cc)), l1 = ld_s8((lsa + 1024) ^ (32 * cc));
+      const uint2 rec[4][2] = {{make_uint2(a0.x, a0.y), make_uint2(b0.x, b0.y)},
+                               {make_uint2(a0.z, a0.w), make_uint2(b0.z, b0.w)},
+                               {make_uint2(a1.x, a1.y), make_uint2(b1.x, b1.y)},
+                               {make_uint2(a1.z, a1.w), make_uint2(b1.z, b1.w)}};
+      int acc[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        uint32_t r0lo, r0hi, r1lo, r1hi;
+        iq2_operand(c, rec[u][0], r0lo, r0hi);
+        iq2_operand(c, rec[u][1], r1lo, r1hi);
+        if (u == 0)
+          mma_s8s8_zero(acc, r0lo, r1lo, r0hi, r1hi, bv[u].x, bv[u].y);
+        else
+          mma_s8s8(acc, r0lo, r1lo, r0hi, r1hi, bv[u].x, bv[u].y);
+      }
+      // this thread's columns are sub-block 4cc+tig, digits hi and lo
+      i0 += (acc[0] * 128 + acc[1]) * static_cast<int>((l0 >> 3) | 1u);
+      i1 += (acc[2] * 128 + acc[3]) * static_cast<int>((l1 >> 3) | 1u);
+      if (cc & 1) {
+        const int sb = cc >> 1;
+        const float xsv = ld_sf(xsc + (2 * j + sb) * 4);
+        const uint32_t w0 = j ? dp[1][0] : dp[0][0], w1 = j ? dp[1][1] : dp[0][1];
+        const float d0 = sb ? half_hi(w0) : half_lo(w0);
+        const float d1 = sb ? half_hi(w1) : half_lo(w1);
+        f0 = fmaf(static_cast<float>(i0), d0 * xsv, f0);
+        f1 = fmaf(static_cast<float>(i1), d1 * xsv, f1);
+        i0 = i1 = 0;
+      }
+    }
+    __syncwarp();
+    if (c.lane == 0) mbar_arrive(&c.empty[s]);
+  }
+  // the four lanes of a quad hold four different sub-blocks of the same rows
+  f0 += __shfl_xor_sync(0xffffffffu, f0, 1);
+  f0 += __shfl_xor_sync(0xffffffffu, f0, 2);
+  f1 += __shfl_xor_sync(0xffffffffu, f1, 1);
+  f1 += __shfl_xor_sync(0xffffffffu, f1, 2);
+  if (tig == 0) {
+    float* out = a.gpart + ((static_cast<size_t>(w.p0) * 2 + w.m) * a.KP + w.kp) * I + w.rb * kBoxRows + row_l;
+    out[0] = f0;
+    out[8] = f1;
+  }
+  return true;
+}
+
+// One unit whose expert holds 2..4*MAXQ assignments. TPG tokens share one set
+// of MMA columns (TPG tokens x 4/TPG sub-block slots x 2 digits); MAXQ column
+// sets reuse the same A operands.
 template <int TPG, int MAXQ>
-__device__ __forceinline__ bool gu_unit(const GuTmaArgs& a, const uint8_t* smem, const GuCtx& c, int& it, int e,
-                                        int m, int rb, int kp, int p0, int ne) {
+__device__ __forceinline__ bool gu_unit_multi(const GuTmaArgs& a, const GuCtx& c, RingPos& rp, const GuUnit& w,
+                                              const uint32_t (&dp)[kMaxNB][2]) {
   constexpr int SPS = 4 / TPG;
-  const int H = a.H, I = a.I;
+  const int H = a.H, I = a.I, ne = w.ne, p0 = w.p0;
   const int ngroups = (ne + TPG - 1) / TPG;
   const int g = c.g, tig = c.tig;
   const int tslot_b = (g >> 1) % TPG, sslot_b = (g >> 1) / TPG, dig_b = g & 1;
   const int tslot_c = tig % TPG, sslot_c = tig / TPG;
-  const int row_l = 16 * c.warp + g;  // row within the box (and +8)
-  const size_t row_g = static_cast<size_t>(e) * I + rb * kBoxRows + row_l;
-  // d of the part's four super-blocks for rows g and g+8
-  const uint16_t* dpl = m ? a.up_d : a.gate_d;
-  const uint2 dq0 = *reinterpret_cast<const uint2*>(dpl + row_g * (H / 256) + kp * 4);
-  const uint2 dq1 = *reinterpret_cast<const uint2*>(dpl + (row_g + 8) * (H / 256) + kp * 4);
+  const int row_l = 16 * c.warp + g;
   const int8_t* xb[MAXQ];
-  bool bval[MAXQ];
   const float* xsc[MAXQ];
+  bool bon[MAXQ];
 #pragma unroll
   for (int q = 0; q < MAXQ; ++q) {
     const int tb = q * TPG + tslot_b, tc = q * TPG + tslot_c;
-    bval[q] = q < ngroups && tb < ne;
-    const int tok = bval[q] ? a.perm[p0 + tb] / a.k : 0;
-    xb[q] = c.xdig + (static_cast<size_t>(tok) * 2 + dig_b) * H + 8 * tig + (kp * 32 + sslot_b) * 32;
-    xsc[q] = (q < ngroups && tc < ne) ? c.xscl + static_cast<size_t>(a.perm[p0 + tc] / a.k) * (H / 256) + kp * 4
-                                      : nullptr;
+    bon[q] = q < ngroups && tb < ne;
+    xb[q] = bon[q] ? c.xdig + (c.tok[p0 + tb] * 2 + dig_b) * c.xpitch + 8 * tig + (w.kp * a.NB * 16 + sslot_b) * 32
+                   : c.zero + 8 * tig;
+    xsc[q] = (q < ngroups && tc < ne) ? c.xscl + c.tok[p0 + tc] * (H / 256) + 2 * a.NB * w.kp : nullptr;
   }
-  int acc[MAXQ][2][4];
+  int acc[MAXQ][4];
   int iacc[MAXQ][2];
   float facc[MAXQ][2];
 #pragma unroll
   for (int q = 0; q < MAXQ; ++q) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) acc[q][h][0] = acc[q][h][1] = acc[q][h][2] = acc[q][h][3] = 0;
     iacc[q][0] = iacc[q][1] = 0;
     facc[q][0] = facc[q][1] = 0.f;
   }
 #pragma unroll 1
-  for (int j = 0; j < 2; ++j, ++it) {
-    const int s = it % c.S;
-    if (!mbar_wait_bounded(&c.full[s], (it / c.S) & 1u, a.err, ERR_TIMEOUT)) return false;
-    const uint8_t* st = c.ring + s * kGuBox;
-    const uint8_t* rg = st + row_l * 128;
-    const uint8_t* rg8 = rg + 8 * 128;
+  for (int j = 0; j < a.NB; ++j) {
+    if (!mbar_wait_bounded(&c.full[rp.s], rp.ph, a.err, ERR_TIMEOUT)) return false;
+    const int s = rp.s;
+    rp.next(c.S);
+    const uint8_t* rg = c.ring + s * kGuBox + row_l * kGuW;
+    const uint32_t dj0 = j ? dp[1][0] : dp[0][0], dj1 = j ? dp[1][1] : dp[0][1];
 #pragma unroll 1
     for (int cc = 0; cc < 4; ++cc) {
       uint2 rec[4][2];
-      {
-        const uint4 a0 = *reinterpret_cast<const uint4*>(rg + (((2 * cc) ^ g) << 4));
-        const uint4 a1 = *reinterpret_cast<const uint4*>(rg + (((2 * cc + 1) ^ g) << 4));
-        const uint4 b0 = *reinterpret_cast<const uint4*>(rg8 + (((2 * cc) ^ g) << 4));
-        const uint4 b1 = *reinterpret_cast<const uint4*>(rg8 + (((2 * cc + 1) ^ g) << 4));
-        rec[0][0] = make_uint2(a0.x, a0.y); rec[1][0] = make_uint2(a0.z, a0.w);
-        rec[2][0] = make_uint2(a1.x, a1.y); rec[3][0] = make_uint2(a1.z, a1.w);
-        rec[0][1] = make_uint2(b0.x, b0.y); rec[1][1] = make_uint2(b0.z, b0.w);
-        rec[2][1] = make_uint2(b1.x, b1.y); rec[3][1] = make_uint2(b1.z, b1.w);
-      }
+      gu_records(rg, cc, g, rec);
       uint32_t af[4][2][2];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const uint32_t al = (rotr(rec[u][r].x, c.rot_idx) & 0x7F80u) | c.lane4;
-          const uint32_t as = (rotr(rec[u][r].y, c.rot_sig) & 0x3F80u) | c.lane4;
-          const uint32_t sel = *reinterpret_cast<const uint32_t*>(smem + kLvlOff + al) |
-                               *reinterpret_cast<const uint32_t*>(smem + kSgnOff + as);
-          af[u][r][0] = prmt(kPosBytes, kNegBytes, sel);
-          af[u][r][1] = prmt(kPosBytes, kNegBytes, sel >> 16);
-        }
-      const int sbo = j * 16 + 4 * cc;  // sub-block offset inside the part
+      for (int u = 0; u < 4; ++u) {
+        iq2_operand(c, rec[u][0], af[u][0][0], af[u][0][1]);
+        iq2_operand(c, rec[u][1], af[u][1][0], af[u][1][1]);
+      }
 #pragma unroll
       for (int q = 0; q < MAXQ; ++q) {
         if (q >= ngroups) break;
-        uint2 bl[TPG];
 #pragma unroll
-        for (int jj = 0; jj < TPG; ++jj)
-          bl[jj] = bval[q] ? *reinterpret_cast<const uint2*>(xb[q] + (sbo + jj * SPS) * 32) : make_uint2(0u, 0u);
+        for (int jj = 0; jj < TPG; ++jj) {
+          // column set jj covers sub-blocks 4cc + jj*SPS .. +SPS-1
+          const int8_t* xp = bon[q] ? xb[q] + j * 512 : xb[q];
+          const uint2 bl = *reinterpret_cast<const uint2*>(xp + (4 * cc + jj * SPS) * 32);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int jj = u / SPS, slot = u % SPS;
-          const bool on = slot == sslot_b;
-          mma_s8s8(acc[q][u & 1], af[u][0][0], af[u][1][0], af[u][0][1], af[u][1][1], on ? bl[jj].x : 0u,
-                   on ? bl[jj].y : 0u);
-          if (slot == SPS - 1) {
-            uint32_t v0 = rec[jj * SPS][0].y, v1 = rec[jj * SPS][1].y;
-#pragma unroll
-            for (int w = 1; w < SPS; ++w)
-              if (sslot_c == w) { v0 = rec[jj * SPS + w][0].y; v1 = rec[jj * SPS + w][1].y; }
-            const int odd0 = static_cast<int>((v0 >> 27) | 1u), odd1 = static_cast<int>((v1 >> 27) | 1u);
-            iacc[q][0] += ((acc[q][0][0] + acc[q][1][0]) * 128 + acc[q][0][1] + acc[q][1][1]) * odd0;
-            iacc[q][1] += ((acc[q][0][2] + acc[q][1][2]) * 128 + acc[q][0][3] + acc[q][1][3]) * odd1;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) acc[q][h][0] = acc[q][h][1] = acc[q][h][2] = acc[q][h][3] = 0;
+          for (int sl = 0; sl < SPS; ++sl) {
+            const int u = jj * SPS + sl;
+            const bool on = sl == sslot_b;
+            const uint32_t b0 = on ? bl.x : 0u, b1 = on ? bl.y : 0u;
+            if (sl == 0)
+              mma_s8s8_zero(acc[q], af[u][0][0], af[u][1][0], af[u][0][1], af[u][1][1], b0, b1);
+            else
+              mma_s8s8(acc[q], af[u][0][0], af[u][1][0], af[u][0][1], af[u][1][1], b0, b1);
           }
+          const int sbi = 4 * cc + jj * SPS + sslot_c;
+          const int odd0 = gu_odd(rg, sbi, g), odd1 = gu_odd(rg + 1024, sbi, g);
+          iacc[q][0] += (acc[q][0] * 128 + acc[q][1]) * odd0;
+          iacc[q][1] += (acc[q][2] * 128 + acc[q][3]) * odd1;
         }
       }
       if (cc & 1) {
-        // super-block done: d (per row) and 2^s/8 (per token)
-        const int sbl = j * 2 + (cc >> 1);
-        const uint32_t w0 = sbl < 2 ? dq0.x : dq0.y, w1 = sbl < 2 ? dq1.x : dq1.y;
-        const float d0 = half_bits_to_float(static_cast<uint16_t>((sbl & 1) ? (w0 >> 16) : (w0 & 0xFFFFu)));
-        const float d1 = half_bits_to_float(static_cast<uint16_t>((sbl & 1) ? (w1 >> 16) : (w1 & 0xFFFFu)));
+        const int sb = cc >> 1;
+        const float d0 = sb ? half_hi(dj0) : half_lo(dj0);
+        const float d1 = sb ? half_hi(dj1) : half_lo(dj1);
 #pragma unroll
         for (int q = 0; q < MAXQ; ++q) {
-          const float xsv = xsc[q] ? xsc[q][sbl] : 0.f;
+          const float xsv = xsc[q] ? xsc[q][2 * j + sb] : 0.f;
           facc[q][0] = fmaf(static_cast<float>(iacc[q][0]), d0 * xsv, facc[q][0]);
           facc[q][1] = fmaf(static_cast<float>(iacc[q][1]), d1 * xsv, facc[q][1]);
           iacc[q][0] = iacc[q][1] = 0;
@@ -189,20 +426,15 @@ __device__ __forceinline__ bool gu_unit(const GuTmaArgs& a, const uint8_t* smem,
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       float v = facc[q][r];
-      if (TPG == 1) {
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-      } else if (TPG == 2) {
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-      }
+      if (TPG == 2) v += __shfl_xor_sync(0xffffffffu, v, 2);
       facc[q][r] = v;
     }
   const bool owner = (TPG == 4) || (tig < TPG);
 #pragma unroll
   for (int q = 0; q < MAXQ; ++q) {
-    const int tok = q * TPG + tslot_c;
-    if (q < ngroups && owner && tok < ne) {
-      float* out = a.gpart + ((static_cast<size_t>(p0 + tok) * 2 + m) * a.KP + kp) * I + rb * kBoxRows + row_l;
+    const int t = q * TPG + tslot_c;
+    if (q < ngroups && owner && t < ne) {
+      float* out = a.gpart + ((static_cast<size_t>(p0 + t) * 2 + w.m) * a.KP + w.kp) * I + w.rb * kBoxRows + row_l;
       out[0] = facc[q][0];
       out[8] = facc[q][1];
     }
@@ -210,22 +442,47 @@ __device__ __forceinline__ bool gu_unit(const GuTmaArgs& a, const uint8_t* smem,
   return true;
 }
 
-template <int MAXQ>
+
+// Shared-memory plan of the gate/up kernel's dynamic part (host and device
+// agree on it); the selector tables are static shared memory.
+struct GuPlan {
+  size_t meta, zero, x, xs, ring, bars, total;
+};
+__host__ __device__ inline GuPlan gu_plan(int E, int T, int k, int H, bool xs_in, int S) {
+  GuPlan p;
+  p.meta = 0;
+  p.zero = p.meta + meta_bytes(E, T * k, true);
+  p.x = p.zero + kZeroBytes;
+  p.xs = p.x + (xs_in ? align_up(static_cast<size_t>(T) * 2 * (H + kRowPad), 128) : 0);
+  const size_t end = p.xs + (xs_in ? align_up(static_cast<size_t>(T) * (H / 256) * 4, 128) : 0);
+  p.ring = align_up(end, 1024);
+  p.bars = p.ring + static_cast<size_t>(S) * kGuBox;
+  p.total = p.bars + 2 * static_cast<size_t>(S) * 8;
+  return p;
+}
+
+template <int MAXQ, bool XS>
 __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_constant__ CUtensorMap tm_gate,
                                                                   const __grid_constant__ CUtensorMap tm_up,
                                                                   GuTmaArgs a) {
+  // replicated selector tables at a fixed shared address, so lookups need no base add
+  __shared__ __align__(128) uint32_t s_tab[kTabWords];
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int H = a.H, I = a.I, T = a.T, S = a.S;
-  const size_t xb_bytes = a.x_in_smem ? align_up(static_cast<size_t>(T) * 2 * H, 128) : 0;
-  const size_t xs_bytes = a.x_in_smem ? align_up(static_cast<size_t>(T) * (H / 256) * 4, 128) : 0;
-  int8_t* xsm = reinterpret_cast<int8_t*>(smem + kXOff);
-  float* xssm = reinterpret_cast<float*>(smem + kXOff + xb_bytes);
-  uint8_t* ring = smem + align_up(kXOff + xb_bytes + xs_bytes, 1024);
-  uint64_t* full = reinterpret_cast<uint64_t*>(ring + static_cast<size_t>(S) * kGuBox);
+  const int H = a.H, I = a.I, T = a.T, S = a.S, NB = a.NB;
+  const int nA = T * a.k;
+  const GuPlan pl = gu_plan(a.E, T, a.k, H, XS, S);
+  MetaSmem ms;
+  ms.off = reinterpret_cast<int32_t*>(smem + pl.meta);
+  ms.act = ms.off + (a.E + 1);
+  ms.tok = ms.act + (a.E + 1);
+  int8_t* zero = reinterpret_cast<int8_t*>(smem + pl.zero);
+  int8_t* xsm = reinterpret_cast<int8_t*>(smem + pl.x);
+  float* xssm = reinterpret_cast<float*>(smem + pl.xs);
+  uint8_t* ring = smem + pl.ring;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + pl.bars);
   uint64_t* empty = full + S;
   const int rbs = I / kBoxRows;
-  const int nunits = a.active[a.E] * 2 * rbs * a.KP;
 
   if ((smem_addr(ring) & 1023u) != 0) {  // the 128-byte swizzle pattern assumes 1024-byte aligned boxes
     if (tid == 0) atomicCAS(a.err, 0, ERR_CUDA);
@@ -238,33 +495,32 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
     }
     fence_barrier_init();
   }
-  for (int i = tid; i < 256 * 32; i += kThreadsT)
-    reinterpret_cast<uint32_t*>(smem + kLvlOff)[i] = d_sel_tables2.level[i >> 5];
-  for (int i = tid; i < 128 * 32; i += kThreadsT)
-    reinterpret_cast<uint32_t*>(smem + kSgnOff)[i] = d_sel_tables2.sign[i >> 5];
-  if (a.x_in_smem) {
-    const int nx = T * 2 * H / 16;
-    for (int i = tid; i < nx; i += kThreadsT) reinterpret_cast<uint4*>(xsm)[i] = reinterpret_cast<const uint4*>(a.xd)[i];
+  for (int i = tid; i < 256 * 32; i += kThreadsT) s_tab[i] = d_sel_tables2.level[i >> 5];
+  for (int i = tid; i < 128 * 32; i += kThreadsT) s_tab[256 * 32 + i] = d_sel_tables2.sign[i >> 5];
+  for (int i = tid; i < kZeroBytes / 16; i += kThreadsT) reinterpret_cast<uint4*>(zero)[i] = make_uint4(0, 0, 0, 0);
+  load_meta(ms, a.offsets, a.active, a.perm, a.E, nA, a.k, tid, kThreadsT);
+  if (XS) {
+    stage_rows(xsm, a.xd, T * 2, H, tid, kThreadsT);
     for (int i = tid; i < T * (H / 256); i += kThreadsT) xssm[i] = a.xs[i];
   }
   __syncthreads();
+  const int nact = ms.act[a.E];
 
   if (warp == kCW) {  // producer
     if (lane == 0) {
       prefetch_tmap(&tm_gate);
       prefetch_tmap(&tm_up);
-      int it = 0;
-      for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-        const int kp = u % a.KP;
-        const int rest = u / a.KP;
-        const int rb = rest % rbs, m = (rest / rbs) & 1, slot = rest / rbs / 2;
-        const int e = a.active[slot];
-        for (int j = 0; j < 2; ++j, ++it) {
-          const int s = it % S;
-          if (!mbar_wait_bounded(&empty[s], ((it / S) & 1u) ^ 1u, a.err, ERR_TIMEOUT)) return;
-          mbar_arrive_expect_tx(&full[s], kGuBox);
-          tma_load_2d(ring + static_cast<size_t>(s) * kGuBox, m ? &tm_up : &tm_gate, kp * 256 + j * 128,
-                      e * I + rb * kBoxRows, &full[s]);
+      RingPos rp{0, 0u};
+      GuIter t;
+      t.init(blockIdx.x, gridDim.x, a.KP, rbs);
+      for (; t.slot < nact; t.next(a.KP, rbs)) {
+        const int e = ms.act[t.slot];
+        for (int j = 0; j < NB; ++j) {
+          if (!mbar_wait_bounded(&empty[rp.s], rp.ph ^ 1u, a.err, ERR_TIMEOUT)) return;
+          mbar_arrive_expect_tx(&full[rp.s], kGuBox);
+          tma_load_2d(ring + rp.s * kGuBox, t.m ? &tm_up : &tm_gate, (t.kp * NB + j) * kGuW, e * I + t.rb * kBoxRows,
+                      &full[rp.s]);
+          rp.next(S);
         }
       }
     }
@@ -272,11 +528,26 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
   }
 
   GuCtx c;
+  c.tab = reinterpret_cast<const char*>(s_tab);
   c.ring = ring;
   c.full = full;
   c.empty = empty;
-  c.xdig = a.x_in_smem ? xsm : a.xd;
-  c.xscl = a.x_in_smem ? xssm : a.xs;
+  if (XS) {
+    c.xdig = xsm;
+    c.xscl = xssm;
+    c.zero = zero;
+    c.xpitch = H + kRowPad;
+  } else {
+    c.xdig = a.xd;
+    c.xscl = a.xs;
+    c.zero = g_zero_operand;
+    c.xpitch = H;
+  }
+  c.ring_s = smem_addr(ring);
+  c.x_s = smem_addr(xsm);
+  c.xs_s = smem_addr(xssm);
+  c.zero_s = smem_addr(zero);
+  c.tok = ms.tok;
   c.warp = warp;
   c.lane = lane;
   c.g = lane >> 2;
@@ -285,24 +556,53 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
   c.lane4 = static_cast<uint32_t>(lane) << 2;
   c.rot_idx = (8u * c.tig - 7u) & 31u;
   c.rot_sig = (7u * c.tig - 7u) & 31u;
-  int it = 0;
-  for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-    const int kp = u % a.KP;
-    const int rest = u / a.KP;
-    const int rb = rest % rbs, m = (rest / rbs) & 1, slot = rest / rbs / 2;
-    const int e = a.active[slot];
-    const int p0 = a.offsets[e], ne = a.offsets[e + 1] - p0;
+  const int row_l = 16 * warp + c.g;
+  const int dstride = H / 256;
+  // per-row fp16 scales of a unit: for box j the pair of super-blocks 2(kp*NB+j), +1
+  auto dload = [&](const GuUnit& w, uint32_t (&d)[kMaxNB][2]) {
+    const uint16_t* dpl = w.m ? a.up_d : a.gate_d;
+    const size_t row = static_cast<size_t>(w.e) * I + w.rb * kBoxRows + row_l;
+    const uint16_t* r0 = dpl + row * dstride + 2 * w.kp * NB;
+    d[0][0] = __ldg(reinterpret_cast<const uint32_t*>(r0));
+    d[0][1] = __ldg(reinterpret_cast<const uint32_t*>(r0 + 8 * dstride));
+    if (NB > 1) {
+      d[1][0] = __ldg(reinterpret_cast<const uint32_t*>(r0 + 2));
+      d[1][1] = __ldg(reinterpret_cast<const uint32_t*>(r0 + 8 * dstride + 2));
+    }
+  };
+  RingPos rp{0, 0u};
+  GuIter t;
+  t.init(blockIdx.x, gridDim.x, a.KP, rbs);
+  uint32_t nd[kMaxNB][2] = {};
+  GuUnit nw{};
+  if (t.slot < nact) {
+    nw = gu_unit_of(t, ms);
+    dload(nw, nd);
+  }
+  while (t.slot < nact) {
+    const GuUnit w = nw;
+    uint32_t d[kMaxNB][2];
+#pragma unroll
+    for (int j = 0; j < kMaxNB; ++j) d[j][0] = nd[j][0], d[j][1] = nd[j][1];
+    t.next(a.KP, rbs);
+    if (t.slot < nact) {
+      nw = gu_unit_of(t, ms);
+      dload(nw, nd);
+    }
     bool ok;
-    if (MAXQ == 1 || ne == 1) ok = gu_unit<1, 1>(a, smem, c, it, e, m, rb, kp, p0, ne);
-    else if (ne == 2) ok = gu_unit<2, 1>(a, smem, c, it, e, m, rb, kp, p0, ne);
-    else ok = gu_unit<4, (MAXQ > 1 ? MAXQ : 1)>(a, smem, c, it, e, m, rb, kp, p0, ne);
+    if (XS && (MAXQ == 1 || w.ne == 1)) ok = gu_unit_one(a, c, rp, w, d);
+    else if (w.ne == 1) ok = gu_unit_multi<4, 1>(a, c, rp, w, d);
+    else if (w.ne == 2) ok = gu_unit_multi<2, 1>(a, c, rp, w, d);
+    else ok = gu_unit_multi<4, (MAXQ > 1 ? MAXQ : 1)>(a, c, rp, w, d);
     if (!ok) return;
   }
 }
 
-// ---------------------------------------------------------------------------
+// ===========================================================================
+// down
+// ===========================================================================
 struct DnTmaArgs {
-  int H, I, E, k, T, DP, S, h_in_smem;
+  int H, I, E, k, T, DP, NB, S;
   const uint32_t* dd;
   const int8_t* hd;
   const float* hsc;
@@ -314,154 +614,276 @@ struct DnTmaArgs {
   int hss;
 };
 
-template <int TPG, int MAXQ>
-__device__ __forceinline__ bool dn_unit(const DnTmaArgs& a, const uint8_t* ring, uint64_t* full, uint64_t* empty,
-                                        const int8_t* hd, const float* hsc, const int32_t* hq, int warp, int lane,
-                                        int& it, int e, int rb, int dp, int p0, int ne) {
-  constexpr int SPP = TPG == 1 ? 2 : 1;  // sub-block pairs per column set
-  const int H = a.H, I = a.I, S = a.S;
-  const int g = lane >> 2, tig = lane & 3;
-  const int ngroups = (ne + TPG - 1) / TPG;
+// Unit u = (slot * rbs + rb) * DP + dp, walked in steps of gridDim.x.
+struct DnIter {
+  int dp, rb, slot, ddp, drb, dslot;
+  __device__ __forceinline__ void init(int u0, int G, int DP, int rbs) {
+    dp = u0 % DP;
+    int r = u0 / DP;
+    rb = r % rbs;
+    slot = r / rbs;
+    ddp = G % DP;
+    r = G / DP;
+    drb = r % rbs;
+    dslot = r / rbs;
+  }
+  __device__ __forceinline__ void next(int DP, int rbs) {
+    dp += ddp;
+    int c = dp >= DP ? 1 : 0;
+    dp -= c * DP;
+    rb += drb + c;
+    c = rb >= rbs ? 1 : 0;
+    rb -= c * rbs;
+    slot += dslot + c;
+  }
+};
+
+struct DnUnit {
+  int e, rb, dp, p0, ne;
+};
+
+__device__ __forceinline__ DnUnit dn_unit_of(const DnIter& t, const MetaSmem& ms) {
+  DnUnit w;
+  w.dp = t.dp;
+  w.rb = t.rb;
+  w.e = ms.act[t.slot];
+  w.p0 = ms.off[w.e];
+  w.ne = ms.off[w.e + 1] - w.p0;
+  return w;
+}
+
+struct DnCtx {
+  const uint8_t* ring;
+  uint64_t* full;
+  uint64_t* empty;
+  const int8_t* hd;    // rows (assignment, digit) of I digits in MMA k order, pitch hpitch
+  const float* hsc;    // [T*k][hss]
+  const int32_t* hq;   // [T*k][I/16]
+  const int8_t* zero;  // 128-byte aligned zero region
+  uint32_t ring_s, hd_s, hsc_s, hq_s, zero_s;  // shared-window addresses (staged variant)
+  int hpitch, warp, lane, g, tig, S;
+};
+
+__device__ __forceinline__ float dn_block(uint32_t dd, float e2, int iA, int iM) {
+  return e2 * fmaf(half_lo(dd), static_cast<float>(iA), -half_hi(dd) * static_cast<float>(iM));
+}
+
+// One down unit for an expert with one assignment. MMA columns:
+// (pair slot 0..1) x (half 0..1) x (digit hi, lo); idle column halves read the
+// zero region.
+// One down unit for an expert with one assignment, h staged in shared memory.
+// MMA columns: (pair slot 0..1) x (half 0..1) x (digit hi, lo); idle column
+// halves read the zero region. All shared-memory addresses are 32-bit with
+// compile-time offsets.
+__device__ __forceinline__ bool dn_unit_one(const DnTmaArgs& a, const DnCtx& c, RingPos& rp, const DnUnit& w,
+                                            const uint32_t (&dd)[kMaxNB][2]) {
+  const int H = a.H, I = a.I, NB = a.NB;
+  const int g = c.g, tig = c.tig;
+  const int row_l = 16 * c.warp + g;
+  const uint32_t sh = 2 * tig;
+  const int sl_b = g >> 2, hb = (g >> 1) & 1, dig_b = g & 1;
+  const uint32_t hrow = c.hd_s + (w.p0 * 2 + dig_b) * c.hpitch + w.dp * NB * 256 + 8 * tig;
+  const uint32_t zrow = c.zero_s + ((64 * (w.p0 & 1) + 64) & 127) + 8 * tig;
+  const uint32_t hqr = c.hq_s + (w.p0 * (I / 16) + w.dp * NB * 16 + tig) * 4;
+  const uint32_t e2p = c.hsc_s + (w.p0 * a.hss + w.dp * NB) * 4;
+  float f0 = 0.f, f1 = 0.f;
+#pragma unroll 1
+  for (int j = 0; j < NB; ++j) {
+    uint32_t bp0[2], bp1[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      bp0[u] = (sl_b == u && hb == 0) ? hrow + j * 256 : zrow;
+      bp1[u] = (sl_b == u && hb == 1) ? hrow + j * 256 + 4 : zrow + 4;
+    }
+    if (!mbar_wait_bounded(&c.full[rp.s], rp.ph, a.err, ERR_TIMEOUT)) return false;
+    const uint32_t rA = c.ring_s + rp.s * kDnBox + row_l * kDnW, rB = rA + 8 * kDnW;
+    const int s = rp.s;
+    rp.next(c.S);
+    int iA0 = 0, iA1 = 0, iM0 = 0, iM1 = 0;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {  // 16 q bytes = four sub-blocks = two MMAs
+      const uint4 qa = ld_s128(rA + 16 + 16 * cc);
+      const uint4 qb = ld_s128(rB + 16 + 16 * cc);
+      uint32_t bv0[2], bv1[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        bv0[u] = ld_s32(bp0[u] + (2 * cc + u) * 32);
+        bv1[u] = ld_s32(bp1[u] + (2 * cc + u) * 32);
+      }
+      // this thread's columns: sub-block 4cc + tig (pair 2cc + tig/2, half tig&1)
+      const uint32_t scA = ld_s8(rA + 4 * cc + tig), scB = ld_s8(rB + 4 * cc + tig);
+      const int hqv = static_cast<int>(ld_s32(hqr + (j * 16 + 4 * cc) * 4));
+      int acc[4];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const uint32_t wa0 = u ? qa.z : qa.x, wa1 = u ? qa.w : qa.y;
+        const uint32_t wb0 = u ? qb.z : qb.x, wb1 = u ? qb.w : qb.y;
+        const uint32_t a0 = (wa0 >> sh) & 0x03030303u, a1 = (wb0 >> sh) & 0x03030303u;
+        const uint32_t a2 = (wa1 >> sh) & 0x03030303u, a3 = (wb1 >> sh) & 0x03030303u;
+        if (u == 0) mma_u8s8_zero(acc, a0, a1, a2, a3, bv0[u], bv1[u]);
+        else mma_u8s8(acc, a0, a1, a2, a3, bv0[u], bv1[u]);
+      }
+      iA0 += (acc[0] * 128 + acc[1]) * static_cast<int>(scA & 15u);
+      iA1 += (acc[2] * 128 + acc[3]) * static_cast<int>(scB & 15u);
+      iM0 += static_cast<int>(scA >> 4) * hqv;
+      iM1 += static_cast<int>(scB >> 4) * hqv;
+    }
+    const float e2 = ld_sf(e2p + j * 4);
+    __syncwarp();
+    if (c.lane == 0) mbar_arrive(&c.empty[s]);
+    const uint32_t dA = j ? dd[1][0] : dd[0][0], dB = j ? dd[1][1] : dd[0][1];
+    f0 += dn_block(dA, e2, iA0, iM0);
+    f1 += dn_block(dB, e2, iA1, iM1);
+  }
+  f0 += __shfl_xor_sync(0xffffffffu, f0, 1);
+  f0 += __shfl_xor_sync(0xffffffffu, f0, 2);
+  f1 += __shfl_xor_sync(0xffffffffu, f1, 1);
+  f1 += __shfl_xor_sync(0xffffffffu, f1, 2);
+  if (tig == 0) {
+    float* out = a.opart + (static_cast<size_t>(w.p0) * a.DP + w.dp) * H + w.rb * kBoxRows + row_l;
+    out[0] = f0;
+    out[8] = f1;
+  }
+  return true;
+}
+
+// One down unit for an expert with 2..2*MAXQ assignments. MMA columns:
+// (token slot 0..1) x (half 0..1) x (digit hi, lo).
+template <int MAXQ>
+__device__ __forceinline__ bool dn_unit_multi(const DnTmaArgs& a, const DnCtx& c, RingPos& rp, const DnUnit& w,
+                                              const uint32_t (&dd)[kMaxNB][2]) {
+  const int H = a.H, I = a.I, ne = w.ne, p0 = w.p0;
+  const int g = c.g, tig = c.tig;
+  const int ngroups = (ne + 1) / 2;
   const int dig_b = g & 1, hb = (g >> 1) & 1, sl_b = g >> 2;
   const int hc = tig & 1, sl_c = tig >> 1;
   const uint32_t sh = 2 * tig;
-  const int row_l = 16 * warp + g;
-  const size_t row_g = static_cast<size_t>(e) * H + rb * kBoxRows + row_l;
-  const int nblk = I / 256;
-  const uint2 ddA = *reinterpret_cast<const uint2*>(a.dd + row_g * nblk + dp * 2);
-  const uint2 ddB = *reinterpret_cast<const uint2*>(a.dd + (row_g + 8) * nblk + dp * 2);
-  const int8_t* hb_ptr[MAXQ];
-  bool hb_on[MAXQ];
-  const float* sc_ptr[MAXQ];
+  const int row_l = 16 * c.warp + g;
+  const int8_t* hrow[MAXQ];
+  bool b0on[MAXQ], b1on[MAXQ];
   const int32_t* hq_ptr[MAXQ];
+  const float* e2p[MAXQ];
 #pragma unroll
   for (int q = 0; q < MAXQ; ++q) {
-    const int tb = q * TPG + (TPG == 1 ? 0 : sl_b);
-    const int tc = q * TPG + (TPG == 1 ? 0 : sl_c);
-    hb_on[q] = q < ngroups && tb < ne;
-    hb_ptr[q] = hd + (static_cast<size_t>(p0 + (hb_on[q] ? tb : 0)) * 2 + dig_b) * I + 8 * tig + dp * 512;
+    const int tb = 2 * q + sl_b, tc = 2 * q + sl_c;
+    const bool on = q < ngroups && tb < ne;
+    hrow[q] = c.hd + ((p0 + (on ? tb : 0)) * 2 + dig_b) * c.hpitch + w.dp * a.NB * 256 + 8 * tig;
+    b0on[q] = on && hb == 0;
+    b1on[q] = on && hb == 1;
     const bool cv = q < ngroups && tc < ne;
-    sc_ptr[q] = cv ? hsc + static_cast<size_t>(p0 + tc) * a.hss + dp * 2 : nullptr;
-    hq_ptr[q] = cv ? hq + static_cast<size_t>(p0 + tc) * (I / 16) + dp * 32 : nullptr;
+    hq_ptr[q] = c.hq + (p0 + (cv ? tc : 0)) * (I / 16) + w.dp * a.NB * 16 + hc;
+    e2p[q] = cv ? c.hsc + (p0 + tc) * a.hss + w.dp * a.NB : nullptr;
   }
-  int acc[MAXQ][4];
-  int iA[MAXQ][2], iM[MAXQ][2];
+  const int8_t* zrow = c.zero + 8 * tig;
   float facc[MAXQ][2];
 #pragma unroll
-  for (int q = 0; q < MAXQ; ++q) {
-    acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0;
-    iA[q][0] = iA[q][1] = iM[q][0] = iM[q][1] = 0;
-    facc[q][0] = facc[q][1] = 0.f;
-  }
-  const int s = it % S;
-  if (!mbar_wait_bounded(&full[s], (it / S) & 1u, a.err, ERR_TIMEOUT)) return false;
-  const uint8_t* rA = ring + static_cast<size_t>(s) * kDnBox + row_l * 160;
-  const uint8_t* rB = rA + 8 * 160;
+  for (int q = 0; q < MAXQ; ++q) facc[q][0] = facc[q][1] = 0.f;
 #pragma unroll 1
-  for (int cc = 0; cc < 4; ++cc) {  // chunks of four sub-block pairs; 16 pairs = two blocks
-    uint32_t af[4][4];
+  for (int j = 0; j < a.NB; ++j) {
+    int acc[4];
+    int iA[MAXQ][2], iM[MAXQ][2];
 #pragma unroll
-    for (int u2 = 0; u2 < 2; ++u2) {
-      const int pr = 4 * cc + 2 * u2;
-      const int off = (pr >> 3) * 80 + 16 + 8 * (pr & 7);
-      const uint4 qa = *reinterpret_cast<const uint4*>(rA + off);
-      const uint4 qb = *reinterpret_cast<const uint4*>(rB + off);
-      af[2 * u2][0] = (qa.x >> sh) & 0x03030303u;
-      af[2 * u2][1] = (qb.x >> sh) & 0x03030303u;
-      af[2 * u2][2] = (qa.y >> sh) & 0x03030303u;
-      af[2 * u2][3] = (qb.y >> sh) & 0x03030303u;
-      af[2 * u2 + 1][0] = (qa.z >> sh) & 0x03030303u;
-      af[2 * u2 + 1][1] = (qb.z >> sh) & 0x03030303u;
-      af[2 * u2 + 1][2] = (qa.w >> sh) & 0x03030303u;
-      af[2 * u2 + 1][3] = (qb.w >> sh) & 0x03030303u;
+    for (int q = 0; q < MAXQ; ++q) iA[q][0] = iA[q][1] = iM[q][0] = iM[q][1] = 0;
+    if (!mbar_wait_bounded(&c.full[rp.s], rp.ph, a.err, ERR_TIMEOUT)) return false;
+    const int s = rp.s;
+    rp.next(c.S);
+    const uint8_t* rA = c.ring + s * kDnBox + row_l * kDnW;
+    const uint8_t* rB = rA + 8 * kDnW;
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+      const uint4 qa = lds128(rA + 16 + 16 * cc);
+      const uint4 qb = lds128(rB + 16 + 16 * cc);
+      uint32_t af[2][4];
+      af[0][0] = (qa.x >> sh) & 0x03030303u; af[0][1] = (qb.x >> sh) & 0x03030303u;
+      af[0][2] = (qa.y >> sh) & 0x03030303u; af[0][3] = (qb.y >> sh) & 0x03030303u;
+      af[1][0] = (qa.z >> sh) & 0x03030303u; af[1][1] = (qb.z >> sh) & 0x03030303u;
+      af[1][2] = (qa.w >> sh) & 0x03030303u; af[1][3] = (qb.w >> sh) & 0x03030303u;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int pr = 2 * cc + u;
+        // this thread's columns: sub-block 2*pr + hc of token 2q + sl_c
+        const int sub = 2 * pr + hc;
+        const uint32_t scA = rA[sub], scB = rB[sub];
+#pragma unroll
+        for (int q = 0; q < MAXQ; ++q) {
+          if (q >= ngroups) break;
+          const int8_t* p0b = b0on[q] ? hrow[q] + j * 256 : zrow;
+          const int8_t* p1b = b1on[q] ? hrow[q] + j * 256 + 4 : zrow + 4;
+          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(p0b + pr * 32);
+          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(p1b + pr * 32);
+          mma_u8s8_zero(acc, af[u][0], af[u][1], af[u][2], af[u][3], b0, b1);
+          const int hqv = hq_ptr[q][j * 16 + 2 * pr];
+          iA[q][0] += (acc[0] * 128 + acc[1]) * static_cast<int>(scA & 15u);
+          iA[q][1] += (acc[2] * 128 + acc[3]) * static_cast<int>(scB & 15u);
+          iM[q][0] += static_cast<int>(scA >> 4) * hqv;
+          iM[q][1] += static_cast<int>(scB >> 4) * hqv;
+        }
+      }
     }
+    __syncwarp();
+    if (c.lane == 0) mbar_arrive(&c.empty[s]);
+    const uint32_t dA = j ? dd[1][0] : dd[0][0], dB = j ? dd[1][1] : dd[0][1];
 #pragma unroll
     for (int q = 0; q < MAXQ; ++q) {
-      if (q >= ngroups) break;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int pr = 4 * cc + u, slot = u % SPP;
-        uint2 bv = make_uint2(0u, 0u);
-        if (hb_on[q] && (SPP == 1 || slot == sl_b)) {
-          bv = *reinterpret_cast<const uint2*>(hb_ptr[q] + pr * 32);
-          if (hb) bv.x = 0u; else bv.y = 0u;
-        }
-        mma_u8s8(acc[q], af[u][0], af[u][1], af[u][2], af[u][3], bv.x, bv.y);
-        if (slot == SPP - 1) {
-          const int sub = 2 * (pr - (SPP - 1) + (TPG == 1 ? sl_c : 0)) + hc;  // sub-block inside the two blocks
-          const int bb = sub >> 4, si = sub & 15;
-          const uint32_t scA = rA[bb * 80 + si], scB = rB[bb * 80 + si];
-          if (hq_ptr[q]) {
-            const int hqv = hq_ptr[q][sub];
-            iA[q][0] += (acc[q][0] * 128 + acc[q][1]) * static_cast<int>(scA & 15u);
-            iA[q][1] += (acc[q][2] * 128 + acc[q][3]) * static_cast<int>(scB & 15u);
-            iM[q][0] += static_cast<int>(scA >> 4) * hqv;
-            iM[q][1] += static_cast<int>(scB >> 4) * hqv;
-          }
-          acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0;
-        }
-      }
-    }
-    if (cc & 1) {
-      // block (super-block) done: 2^e * (d * A - dmin * M)
-      const int bl = cc >> 1;
-      const uint32_t wA = bl ? ddA.y : ddA.x, wB = bl ? ddB.y : ddB.x;
-      const float dA = half_bits_to_float(static_cast<uint16_t>(wA & 0xFFFFu));
-      const float nA = half_bits_to_float(static_cast<uint16_t>(wA >> 16));
-      const float dB = half_bits_to_float(static_cast<uint16_t>(wB & 0xFFFFu));
-      const float nB = half_bits_to_float(static_cast<uint16_t>(wB >> 16));
-#pragma unroll
-      for (int q = 0; q < MAXQ; ++q) {
-        const float e2 = sc_ptr[q] ? sc_ptr[q][bl] : 0.f;
-        facc[q][0] = fmaf(e2, fmaf(dA, static_cast<float>(iA[q][0]), -nA * static_cast<float>(iM[q][0])), facc[q][0]);
-        facc[q][1] = fmaf(e2, fmaf(dB, static_cast<float>(iA[q][1]), -nB * static_cast<float>(iM[q][1])), facc[q][1]);
-        iA[q][0] = iA[q][1] = iM[q][0] = iM[q][1] = 0;
-      }
+      const float e2 = e2p[q] ? e2p[q][j] : 0.f;
+      facc[q][0] += dn_block(dA, e2, iA[q][0], iM[q][0]);
+      facc[q][1] += dn_block(dB, e2, iA[q][1], iM[q][1]);
     }
   }
-  __syncwarp();
-  if (lane == 0) mbar_arrive(&empty[s]);
-  ++it;
-#pragma unroll
-  for (int q = 0; q < MAXQ; ++q)
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      float v = facc[q][r];
-      v += __shfl_xor_sync(0xffffffffu, v, 1);
-      if (TPG == 1) v += __shfl_xor_sync(0xffffffffu, v, 2);
-      facc[q][r] = v;
-    }
-  const bool owner = TPG == 1 ? (tig == 0) : (hc == 0);
 #pragma unroll
   for (int q = 0; q < MAXQ; ++q) {
-    const int tok = q * TPG + (TPG == 1 ? 0 : sl_c);
-    if (q < ngroups && owner && tok < ne) {
-      float* out = a.opart + (static_cast<size_t>(p0 + tok) * a.DP + dp) * H + rb * kBoxRows + row_l;
-      out[0] = facc[q][0];
-      out[8] = facc[q][1];
+    if (q >= ngroups) break;
+    float f0 = facc[q][0], f1 = facc[q][1];
+    f0 += __shfl_xor_sync(0xffffffffu, f0, 1);
+    f1 += __shfl_xor_sync(0xffffffffu, f1, 1);
+    const int t = 2 * q + sl_c;
+    if (hc == 0 && t < ne) {
+      float* out = a.opart + (static_cast<size_t>(p0 + t) * a.DP + w.dp) * H + w.rb * kBoxRows + row_l;
+      out[0] = f0;
+      out[8] = f1;
     }
   }
   return true;
 }
 
-template <int MAXQ>
+// Shared-memory plan of the down kernel.
+struct DnPlan {
+  size_t meta, zero, hd, hsc, hq, ring, bars, total;
+};
+__host__ __device__ inline DnPlan dn_plan(int E, int nA, int I, int hss, bool hs_in, int S) {
+  DnPlan p;
+  p.meta = 0;
+  p.zero = meta_bytes(E, nA, false);
+  p.hd = p.zero + kZeroBytes;
+  p.hsc = p.hd + (hs_in ? align_up(static_cast<size_t>(nA) * 2 * (I + kRowPad), 128) : 0);
+  p.hq = p.hsc + (hs_in ? align_up(static_cast<size_t>(nA) * hss * 4, 128) : 0);
+  const size_t end = p.hq + (hs_in ? align_up(static_cast<size_t>(nA) * (I / 16) * 4, 128) : 0);
+  p.ring = align_up(end, 1024);
+  p.bars = p.ring + static_cast<size_t>(S) * kDnBox;
+  p.total = p.bars + 2 * static_cast<size_t>(S) * 8;
+  return p;
+}
+
+template <int MAXQ, bool HS>
 __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_constant__ CUtensorMap tm_down,
                                                                 DnTmaArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int H = a.H, I = a.I, S = a.S;
+  const int H = a.H, I = a.I, S = a.S, NB = a.NB;
   const int nA = a.T * a.k;
-  const size_t hd_bytes = a.h_in_smem ? align_up(static_cast<size_t>(nA) * 2 * I, 128) : 0;
-  const size_t hsc_bytes = a.h_in_smem ? align_up(static_cast<size_t>(nA) * a.hss * 4, 128) : 0;
-  const size_t hq_bytes = a.h_in_smem ? align_up(static_cast<size_t>(nA) * (I / 16) * 4, 128) : 0;
-  int8_t* hd_s = reinterpret_cast<int8_t*>(smem);
-  float* hsc_s = reinterpret_cast<float*>(smem + hd_bytes);
-  int32_t* hq_s = reinterpret_cast<int32_t*>(smem + hd_bytes + hsc_bytes);
-  uint8_t* ring = smem + align_up(hd_bytes + hsc_bytes + hq_bytes, 1024);
-  uint64_t* full = reinterpret_cast<uint64_t*>(ring + static_cast<size_t>(S) * kDnBox);
+  const DnPlan pl = dn_plan(a.E, nA, I, a.hss, HS, S);
+  MetaSmem ms;
+  ms.off = reinterpret_cast<int32_t*>(smem + pl.meta);
+  ms.act = ms.off + (a.E + 1);
+  ms.tok = nullptr;
+  int8_t* zero = reinterpret_cast<int8_t*>(smem + pl.zero);
+  int8_t* hd_s = reinterpret_cast<int8_t*>(smem + pl.hd);
+  float* hsc_s = reinterpret_cast<float*>(smem + pl.hsc);
+  int32_t* hq_s = reinterpret_cast<int32_t*>(smem + pl.hq);
+  uint8_t* ring = smem + pl.ring;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + pl.bars);
   uint64_t* empty = full + S;
   const int rbs = H / kBoxRows;
-  const int nunits = a.active[a.E] * rbs * a.DP;
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -470,44 +892,95 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
     }
     fence_barrier_init();
   }
-  if (a.h_in_smem) {
-    for (int i = tid; i < nA * 2 * I / 16; i += kThreadsT)
-      reinterpret_cast<uint4*>(hd_s)[i] = reinterpret_cast<const uint4*>(a.hd)[i];
+  for (int i = tid; i < kZeroBytes / 16; i += kThreadsT) reinterpret_cast<uint4*>(zero)[i] = make_uint4(0, 0, 0, 0);
+  load_meta(ms, a.offsets, a.active, nullptr, a.E, nA, a.k, tid, kThreadsT);
+  if (HS) {
+    stage_rows(hd_s, a.hd, nA * 2, I, tid, kThreadsT);
     for (int i = tid; i < nA * a.hss; i += kThreadsT) hsc_s[i] = a.hsc[i];
     for (int i = tid; i < nA * (I / 16); i += kThreadsT) hq_s[i] = a.hq[i];
   }
   __syncthreads();
+  const int nact = ms.act[a.E];
 
   if (warp == kCW) {  // producer
     if (lane == 0) {
       prefetch_tmap(&tm_down);
-      int it = 0;
-      for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
-        const int dp = u % a.DP;
-        const int rest = u / a.DP;
-        const int rb = rest % rbs, slot = rest / rbs;
-        const int e = a.active[slot];
-        const int s = it % S;
-        if (!mbar_wait_bounded(&empty[s], ((it / S) & 1u) ^ 1u, a.err, ERR_TIMEOUT)) return;
-        mbar_arrive_expect_tx(&full[s], kDnBox);
-        tma_load_2d(ring + static_cast<size_t>(s) * kDnBox, &tm_down, dp * 160, e * H + rb * kBoxRows, &full[s]);
+      RingPos rp{0, 0u};
+      DnIter t;
+      t.init(blockIdx.x, gridDim.x, a.DP, rbs);
+      for (; t.slot < nact; t.next(a.DP, rbs)) {
+        const int e = ms.act[t.slot];
+        for (int j = 0; j < NB; ++j) {
+          if (!mbar_wait_bounded(&empty[rp.s], rp.ph ^ 1u, a.err, ERR_TIMEOUT)) return;
+          mbar_arrive_expect_tx(&full[rp.s], kDnBox);
+          tma_load_2d(ring + rp.s * kDnBox, &tm_down, (t.dp * NB + j) * kDnW, e * H + t.rb * kBoxRows, &full[rp.s]);
+          rp.next(S);
+        }
       }
     }
     return;
   }
-  const int8_t* hd = a.h_in_smem ? hd_s : a.hd;
-  const float* hsc = a.h_in_smem ? hsc_s : a.hsc;
-  const int32_t* hq = a.h_in_smem ? hq_s : a.hq;
-  int it = 0;
-  for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-    const int dp = u % a.DP;
-    const int rest = u / a.DP;
-    const int rb = rest % rbs, slot = rest / rbs;
-    const int e = a.active[slot];
-    const int p0 = a.offsets[e], ne = a.offsets[e + 1] - p0;
+  DnCtx c;
+  c.ring = ring;
+  c.ring_s = smem_addr(ring);
+  c.full = full;
+  c.empty = empty;
+  if (HS) {
+    c.hd = hd_s;
+    c.hsc = hsc_s;
+    c.hq = hq_s;
+    c.zero = zero;
+    c.hpitch = I + kRowPad;
+    c.hd_s = smem_addr(hd_s);
+    c.hsc_s = smem_addr(hsc_s);
+    c.hq_s = smem_addr(hq_s);
+    c.zero_s = smem_addr(zero);
+  } else {
+    c.hd = a.hd;
+    c.hsc = a.hsc;
+    c.hq = a.hq;
+    c.zero = g_zero_operand;
+    c.hpitch = I;
+  }
+  c.warp = warp;
+  c.lane = lane;
+  c.g = lane >> 2;
+  c.tig = lane & 3;
+  c.S = S;
+  const int row_l = 16 * warp + c.g;
+  const int nblk = I / 256;
+  auto ddload = [&](const DnUnit& w, uint32_t (&d)[kMaxNB][2]) {
+    const size_t row = static_cast<size_t>(w.e) * H + w.rb * kBoxRows + row_l;
+    const uint32_t* r0 = a.dd + row * nblk + w.dp * NB;
+    d[0][0] = __ldg(r0);
+    d[0][1] = __ldg(r0 + 8 * nblk);
+    if (NB > 1) {
+      d[1][0] = __ldg(r0 + 1);
+      d[1][1] = __ldg(r0 + 8 * nblk + 1);
+    }
+  };
+  RingPos rp{0, 0u};
+  DnIter t;
+  t.init(blockIdx.x, gridDim.x, a.DP, rbs);
+  uint32_t nd[kMaxNB][2] = {};
+  DnUnit nw{};
+  if (t.slot < nact) {
+    nw = dn_unit_of(t, ms);
+    ddload(nw, nd);
+  }
+  while (t.slot < nact) {
+    const DnUnit w = nw;
+    uint32_t d[kMaxNB][2];
+#pragma unroll
+    for (int j = 0; j < kMaxNB; ++j) d[j][0] = nd[j][0], d[j][1] = nd[j][1];
+    t.next(a.DP, rbs);
+    if (t.slot < nact) {
+      nw = dn_unit_of(t, ms);
+      ddload(nw, nd);
+    }
     bool ok;
-    if (MAXQ == 1 || ne == 1) ok = dn_unit<1, 1>(a, ring, full, empty, hd, hsc, hq, warp, lane, it, e, rb, dp, p0, ne);
-    else ok = dn_unit<2, (MAXQ > 1 ? MAXQ : 1)>(a, ring, full, empty, hd, hsc, hq, warp, lane, it, e, rb, dp, p0, ne);
+    if (HS && (MAXQ == 1 || w.ne == 1)) ok = dn_unit_one(a, c, rp, w, d);
+    else ok = dn_unit_multi<(MAXQ > 1 ? MAXQ : 1)>(a, c, rp, w, d);
     if (!ok) return;
   }
 }
@@ -544,43 +1017,64 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t row
 
 constexpr size_t kBudget = 227 * 1024;
 
+int nb_for(int T) { return T == 1 ? 1 : 2; }
+
+template <typename K>
+void launch_k(K kern, int grid, size_t smem, cudaStream_t st, const CUtensorMap& m0, const CUtensorMap& m1,
+              const GuTmaArgs& a) {
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  kern<<<grid, kThreadsT, smem, st>>>(m0, m1, a);
+}
+
+template <typename K>
+void launch_k(K kern, int grid, size_t smem, cudaStream_t st, const CUtensorMap& m0, const DnTmaArgs& a) {
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  kern<<<grid, kThreadsT, smem, st>>>(m0, a);
+}
+
 }  // namespace
 
 bool tma_path_supported(const LayerShape& s, int T) {
-  return s.H % 1024 == 0 && s.I % 512 == 0 && T <= 16 && encode_fn() != nullptr;
+  return s.H % 1024 == 0 && s.I % 512 == 0 && T >= 1 && T <= 16 && s.E <= kMaxExpertsTma &&
+         encode_fn() != nullptr;
 }
-// A gate/up unit covers 1024 of H and a down unit 512 of I, so the reduction
-// axis is always split into this many parts.
-int tma_gu_parts(const LayerShape& s, int) { return s.H / 1024; }
-int tma_dn_parts(const LayerShape& s, int) { return s.I / 512; }
+// A gate/up unit covers NB*512 of H and a down unit NB*256 of I, so the
+// reduction axis is always split into this many parts.
+int tma_gu_parts(const LayerShape& s, int T) { return s.H / (512 * nb_for(T)); }
+int tma_dn_parts(const LayerShape& s, int T) { return s.I / (256 * nb_for(T)); }
 
 int launch_gateup_tma(const LayerShape& sh, const uint8_t* gate_codes, const uint16_t* gate_d,
                       const uint8_t* up_codes, const uint16_t* up_d, const int8_t* xd, const float* xs, int T,
                       const Routing& r, float* gpart, int* err, int sms, cudaStream_t st) {
   CUtensorMap tg, tu;
   const uint64_t rb = sh.H / 4, rows = static_cast<uint64_t>(sh.E) * sh.I;
-  if (!make_map(&tg, gate_codes, rb, rows, 128, kBoxRows, true) || !make_map(&tu, up_codes, rb, rows, 128, kBoxRows, true))
+  if (!make_map(&tg, gate_codes, rb, rows, kGuW, kBoxRows, true) ||
+      !make_map(&tu, up_codes, rb, rows, kGuW, kBoxRows, true))
     return ERR_CUDA;
   GuTmaArgs a{};
-  a.H = sh.H; a.I = sh.I; a.E = sh.E; a.k = sh.k; a.T = T; a.KP = tma_gu_parts(sh, T);
+  a.H = sh.H; a.I = sh.I; a.E = sh.E; a.k = sh.k; a.T = T;
+  a.NB = nb_for(T); a.KP = tma_gu_parts(sh, T);
   a.gate_d = gate_d; a.up_d = up_d; a.xd = xd; a.xs = xs;
   a.offsets = r.offsets; a.perm = r.perm; a.active = r.active; a.gpart = gpart; a.err = err;
-  const size_t xbytes = align_up(static_cast<size_t>(T) * 2 * sh.H, 128) + align_up(static_cast<size_t>(T) * (sh.H / 256) * 4, 128);
-  a.x_in_smem = (kXOff + xbytes + 4 * kGuBox + 1024 <= kBudget) ? 1 : 0;
-  const size_t ring_off = align_up(kXOff + (a.x_in_smem ? xbytes : 0), 1024);
-  int S = static_cast<int>((kBudget - ring_off - 256) / kGuBox);
-  S = std::max(2, std::min(S, 10));
+  // stage the activations when that still leaves three ring stages
+  const size_t budget = kBudget - kTabWords * 4;  // the selector tables are static shared memory
+  const bool xs_in = gu_plan(sh.E, T, sh.k, sh.H, true, 3).total <= budget;
+  int S = 2;
+  while (S < 6 && gu_plan(sh.E, T, sh.k, sh.H, xs_in, S + 1).total <= budget) ++S;
+  if (gu_plan(sh.E, T, sh.k, sh.H, xs_in, S).total > budget) return ERR_SHAPE;
   a.S = S;
-  const size_t smem = ring_off + static_cast<size_t>(S) * kGuBox + 2 * S * 8;
-  const int slots = static_cast<int>(std::min<size_t>(static_cast<size_t>(T) * sh.k, static_cast<size_t>(sh.E)));
+  const size_t smem = gu_plan(sh.E, T, sh.k, sh.H, xs_in, S).total;
+  const size_t nA = static_cast<size_t>(T) * sh.k;
+  const int slots = static_cast<int>(std::min<size_t>(nA, static_cast<size_t>(sh.E)));
   const int units = slots * 2 * (sh.I / kBoxRows) * a.KP;
   const int grid = std::max(1, std::min(units, sms));
-  if (T == 1) {
-    cudaFuncSetAttribute(gateup_tma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    gateup_tma_kernel<1><<<grid, kThreadsT, smem, st>>>(tg, tu, a);
-  } else {  // at most 16 tokens per expert: four groups of four
-    cudaFuncSetAttribute(gateup_tma_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    gateup_tma_kernel<4><<<grid, kThreadsT, smem, st>>>(tg, tu, a);
+  if (T == 1) {  // one token: the single-assignment variant with staged activations
+    if (!xs_in) return ERR_SHAPE;
+    launch_k(gateup_tma_kernel<1, true>, grid, smem, st, tg, tu, a);
+  } else if (xs_in) {  // at most 16 tokens per expert: four groups of four
+    launch_k(gateup_tma_kernel<4, true>, grid, smem, st, tg, tu, a);
+  } else {
+    launch_k(gateup_tma_kernel<4, false>, grid, smem, st, tg, tu, a);
   }
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
 }
@@ -589,30 +1083,30 @@ int launch_down_tma(const LayerShape& sh, const uint8_t* down_codes, const uint3
                     const float* hsc, const int32_t* hq, int hss, int T, const Routing& r, float* opart, int* err,
                     int sms, cudaStream_t st) {
   CUtensorMap td;
-  const uint64_t rb = static_cast<uint64_t>(sh.I / 256) * 80, rows = static_cast<uint64_t>(sh.E) * sh.H;
-  if (!make_map(&td, down_codes, rb, rows, 160, kBoxRows, false)) return ERR_CUDA;
+  const uint64_t rb = static_cast<uint64_t>(sh.I / 256) * kDnW, rows = static_cast<uint64_t>(sh.E) * sh.H;
+  if (!make_map(&td, down_codes, rb, rows, kDnW, kBoxRows, false)) return ERR_CUDA;
   DnTmaArgs a{};
-  a.H = sh.H; a.I = sh.I; a.E = sh.E; a.k = sh.k; a.T = T; a.DP = tma_dn_parts(sh, T); a.hss = hss;
+  a.H = sh.H; a.I = sh.I; a.E = sh.E; a.k = sh.k; a.T = T; a.hss = hss;
+  a.NB = nb_for(T); a.DP = tma_dn_parts(sh, T);
   a.dd = down_dd; a.hd = hd; a.hsc = hsc; a.hq = hq;
   a.offsets = r.offsets; a.active = r.active; a.opart = opart; a.err = err;
-  const size_t nA = static_cast<size_t>(T) * sh.k;
-  const size_t hbytes = align_up(nA * 2 * sh.I, 128) + align_up(nA * hss * 4, 128) + align_up(nA * (sh.I / 16) * 4, 128);
-  a.h_in_smem = (hbytes + 4 * kDnBox + 1024 <= kBudget) ? 1 : 0;
-  const size_t ring_off = align_up(a.h_in_smem ? hbytes : 0, 1024);
-  int S = static_cast<int>((kBudget - ring_off - 256) / kDnBox);
-  S = std::max(2, std::min(S, 8));
+  const int nA = T * sh.k;
+  const bool hs_in = dn_plan(sh.E, nA, sh.I, hss, true, 4).total <= kBudget;
+  int S = 2;
+  while (S < 8 && dn_plan(sh.E, nA, sh.I, hss, hs_in, S + 1).total <= kBudget) ++S;
+  if (dn_plan(sh.E, nA, sh.I, hss, hs_in, S).total > kBudget) return ERR_SHAPE;
   a.S = S;
-  const size_t smem = ring_off + static_cast<size_t>(S) * kDnBox + 2 * S * 8;
-  const int slots = static_cast<int>(std::min<size_t>(nA, static_cast<size_t>(sh.E)));
+  const size_t smem = dn_plan(sh.E, nA, sh.I, hss, hs_in, S).total;
+  const int slots = std::min(nA, sh.E);
   const int units = slots * (sh.H / kBoxRows) * a.DP;
   const int grid = std::max(1, std::min(units, sms));
-  if (T == 1) {
-    cudaFuncSetAttribute(down_tma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    down_tma_kernel<1><<<grid, kThreadsT, smem, st>>>(td, a);
+  if (T == 1) {  // one token: the single-assignment variant with h staged
+    if (!hs_in) return ERR_SHAPE;
+    launch_k(down_tma_kernel<1, true>, grid, smem, st, td, a);
+  } else if (hs_in) {  // at most 16 tokens per expert: eight groups of two
+    launch_k(down_tma_kernel<8, true>, grid, smem, st, td, a);
   } else {
-    // at most 16 tokens per expert: eight groups of two
-    cudaFuncSetAttribute(down_tma_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    down_tma_kernel<8><<<grid, kThreadsT, smem, st>>>(td, a);
+    launch_k(down_tma_kernel<8, false>, grid, smem, st, td, a);
   }
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
 }
