@@ -129,6 +129,29 @@ def traffic_record(kernel: str):
         return None
 
 
+# ------------------------------------------------------------ multi-rank
+def max_over_ranks(vals, world, device):
+    """Element-wise max of per-rank timings; every rank calls it at the same
+    point (one all-reduce of a few scalars, outside the data path)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def job_tokens_per_s(tokens_per_rank_step, world, ms_per_step):
+    """Whole-job throughput: every rank processes its own tokens (replicas)."""
+    return tokens_per_rank_step * world / (ms_per_step * 1e-3)
+
+
+def rank_seed(cfg_seed, rank):
+    """Input seed of a rank: replicas work on distinct synthetic tokens."""
+    return cfg_seed + 7919 * rank
+
+
 # --------------------------------------------------------------- reference
 def run_reference(args, cfg):
     import oracle
@@ -206,7 +229,7 @@ def run_ours(args, cfg):
         layers.append(moe2bit.to_device(lw))
         del lw
     n_slots = 4
-    xs_host = [synth.make_x_fast(cfg, T, layer=100 + s, cfg_seed=cfg.seed + 7919 * rank) for s in range(n_slots)]
+    xs_host = [synth.make_x_fast(cfg, T, layer=100 + s, cfg_seed=rank_seed(cfg.seed, rank)) for s in range(n_slots)]
     xdt = torch.bfloat16 if cfg.x_dtype == "bf16" else torch.float32
 
     def dev_x(a):
@@ -320,10 +343,7 @@ def run_ours(args, cfg):
     ms_e2e = e0.elapsed_time(e1) / args.steps
     clocks = clk.stop()
 
-    mx = torch.tensor([ms, ms_e2e], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-    ms, ms_e2e = float(mx[0]), float(mx[1])
+    ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, "cuda")
 
     # realised active experts per step, from the library's own routing
     act = []
@@ -365,7 +385,7 @@ def run_ours(args, cfg):
         n_layers if cfg.name == "stack" else 1)
     bytes_x = T * cfg.H * (2 if cfg.x_dtype == "bf16" else 4)
     line = {
-        "metric": "moe_layer_tokens_per_s", "value": tokens_per_step * world / (ms * 1e-3), "unit": "tokens/s",
+        "metric": "moe_layer_tokens_per_s", "value": job_tokens_per_s(tokens_per_step, world, ms), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
         "config": {"workload": cfg.name, "tokens_per_step": T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
@@ -378,7 +398,7 @@ def run_ours(args, cfg):
         "kernels": {k: {"avg_ms": avg_ms[k], "launches_per_step": launches_per_step[k]} for k in prof},
         "gpu_launches": int(round(sum(launches_per_step.values()) * args.steps)),
         "clocks": clocks,
-        "e2e": {"value": tokens_per_step * world / (ms_e2e * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(tokens_per_step, world, ms_e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": bytes_x, "d2h_bytes_per_step": T * cfg.H * 4},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

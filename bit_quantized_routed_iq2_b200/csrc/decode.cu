@@ -497,7 +497,7 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
   // bf16 activations feed the shared expert's MMAs as one part, fp32 as two
   const int xparts = x_dtype == 0 ? 2 : 1;
   const uint16_t* xbp = x_dtype == 0 ? fw.xb : static_cast<const uint16_t*>(x);
-  const bool sh_mma = s.Is > 0 && shared_mma_supported(s.H, s.Is, T, xparts);
+  const bool sh_mma = s.Is > 0 && shared_mma_supported(s.H, s.Is, T, xparts, s.k);
   if (tma) {
     ProfScope ps(MOE_K_GATEUP, st);
     rc |= launch_gateup_tma(s, w.gate_codes, w.gate_d, w.up_codes, w.up_d, xd, xs, T, r, gu, err, sms, st);

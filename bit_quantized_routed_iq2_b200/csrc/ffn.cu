@@ -11,6 +11,8 @@
 // lanes striding over 8-weight groups along the reduction axis. It is the path
 // for shapes the tuned kernels do not cover and the baseline they are measured
 // against.
+#include <algorithm>
+
 #include "common.cuh"
 #include "dequant.cuh"
 #include "kernels.cuh"
@@ -233,8 +235,14 @@ static size_t simple_ffn_workspace_bytes(const LayerShape& s, int T) {
   return b;
 }
 
+// Token counts above the decode GEMVs' range go through the tensor-core grouped
+// GEMM (prefill.cu) when the shape allows it.
+static bool use_prefill(const LayerShape& s, int T) { return T > kPrefillMinT && prefill_path_supported(s, T); }
+
 size_t ffn_workspace_bytes(const LayerShape& s, int T) {
-  return fast_path_supported(s) ? fast_ffn_workspace_bytes(s, T) : simple_ffn_workspace_bytes(s, T);
+  size_t b = fast_path_supported(s) ? fast_ffn_workspace_bytes(s, T) : simple_ffn_workspace_bytes(s, T);
+  if (use_prefill(s, T)) b = std::max(b, prefill_workspace_bytes(s, T));
+  return b;
 }
 
 static int launch_ffn_simple(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T,
@@ -288,6 +296,12 @@ static int launch_ffn_simple(const LayerShape& s, const WeightPtrs& w, const voi
 
 int launch_ffn(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
                const float* residual, float* y, void* ws, int* err, cudaStream_t st) {
+  if (use_prefill(s, T)) {
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return launch_ffn_prefill(s, w, x, x_dtype, T, r, residual, y, ws, err, sms > 0 ? sms : 148, st);
+  }
   if (fast_path_supported(s)) return launch_ffn_fast(s, w, x, x_dtype, T, r, residual, y, ws, err, st);
   return launch_ffn_simple(s, w, x, x_dtype, T, r, residual, y, ws, st);
 }

@@ -61,12 +61,19 @@ int launch_down_tma(const LayerShape& sh, const uint8_t* down_codes, const uint3
 
 // Shared expert on bf16 warp MMAs for up to 32 tokens (shared_mma.cu). xb holds
 // P bf16 parts of x as [P][T][H]; hb receives h as two parts [2][T][Is].
-bool shared_mma_supported(int H, int Is, int T, int x_parts);
+bool shared_mma_supported(int H, int Is, int T, int x_parts, int k);
 int launch_shared_gateup_mma(int H, int Is, const uint16_t* wg, const uint16_t* wu, const uint16_t* xb, int P,
                              int T, uint16_t* hb, cudaStream_t st);
 int launch_shared_down_combine_mma(int H, int Is, const uint16_t* wd, const uint16_t* hb, int T, int k,
                                    const float* topk_w, const int32_t* inv, const float* obuf, int DP,
                                    const float* residual, float* y, cudaStream_t st);
+
+// Tensor-core grouped GEMM for many tokens (prefill.cu).
+constexpr int kPrefillMinT = 16;
+bool prefill_path_supported(const LayerShape& s, int T);
+size_t prefill_workspace_bytes(const LayerShape& s, int T);
+int launch_ffn_prefill(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
+                       const float* residual, float* y, void* ws, int* err, int sms, cudaStream_t st);
 
 int launch_debug_dequant_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, float* out, cudaStream_t st);
 int launch_debug_dequant_q2k(const uint8_t* codes, const uint32_t* dd, int64_t nblocks, float* out,

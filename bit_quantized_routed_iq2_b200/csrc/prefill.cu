@@ -1,0 +1,730 @@
+// prefill.cu - the many-token path: a grouped GEMM per routed expert on the
+// 5th-generation tensor cores (tcgen05.mma kind::f16, accumulators in TMEM),
+// with the 2-bit expert tiles dequantised into shared memory by dedicated
+// warps, and the unquantized shared expert as a dense GEMM on the same engine.
+//
+// Sources: "ds4 : analyse pratique pour un usage documenté", section « Support
+// de modèles et choix de quantification » (routed up/gate IQ2_XXS, down Q2_K;
+// shared expert unquantized); "Un modèle de 284 milliards de paramètres tourne
+// désormais sur un Mac de 128 Go. Qui y perd ?", section « Comment un modèle de
+// 284 milliards de paramètres tient sur une seule machine » (each token uses a
+// few routed experts). The weight formats are the library's own (see dequant.cuh).
+//
+// Weights are the M operand (128 rows per tile) and the tokens routed to an
+// expert are the N operand (up to 128 per tile), so one dequantised weight tile
+// is multiplied by all of the expert's tokens. Per CTA (one per SM, 512
+// threads):
+//   warps 0-3   epilogue: TMEM -> registers -> SwiGLU / scaling -> global
+//   warp 4      producer: TMA loads of the token tiles (and bf16 weight tiles)
+//   warp 5      TMEM allocation; one lane issues the MMAs and commits
+//   warps 8-15  dequantisers: 2-bit codes -> fp16 weight tiles (128-byte swizzle)
+// Stages of (A tiles, B tile) circulate through full/empty mbarriers; the MMA
+// completion (tcgen05.commit) frees a stage. Two accumulator buffers in TMEM
+// let the epilogue of one tile overlap the MMAs of the next. Every wait is
+// bounded: a time-out records MOE_ERR_TIMEOUT, all roles stop, and the CTA
+// drains its in-flight copies and MMAs before freeing TMEM.
+//
+// Precision: routed weights enter the MMA as fp16. IQ2 values are formed as
+// fp16(d*(2ls+1)*2^10/8) * grid * sign, which keeps them clear of fp16
+// subnormals for the scales this library's generator and real checkpoints use
+// (|d| in [2^-24, 2^5]); the 2^10 is taken out in the fp32 epilogue. Q2K values
+// q*d*sc - dmin*m are formed in fp32 per sub-block and rounded once to fp16.
+// Activations and h enter as fp16 (routed) or as bf16 hi + lo parts (shared).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "decode.cuh"
+#include "kernels.cuh"
+#include "profile.cuh"
+#include "ptx.cuh"
+#include "tc.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kTcThreads = 512;
+constexpr int kEpiWarps = 4;     // warps 0-3
+constexpr int kProdWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kDqWarp0 = 8;      // warps 8-15
+constexpr int kDqWarps = 8;
+constexpr int kMT = 128;         // weight rows per tile (MMA M)
+constexpr int kNT = 128;         // max tokens per tile (MMA N)
+constexpr int kKS = 64;          // K per stage: 128 bytes of fp16 per row
+constexpr int kTile = 128 * 128; // one 128-row x 128-byte operand tile
+constexpr int kStages = 4;
+constexpr int kTmemCols = 512;   // two accumulator buffers of (gate, up) x 128 columns
+
+__device__ const Iq2Codebook d_codebook_tc = kCodebook;
+
+// A tile source and epilogue kind.
+enum TcKind : int {
+  TC_IQ2_PAIR = 0,   // routed gate+up: dequantised IQ2 pair, SwiGLU, fp16 h out
+  TC_Q2K = 1,        // routed down: dequantised Q2K, fp32 out
+  TC_BF16_PAIR = 2,  // shared gate+up: bf16 tiles by TMA, SwiGLU, bf16 hi/lo h out
+  TC_BF16 = 3,       // shared down: bf16 tiles by TMA, fp32 out
+};
+
+struct TcPair {
+  int e, p0, n, pad;  // expert (weight block), first B row, rows of B used
+};
+
+struct TcArgs {
+  int rows_e;    // weight rows per expert
+  int K;         // reduction length of one plane
+  int mt;        // 128-row tiles per expert
+  int planes;    // B planes summed along K (bf16 hi/lo parts), A re-read per plane
+  const uint8_t* c0;
+  const uint16_t* d0;
+  const uint8_t* c1;
+  const uint16_t* d1;
+  const uint32_t* dd;
+  const TcPair* pairs;
+  const int32_t* npairs;
+  void* out;
+  int ldo;        // output row stride in elements
+  int out_rows;   // rows of one output plane (bf16 hi/lo output)
+  float oscale;
+  int* err;
+};
+
+struct TcSmem {
+  static constexpr size_t stage_bytes = 3 * kTile;  // A0, A1, B
+  static constexpr size_t stages = 0;
+  static constexpr size_t tabs = stages + kStages * stage_bytes;  // IQ2 tables / Q2K selectors
+  static constexpr size_t tab_bytes = 256 * 64 + 128 * 64;      // 4 copies of 16-byte entries
+  static constexpr size_t bars = tabs + tab_bytes;
+  static constexpr size_t total = bars + 1024;
+};
+
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, int* err, volatile int* abort_flag) {
+  if (*abort_flag) return false;
+  if (mbar_wait_bounded(bar, parity, err, ERR_TIMEOUT)) return true;
+  *abort_flag = 1;
+  return false;
+}
+
+// The same for all 32 lanes of a warp, with one outcome for the whole warp.
+__device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, int* err, volatile int* abort_flag) {
+  const bool ok = tc_wait(bar, parity, err, abort_flag);
+  return __all_sync(0xffffffffu, ok) != 0;
+}
+
+__device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t f2_to_h2(float lo, float hi) {
+  __half2 r = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+__device__ __forceinline__ uint4 lds128s(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32s(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+
+// One IQ2 row slice (64 weights = two sub-blocks) -> 128 bytes of fp16 in the
+// swizzled tile row at `dst` (row index r within its 8-row atom = r & 7).
+__device__ __forceinline__ void dq_iq2_step(uint4 cw, float dsc, uint32_t dst, int r7, uint32_t tabG, uint32_t tabS,
+                                            uint32_t rep16) {
+#pragma unroll
+  for (int sb = 0; sb < 2; ++sb) {
+    const uint32_t idx = sb ? cw.z : cw.x, v = sb ? cw.w : cw.y;
+    const float sf = dsc * static_cast<float>(2 * (v >> 28) + 1);
+    const uint32_t s2 = f2_to_h2(sf, sf);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t gi = (idx >> (8 * e)) & 0xFFu;
+      const uint32_t si = (v >> (7 * e)) & 0x7Fu;
+      const uint4 G = lds128s(tabG + gi * 64 + rep16);
+      const uint4 S = lds128s(tabS + si * 64 + rep16);
+      uint4 o;
+      o.x = hmul2_u(G.x ^ S.x, s2);
+      o.y = hmul2_u(G.y ^ S.y, s2);
+      o.z = hmul2_u(G.z ^ S.z, s2);
+      o.w = hmul2_u(G.w ^ S.w, s2);
+      sts128(dst + (((sb * 4 + e) ^ r7) << 4), o);
+    }
+  }
+}
+
+// Half a Q2K row slice (32 weights = two 16-weight sub-blocks) -> 64 bytes of
+// fp16 at chunks c0, c0+1, c0+2, c0+3 of the swizzled tile row.
+__device__ __forceinline__ void dq_q2k_half(uint2 qw, uint32_t sc2, float d, float dmin, uint32_t dst, int r7, int c0,
+                                            uint32_t tabQ) {
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const uint32_t scb = (sc2 >> (8 * j)) & 0xFFu;
+    const float A = d * static_cast<float>(scb & 15u), B = dmin * static_cast<float>(scb >> 4);
+    const uint32_t tlo = f2_to_h2(-B, A - B), thi = f2_to_h2(2.f * A - B, 3.f * A - B);
+    const uint32_t w = j ? qw.y : qw.x;  // 16 weights, weight 4b+i at bits 8b+2i
+    uint32_t o[8];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const uint32_t sel = lds32s(tabQ + ((w >> (8 * b)) & 0xFFu) * 4);
+      o[2 * b] = prmt(tlo, thi, sel);
+      o[2 * b + 1] = prmt(tlo, thi, sel >> 16);
+    }
+    sts128(dst + (((c0 + 2 * j) ^ r7) << 4), make_uint4(o[0], o[1], o[2], o[3]));
+    sts128(dst + (((c0 + 2 * j + 1) ^ r7) << 4), make_uint4(o[4], o[5], o[6], o[7]));
+  }
+}
+
+__device__ __forceinline__ float silu_mul_tc(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+template <int KIND>
+__global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_b,
+                                                                const __grid_constant__ CUtensorMap tm_a0,
+                                                                const __grid_constant__ CUtensorMap tm_a1, TcArgs a) {
+  constexpr bool PAIR = (KIND == TC_IQ2_PAIR || KIND == TC_BF16_PAIR);
+  constexpr bool DQ = (KIND == TC_IQ2_PAIR || KIND == TC_Q2K);
+  constexpr bool BF16 = (KIND == TC_BF16_PAIR || KIND == TC_BF16);
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + TcSmem::bars);
+  uint64_t* fullB = fullA + kStages;
+  uint64_t* empty = fullB + kStages;
+  uint64_t* accf = empty + kStages;  // [2]
+  uint64_t* acce = accf + 2;         // [2]
+  uint64_t* drain = acce + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t sbase = smem_addr(smem);
+
+  if ((sbase & 1023u) != 0) {  // the swizzled tiles need 1024-byte alignment
+    if (tid == 0) atomicCAS(a.err, 0, ERR_CUDA);
+    return;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&fullA[s], kDqWarps);
+      mbar_init(&fullB[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf[b], 1);
+      mbar_init(&acce[b], kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  // dequantisation tables (4 copies of each 16-byte entry, picked by lane & 3)
+  const uint32_t tabG = sbase + TcSmem::tabs, tabS = tabG + 256 * 64, tabQ = tabG;
+  if (KIND == TC_IQ2_PAIR) {
+    for (int i = tid; i < 256 * 4 * 4; i += kTcThreads) {  // (entry, copy, word)
+      const int ent = i >> 4, w = i & 3;
+      const uint32_t lv = d_codebook_tc.val[ent][2 * w], hv = d_codebook_tc.val[ent][2 * w + 1];
+      const uint32_t h0 = __half_as_ushort(__float2half_rn(static_cast<float>(lv)));
+      const uint32_t h1 = __half_as_ushort(__float2half_rn(static_cast<float>(hv)));
+      reinterpret_cast<uint32_t*>(smem + TcSmem::tabs)[i] = h0 | (h1 << 16);
+    }
+    for (int i = tid; i < 128 * 4 * 4; i += kTcThreads) {
+      const int ent = i >> 4, w = i & 3;
+      uint32_t par = 0;
+      for (int b = 0; b < 7; ++b) par ^= (ent >> b) & 1;
+      const uint32_t s0 = (2 * w < 7) ? ((ent >> (2 * w)) & 1) : par;
+      const uint32_t s1 = (2 * w + 1 < 7) ? ((ent >> (2 * w + 1)) & 1) : par;
+      reinterpret_cast<uint32_t*>(smem + TcSmem::tabs + 256 * 64)[i] = (s0 << 15) | (s1 << 31);
+    }
+  } else if (KIND == TC_Q2K) {
+    for (int i = tid; i < 256; i += kTcThreads) {  // byte of four 2-bit codes -> two PRMT selectors
+      uint32_t sel = 0;
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t c = (i >> (2 * q)) & 3u;
+        const uint32_t pair = (2 * c) | ((2 * c + 1) << 4);
+        sel |= pair << (8 * q);
+      }
+      reinterpret_cast<uint32_t*>(smem + TcSmem::tabs)[i] = sel;
+    }
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int npairs = *a.npairs;
+  const int nunits = npairs * a.mt;
+  const int nks = a.planes * (a.K / kKS);
+  const int ks_plane = a.K / kKS;
+
+  if (warp == kProdWarp) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_b);
+      int s = 0;
+      uint32_t ph = 0;
+      int issued = 0;
+      for (int u = blockIdx.x; u < nunits && !*abort_flag; u += gridDim.x) {
+        const TcPair pr = a.pairs[u / a.mt];
+        const int m0 = (u % a.mt) * kMT;
+        for (int ks = 0; ks < nks; ++ks) {
+          if (!tc_wait(&empty[s], ph ^ 1u, a.err, abort_flag)) break;
+          uint8_t* st = smem + TcSmem::stages + s * TcSmem::stage_bytes;
+          const int kx = (ks % ks_plane) * kKS, pl = ks / ks_plane;
+          if (BF16) {
+            mbar_arrive_expect_tx(&fullB[s], (PAIR ? 3 : 2) * kTile);
+            // the weight maps are 3-D like every map of this file (one plane)
+            tma_load_3d(st, &tm_a0, kx, pr.e * a.rows_e + m0, 0, &fullB[s]);
+            if (PAIR) tma_load_3d(st + kTile, &tm_a1, kx, pr.e * a.rows_e + m0, 0, &fullB[s]);
+          } else {
+            mbar_arrive_expect_tx(&fullB[s], kTile);
+          }
+          tma_load_3d(st + 2 * kTile, &tm_b, kx, pr.p0, pl, &fullB[s]);
+          ++issued;
+          if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (*abort_flag) {  // let every copy issued into a stage land before the CTA can exit
+        for (int i = 0; i < kStages && i < issued; ++i) {
+          if (--s < 0) { s = kStages - 1; ph ^= 1u; }
+          mbar_wait_bounded(&fullB[s], ph, nullptr, 0);
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_f16(kMT, 16, BF16);  // N patched per tile
+      int s = 0;
+      uint32_t ph = 0;
+      int t = 0;
+      for (int u = blockIdx.x; u < nunits && !*abort_flag; u += gridDim.x, ++t) {
+        const TcPair pr = a.pairs[u / a.mt];
+        const int n16 = (pr.n + 15) & ~15;
+        const uint32_t id = (idesc & ~(0x3Fu << 17)) | (static_cast<uint32_t>(n16 >> 3) << 17);
+        const int buf = t & 1;
+        if (!tc_wait(&acce[buf], ((t >> 1) & 1) ^ 1u, a.err, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem + buf * 256, d1 = d0 + 128;
+        bool ok = true;
+        for (int ks = 0; ks < nks; ++ks) {
+          if (!tc_wait(&fullB[s], ph, a.err, abort_flag)) { ok = false; break; }
+          if (DQ && !tc_wait(&fullA[s], ph, a.err, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t st = sbase + TcSmem::stages + s * TcSmem::stage_bytes;
+          const uint64_t da0 = umma_desc_sw128(st), da1 = umma_desc_sw128(st + kTile);
+          const uint64_t db = umma_desc_sw128(st + 2 * kTile);
+#pragma unroll
+          for (int kk = 0; kk < kKS / 16; ++kk) {
+            const uint32_t acc = (ks | kk) ? 1u : 0u;
+            umma_f16(d0, da0 + 2 * kk, db + 2 * kk, id, acc);  // +32 bytes along K per step
+            if (PAIR) umma_f16(d1, da1 + 2 * kk, db + 2 * kk, id, acc);
+          }
+          umma_commit(&empty[s]);
+          if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&accf[buf]);
+      }
+      // drain: every MMA issued by this thread completes before TMEM is freed
+      umma_commit(drain);
+      mbar_wait_bounded(drain, 0, nullptr, 0);
+    }
+  } else if (DQ && warp >= kDqWarp0) {
+    const int dt = tid - kDqWarp0 * 32;  // 0..255
+    const uint32_t rep16 = (lane & 3) * 16;
+    int s = 0;
+    uint32_t ph = 0;
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+      const TcPair pr = a.pairs[u / a.mt];
+      const int m0 = (u % a.mt) * kMT;
+      bool ok = true;
+      if (KIND == TC_IQ2_PAIR) {
+        const int mat = dt >> 7, r = dt & 127;
+        const size_t grow = static_cast<size_t>(pr.e) * a.rows_e + m0 + r;
+        const uint8_t* crow = (mat ? a.c1 : a.c0) + grow * (a.K / 4);
+        const uint16_t* drow = (mat ? a.d1 : a.d0) + grow * (a.K / 256);
+        const uint32_t roff = (r >> 3) * 1024 + (r & 7) * 128 + mat * kTile;
+        float dsc = 0.f;
+        for (int ks = 0; ks < nks; ++ks) {
+          const uint4 cw = __ldg(reinterpret_cast<const uint4*>(crow + ks * 16));
+          if ((ks & 3) == 0) dsc = half_bits_to_float(__ldg(drow + (ks >> 2))) * 128.0f;  // d / 8 * 2^10
+          if (!tc_wait_warp(&empty[s], ph ^ 1u, a.err, abort_flag)) { ok = false; break; }
+          const uint32_t st = sbase + TcSmem::stages + s * TcSmem::stage_bytes;
+          dq_iq2_step(cw, dsc, st + roff, r & 7, tabG, tabS, rep16);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&fullA[s]);
+          if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
+      } else {  // TC_Q2K: two threads per row, each half of the 64 weights
+        const int half = dt >> 7, r = dt & 127;
+        const size_t grow = static_cast<size_t>(pr.e) * a.rows_e + m0 + r;
+        const int nblk = a.K / 256;
+        const uint8_t* brow = a.c0 + grow * nblk * 80;
+        const uint32_t* ddrow = a.dd + grow * nblk;
+        const uint32_t roff = (r >> 3) * 1024 + (r & 7) * 128;
+        float d = 0.f, dmin = 0.f;
+        for (int ks = 0; ks < nks; ++ks) {
+          const int b = ks >> 2, q4 = ks & 3;
+          const uint8_t* blk = brow + b * 80;
+          const uint2 qw = __ldg(reinterpret_cast<const uint2*>(blk + 16 + q4 * 16 + 8 * half));
+          const uint32_t sc2 = __ldg(reinterpret_cast<const uint16_t*>(blk + q4 * 4 + 2 * half));
+          if (q4 == 0) {
+            const uint32_t w = __ldg(ddrow + b);
+            d = half_bits_to_float(static_cast<uint16_t>(w & 0xFFFFu));
+            dmin = half_bits_to_float(static_cast<uint16_t>(w >> 16));
+          }
+          if (!tc_wait_warp(&empty[s], ph ^ 1u, a.err, abort_flag)) { ok = false; break; }
+          const uint32_t st = sbase + TcSmem::stages + s * TcSmem::stage_bytes;
+          dq_q2k_half(qw, sc2, d, dmin, st + roff, r & 7, 4 * half, tabQ);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&fullA[s]);
+          if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (!ok) break;
+    }
+  } else if (warp < kEpiWarps) {
+    const int r = 32 * warp + lane;  // TMEM lane = weight row of the tile
+    int t = 0;
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++t) {
+      const TcPair pr = a.pairs[u / a.mt];
+      const int m0 = (u % a.mt) * kMT;
+      const int buf = t & 1;
+      if (!tc_wait_warp(&accf[buf], (t >> 1) & 1, a.err, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tl = tmem + buf * 256 + (static_cast<uint32_t>(32 * warp) << 16);
+      const int row = m0 + r;
+      for (int c0 = 0; c0 < pr.n; c0 += 16) {
+        uint32_t g[16], v[16];
+        tmem_ld16(tl + c0, g);
+        if (PAIR) tmem_ld16(tl + 128 + c0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int n = c0 + j;
+          if (n >= pr.n) break;
+          const size_t orow = static_cast<size_t>(pr.p0 + n);
+          if (KIND == TC_IQ2_PAIR) {
+            const float h = silu_mul_tc(__uint_as_float(g[j]) * a.oscale, __uint_as_float(v[j]) * a.oscale);
+            reinterpret_cast<__half*>(a.out)[orow * a.ldo + row] = __float2half_rn(h);
+          } else if (KIND == TC_BF16_PAIR) {
+            const float h = silu_mul_tc(__uint_as_float(g[j]), __uint_as_float(v[j]));
+            const __nv_bfloat16 hi = __float2bfloat16_rn(h);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
+            reinterpret_cast<__nv_bfloat16*>(a.out)[orow * a.ldo + row] = hi;
+            reinterpret_cast<__nv_bfloat16*>(a.out)[(static_cast<size_t>(a.out_rows) + orow) * a.ldo + row] = lo;
+          } else {
+            reinterpret_cast<float*>(a.out)[orow * a.ldo + row] = __uint_as_float(g[j]) * a.oscale;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[buf]);
+    }
+  }
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+}  // namespace moe
+
+namespace moe {
+namespace {
+
+// Expert-sorted fp16 copy of the activations for the routed B operand, and the
+// tile lists: routed (expert, first assignment, count) tiles of up to 128
+// assignments, and shared tiles of up to 128 tokens. Block 0 also clears the
+// call's status word.
+template <typename XT>
+__global__ void __launch_bounds__(256) prefill_prep_kernel(const XT* __restrict__ x, int T, int H, int k,
+                                                           const int32_t* __restrict__ perm, __half* __restrict__ xp,
+                                                           const int32_t* __restrict__ offsets,
+                                                           const int32_t* __restrict__ active, int E,
+                                                           TcPair* __restrict__ pairs, int32_t* __restrict__ npairs,
+                                                           TcPair* __restrict__ spairs, int32_t* __restrict__ nspairs,
+                                                           int* __restrict__ err_word) {
+  const int nA = T * k;
+  if (blockIdx.x == 0 && threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    if (lane == 0 && err_word) *err_word = 0;
+    const int nact = active[E];
+    int base = 0;
+    for (int s0 = 0; s0 < nact; s0 += 32) {
+      const int s = s0 + lane;
+      int e = 0, p0 = 0, ne = 0;
+      if (s < nact) {
+        e = active[s];
+        p0 = offsets[e];
+        ne = offsets[e + 1] - p0;
+      }
+      const int nt = (ne + kNT - 1) / kNT;
+      int incl = nt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      for (int j = 0; j < nt; ++j) {
+        TcPair pr;
+        pr.e = e;
+        pr.p0 = p0 + j * kNT;
+        pr.n = min(kNT, ne - j * kNT);
+        pr.pad = 0;
+        pairs[base + incl - nt + j] = pr;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) *npairs = base;
+    const int ns = (T + kNT - 1) / kNT;
+    for (int j = lane; j < ns; j += 32) {
+      TcPair pr;
+      pr.e = 0;
+      pr.p0 = j * kNT;
+      pr.n = min(kNT, T - j * kNT);
+      pr.pad = 0;
+      spairs[j] = pr;
+    }
+    if (lane == 0) *nspairs = ns;
+  }
+  const int per = H / 8;
+  const size_t n8 = static_cast<size_t>(nA) * per;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int p = static_cast<int>(i / per), c = static_cast<int>(i % per);
+    const size_t src = static_cast<size_t>(perm[p] / k) * H + c * 8;
+    float v[8];
+    if constexpr (sizeof(XT) == 4) {
+      const float4 a0 = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + src);
+      const float4 a1 = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + src + 4);
+      v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w; v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
+    } else {
+      const uint4 w = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(x) + src);
+      v[0] = __uint_as_float(w.x << 16); v[1] = __uint_as_float(w.x & 0xFFFF0000u);
+      v[2] = __uint_as_float(w.y << 16); v[3] = __uint_as_float(w.y & 0xFFFF0000u);
+      v[4] = __uint_as_float(w.z << 16); v[5] = __uint_as_float(w.z & 0xFFFF0000u);
+      v[6] = __uint_as_float(w.w << 16); v[7] = __uint_as_float(w.w & 0xFFFF0000u);
+    }
+    uint4 o;
+    o.x = f2_to_h2(v[0], v[1]);
+    o.y = f2_to_h2(v[2], v[3]);
+    o.z = f2_to_h2(v[4], v[5]);
+    o.w = f2_to_h2(v[6], v[7]);
+    *reinterpret_cast<uint4*>(xp + static_cast<size_t>(p) * H + c * 8) = o;
+  }
+}
+
+// fp32 activations as two bf16 parts [2][T][H] for the shared expert.
+__global__ void __launch_bounds__(256) bf16_parts_kernel(const float* __restrict__ x, size_t n,
+                                                         __nv_bfloat16* __restrict__ xb) {
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float v = x[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    xb[i] = hi;
+    xb[n + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
+  }
+}
+
+// y[t][h] = sum_j w[t][j] o[inv[t*k+j]][h] (j ascending) + s[t][h] (+ residual).
+__global__ void __launch_bounds__(256) prefill_combine_kernel(int T, int H, int k, const float* __restrict__ topk_w,
+                                                              const int32_t* __restrict__ inv,
+                                                              const float* __restrict__ o, const float* s,
+                                                              const float* residual, float* y) {
+  const size_t n4 = static_cast<size_t>(T) * H / 4;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int t = static_cast<int>((i * 4) / H), h = static_cast<int>((i * 4) % H);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const float w = topk_w[t * k + j];
+      const float4 v = *reinterpret_cast<const float4*>(o + static_cast<size_t>(inv[t * k + j]) * H + h);
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+    if (s) {
+      const float4 v = *reinterpret_cast<const float4*>(s + i * 4);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    if (residual) {
+      const float4 v = *reinterpret_cast<const float4*>(residual + i * 4);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    *reinterpret_cast<float4*>(y + i * 4) = acc;
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tc_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [planes][rows][K] 16-bit elements, box 64 (K) x 128 rows x 1 plane, 128-byte swizzle.
+bool tc_map(CUtensorMap* m, const void* base, bool bf16, uint64_t K, uint64_t rows, uint64_t planes) {
+  auto fn = tc_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {K, rows, planes};
+  const cuuint64_t strides[2] = {K * 2, K * 2 * rows};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int KIND>
+int launch_tc(const CUtensorMap& mb, const CUtensorMap& ma0, const CUtensorMap& ma1, const TcArgs& a, int sms,
+              cudaStream_t st) {
+  const size_t smem = TcSmem::total;
+  cudaFuncSetAttribute(tc_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  tc_gemm_kernel<KIND><<<sms, kTcThreads, smem, st>>>(mb, ma0, ma1, a);
+  return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
+}
+
+struct PrefillWs {
+  __half* xp;
+  __half* hh;
+  float* o;
+  __nv_bfloat16* xb;
+  __nv_bfloat16* hs;
+  float* s;
+  TcPair* pairs;
+  TcPair* spairs;
+  int32_t* counts;
+  size_t bytes;
+};
+
+PrefillWs carve_prefill(const LayerShape& sh, int T, char* base) {
+  const size_t nA = static_cast<size_t>(T) * sh.k;
+  PrefillWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* q = base ? base + off : nullptr;
+    off += align_up(bytes > 0 ? bytes : 1, 1024);
+    return q;
+  };
+  w.xp = reinterpret_cast<__half*>(take(nA * sh.H * 2));
+  w.hh = reinterpret_cast<__half*>(take(nA * sh.I * 2));
+  w.o = reinterpret_cast<float*>(take(nA * sh.H * 4));
+  w.xb = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(T) * sh.H * 2 * 2));
+  w.hs = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(T) * (sh.Is > 0 ? sh.Is : 1) * 2 * 2));
+  w.s = reinterpret_cast<float*>(take(static_cast<size_t>(T) * sh.H * 4));
+  w.pairs = reinterpret_cast<TcPair*>(take((static_cast<size_t>(sh.E) + nA / kNT + 1) * sizeof(TcPair)));
+  w.spairs = reinterpret_cast<TcPair*>(take((static_cast<size_t>(T) / kNT + 1) * sizeof(TcPair)));
+  w.counts = reinterpret_cast<int32_t*>(take(64));
+  w.bytes = off;
+  return w;
+}
+
+}  // namespace
+
+bool prefill_path_supported(const LayerShape& s, int T) {
+  if (T < 1 || s.H % 256 != 0 || s.I % 256 != 0 || s.H % kMT != 0 || s.I % kMT != 0) return false;
+  if (s.Is > 0 && (s.Is % kMT != 0 || s.Is % kKS != 0)) return false;
+  return tc_encode_fn() != nullptr;
+}
+
+size_t prefill_workspace_bytes(const LayerShape& s, int T) { return carve_prefill(s, T, nullptr).bytes; }
+
+int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x, int x_dtype, int T,
+                       const Routing& r, const float* residual, float* y, void* ws, int* err, int sms,
+                       cudaStream_t st) {
+  const PrefillWs pw = carve_prefill(sh, T, static_cast<char*>(ws));
+  const int nA = T * sh.k;
+  int rc = OK;
+  {
+    ProfScope ps(MOE_K_PREP, st);
+    const int grid = std::max(1, std::min(sms * 4, (nA * (sh.H / 8) + 255) / 256));
+    if (x_dtype == 0)
+      prefill_prep_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), T, sh.H, sh.k, r.perm, pw.xp,
+                                                       r.offsets, r.active, sh.E, pw.pairs, pw.counts, pw.spairs,
+                                                       pw.counts + 1, err);
+    else
+      prefill_prep_kernel<uint16_t><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), T, sh.H, sh.k, r.perm,
+                                                          pw.xp, r.offsets, r.active, sh.E, pw.pairs, pw.counts,
+                                                          pw.spairs, pw.counts + 1, err);
+    if (sh.Is > 0 && x_dtype == 0) {
+      const size_t n = static_cast<size_t>(T) * sh.H;
+      bf16_parts_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const float*>(x), n, pw.xb);
+    }
+  }
+  CUtensorMap mb, ma0, ma1;
+  // routed gate/up: A = IQ2 gate/up rows (dequantised), B = expert-sorted fp16 activations
+  {
+    ProfScope ps(MOE_K_PREFILL_GATEUP, st);
+    if (!tc_map(&mb, pw.xp, false, sh.H, nA, 1)) return ERR_CUDA;
+    TcArgs a{};
+    a.rows_e = sh.I; a.K = sh.H; a.mt = sh.I / kMT; a.planes = 1;
+    a.c0 = w.gate_codes; a.d0 = w.gate_d; a.c1 = w.up_codes; a.d1 = w.up_d;
+    a.pairs = pw.pairs; a.npairs = pw.counts; a.out = pw.hh; a.ldo = sh.I; a.out_rows = nA;
+    a.oscale = 1.0f / 1024.0f; a.err = err;
+    rc |= launch_tc<TC_IQ2_PAIR>(mb, mb, mb, a, sms, st);
+  }
+  if (sh.Is > 0) {
+    ProfScope ps(MOE_K_SHARED_GATEUP, st);
+    const int planes = x_dtype == 0 ? 2 : 1;
+    const void* xsrc = x_dtype == 0 ? static_cast<const void*>(pw.xb) : x;
+    if (!tc_map(&mb, xsrc, true, sh.H, T, planes) || !tc_map(&ma0, w.sh_gate, true, sh.H, sh.Is, 1) ||
+        !tc_map(&ma1, w.sh_up, true, sh.H, sh.Is, 1))
+      return ERR_CUDA;
+    TcArgs a{};
+    a.rows_e = sh.Is; a.K = sh.H; a.mt = sh.Is / kMT; a.planes = planes;
+    a.pairs = pw.spairs; a.npairs = pw.counts + 1; a.out = pw.hs; a.ldo = sh.Is; a.out_rows = T;
+    a.oscale = 1.0f; a.err = err;
+    rc |= launch_tc<TC_BF16_PAIR>(mb, ma0, ma1, a, sms, st);
+  }
+  {
+    ProfScope ps(MOE_K_PREFILL_DOWN, st);
+    if (!tc_map(&mb, pw.hh, false, sh.I, nA, 1)) return ERR_CUDA;
+    TcArgs a{};
+    a.rows_e = sh.H; a.K = sh.I; a.mt = sh.H / kMT; a.planes = 1;
+    a.c0 = w.down_codes; a.dd = w.down_dd;
+    a.pairs = pw.pairs; a.npairs = pw.counts; a.out = pw.o; a.ldo = sh.H; a.out_rows = nA;
+    a.oscale = 1.0f; a.err = err;
+    rc |= launch_tc<TC_Q2K>(mb, mb, mb, a, sms, st);
+  }
+  if (sh.Is > 0) {
+    ProfScope ps(MOE_K_SHARED_DOWN, st);
+    if (!tc_map(&mb, pw.hs, true, sh.Is, T, 2) || !tc_map(&ma0, w.sh_down, true, sh.Is, sh.H, 1)) return ERR_CUDA;
+    TcArgs a{};
+    a.rows_e = sh.H; a.K = sh.Is; a.mt = sh.H / kMT; a.planes = 2;
+    a.pairs = pw.spairs; a.npairs = pw.counts + 1; a.out = pw.s; a.ldo = sh.H; a.out_rows = T;
+    a.oscale = 1.0f; a.err = err;
+    rc |= launch_tc<TC_BF16>(mb, ma0, ma0, a, sms, st);
+  }
+  {
+    ProfScope ps(MOE_K_COMBINE, st);
+    const int grid = std::max(1, std::min(sms * 8, static_cast<int>((static_cast<size_t>(T) * sh.H / 4 + 255) / 256)));
+    prefill_combine_kernel<<<grid, 256, 0, st>>>(T, sh.H, sh.k, r.topk_w, r.inv, pw.o, sh.Is > 0 ? pw.s : nullptr,
+                                                 residual, y);
+  }
+  if (rc != OK) return ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
+}
+
+}  // namespace moe

@@ -325,6 +325,52 @@ __global__ void __launch_bounds__(1024) topk_permute_kernel(const float* __restr
   permute_block(idx_s, T * k, E, offsets, perm, inv, active, pbuf);
 }
 
+// Decode routing for few assignments (T*k <= 1024, T <= 32, E <= 1024) in one
+// CTA: warp t takes the top-k of token t; then an integer histogram (shared
+// atomics, order-independent), one exclusive scan for the offsets, one for the
+// active-expert list, and the stable rank of each assignment among the earlier
+// ones routed to the same expert by direct counting.
+template <int EPL>
+__global__ void __launch_bounds__(1024) topk_permute_small_kernel(const float* __restrict__ logits, int T, int E,
+                                                                  int k, int32_t* __restrict__ topk_idx,
+                                                                  float* __restrict__ topk_w,
+                                                                  int32_t* __restrict__ offsets,
+                                                                  int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                                  int32_t* __restrict__ active) {
+  __shared__ int idx_s[1024];
+  __shared__ int cnt[1024];
+  __shared__ int warp_sums[32];
+  __shared__ int total;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int n = T * k;
+  if (tid < E) cnt[tid] = 0;
+  if (warp < T)
+    topk_warp<EPL>(logits + static_cast<size_t>(warp) * E, E, k, topk_idx + static_cast<size_t>(warp) * k,
+                   topk_w + static_cast<size_t>(warp) * k, idx_s + warp * k);
+  __syncthreads();
+  const int e = tid < n ? idx_s[tid] : 0;
+  if (tid < n) atomicAdd(&cnt[e], 1);
+  __syncthreads();
+  const int c = tid < E ? cnt[tid] : 0;
+  const int ex = block_exclusive_scan_1024(c, warp_sums, &total);
+  if (tid < E) {
+    offsets[tid] = ex;
+    cnt[tid] = ex;  // becomes the offset table (each thread rewrites only its own entry)
+  }
+  if (tid == 0) offsets[E] = n;
+  const int flag = (tid < E && c > 0) ? 1 : 0;
+  const int pos = block_exclusive_scan_1024(flag, warp_sums, &total);
+  if (flag) active[pos] = tid;
+  if (tid == 0) active[E] = total;
+  if (tid < n) {
+    int rank = 0;
+    for (int b = 0; b < tid; ++b) rank += idx_s[b] == e ? 1 : 0;
+    const int p = cnt[e] + rank;
+    perm[p] = tid;
+    inv[tid] = p;
+  }
+}
+
 // Active-expert list from caller-provided offsets (used by moe_expert_ffn).
 __global__ void __launch_bounds__(1024) active_from_offsets_kernel(const int32_t* __restrict__ offsets, int E,
                                                                    int32_t* __restrict__ active) {
@@ -368,7 +414,14 @@ int launch_route(const uint16_t* Wr, const float* bias, const void* x, int x_dty
     }
   }
   const size_t psmem = 32 * E * sizeof(uint16_t) + 3 * E * sizeof(int);
-  if (T * k <= 1024 && T <= 32) {
+  if (T * k <= 1024 && T <= 32 && E <= 1024) {
+    ProfScope ps(MOE_K_PERMUTE, st);
+    if (E <= 256)
+      topk_permute_small_kernel<8><<<1, 1024, 0, st>>>(logits, T, E, k, topk_idx, topk_w, offsets, perm, inv, active);
+    else
+      topk_permute_small_kernel<32><<<1, 1024, 0, st>>>(logits, T, E, k, topk_idx, topk_w, offsets, perm, inv,
+                                                        active);
+  } else if (T * k <= 1024 && T <= 32) {
     ProfScope ps(MOE_K_PERMUTE, st);
     const size_t sm = 1024 * sizeof(int32_t) + psmem;
     if (E <= 256) {

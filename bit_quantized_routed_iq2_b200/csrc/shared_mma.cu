@@ -159,15 +159,26 @@ __global__ void __launch_bounds__(512) shared_gateup_mma_kernel(int H, int Is, c
 }
 
 // y[t][r] = sum_j w[t][j] sum_dp o[inv[t*k+j]][dp][r] + (Wsd h_t)[r] (+ residual),
-// 16 rows of H per CTA; h arrives as two bf16 parts.
+// 16 rows of H per CTA; h arrives as two bf16 parts. The routed partial rows
+// are gathered first by all threads (one (row, token, slot) each, parts added
+// in order) into shared memory; each output then adds its k slots in slot
+// order.
 template <int NG>
 __global__ void __launch_bounds__(512) shared_down_combine_mma_kernel(
     int H, int Is, const uint16_t* __restrict__ wd, const uint16_t* __restrict__ hb, int T, int KS, int k,
     const float* __restrict__ topk_w, const int32_t* __restrict__ inv, const float* __restrict__ obuf, int DP,
     const float* residual, float* y) {
   __shared__ __align__(16) float red[ks_max<NG>() * NG * 8 * kRows];
+  extern __shared__ float osum[];  // [T*k][kRows]
   const int warp = threadIdx.x >> 5;
   const int r0 = blockIdx.x * kRows;
+  for (int i = threadIdx.x; i < kRows * T * k; i += blockDim.x) {
+    const int r = i % kRows, a = i / kRows;
+    const float* o = obuf + static_cast<size_t>(inv[a]) * DP * H + r0 + r;
+    float s = 0.f;
+    for (int dp = 0; dp < DP; ++dp) s += o[static_cast<size_t>(dp) * H];
+    osum[i] = s;
+  }
   const int span = Is / KS;
   float acc[1][NG][4];
   const uint16_t* const W[1] = {wd};
@@ -178,13 +189,7 @@ __global__ void __launch_bounds__(512) shared_down_combine_mma_kernel(
     const int r = i % kRows, t = i / kRows;
     const int row = r0 + r;
     float v = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int a = t * k + j;
-      const float* o = obuf + static_cast<size_t>(inv[a]) * DP * H + row;
-      float s = 0.f;
-      for (int dp = 0; dp < DP; ++dp) s += o[static_cast<size_t>(dp) * H];
-      v = fmaf(topk_w[a], s, v);
-    }
+    for (int j = 0; j < k; ++j) v = fmaf(topk_w[t * k + j], osum[(t * k + j) * kRows + r], v);
     v += skinny_value<1, NG>(red, KS, 0, r, t, 2);
     if (residual) v += residual[static_cast<size_t>(t) * H + row];
     y[static_cast<size_t>(t) * H + row] = v;
@@ -203,8 +208,9 @@ int ksmax_for(int ng) { return ng <= 2 ? 16 : (ng == 4 ? 8 : 4); }
 
 }  // namespace
 
-bool shared_mma_supported(int H, int Is, int T, int x_parts) {
+bool shared_mma_supported(int H, int Is, int T, int x_parts, int k) {
   if (Is <= 0 || H % kRows != 0 || Is % kRows != 0 || T < 1) return false;
+  if (static_cast<size_t>(kRows) * T * k * sizeof(float) > 48 * 1024 - 16 * 1024) return false;
   const int ng_gu = groups_for(T * x_parts), ng_dn = groups_for(2 * T);
   if (ng_gu == 0 || ng_gu > 4 || ng_dn == 0) return false;
   return pick_ks(H, ksmax_for(ng_gu)) > 0 && pick_ks(Is, ksmax_for(ng_dn)) > 0;
@@ -232,21 +238,22 @@ int launch_shared_down_combine_mma(int H, int Is, const uint16_t* wd, const uint
   const int ks = pick_ks(Is, ksmax_for(ng));
   if (ks == 0) return ERR_SHAPE;
   const dim3 grid(H / kRows), block(32 * ks);
+  const size_t dyn = static_cast<size_t>(kRows) * T * k * sizeof(float);
   switch (ng) {
     case 1:
-      shared_down_combine_mma_kernel<1><<<grid, block, 0, st>>>(H, Is, wd, hb, T, ks, k, topk_w, inv, obuf, DP,
+      shared_down_combine_mma_kernel<1><<<grid, block, dyn, st>>>(H, Is, wd, hb, T, ks, k, topk_w, inv, obuf, DP,
                                                                 residual, y);
       break;
     case 2:
-      shared_down_combine_mma_kernel<2><<<grid, block, 0, st>>>(H, Is, wd, hb, T, ks, k, topk_w, inv, obuf, DP,
+      shared_down_combine_mma_kernel<2><<<grid, block, dyn, st>>>(H, Is, wd, hb, T, ks, k, topk_w, inv, obuf, DP,
                                                                 residual, y);
       break;
     case 4:
-      shared_down_combine_mma_kernel<4><<<grid, block, 0, st>>>(H, Is, wd, hb, T, ks, k, topk_w, inv, obuf, DP,
+      shared_down_combine_mma_kernel<4><<<grid, block, dyn, st>>>(H, Is, wd, hb, T, ks, k, topk_w, inv, obuf, DP,
                                                                 residual, y);
       break;
     case 8:
-      shared_down_combine_mma_kernel<8><<<grid, block, 0, st>>>(H, Is, wd, hb, T, ks, k, topk_w, inv, obuf, DP,
+      shared_down_combine_mma_kernel<8><<<grid, block, dyn, st>>>(H, Is, wd, hb, T, ks, k, topk_w, inv, obuf, DP,
                                                                 residual, y);
       break;
     default: return ERR_SHAPE;

@@ -163,6 +163,11 @@ SMALL_CASES = {
     "tma_t5": _small(H=2048, I=1024, E=8, k=4, Is=128, T=5, seed=0x5A18),
     "tma_t16": _small(H=1024, I=512, E=8, k=4, Is=64, T=16, seed=0x5A19),
     "tma_t16_zipf_f32": _small(H=1024, I=1024, E=12, k=3, Is=0, T=16, x_dtype="f32", zipf=True, seed=0x5A1A),
+    # shapes served by the tensor-core grouped GEMM (T > 16, H, I, I_s multiples of 128 / 256)
+    "tc_t17": _small(H=512, I=256, E=4, k=2, Is=128, T=17, seed=0x5A1B),
+    "tc_t64_f32": _small(H=1024, I=512, E=8, k=2, Is=256, T=64, x_dtype="f32", seed=0x5A1C),
+    "tc_t200_zipf": _small(H=768, I=512, E=16, k=4, Is=0, T=200, zipf=True, seed=0x5A1D),
+    "tc_t300_many_tiles": _small(H=1280, I=768, E=2, k=1, Is=384, T=300, seed=0x5A1E),
 }
 
 
