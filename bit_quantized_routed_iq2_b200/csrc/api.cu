@@ -133,7 +133,7 @@ moe_status moe_route(const moe_layer_desc* desc, const uint16_t* router_w, const
   RouteWs w = carve(desc, T, ws);
   if (ws_bytes < w.bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
   return to_status(launch_route(router_w, router_bias, x, x_dtype, T, desc->hidden, desc->n_experts,
-                                desc->top_k, w.logits, topk_idx, topk_w, offsets, perm, inv, w.active,
+                                desc->top_k, w.logits, topk_idx, topk_w, offsets, perm, inv, w.active, w.status,
                                 static_cast<cudaStream_t>(stream)));
 }
 
@@ -158,7 +158,7 @@ moe_status moe_expert_ffn(const moe_layer_desc* desc, const moe_layer_weights* w
   if (rc != OK) return to_status(rc);
   Routing r{topk_w, offsets, perm, inv, w.active};
   return to_status(
-      launch_ffn(shape_of(desc), weights_of(weights), x, x_dtype, T, r, residual, y, w.ffn, w.status, s));
+      launch_ffn(shape_of(desc), weights_of(weights), x, x_dtype, T, r, residual, y, w.ffn, w.status, true, s));
 }
 
 moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights* weights, const void* x,
@@ -180,11 +180,14 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights
   if (ws_bytes < w.bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int rc = launch_route(weights->router_w, weights->router_bias, x, x_dtype, T, desc->hidden, desc->n_experts,
-                        desc->top_k, w.logits, w.topk_idx, w.topk_w, w.offsets, w.perm, w.inv, w.active, s);
+                        desc->top_k, w.logits, w.topk_idx, w.topk_w, w.offsets, w.perm, w.inv, w.active, w.status,
+                        s);
   if (rc != OK) return to_status(rc);
   Routing r{w.topk_w, w.offsets, w.perm, w.inv, w.active};
-  return to_status(
-      launch_ffn(shape_of(desc), weights_of(weights), x, x_dtype, T, r, residual, y, w.ffn, w.status, s));
+  // the tensor-core router (many bf16 tokens) already cleared the status word
+  const bool routed_clears = x_dtype == MOE_BF16 && router_tc_supported(T, desc->hidden, desc->n_experts);
+  return to_status(launch_ffn(shape_of(desc), weights_of(weights), x, x_dtype, T, r, residual, y, w.ffn, w.status,
+                              !routed_clears, s));
 }
 
 moe_status moe_debug_dequant_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, float* out,

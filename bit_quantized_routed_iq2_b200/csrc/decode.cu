@@ -469,7 +469,7 @@ size_t fast_ffn_workspace_bytes(const LayerShape& s, int T) {
 }
 
 int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
-                    const float* residual, float* y, void* ws, int* err, cudaStream_t st) {
+                    const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st) {
   const size_t nA = static_cast<size_t>(T) * s.k;
   const bool tma = tma_shape(s, T) && tma_path_supported(s, T);
   const int KP = tma ? tma_gu_parts(s, T) : 1, DP = tma ? tma_dn_parts(s, T) : 1;
@@ -490,9 +490,11 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
     ProfScope ps(MOE_K_PREP, st);
     dim3 g(T, (s.H / 256 + 7) / 8);
     if (x_dtype == 0)
-      x_digits_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(x), T, s.H, xd, xs, fw.xb, err);
+      x_digits_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(x), T, s.H, xd, xs, fw.xb,
+                                                clear_status ? err : nullptr);
     else
-      x_digits_kernel<uint16_t><<<g, 256, 0, st>>>(static_cast<const uint16_t*>(x), T, s.H, xd, xs, nullptr, err);
+      x_digits_kernel<uint16_t><<<g, 256, 0, st>>>(static_cast<const uint16_t*>(x), T, s.H, xd, xs, nullptr,
+                                                   clear_status ? err : nullptr);
   }
   // bf16 activations feed the shared expert's MMAs as one part, fp32 as two
   const int xparts = x_dtype == 0 ? 2 : 1;

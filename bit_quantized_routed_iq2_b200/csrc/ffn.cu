@@ -295,14 +295,14 @@ static int launch_ffn_simple(const LayerShape& s, const WeightPtrs& w, const voi
 }
 
 int launch_ffn(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
-               const float* residual, float* y, void* ws, int* err, cudaStream_t st) {
+               const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st) {
   if (use_prefill(s, T)) {
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return launch_ffn_prefill(s, w, x, x_dtype, T, r, residual, y, ws, err, sms > 0 ? sms : 148, st);
+    return launch_ffn_prefill(s, w, x, x_dtype, T, r, residual, y, ws, err, clear_status, sms > 0 ? sms : 148, st);
   }
-  if (fast_path_supported(s)) return launch_ffn_fast(s, w, x, x_dtype, T, r, residual, y, ws, err, st);
+  if (fast_path_supported(s)) return launch_ffn_fast(s, w, x, x_dtype, T, r, residual, y, ws, err, clear_status, st);
   return launch_ffn_simple(s, w, x, x_dtype, T, r, residual, y, ws, st);
 }
 

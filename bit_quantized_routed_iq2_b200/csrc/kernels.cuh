@@ -34,19 +34,21 @@ struct Routing {
 
 int launch_route(const uint16_t* Wr, const float* bias, const void* x, int x_dtype, int T, int H, int E, int k,
                  float* logits, int32_t* topk_idx, float* topk_w, int32_t* offsets, int32_t* perm, int32_t* inv,
-                 int32_t* active, cudaStream_t st);
+                 int32_t* active, int* err, cudaStream_t st);
 int launch_active_from_offsets(const int32_t* offsets, int E, int32_t* active, cudaStream_t st);
 
 // Workspace needed by the FFN stage for T tokens (bytes) and the launcher.
 size_t ffn_workspace_bytes(const LayerShape& s, int T);
+// clear_status: the FFN's first kernel clears *err (false when an earlier
+// kernel of the same call already did).
 int launch_ffn(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
-               const float* residual, float* y, void* ws, int* err, cudaStream_t st);
+               const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st);
 
 // Tensor-core dequant-GEMV path (decode.cu): shapes with H % 256 == 0 and I % 256 == 0.
 bool fast_path_supported(const LayerShape& s);
 size_t fast_ffn_workspace_bytes(const LayerShape& s, int T);
 int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
-                    const float* residual, float* y, void* ws, int* err, cudaStream_t st);
+                    const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st);
 
 // TMA-fed GEMVs (gemv_tma.cu).
 bool tma_path_supported(const LayerShape& s, int T);
@@ -68,12 +70,18 @@ int launch_shared_down_combine_mma(int H, int Is, const uint16_t* wd, const uint
                                    const float* topk_w, const int32_t* inv, const float* obuf, int DP,
                                    const float* residual, float* y, cudaStream_t st);
 
+// Router logits on the tensor cores for many bf16 tokens (prefill.cu).
+bool router_tc_supported(int T, int H, int E);
+int launch_router_tc(const uint16_t* Wr, const float* bias, const uint16_t* x, int T, int H, int E, float* logits,
+                     int* err, int sms, cudaStream_t st);
+
 // Tensor-core grouped GEMM for many tokens (prefill.cu).
 constexpr int kPrefillMinT = 16;
 bool prefill_path_supported(const LayerShape& s, int T);
 size_t prefill_workspace_bytes(const LayerShape& s, int T);
 int launch_ffn_prefill(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
-                       const float* residual, float* y, void* ws, int* err, int sms, cudaStream_t st);
+                       const float* residual, float* y, void* ws, int* err, bool clear_status, int sms,
+                       cudaStream_t st);
 
 int launch_debug_dequant_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, float* out, cudaStream_t st);
 int launch_debug_dequant_q2k(const uint8_t* codes, const uint32_t* dd, int64_t nblocks, float* out,

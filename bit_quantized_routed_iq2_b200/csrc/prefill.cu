@@ -84,13 +84,16 @@ struct TcArgs {
   const uint8_t* c1;
   const uint16_t* d1;
   const uint32_t* dd;
-  const TcPair* pairs;
+  const TcPair* pairs;     // tile list (expert, first B row, rows), or null for dense tiles
   const int32_t* npairs;
+  int dense_rows;          // with pairs == null: tiles of 128 rows over this many B rows, expert 0
+  const float* bias;       // TC_BF16 only: added per weight row (router bias), may be null
   void* out;
   int ldo;        // output row stride in elements
   int out_rows;   // rows of one output plane (bf16 hi/lo output)
   float oscale;
   int* err;
+  int clear_err;  // CTA 0 clears *err at start (first kernel of a call)
 };
 
 struct TcSmem {
@@ -186,6 +189,16 @@ __device__ __forceinline__ void dq_q2k_half(uint2 qw, uint32_t sc2, float d, flo
 
 __device__ __forceinline__ float silu_mul_tc(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
+__device__ __forceinline__ TcPair tc_pair(const TcArgs& a, int i) {
+  if (a.pairs) return a.pairs[i];
+  TcPair p;
+  p.e = 0;
+  p.p0 = i * kNT;
+  p.n = min(kNT, a.dense_rows - i * kNT);
+  p.pad = 0;
+  return p;
+}
+
 template <int KIND>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_b,
                                                                 const __grid_constant__ CUtensorMap tm_a0,
@@ -209,6 +222,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     if (tid == 0) atomicCAS(a.err, 0, ERR_CUDA);
     return;
   }
+  if (tid == 0 && blockIdx.x == 0 && a.clear_err) *a.err = 0;
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&fullA[s], kDqWarps);
@@ -260,7 +274,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int npairs = *a.npairs;
+  const int npairs = a.pairs ? *a.npairs : (a.dense_rows + kNT - 1) / kNT;
   const int nunits = npairs * a.mt;
   const int nks = a.planes * (a.K / kKS);
   const int ks_plane = a.K / kKS;
@@ -272,7 +286,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       uint32_t ph = 0;
       int issued = 0;
       for (int u = blockIdx.x; u < nunits && !*abort_flag; u += gridDim.x) {
-        const TcPair pr = a.pairs[u / a.mt];
+        const TcPair pr = tc_pair(a, u / a.mt);
         const int m0 = (u % a.mt) * kMT;
         for (int ks = 0; ks < nks; ++ks) {
           if (!tc_wait(&empty[s], ph ^ 1u, a.err, abort_flag)) break;
@@ -305,7 +319,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       uint32_t ph = 0;
       int t = 0;
       for (int u = blockIdx.x; u < nunits && !*abort_flag; u += gridDim.x, ++t) {
-        const TcPair pr = a.pairs[u / a.mt];
+        const TcPair pr = tc_pair(a, u / a.mt);
         const int n16 = (pr.n + 15) & ~15;
         const uint32_t id = (idesc & ~(0x3Fu << 17)) | (static_cast<uint32_t>(n16 >> 3) << 17);
         const int buf = t & 1;
@@ -342,7 +356,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     int s = 0;
     uint32_t ph = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-      const TcPair pr = a.pairs[u / a.mt];
+      const TcPair pr = tc_pair(a, u / a.mt);
       const int m0 = (u % a.mt) * kMT;
       bool ok = true;
       if (KIND == TC_IQ2_PAIR) {
@@ -351,17 +365,35 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         const uint8_t* crow = (mat ? a.c1 : a.c0) + grow * (a.K / 4);
         const uint16_t* drow = (mat ? a.d1 : a.d0) + grow * (a.K / 256);
         const uint32_t roff = (r >> 3) * 1024 + (r & 7) * 128 + mat * kTile;
-        float dsc = 0.f;
-        for (int ks = 0; ks < nks; ++ks) {
-          const uint4 cw = __ldg(reinterpret_cast<const uint4*>(crow + ks * 16));
-          if ((ks & 3) == 0) dsc = half_bits_to_float(__ldg(drow + (ks >> 2))) * 128.0f;  // d / 8 * 2^10
-          if (!tc_wait_warp(&empty[s], ph ^ 1u, a.err, abort_flag)) { ok = false; break; }
-          const uint32_t st = sbase + TcSmem::stages + s * TcSmem::stage_bytes;
-          dq_iq2_step(cw, dsc, st + roff, r & 7, tabG, tabS, rep16);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&fullA[s]);
-          if (++s == kStages) { s = 0; ph ^= 1u; }
+        // one 256-weight block (four stages) per step; loads run two blocks ahead
+        const int nblk = nks / 4;
+        uint4 cur[4], nxt[4], nn[4];
+        uint32_t dcur = 0, dnxt = 0, dnn = 0;
+        auto load_blk = [&](int b, uint4 (&dst)[4], uint32_t& dv) {
+          const uint4* src = reinterpret_cast<const uint4*>(crow + b * 64);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dst[q] = __ldg(src + q);
+          dv = __ldg(drow + b);
+        };
+        load_blk(0, cur, dcur);
+        if (nblk > 1) load_blk(1, nxt, dnxt);
+        for (int b = 0; b < nblk && ok; ++b) {
+          if (b + 2 < nblk) load_blk(b + 2, nn, dnn);
+          const float dsc = half_bits_to_float(static_cast<uint16_t>(dcur)) * 128.0f;  // d / 8 * 2^10
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (!tc_wait_warp(&empty[s], ph ^ 1u, a.err, abort_flag)) { ok = false; break; }
+            const uint32_t st = sbase + TcSmem::stages + s * TcSmem::stage_bytes;
+            dq_iq2_step(cur[q], dsc, st + roff, r & 7, tabG, tabS, rep16);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&fullA[s]);
+            if (++s == kStages) { s = 0; ph ^= 1u; }
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) { cur[q] = nxt[q]; nxt[q] = nn[q]; }
+          dcur = dnxt;
+          dnxt = dnn;
         }
       } else {  // TC_Q2K: two threads per row, each half of the 64 weights
         const int half = dt >> 7, r = dt & 127;
@@ -370,24 +402,41 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         const uint8_t* brow = a.c0 + grow * nblk * 80;
         const uint32_t* ddrow = a.dd + grow * nblk;
         const uint32_t roff = (r >> 3) * 1024 + (r & 7) * 128;
-        float d = 0.f, dmin = 0.f;
-        for (int ks = 0; ks < nks; ++ks) {
-          const int b = ks >> 2, q4 = ks & 3;
-          const uint8_t* blk = brow + b * 80;
-          const uint2 qw = __ldg(reinterpret_cast<const uint2*>(blk + 16 + q4 * 16 + 8 * half));
-          const uint32_t sc2 = __ldg(reinterpret_cast<const uint16_t*>(blk + q4 * 4 + 2 * half));
-          if (q4 == 0) {
-            const uint32_t w = __ldg(ddrow + b);
-            d = half_bits_to_float(static_cast<uint16_t>(w & 0xFFFFu));
-            dmin = half_bits_to_float(static_cast<uint16_t>(w >> 16));
+        // one 80-byte block (four stages) per step; loads run two blocks ahead
+        const int nbk = nks / 4;
+        uint4 cur[5], nxt[5], nn[5];
+        uint32_t dcur = 0, dnxt = 0, dnn = 0;
+        auto load_blk = [&](int b, uint4 (&dst)[5], uint32_t& dv) {
+          const uint4* src = reinterpret_cast<const uint4*>(brow + b * 80);
+#pragma unroll
+          for (int q = 0; q < 5; ++q) dst[q] = __ldg(src + q);
+          dv = __ldg(ddrow + b);
+        };
+        load_blk(0, cur, dcur);
+        if (nbk > 1) load_blk(1, nxt, dnxt);
+        for (int b = 0; b < nbk && ok; ++b) {
+          if (b + 2 < nbk) load_blk(b + 2, nn, dnn);
+          const float d = half_bits_to_float(static_cast<uint16_t>(dcur & 0xFFFFu));
+          const float dmin = half_bits_to_float(static_cast<uint16_t>(dcur >> 16));
+          const uint32_t scw[4] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w};
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            // sub-blocks 4q4 + 2half, +1: q bytes 16 + 16q4 + 8half, scale bytes 4q4 + 2half
+            const uint4 qv = cur[1 + q4];
+            const uint2 qw = half ? make_uint2(qv.z, qv.w) : make_uint2(qv.x, qv.y);
+            const uint32_t sc2 = (scw[q4] >> (16 * half)) & 0xFFFFu;
+            if (!tc_wait_warp(&empty[s], ph ^ 1u, a.err, abort_flag)) { ok = false; break; }
+            const uint32_t st = sbase + TcSmem::stages + s * TcSmem::stage_bytes;
+            dq_q2k_half(qw, sc2, d, dmin, st + roff, r & 7, 4 * half, tabQ);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&fullA[s]);
+            if (++s == kStages) { s = 0; ph ^= 1u; }
           }
-          if (!tc_wait_warp(&empty[s], ph ^ 1u, a.err, abort_flag)) { ok = false; break; }
-          const uint32_t st = sbase + TcSmem::stages + s * TcSmem::stage_bytes;
-          dq_q2k_half(qw, sc2, d, dmin, st + roff, r & 7, 4 * half, tabQ);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&fullA[s]);
-          if (++s == kStages) { s = 0; ph ^= 1u; }
+#pragma unroll
+          for (int q = 0; q < 5; ++q) { cur[q] = nxt[q]; nxt[q] = nn[q]; }
+          dcur = dnxt;
+          dnxt = dnn;
         }
       }
       if (!ok) break;
@@ -396,7 +445,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     const int r = 32 * warp + lane;  // TMEM lane = weight row of the tile
     int t = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++t) {
-      const TcPair pr = a.pairs[u / a.mt];
+      const TcPair pr = tc_pair(a, u / a.mt);
       const int m0 = (u % a.mt) * kMT;
       const int buf = t & 1;
       if (!tc_wait_warp(&accf[buf], (t >> 1) & 1, a.err, abort_flag)) break;
@@ -422,8 +471,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
             reinterpret_cast<__nv_bfloat16*>(a.out)[orow * a.ldo + row] = hi;
             reinterpret_cast<__nv_bfloat16*>(a.out)[(static_cast<size_t>(a.out_rows) + orow) * a.ldo + row] = lo;
+          } else if (KIND == TC_Q2K) {  // routed expert outputs, combined later in slot order
+            reinterpret_cast<__half*>(a.out)[orow * a.ldo + row] = __float2half_rn(__uint_as_float(g[j]) * a.oscale);
           } else {
-            reinterpret_cast<float*>(a.out)[orow * a.ldo + row] = __uint_as_float(g[j]) * a.oscale;
+            const float bv = (KIND == TC_BF16 && a.bias) ? a.bias[row] : 0.f;
+            reinterpret_cast<float*>(a.out)[orow * a.ldo + row] = __uint_as_float(g[j]) * a.oscale + bv;
           }
         }
       }
@@ -539,10 +591,12 @@ __global__ void __launch_bounds__(256) bf16_parts_kernel(const float* __restrict
   }
 }
 
-// y[t][h] = sum_j w[t][j] o[inv[t*k+j]][h] (j ascending) + s[t][h] (+ residual).
+// y[t][h] = sum_j w[t][j] o[inv[t*k+j]][h] (j ascending) + s[t][h] (+ residual),
+// with the routed expert outputs o stored as fp16 (relative rounding 2^-11,
+// an order below the 2e-3 bound) to halve the traffic of this pass.
 __global__ void __launch_bounds__(256) prefill_combine_kernel(int T, int H, int k, const float* __restrict__ topk_w,
                                                               const int32_t* __restrict__ inv,
-                                                              const float* __restrict__ o, const float* s,
+                                                              const __half* __restrict__ o, const float* s,
                                                               const float* residual, float* y) {
   const size_t n4 = static_cast<size_t>(T) * H / 4;
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
@@ -551,11 +605,13 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(int T, int H, int 
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < k; ++j) {
       const float w = topk_w[t * k + j];
-      const float4 v = *reinterpret_cast<const float4*>(o + static_cast<size_t>(inv[t * k + j]) * H + h);
-      acc.x = fmaf(w, v.x, acc.x);
-      acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z);
-      acc.w = fmaf(w, v.w, acc.w);
+      const uint2 hv = *reinterpret_cast<const uint2*>(o + static_cast<size_t>(inv[t * k + j]) * H + h);
+      const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
+      const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
+      acc.x = fmaf(w, v01.x, acc.x);
+      acc.y = fmaf(w, v01.y, acc.y);
+      acc.z = fmaf(w, v23.x, acc.z);
+      acc.w = fmaf(w, v23.y, acc.w);
     }
     if (s) {
       const float4 v = *reinterpret_cast<const float4*>(s + i * 4);
@@ -609,7 +665,7 @@ int launch_tc(const CUtensorMap& mb, const CUtensorMap& ma0, const CUtensorMap& 
 struct PrefillWs {
   __half* xp;
   __half* hh;
-  float* o;
+  __half* o;  // routed expert outputs [T*k][H], fp16
   __nv_bfloat16* xb;
   __nv_bfloat16* hs;
   float* s;
@@ -630,7 +686,7 @@ PrefillWs carve_prefill(const LayerShape& sh, int T, char* base) {
   };
   w.xp = reinterpret_cast<__half*>(take(nA * sh.H * 2));
   w.hh = reinterpret_cast<__half*>(take(nA * sh.I * 2));
-  w.o = reinterpret_cast<float*>(take(nA * sh.H * 4));
+  w.o = reinterpret_cast<__half*>(take(nA * sh.H * 2));
   w.xb = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(T) * sh.H * 2 * 2));
   w.hs = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(T) * (sh.Is > 0 ? sh.Is : 1) * 2 * 2));
   w.s = reinterpret_cast<float*>(take(static_cast<size_t>(T) * sh.H * 4));
@@ -643,6 +699,24 @@ PrefillWs carve_prefill(const LayerShape& sh, int T, char* base) {
 
 }  // namespace
 
+// Router logits for many bf16 tokens on the same tensor-core GEMM: weights
+// Wr [E][H] (bf16, by TMA) are the M operand, tokens the N operand, the bias is
+// added in the epilogue: logits[t][e] = sum_h Wr[e][h] x[t][h] + bias[e].
+bool router_tc_supported(int T, int H, int E) {
+  return T > 64 && H % kKS == 0 && E % kMT == 0 && tc_encode_fn() != nullptr;
+}
+
+int launch_router_tc(const uint16_t* Wr, const float* bias, const uint16_t* x, int T, int H, int E, float* logits,
+                     int* err, int sms, cudaStream_t st) {
+  CUtensorMap mb, ma;
+  if (!tc_map(&mb, x, true, H, T, 1) || !tc_map(&ma, Wr, true, H, E, 1)) return ERR_CUDA;
+  TcArgs a{};
+  a.rows_e = E; a.K = H; a.mt = E / kMT; a.planes = 1;
+  a.dense_rows = T; a.bias = bias; a.out = logits; a.ldo = E; a.out_rows = T;
+  a.oscale = 1.0f; a.err = err; a.clear_err = 1;
+  return launch_tc<TC_BF16>(mb, ma, ma, a, sms, st);
+}
+
 bool prefill_path_supported(const LayerShape& s, int T) {
   if (T < 1 || s.H % 256 != 0 || s.I % 256 != 0 || s.H % kMT != 0 || s.I % kMT != 0) return false;
   if (s.Is > 0 && (s.Is % kMT != 0 || s.Is % kKS != 0)) return false;
@@ -652,8 +726,8 @@ bool prefill_path_supported(const LayerShape& s, int T) {
 size_t prefill_workspace_bytes(const LayerShape& s, int T) { return carve_prefill(s, T, nullptr).bytes; }
 
 int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x, int x_dtype, int T,
-                       const Routing& r, const float* residual, float* y, void* ws, int* err, int sms,
-                       cudaStream_t st) {
+                       const Routing& r, const float* residual, float* y, void* ws, int* err, bool clear_status,
+                       int sms, cudaStream_t st) {
   const PrefillWs pw = carve_prefill(sh, T, static_cast<char*>(ws));
   const int nA = T * sh.k;
   int rc = OK;
@@ -663,11 +737,11 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
     if (x_dtype == 0)
       prefill_prep_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), T, sh.H, sh.k, r.perm, pw.xp,
                                                        r.offsets, r.active, sh.E, pw.pairs, pw.counts, pw.spairs,
-                                                       pw.counts + 1, err);
+                                                       pw.counts + 1, clear_status ? err : nullptr);
     else
       prefill_prep_kernel<uint16_t><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), T, sh.H, sh.k, r.perm,
                                                           pw.xp, r.offsets, r.active, sh.E, pw.pairs, pw.counts,
-                                                          pw.spairs, pw.counts + 1, err);
+                                                          pw.spairs, pw.counts + 1, clear_status ? err : nullptr);
     if (sh.Is > 0 && x_dtype == 0) {
       const size_t n = static_cast<size_t>(T) * sh.H;
       bf16_parts_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const float*>(x), n, pw.xb);
@@ -694,7 +768,7 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
       return ERR_CUDA;
     TcArgs a{};
     a.rows_e = sh.Is; a.K = sh.H; a.mt = sh.Is / kMT; a.planes = planes;
-    a.pairs = pw.spairs; a.npairs = pw.counts + 1; a.out = pw.hs; a.ldo = sh.Is; a.out_rows = T;
+    a.dense_rows = T; a.out = pw.hs; a.ldo = sh.Is; a.out_rows = T;
     a.oscale = 1.0f; a.err = err;
     rc |= launch_tc<TC_BF16_PAIR>(mb, ma0, ma1, a, sms, st);
   }
@@ -713,7 +787,7 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
     if (!tc_map(&mb, pw.hs, true, sh.Is, T, 2) || !tc_map(&ma0, w.sh_down, true, sh.Is, sh.H, 1)) return ERR_CUDA;
     TcArgs a{};
     a.rows_e = sh.H; a.K = sh.Is; a.mt = sh.H / kMT; a.planes = 2;
-    a.pairs = pw.spairs; a.npairs = pw.counts + 1; a.out = pw.s; a.ldo = sh.H; a.out_rows = T;
+    a.dense_rows = T; a.out = pw.s; a.ldo = sh.H; a.out_rows = T;
     a.oscale = 1.0f; a.err = err;
     rc |= launch_tc<TC_BF16>(mb, ma0, ma0, a, sms, st);
   }

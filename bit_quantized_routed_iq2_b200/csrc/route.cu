@@ -391,10 +391,17 @@ static void set_smem(K kernel, size_t bytes) {
 
 int launch_route(const uint16_t* Wr, const float* bias, const void* x, int x_dtype, int T, int H, int E, int k,
                  float* logits, int32_t* topk_idx, float* topk_w, int32_t* offsets, int32_t* perm, int32_t* inv,
-                 int32_t* active, cudaStream_t st) {
+                 int32_t* active, int* err, cudaStream_t st) {
   {
     ProfScope ps(MOE_K_ROUTER_LOGITS, st);
-    if (T <= 64) {
+    if (x_dtype == 1 && router_tc_supported(T, H, E)) {
+      int dev = 0, sms = 0;
+      cudaGetDevice(&dev);
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      const int rc = launch_router_tc(Wr, bias, static_cast<const uint16_t*>(x), T, H, E, logits, err,
+                                      sms > 0 ? sms : 148, st);
+      if (rc != OK) return rc;
+    } else if (T <= 64) {
       constexpr int TT = 4;
       dim3 g((T + TT - 1) / TT, E);
       if (x_dtype == 0)

@@ -45,7 +45,7 @@ constexpr int kRows = 16;
 // Accumulate D[r][c] += sum_{k in [kbeg, kend)} W_m[r0 + r][k] * B[c][k] for
 // NM weight matrices sharing the B columns. B column c of group q is
 // (token, part) = ((8q + c) / P, (8q + c) % P).
-template <int NM, int NG>
+template <int NM, int NG, int U = (NG == 1 ? 4 : 2)>
 __device__ __forceinline__ void skinny_mainloop(const uint16_t* const (&W)[NM], int K, int r0, const uint16_t* xb,
                                                 int P, int T, int kbeg, int kend, float (&acc)[NM][NG][4]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
@@ -67,7 +67,7 @@ __device__ __forceinline__ void skinny_mainloop(const uint16_t* const (&W)[NM], 
   for (int m = 0; m < NM; ++m)
 #pragma unroll
     for (int q = 0; q < NG; ++q) acc[m][q][0] = acc[m][q][1] = acc[m][q][2] = acc[m][q][3] = 0.f;
-  constexpr int U = 2;  // steps of 32 columns in flight
+  // U steps of 32 columns in flight per warp
   for (int k0 = kbeg; k0 < kend; k0 += 32 * U) {
     uint4 av[U][NM][2];
     uint4 bv[U][NG];
@@ -159,10 +159,10 @@ __global__ void __launch_bounds__(512) shared_gateup_mma_kernel(int H, int Is, c
 }
 
 // y[t][r] = sum_j w[t][j] sum_dp o[inv[t*k+j]][dp][r] + (Wsd h_t)[r] (+ residual),
-// 16 rows of H per CTA; h arrives as two bf16 parts. The routed partial rows
-// are gathered first by all threads (one (row, token, slot) each, parts added
-// in order) into shared memory; each output then adds its k slots in slot
-// order.
+// 16 rows of H per CTA; h arrives as two bf16 parts. After the weight stream,
+// all threads gather the routed partial rows (one (row, token, slot) each,
+// parts added in order; the first slot index is loaded before the stream) into
+// shared memory; each output then adds its k slots in slot order.
 template <int NG>
 __global__ void __launch_bounds__(512) shared_down_combine_mma_kernel(
     int H, int Is, const uint16_t* __restrict__ wd, const uint16_t* __restrict__ hb, int T, int KS, int k,
@@ -172,18 +172,21 @@ __global__ void __launch_bounds__(512) shared_down_combine_mma_kernel(
   extern __shared__ float osum[];  // [T*k][kRows]
   const int warp = threadIdx.x >> 5;
   const int r0 = blockIdx.x * kRows;
-  for (int i = threadIdx.x; i < kRows * T * k; i += blockDim.x) {
-    const int r = i % kRows, a = i / kRows;
-    const float* o = obuf + static_cast<size_t>(inv[a]) * DP * H + r0 + r;
-    float s = 0.f;
-    for (int dp = 0; dp < DP; ++dp) s += o[static_cast<size_t>(dp) * H];
-    osum[i] = s;
-  }
+  // the assignment rows of this thread's first gather item, loaded before the weight stream
+  const int nitems = kRows * T * k;
+  const int a0 = threadIdx.x < nitems ? inv[threadIdx.x / kRows] : 0;
   const int span = Is / KS;
   float acc[1][NG][4];
   const uint16_t* const W[1] = {wd};
   skinny_mainloop<1, NG>(W, Is, r0, hb, 2, T, warp * span, (warp + 1) * span, acc);
   skinny_store<1, NG>(red, acc);
+  for (int i = threadIdx.x; i < nitems; i += blockDim.x) {
+    const int r = i % kRows, a = i / kRows;
+    const float* o = obuf + static_cast<size_t>(i < static_cast<int>(blockDim.x) ? a0 : inv[a]) * DP * H + r0 + r;
+    float sacc = 0.f;
+    for (int dp = 0; dp < DP; ++dp) sacc += o[static_cast<size_t>(dp) * H];
+    osum[i] = sacc;
+  }
   __syncthreads();
   for (int i = threadIdx.x; i < kRows * T; i += blockDim.x) {
     const int r = i % kRows, t = i / kRows;

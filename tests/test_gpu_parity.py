@@ -168,6 +168,8 @@ SMALL_CASES = {
     "tc_t64_f32": _small(H=1024, I=512, E=8, k=2, Is=256, T=64, x_dtype="f32", seed=0x5A1C),
     "tc_t200_zipf": _small(H=768, I=512, E=16, k=4, Is=0, T=200, zipf=True, seed=0x5A1D),
     "tc_t300_many_tiles": _small(H=1280, I=768, E=2, k=1, Is=384, T=300, seed=0x5A1E),
+    # router logits on the tensor cores too (bf16 x, T > 64, E % 128 == 0)
+    "tc_router_t130": _small(H=512, I=256, E=128, k=4, Is=128, T=130, seed=0x5A1F),
 }
 
 
