@@ -350,68 +350,7 @@ __global__ void __launch_bounds__(256) hquant_kernel(int I, int KP, const float*
                                                      int32_t* __restrict__ hq, int hss) {
   const int p = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float* g = gu + static_cast<size_t>(p) * 2 * KP * I;
-  const float* u = g + static_cast<size_t>(KP) * I;
-  for (int sb = warp; sb < I / 256; sb += 8) {
-    const int base = sb * 256 + lane * 8;
-    float gv[8], uv[8];
-    {
-      const float4 g0 = *reinterpret_cast<const float4*>(g + base), g1 = *reinterpret_cast<const float4*>(g + base + 4);
-      const float4 u0 = *reinterpret_cast<const float4*>(u + base), u1 = *reinterpret_cast<const float4*>(u + base + 4);
-      gv[0] = g0.x; gv[1] = g0.y; gv[2] = g0.z; gv[3] = g0.w; gv[4] = g1.x; gv[5] = g1.y; gv[6] = g1.z; gv[7] = g1.w;
-      uv[0] = u0.x; uv[1] = u0.y; uv[2] = u0.z; uv[3] = u0.w; uv[4] = u1.x; uv[5] = u1.y; uv[6] = u1.z; uv[7] = u1.w;
-    }
-    // parts are added in order; loads of up to eight parts are in flight at once
-    for (int k0 = 1; k0 < KP; k0 += 8) {
-      float4 lg[8][2], lu[8][2];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (k0 + q < KP) {
-          const float* gp = g + static_cast<size_t>(k0 + q) * I + base;
-          const float* up = u + static_cast<size_t>(k0 + q) * I + base;
-          lg[q][0] = *reinterpret_cast<const float4*>(gp);
-          lg[q][1] = *reinterpret_cast<const float4*>(gp + 4);
-          lu[q][0] = *reinterpret_cast<const float4*>(up);
-          lu[q][1] = *reinterpret_cast<const float4*>(up + 4);
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (k0 + q < KP) {
-          gv[0] += lg[q][0].x; gv[1] += lg[q][0].y; gv[2] += lg[q][0].z; gv[3] += lg[q][0].w;
-          gv[4] += lg[q][1].x; gv[5] += lg[q][1].y; gv[6] += lg[q][1].z; gv[7] += lg[q][1].w;
-          uv[0] += lu[q][0].x; uv[1] += lu[q][0].y; uv[2] += lu[q][0].z; uv[3] += lu[q][0].w;
-          uv[4] += lu[q][1].x; uv[5] += lu[q][1].y; uv[6] += lu[q][1].z; uv[7] += lu[q][1].w;
-        }
-      }
-    }
-    float h[8], m = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      h[i] = silu_mul(gv[i], uv[i]);
-      m = fmaxf(m, fabsf(h[i]));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const int e = m > 0.f ? floor_log2_pos(m) - 11 : 0;
-    int qs = 0;
-    int8_t* hi_row = hd + static_cast<size_t>(p) * 2 * I;
-    int8_t* lo_row = hi_row + I;
-    const int blk32 = base >> 5, jj0 = base & 31;  // this lane's 8 elements sit in one 32-block
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      int hi = 0, lo = 0;
-      if (m > 0.f) split_digits(h[i], e, hi, lo);
-      qs += hi * 128 + lo;
-      const int jj = jj0 + i, sub = jj >> 4, j = jj & 15;
-      const int pos = blk32 * 32 + 8 * (j & 3) + 4 * sub + (j >> 2);
-      hi_row[pos] = static_cast<int8_t>(hi);
-      lo_row[pos] = static_cast<int8_t>(lo);
-    }
-    qs += __shfl_xor_sync(0xffffffffu, qs, 1);  // lanes 2i, 2i+1 hold one 16-element sub-block
-    if ((lane & 1) == 0) hq[static_cast<size_t>(p) * (I / 16) + sb * 16 + (lane >> 1)] = qs;
-    if (lane == 0) hsc[static_cast<size_t>(p) * hss + sb] = m > 0.f ? ldexpf(1.0f, e) : 0.f;
-  }
+  for (int sb = warp; sb < I / 256; sb += 8) hquant_block_warp(I, KP, gu, p, sb, hd, hsc, hq, hss, lane);
 }
 
 // The TMA-fed GEMVs (gemv_tma.cu) serve shapes with H % 1024 == 0 and

@@ -57,7 +57,6 @@ constexpr int kMT = 128;         // weight rows per tile (MMA M)
 constexpr int kNT = 128;         // max tokens per tile (MMA N)
 constexpr int kKS = 64;          // K per stage: 128 bytes of fp16 per row
 constexpr int kTile = 128 * 128; // one 128-row x 128-byte operand tile
-constexpr int kStages = 4;
 constexpr int kTmemCols = 512;   // two accumulator buffers of (gate, up) x 128 columns
 
 __device__ const Iq2Codebook d_codebook_tc = kCodebook;
@@ -96,14 +95,28 @@ struct TcArgs {
   int clear_err;  // CTA 0 clears *err at start (first kernel of a call)
 };
 
-struct TcSmem {
-  static constexpr size_t stage_bytes = 3 * kTile;  // A0, A1, B
-  static constexpr size_t stages = 0;
-  static constexpr size_t tabs = stages + kStages * stage_bytes;  // IQ2 tables / Q2K selectors
-  static constexpr size_t tab_bytes = 256 * 64 + 128 * 64;      // 4 copies of 16-byte entries
+// Shared-memory layout per kernel kind: stages of (A0, A1 for the pair kinds,
+// B), the replicated dequantisation tables, barriers. Every lookup table is
+// replicated so that the lanes of one load phase read distinct banks: IQ2
+// level selectors (8 bytes, 16 copies), IQ2 sign masks (16 bytes, 8 copies),
+// Q2K selectors (4 bytes, 32 copies).
+template <int KIND>
+struct TcLayout {
+  static constexpr bool pair = (KIND == TC_IQ2_PAIR || KIND == TC_BF16_PAIR);
+  static constexpr int stages = pair ? 3 : 4;
+  static constexpr size_t stage_bytes = (pair ? 3 : 2) * kTile;
+  static constexpr size_t b_off = (pair ? 2 : 1) * kTile;  // B tile inside a stage
+  static constexpr size_t tabs = stages * stage_bytes;
+  static constexpr size_t tab_bytes =
+      KIND == TC_IQ2_PAIR ? (256 * 128 + 128 * 128) : (KIND == TC_Q2K ? 256 * 128 : 0);
   static constexpr size_t bars = tabs + tab_bytes;
   static constexpr size_t total = bars + 1024;
 };
+
+// fp16 bytes of the grid levels 8, 25, 43 for prmt: low bytes at 0..2, high
+// bytes at 3..5, so level L is the byte pair (L, 3 + L).
+constexpr uint32_t kHalfLevelsA = 0x48604000u;  // bytes 0x00, 0x40, 0x60, 0x48
+constexpr uint32_t kHalfLevelsB = 0x0000514Eu;  // bytes 0x4E, 0x51
 
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, int* err, volatile int* abort_flag) {
   if (*abort_flag) return false;
@@ -134,6 +147,11 @@ __device__ __forceinline__ uint4 lds128s(uint32_t a) {
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
   return v;
 }
+__device__ __forceinline__ uint2 lds64s(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
 __device__ __forceinline__ uint32_t lds32s(uint32_t a) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
@@ -141,9 +159,11 @@ __device__ __forceinline__ uint32_t lds32s(uint32_t a) {
 }
 
 // One IQ2 row slice (64 weights = two sub-blocks) -> 128 bytes of fp16 in the
-// swizzled tile row at `dst` (row index r within its 8-row atom = r & 7).
-__device__ __forceinline__ void dq_iq2_step(uint4 cw, float dsc, uint32_t dst, int r7, uint32_t tabG, uint32_t tabS,
-                                            uint32_t rep16) {
+// swizzled tile row at `dst` (row index r within its 8-row atom = r & 7). Per
+// group of 8: the grid row gives four prmt selectors (unsigned fp16 pairs),
+// the sign field gives four sign masks, and the sub-block scale multiplies.
+__device__ __forceinline__ void dq_iq2_step(uint4 cw, float dsc, uint32_t dst, int r7, uint32_t tabL, uint32_t tabS,
+                                            uint32_t rep8, uint32_t rep16) {
 #pragma unroll
   for (int sb = 0; sb < 2; ++sb) {
     const uint32_t idx = sb ? cw.z : cw.x, v = sb ? cw.w : cw.y;
@@ -153,13 +173,13 @@ __device__ __forceinline__ void dq_iq2_step(uint4 cw, float dsc, uint32_t dst, i
     for (int e = 0; e < 4; ++e) {
       const uint32_t gi = (idx >> (8 * e)) & 0xFFu;
       const uint32_t si = (v >> (7 * e)) & 0x7Fu;
-      const uint4 G = lds128s(tabG + gi * 64 + rep16);
-      const uint4 S = lds128s(tabS + si * 64 + rep16);
+      const uint2 L = lds64s(tabL + gi * 128 + rep8);
+      const uint4 S = lds128s(tabS + si * 128 + rep16);
       uint4 o;
-      o.x = hmul2_u(G.x ^ S.x, s2);
-      o.y = hmul2_u(G.y ^ S.y, s2);
-      o.z = hmul2_u(G.z ^ S.z, s2);
-      o.w = hmul2_u(G.w ^ S.w, s2);
+      o.x = hmul2_u(prmt(kHalfLevelsA, kHalfLevelsB, L.x) ^ S.x, s2);
+      o.y = hmul2_u(prmt(kHalfLevelsA, kHalfLevelsB, L.x >> 16) ^ S.y, s2);
+      o.z = hmul2_u(prmt(kHalfLevelsA, kHalfLevelsB, L.y) ^ S.z, s2);
+      o.w = hmul2_u(prmt(kHalfLevelsA, kHalfLevelsB, L.y >> 16) ^ S.w, s2);
       sts128(dst + (((sb * 4 + e) ^ r7) << 4), o);
     }
   }
@@ -178,7 +198,7 @@ __device__ __forceinline__ void dq_q2k_half(uint2 qw, uint32_t sc2, float d, flo
     uint32_t o[8];
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-      const uint32_t sel = lds32s(tabQ + ((w >> (8 * b)) & 0xFFu) * 4);
+      const uint32_t sel = lds32s(tabQ + ((w >> (8 * b)) & 0xFFu) * 128);  // tabQ includes lane * 4
       o[2 * b] = prmt(tlo, thi, sel);
       o[2 * b + 1] = prmt(tlo, thi, sel >> 16);
     }
@@ -206,9 +226,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
   constexpr bool PAIR = (KIND == TC_IQ2_PAIR || KIND == TC_BF16_PAIR);
   constexpr bool DQ = (KIND == TC_IQ2_PAIR || KIND == TC_Q2K);
   constexpr bool BF16 = (KIND == TC_BF16_PAIR || KIND == TC_BF16);
+  using L = TcLayout<KIND>;
+  constexpr int kStages = L::stages;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + TcSmem::bars);
+  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + L::bars);
   uint64_t* fullB = fullA + kStages;
   uint64_t* empty = fullB + kStages;
   uint64_t* accf = empty + kStages;  // [2]
@@ -237,33 +259,41 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     *abort_flag = 0;
     fence_barrier_init();
   }
-  // dequantisation tables (4 copies of each 16-byte entry, picked by lane & 3)
-  const uint32_t tabG = sbase + TcSmem::tabs, tabS = tabG + 256 * 64, tabQ = tabG;
+  // dequantisation tables, replicated per load phase (see TcLayout)
+  const uint32_t tabL = sbase + L::tabs, tabS = tabL + 256 * 128, tabQ = sbase + L::tabs + lane * 4;
   if (KIND == TC_IQ2_PAIR) {
-    for (int i = tid; i < 256 * 4 * 4; i += kTcThreads) {  // (entry, copy, word)
-      const int ent = i >> 4, w = i & 3;
-      const uint32_t lv = d_codebook_tc.val[ent][2 * w], hv = d_codebook_tc.val[ent][2 * w + 1];
-      const uint32_t h0 = __half_as_ushort(__float2half_rn(static_cast<float>(lv)));
-      const uint32_t h1 = __half_as_ushort(__float2half_rn(static_cast<float>(hv)));
-      reinterpret_cast<uint32_t*>(smem + TcSmem::tabs)[i] = h0 | (h1 << 16);
+    for (int i = tid; i < 256 * 16 * 2; i += kTcThreads) {  // (row, copy, word): two prmt selectors per word
+      const int ent = i >> 5, w = i & 1;
+      uint32_t word = 0;
+      for (int h = 0; h < 2; ++h) {
+        const int e0 = 4 * w + 2 * h;
+        uint32_t lv[2];
+        for (int q = 0; q < 2; ++q) {
+          const uint32_t v = d_codebook_tc.val[ent][e0 + q];
+          lv[q] = v == 8 ? 0u : (v == 25 ? 1u : 2u);
+        }
+        const uint32_t sel = lv[0] | ((3 + lv[0]) << 4) | (lv[1] << 8) | ((3 + lv[1]) << 12);
+        word |= sel << (16 * h);
+      }
+      reinterpret_cast<uint32_t*>(smem + L::tabs)[i] = word;
     }
-    for (int i = tid; i < 128 * 4 * 4; i += kTcThreads) {
-      const int ent = i >> 4, w = i & 3;
+    for (int i = tid; i < 128 * 8 * 4; i += kTcThreads) {  // (sign field, copy, word)
+      const int ent = i >> 5, w = i & 3;
       uint32_t par = 0;
       for (int b = 0; b < 7; ++b) par ^= (ent >> b) & 1;
       const uint32_t s0 = (2 * w < 7) ? ((ent >> (2 * w)) & 1) : par;
       const uint32_t s1 = (2 * w + 1 < 7) ? ((ent >> (2 * w + 1)) & 1) : par;
-      reinterpret_cast<uint32_t*>(smem + TcSmem::tabs + 256 * 64)[i] = (s0 << 15) | (s1 << 31);
+      reinterpret_cast<uint32_t*>(smem + L::tabs + 256 * 128)[i] = (s0 << 15) | (s1 << 31);
     }
   } else if (KIND == TC_Q2K) {
-    for (int i = tid; i < 256; i += kTcThreads) {  // byte of four 2-bit codes -> two PRMT selectors
+    for (int i = tid; i < 256 * 32; i += kTcThreads) {  // (byte of four 2-bit codes, copy) -> two selectors
+      const int byte = i >> 5;
       uint32_t sel = 0;
       for (int q = 0; q < 4; ++q) {
-        const uint32_t c = (i >> (2 * q)) & 3u;
-        const uint32_t pair = (2 * c) | ((2 * c + 1) << 4);
-        sel |= pair << (8 * q);
+        const uint32_t c = (byte >> (2 * q)) & 3u;
+        sel |= ((2 * c) | ((2 * c + 1) << 4)) << (8 * q);
       }
-      reinterpret_cast<uint32_t*>(smem + TcSmem::tabs)[i] = sel;
+      reinterpret_cast<uint32_t*>(smem + L::tabs)[i] = sel;
     }
   }
   if (warp == kMmaWarp) {
@@ -290,17 +320,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         const int m0 = (u % a.mt) * kMT;
         for (int ks = 0; ks < nks; ++ks) {
           if (!tc_wait(&empty[s], ph ^ 1u, a.err, abort_flag)) break;
-          uint8_t* st = smem + TcSmem::stages + s * TcSmem::stage_bytes;
+          uint8_t* st = smem + s * L::stage_bytes;
           const int kx = (ks % ks_plane) * kKS, pl = ks / ks_plane;
           if (BF16) {
-            mbar_arrive_expect_tx(&fullB[s], (PAIR ? 3 : 2) * kTile);
+            mbar_arrive_expect_tx(&fullB[s], L::stage_bytes);
             // the weight maps are 3-D like every map of this file (one plane)
             tma_load_3d(st, &tm_a0, kx, pr.e * a.rows_e + m0, 0, &fullB[s]);
             if (PAIR) tma_load_3d(st + kTile, &tm_a1, kx, pr.e * a.rows_e + m0, 0, &fullB[s]);
           } else {
             mbar_arrive_expect_tx(&fullB[s], kTile);
           }
-          tma_load_3d(st + 2 * kTile, &tm_b, kx, pr.p0, pl, &fullB[s]);
+          tma_load_3d(st + L::b_off, &tm_b, kx, pr.p0, pl, &fullB[s]);
           ++issued;
           if (++s == kStages) { s = 0; ph ^= 1u; }
         }
@@ -331,9 +361,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           if (!tc_wait(&fullB[s], ph, a.err, abort_flag)) { ok = false; break; }
           if (DQ && !tc_wait(&fullA[s], ph, a.err, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t st = sbase + TcSmem::stages + s * TcSmem::stage_bytes;
+          const uint32_t st = sbase + s * L::stage_bytes;
           const uint64_t da0 = umma_desc_sw128(st), da1 = umma_desc_sw128(st + kTile);
-          const uint64_t db = umma_desc_sw128(st + 2 * kTile);
+          const uint64_t db = umma_desc_sw128(st + L::b_off);
 #pragma unroll
           for (int kk = 0; kk < kKS / 16; ++kk) {
             const uint32_t acc = (ks | kk) ? 1u : 0u;
@@ -352,7 +382,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     }
   } else if (DQ && warp >= kDqWarp0) {
     const int dt = tid - kDqWarp0 * 32;  // 0..255
-    const uint32_t rep16 = (lane & 3) * 16;
+    const uint32_t rep8 = (lane & 15) * 8, rep16 = (lane & 7) * 16;
     int s = 0;
     uint32_t ph = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
@@ -365,35 +395,41 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         const uint8_t* crow = (mat ? a.c1 : a.c0) + grow * (a.K / 4);
         const uint16_t* drow = (mat ? a.d1 : a.d0) + grow * (a.K / 256);
         const uint32_t roff = (r >> 3) * 1024 + (r & 7) * 128 + mat * kTile;
-        // one 256-weight block (four stages) per step; loads run two blocks ahead
+        // one 256-weight block (four stages) per step; loads run two blocks
+        // ahead into three rotating register buffers (no copies of in-flight loads)
         const int nblk = nks / 4;
-        uint4 cur[4], nxt[4], nn[4];
-        uint32_t dcur = 0, dnxt = 0, dnn = 0;
+        uint4 c0[4], c1[4], c2[4];
+        uint32_t e0 = 0, e1 = 0, e2 = 0;
         auto load_blk = [&](int b, uint4 (&dst)[4], uint32_t& dv) {
+          if (b >= nblk) return;
           const uint4* src = reinterpret_cast<const uint4*>(crow + b * 64);
 #pragma unroll
           for (int q = 0; q < 4; ++q) dst[q] = __ldg(src + q);
           dv = __ldg(drow + b);
         };
-        load_blk(0, cur, dcur);
-        if (nblk > 1) load_blk(1, nxt, dnxt);
-        for (int b = 0; b < nblk && ok; ++b) {
-          if (b + 2 < nblk) load_blk(b + 2, nn, dnn);
-          const float dsc = half_bits_to_float(static_cast<uint16_t>(dcur)) * 128.0f;  // d / 8 * 2^10
+        auto run_blk = [&](int b, const uint4 (&cb)[4], uint32_t dv) {
+          if (b >= nblk || !ok) return;
+          const float dsc = half_bits_to_float(static_cast<uint16_t>(dv)) * 128.0f;  // d / 8 * 2^10
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            if (!tc_wait_warp(&empty[s], ph ^ 1u, a.err, abort_flag)) { ok = false; break; }
-            const uint32_t st = sbase + TcSmem::stages + s * TcSmem::stage_bytes;
-            dq_iq2_step(cur[q], dsc, st + roff, r & 7, tabG, tabS, rep16);
+            if (!tc_wait_warp(&empty[s], ph ^ 1u, a.err, abort_flag)) { ok = false; return; }
+            const uint32_t st = sbase + s * L::stage_bytes;
+            dq_iq2_step(cb[q], dsc, st + roff, r & 7, tabL, tabS, rep8, rep16);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&fullA[s]);
             if (++s == kStages) { s = 0; ph ^= 1u; }
           }
-#pragma unroll
-          for (int q = 0; q < 4; ++q) { cur[q] = nxt[q]; nxt[q] = nn[q]; }
-          dcur = dnxt;
-          dnxt = dnn;
+        };
+        load_blk(0, c0, e0);
+        load_blk(1, c1, e1);
+        for (int b = 0; b < nblk && ok; b += 3) {
+          load_blk(b + 2, c2, e2);
+          run_blk(b, c0, e0);
+          load_blk(b + 3, c0, e0);
+          run_blk(b + 1, c1, e1);
+          load_blk(b + 4, c1, e1);
+          run_blk(b + 2, c2, e2);
         }
       } else {  // TC_Q2K: two threads per row, each half of the 64 weights
         const int half = dt >> 7, r = dt & 127;
@@ -403,40 +439,46 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         const uint32_t* ddrow = a.dd + grow * nblk;
         const uint32_t roff = (r >> 3) * 1024 + (r & 7) * 128;
         // one 80-byte block (four stages) per step; loads run two blocks ahead
+        // into three rotating register buffers (no copies of in-flight loads)
         const int nbk = nks / 4;
-        uint4 cur[5], nxt[5], nn[5];
-        uint32_t dcur = 0, dnxt = 0, dnn = 0;
+        uint4 c0[5], c1[5], c2[5];
+        uint32_t e0 = 0, e1 = 0, e2 = 0;
         auto load_blk = [&](int b, uint4 (&dst)[5], uint32_t& dv) {
+          if (b >= nbk) return;
           const uint4* src = reinterpret_cast<const uint4*>(brow + b * 80);
 #pragma unroll
           for (int q = 0; q < 5; ++q) dst[q] = __ldg(src + q);
           dv = __ldg(ddrow + b);
         };
-        load_blk(0, cur, dcur);
-        if (nbk > 1) load_blk(1, nxt, dnxt);
-        for (int b = 0; b < nbk && ok; ++b) {
-          if (b + 2 < nbk) load_blk(b + 2, nn, dnn);
-          const float d = half_bits_to_float(static_cast<uint16_t>(dcur & 0xFFFFu));
-          const float dmin = half_bits_to_float(static_cast<uint16_t>(dcur >> 16));
-          const uint32_t scw[4] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w};
+        auto run_blk = [&](int b, const uint4 (&cb)[5], uint32_t dv) {
+          if (b >= nbk || !ok) return;
+          const float d = half_bits_to_float(static_cast<uint16_t>(dv & 0xFFFFu));
+          const float dmin = half_bits_to_float(static_cast<uint16_t>(dv >> 16));
+          const uint32_t scw[4] = {cb[0].x, cb[0].y, cb[0].z, cb[0].w};
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             // sub-blocks 4q4 + 2half, +1: q bytes 16 + 16q4 + 8half, scale bytes 4q4 + 2half
-            const uint4 qv = cur[1 + q4];
+            const uint4 qv = cb[1 + q4];
             const uint2 qw = half ? make_uint2(qv.z, qv.w) : make_uint2(qv.x, qv.y);
             const uint32_t sc2 = (scw[q4] >> (16 * half)) & 0xFFFFu;
-            if (!tc_wait_warp(&empty[s], ph ^ 1u, a.err, abort_flag)) { ok = false; break; }
-            const uint32_t st = sbase + TcSmem::stages + s * TcSmem::stage_bytes;
+            if (!tc_wait_warp(&empty[s], ph ^ 1u, a.err, abort_flag)) { ok = false; return; }
+            const uint32_t st = sbase + s * L::stage_bytes;
             dq_q2k_half(qw, sc2, d, dmin, st + roff, r & 7, 4 * half, tabQ);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&fullA[s]);
             if (++s == kStages) { s = 0; ph ^= 1u; }
           }
-#pragma unroll
-          for (int q = 0; q < 5; ++q) { cur[q] = nxt[q]; nxt[q] = nn[q]; }
-          dcur = dnxt;
-          dnxt = dnn;
+        };
+        load_blk(0, c0, e0);
+        load_blk(1, c1, e1);
+        for (int b = 0; b < nbk && ok; b += 3) {
+          load_blk(b + 2, c2, e2);
+          run_blk(b, c0, e0);
+          load_blk(b + 3, c0, e0);
+          run_blk(b + 1, c1, e1);
+          load_blk(b + 4, c1, e1);
+          run_blk(b + 2, c2, e2);
         }
       }
       if (!ok) break;
@@ -656,7 +698,7 @@ bool tc_map(CUtensorMap* m, const void* base, bool bf16, uint64_t K, uint64_t ro
 template <int KIND>
 int launch_tc(const CUtensorMap& mb, const CUtensorMap& ma0, const CUtensorMap& ma1, const TcArgs& a, int sms,
               cudaStream_t st) {
-  const size_t smem = TcSmem::total;
+  const size_t smem = TcLayout<KIND>::total;
   cudaFuncSetAttribute(tc_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   tc_gemm_kernel<KIND><<<sms, kTcThreads, smem, st>>>(mb, ma0, ma1, a);
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
