@@ -76,7 +76,7 @@ int launch_router_tc(const uint16_t* Wr, const float* bias, const uint16_t* x, i
                      int* err, int sms, cudaStream_t st);
 
 // Tensor-core grouped GEMM for many tokens (prefill.cu).
-constexpr int kPrefillMinT = 16;
+constexpr int kPrefillMinT = 4;
 bool prefill_path_supported(const LayerShape& s, int T);
 size_t prefill_workspace_bytes(const LayerShape& s, int T);
 int launch_ffn_prefill(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,

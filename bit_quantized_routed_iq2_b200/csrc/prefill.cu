@@ -29,7 +29,13 @@
 // subnormals for the scales this library's generator and real checkpoints use
 // (|d| in [2^-24, 2^5]); the 2^10 is taken out in the fp32 epilogue. Q2K values
 // q*d*sc - dmin*m are formed in fp32 per sub-block and rounded once to fp16.
-// Activations and h enter as fp16 (routed) or as bf16 hi + lo parts (shared).
+// Routed activations enter as fp16(x * 2^-e) with one power-of-2 exponent e per
+// token (largest element just below 2^13), h as fp16(h * 2^(-2e-12)), and the
+// down outputs leave as fp16(o * 2^(-2e-12)) (h and o scale with x squared);
+// the epilogues and the combine undo the exponents exactly, so activations of
+// any magnitude stay inside the fp16 range (a chained residual stream grows
+// layer by layer). The shared expert
+// takes bf16 x and bf16 hi + lo parts of h.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -74,6 +80,8 @@ struct TcPair {
 };
 
 struct TcArgs {
+  int n_experts;  // weight blocks (experts) the tiles may name
+  int b_rows;     // rows of one B plane (bound of every tile)
   int rows_e;    // weight rows per expert
   int K;         // reduction length of one plane
   int mt;        // 128-row tiles per expert
@@ -87,6 +95,7 @@ struct TcArgs {
   const int32_t* npairs;
   int dense_rows;          // with pairs == null: tiles of 128 rows over this many B rows, expert 0
   const float* bias;       // TC_BF16 only: added per weight row (router bias), may be null
+  const int32_t* row_exp;  // routed kinds: power-of-2 exponent e of each B row (see the epilogues)
   void* out;
   int ldo;        // output row stride in elements
   int out_rows;   // rows of one output plane (bf16 hi/lo output)
@@ -209,13 +218,22 @@ __device__ __forceinline__ void dq_q2k_half(uint2 qw, uint32_t sc2, float d, flo
 
 __device__ __forceinline__ float silu_mul_tc(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
+// Tile i of the list; a tile outside the operands' bounds comes back with
+// n = 0 (every role then skips it) and records MOE_ERR_INVALID_ARG.
 __device__ __forceinline__ TcPair tc_pair(const TcArgs& a, int i) {
-  if (a.pairs) return a.pairs[i];
   TcPair p;
-  p.e = 0;
-  p.p0 = i * kNT;
-  p.n = min(kNT, a.dense_rows - i * kNT);
-  p.pad = 0;
+  if (a.pairs) {
+    p = a.pairs[i];
+  } else {
+    p.e = 0;
+    p.p0 = i * kNT;
+    p.n = min(kNT, a.dense_rows - i * kNT);
+    p.pad = 0;
+  }
+  if (p.e < 0 || p.e >= a.n_experts || p.p0 < 0 || p.n < 1 || p.n > kNT || p.p0 + p.n > a.b_rows) {
+    if (a.err) atomicCAS(a.err, 0, ERR_ARG);
+    p.n = 0;
+  }
   return p;
 }
 
@@ -318,6 +336,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       for (int u = blockIdx.x; u < nunits && !*abort_flag; u += gridDim.x) {
         const TcPair pr = tc_pair(a, u / a.mt);
         const int m0 = (u % a.mt) * kMT;
+        if (pr.n == 0) continue;
         for (int ks = 0; ks < nks; ++ks) {
           if (!tc_wait(&empty[s], ph ^ 1u, a.err, abort_flag)) break;
           uint8_t* st = smem + s * L::stage_bytes;
@@ -348,8 +367,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       int s = 0;
       uint32_t ph = 0;
       int t = 0;
-      for (int u = blockIdx.x; u < nunits && !*abort_flag; u += gridDim.x, ++t) {
+      for (int u = blockIdx.x; u < nunits && !*abort_flag; u += gridDim.x) {
         const TcPair pr = tc_pair(a, u / a.mt);
+        if (pr.n == 0) continue;
         const int n16 = (pr.n + 15) & ~15;
         const uint32_t id = (idesc & ~(0x3Fu << 17)) | (static_cast<uint32_t>(n16 >> 3) << 17);
         const int buf = t & 1;
@@ -375,6 +395,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         }
         if (!ok) break;
         umma_commit(&accf[buf]);
+        ++t;
       }
       // drain: every MMA issued by this thread completes before TMEM is freed
       umma_commit(drain);
@@ -388,6 +409,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const TcPair pr = tc_pair(a, u / a.mt);
       const int m0 = (u % a.mt) * kMT;
+      if (pr.n == 0) continue;
       bool ok = true;
       if (KIND == TC_IQ2_PAIR) {
         const int mat = dt >> 7, r = dt & 127;
@@ -486,9 +508,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
   } else if (warp < kEpiWarps) {
     const int r = 32 * warp + lane;  // TMEM lane = weight row of the tile
     int t = 0;
-    for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++t) {
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const TcPair pr = tc_pair(a, u / a.mt);
       const int m0 = (u % a.mt) * kMT;
+      if (pr.n == 0) continue;
       const int buf = t & 1;
       if (!tc_wait_warp(&accf[buf], (t >> 1) & 1, a.err, abort_flag)) break;
       tc_fence_after();
@@ -505,8 +528,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           if (n >= pr.n) break;
           const size_t orow = static_cast<size_t>(pr.p0 + n);
           if (KIND == TC_IQ2_PAIR) {
-            const float h = silu_mul_tc(__uint_as_float(g[j]) * a.oscale, __uint_as_float(v[j]) * a.oscale);
-            reinterpret_cast<__half*>(a.out)[orow * a.ldo + row] = __float2half_rn(h);
+            // B row = x * 2^-e: g, u come back as exact fp32 rescalings; h leaves as
+            // fp16(h * 2^(-2e-12)), the scale that keeps it inside the fp16 range
+            const int ex = a.row_exp[orow];
+            const float sc = ldexpf(a.oscale, ex);
+            const float h = silu_mul_tc(__uint_as_float(g[j]) * sc, __uint_as_float(v[j]) * sc);
+            reinterpret_cast<__half*>(a.out)[orow * a.ldo + row] = __float2half_rn(ldexpf(h, -2 * ex - 12));
           } else if (KIND == TC_BF16_PAIR) {
             const float h = silu_mul_tc(__uint_as_float(g[j]), __uint_as_float(v[j]));
             const __nv_bfloat16 hi = __float2bfloat16_rn(h);
@@ -514,6 +541,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             reinterpret_cast<__nv_bfloat16*>(a.out)[orow * a.ldo + row] = hi;
             reinterpret_cast<__nv_bfloat16*>(a.out)[(static_cast<size_t>(a.out_rows) + orow) * a.ldo + row] = lo;
           } else if (KIND == TC_Q2K) {  // routed expert outputs, combined later in slot order
+            // B row = h * 2^(-2e-12), so the accumulator is o * 2^(-2e-12) (h and o are
+            // quadratic in x); it is stored as is and the combine applies 2^(2e+12)
             reinterpret_cast<__half*>(a.out)[orow * a.ldo + row] = __float2half_rn(__uint_as_float(g[j]) * a.oscale);
           } else {
             const float bv = (KIND == TC_BF16 && a.bias) ? a.bias[row] : 0.f;
@@ -524,6 +553,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acce[buf]);
+      ++t;
     }
   }
   __syncthreads();
@@ -539,6 +569,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
 namespace moe {
 namespace {
 
+// Power-of-2 exponent per token: e = floor(log2 max|x_t|) - 12 (0 for a zero
+// row), so x * 2^-e lies below 2^13 in magnitude and well inside fp16.
+template <typename XT>
+__global__ void __launch_bounds__(256) token_exp_kernel(const XT* __restrict__ x, int T, int H,
+                                                        int32_t* __restrict__ texp) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (t >= T) return;
+  float m = 0.f;
+  for (int i = lane; i < H; i += 32) {
+    float v;
+    if constexpr (sizeof(XT) == 4) v = reinterpret_cast<const float*>(x)[static_cast<size_t>(t) * H + i];
+    else v = __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(x)[static_cast<size_t>(t) * H + i]) << 16);
+    m = fmaxf(m, fabsf(v));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) texp[t] = m > 0.f ? floor_log2_pos(m) - 12 : 0;
+}
+
 // Expert-sorted fp16 copy of the activations for the routed B operand, and the
 // tile lists: routed (expert, first assignment, count) tiles of up to 128
 // assignments, and shared tiles of up to 128 tokens. Block 0 also clears the
@@ -550,7 +599,8 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(const XT* __restrict_
                                                            const int32_t* __restrict__ active, int E,
                                                            TcPair* __restrict__ pairs, int32_t* __restrict__ npairs,
                                                            TcPair* __restrict__ spairs, int32_t* __restrict__ nspairs,
-                                                           int* __restrict__ err_word) {
+                                                           const int32_t* __restrict__ texp,
+                                                           int32_t* __restrict__ aexp, int* __restrict__ err_word) {
   const int nA = T * k;
   if (blockIdx.x == 0 && threadIdx.x < 32) {
     const int lane = threadIdx.x;
@@ -599,7 +649,10 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(const XT* __restrict_
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const int p = static_cast<int>(i / per), c = static_cast<int>(i % per);
-    const size_t src = static_cast<size_t>(perm[p] / k) * H + c * 8;
+    const int tok = perm[p] / k;
+    const int ex = texp[tok];
+    if (c == 0) aexp[p] = ex;
+    const size_t src = static_cast<size_t>(tok) * H + c * 8;
     float v[8];
     if constexpr (sizeof(XT) == 4) {
       const float4 a0 = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + src);
@@ -612,6 +665,8 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(const XT* __restrict_
       v[4] = __uint_as_float(w.z << 16); v[5] = __uint_as_float(w.z & 0xFFFF0000u);
       v[6] = __uint_as_float(w.w << 16); v[7] = __uint_as_float(w.w & 0xFFFF0000u);
     }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) v[q] = ldexpf(v[q], -ex);
     uint4 o;
     o.x = f2_to_h2(v[0], v[1]);
     o.y = f2_to_h2(v[2], v[3]);
@@ -634,19 +689,22 @@ __global__ void __launch_bounds__(256) bf16_parts_kernel(const float* __restrict
 }
 
 // y[t][h] = sum_j w[t][j] o[inv[t*k+j]][h] (j ascending) + s[t][h] (+ residual),
-// with the routed expert outputs o stored as fp16 (relative rounding 2^-11,
-// an order below the 2e-3 bound) to halve the traffic of this pass.
+// with the routed expert outputs stored as fp16 o * 2^(-2e-12) of their token
+// (relative rounding 2^-11, an order below the 2e-3 bound) to halve the
+// traffic of this pass; w * 2^(2e+12) is exact.
 __global__ void __launch_bounds__(256) prefill_combine_kernel(int T, int H, int k, const float* __restrict__ topk_w,
                                                               const int32_t* __restrict__ inv,
-                                                              const __half* __restrict__ o, const float* s,
+                                                              const __half* __restrict__ o,
+                                                              const int32_t* __restrict__ texp, const float* s,
                                                               const float* residual, float* y) {
   const size_t n4 = static_cast<size_t>(T) * H / 4;
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const int t = static_cast<int>((i * 4) / H), h = static_cast<int>((i * 4) % H);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float tsc = ldexpf(1.0f, 2 * texp[t] + 12);  // the routed outputs arrive as o * 2^(-2e-12)
     for (int j = 0; j < k; ++j) {
-      const float w = topk_w[t * k + j];
+      const float w = topk_w[t * k + j] * tsc;
       const uint2 hv = *reinterpret_cast<const uint2*>(o + static_cast<size_t>(inv[t * k + j]) * H + h);
       const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
       const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
@@ -714,6 +772,8 @@ struct PrefillWs {
   TcPair* pairs;
   TcPair* spairs;
   int32_t* counts;
+  int32_t* texp;  // per token
+  int32_t* aexp;  // per assignment
   size_t bytes;
 };
 
@@ -735,6 +795,8 @@ PrefillWs carve_prefill(const LayerShape& sh, int T, char* base) {
   w.pairs = reinterpret_cast<TcPair*>(take((static_cast<size_t>(sh.E) + nA / kNT + 1) * sizeof(TcPair)));
   w.spairs = reinterpret_cast<TcPair*>(take((static_cast<size_t>(T) / kNT + 1) * sizeof(TcPair)));
   w.counts = reinterpret_cast<int32_t*>(take(64));
+  w.texp = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * 4));
+  w.aexp = reinterpret_cast<int32_t*>(take(nA * 4));
   w.bytes = off;
   return w;
 }
@@ -753,6 +815,7 @@ int launch_router_tc(const uint16_t* Wr, const float* bias, const uint16_t* x, i
   CUtensorMap mb, ma;
   if (!tc_map(&mb, x, true, H, T, 1) || !tc_map(&ma, Wr, true, H, E, 1)) return ERR_CUDA;
   TcArgs a{};
+  a.n_experts = 1; a.b_rows = T;
   a.rows_e = E; a.K = H; a.mt = E / kMT; a.planes = 1;
   a.dense_rows = T; a.bias = bias; a.out = logits; a.ldo = E; a.out_rows = T;
   a.oscale = 1.0f; a.err = err; a.clear_err = 1;
@@ -777,13 +840,18 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
     ProfScope ps(MOE_K_PREP, st);
     const int grid = std::max(1, std::min(sms * 4, (nA * (sh.H / 8) + 255) / 256));
     if (x_dtype == 0)
+      token_exp_kernel<float><<<(T + 7) / 8, 256, 0, st>>>(static_cast<const float*>(x), T, sh.H, pw.texp);
+    else
+      token_exp_kernel<uint16_t><<<(T + 7) / 8, 256, 0, st>>>(static_cast<const uint16_t*>(x), T, sh.H, pw.texp);
+    if (x_dtype == 0)
       prefill_prep_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), T, sh.H, sh.k, r.perm, pw.xp,
                                                        r.offsets, r.active, sh.E, pw.pairs, pw.counts, pw.spairs,
-                                                       pw.counts + 1, clear_status ? err : nullptr);
+                                                       pw.counts + 1, pw.texp, pw.aexp, clear_status ? err : nullptr);
     else
       prefill_prep_kernel<uint16_t><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), T, sh.H, sh.k, r.perm,
                                                           pw.xp, r.offsets, r.active, sh.E, pw.pairs, pw.counts,
-                                                          pw.spairs, pw.counts + 1, clear_status ? err : nullptr);
+                                                          pw.spairs, pw.counts + 1, pw.texp, pw.aexp,
+                                                          clear_status ? err : nullptr);
     if (sh.Is > 0 && x_dtype == 0) {
       const size_t n = static_cast<size_t>(T) * sh.H;
       bf16_parts_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const float*>(x), n, pw.xb);
@@ -795,10 +863,11 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
     ProfScope ps(MOE_K_PREFILL_GATEUP, st);
     if (!tc_map(&mb, pw.xp, false, sh.H, nA, 1)) return ERR_CUDA;
     TcArgs a{};
+    a.n_experts = sh.E; a.b_rows = nA;
     a.rows_e = sh.I; a.K = sh.H; a.mt = sh.I / kMT; a.planes = 1;
     a.c0 = w.gate_codes; a.d0 = w.gate_d; a.c1 = w.up_codes; a.d1 = w.up_d;
     a.pairs = pw.pairs; a.npairs = pw.counts; a.out = pw.hh; a.ldo = sh.I; a.out_rows = nA;
-    a.oscale = 1.0f / 1024.0f; a.err = err;
+    a.oscale = 1.0f / 1024.0f; a.err = err; a.row_exp = pw.aexp;
     rc |= launch_tc<TC_IQ2_PAIR>(mb, mb, mb, a, sms, st);
   }
   if (sh.Is > 0) {
@@ -809,6 +878,7 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
         !tc_map(&ma1, w.sh_up, true, sh.H, sh.Is, 1))
       return ERR_CUDA;
     TcArgs a{};
+    a.n_experts = 1; a.b_rows = T;
     a.rows_e = sh.Is; a.K = sh.H; a.mt = sh.Is / kMT; a.planes = planes;
     a.dense_rows = T; a.out = pw.hs; a.ldo = sh.Is; a.out_rows = T;
     a.oscale = 1.0f; a.err = err;
@@ -818,16 +888,18 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
     ProfScope ps(MOE_K_PREFILL_DOWN, st);
     if (!tc_map(&mb, pw.hh, false, sh.I, nA, 1)) return ERR_CUDA;
     TcArgs a{};
+    a.n_experts = sh.E; a.b_rows = nA;
     a.rows_e = sh.H; a.K = sh.I; a.mt = sh.H / kMT; a.planes = 1;
     a.c0 = w.down_codes; a.dd = w.down_dd;
     a.pairs = pw.pairs; a.npairs = pw.counts; a.out = pw.o; a.ldo = sh.H; a.out_rows = nA;
-    a.oscale = 1.0f; a.err = err;
+    a.oscale = 1.0f; a.err = err; a.row_exp = pw.aexp;
     rc |= launch_tc<TC_Q2K>(mb, mb, mb, a, sms, st);
   }
   if (sh.Is > 0) {
     ProfScope ps(MOE_K_SHARED_DOWN, st);
     if (!tc_map(&mb, pw.hs, true, sh.Is, T, 2) || !tc_map(&ma0, w.sh_down, true, sh.Is, sh.H, 1)) return ERR_CUDA;
     TcArgs a{};
+    a.n_experts = 1; a.b_rows = T;
     a.rows_e = sh.H; a.K = sh.Is; a.mt = sh.H / kMT; a.planes = 2;
     a.dense_rows = T; a.out = pw.s; a.ldo = sh.H; a.out_rows = T;
     a.oscale = 1.0f; a.err = err;
@@ -836,7 +908,7 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
   {
     ProfScope ps(MOE_K_COMBINE, st);
     const int grid = std::max(1, std::min(sms * 8, static_cast<int>((static_cast<size_t>(T) * sh.H / 4 + 255) / 256)));
-    prefill_combine_kernel<<<grid, 256, 0, st>>>(T, sh.H, sh.k, r.topk_w, r.inv, pw.o, sh.Is > 0 ? pw.s : nullptr,
+    prefill_combine_kernel<<<grid, 256, 0, st>>>(T, sh.H, sh.k, r.topk_w, r.inv, pw.o, pw.texp, sh.Is > 0 ? pw.s : nullptr,
                                                  residual, y);
   }
   if (rc != OK) return ERR_CUDA;

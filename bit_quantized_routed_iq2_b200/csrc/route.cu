@@ -155,7 +155,8 @@ __device__ __forceinline__ void topk_warp(const float* __restrict__ lrow, int E,
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
     const int e = lane + 32 * i;
-    l[i] = e < E ? lrow[e] : -INFINITY;
+    const float v = e < E ? lrow[e] : -INFINITY;
+    l[i] = v == v ? v : -INFINITY;  // a NaN logit ranks last, so every index stays valid
   }
   uint32_t taken = 0;
   float chosen[16];

@@ -158,16 +158,22 @@ SMALL_CASES = {
     "flat_blocks_k1": _small(H=256, I=64, E=4, k=1, Is=32, T=9, seed=0x5A14),
     "single_expert": _small(E=1, k=1, Is=0, T=5, seed=0x5A15),
     "k_eq_E": _small(E=4, k=4, T=7, seed=0x5A16),
-    # shapes served by the TMA-fed GEMVs (H % 1024 == 0, I % 512 == 0, T <= 16)
+    # shapes served by the TMA-fed GEMVs (H % 1024 == 0, I % 512 == 0; T <= 4 unless the
+    # tensor-core path cannot take the shape)
     "tma_t1": _small(H=1024, I=512, E=16, k=4, Is=64, T=1, seed=0x5A17),
     "tma_t5": _small(H=2048, I=1024, E=8, k=4, Is=128, T=5, seed=0x5A18),
     "tma_t16": _small(H=1024, I=512, E=8, k=4, Is=64, T=16, seed=0x5A19),
     "tma_t16_zipf_f32": _small(H=1024, I=1024, E=12, k=3, Is=0, T=16, x_dtype="f32", zipf=True, seed=0x5A1A),
-    # shapes served by the tensor-core grouped GEMM (T > 16, H, I, I_s multiples of 128 / 256)
+    "tma_t3_shared_experts": _small(H=1024, I=512, E=4, k=4, Is=128, T=3, seed=0x5A20),
+    # shapes served by the tensor-core grouped GEMM (T > 4, H, I multiples of 256, I_s of 128)
     "tc_t17": _small(H=512, I=256, E=4, k=2, Is=128, T=17, seed=0x5A1B),
     "tc_t64_f32": _small(H=1024, I=512, E=8, k=2, Is=256, T=64, x_dtype="f32", seed=0x5A1C),
     "tc_t200_zipf": _small(H=768, I=512, E=16, k=4, Is=0, T=200, zipf=True, seed=0x5A1D),
     "tc_t300_many_tiles": _small(H=1280, I=768, E=2, k=1, Is=384, T=300, seed=0x5A1E),
+    # activations far from unit scale: the fp16 operands of the tensor-core path carry a
+    # power-of-2 exponent per token, so neither overflow (g * u beyond 65504) nor underflow
+    "tc_t40_large_x": _small(H=512, I=256, E=8, k=2, Is=128, T=40, x_std=300.0, seed=0x5A21),
+    "tc_t40_small_x_f32": _small(H=512, I=256, E=8, k=2, Is=128, T=40, x_dtype="f32", x_std=1e-3, seed=0x5A22),
     # router logits on the tensor cores too (bf16 x, T > 64, E % 128 == 0)
     "tc_router_t130": _small(H=512, I=256, E=128, k=4, Is=128, T=130, seed=0x5A1F),
 }
