@@ -53,8 +53,10 @@ constexpr int kGuW = 128;                    // code bytes per gate/up box row (
 constexpr int kGuBox = kBoxRows * kGuW;      // 32 KB
 constexpr int kDnW = 80;                     // one Q2K-style block per down box row
 constexpr int kDnBox = kBoxRows * kDnW;      // 20 KB
-constexpr uint32_t kSgnOff = 32768;          // sign table after the level table (32 KB)
-constexpr int kTabWords = (256 + 128) * 32;  // both tables, each entry replicated for the 32 lanes
+// Selector tables, each entry replicated for the 32 lanes: grid row i at byte
+// 256*i + 4*lane, sign field s at byte 256*s + 128 + 4*lane (interleaved, so
+// that one prmt turns a grid index byte into its table address).
+constexpr int kTabBytes = 256 * 256;
 constexpr int kZeroBytes = 1024;             // zero operand region for idle MMA columns
 constexpr int kRowPad = 32;                  // padding of a staged activation row
 constexpr int kMaxExpertsTma = 1024;
@@ -203,7 +205,7 @@ __device__ __forceinline__ GuUnit gu_unit_of(const GuIter& t, const MetaSmem& ms
 }
 
 struct GuCtx {
-  const char* tab;      // level table, then sign table at +kSgnOff (static shared memory)
+  const char* tab;      // interleaved level and sign tables (start of dynamic shared memory)
   const uint8_t* ring;
   uint64_t* full;
   uint64_t* empty;
@@ -213,16 +215,16 @@ struct GuCtx {
   const int32_t* tok;
   uint32_t ring_s, x_s, xs_s, zero_s;  // shared-window addresses (staged variant)
   int xpitch, warp, lane, g, tig, S;
-  uint32_t lane4, rot_idx, rot_sig;
+  uint32_t lane4, sel_idx, rot_sig, sgn_lane;
 };
 
 // Selector word (level nibbles | sign bits) of grid group `tig` of one 8-byte
 // sub-block record -> two int8x4 A registers.
 __device__ __forceinline__ void iq2_operand(const GuCtx& c, uint2 rec, uint32_t& lo, uint32_t& hi) {
-  const uint32_t al = (rotr(rec.x, c.rot_idx) & 0x7F80u) | c.lane4;
-  const uint32_t as = (rotr(rec.y, c.rot_sig) & 0x3F80u) | c.lane4;
-  const uint32_t sel = *reinterpret_cast<const uint32_t*>(c.tab + al) |
-                       *reinterpret_cast<const uint32_t*>(c.tab + kSgnOff + as);
+  const uint32_t al = prmt(rec.x, c.lane4, c.sel_idx);                  // 256 * index byte + 4 * lane
+  const uint32_t as = (rotr(rec.y, c.rot_sig) & 0x7F00u) | c.sgn_lane;  // 256 * sign field + 128 + 4 * lane
+  // level codes sit in bits 0-1 of each nibble and signs in bit 2: the sum is the union
+  const uint32_t sel = *reinterpret_cast<const uint32_t*>(c.tab + al) + *reinterpret_cast<const uint32_t*>(c.tab + as);
   lo = prmt(kPosBytes, kNegBytes, sel);
   hi = prmt(kPosBytes, kNegBytes, __umulhi(sel, 0x10000u));
 }
@@ -443,14 +445,16 @@ __device__ __forceinline__ bool gu_unit_multi(const GuTmaArgs& a, const GuCtx& c
 }
 
 
-// Shared-memory plan of the gate/up kernel's dynamic part (host and device
-// agree on it); the selector tables are static shared memory.
+// Shared-memory plan of the gate/up kernel (host and device agree on it); the
+// selector tables come first, at a fixed shared address, so lookups need no
+// base add.
 struct GuPlan {
-  size_t meta, zero, x, xs, ring, bars, total;
+  size_t tab, meta, zero, x, xs, ring, bars, total;
 };
 __host__ __device__ inline GuPlan gu_plan(int E, int T, int k, int H, bool xs_in, int S) {
   GuPlan p;
-  p.meta = 0;
+  p.tab = 0;
+  p.meta = kTabBytes;
   p.zero = p.meta + meta_bytes(E, T * k, true);
   p.x = p.zero + kZeroBytes;
   p.xs = p.x + (xs_in ? align_up(static_cast<size_t>(T) * 2 * (H + kRowPad), 128) : 0);
@@ -465,8 +469,6 @@ template <int MAXQ, bool XS>
 __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_constant__ CUtensorMap tm_gate,
                                                                   const __grid_constant__ CUtensorMap tm_up,
                                                                   GuTmaArgs a) {
-  // replicated selector tables at a fixed shared address, so lookups need no base add
-  __shared__ __align__(128) uint32_t s_tab[kTabWords];
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H, I = a.I, T = a.T, S = a.S, NB = a.NB;
@@ -495,8 +497,11 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
     }
     fence_barrier_init();
   }
-  for (int i = tid; i < 256 * 32; i += kThreadsT) s_tab[i] = d_sel_tables2.level[i >> 5];
-  for (int i = tid; i < 128 * 32; i += kThreadsT) s_tab[256 * 32 + i] = d_sel_tables2.sign[i >> 5];
+  for (int i = tid; i < kTabBytes / 4; i += kThreadsT) {
+    const int ent = i >> 6;
+    reinterpret_cast<uint32_t*>(smem + pl.tab)[i] =
+        (i & 32) == 0 ? d_sel_tables2.level[ent] : (ent < 128 ? d_sel_tables2.sign[ent] : 0u);
+  }
   for (int i = tid; i < kZeroBytes / 16; i += kThreadsT) reinterpret_cast<uint4*>(zero)[i] = make_uint4(0, 0, 0, 0);
   load_meta(ms, a.offsets, a.active, a.perm, a.E, nA, a.k, tid, kThreadsT);
   if (XS) {
@@ -528,7 +533,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
   }
 
   GuCtx c;
-  c.tab = reinterpret_cast<const char*>(s_tab);
+  c.tab = reinterpret_cast<const char*>(smem + pl.tab);
   c.ring = ring;
   c.full = full;
   c.empty = empty;
@@ -554,8 +559,9 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
   c.tig = lane & 3;
   c.S = S;
   c.lane4 = static_cast<uint32_t>(lane) << 2;
-  c.rot_idx = (8u * c.tig - 7u) & 31u;
-  c.rot_sig = (7u * c.tig - 7u) & 31u;
+  c.sel_idx = 0x5504u | (static_cast<uint32_t>(c.tig) << 4);  // bytes: lane4, index byte tig, 0, 0
+  c.rot_sig = (7u * c.tig - 8u) & 31u;                          // sign field tig to bits 8..14
+  c.sgn_lane = 128u + c.lane4;
   const int row_l = 16 * warp + c.g;
   const int dstride = H / 256;
   // per-row fp16 scales of a unit: for box j the pair of super-blocks 2(kp*NB+j), +1
@@ -1057,7 +1063,7 @@ int launch_gateup_tma(const LayerShape& sh, const uint8_t* gate_codes, const uin
   a.gate_d = gate_d; a.up_d = up_d; a.xd = xd; a.xs = xs;
   a.offsets = r.offsets; a.perm = r.perm; a.active = r.active; a.gpart = gpart; a.err = err;
   // stage the activations when that still leaves three ring stages
-  const size_t budget = kBudget - kTabWords * 4;  // the selector tables are static shared memory
+  const size_t budget = kBudget;
   const bool xs_in = gu_plan(sh.E, T, sh.k, sh.H, true, 3).total <= budget;
   int S = 2;
   while (S < 6 && gu_plan(sh.E, T, sh.k, sh.H, xs_in, S + 1).total <= budget) ++S;

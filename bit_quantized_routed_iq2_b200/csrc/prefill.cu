@@ -12,20 +12,22 @@
 //
 // Weights are the M operand (128 rows per tile) and the tokens routed to an
 // expert are the N operand (up to 128 per tile), so one dequantised weight tile
-// is multiplied by all of the expert's tokens. Per CTA (one per SM, 512
+// is multiplied by all of the expert's tokens. Per CTA (one per SM, 768
 // threads):
 //   warps 0-3   epilogue: TMEM -> registers -> SwiGLU / scaling -> global
 //   warp 4      producer: TMA loads of the token tiles (and bf16 weight tiles)
 //   warp 5      TMEM allocation; one lane issues the MMAs and commits
-//   warps 8-15  dequantisers: 2-bit codes -> fp16 weight tiles (128-byte swizzle)
+//   warps 8-23  dequantisers: 2-bit codes -> fp16 weight tiles (128-byte swizzle),
+//               each thread one sub-block of one row per stage
 // Stages of (A tiles, B tile) circulate through full/empty mbarriers; the MMA
 // completion (tcgen05.commit) frees a stage. Two accumulator buffers in TMEM
 // let the epilogue of one tile overlap the MMAs of the next. Every wait is
 // bounded: a time-out records MOE_ERR_TIMEOUT, all roles stop, and the CTA
 // drains its in-flight copies and MMAs before freeing TMEM.
 //
-// Precision: routed weights enter the MMA as fp16. IQ2 values are formed as
-// fp16(d*(2ls+1)*2^10/8) * grid * sign, which keeps them clear of fp16
+// Precision: routed weights enter the MMA as fp16. IQ2 values are the fp16
+// rounding of s * grid with s = fp16(d*(2ls+1)*2^10/8), the sign applied
+// exactly afterwards, which keeps them clear of fp16
 // subnormals for the scales this library's generator and real checkpoints use
 // (|d| in [2^-24, 2^5]); the 2^10 is taken out in the fp32 epilogue. Q2K values
 // q*d*sc - dmin*m are formed in fp32 per sub-block and rounded once to fp16.
@@ -53,12 +55,12 @@
 namespace moe {
 namespace {
 
-constexpr int kTcThreads = 512;
+constexpr int kTcThreads = 768;
 constexpr int kEpiWarps = 4;     // warps 0-3
 constexpr int kProdWarp = 4;
 constexpr int kMmaWarp = 5;
-constexpr int kDqWarp0 = 8;      // warps 8-15
-constexpr int kDqWarps = 8;
+constexpr int kDqWarp0 = 8;      // warps 8-23
+constexpr int kDqWarps = 16;
 constexpr int kMT = 128;         // weight rows per tile (MMA M)
 constexpr int kNT = 128;         // max tokens per tile (MMA N)
 constexpr int kKS = 64;          // K per stage: 128 bytes of fp16 per row
@@ -122,10 +124,10 @@ struct TcLayout {
   static constexpr size_t total = bars + 1024;
 };
 
-// fp16 bytes of the grid levels 8, 25, 43 for prmt: low bytes at 0..2, high
-// bytes at 3..5, so level L is the byte pair (L, 3 + L).
-constexpr uint32_t kHalfLevelsA = 0x48604000u;  // bytes 0x00, 0x40, 0x60, 0x48
-constexpr uint32_t kHalfLevelsB = 0x0000514Eu;  // bytes 0x4E, 0x51
+// fp16 grid levels; scaled per sub-block into prmt source bytes with the low
+// bytes at 0..2 and the high bytes at 3..5, so level L is the byte pair (L, 3 + L).
+constexpr uint32_t kHalf8And25 = 0x4E404800u;   // fp16 pair (8, 25)
+constexpr uint32_t kHalf43Twice = 0x51605160u;  // fp16 pair (43, 43)
 
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, int* err, volatile int* abort_flag) {
   if (*abort_flag) return false;
@@ -167,53 +169,57 @@ __device__ __forceinline__ uint32_t lds32s(uint32_t a) {
   return v;
 }
 
-// One IQ2 row slice (64 weights = two sub-blocks) -> 128 bytes of fp16 in the
-// swizzled tile row at `dst` (row index r within its 8-row atom = r & 7). Per
-// group of 8: the grid row gives four prmt selectors (unsigned fp16 pairs),
-// the sign field gives four sign masks, and the sub-block scale multiplies.
-__device__ __forceinline__ void dq_iq2_step(uint4 cw, float dsc, uint32_t dst, int r7, uint32_t tabL, uint32_t tabS,
-                                            uint32_t rep8, uint32_t rep16) {
+// One IQ2 sub-block of a row (32 weights: an 8-byte record of four grid
+// index bytes and a word holding four 7-bit sign fields and the 4-bit scale)
+// -> 64 bytes of fp16 at four 16-byte chunks of the swizzled tile row; `dst`
+// already carries the row's swizzle and the sub-block's chunk base, and chunk
+// e is reached by XOR with 16e. The three scaled levels s*8, s*25, s*43 are
+// rounded to fp16 once and laid out as prmt source bytes (low bytes at 0..2,
+// high bytes at 3..5, the byte positions the level selectors expect); per
+// group of 8 the grid row gives four prmt selectors and the sign field four
+// fp16 pairs of +-1 that multiply exactly, so each weight is the fp16 rounding
+// of (+-level) * s. Shifts are written as multiplications so that the
+// compiler may place them on the multiply-add pipe beside the prmt work.
+__device__ __forceinline__ void dq_iq2_sub(uint2 rec, float dsc, uint32_t dst, uint32_t tabL, uint32_t tabS) {
+  const uint32_t idx = rec.x, v = rec.y;
+  const float sf = dsc * static_cast<float>(2 * __umulhi(v, 16u) + 1);  // v >> 28 = ls
+  const uint32_t s2 = f2_to_h2(sf, sf);
+  const uint32_t t01 = hmul2_u(kHalf8And25, s2), t2 = hmul2_u(kHalf43Twice, s2);
+  const uint32_t srcA = prmt(t01, t2, 0x1420u), srcB = prmt(t01, t2, 0x0053u);
 #pragma unroll
-  for (int sb = 0; sb < 2; ++sb) {
-    const uint32_t idx = sb ? cw.z : cw.x, v = sb ? cw.w : cw.y;
-    const float sf = dsc * static_cast<float>(2 * (v >> 28) + 1);
-    const uint32_t s2 = f2_to_h2(sf, sf);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t gi = (idx >> (8 * e)) & 0xFFu;
-      const uint32_t si = (v >> (7 * e)) & 0x7Fu;
-      const uint2 L = lds64s(tabL + gi * 128 + rep8);
-      const uint4 S = lds128s(tabS + si * 128 + rep16);
-      uint4 o;
-      o.x = hmul2_u(prmt(kHalfLevelsA, kHalfLevelsB, L.x) ^ S.x, s2);
-      o.y = hmul2_u(prmt(kHalfLevelsA, kHalfLevelsB, L.x >> 16) ^ S.y, s2);
-      o.z = hmul2_u(prmt(kHalfLevelsA, kHalfLevelsB, L.y) ^ S.z, s2);
-      o.w = hmul2_u(prmt(kHalfLevelsA, kHalfLevelsB, L.y >> 16) ^ S.w, s2);
-      sts128(dst + (((sb * 4 + e) ^ r7) << 4), o);
-    }
+  for (int e = 0; e < 4; ++e) {
+    // byte e of idx at bits 7..14 (x 128-byte entries), sign field e likewise
+    const uint32_t gsh = e == 0 ? idx * 128u : __umulhi(idx, 1u << (39 - 8 * e));
+    const uint32_t ssh = e == 0 ? v * 128u : (e == 1 ? v : __umulhi(v, 1u << (39 - 7 * e)));
+    const uint2 L = lds64s(tabL + (gsh & 0x7F80u));
+    const uint4 S = lds128s(tabS + (ssh & 0x3F80u));
+    uint4 o;
+    o.x = hmul2_u(prmt(srcA, srcB, L.x), S.x);
+    o.y = hmul2_u(prmt(srcA, srcB, __umulhi(L.x, 0x10000u)), S.y);
+    o.z = hmul2_u(prmt(srcA, srcB, L.y), S.z);
+    o.w = hmul2_u(prmt(srcA, srcB, __umulhi(L.y, 0x10000u)), S.w);
+    sts128(dst ^ (e << 4), o);
   }
 }
 
-// Half a Q2K row slice (32 weights = two 16-weight sub-blocks) -> 64 bytes of
-// fp16 at chunks c0, c0+1, c0+2, c0+3 of the swizzled tile row.
-__device__ __forceinline__ void dq_q2k_half(uint2 qw, uint32_t sc2, float d, float dmin, uint32_t dst, int r7, int c0,
-                                            uint32_t tabQ) {
+// One Q2K sub-block of a row (16 weights, four per byte of `w`: weight 4b+i at
+// bits 8b+2i) with scale byte `scb` (sc | m << 4) -> 32 bytes of fp16 at two
+// 16-byte chunks (dst, dst ^ 16) of the swizzled tile row. The four values
+// d*sc*q - dmin*m, q = 0..3, are the prmt source bytes.
+__device__ __forceinline__ void dq_q2k_sub(uint32_t w, uint32_t scb, float d, float dmin, uint32_t dst,
+                                           uint32_t tabQ) {
+  const float A = d * static_cast<float>(scb & 15u), B = dmin * static_cast<float>(scb >> 4);
+  const uint32_t tlo = f2_to_h2(-B, A - B), thi = f2_to_h2(2.f * A - B, 3.f * A - B);
+  uint32_t o[8];
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const uint32_t scb = (sc2 >> (8 * j)) & 0xFFu;
-    const float A = d * static_cast<float>(scb & 15u), B = dmin * static_cast<float>(scb >> 4);
-    const uint32_t tlo = f2_to_h2(-B, A - B), thi = f2_to_h2(2.f * A - B, 3.f * A - B);
-    const uint32_t w = j ? qw.y : qw.x;  // 16 weights, weight 4b+i at bits 8b+2i
-    uint32_t o[8];
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const uint32_t sel = lds32s(tabQ + ((w >> (8 * b)) & 0xFFu) * 128);  // tabQ includes lane * 4
-      o[2 * b] = prmt(tlo, thi, sel);
-      o[2 * b + 1] = prmt(tlo, thi, sel >> 16);
-    }
-    sts128(dst + (((c0 + 2 * j) ^ r7) << 4), make_uint4(o[0], o[1], o[2], o[3]));
-    sts128(dst + (((c0 + 2 * j + 1) ^ r7) << 4), make_uint4(o[4], o[5], o[6], o[7]));
+  for (int b = 0; b < 4; ++b) {
+    const uint32_t ent = b == 0 ? w * 128u : __umulhi(w, 1u << (39 - 8 * b));  // byte b at bits 7..14
+    const uint32_t sel = lds32s(tabQ + (ent & 0x7F80u));                       // tabQ includes lane * 4
+    o[2 * b] = prmt(tlo, thi, sel);
+    o[2 * b + 1] = prmt(tlo, thi, __umulhi(sel, 0x10000u));
   }
+  sts128(dst, make_uint4(o[0], o[1], o[2], o[3]));
+  sts128(dst ^ 16u, make_uint4(o[4], o[5], o[6], o[7]));
 }
 
 __device__ __forceinline__ float silu_mul_tc(float g, float u) { return g / (1.0f + expf(-g)) * u; }
@@ -278,7 +284,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     fence_barrier_init();
   }
   // dequantisation tables, replicated per load phase (see TcLayout)
-  const uint32_t tabL = sbase + L::tabs, tabS = tabL + 256 * 128, tabQ = sbase + L::tabs + lane * 4;
+  // replica of this lane folded into the table bases (entries are 128 bytes apart)
+  const uint32_t tabL = sbase + L::tabs + (lane & 15) * 8, tabS = sbase + L::tabs + 256 * 128 + (lane & 7) * 16,
+                 tabQ = sbase + L::tabs + lane * 4;
   if (KIND == TC_IQ2_PAIR) {
     for (int i = tid; i < 256 * 16 * 2; i += kTcThreads) {  // (row, copy, word): two prmt selectors per word
       const int ent = i >> 5, w = i & 1;
@@ -301,7 +309,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       for (int b = 0; b < 7; ++b) par ^= (ent >> b) & 1;
       const uint32_t s0 = (2 * w < 7) ? ((ent >> (2 * w)) & 1) : par;
       const uint32_t s1 = (2 * w + 1 < 7) ? ((ent >> (2 * w + 1)) & 1) : par;
-      reinterpret_cast<uint32_t*>(smem + L::tabs + 256 * 128)[i] = (s0 << 15) | (s1 << 31);
+      // fp16 pair of +-1 (0x3C00 / 0xBC00)
+      reinterpret_cast<uint32_t*>(smem + L::tabs + 256 * 128)[i] = 0x3C003C00u | (s0 << 15) | (s1 << 31);
     }
   } else if (KIND == TC_Q2K) {
     for (int i = tid; i < 256 * 32; i += kTcThreads) {  // (byte of four 2-bit codes, copy) -> two selectors
@@ -402,8 +411,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       mbar_wait_bounded(drain, 0, nullptr, 0);
     }
   } else if (DQ && warp >= kDqWarp0) {
-    const int dt = tid - kDqWarp0 * 32;  // 0..255
-    const uint32_t rep8 = (lane & 15) * 8, rep16 = (lane & 7) * 16;
+    // sixteen warps; each thread turns one sub-block of one row into fp16 per stage
+    const int dt = tid - kDqWarp0 * 32;  // 0..511
     int s = 0;
     uint32_t ph = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
@@ -412,31 +421,34 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       if (pr.n == 0) continue;
       bool ok = true;
       if (KIND == TC_IQ2_PAIR) {
-        const int mat = dt >> 7, r = dt & 127;
+        // thread = (matrix, row, sub-block half of the stage's 64 weights)
+        const int mat = dt >> 8, r = (dt >> 1) & 127, hf = dt & 1;
         const size_t grow = static_cast<size_t>(pr.e) * a.rows_e + m0 + r;
-        const uint8_t* crow = (mat ? a.c1 : a.c0) + grow * (a.K / 4);
+        const uint8_t* crow = (mat ? a.c1 : a.c0) + grow * (a.K / 4) + 8 * hf;
         const uint16_t* drow = (mat ? a.d1 : a.d0) + grow * (a.K / 256);
-        const uint32_t roff = (r >> 3) * 1024 + (r & 7) * 128 + mat * kTile;
-        // one 256-weight block (four stages) per step; loads run two blocks
-        // ahead into three rotating register buffers (no copies of in-flight loads)
+        // row base in the stage | the row's swizzle | chunk base 4*hf (chunks c ^ (r & 7))
+        const uint32_t roff = ((r >> 3) * 1024 + (r & 7) * 128 + mat * kTile) | ((r & 7) << 4);
+        const uint32_t cx = static_cast<uint32_t>(hf) << 6;
+        // one 256-weight block (four stages, one record each) per step; loads run two
+        // blocks ahead into three rotating register buffers (no copies of in-flight loads)
         const int nblk = nks / 4;
-        uint4 c0[4], c1[4], c2[4];
+        uint2 c0[4], c1[4], c2[4];
         uint32_t e0 = 0, e1 = 0, e2 = 0;
-        auto load_blk = [&](int b, uint4 (&dst)[4], uint32_t& dv) {
+        auto load_blk = [&](int b, uint2 (&dst)[4], uint32_t& dv) {
           if (b >= nblk) return;
-          const uint4* src = reinterpret_cast<const uint4*>(crow + b * 64);
+          const uint8_t* src = crow + b * 64;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) dst[q] = __ldg(src + q);
+          for (int q = 0; q < 4; ++q) dst[q] = __ldg(reinterpret_cast<const uint2*>(src + 16 * q));
           dv = __ldg(drow + b);
         };
-        auto run_blk = [&](int b, const uint4 (&cb)[4], uint32_t dv) {
+        auto run_blk = [&](int b, const uint2 (&cb)[4], uint32_t dv) {
           if (b >= nblk || !ok) return;
           const float dsc = half_bits_to_float(static_cast<uint16_t>(dv)) * 128.0f;  // d / 8 * 2^10
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             if (!tc_wait_warp(&empty[s], ph ^ 1u, a.err, abort_flag)) { ok = false; return; }
             const uint32_t st = sbase + s * L::stage_bytes;
-            dq_iq2_step(cb[q], dsc, st + roff, r & 7, tabL, tabS, rep8, rep16);
+            dq_iq2_sub(cb[q], dsc, (st + roff) ^ cx, tabL, tabS);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&fullA[s]);
@@ -453,54 +465,56 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           load_blk(b + 4, c1, e1);
           run_blk(b + 2, c2, e2);
         }
-      } else {  // TC_Q2K: two threads per row, each half of the 64 weights
-        const int half = dt >> 7, r = dt & 127;
+      } else {  // TC_Q2K: thread = (row, quarter qt of the stage's 64 weights = one sub-block)
+        const int r = dt >> 2, qt = dt & 3;
         const size_t grow = static_cast<size_t>(pr.e) * a.rows_e + m0 + r;
         const int nblk = a.K / 256;
         const uint8_t* brow = a.c0 + grow * nblk * 80;
         const uint32_t* ddrow = a.dd + grow * nblk;
-        const uint32_t roff = (r >> 3) * 1024 + (r & 7) * 128;
-        // one 80-byte block (four stages) per step; loads run two blocks ahead
-        // into three rotating register buffers (no copies of in-flight loads)
+        const uint32_t roff = ((r >> 3) * 1024 + (r & 7) * 128) | ((r & 7) << 4);
+        const uint32_t cx = static_cast<uint32_t>(qt) << 5;  // chunks 2qt, 2qt + 1
+        const uint32_t sshift = 8u * qt;
+        // one 80-byte block (four stages) per step: the 16 scale bytes, the thread's four
+        // q words (sub-blocks 4q + qt) and dd; loads run two blocks ahead as above
         const int nbk = nks / 4;
-        uint4 c0[5], c1[5], c2[5];
+        uint4 s0, s1, s2, w0, w1, w2;
         uint32_t e0 = 0, e1 = 0, e2 = 0;
-        auto load_blk = [&](int b, uint4 (&dst)[5], uint32_t& dv) {
+        auto load_blk = [&](int b, uint4& sc, uint4& qw, uint32_t& dv) {
           if (b >= nbk) return;
-          const uint4* src = reinterpret_cast<const uint4*>(brow + b * 80);
-#pragma unroll
-          for (int q = 0; q < 5; ++q) dst[q] = __ldg(src + q);
+          const uint8_t* src = brow + b * 80;
+          sc = __ldg(reinterpret_cast<const uint4*>(src));
+          qw.x = __ldg(reinterpret_cast<const uint32_t*>(src + 16 + 4 * qt));
+          qw.y = __ldg(reinterpret_cast<const uint32_t*>(src + 32 + 4 * qt));
+          qw.z = __ldg(reinterpret_cast<const uint32_t*>(src + 48 + 4 * qt));
+          qw.w = __ldg(reinterpret_cast<const uint32_t*>(src + 64 + 4 * qt));
           dv = __ldg(ddrow + b);
         };
-        auto run_blk = [&](int b, const uint4 (&cb)[5], uint32_t dv) {
+        auto run_blk = [&](int b, const uint4& sc, const uint4& qw, uint32_t dv) {
           if (b >= nbk || !ok) return;
           const float d = half_bits_to_float(static_cast<uint16_t>(dv & 0xFFFFu));
           const float dmin = half_bits_to_float(static_cast<uint16_t>(dv >> 16));
-          const uint32_t scw[4] = {cb[0].x, cb[0].y, cb[0].z, cb[0].w};
+          const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
+          const uint32_t qws[4] = {qw.x, qw.y, qw.z, qw.w};
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            // sub-blocks 4q4 + 2half, +1: q bytes 16 + 16q4 + 8half, scale bytes 4q4 + 2half
-            const uint4 qv = cb[1 + q4];
-            const uint2 qw = half ? make_uint2(qv.z, qv.w) : make_uint2(qv.x, qv.y);
-            const uint32_t sc2 = (scw[q4] >> (16 * half)) & 0xFFFFu;
+          for (int q = 0; q < 4; ++q) {
             if (!tc_wait_warp(&empty[s], ph ^ 1u, a.err, abort_flag)) { ok = false; return; }
             const uint32_t st = sbase + s * L::stage_bytes;
-            dq_q2k_half(qw, sc2, d, dmin, st + roff, r & 7, 4 * half, tabQ);
+            dq_q2k_sub(qws[q], (scw[q] >> sshift) & 0xFFu, d, dmin, (st + roff) ^ cx, tabQ);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&fullA[s]);
             if (++s == kStages) { s = 0; ph ^= 1u; }
           }
         };
-        load_blk(0, c0, e0);
-        load_blk(1, c1, e1);
+        load_blk(0, s0, w0, e0);
+        load_blk(1, s1, w1, e1);
         for (int b = 0; b < nbk && ok; b += 3) {
-          load_blk(b + 2, c2, e2);
-          run_blk(b, c0, e0);
-          load_blk(b + 3, c0, e0);
-          run_blk(b + 1, c1, e1);
-          load_blk(b + 4, c1, e1);
-          run_blk(b + 2, c2, e2);
+          load_blk(b + 2, s2, w2, e2);
+          run_blk(b, s0, w0, e0);
+          load_blk(b + 3, s0, w0, e0);
+          run_blk(b + 1, s1, w1, e1);
+          load_blk(b + 4, s1, w1, e1);
+          run_blk(b + 2, s2, w2, e2);
         }
       }
       if (!ok) break;
