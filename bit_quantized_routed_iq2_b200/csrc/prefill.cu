@@ -106,22 +106,35 @@ struct TcArgs {
   int clear_err;  // CTA 0 clears *err at start (first kernel of a call)
 };
 
-// Shared-memory layout per kernel kind: stages of (A0, A1 for the pair kinds,
-// B), the replicated dequantisation tables, barriers. Every lookup table is
-// replicated so that the lanes of one load phase read distinct banks: IQ2
-// level selectors (8 bytes, 16 copies), IQ2 sign masks (16 bytes, 8 copies),
-// Q2K selectors (4 bytes, 32 copies).
+// Memory plan per kernel kind.
+// Dequantising kinds: the fp16 weight tiles (A) go from registers into TMEM
+// (tcgen05.st) and the MMA reads A from there, so shared memory carries only
+// the token tiles (B, a TMA ring of its own) and the replicated lookup tables:
+// IQ2 level selectors (8 bytes, 16 copies), IQ2 signs as fp16 +-1 pairs (16
+// bytes, 8 copies), Q2K selectors (4 bytes, 32 copies); every copy serves the
+// lanes of one load phase, so lookups are free of bank conflicts.
+// bf16 kinds: A and B tiles both arrive by TMA into one ring of stages.
+// TMEM (512 columns): A stages at columns [0, 256) for the dequantising kinds,
+// accumulators above them; the bf16 kinds double-buffer the accumulators over
+// all 512 columns.
 template <int KIND>
 struct TcLayout {
+  static constexpr bool dq = (KIND == TC_IQ2_PAIR || KIND == TC_Q2K);
   static constexpr bool pair = (KIND == TC_IQ2_PAIR || KIND == TC_BF16_PAIR);
-  static constexpr int stages = pair ? 3 : 4;
-  static constexpr size_t stage_bytes = (pair ? 3 : 2) * kTile;
-  static constexpr size_t b_off = (pair ? 2 : 1) * kTile;  // B tile inside a stage
+  static constexpr int stages = dq ? 8 : (pair ? 4 : 6);                 // shared-memory ring
+  static constexpr size_t stage_bytes = (dq ? 1 : (pair ? 3 : 2)) * kTile;
+  static constexpr size_t b_off = dq ? 0 : (pair ? 2 : 1) * kTile;      // B tile inside a stage
+  static constexpr int a_stages = KIND == TC_IQ2_PAIR ? 4 : 8;           // TMEM A ring (dq kinds)
+  static constexpr uint32_t a_cols = pair ? 64 : 32;                     // TMEM columns per A stage
+  static constexpr int acc_bufs = KIND == TC_IQ2_PAIR ? 1 : 2;
+  static constexpr uint32_t acc_base = dq ? 256 : 0;
+  static constexpr uint32_t acc_stride = KIND == TC_Q2K ? 128 : 256;    // columns per accumulator buffer
   static constexpr size_t tabs = stages * stage_bytes;
   static constexpr size_t tab_bytes =
       KIND == TC_IQ2_PAIR ? (256 * 128 + 128 * 128) : (KIND == TC_Q2K ? 256 * 128 : 0);
   static constexpr size_t bars = tabs + tab_bytes;
   static constexpr size_t total = bars + 1024;
+  static_assert(total <= 227 * 1024, "shared memory plan too large");
 };
 
 // fp16 grid levels; scaled per sub-block into prmt source bytes with the low
@@ -171,16 +184,14 @@ __device__ __forceinline__ uint32_t lds32s(uint32_t a) {
 
 // One IQ2 sub-block of a row (32 weights: an 8-byte record of four grid
 // index bytes and a word holding four 7-bit sign fields and the 4-bit scale)
-// -> 64 bytes of fp16 at four 16-byte chunks of the swizzled tile row; `dst`
-// already carries the row's swizzle and the sub-block's chunk base, and chunk
-// e is reached by XOR with 16e. The three scaled levels s*8, s*25, s*43 are
-// rounded to fp16 once and laid out as prmt source bytes (low bytes at 0..2,
-// high bytes at 3..5, the byte positions the level selectors expect); per
-// group of 8 the grid row gives four prmt selectors and the sign field four
-// fp16 pairs of +-1 that multiply exactly, so each weight is the fp16 rounding
-// of (+-level) * s. Shifts are written as multiplications so that the
-// compiler may place them on the multiply-add pipe beside the prmt work.
-__device__ __forceinline__ void dq_iq2_sub(uint2 rec, float dsc, uint32_t dst, uint32_t tabL, uint32_t tabS) {
+// -> 16 words of fp16 pairs in K order. The three scaled levels s*8, s*25,
+// s*43 are rounded to fp16 once and laid out as prmt source bytes (low bytes
+// at 0..2, high bytes at 3..5, the byte positions the level selectors
+// expect); per group of 8 the grid row gives four prmt selectors and the sign
+// field four fp16 pairs of +-1 that multiply exactly, so each weight is the
+// fp16 rounding of (+-level) * s. Shifts are written as multiplications so
+// that the compiler may place them on the multiply-add pipe beside the prmt work.
+__device__ __forceinline__ void dq_iq2_sub(uint2 rec, float dsc, uint32_t tabL, uint32_t tabS, uint32_t (&o)[16]) {
   const uint32_t idx = rec.x, v = rec.y;
   const float sf = dsc * static_cast<float>(2 * __umulhi(v, 16u) + 1);  // v >> 28 = ls
   const uint32_t s2 = f2_to_h2(sf, sf);
@@ -193,24 +204,20 @@ __device__ __forceinline__ void dq_iq2_sub(uint2 rec, float dsc, uint32_t dst, u
     const uint32_t ssh = e == 0 ? v * 128u : (e == 1 ? v : __umulhi(v, 1u << (39 - 7 * e)));
     const uint2 L = lds64s(tabL + (gsh & 0x7F80u));
     const uint4 S = lds128s(tabS + (ssh & 0x3F80u));
-    uint4 o;
-    o.x = hmul2_u(prmt(srcA, srcB, L.x), S.x);
-    o.y = hmul2_u(prmt(srcA, srcB, __umulhi(L.x, 0x10000u)), S.y);
-    o.z = hmul2_u(prmt(srcA, srcB, L.y), S.z);
-    o.w = hmul2_u(prmt(srcA, srcB, __umulhi(L.y, 0x10000u)), S.w);
-    sts128(dst ^ (e << 4), o);
+    o[4 * e + 0] = hmul2_u(prmt(srcA, srcB, L.x), S.x);
+    o[4 * e + 1] = hmul2_u(prmt(srcA, srcB, __umulhi(L.x, 0x10000u)), S.y);
+    o[4 * e + 2] = hmul2_u(prmt(srcA, srcB, L.y), S.z);
+    o[4 * e + 3] = hmul2_u(prmt(srcA, srcB, __umulhi(L.y, 0x10000u)), S.w);
   }
 }
 
 // One Q2K sub-block of a row (16 weights, four per byte of `w`: weight 4b+i at
-// bits 8b+2i) with scale byte `scb` (sc | m << 4) -> 32 bytes of fp16 at two
-// 16-byte chunks (dst, dst ^ 16) of the swizzled tile row. The four values
-// d*sc*q - dmin*m, q = 0..3, are the prmt source bytes.
-__device__ __forceinline__ void dq_q2k_sub(uint32_t w, uint32_t scb, float d, float dmin, uint32_t dst,
-                                           uint32_t tabQ) {
+// bits 8b+2i) with scale byte `scb` (sc | m << 4) -> 8 words of fp16 pairs in
+// K order. The four values d*sc*q - dmin*m, q = 0..3, are the prmt source bytes.
+__device__ __forceinline__ void dq_q2k_sub(uint32_t w, uint32_t scb, float d, float dmin, uint32_t tabQ,
+                                           uint32_t (&o)[8]) {
   const float A = d * static_cast<float>(scb & 15u), B = dmin * static_cast<float>(scb >> 4);
   const uint32_t tlo = f2_to_h2(-B, A - B), thi = f2_to_h2(2.f * A - B, 3.f * A - B);
-  uint32_t o[8];
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     const uint32_t ent = b == 0 ? w * 128u : __umulhi(w, 1u << (39 - 8 * b));  // byte b at bits 7..14
@@ -218,11 +225,25 @@ __device__ __forceinline__ void dq_q2k_sub(uint32_t w, uint32_t scb, float d, fl
     o[2 * b] = prmt(tlo, thi, sel);
     o[2 * b + 1] = prmt(tlo, thi, __umulhi(sel, 0x10000u));
   }
-  sts128(dst, make_uint4(o[0], o[1], o[2], o[3]));
-  sts128(dst ^ 16u, make_uint4(o[4], o[5], o[6], o[7]));
+}
+
+// One lane of the (converged) warp returns true, the same lane every time.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile("{\n .reg .pred P;\n elect.sync _|P, 0xffffffff;\n selp.u32 %0, 1, 0, P;\n}\n" : "=r"(p));
+  return p != 0;
 }
 
 __device__ __forceinline__ float silu_mul_tc(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+// x * 2^k as two exact power-of-2 multiplications (each factor a normal
+// float), the same value as ldexpf for results in the normal range; k is
+// clamped to [-252, 252], beyond which every finite fp32 x under- or overflows.
+__device__ __forceinline__ float mul_pow2(float x, int k) {
+  k = max(-252, min(252, k));
+  const int k1 = k >> 1, k2 = k - k1;
+  return x * __int_as_float((k1 + 127) << 23) * __int_as_float((k2 + 127) << 23);
+}
 
 // Tile i of the list; a tile outside the operands' bounds comes back with
 // n = 0 (every role then skips it) and records MOE_ERR_INVALID_ARG.
@@ -252,14 +273,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
   constexpr bool BF16 = (KIND == TC_BF16_PAIR || KIND == TC_BF16);
   using L = TcLayout<KIND>;
   constexpr int kStages = L::stages;
+  constexpr int kAStages = L::a_stages;
+  constexpr int kAccBufs = L::acc_bufs;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + L::bars);
-  uint64_t* fullB = fullA + kStages;
-  uint64_t* empty = fullB + kStages;
-  uint64_t* accf = empty + kStages;  // [2]
-  uint64_t* acce = accf + 2;         // [2]
-  uint64_t* drain = acce + 2;
+  uint64_t* fullB = reinterpret_cast<uint64_t*>(smem + L::bars);  // [kStages] shared-memory ring
+  uint64_t* emptyB = fullB + kStages;
+  uint64_t* fullA = emptyB + kStages;  // [kAStages] TMEM A ring (dequantising kinds)
+  uint64_t* emptyA = fullA + kAStages;
+  uint64_t* accf = emptyA + kAStages;  // [kAccBufs]
+  uint64_t* acce = accf + kAccBufs;    // [kAccBufs]
+  uint64_t* drain = acce + kAccBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t sbase = smem_addr(smem);
@@ -271,11 +295,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
   if (tid == 0 && blockIdx.x == 0 && a.clear_err) *a.err = 0;
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&fullA[s], kDqWarps);
       mbar_init(&fullB[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&emptyB[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(&fullA[s], kDqWarps);
+      mbar_init(&emptyA[s], 1);
+    }
+    for (int b = 0; b < kAccBufs; ++b) {
       mbar_init(&accf[b], 1);
       mbar_init(&acce[b], kEpiWarps);
     }
@@ -283,8 +310,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     *abort_flag = 0;
     fence_barrier_init();
   }
-  // dequantisation tables, replicated per load phase (see TcLayout)
-  // replica of this lane folded into the table bases (entries are 128 bytes apart)
+  // dequantisation tables, replicated per load phase (see TcLayout); the
+  // replica of this lane is folded into the table bases (entries 128 bytes apart)
   const uint32_t tabL = sbase + L::tabs + (lane & 15) * 8, tabS = sbase + L::tabs + 256 * 128 + (lane & 7) * 16,
                  tabQ = sbase + L::tabs + lane * 4;
   if (KIND == TC_IQ2_PAIR) {
@@ -347,7 +374,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         const int m0 = (u % a.mt) * kMT;
         if (pr.n == 0) continue;
         for (int ks = 0; ks < nks; ++ks) {
-          if (!tc_wait(&empty[s], ph ^ 1u, a.err, abort_flag)) break;
+          if (!tc_wait(&emptyB[s], ph ^ 1u, a.err, abort_flag)) break;
           uint8_t* st = smem + s * L::stage_bytes;
           const int kx = (ks % ks_plane) * kKS, pl = ks / ks_plane;
           if (BF16) {
@@ -371,64 +398,97 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       }
     }
   } else if (warp == kMmaWarp) {
-    if (lane == 0) {
-      const uint32_t idesc = umma_idesc_f16(kMT, 16, BF16);  // N patched per tile
-      int s = 0;
-      uint32_t ph = 0;
-      int t = 0;
-      for (int u = blockIdx.x; u < nunits && !*abort_flag; u += gridDim.x) {
-        const TcPair pr = tc_pair(a, u / a.mt);
-        if (pr.n == 0) continue;
-        const int n16 = (pr.n + 15) & ~15;
-        const uint32_t id = (idesc & ~(0x3Fu << 17)) | (static_cast<uint32_t>(n16 >> 3) << 17);
-        const int buf = t & 1;
-        if (!tc_wait(&acce[buf], ((t >> 1) & 1) ^ 1u, a.err, abort_flag)) break;
+    // the whole warp runs the loop (waits and operand arithmetic stay warp-uniform)
+    // and one elected lane issues the MMAs and their commits
+    const uint32_t idesc = umma_idesc_f16(kMT, 16, BF16);  // N patched per tile
+    const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+    int s = 0, sa = 0;
+    uint32_t ph = 0, pha = 0;
+    int t = 0;
+    // the abort flag is read once per lane, so its test is made warp-uniform
+    for (int u = blockIdx.x; u < nunits && !__any_sync(0xffffffffu, *abort_flag != 0); u += gridDim.x) {
+      const TcPair pr = tc_pair(a, u / a.mt);
+      if (pr.n == 0) continue;
+      const int n16 = (pr.n + 15) & ~15;
+      const uint32_t id = (idesc & ~(0x3Fu << 17)) | (static_cast<uint32_t>(n16 >> 3) << 17);
+      const int buf = t % kAccBufs;
+      if (!tc_wait_warp(&acce[buf], ((t / kAccBufs) & 1) ^ 1u, a.err, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t d0 = tm + L::acc_base + buf * L::acc_stride, d1 = d0 + 128;
+      bool ok = true;
+      for (int ks = 0; ks < nks; ++ks) {
+        if (!tc_wait_warp(&fullB[s], ph, a.err, abort_flag)) { ok = false; break; }
+        if (DQ && !tc_wait_warp(&fullA[sa], pha, a.err, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d0 = tmem + buf * 256, d1 = d0 + 128;
-        bool ok = true;
-        for (int ks = 0; ks < nks; ++ks) {
-          if (!tc_wait(&fullB[s], ph, a.err, abort_flag)) { ok = false; break; }
-          if (DQ && !tc_wait(&fullA[s], ph, a.err, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t st = sbase + s * L::stage_bytes;
-          const uint64_t da0 = umma_desc_sw128(st), da1 = umma_desc_sw128(st + kTile);
-          const uint64_t db = umma_desc_sw128(st + L::b_off);
+        const uint32_t st = sbase + s * L::stage_bytes;
+        const uint64_t db = umma_desc_sw128(st + L::b_off);
+        if (DQ) {
+          const uint32_t at = tm + sa * L::a_cols;  // gate (or the single matrix), up at +32
+          if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < kKS / 16; ++kk) {
-            const uint32_t acc = (ks | kk) ? 1u : 0u;
-            umma_f16(d0, da0 + 2 * kk, db + 2 * kk, id, acc);  // +32 bytes along K per step
-            if (PAIR) umma_f16(d1, da1 + 2 * kk, db + 2 * kk, id, acc);
+            for (int kk = 0; kk < kKS / 16; ++kk) {
+              const uint32_t acc = (ks | kk) ? 1u : 0u;
+              umma_f16_ts(d0, at + 8 * kk, db + 2 * kk, id, acc);  // 16 fp16 = 8 columns of A per step
+              if (PAIR) umma_f16_ts(d1, at + 32 + 8 * kk, db + 2 * kk, id, acc);
+            }
+            umma_commit(&emptyA[sa]);
+            umma_commit(&emptyB[s]);
           }
-          umma_commit(&empty[s]);
-          if (++s == kStages) { s = 0; ph ^= 1u; }
+          __syncwarp();
+          if (++sa == kAStages) { sa = 0; pha ^= 1u; }
+        } else {
+          const uint64_t da0 = umma_desc_sw128(st), da1 = umma_desc_sw128(st + kTile);
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < kKS / 16; ++kk) {
+              const uint32_t acc = (ks | kk) ? 1u : 0u;
+              umma_f16(d0, da0 + 2 * kk, db + 2 * kk, id, acc);  // +32 bytes along K per step
+              if (PAIR) umma_f16(d1, da1 + 2 * kk, db + 2 * kk, id, acc);
+            }
+            umma_commit(&emptyB[s]);
+          }
+          __syncwarp();
         }
-        if (!ok) break;
-        umma_commit(&accf[buf]);
-        ++t;
+        if (++s == kStages) { s = 0; ph ^= 1u; }
       }
-      // drain: every MMA issued by this thread completes before TMEM is freed
-      umma_commit(drain);
-      mbar_wait_bounded(drain, 0, nullptr, 0);
+      if (!ok) break;
+      if (elect_one()) umma_commit(&accf[buf]);
+      __syncwarp();
+      ++t;
     }
+    // drain: every MMA issued by this warp completes before TMEM is freed
+    if (elect_one()) umma_commit(drain);
+    __syncwarp();
+    mbar_wait_bounded(drain, 0, nullptr, 0);
   } else if (DQ && warp >= kDqWarp0) {
-    // sixteen warps; each thread turns one sub-block of one row into fp16 per stage
-    const int dt = tid - kDqWarp0 * 32;  // 0..511
-    int s = 0;
-    uint32_t ph = 0;
+    // sixteen warps; warp w may write TMEM lanes 32*(w%4)..+31, so the row is
+    // 32*(w%4) + lane and the four warps of a lane quarter split each stage's
+    // weights of their rows; each thread turns one sub-block into fp16 per stage
+    const int quarter = warp & 3, part = (warp - kDqWarp0) >> 2;  // part 0..3
+    const int r = 32 * quarter + lane;
+    const uint32_t tlane = static_cast<uint32_t>(32 * quarter) << 16;
+    int sa = 0;
+    uint32_t pha = 0;
+    // one stage: wait for the A slot, fill this thread's columns, publish
+    auto publish = [&](bool ok) {
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (ok && lane == 0) mbar_arrive(&fullA[sa]);
+      if (++sa == kAStages) { sa = 0; pha ^= 1u; }
+    };
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const TcPair pr = tc_pair(a, u / a.mt);
       const int m0 = (u % a.mt) * kMT;
       if (pr.n == 0) continue;
       bool ok = true;
       if (KIND == TC_IQ2_PAIR) {
-        // thread = (matrix, row, sub-block half of the stage's 64 weights)
-        const int mat = dt >> 8, r = (dt >> 1) & 127, hf = dt & 1;
+        // part = (matrix, sub-block half of the stage's 64 weights)
+        const int mat = part >> 1, hf = part & 1;
         const size_t grow = static_cast<size_t>(pr.e) * a.rows_e + m0 + r;
         const uint8_t* crow = (mat ? a.c1 : a.c0) + grow * (a.K / 4) + 8 * hf;
         const uint16_t* drow = (mat ? a.d1 : a.d0) + grow * (a.K / 256);
-        // row base in the stage | the row's swizzle | chunk base 4*hf (chunks c ^ (r & 7))
-        const uint32_t roff = ((r >> 3) * 1024 + (r & 7) * 128 + mat * kTile) | ((r & 7) << 4);
-        const uint32_t cx = static_cast<uint32_t>(hf) << 6;
+        const uint32_t tcol = tlane + mat * 32 + hf * 16;
         // one 256-weight block (four stages, one record each) per step; loads run two
         // blocks ahead into three rotating register buffers (no copies of in-flight loads)
         const int nblk = nks / 4;
@@ -446,13 +506,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           const float dsc = half_bits_to_float(static_cast<uint16_t>(dv)) * 128.0f;  // d / 8 * 2^10
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            if (!tc_wait_warp(&empty[s], ph ^ 1u, a.err, abort_flag)) { ok = false; return; }
-            const uint32_t st = sbase + s * L::stage_bytes;
-            dq_iq2_sub(cb[q], dsc, (st + roff) ^ cx, tabL, tabS);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&fullA[s]);
-            if (++s == kStages) { s = 0; ph ^= 1u; }
+            if (!tc_wait_warp(&emptyA[sa], pha ^ 1u, a.err, abort_flag)) { ok = false; return; }
+            tc_fence_after();
+            uint32_t o[16];
+            dq_iq2_sub(cb[q], dsc, tabL, tabS, o);
+            tmem_st16(tmem + tcol + sa * L::a_cols, o);
+            publish(true);
           }
         };
         load_blk(0, c0, e0);
@@ -465,14 +524,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           load_blk(b + 4, c1, e1);
           run_blk(b + 2, c2, e2);
         }
-      } else {  // TC_Q2K: thread = (row, quarter qt of the stage's 64 weights = one sub-block)
-        const int r = dt >> 2, qt = dt & 3;
+      } else {  // TC_Q2K: part = quarter of the stage's 64 weights = one 16-weight sub-block
+        const int qt = part;
         const size_t grow = static_cast<size_t>(pr.e) * a.rows_e + m0 + r;
         const int nblk = a.K / 256;
         const uint8_t* brow = a.c0 + grow * nblk * 80;
         const uint32_t* ddrow = a.dd + grow * nblk;
-        const uint32_t roff = ((r >> 3) * 1024 + (r & 7) * 128) | ((r & 7) << 4);
-        const uint32_t cx = static_cast<uint32_t>(qt) << 5;  // chunks 2qt, 2qt + 1
+        const uint32_t tcol = tlane + qt * 8;
         const uint32_t sshift = 8u * qt;
         // one 80-byte block (four stages) per step: the 16 scale bytes, the thread's four
         // q words (sub-blocks 4q + qt) and dd; loads run two blocks ahead as above
@@ -497,13 +555,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           const uint32_t qws[4] = {qw.x, qw.y, qw.z, qw.w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            if (!tc_wait_warp(&empty[s], ph ^ 1u, a.err, abort_flag)) { ok = false; return; }
-            const uint32_t st = sbase + s * L::stage_bytes;
-            dq_q2k_sub(qws[q], (scw[q] >> sshift) & 0xFFu, d, dmin, (st + roff) ^ cx, tabQ);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&fullA[s]);
-            if (++s == kStages) { s = 0; ph ^= 1u; }
+            if (!tc_wait_warp(&emptyA[sa], pha ^ 1u, a.err, abort_flag)) { ok = false; return; }
+            tc_fence_after();
+            uint32_t o[8];
+            dq_q2k_sub(qws[q], (scw[q] >> sshift) & 0xFFu, d, dmin, tabQ, o);
+            tmem_st8(tmem + tcol + sa * L::a_cols, o);
+            publish(true);
           }
         };
         load_blk(0, s0, w0, e0);
@@ -526,15 +583,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       const TcPair pr = tc_pair(a, u / a.mt);
       const int m0 = (u % a.mt) * kMT;
       if (pr.n == 0) continue;
-      const int buf = t & 1;
-      if (!tc_wait_warp(&accf[buf], (t >> 1) & 1, a.err, abort_flag)) break;
+      const int buf = t % kAccBufs;
+      // the tile's per-row exponents (lane n % 32 of word n / 32), loaded before the wait
+      int ex4[4] = {0, 0, 0, 0};
+      if (KIND == TC_IQ2_PAIR) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (32 * i + lane < pr.n) ex4[i] = __ldg(a.row_exp + pr.p0 + 32 * i + lane);
+      }
+      if (!tc_wait_warp(&accf[buf], (t / kAccBufs) & 1, a.err, abort_flag)) break;
       tc_fence_after();
-      const uint32_t tl = tmem + buf * 256 + (static_cast<uint32_t>(32 * warp) << 16);
+      const uint32_t tl = tmem + L::acc_base + buf * L::acc_stride + (static_cast<uint32_t>(32 * warp) << 16);
       const int row = m0 + r;
       for (int c0 = 0; c0 < pr.n; c0 += 16) {
         uint32_t g[16], v[16];
         tmem_ld16(tl + c0, g);
         if (PAIR) tmem_ld16(tl + 128 + c0, v);
+        const int exw = (c0 < 64) ? (c0 < 32 ? ex4[0] : ex4[1]) : (c0 < 96 ? ex4[2] : ex4[3]);
         tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -544,10 +609,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           if (KIND == TC_IQ2_PAIR) {
             // B row = x * 2^-e: g, u come back as exact fp32 rescalings; h leaves as
             // fp16(h * 2^(-2e-12)), the scale that keeps it inside the fp16 range
-            const int ex = a.row_exp[orow];
-            const float sc = ldexpf(a.oscale, ex);
-            const float h = silu_mul_tc(__uint_as_float(g[j]) * sc, __uint_as_float(v[j]) * sc);
-            reinterpret_cast<__half*>(a.out)[orow * a.ldo + row] = __float2half_rn(ldexpf(h, -2 * ex - 12));
+            const int ex = __shfl_sync(0xffffffffu, exw, (c0 & 31) + j);
+            const float gs = mul_pow2(__uint_as_float(g[j]) * a.oscale, ex);
+            const float us = mul_pow2(__uint_as_float(v[j]) * a.oscale, ex);
+            const float h = silu_mul_tc(gs, us);
+            reinterpret_cast<__half*>(a.out)[orow * a.ldo + row] = __float2half_rn(mul_pow2(h, -2 * ex - 12));
           } else if (KIND == TC_BF16_PAIR) {
             const float h = silu_mul_tc(__uint_as_float(g[j]), __uint_as_float(v[j]));
             const __nv_bfloat16 hi = __float2bfloat16_rn(h);
