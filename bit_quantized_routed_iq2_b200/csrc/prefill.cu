@@ -66,6 +66,7 @@ constexpr int kNT = 128;         // max tokens per tile (MMA N)
 constexpr int kKS = 64;          // K per stage: 128 bytes of fp16 per row
 constexpr int kTile = 128 * 128; // one 128-row x 128-byte operand tile
 constexpr int kTmemCols = 512;   // two accumulator buffers of (gate, up) x 128 columns
+constexpr int kCodeChunk = 128 * 16;  // code bytes of one stage: 128 rows x 16 bytes
 
 __device__ const Iq2Codebook d_codebook_tc = kCodebook;
 
@@ -109,7 +110,9 @@ struct TcArgs {
 // Memory plan per kernel kind.
 // Dequantising kinds: the fp16 weight tiles (A) go from registers into TMEM
 // (tcgen05.st) and the MMA reads A from there, so shared memory carries only
-// the token tiles (B, a TMA ring of its own) and the replicated lookup tables:
+// the TMA ring of token tiles (B) with each stage's code bytes beside them
+// (IQ2: 16 bytes per row of gate and of up; Q2K: the 16 q bytes of the stage
+// and the block's 16 scale bytes) and the replicated lookup tables:
 // IQ2 level selectors (8 bytes, 16 copies), IQ2 signs as fp16 +-1 pairs (16
 // bytes, 8 copies), Q2K selectors (4 bytes, 32 copies); every copy serves the
 // lanes of one load phase, so lookups are free of bank conflicts.
@@ -122,7 +125,8 @@ struct TcLayout {
   static constexpr bool dq = (KIND == TC_IQ2_PAIR || KIND == TC_Q2K);
   static constexpr bool pair = (KIND == TC_IQ2_PAIR || KIND == TC_BF16_PAIR);
   static constexpr int stages = dq ? 8 : (pair ? 4 : 6);                 // shared-memory ring
-  static constexpr size_t stage_bytes = (dq ? 1 : (pair ? 3 : 2)) * kTile;
+  // dequantising kinds: B tile + two 2 KB chunks of code bytes (128 rows x 16 bytes)
+  static constexpr size_t stage_bytes = dq ? kTile + 2 * kCodeChunk : (pair ? 3 : 2) * kTile;
   static constexpr size_t b_off = dq ? 0 : (pair ? 2 : 1) * kTile;      // B tile inside a stage
   static constexpr int a_stages = KIND == TC_IQ2_PAIR ? 4 : 8;           // TMEM A ring (dq kinds)
   static constexpr uint32_t a_cols = pair ? 64 : 32;                     // TMEM columns per A stage
@@ -174,6 +178,11 @@ __device__ __forceinline__ uint4 lds128s(uint32_t a) {
 __device__ __forceinline__ uint2 lds64s(uint32_t a) {
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds8s(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
 __device__ __forceinline__ uint32_t lds32s(uint32_t a) {
@@ -383,7 +392,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             tma_load_3d(st, &tm_a0, kx, pr.e * a.rows_e + m0, 0, &fullB[s]);
             if (PAIR) tma_load_3d(st + kTile, &tm_a1, kx, pr.e * a.rows_e + m0, 0, &fullB[s]);
           } else {
-            mbar_arrive_expect_tx(&fullB[s], kTile);
+            mbar_arrive_expect_tx(&fullB[s], L::stage_bytes);
+            const int wrow = pr.e * a.rows_e + m0;
+            if (KIND == TC_IQ2_PAIR) {  // 16 code bytes per row = 64 weights of gate and of up
+              tma_load_2d(st + kTile, &tm_a0, 16 * ks, wrow, &fullB[s]);
+              tma_load_2d(st + kTile + kCodeChunk, &tm_a1, 16 * ks, wrow, &fullB[s]);
+            } else {  // the stage's 16 q bytes and its block's 16 scale bytes
+              const int blk = 80 * (ks >> 2);
+              tma_load_2d(st + kTile, &tm_a0, blk + 16 + 16 * (ks & 3), wrow, &fullB[s]);
+              tma_load_2d(st + kTile + kCodeChunk, &tm_a0, blk, wrow, &fullB[s]);
+            }
           }
           tma_load_3d(st + L::b_off, &tm_b, kx, pr.p0, pl, &fullB[s]);
           ++issued;
@@ -463,118 +481,76 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
   } else if (DQ && warp >= kDqWarp0) {
     // sixteen warps; warp w may write TMEM lanes 32*(w%4)..+31, so the row is
     // 32*(w%4) + lane and the four warps of a lane quarter split each stage's
-    // weights of their rows; each thread turns one sub-block into fp16 per stage
+    // weights of their rows; each thread turns one sub-block into fp16 per stage,
+    // reading its code bytes from the stage the producer filled
     const int quarter = warp & 3, part = (warp - kDqWarp0) >> 2;  // part 0..3
     const int r = 32 * quarter + lane;
     const uint32_t tlane = static_cast<uint32_t>(32 * quarter) << 16;
-    int sa = 0;
-    uint32_t pha = 0;
-    // one stage: wait for the A slot, fill this thread's columns, publish
-    auto publish = [&](bool ok) {
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (ok && lane == 0) mbar_arrive(&fullA[sa]);
-      if (++sa == kAStages) { sa = 0; pha ^= 1u; }
+    int sa = 0, s = 0;
+    uint32_t pha = 0, ph = 0;
+    const int nblk = nks / 4;
+    // per-block scales of this row (IQ2 d, Q2K d | dmin << 16), loaded one block
+    // ahead along the sequence of this CTA's tiles (the next tile's first block
+    // is requested during the last block of the current one)
+    auto next_tile = [&](int uu) {
+      while (uu < nunits && tc_pair(a, uu / a.mt).n == 0) uu += gridDim.x;
+      return uu;
     };
-    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-      const TcPair pr = tc_pair(a, u / a.mt);
-      const int m0 = (u % a.mt) * kMT;
-      if (pr.n == 0) continue;
+    auto row_of = [&](int uu) -> size_t {
+      return static_cast<size_t>(tc_pair(a, uu / a.mt).e) * a.rows_e + (uu % a.mt) * kMT + r;
+    };
+    auto ldscale = [&](size_t grow, int b) -> uint32_t {
+      if (KIND == TC_IQ2_PAIR) return static_cast<uint32_t>(__ldg(((part >> 1) ? a.d1 : a.d0) + grow * nblk + b));
+      return __ldg(a.dd + grow * nblk + b);
+    };
+    int u = next_tile(blockIdx.x);
+    uint32_t dq1 = u < nunits ? ldscale(row_of(u), 0) : 0u;
+    while (u < nunits) {
+      const int un = next_tile(u + gridDim.x);
+      const size_t grow = row_of(u);
+      const size_t grow_n = un < nunits ? row_of(un) : 0;
       bool ok = true;
-      if (KIND == TC_IQ2_PAIR) {
-        // part = (matrix, sub-block half of the stage's 64 weights)
-        const int mat = part >> 1, hf = part & 1;
-        const size_t grow = static_cast<size_t>(pr.e) * a.rows_e + m0 + r;
-        const uint8_t* crow = (mat ? a.c1 : a.c0) + grow * (a.K / 4) + 8 * hf;
-        const uint16_t* drow = (mat ? a.d1 : a.d0) + grow * (a.K / 256);
-        const uint32_t tcol = tlane + mat * 32 + hf * 16;
-        // one 256-weight block (four stages, one record each) per step; loads run two
-        // blocks ahead into three rotating register buffers (no copies of in-flight loads)
-        const int nblk = nks / 4;
-        uint2 c0[4], c1[4], c2[4];
-        uint32_t e0 = 0, e1 = 0, e2 = 0;
-        auto load_blk = [&](int b, uint2 (&dst)[4], uint32_t& dv) {
-          if (b >= nblk) return;
-          const uint8_t* src = crow + b * 64;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) dst[q] = __ldg(reinterpret_cast<const uint2*>(src + 16 * q));
-          dv = __ldg(drow + b);
-        };
-        auto run_blk = [&](int b, const uint2 (&cb)[4], uint32_t dv) {
-          if (b >= nblk || !ok) return;
-          const float dsc = half_bits_to_float(static_cast<uint16_t>(dv)) * 128.0f;  // d / 8 * 2^10
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (!tc_wait_warp(&emptyA[sa], pha ^ 1u, a.err, abort_flag)) { ok = false; return; }
-            tc_fence_after();
-            uint32_t o[16];
-            dq_iq2_sub(cb[q], dsc, tabL, tabS, o);
-            tmem_st16(tmem + tcol + sa * L::a_cols, o);
-            publish(true);
-          }
-        };
-        load_blk(0, c0, e0);
-        load_blk(1, c1, e1);
-        for (int b = 0; b < nblk && ok; b += 3) {
-          load_blk(b + 2, c2, e2);
-          run_blk(b, c0, e0);
-          load_blk(b + 3, c0, e0);
-          run_blk(b + 1, c1, e1);
-          load_blk(b + 4, c1, e1);
-          run_blk(b + 2, c2, e2);
+      uint32_t dq0 = 0;
+      for (int ks = 0; ks < nks && ok; ++ks) {
+        if ((ks & 3) == 0) {
+          const int b = ks >> 2;
+          dq0 = dq1;
+          dq1 = b + 1 < nblk ? ldscale(grow, b + 1) : (un < nunits ? ldscale(grow_n, 0) : 0u);
         }
-      } else {  // TC_Q2K: part = quarter of the stage's 64 weights = one 16-weight sub-block
-        const int qt = part;
-        const size_t grow = static_cast<size_t>(pr.e) * a.rows_e + m0 + r;
-        const int nblk = a.K / 256;
-        const uint8_t* brow = a.c0 + grow * nblk * 80;
-        const uint32_t* ddrow = a.dd + grow * nblk;
-        const uint32_t tcol = tlane + qt * 8;
-        const uint32_t sshift = 8u * qt;
-        // one 80-byte block (four stages) per step: the 16 scale bytes, the thread's four
-        // q words (sub-blocks 4q + qt) and dd; loads run two blocks ahead as above
-        const int nbk = nks / 4;
-        uint4 s0, s1, s2, w0, w1, w2;
-        uint32_t e0 = 0, e1 = 0, e2 = 0;
-        auto load_blk = [&](int b, uint4& sc, uint4& qw, uint32_t& dv) {
-          if (b >= nbk) return;
-          const uint8_t* src = brow + b * 80;
-          sc = __ldg(reinterpret_cast<const uint4*>(src));
-          qw.x = __ldg(reinterpret_cast<const uint32_t*>(src + 16 + 4 * qt));
-          qw.y = __ldg(reinterpret_cast<const uint32_t*>(src + 32 + 4 * qt));
-          qw.z = __ldg(reinterpret_cast<const uint32_t*>(src + 48 + 4 * qt));
-          qw.w = __ldg(reinterpret_cast<const uint32_t*>(src + 64 + 4 * qt));
-          dv = __ldg(ddrow + b);
-        };
-        auto run_blk = [&](int b, const uint4& sc, const uint4& qw, uint32_t dv) {
-          if (b >= nbk || !ok) return;
-          const float d = half_bits_to_float(static_cast<uint16_t>(dv & 0xFFFFu));
-          const float dmin = half_bits_to_float(static_cast<uint16_t>(dv >> 16));
-          const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
-          const uint32_t qws[4] = {qw.x, qw.y, qw.z, qw.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (!tc_wait_warp(&emptyA[sa], pha ^ 1u, a.err, abort_flag)) { ok = false; return; }
-            tc_fence_after();
-            uint32_t o[8];
-            dq_q2k_sub(qws[q], (scw[q] >> sshift) & 0xFFu, d, dmin, tabQ, o);
-            tmem_st8(tmem + tcol + sa * L::a_cols, o);
-            publish(true);
-          }
-        };
-        load_blk(0, s0, w0, e0);
-        load_blk(1, s1, w1, e1);
-        for (int b = 0; b < nbk && ok; b += 3) {
-          load_blk(b + 2, s2, w2, e2);
-          run_blk(b, s0, w0, e0);
-          load_blk(b + 3, s0, w0, e0);
-          run_blk(b + 1, s1, w1, e1);
-          load_blk(b + 4, s1, w1, e1);
-          run_blk(b + 2, s2, w2, e2);
+        if (!tc_wait_warp(&emptyA[sa], pha ^ 1u, a.err, abort_flag) ||
+            !tc_wait_warp(&fullB[s], ph, a.err, abort_flag)) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        const uint32_t code = sbase + s * L::stage_bytes + kTile + r * 16;
+        if (KIND == TC_IQ2_PAIR) {
+          // part = (matrix, sub-block half of the stage's 64 weights)
+          const int mat = part >> 1, hf = part & 1;
+          const uint2 rec = lds64s(code + mat * kCodeChunk + 8 * hf);
+          const float dsc = half_bits_to_float(static_cast<uint16_t>(dq0)) * 128.0f;  // d / 8 * 2^10
+          uint32_t o[16];
+          dq_iq2_sub(rec, dsc, tabL, tabS, o);
+          tmem_st16(tmem + tlane + mat * 32 + hf * 16 + sa * L::a_cols, o);
+        } else {
+          // part = quarter of the stage's 64 weights = sub-block 4 * (ks % 4) + part of the block
+          const uint32_t w = lds32s(code + 4 * part);
+          const uint32_t scb = lds8s(code + kCodeChunk + 4 * (ks & 3) + part);
+          const float d = half_bits_to_float(static_cast<uint16_t>(dq0 & 0xFFFFu));
+          const float dmin = half_bits_to_float(static_cast<uint16_t>(dq0 >> 16));
+          uint32_t o[8];
+          dq_q2k_sub(w, scb, d, dmin, tabQ, o);
+          tmem_st8(tmem + tlane + part * 8 + sa * L::a_cols, o);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&fullA[sa]);
+        if (++sa == kAStages) { sa = 0; pha ^= 1u; }
+        if (++s == kStages) { s = 0; ph ^= 1u; }
       }
       if (!ok) break;
+      u = un;
     }
   } else if (warp < kEpiWarps) {
     const int r = 32 * warp + lane;  // TMEM lane = weight row of the tile
@@ -833,6 +809,20 @@ bool tc_map(CUtensorMap* m, const void* base, bool bf16, uint64_t K, uint64_t ro
   return r == CUDA_SUCCESS;
 }
 
+// 2-D map over a plane of code bytes: rows of `row_bytes`, boxes of 16 bytes x 128 rows.
+bool code_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows) {
+  auto fn = tc_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {16, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int KIND>
 int launch_tc(const CUtensorMap& mb, const CUtensorMap& ma0, const CUtensorMap& ma1, const TcArgs& a, int sms,
               cudaStream_t st) {
@@ -941,14 +931,17 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
   // routed gate/up: A = IQ2 gate/up rows (dequantised), B = expert-sorted fp16 activations
   {
     ProfScope ps(MOE_K_PREFILL_GATEUP, st);
-    if (!tc_map(&mb, pw.xp, false, sh.H, nA, 1)) return ERR_CUDA;
+    const uint64_t wrows = static_cast<uint64_t>(sh.E) * sh.I;
+    if (!tc_map(&mb, pw.xp, false, sh.H, nA, 1) || !code_map(&ma0, w.gate_codes, sh.H / 4, wrows) ||
+        !code_map(&ma1, w.up_codes, sh.H / 4, wrows))
+      return ERR_CUDA;
     TcArgs a{};
     a.n_experts = sh.E; a.b_rows = nA;
     a.rows_e = sh.I; a.K = sh.H; a.mt = sh.I / kMT; a.planes = 1;
     a.c0 = w.gate_codes; a.d0 = w.gate_d; a.c1 = w.up_codes; a.d1 = w.up_d;
     a.pairs = pw.pairs; a.npairs = pw.counts; a.out = pw.hh; a.ldo = sh.I; a.out_rows = nA;
     a.oscale = 1.0f / 1024.0f; a.err = err; a.row_exp = pw.aexp;
-    rc |= launch_tc<TC_IQ2_PAIR>(mb, mb, mb, a, sms, st);
+    rc |= launch_tc<TC_IQ2_PAIR>(mb, ma0, ma1, a, sms, st);
   }
   if (sh.Is > 0) {
     ProfScope ps(MOE_K_SHARED_GATEUP, st);
@@ -966,14 +959,16 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
   }
   {
     ProfScope ps(MOE_K_PREFILL_DOWN, st);
-    if (!tc_map(&mb, pw.hh, false, sh.I, nA, 1)) return ERR_CUDA;
+    if (!tc_map(&mb, pw.hh, false, sh.I, nA, 1) ||
+        !code_map(&ma0, w.down_codes, static_cast<uint64_t>(sh.I / 256) * 80, static_cast<uint64_t>(sh.E) * sh.H))
+      return ERR_CUDA;
     TcArgs a{};
     a.n_experts = sh.E; a.b_rows = nA;
     a.rows_e = sh.H; a.K = sh.I; a.mt = sh.H / kMT; a.planes = 1;
     a.c0 = w.down_codes; a.dd = w.down_dd;
     a.pairs = pw.pairs; a.npairs = pw.counts; a.out = pw.o; a.ldo = sh.H; a.out_rows = nA;
     a.oscale = 1.0f; a.err = err; a.row_exp = pw.aexp;
-    rc |= launch_tc<TC_Q2K>(mb, mb, mb, a, sms, st);
+    rc |= launch_tc<TC_Q2K>(mb, ma0, ma0, a, sms, st);
   }
   if (sh.Is > 0) {
     ProfScope ps(MOE_K_SHARED_DOWN, st);
