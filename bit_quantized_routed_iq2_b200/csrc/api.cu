@@ -179,6 +179,12 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights
   RouteWs w = carve(desc, T, ws);
   if (ws_bytes < w.bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the shared expert does not depend on routing: its gate/up starts first, on a side stream
+  const bool early = shared_early_ok(shape_of(desc), x_dtype, T);
+  if (early) {
+    const int rc0 = launch_shared_early(shape_of(desc), weights_of(weights), x, T, w.ffn, s);
+    if (rc0 != OK) return to_status(rc0);
+  }
   int rc = launch_route(weights->router_w, weights->router_bias, x, x_dtype, T, desc->hidden, desc->n_experts,
                         desc->top_k, w.logits, w.topk_idx, w.topk_w, w.offsets, w.perm, w.inv, w.active, w.status,
                         s);
@@ -187,7 +193,7 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights
   // the tensor-core router (many bf16 tokens) already cleared the status word
   const bool routed_clears = x_dtype == MOE_BF16 && router_tc_supported(T, desc->hidden, desc->n_experts);
   return to_status(launch_ffn(shape_of(desc), weights_of(weights), x, x_dtype, T, r, residual, y, w.ffn, w.status,
-                              !routed_clears, s));
+                              !routed_clears, s, early));
 }
 
 moe_status moe_debug_dequant_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, float* out,

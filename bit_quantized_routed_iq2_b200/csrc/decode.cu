@@ -13,6 +13,9 @@
 
 #include <algorithm>
 
+#include <map>
+#include <mutex>
+
 #include "decode.cuh"
 #include "kernels.cuh"
 #include "profile.cuh"
@@ -407,8 +410,54 @@ size_t fast_ffn_workspace_bytes(const LayerShape& s, int T) {
   return b;
 }
 
+// Side stream and fork/join events per (device, caller stream), created on first use.
+struct SideCtx {
+  cudaStream_t st = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+static SideCtx* side_ctx(cudaStream_t st) {
+  static std::mutex mu;
+  static std::map<std::pair<int, cudaStream_t>, SideCtx> table;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  SideCtx& c = table[{dev, st}];
+  if (!c.st) {
+    if (cudaStreamCreateWithFlags(&c.st, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming) != cudaSuccess) {
+      table.erase({dev, st});
+      return nullptr;
+    }
+  }
+  return &c;
+}
+
+bool shared_early_ok(const LayerShape& s, int x_dtype, int T) {
+  return x_dtype == 1 && s.Is > 0 && !use_prefill(s, T) && fast_path_supported(s) &&
+         shared_mma_supported(s.H, s.Is, T, 1, s.k);
+}
+
+int launch_shared_early(const LayerShape& s, const WeightPtrs& w, const void* x, int T, void* ws, cudaStream_t st) {
+  SideCtx* c = side_ctx(st);
+  if (!c) return ERR_CUDA;
+  const bool tma = tma_shape(s, T) && tma_path_supported(s, T);
+  const int KP = tma ? tma_gu_parts(s, T) : 1, DP = tma ? tma_dn_parts(s, T) : 1;
+  const FastWs fw = carve_fast(s, T, KP, DP, static_cast<char*>(ws));
+  if (cudaEventRecord(c->fork, st) != cudaSuccess || cudaStreamWaitEvent(c->st, c->fork, 0) != cudaSuccess)
+    return ERR_CUDA;
+  int rc;
+  {
+    ProfScope ps(MOE_K_SHARED_GATEUP, c->st);
+    rc = launch_shared_gateup_mma(s.H, s.Is, w.sh_gate, w.sh_up, static_cast<const uint16_t*>(x), 1, T, fw.hb, c->st);
+  }
+  if (cudaEventRecord(c->join, c->st) != cudaSuccess) return ERR_CUDA;
+  return rc;
+}
+
 int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
-                    const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st) {
+                    const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st,
+                    bool shared_early) {
   const size_t nA = static_cast<size_t>(T) * s.k;
   const bool tma = tma_shape(s, T) && tma_path_supported(s, T);
   const int KP = tma ? tma_gu_parts(s, T) : 1, DP = tma ? tma_dn_parts(s, T) : 1;
@@ -451,7 +500,9 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
     ProfScope ps(MOE_K_GATEUP, st);
     rc |= launch_gateup(ga, slots, sms, st);
   }
-  if (sh_mma) {
+  if (sh_mma && shared_early) {
+    // launched before routing on the side stream (launch_shared_early)
+  } else if (sh_mma) {
     ProfScope ps(MOE_K_SHARED_GATEUP, st);
     rc |= launch_shared_gateup_mma(s.H, s.Is, w.sh_gate, w.sh_up, xbp, xparts, T, fw.hb, st);
   } else if (s.Is > 0) {
@@ -488,6 +539,10 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
     rc |= launch_down(da, slots, T, sms, st);
   }
   if (sh_mma) {
+    if (shared_early) {
+      SideCtx* c = side_ctx(st);
+      if (!c || cudaStreamWaitEvent(st, c->join, 0) != cudaSuccess) return ERR_CUDA;
+    }
     ProfScope ps(MOE_K_COMBINE, st);
     rc |= launch_shared_down_combine_mma(s.H, s.Is, w.sh_down, fw.hb, T, s.k, r.topk_w, r.inv, obuf, DP, residual,
                                          y, st);

@@ -237,7 +237,7 @@ static size_t simple_ffn_workspace_bytes(const LayerShape& s, int T) {
 
 // Token counts above the decode GEMVs' range go through the tensor-core grouped
 // GEMM (prefill.cu) when the shape allows it.
-static bool use_prefill(const LayerShape& s, int T) { return T > kPrefillMinT && prefill_path_supported(s, T); }
+bool use_prefill(const LayerShape& s, int T) { return T > kPrefillMinT && prefill_path_supported(s, T); }
 
 size_t ffn_workspace_bytes(const LayerShape& s, int T) {
   size_t b = fast_path_supported(s) ? fast_ffn_workspace_bytes(s, T) : simple_ffn_workspace_bytes(s, T);
@@ -295,14 +295,16 @@ static int launch_ffn_simple(const LayerShape& s, const WeightPtrs& w, const voi
 }
 
 int launch_ffn(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
-               const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st) {
+               const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st,
+               bool shared_early) {
   if (use_prefill(s, T)) {
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     return launch_ffn_prefill(s, w, x, x_dtype, T, r, residual, y, ws, err, clear_status, sms > 0 ? sms : 148, st);
   }
-  if (fast_path_supported(s)) return launch_ffn_fast(s, w, x, x_dtype, T, r, residual, y, ws, err, clear_status, st);
+  if (fast_path_supported(s))
+    return launch_ffn_fast(s, w, x, x_dtype, T, r, residual, y, ws, err, clear_status, st, shared_early);
   return launch_ffn_simple(s, w, x, x_dtype, T, r, residual, y, ws, st);
 }
 

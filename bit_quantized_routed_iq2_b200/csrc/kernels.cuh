@@ -42,13 +42,17 @@ size_t ffn_workspace_bytes(const LayerShape& s, int T);
 // clear_status: the FFN's first kernel clears *err (false when an earlier
 // kernel of the same call already did).
 int launch_ffn(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
-               const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st);
+               const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st,
+               bool shared_early = false);
 
 // Tensor-core dequant-GEMV path (decode.cu): shapes with H % 256 == 0 and I % 256 == 0.
 bool fast_path_supported(const LayerShape& s);
+// true when launch_ffn takes the tensor-core grouped GEMM for T tokens
+bool use_prefill(const LayerShape& s, int T);
 size_t fast_ffn_workspace_bytes(const LayerShape& s, int T);
 int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
-                    const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st);
+                    const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st,
+                    bool shared_early = false);
 
 // TMA-fed GEMVs (gemv_tma.cu).
 bool tma_path_supported(const LayerShape& s, int T);
@@ -64,6 +68,11 @@ int launch_down_tma(const LayerShape& sh, const uint8_t* down_codes, const uint3
 // Shared expert on bf16 warp MMAs for up to 32 tokens (shared_mma.cu). xb holds
 // P bf16 parts of x as [P][T][H]; hb receives h as two parts [2][T][Is].
 bool shared_mma_supported(int H, int Is, int T, int x_parts, int k);
+// Shared expert ahead of routing: for bf16 activations on the decode path the
+// shared gate/up runs on a side stream forked from `st` before the router, and
+// the decode path's combine waits for it. Returns true when it was launched.
+bool shared_early_ok(const LayerShape& s, int x_dtype, int T);
+int launch_shared_early(const LayerShape& s, const WeightPtrs& w, const void* x, int T, void* ffn_ws, cudaStream_t st);
 int launch_shared_gateup_mma(int H, int Is, const uint16_t* wg, const uint16_t* wu, const uint16_t* xb, int P,
                              int T, uint16_t* hb, cudaStream_t st);
 int launch_shared_down_combine_mma(int H, int Is, const uint16_t* wd, const uint16_t* hb, int T, int k,
@@ -75,8 +84,10 @@ bool router_tc_supported(int T, int H, int E);
 int launch_router_tc(const uint16_t* Wr, const float* bias, const uint16_t* x, int T, int H, int E, float* logits,
                      int* err, int sms, cudaStream_t st);
 
-// Tensor-core grouped GEMM for many tokens (prefill.cu).
-constexpr int kPrefillMinT = 4;
+// Tensor-core grouped GEMM for many tokens (prefill.cu). Up to 16 tokens the
+// int8 dequant-GEMVs are faster (an 8-layer chain of 16-token steps measured
+// 9.3 ms on the GEMVs against 10.3 ms on the grouped GEMM).
+constexpr int kPrefillMinT = 16;
 bool prefill_path_supported(const LayerShape& s, int T);
 size_t prefill_workspace_bytes(const LayerShape& s, int T);
 int launch_ffn_prefill(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
