@@ -153,6 +153,15 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, int* err
   return false;
 }
 
+// The same with sleeps between polls, for waits whose latency matters little.
+__device__ __forceinline__ bool tc_wait_sleepy(uint64_t* bar, uint32_t parity, int* err, volatile int* abort_flag,
+                                               unsigned max_ns = 2048) {
+  if (*abort_flag) return false;
+  if (mbar_wait_bounded_sleepy(bar, parity, err, ERR_TIMEOUT, max_ns)) return true;
+  *abort_flag = 1;
+  return false;
+}
+
 // The same for all 32 lanes of a warp, with one outcome for the whole warp.
 __device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, int* err, volatile int* abort_flag) {
   const bool ok = tc_wait(bar, parity, err, abort_flag);
@@ -178,6 +187,11 @@ __device__ __forceinline__ uint4 lds128s(uint32_t a) {
 __device__ __forceinline__ uint2 lds64s(uint32_t a) {
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds16s(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
 __device__ __forceinline__ uint32_t lds8s(uint32_t a) {
@@ -243,7 +257,9 @@ __device__ __forceinline__ bool elect_one() {
   return p != 0;
 }
 
-__device__ __forceinline__ float silu_mul_tc(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+// silu(g) * u with the fast exponential and division: relative error near
+// 1e-6, far below the fp16 rounding that follows; g -> -inf gives -0.
+__device__ __forceinline__ float silu_mul_fast(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
 // x * 2^k as two exact power-of-2 multiplications (each factor a normal
 // float), the same value as ldexpf for results in the normal range; k is
@@ -308,7 +324,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       mbar_init(&emptyB[s], 1);
     }
     for (int s = 0; s < kAStages; ++s) {
-      mbar_init(&fullA[s], kDqWarps);
+      mbar_init(&fullA[s], kDqWarps / 2);  // one group of eight warps fills a stage
       mbar_init(&emptyA[s], 1);
     }
     for (int b = 0; b < kAccBufs; ++b) {
@@ -383,7 +399,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         const int m0 = (u % a.mt) * kMT;
         if (pr.n == 0) continue;
         for (int ks = 0; ks < nks; ++ks) {
-          if (!tc_wait(&emptyB[s], ph ^ 1u, a.err, abort_flag)) break;
+          if (!tc_wait_sleepy(&emptyB[s], ph ^ 1u, a.err, abort_flag, 256)) break;  // the ring runs ahead
           uint8_t* st = smem + s * L::stage_bytes;
           const int kx = (ks % ks_plane) * kKS, pl = ks / ks_plane;
           if (BF16) {
@@ -479,15 +495,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     __syncwarp();
     mbar_wait_bounded(drain, 0, nullptr, 0);
   } else if (DQ && warp >= kDqWarp0) {
-    // sixteen warps; warp w may write TMEM lanes 32*(w%4)..+31, so the row is
-    // 32*(w%4) + lane and the four warps of a lane quarter split each stage's
-    // weights of their rows; each thread turns one sub-block into fp16 per stage,
-    // reading its code bytes from the stage the producer filled
-    const int quarter = warp & 3, part = (warp - kDqWarp0) >> 2;  // part 0..3
+    // sixteen warps in two groups of eight: group g fills the stages ks = g (mod 2),
+    // so the two groups' latencies overlap. Warp w may write TMEM lanes
+    // 32*(w%4)..+31, so the row is 32*(w%4) + lane; the two warps of a lane
+    // quarter in a group split the stage's weights of their rows, each thread
+    // turning two sub-blocks of one row into fp16, from the code bytes the
+    // producer put beside the stage's token tile
+    const int grp = (warp - kDqWarp0) >> 3, part = ((warp - kDqWarp0) >> 2) & 1;
+    const int quarter = warp & 3;
     const int r = 32 * quarter + lane;
     const uint32_t tlane = static_cast<uint32_t>(32 * quarter) << 16;
-    int sa = 0, s = 0;
-    uint32_t pha = 0, ph = 0;
+    long long gs = grp;  // global stage index (over this CTA's tiles) of this group's next stage
     const int nblk = nks / 4;
     // per-block scales of this row (IQ2 d, Q2K d | dmin << 16), loaded one block
     // ahead along the sequence of this CTA's tiles (the next tile's first block
@@ -500,7 +518,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       return static_cast<size_t>(tc_pair(a, uu / a.mt).e) * a.rows_e + (uu % a.mt) * kMT + r;
     };
     auto ldscale = [&](size_t grow, int b) -> uint32_t {
-      if (KIND == TC_IQ2_PAIR) return static_cast<uint32_t>(__ldg(((part >> 1) ? a.d1 : a.d0) + grow * nblk + b));
+      if (KIND == TC_IQ2_PAIR) return static_cast<uint32_t>(__ldg((part ? a.d1 : a.d0) + grow * nblk + b));
       return __ldg(a.dd + grow * nblk + b);
     };
     int u = next_tile(blockIdx.x);
@@ -511,12 +529,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       const size_t grow_n = un < nunits ? row_of(un) : 0;
       bool ok = true;
       uint32_t dq0 = 0;
-      for (int ks = 0; ks < nks && ok; ++ks) {
-        if ((ks & 3) == 0) {
+      for (int ks = grp; ks < nks && ok; ks += 2, gs += 2) {  // nks is a multiple of 4
+        if ((ks & 3) == grp) {  // the group's first stage of a block
           const int b = ks >> 2;
           dq0 = dq1;
           dq1 = b + 1 < nblk ? ldscale(grow, b + 1) : (un < nunits ? ldscale(grow_n, 0) : 0u);
         }
+        const int sa = static_cast<int>(gs % kAStages), s = static_cast<int>(gs % kStages);
+        const uint32_t pha = static_cast<uint32_t>((gs / kAStages) & 1), ph = static_cast<uint32_t>((gs / kStages) & 1);
         if (!tc_wait_warp(&emptyA[sa], pha ^ 1u, a.err, abort_flag) ||
             !tc_wait_warp(&fullB[s], ph, a.err, abort_flag)) {
           ok = false;
@@ -525,29 +545,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         tc_fence_after();
         const uint32_t code = sbase + s * L::stage_bytes + kTile + r * 16;
         if (KIND == TC_IQ2_PAIR) {
-          // part = (matrix, sub-block half of the stage's 64 weights)
-          const int mat = part >> 1, hf = part & 1;
-          const uint2 rec = lds64s(code + mat * kCodeChunk + 8 * hf);
+          // part = matrix; the row's two 8-byte records of this stage (32 weights each)
+          const uint4 rec = lds128s(code + part * kCodeChunk);
           const float dsc = half_bits_to_float(static_cast<uint16_t>(dq0)) * 128.0f;  // d / 8 * 2^10
-          uint32_t o[16];
-          dq_iq2_sub(rec, dsc, tabL, tabS, o);
-          tmem_st16(tmem + tlane + mat * 32 + hf * 16 + sa * L::a_cols, o);
+          uint32_t o0[16], o1[16];
+          dq_iq2_sub(make_uint2(rec.x, rec.y), dsc, tabL, tabS, o0);
+          dq_iq2_sub(make_uint2(rec.z, rec.w), dsc, tabL, tabS, o1);
+          const uint32_t tc = tmem + tlane + part * 32 + sa * L::a_cols;
+          tmem_st16(tc, o0);
+          tmem_st16(tc + 16, o1);
         } else {
-          // part = quarter of the stage's 64 weights = sub-block 4 * (ks % 4) + part of the block
-          const uint32_t w = lds32s(code + 4 * part);
-          const uint32_t scb = lds8s(code + kCodeChunk + 4 * (ks & 3) + part);
+          // part = half of the stage's 64 weights = sub-blocks 4 * (ks % 4) + 2 * part, +1 of the block
+          const uint2 w = lds64s(code + 8 * part);
+          const uint32_t scb = lds16s(code + kCodeChunk + 4 * (ks & 3) + 2 * part);
           const float d = half_bits_to_float(static_cast<uint16_t>(dq0 & 0xFFFFu));
           const float dmin = half_bits_to_float(static_cast<uint16_t>(dq0 >> 16));
-          uint32_t o[8];
-          dq_q2k_sub(w, scb, d, dmin, tabQ, o);
-          tmem_st8(tmem + tlane + part * 8 + sa * L::a_cols, o);
+          uint32_t o0[8], o1[8];
+          dq_q2k_sub(w.x, scb & 0xFFu, d, dmin, tabQ, o0);
+          dq_q2k_sub(w.y, scb >> 8, d, dmin, tabQ, o1);
+          const uint32_t tc = tmem + tlane + part * 16 + sa * L::a_cols;
+          tmem_st8(tc, o0);
+          tmem_st8(tc + 8, o1);
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&fullA[sa]);
-        if (++sa == kAStages) { sa = 0; pha ^= 1u; }
-        if (++s == kStages) { s = 0; ph ^= 1u; }
       }
       if (!ok) break;
       u = un;
@@ -567,7 +590,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         for (int i = 0; i < 4; ++i)
           if (32 * i + lane < pr.n) ex4[i] = __ldg(a.row_exp + pr.p0 + 32 * i + lane);
       }
-      if (!tc_wait_warp(&accf[buf], (t / kAccBufs) & 1, a.err, abort_flag)) break;
+      // the epilogue waits out a whole tile of MMAs: it sleeps between polls
+      const bool got = tc_wait_sleepy(&accf[buf], (t / kAccBufs) & 1, a.err, abort_flag, kAccBufs > 1 ? 2048 : 256);
+      if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t tl = tmem + L::acc_base + buf * L::acc_stride + (static_cast<uint32_t>(32 * warp) << 16);
       const int row = m0 + r;
@@ -586,12 +611,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             // B row = x * 2^-e: g, u come back as exact fp32 rescalings; h leaves as
             // fp16(h * 2^(-2e-12)), the scale that keeps it inside the fp16 range
             const int ex = __shfl_sync(0xffffffffu, exw, (c0 & 31) + j);
-            const float gs = mul_pow2(__uint_as_float(g[j]) * a.oscale, ex);
-            const float us = mul_pow2(__uint_as_float(v[j]) * a.oscale, ex);
-            const float h = silu_mul_tc(gs, us);
-            reinterpret_cast<__half*>(a.out)[orow * a.ldo + row] = __float2half_rn(mul_pow2(h, -2 * ex - 12));
+            float gs = __uint_as_float(g[j]) * a.oscale, us = __uint_as_float(v[j]) * a.oscale;
+            float h;
+            if (ex >= -60 && ex <= 55) {  // both factors are normal floats: build them from exponent bits
+              const float up = __int_as_float((ex + 127) << 23), down = __int_as_float((127 - 12 - 2 * ex) << 23);
+              h = silu_mul_fast(gs * up, us * up) * down;
+            } else {
+              h = mul_pow2(silu_mul_fast(mul_pow2(gs, ex), mul_pow2(us, ex)), -2 * ex - 12);
+            }
+            reinterpret_cast<__half*>(a.out)[orow * a.ldo + row] = __float2half_rn(h);
           } else if (KIND == TC_BF16_PAIR) {
-            const float h = silu_mul_tc(__uint_as_float(g[j]), __uint_as_float(v[j]));
+            const float h = silu_mul_fast(__uint_as_float(g[j]), __uint_as_float(v[j]));
             const __nv_bfloat16 hi = __float2bfloat16_rn(h);
             const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
             reinterpret_cast<__nv_bfloat16*>(a.out)[orow * a.ldo + row] = hi;

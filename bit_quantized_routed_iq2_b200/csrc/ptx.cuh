@@ -45,31 +45,37 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-// try_wait with a suspend-time hint: a thread whose phase is not complete
-// sleeps until it completes or about `ns` nanoseconds pass, instead of
-// returning at once, so waiting warps take few issue slots from working ones.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity), "r"(ns)
-      : "memory");
-  return ok != 0;
-}
-
 // Wait for phase `parity` of `bar` for at most ~`limit_cycles` SM clock cycles
 // (4e9 is about two seconds at B200 clocks); on time-out record `code` in *err
-// (first writer wins) and return false. Never waits unbounded: each poll sleeps
-// at most 20 us, and the cycle counter is read once per 64 polls.
+// (first writer wins) and return false. Never spins unbounded. The cycle
+// counter is read once per 1024 polls so the poll loop stays tight.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err, int code,
                                                   long long limit_cycles = 4000000000ll) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    for (int i = 0; i < 1024; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (clock64() - t0 > limit_cycles) {
+      if (err) atomicCAS(err, 0, code);
+      return false;
+    }
+  }
+}
+
+// The same bound for waits whose latency matters little (a warp that waits for
+// a whole tile): between polls the warp sleeps, from 64 ns doubling up to
+// `max_ns`, so it takes almost no issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_wait_bounded_sleepy(uint64_t* bar, uint32_t parity, int* err, int code,
+                                                         unsigned max_ns = 2048, long long limit_cycles = 4000000000ll) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  unsigned ns = 64;
+  while (true) {
+    __nanosleep(ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    ns = ns < max_ns ? 2 * ns : max_ns;
     if (clock64() - t0 > limit_cycles) {
       if (err) atomicCAS(err, 0, code);
       return false;
