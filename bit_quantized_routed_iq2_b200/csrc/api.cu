@@ -187,13 +187,14 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights
   }
   int rc = launch_route(weights->router_w, weights->router_bias, x, x_dtype, T, desc->hidden, desc->n_experts,
                         desc->top_k, w.logits, w.topk_idx, w.topk_w, w.offsets, w.perm, w.inv, w.active, w.status,
-                        s);
+                        s, early);
   if (rc != OK) return to_status(rc);
   Routing r{w.topk_w, w.offsets, w.perm, w.inv, w.active};
-  // the tensor-core router (many bf16 tokens) already cleared the status word
+  // the status word is cleared by the first kernel on the caller's stream: the router when the shared
+  // expert and the digits run ahead on the side stream, the tensor-core router for many bf16 tokens
   const bool routed_clears = x_dtype == MOE_BF16 && router_tc_supported(T, desc->hidden, desc->n_experts);
   return to_status(launch_ffn(shape_of(desc), weights_of(weights), x, x_dtype, T, r, residual, y, w.ffn, w.status,
-                              !routed_clears, s, early));
+                              !routed_clears && !early, s, early));
 }
 
 moe_status moe_debug_dequant_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, float* out,

@@ -33,6 +33,8 @@ template <typename XT>
 __global__ void __launch_bounds__(256) x_digits_kernel(const XT* __restrict__ x, int T, int H,
                                                        int8_t* __restrict__ xd, float* __restrict__ xs,
                                                        uint16_t* __restrict__ xb, int* __restrict__ err_word) {
+  pdl_trigger();
+  pdl_wait();
   if (err_word && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *err_word = 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x;
@@ -351,6 +353,8 @@ int hsc_stride(int I) { return ((I / 256) + 3) & ~3; }
 __global__ void __launch_bounds__(256) hquant_kernel(int I, int KP, const float* __restrict__ gu,
                                                      int8_t* __restrict__ hd, float* __restrict__ hsc,
                                                      int32_t* __restrict__ hq, int hss) {
+  pdl_trigger();
+  pdl_wait();
   const int p = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int sb = warp; sb < I / 256; sb += 8) hquant_block_warp(I, KP, gu, p, sb, hd, hsc, hq, hss, lane);
@@ -413,7 +417,7 @@ size_t fast_ffn_workspace_bytes(const LayerShape& s, int T) {
 // Side stream and fork/join events per (device, caller stream), created on first use.
 struct SideCtx {
   cudaStream_t st = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaEvent_t fork = nullptr, digits = nullptr, join = nullptr;
 };
 static SideCtx* side_ctx(cudaStream_t st) {
   static std::mutex mu;
@@ -425,6 +429,7 @@ static SideCtx* side_ctx(cudaStream_t st) {
   if (!c.st) {
     if (cudaStreamCreateWithFlags(&c.st, cudaStreamNonBlocking) != cudaSuccess ||
         cudaEventCreateWithFlags(&c.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c.digits, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming) != cudaSuccess) {
       table.erase({dev, st});
       return nullptr;
@@ -446,6 +451,14 @@ int launch_shared_early(const LayerShape& s, const WeightPtrs& w, const void* x,
   const FastWs fw = carve_fast(s, T, KP, DP, static_cast<char*>(ws));
   if (cudaEventRecord(c->fork, st) != cudaSuccess || cudaStreamWaitEvent(c->st, c->fork, 0) != cudaSuccess)
     return ERR_CUDA;
+  // the activation digits of the routed GEMVs do not depend on routing either
+  {
+    ProfScope ps(MOE_K_PREP, c->st);
+    dim3 g(T, (s.H / 256 + 7) / 8);
+    x_digits_kernel<uint16_t><<<g, 256, 0, c->st>>>(static_cast<const uint16_t*>(x), T, s.H, fw.xd, fw.xs, nullptr,
+                                                    nullptr);
+  }
+  if (cudaEventRecord(c->digits, c->st) != cudaSuccess) return ERR_CUDA;
   int rc;
   {
     ProfScope ps(MOE_K_SHARED_GATEUP, c->st);
@@ -474,15 +487,18 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
   const int sms = num_sms();
   const int slots = static_cast<int>(std::min<size_t>(nA, static_cast<size_t>(s.E)));
   int rc = OK;
-  {
+  if (shared_early) {  // the digits come from the side stream (launch_shared_early)
+    SideCtx* c = side_ctx(st);
+    if (!c || cudaStreamWaitEvent(st, c->digits, 0) != cudaSuccess) return ERR_CUDA;
+  } else {
     ProfScope ps(MOE_K_PREP, st);
     dim3 g(T, (s.H / 256 + 7) / 8);
     if (x_dtype == 0)
-      x_digits_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(x), T, s.H, xd, xs, fw.xb,
-                                                clear_status ? err : nullptr);
+      launch_pdl(x_digits_kernel<float>, g, dim3(256), 0, st, static_cast<const float*>(x), T, s.H, xd, xs, fw.xb,
+                 clear_status ? err : nullptr);
     else
-      x_digits_kernel<uint16_t><<<g, 256, 0, st>>>(static_cast<const uint16_t*>(x), T, s.H, xd, xs, nullptr,
-                                                   clear_status ? err : nullptr);
+      launch_pdl(x_digits_kernel<uint16_t>, g, dim3(256), 0, st, static_cast<const uint16_t*>(x), T, s.H, xd, xs,
+                 static_cast<uint16_t*>(nullptr), clear_status ? err : nullptr);
   }
   // bf16 activations feed the shared expert's MMAs as one part, fp32 as two
   const int xparts = x_dtype == 0 ? 2 : 1;
@@ -525,7 +541,8 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
   }
   {
     ProfScope ps(MOE_K_HQUANT, st);
-    hquant_kernel<<<static_cast<unsigned>(nA), 256, 0, st>>>(s.I, KP, gu, hd, hsc, hq, hsc_stride(s.I));
+    launch_pdl(hquant_kernel, dim3(static_cast<unsigned>(nA)), dim3(256), 0, st, s.I, KP, static_cast<const float*>(gu),
+               hd, hsc, hq, hsc_stride(s.I));
   }
   if (tma) {
     ProfScope ps(MOE_K_DOWN, st);

@@ -470,6 +470,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
                                                                   const __grid_constant__ CUtensorMap tm_up,
                                                                   GuTmaArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
+  pdl_trigger();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H, I = a.I, T = a.T, S = a.S, NB = a.NB;
   const int nA = T * a.k;
@@ -503,6 +504,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
         (i & 32) == 0 ? d_sel_tables2.level[ent] : (ent < 128 ? d_sel_tables2.sign[ent] : 0u);
   }
   for (int i = tid; i < kZeroBytes / 16; i += kThreadsT) reinterpret_cast<uint4*>(zero)[i] = make_uint4(0, 0, 0, 0);
+  pdl_wait();  // routing and activations come from the kernels before this one
   load_meta(ms, a.offsets, a.active, a.perm, a.E, nA, a.k, tid, kThreadsT);
   if (XS) {
     stage_rows(xsm, a.xd, T * 2, H, tid, kThreadsT);
@@ -874,6 +876,7 @@ template <int MAXQ, bool HS>
 __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_constant__ CUtensorMap tm_down,
                                                                 DnTmaArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
+  pdl_trigger();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H, I = a.I, S = a.S, NB = a.NB;
   const int nA = a.T * a.k;
@@ -899,6 +902,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
     fence_barrier_init();
   }
   for (int i = tid; i < kZeroBytes / 16; i += kThreadsT) reinterpret_cast<uint4*>(zero)[i] = make_uint4(0, 0, 0, 0);
+  pdl_wait();  // routing and h come from the kernels before this one
   load_meta(ms, a.offsets, a.active, nullptr, a.E, nA, a.k, tid, kThreadsT);
   if (HS) {
     stage_rows(hd_s, a.hd, nA * 2, I, tid, kThreadsT);
@@ -1029,13 +1033,13 @@ template <typename K>
 void launch_k(K kern, int grid, size_t smem, cudaStream_t st, const CUtensorMap& m0, const CUtensorMap& m1,
               const GuTmaArgs& a) {
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  kern<<<grid, kThreadsT, smem, st>>>(m0, m1, a);
+  launch_pdl(kern, dim3(grid), dim3(kThreadsT), smem, st, m0, m1, a);
 }
 
 template <typename K>
 void launch_k(K kern, int grid, size_t smem, cudaStream_t st, const CUtensorMap& m0, const DnTmaArgs& a) {
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  kern<<<grid, kThreadsT, smem, st>>>(m0, a);
+  launch_pdl(kern, dim3(grid), dim3(kThreadsT), smem, st, m0, a);
 }
 
 }  // namespace

@@ -34,7 +34,8 @@ struct Routing {
 
 int launch_route(const uint16_t* Wr, const float* bias, const void* x, int x_dtype, int T, int H, int E, int k,
                  float* logits, int32_t* topk_idx, float* topk_w, int32_t* offsets, int32_t* perm, int32_t* inv,
-                 int32_t* active, int* err, cudaStream_t st);
+                 int32_t* active, int* err, cudaStream_t st,
+                 bool clear_status = false);
 int launch_active_from_offsets(const int32_t* offsets, int E, int32_t* active, cudaStream_t st);
 
 // Workspace needed by the FFN stage for T tokens (bytes) and the launcher.

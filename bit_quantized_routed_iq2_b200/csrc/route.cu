@@ -10,6 +10,7 @@
 // to the lower index), weights = softmax over the chosen k.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "ptx.cuh"
 #include "profile.cuh"
 
 namespace moe {
@@ -40,13 +41,14 @@ template <typename XT, int TT>
 __global__ void __launch_bounds__(128) router_logits_small_kernel(const uint16_t* __restrict__ Wr,
                                                                   const float* __restrict__ bias,
                                                                   const XT* __restrict__ x, int T, int H, int E,
-                                                                  float* __restrict__ logits) {
+                                                                  float* __restrict__ logits, int* clear_word) {
   constexpr int MAXJ = 16;  // H <= 16 * 1024
   __shared__ float part[4][TT];
   const int e = blockIdx.y;
   const int t0 = blockIdx.x * TT;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nj = H / 1024 + ((H % 1024) ? 1 : 0);
+  pdl_trigger();
   uint4 wv[MAXJ];
 #pragma unroll
   for (int j = 0; j < MAXJ; ++j) {
@@ -54,6 +56,9 @@ __global__ void __launch_bounds__(128) router_logits_small_kernel(const uint16_t
     wv[j] = (j < nj && c < H) ? *reinterpret_cast<const uint4*>(Wr + static_cast<size_t>(e) * H + c)
                               : make_uint4(0u, 0u, 0u, 0u);
   }
+  // the router weights are constants; x and the logits belong to the step
+  pdl_wait();
+  if (clear_word && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *clear_word = 0;  // first kernel of a call
   float acc[TT];
 #pragma unroll
   for (int t = 0; t < TT; ++t) acc[t] = 0.f;
@@ -344,6 +349,8 @@ __global__ void __launch_bounds__(1024) topk_permute_small_kernel(const float* _
   __shared__ int total;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int n = T * k;
+  pdl_trigger();
+  pdl_wait();
   if (tid < E) cnt[tid] = 0;
   if (warp < T)
     topk_warp<EPL>(logits + static_cast<size_t>(warp) * E, E, k, topk_idx + static_cast<size_t>(warp) * k,
@@ -372,6 +379,56 @@ __global__ void __launch_bounds__(1024) topk_permute_small_kernel(const float* _
   }
 }
 
+// Decode routing for at most 32 assignments (T*k <= 32, E <= 32*EPL) in one
+// warp: the top-k of each token in turn, then (lane j = assignment j) the
+// offsets as counts of smaller expert indices, the stable rank among equal
+// experts by match, and the active list by ballot prefix sums. Same outputs
+// as topk_permute_small_kernel, without block barriers or shared atomics.
+template <int EPL>
+__global__ void __launch_bounds__(32) topk_permute_warp_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                               int32_t* __restrict__ topk_idx,
+                                                               float* __restrict__ topk_w,
+                                                               int32_t* __restrict__ offsets,
+                                                               int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                               int32_t* __restrict__ active) {
+  __shared__ int idx_s[32];
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x;
+  const int n = T * k;
+  for (int t = 0; t < T; ++t)
+    topk_warp<EPL>(logits + static_cast<size_t>(t) * E, E, k, topk_idx + static_cast<size_t>(t) * k,
+                   topk_w + static_cast<size_t>(t) * k, idx_s + t * k);
+  __syncwarp();
+  const int e = lane < n ? idx_s[lane] : 0x7fffffff;  // above every expert index
+  // assignment j: position = (assignments with a smaller expert) + (earlier ones with the same expert)
+  int below = 0;
+  for (int j = 0; j < n; ++j) below += __shfl_sync(0xffffffffu, e, j) < e ? 1 : 0;
+  const unsigned same = __match_any_sync(0xffffffffu, e);
+  const int p = below + __popc(same & ((1u << lane) - 1u));
+  if (lane < n) {
+    perm[p] = lane;
+    inv[lane] = p;
+  }
+  // offsets[x] for x = 0..E and the ascending list of experts with at least one assignment
+  int nact = 0;
+  for (int base = 0; base <= E; base += 32) {
+    const int x = base + lane;
+    int lt = 0, eq = 0;
+    for (int j = 0; j < n; ++j) {
+      const int ej = __shfl_sync(0xffffffffu, e, j);
+      lt += ej < x ? 1 : 0;
+      eq += ej == x ? 1 : 0;
+    }
+    if (x <= E) offsets[x] = x == E ? n : lt;
+    const bool has = x < E && eq > 0;
+    const unsigned m = __ballot_sync(0xffffffffu, has);
+    if (has) active[nact + __popc(m & ((1u << lane) - 1u))] = x;
+    nact += __popc(m);
+  }
+  if (lane == 0) active[E] = nact;
+}
+
 // Active-expert list from caller-provided offsets (used by moe_expert_ffn).
 __global__ void __launch_bounds__(1024) active_from_offsets_kernel(const int32_t* __restrict__ offsets, int E,
                                                                    int32_t* __restrict__ active) {
@@ -392,7 +449,7 @@ static void set_smem(K kernel, size_t bytes) {
 
 int launch_route(const uint16_t* Wr, const float* bias, const void* x, int x_dtype, int T, int H, int E, int k,
                  float* logits, int32_t* topk_idx, float* topk_w, int32_t* offsets, int32_t* perm, int32_t* inv,
-                 int32_t* active, int* err, cudaStream_t st) {
+                 int32_t* active, int* err, cudaStream_t st, bool clear_status) {
   {
     ProfScope ps(MOE_K_ROUTER_LOGITS, st);
     if (x_dtype == 1 && router_tc_supported(T, H, E)) {
@@ -406,11 +463,11 @@ int launch_route(const uint16_t* Wr, const float* bias, const void* x, int x_dty
       constexpr int TT = 4;
       dim3 g((T + TT - 1) / TT, E);
       if (x_dtype == 0)
-        router_logits_small_kernel<float, TT><<<g, 128, 0, st>>>(Wr, bias, static_cast<const float*>(x), T, H, E,
-                                                                 logits);
+        launch_pdl(router_logits_small_kernel<float, TT>, g, dim3(128), 0, st, Wr, bias,
+                   static_cast<const float*>(x), T, H, E, logits, clear_status ? err : nullptr);
       else
-        router_logits_small_kernel<uint16_t, TT><<<g, 128, 0, st>>>(Wr, bias, static_cast<const uint16_t*>(x), T, H,
-                                                                    E, logits);
+        launch_pdl(router_logits_small_kernel<uint16_t, TT>, g, dim3(128), 0, st, Wr, bias,
+                   static_cast<const uint16_t*>(x), T, H, E, logits, clear_status ? err : nullptr);
     } else {
       constexpr int TT = 8;
       dim3 g((T + TT - 1) / TT, (E + 7) / 8);
@@ -422,13 +479,18 @@ int launch_route(const uint16_t* Wr, const float* bias, const void* x, int x_dty
     }
   }
   const size_t psmem = 32 * E * sizeof(uint16_t) + 3 * E * sizeof(int);
-  if (T * k <= 1024 && T <= 32 && E <= 1024) {
+  if (T * k <= 32 && E <= 256) {
+    ProfScope ps(MOE_K_PERMUTE, st);
+    launch_pdl(topk_permute_warp_kernel<8>, dim3(1), dim3(32), 0, st, logits, T, E, k, topk_idx, topk_w, offsets,
+               perm, inv, active);
+  } else if (T * k <= 1024 && T <= 32 && E <= 1024) {
     ProfScope ps(MOE_K_PERMUTE, st);
     if (E <= 256)
-      topk_permute_small_kernel<8><<<1, 1024, 0, st>>>(logits, T, E, k, topk_idx, topk_w, offsets, perm, inv, active);
+      launch_pdl(topk_permute_small_kernel<8>, dim3(1), dim3(1024), 0, st, logits, T, E, k, topk_idx, topk_w,
+                 offsets, perm, inv, active);
     else
-      topk_permute_small_kernel<32><<<1, 1024, 0, st>>>(logits, T, E, k, topk_idx, topk_w, offsets, perm, inv,
-                                                        active);
+      launch_pdl(topk_permute_small_kernel<32>, dim3(1), dim3(1024), 0, st, logits, T, E, k, topk_idx, topk_w,
+                 offsets, perm, inv, active);
   } else if (T * k <= 1024 && T <= 32) {
     ProfScope ps(MOE_K_PERMUTE, st);
     const size_t sm = 1024 * sizeof(int32_t) + psmem;

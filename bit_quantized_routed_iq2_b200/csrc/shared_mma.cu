@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace moe {
 namespace {
@@ -170,6 +171,8 @@ __global__ void __launch_bounds__(512) shared_down_combine_mma_kernel(
     const float* residual, float* y) {
   __shared__ __align__(16) float red[ks_max<NG>() * NG * 8 * kRows];
   extern __shared__ float osum[];  // [T*k][kRows]
+  pdl_trigger();
+  pdl_wait();  // h, the routed partials and the routing come from the kernels before this one
   const int warp = threadIdx.x >> 5;
   const int r0 = blockIdx.x * kRows;
   // the assignment rows of this thread's first gather item, loaded before the weight stream
@@ -244,20 +247,20 @@ int launch_shared_down_combine_mma(int H, int Is, const uint16_t* wd, const uint
   const size_t dyn = static_cast<size_t>(kRows) * T * k * sizeof(float);
   switch (ng) {
     case 1:
-      shared_down_combine_mma_kernel<1><<<grid, block, dyn, st>>>(H, Is, wd, hb, T, ks, k, topk_w, inv, obuf, DP,
-                                                                residual, y);
+      launch_pdl(shared_down_combine_mma_kernel<1>, grid, block, dyn, st, H, Is, wd, hb, T, ks, k, topk_w, inv, obuf,
+                 DP, residual, y);
       break;
     case 2:
-      shared_down_combine_mma_kernel<2><<<grid, block, dyn, st>>>(H, Is, wd, hb, T, ks, k, topk_w, inv, obuf, DP,
-                                                                residual, y);
+      launch_pdl(shared_down_combine_mma_kernel<2>, grid, block, dyn, st, H, Is, wd, hb, T, ks, k, topk_w, inv, obuf,
+                 DP, residual, y);
       break;
     case 4:
-      shared_down_combine_mma_kernel<4><<<grid, block, dyn, st>>>(H, Is, wd, hb, T, ks, k, topk_w, inv, obuf, DP,
-                                                                residual, y);
+      launch_pdl(shared_down_combine_mma_kernel<4>, grid, block, dyn, st, H, Is, wd, hb, T, ks, k, topk_w, inv, obuf,
+                 DP, residual, y);
       break;
     case 8:
-      shared_down_combine_mma_kernel<8><<<grid, block, dyn, st>>>(H, Is, wd, hb, T, ks, k, topk_w, inv, obuf, DP,
-                                                                residual, y);
+      launch_pdl(shared_down_combine_mma_kernel<8>, grid, block, dyn, st, H, Is, wd, hb, T, ks, k, topk_w, inv, obuf,
+                 DP, residual, y);
       break;
     default: return ERR_SHAPE;
   }
