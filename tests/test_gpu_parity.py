@@ -170,6 +170,9 @@ SMALL_CASES = {
     "tc_t64_f32": _small(H=1024, I=512, E=8, k=2, Is=256, T=64, x_dtype="f32", seed=0x5A1C),
     "tc_t200_zipf": _small(H=768, I=512, E=16, k=4, Is=0, T=200, zipf=True, seed=0x5A1D),
     "tc_t300_many_tiles": _small(H=1280, I=768, E=2, k=1, Is=384, T=300, seed=0x5A1E),
+    # routing in one warp up to 32 assignments (here exactly 32), the block kernel above (here 40)
+    "route_n32": _small(H=512, I=256, E=64, k=8, Is=64, T=4, seed=0x5A23),
+    "route_n40": _small(H=512, I=256, E=64, k=8, Is=64, T=5, seed=0x5A24),
     # activations far from unit scale: the fp16 operands of the tensor-core path carry a
     # power-of-2 exponent per token, so neither overflow (g * u beyond 65504) nor underflow
     "tc_t40_large_x": _small(H=512, I=256, E=8, k=2, Is=128, T=40, x_std=300.0, seed=0x5A21),
