@@ -66,7 +66,7 @@ constexpr int kNT = 128;         // max tokens per tile (MMA N)
 constexpr int kKS = 64;          // K per stage: 128 bytes of fp16 per row
 constexpr int kTile = 128 * 128; // one 128-row x 128-byte operand tile
 constexpr int kTmemCols = 512;   // two accumulator buffers of (gate, up) x 128 columns
-constexpr int kCodeChunk = 128 * 16;  // code bytes of one stage: 128 rows x 16 bytes
+constexpr int kCStages = 3;  // code-block ring of the dequantising kinds (one entry per 256-weight block)
 
 __device__ const Iq2Codebook d_codebook_tc = kCodebook;
 
@@ -110,9 +110,9 @@ struct TcArgs {
 // Memory plan per kernel kind.
 // Dequantising kinds: the fp16 weight tiles (A) go from registers into TMEM
 // (tcgen05.st) and the MMA reads A from there, so shared memory carries only
-// the TMA ring of token tiles (B) with each stage's code bytes beside them
-// (IQ2: 16 bytes per row of gate and of up; Q2K: the 16 q bytes of the stage
-// and the block's 16 scale bytes) and the replicated lookup tables:
+// the TMA ring of token tiles (B), a ring of code blocks (the code bytes of one
+// 256-weight block of the tile's rows, one TMA box per matrix and block) and
+// the replicated lookup tables:
 // IQ2 level selectors (8 bytes, 16 copies), IQ2 signs as fp16 +-1 pairs (16
 // bytes, 8 copies), Q2K selectors (4 bytes, 32 copies); every copy serves the
 // lanes of one load phase, so lookups are free of bank conflicts.
@@ -125,15 +125,18 @@ struct TcLayout {
   static constexpr bool dq = (KIND == TC_IQ2_PAIR || KIND == TC_Q2K);
   static constexpr bool pair = (KIND == TC_IQ2_PAIR || KIND == TC_BF16_PAIR);
   static constexpr int stages = dq ? 8 : (pair ? 4 : 6);                 // shared-memory ring
-  // dequantising kinds: B tile + two 2 KB chunks of code bytes (128 rows x 16 bytes)
-  static constexpr size_t stage_bytes = dq ? kTile + 2 * kCodeChunk : (pair ? 3 : 2) * kTile;
+  static constexpr size_t stage_bytes = dq ? kTile : (pair ? 3 : 2) * kTile;
+  // code bytes of one 256-weight block for the tile's 128 rows: IQ2 64 bytes per row of gate and of up,
+  // Q2K the whole 80-byte block
+  static constexpr size_t code_bytes = KIND == TC_IQ2_PAIR ? 2 * 128 * 64 : (KIND == TC_Q2K ? 128 * 80 : 0);
+  static constexpr size_t code_off = stages * stage_bytes;
   static constexpr size_t b_off = dq ? 0 : (pair ? 2 : 1) * kTile;      // B tile inside a stage
   static constexpr int a_stages = KIND == TC_IQ2_PAIR ? 4 : 8;           // TMEM A ring (dq kinds)
   static constexpr uint32_t a_cols = pair ? 64 : 32;                     // TMEM columns per A stage
   static constexpr int acc_bufs = KIND == TC_IQ2_PAIR ? 1 : 2;
   static constexpr uint32_t acc_base = dq ? 256 : 0;
   static constexpr uint32_t acc_stride = KIND == TC_Q2K ? 128 : 256;    // columns per accumulator buffer
-  static constexpr size_t tabs = stages * stage_bytes;
+  static constexpr size_t tabs = code_off + (dq ? kCStages * code_bytes : 0);
   static constexpr size_t tab_bytes =
       KIND == TC_IQ2_PAIR ? (256 * 128 + 128 * 128) : (KIND == TC_Q2K ? 256 * 128 : 0);
   static constexpr size_t bars = tabs + tab_bytes;
@@ -306,7 +309,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
   uint64_t* emptyB = fullB + kStages;
   uint64_t* fullA = emptyB + kStages;  // [kAStages] TMEM A ring (dequantising kinds)
   uint64_t* emptyA = fullA + kAStages;
-  uint64_t* accf = emptyA + kAStages;  // [kAccBufs]
+  uint64_t* fullC = emptyA + kAStages;  // [kCStages] code-block ring (dequantising kinds)
+  uint64_t* emptyC = fullC + kCStages;
+  uint64_t* accf = emptyC + kCStages;  // [kAccBufs]
   uint64_t* acce = accf + kAccBufs;    // [kAccBufs]
   uint64_t* drain = acce + kAccBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -326,6 +331,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     for (int s = 0; s < kAStages; ++s) {
       mbar_init(&fullA[s], kDqWarps / 2);  // one group of eight warps fills a stage
       mbar_init(&emptyA[s], 1);
+    }
+    for (int c = 0; c < kCStages; ++c) {
+      mbar_init(&fullC[c], 1);
+      mbar_init(&emptyC[c], kDqWarps);  // every dequantising warp reads every block
     }
     for (int b = 0; b < kAccBufs; ++b) {
       mbar_init(&accf[b], 1);
@@ -393,12 +402,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       prefetch_tmap(&tm_b);
       int s = 0;
       uint32_t ph = 0;
-      int issued = 0;
+      int issued = 0, c = 0, issued_c = 0;
+      uint32_t pc = 0;
       for (int u = blockIdx.x; u < nunits && !*abort_flag; u += gridDim.x) {
         const TcPair pr = tc_pair(a, u / a.mt);
         const int m0 = (u % a.mt) * kMT;
         if (pr.n == 0) continue;
         for (int ks = 0; ks < nks; ++ks) {
+          if (DQ && (ks & 3) == 0) {  // a new 256-weight block: its code bytes for all four stages
+            if (!tc_wait_sleepy(&emptyC[c], pc ^ 1u, a.err, abort_flag, 256)) break;
+            uint8_t* ce = smem + L::code_off + c * L::code_bytes;
+            const int wrow = pr.e * a.rows_e + m0;
+            mbar_arrive_expect_tx(&fullC[c], L::code_bytes);
+            if (KIND == TC_IQ2_PAIR) {
+              tma_load_2d(ce, &tm_a0, 64 * (ks >> 2), wrow, &fullC[c]);
+              tma_load_2d(ce + 128 * 64, &tm_a1, 64 * (ks >> 2), wrow, &fullC[c]);
+            } else {
+              tma_load_2d(ce, &tm_a0, 80 * (ks >> 2), wrow, &fullC[c]);
+            }
+            ++issued_c;
+            if (++c == kCStages) { c = 0; pc ^= 1u; }
+          }
           if (!tc_wait_sleepy(&emptyB[s], ph ^ 1u, a.err, abort_flag, 256)) break;  // the ring runs ahead
           uint8_t* st = smem + s * L::stage_bytes;
           const int kx = (ks % ks_plane) * kKS, pl = ks / ks_plane;
@@ -409,15 +433,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             if (PAIR) tma_load_3d(st + kTile, &tm_a1, kx, pr.e * a.rows_e + m0, 0, &fullB[s]);
           } else {
             mbar_arrive_expect_tx(&fullB[s], L::stage_bytes);
-            const int wrow = pr.e * a.rows_e + m0;
-            if (KIND == TC_IQ2_PAIR) {  // 16 code bytes per row = 64 weights of gate and of up
-              tma_load_2d(st + kTile, &tm_a0, 16 * ks, wrow, &fullB[s]);
-              tma_load_2d(st + kTile + kCodeChunk, &tm_a1, 16 * ks, wrow, &fullB[s]);
-            } else {  // the stage's 16 q bytes and its block's 16 scale bytes
-              const int blk = 80 * (ks >> 2);
-              tma_load_2d(st + kTile, &tm_a0, blk + 16 + 16 * (ks & 3), wrow, &fullB[s]);
-              tma_load_2d(st + kTile + kCodeChunk, &tm_a0, blk, wrow, &fullB[s]);
-            }
           }
           tma_load_3d(st + L::b_off, &tm_b, kx, pr.p0, pl, &fullB[s]);
           ++issued;
@@ -428,6 +443,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         for (int i = 0; i < kStages && i < issued; ++i) {
           if (--s < 0) { s = kStages - 1; ph ^= 1u; }
           mbar_wait_bounded(&fullB[s], ph, nullptr, 0);
+        }
+        for (int i = 0; i < kCStages && i < issued_c; ++i) {
+          if (--c < 0) { c = kCStages - 1; pc ^= 1u; }
+          mbar_wait_bounded(&fullC[c], pc, nullptr, 0);
         }
       }
     }
@@ -499,13 +518,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     // so the two groups' latencies overlap. Warp w may write TMEM lanes
     // 32*(w%4)..+31, so the row is 32*(w%4) + lane; the two warps of a lane
     // quarter in a group split the stage's weights of their rows, each thread
-    // turning two sub-blocks of one row into fp16, from the code bytes the
-    // producer put beside the stage's token tile
+    // turning two sub-blocks of one row into fp16, from the code-block ring the
+    // producer fills (one entry per 256-weight block, released by all sixteen warps)
     const int grp = (warp - kDqWarp0) >> 3, part = ((warp - kDqWarp0) >> 2) & 1;
     const int quarter = warp & 3;
     const int r = 32 * quarter + lane;
     const uint32_t tlane = static_cast<uint32_t>(32 * quarter) << 16;
     long long gs = grp;  // global stage index (over this CTA's tiles) of this group's next stage
+    int cb = 0;          // code-block ring position and phase
+    uint32_t pcb = 0;
     const int nblk = nks / 4;
     // per-block scales of this row (IQ2 d, Q2K d | dmin << 16), loaded one block
     // ahead along the sequence of this CTA's tiles (the next tile's first block
@@ -530,23 +551,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       bool ok = true;
       uint32_t dq0 = 0;
       for (int ks = grp; ks < nks && ok; ks += 2, gs += 2) {  // nks is a multiple of 4
+        const int q = ks & 3;
+        if (q == grp && !tc_wait_warp(&fullC[cb], pcb, a.err, abort_flag)) {  // the block's code bytes
+          ok = false;
+          break;
+        }
         if ((ks & 3) == grp) {  // the group's first stage of a block
           const int b = ks >> 2;
           dq0 = dq1;
           dq1 = b + 1 < nblk ? ldscale(grow, b + 1) : (un < nunits ? ldscale(grow_n, 0) : 0u);
         }
-        const int sa = static_cast<int>(gs % kAStages), s = static_cast<int>(gs % kStages);
-        const uint32_t pha = static_cast<uint32_t>((gs / kAStages) & 1), ph = static_cast<uint32_t>((gs / kStages) & 1);
-        if (!tc_wait_warp(&emptyA[sa], pha ^ 1u, a.err, abort_flag) ||
-            !tc_wait_warp(&fullB[s], ph, a.err, abort_flag)) {
+        const int sa = static_cast<int>(gs % kAStages);
+        const uint32_t pha = static_cast<uint32_t>((gs / kAStages) & 1);
+        if (!tc_wait_warp(&emptyA[sa], pha ^ 1u, a.err, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t code = sbase + s * L::stage_bytes + kTile + r * 16;
+        const uint32_t ce = sbase + L::code_off + cb * L::code_bytes;
         if (KIND == TC_IQ2_PAIR) {
           // part = matrix; the row's two 8-byte records of this stage (32 weights each)
-          const uint4 rec = lds128s(code + part * kCodeChunk);
+          const uint4 rec = lds128s(ce + part * (128 * 64) + r * 64 + 16 * q);
           const float dsc = half_bits_to_float(static_cast<uint16_t>(dq0)) * 128.0f;  // d / 8 * 2^10
           uint32_t o0[16], o1[16];
           dq_iq2_sub(make_uint2(rec.x, rec.y), dsc, tabL, tabS, o0);
@@ -556,8 +581,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           tmem_st16(tc + 16, o1);
         } else {
           // part = half of the stage's 64 weights = sub-blocks 4 * (ks % 4) + 2 * part, +1 of the block
-          const uint2 w = lds64s(code + 8 * part);
-          const uint32_t scb = lds16s(code + kCodeChunk + 4 * (ks & 3) + 2 * part);
+          const uint2 w = lds64s(ce + r * 80 + 16 + 16 * q + 8 * part);
+          const uint32_t scb = lds16s(ce + r * 80 + 4 * q + 2 * part);
           const float d = half_bits_to_float(static_cast<uint16_t>(dq0 & 0xFFFFu));
           const float dmin = half_bits_to_float(static_cast<uint16_t>(dq0 >> 16));
           uint32_t o0[8], o1[8];
@@ -571,6 +596,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&fullA[sa]);
+        if (q == grp + 2) {  // this group's last stage of the block: the code entry is free for this warp
+          if (lane == 0) mbar_arrive(&emptyC[cb]);
+          if (++cb == kCStages) { cb = 0; pcb ^= 1u; }
+        }
       }
       if (!ok) break;
       u = un;
@@ -839,13 +868,13 @@ bool tc_map(CUtensorMap* m, const void* base, bool bf16, uint64_t K, uint64_t ro
   return r == CUDA_SUCCESS;
 }
 
-// 2-D map over a plane of code bytes: rows of `row_bytes`, boxes of 16 bytes x 128 rows.
-bool code_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows) {
+// 2-D map over a plane of code bytes: rows of `row_bytes`, boxes of `box_bytes` x 128 rows.
+bool code_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_bytes) {
   auto fn = tc_encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {row_bytes, rows};
   const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {16, 128};
+  const cuuint32_t box[2] = {box_bytes, 128};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -962,8 +991,8 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
   {
     ProfScope ps(MOE_K_PREFILL_GATEUP, st);
     const uint64_t wrows = static_cast<uint64_t>(sh.E) * sh.I;
-    if (!tc_map(&mb, pw.xp, false, sh.H, nA, 1) || !code_map(&ma0, w.gate_codes, sh.H / 4, wrows) ||
-        !code_map(&ma1, w.up_codes, sh.H / 4, wrows))
+    if (!tc_map(&mb, pw.xp, false, sh.H, nA, 1) || !code_map(&ma0, w.gate_codes, sh.H / 4, wrows, 64) ||
+        !code_map(&ma1, w.up_codes, sh.H / 4, wrows, 64))
       return ERR_CUDA;
     TcArgs a{};
     a.n_experts = sh.E; a.b_rows = nA;
@@ -990,7 +1019,7 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
   {
     ProfScope ps(MOE_K_PREFILL_DOWN, st);
     if (!tc_map(&mb, pw.hh, false, sh.I, nA, 1) ||
-        !code_map(&ma0, w.down_codes, static_cast<uint64_t>(sh.I / 256) * 80, static_cast<uint64_t>(sh.E) * sh.H))
+        !code_map(&ma0, w.down_codes, static_cast<uint64_t>(sh.I / 256) * 80, static_cast<uint64_t>(sh.E) * sh.H, 80))
       return ERR_CUDA;
     TcArgs a{};
     a.n_experts = sh.E; a.b_rows = nA;
