@@ -179,9 +179,6 @@ __device__ __forceinline__ uint32_t f2_to_h2(float lo, float hi) {
   __half2 r = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&r);
 }
-__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
-  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
-}
 __device__ __forceinline__ uint4 lds128s(uint32_t a) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
@@ -195,11 +192,6 @@ __device__ __forceinline__ uint2 lds64s(uint32_t a) {
 __device__ __forceinline__ uint32_t lds16s(uint32_t a) {
   uint32_t v;
   asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ uint32_t lds8s(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
 __device__ __forceinline__ uint32_t lds32s(uint32_t a) {
