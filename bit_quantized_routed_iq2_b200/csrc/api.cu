@@ -188,7 +188,10 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights
   int rc = launch_route(weights->router_w, weights->router_bias, x, x_dtype, T, desc->hidden, desc->n_experts,
                         desc->top_k, w.logits, w.topk_idx, w.topk_w, w.offsets, w.perm, w.inv, w.active, w.status,
                         s, early);
-  if (rc != OK) return to_status(rc);
+  if (rc != OK) {
+    if (early) join_shared_early(s);  // leave no forked work unjoined (graph capture requires it)
+    return to_status(rc);
+  }
   Routing r{w.topk_w, w.offsets, w.perm, w.inv, w.active};
   // the status word is cleared by the first kernel on the caller's stream: the router when the shared
   // expert and the digits run ahead on the side stream, the tensor-core router for many bf16 tokens

@@ -443,6 +443,10 @@ bool shared_early_ok(const LayerShape& s, int x_dtype, int T) {
          shared_mma_supported(s.H, s.Is, T, 1, s.k);
 }
 
+void join_shared_early(cudaStream_t st) {
+  if (SideCtx* c = side_ctx(st)) cudaStreamWaitEvent(st, c->join, 0);
+}
+
 int launch_shared_early(const LayerShape& s, const WeightPtrs& w, const void* x, int T, void* ws, cudaStream_t st) {
   SideCtx* c = side_ctx(st);
   if (!c) return ERR_CUDA;

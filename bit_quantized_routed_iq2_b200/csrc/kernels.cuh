@@ -74,6 +74,8 @@ bool shared_mma_supported(int H, int Is, int T, int x_parts, int k);
 // the decode path's combine waits for it. Returns true when it was launched.
 bool shared_early_ok(const LayerShape& s, int x_dtype, int T);
 int launch_shared_early(const LayerShape& s, const WeightPtrs& w, const void* x, int T, void* ffn_ws, cudaStream_t st);
+// Joins the side stream back into `st` (the error path of a call that forked it).
+void join_shared_early(cudaStream_t st);
 int launch_shared_gateup_mma(int H, int Is, const uint16_t* wg, const uint16_t* wu, const uint16_t* xb, int P,
                              int T, uint16_t* hb, cudaStream_t st);
 int launch_shared_down_combine_mma(int H, int Is, const uint16_t* wd, const uint16_t* hb, int T, int k,
