@@ -25,8 +25,13 @@
  * Conventions for every call:
  *   - Pointers marked "device" must be device-accessible memory of the current
  *     CUDA device; "host" pointers are ordinary host memory. All buffers are
- *     owned by the caller. The library never allocates or frees device memory,
- *     never synchronises, and only enqueues work on `stream`.
+ *     owned by the caller. The library never allocates or frees device memory
+ *     and never synchronises. Work is ordered on `stream`: it starts after the
+ *     work already enqueued there and finishes before anything enqueued later.
+ *     moe_layer_forward may run part of it on a side stream that it forks from
+ *     `stream` and joins back with events (created once per device and caller
+ *     stream, kept for the life of the process); this is safe inside CUDA graph
+ *     capture.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *   - Argument and shape errors are detected on the host before anything is
  *     enqueued and are returned as a status; nothing is launched in that case.
@@ -170,7 +175,10 @@ MOE_API moe_status moe_expert_ffn(const moe_layer_desc* desc, const moe_layer_we
 
 /*
  * The whole layer: moe_route then moe_expert_ffn, with the routing kept in the
- * workspace. Same argument meanings as above.
+ * workspace. Same argument meanings as above. For bf16 x on the decode path
+ * (T <= 16) the shared expert's gate/up and the activation digits, which do not
+ * depend on routing, run on a side stream forked from `stream` before the
+ * router and joined back before the combine.
  */
 MOE_API moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights* w, const void* x,
                              moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws,
