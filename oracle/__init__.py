@@ -14,8 +14,10 @@ import subprocess
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SO = os.path.join(_HERE, "liboracle.so")
+_SO = os.path.join(_HERE, "liboracle.so")          # single-threaded build
+_SO_OMP = os.path.join(_HERE, "liboracle_omp.so")  # the same source with OpenMP on
 _lib = None
+_openmp = os.environ.get("MOEREF_OPENMP", "1") != "0"
 
 F32, BF16 = 0, 1
 
@@ -34,21 +36,46 @@ class Weights(ctypes.Structure):
     ]
 
 
-def build(force: bool = False, openmp: bool = False) -> str:
-    """Compile the oracle: plain C99, -O2, no fast-math, no FMA contraction."""
+def build(force: bool = False, openmp: bool | None = None) -> str:
+    """Compile the oracle: plain C99, -O2, no fast-math, no FMA contraction.
+
+    Two builds of the one source: ``liboracle.so`` (single thread) and
+    ``liboracle_omp.so`` (-fopenmp: independent tokens, assignments, rows and
+    blocks spread over threads; every output is still computed by one thread
+    with the same sequential loop, so both builds return identical bits).
+    ``openmp=None`` builds both and returns the path of the one in use."""
     src = os.path.join(_HERE, "moeref.c")
-    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(src):
-        cmd = ["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c99", "-fPIC", "-shared",
-               "-o", _SO, src, "-lm"]
-        subprocess.check_call(cmd)
-    return _SO
+    base = ["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c99", "-fPIC", "-shared"]
+    for so, extra in ((_SO, ["-Wno-unknown-pragmas"]), (_SO_OMP, ["-fopenmp"])):
+        if openmp is not None and (so == _SO_OMP) != openmp:
+            continue
+        if force or not os.path.exists(so) or os.path.getmtime(so) < os.path.getmtime(src):
+            subprocess.check_call([*base, *extra, "-o", so, src, "-lm"])
+    if openmp is None:
+        return _SO_OMP if _openmp else _SO
+    return _SO_OMP if openmp else _SO
+
+
+def use_openmp(on: bool) -> None:
+    """Select the build that lib() loads (before its first call)."""
+    global _openmp
+    if _lib is not None and on != _openmp:
+        raise RuntimeError("the oracle library is already loaded")
+    _openmp = on
+
+
+def threads() -> int:
+    """Threads the loaded build may use (1 for the single-threaded build)."""
+    if not _openmp:
+        return 1
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n and n.isdigit() else (os.cpu_count() or 1)
 
 
 def lib():
     global _lib
     if _lib is None:
-        build()
-        L = ctypes.CDLL(_SO)
+        L = ctypes.CDLL(build(openmp=_openmp))
         vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
         L.moeref_f16_to_f64.restype = ctypes.c_double
         L.moeref_f16_to_f64.argtypes = [ctypes.c_uint16]

@@ -127,6 +127,8 @@ void moeref_grid(uint8_t out[256 * 8]) {
 void moeref_dequant_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, float* out) {
   uint8_t grid[256 * 8];
   moeref_grid(grid);
+  /* blocks are independent */
+#pragma omp parallel for schedule(static)
   for (int64_t b = 0; b < nblocks; ++b) {
     const uint8_t* q = codes + b * IQ2_BYTES;
     double db = moeref_f16_to_f64(d[b]);
@@ -157,6 +159,8 @@ void moeref_dequant_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks
  * double and the difference is exact in double; the cast to fp32 is the only
  * rounding. Parity: pinned by hand-worked blocks and exhaustive checks. */
 void moeref_dequant_q2k(const uint8_t* codes, const uint32_t* dd, int64_t nblocks, float* out) {
+  /* blocks are independent */
+#pragma omp parallel for schedule(static)
   for (int64_t b = 0; b < nblocks; ++b) {
     const uint8_t* q = codes + b * Q2K_BYTES;
     double dv = moeref_f16_to_f64((uint16_t)(dd[b] & 0xFFFFu));
@@ -195,11 +199,20 @@ int moeref_route(int H, int E, int k, const uint16_t* router_w, const float* rou
                  int x_dtype, int T, int32_t* topk_idx, float* topk_w, double* logits_out) {
   if (H <= 0 || E <= 0 || k <= 0 || k > E || T < 0 || !router_w || (T && (!x || !topk_idx || !topk_w)))
     return REF_ERR_ARG;
-  double* l = (double*)malloc(sizeof(double) * (size_t)E);
-  char* taken = (char*)malloc((size_t)E);
-  double* lw = (double*)malloc(sizeof(double) * (size_t)k);
-  if (!l || !taken || !lw) { free(l); free(taken); free(lw); return REF_ERR_NOMEM; }
+  int rc = REF_OK;
+  /* tokens are independent; with OpenMP they are spread over threads (the
+     arithmetic of each token is the same sequential loop either way) */
+#pragma omp parallel for schedule(dynamic, 1)
   for (int t = 0; t < T; ++t) {
+    double* l = (double*)malloc(sizeof(double) * (size_t)E);
+    char* taken = (char*)malloc((size_t)E);
+    double* lw = (double*)malloc(sizeof(double) * (size_t)k);
+    if (!l || !taken || !lw) {
+      free(l); free(taken); free(lw);
+#pragma omp critical
+      rc = REF_ERR_NOMEM;
+      continue;
+    }
     for (int e = 0; e < E; ++e) {
       double acc = 0.0;
       for (int h = 0; h < H; ++h)
@@ -220,11 +233,11 @@ int moeref_route(int H, int E, int k, const uint16_t* router_w, const float* rou
     double z = 0.0;
     for (int j = 0; j < k; ++j) z += exp(lw[j] - lw[0]);
     for (int j = 0; j < k; ++j) topk_w[(int64_t)t * k + j] = (float)(exp(lw[j] - lw[0]) / z);
+    free(l);
+    free(taken);
+    free(lw);
   }
-  free(l);
-  free(taken);
-  free(lw);
-  return REF_OK;
+  return rc;
 }
 
 /* ------------------------------------------------------------- permutation
@@ -284,49 +297,71 @@ int moeref_expert_ffn(const moeref_desc* desc, const moeref_weights* W, const vo
   float* wg = (float*)malloc(sizeof(float) * (size_t)I * H);
   float* wu = (float*)malloc(sizeof(float) * (size_t)I * H);
   float* wd = (float*)malloc(sizeof(float) * (size_t)H * I);
-  double* h = (double*)malloc(sizeof(double) * (size_t)I);
-  if (!o || !wg || !wu || !wd || !h) { free(o); free(wg); free(wu); free(wd); free(h); return REF_ERR_NOMEM; }
+  if (!o || !wg || !wu || !wd) { free(o); free(wg); free(wu); free(wd); return REF_ERR_NOMEM; }
 
+  int64_t* mine = (int64_t*)malloc(sizeof(int64_t) * (size_t)(nA > 0 ? nA : 1));
+  if (!mine) { free(o); free(wg); free(wu); free(wd); return REF_ERR_NOMEM; }
   for (int e = 0; e < E; ++e) {
-    int used = 0;
-    for (int64_t a = 0; a < nA; ++a) used |= topk_idx[a] == e;
-    if (!used) continue;
+    int64_t na = 0;
+    for (int64_t a = 0; a < nA; ++a)
+      if (topk_idx[a] == e) mine[na++] = a;
+    if (!na) continue;
     dequant_matrix_iq2(W->gate_codes, W->gate_d, e, I, H, wg);
     dequant_matrix_iq2(W->up_codes, W->up_d, e, I, H, wu);
     dequant_matrix_q2k(W->down_codes, W->down_dd, e, H, I, wd);
-    for (int64_t a = 0; a < nA; ++a) {
-      if (topk_idx[a] != e) continue;
-      int64_t t = a / k;
+    /* the assignments of expert e (and, with OpenMP, their rows) are
+       independent; each dot product is the same sequential loop */
+    double* hh = (double*)malloc(sizeof(double) * (size_t)na * I);
+    double* xa = (double*)malloc(sizeof(double) * (size_t)na * H); /* exact widening of x_t */
+    if (!hh || !xa) { free(hh); free(xa); free(mine); free(o); free(wg); free(wu); free(wd); return REF_ERR_NOMEM; }
+    for (int64_t i = 0; i < na; ++i)
+      for (int c = 0; c < H; ++c) xa[i * H + c] = act_in(x, x_dtype, (mine[i] / k) * H + c);
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t i = 0; i < na; ++i)
       for (int r = 0; r < I; ++r) {
         double g = 0.0, u = 0.0;
         for (int c = 0; c < H; ++c) {
-          double xv = act_in(x, x_dtype, t * H + c);
+          double xv = xa[i * H + c];
           g += (double)wg[(int64_t)r * H + c] * xv;
           u += (double)wu[(int64_t)r * H + c] * xv;
         }
-        h[r] = silu(g) * u;
+        hh[i * I + r] = silu(g) * u;
       }
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t i = 0; i < na; ++i)
       for (int r = 0; r < H; ++r) {
         double acc = 0.0;
-        for (int c = 0; c < I; ++c) acc += (double)wd[(int64_t)r * I + c] * h[c];
-        o[a * H + r] = acc;
+        for (int c = 0; c < I; ++c) acc += (double)wd[(int64_t)r * I + c] * hh[i * I + c];
+        o[mine[i] * H + r] = acc;
       }
-    }
+    free(hh);
+    free(xa);
   }
+  free(mine);
   free(wg);
   free(wu);
   free(wd);
 
-  double* hs = (double*)malloc(sizeof(double) * (size_t)(Is > 0 ? Is : 1));
-  double* s = (double*)malloc(sizeof(double) * (size_t)H);
-  if (!hs || !s) { free(o); free(h); free(hs); free(s); return REF_ERR_NOMEM; }
+  int rc = REF_OK;
+  /* tokens are independent (shared expert and combine) */
+#pragma omp parallel for schedule(dynamic, 1)
   for (int64_t t = 0; t < T; ++t) {
+    double* hs = (double*)malloc(sizeof(double) * (size_t)(Is > 0 ? Is : 1));
+    double* s = (double*)malloc(sizeof(double) * (size_t)H);
+    double* xt = (double*)malloc(sizeof(double) * (size_t)H); /* exact widening of x_t */
+    if (!hs || !s || !xt) {
+      free(hs); free(s); free(xt);
+#pragma omp critical
+      rc = REF_ERR_NOMEM;
+      continue;
+    }
     for (int r = 0; r < H; ++r) s[r] = 0.0;
+    for (int c = 0; c < H; ++c) xt[c] = act_in(x, x_dtype, t * H + c);
     if (Is > 0) {
       for (int r = 0; r < Is; ++r) {
         double g = 0.0, u = 0.0;
         for (int c = 0; c < H; ++c) {
-          double xv = act_in(x, x_dtype, t * H + c);
+          double xv = xt[c];
           g += moeref_bf16_to_f64(W->sh_gate[(int64_t)r * H + c]) * xv;
           u += moeref_bf16_to_f64(W->sh_up[(int64_t)r * H + c]) * xv;
         }
@@ -345,12 +380,12 @@ int moeref_expert_ffn(const moeref_desc* desc, const moeref_weights* W, const vo
       if (residual) acc += (double)residual[t * H + r];
       y[t * H + r] = (float)acc;
     }
+    free(hs);
+    free(s);
+    free(xt);
   }
   free(o);
-  free(h);
-  free(hs);
-  free(s);
-  return REF_OK;
+  return rc;
 }
 
 /* ------------------------------------------------------------ whole layer

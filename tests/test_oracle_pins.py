@@ -350,3 +350,32 @@ def test_token_permutation_equivariance():
     p = np.array([2, 0, 3, 1])
     y1, _, _ = oracle.layer_forward(lw, np.ascontiguousarray(x[p]))
     assert np.array_equal(y1, y0[p])
+
+
+# ------------------------------------------------------- OpenMP build identity
+def test_openmp_build_returns_identical_bits(tmp_path):
+    """The OpenMP build spreads independent outputs over threads; each output is
+    still one sequential loop, so its bits equal the single-threaded build's."""
+    import subprocess
+    import sys
+
+    code = r'''
+import os, sys, numpy as np
+sys.path.insert(0, sys.argv[1])
+import oracle, synth
+sys.path.insert(0, os.path.join(sys.argv[1], "tests"))
+cfg = synth.Config("omp_pin", 9, 512, 256, 8, 3, 64, "bf16", 1.0, True, 1, 0x0B5E)
+lw = synth.make_layer(cfg)
+x = synth.make_x(cfg)
+y, idx, w = oracle.layer_forward(lw, x, synth.make_residual(cfg, cfg.T))
+np.savez(sys.argv[2], y=y, idx=idx, w=w)
+'''
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    outs = {}
+    for flag in ("0", "1"):
+        out = str(tmp_path / f"o{flag}.npz")
+        env = dict(os.environ, MOEREF_OPENMP=flag, OMP_NUM_THREADS="4")
+        subprocess.check_call([sys.executable, "-c", code, root, out], env=env)
+        outs[flag] = np.load(out)
+    for key in ("y", "idx", "w"):
+        assert np.array_equal(outs["0"][key], outs["1"][key]), key
