@@ -88,6 +88,10 @@ def lib():
         L.moeref_dequant_q2k.argtypes = [vp, vp, i64, vp]
         L.moeref_route.argtypes = [i32, i32, i32, vp, vp, vp, i32, i32, vp, vp, vp]
         L.moeref_permute.argtypes = [i32, i32, i32, vp, vp, vp, vp]
+        L.moeref_f32_to_f16.restype = ctypes.c_uint16
+        L.moeref_f32_to_f16.argtypes = [ctypes.c_float]
+        L.moeref_quantize_q2k.argtypes = [vp, i64, vp, vp]
+        L.moeref_quantize_iq2.argtypes = [vp, i64, vp, vp]
         L.moeref_expert_ffn.argtypes = [ctypes.POINTER(Desc), ctypes.POINTER(Weights), vp, i32, i32, vp, vp, vp, vp]
         L.moeref_layer_forward.argtypes = [ctypes.POINTER(Desc), ctypes.POINTER(Weights), vp, i32, i32, vp, vp, vp, vp]
         _lib = L
@@ -145,6 +149,33 @@ def dequant_q2k(codes: np.ndarray, dd: np.ndarray) -> np.ndarray:
     out = np.zeros(codes.shape[0] * 256, np.float32)
     lib().moeref_dequant_q2k(_p(codes), _p(dd), codes.shape[0], _p(out))
     return out
+
+
+def f32_to_f16(v: float) -> int:
+    return int(lib().moeref_f32_to_f16(float(v)))
+
+
+def quantize_q2k(w: np.ndarray):
+    """Float weights (a multiple of 256, blocks along the flattened array) ->
+    (codes [nb][80] u8, dd [nb] u32)."""
+    w = np.ascontiguousarray(w, np.float32).reshape(-1)
+    assert w.size % 256 == 0
+    nb = w.size // 256
+    codes = np.zeros((nb, 80), np.uint8)
+    dd = np.zeros(nb, np.uint32)
+    lib().moeref_quantize_q2k(_p(w), nb, _p(codes), _p(dd))
+    return codes, dd
+
+
+def quantize_iq2(w: np.ndarray):
+    """Float weights -> (codes [nb][64] u8, d [nb] fp16 bits)."""
+    w = np.ascontiguousarray(w, np.float32).reshape(-1)
+    assert w.size % 256 == 0
+    nb = w.size // 256
+    codes = np.zeros((nb, 64), np.uint8)
+    d = np.zeros(nb, np.uint16)
+    lib().moeref_quantize_iq2(_p(w), nb, _p(codes), _p(d))
+    return codes, d
 
 
 def route(router_w, router_bias, x, k: int, want_logits: bool = False):

@@ -399,3 +399,157 @@ int moeref_layer_forward(const moeref_desc* desc, const moeref_weights* W, const
   if (rc) return rc;
   return moeref_expert_ffn(desc, W, x, x_dtype, T, topk_idx, topk_w, residual, y);
 }
+
+/* ------------------------------------------------------------- quantisers
+ * Float weights -> the two block formats, without an importance matrix. The
+ * pages say the routed experts are quantized (IQ2_XXS for up/gate, Q2_K for
+ * down) and that the project's own 2-bit files were made with an imatrix
+ * ("ds4 : un MoE de 284 milliards sur un Mac de 128 Go", « Comment un 284B
+ * tient »); they give no algorithm. These are this project's plain rules:
+ * round-to-nearest for Q2K and an exhaustive codebook search for IQ2. Every
+ * decision (a scale byte, a code, a codebook row) is taken in fp32 with the
+ * operations below in the order written, each rounded to nearest even and
+ * none fused, so that another implementation can reproduce the codes bit for
+ * bit. Parity: pinned by hand-worked blocks, reconstruction bounds and a
+ * brute-force optimality check of the IQ2 search. */
+
+/* fp32 -> IEEE binary16, round to nearest even; finite inputs below 65520. */
+uint16_t moeref_f32_to_f16(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+  uint32_t a = u & 0x7FFFFFFFu;
+  if (a >= 0x477FF000u) return sign | 0x7C00u; /* rounds to inf */
+  if (a < 0x33000001u) return sign;             /* below half the smallest subnormal: +-0 */
+  int e = (int)(a >> 23) - 127;
+  uint32_t m = (a & 0x7FFFFFu) | 0x800000u;    /* 24-bit significand */
+  int shift;                                    /* bits dropped from m */
+  uint32_t base;
+  if (e < -14) { /* subnormal half: value = m * 2^(e-23) = k * 2^-24 with k = m * 2^(e+1) */
+    shift = -1 - e;
+    base = 0;
+  } else {
+    shift = 13;
+    base = (uint32_t)(e + 15) << 10;
+    m &= 0x7FFFFFu; /* drop the implicit bit: the mantissa field */
+  }
+  uint32_t q = m >> shift, rem = m & ((1u << shift) - 1u), half = 1u << (shift - 1);
+  if (rem > half || (rem == half && (q & 1u))) q += 1; /* a carry into the exponent is correct rounding */
+  return (uint16_t)(sign | (base + q));
+}
+
+static float f16_to_f32(uint16_t h) { return (float)moeref_f16_to_f64(h); }
+
+static float clampf_(float v, float lo, float hi) { return v < lo ? lo : (v > hi ? hi : v); }
+
+/* Q2K round-to-nearest, per 256-weight block:
+ *   sub-block s (16 weights): lo_s = min(0, min w), hi_s = max w,
+ *     step_s = (hi_s - lo_s) / 3, off_s = -lo_s;
+ *   d = fp16(max_s step_s / 15), dmin = fp16(max_s off_s / 15);
+ *   sc_s = clamp(rint(step_s / d), 0, 15) (0 if d == 0),
+ *   m_s = clamp(rint(off_s / dmin), 0, 15) (0 if dmin == 0);
+ *   q = clamp(rint((w + dmin * m_s) / (d * sc_s)), 0, 3) (0 if d * sc_s == 0). */
+void moeref_quantize_q2k(const float* w, int64_t nblocks, uint8_t* codes, uint32_t* dd) {
+#pragma omp parallel for schedule(static)
+  for (int64_t b = 0; b < nblocks; ++b) {
+    const float* x = w + b * QK;
+    uint8_t* q = codes + b * Q2K_BYTES;
+    float step[16], off[16], smax = 0.f, omax = 0.f;
+    for (int s = 0; s < 16; ++s) {
+      float lo = 0.f, hi = x[16 * s];
+      for (int i = 0; i < 16; ++i) {
+        if (x[16 * s + i] < lo) lo = x[16 * s + i];
+        if (x[16 * s + i] > hi) hi = x[16 * s + i];
+      }
+      step[s] = (hi - lo) / 3.0f;
+      off[s] = -lo;
+      if (step[s] > smax) smax = step[s];
+      if (off[s] > omax) omax = off[s];
+    }
+    uint16_t d16 = moeref_f32_to_f16(smax / 15.0f), m16 = moeref_f32_to_f16(omax / 15.0f);
+    float df = f16_to_f32(d16), mf = f16_to_f32(m16);
+    dd[b] = (uint32_t)d16 | ((uint32_t)m16 << 16);
+    memset(q, 0, Q2K_BYTES);
+    for (int s = 0; s < 16; ++s) {
+      int sc = df > 0.f ? (int)clampf_(rintf(step[s] / df), 0.f, 15.f) : 0;
+      int m = mf > 0.f ? (int)clampf_(rintf(off[s] / mf), 0.f, 15.f) : 0;
+      q[s] = (uint8_t)(sc | (m << 4));
+      float st = df * (float)sc, of = mf * (float)m;
+      for (int i = 0; i < 16; ++i) {
+        int v = st > 0.f ? (int)clampf_(rintf((x[16 * s + i] + of) / st), 0.f, 3.f) : 0;
+        int k = 16 * s + i;
+        q[16 + k / 4] |= (uint8_t)(v << (2 * (k % 4)));
+      }
+    }
+  }
+}
+
+/* IQ2 codebook search, per 256-weight block:
+ *   d = fp16(max |w| * 8 / (31 * 43)) (the largest magnitude the format holds
+ *   is d * 31 * 43 / 8); with d == 0 every code is 0;
+ *   sub-block s (32 weights): ls = clamp(rint((max|w| * 8 / (d * 43) - 1) / 2), 0, 15),
+ *   c = d * (2 ls + 1) / 8;
+ *   group j (8 weights): element signs follow w (w < 0 is negative); if their
+ *   count is odd, the element of smallest |w| (lowest e on ties) is flipped,
+ *   since the format's eighth sign is the parity of the other seven. For every
+ *   codebook row r the error sum_e (|w_e| -+ c * grid[r][e])^2 is formed in
+ *   fp32 with e ascending (the flipped element takes +); the row of least error
+ *   wins, the lower row on ties. */
+void moeref_quantize_iq2(const float* w, int64_t nblocks, uint8_t* codes, uint16_t* d) {
+  uint8_t grid[256 * 8];
+  moeref_grid(grid);
+#pragma omp parallel for schedule(static)
+  for (int64_t b = 0; b < nblocks; ++b) {
+    const float* x = w + b * QK;
+    uint8_t* q = codes + b * IQ2_BYTES;
+    float amax = 0.f;
+    for (int i = 0; i < QK; ++i) amax = fabsf(x[i]) > amax ? fabsf(x[i]) : amax;
+    uint16_t d16 = moeref_f32_to_f16(amax * 8.0f / 1333.0f);
+    float df = f16_to_f32(d16);
+    d[b] = d16;
+    memset(q, 0, IQ2_BYTES);
+    if (!(df > 0.f)) continue;
+    for (int s = 0; s < 8; ++s) {
+      float smax = 0.f;
+      for (int i = 0; i < 32; ++i) smax = fabsf(x[32 * s + i]) > smax ? fabsf(x[32 * s + i]) : smax;
+      int ls = (int)clampf_(rintf((smax * 8.0f / (df * 43.0f) - 1.0f) / 2.0f), 0.f, 15.f);
+      float c = df * (float)(2 * ls + 1) / 8.0f;
+      uint32_t v = (uint32_t)ls << 28;
+      for (int j = 0; j < 4; ++j) {
+        const float* g = x + 32 * s + 8 * j;
+        int neg[8], nneg = 0, flip = -1;
+        float a[8];
+        for (int e = 0; e < 8; ++e) {
+          a[e] = fabsf(g[e]);
+          neg[e] = g[e] < 0.f;
+          nneg += neg[e];
+        }
+        if (nneg & 1) {
+          flip = 0;
+          for (int e = 1; e < 8; ++e)
+            if (a[e] < a[flip]) flip = e;
+        }
+        int best = 0;
+        float best_err = 0.f;
+        for (int r = 0; r < 256; ++r) {
+          float err = 0.f;
+          for (int e = 0; e < 8; ++e) {
+            float t = c * (float)grid[r * 8 + e];
+            float diff = e == flip ? a[e] + t : a[e] - t;
+            err = err + diff * diff;
+          }
+          if (r == 0 || err < best_err) {
+            best = r;
+            best_err = err;
+          }
+        }
+        q[8 * s + j] = (uint8_t)best;
+        for (int e = 0; e < 7; ++e) v |= (uint32_t)(neg[e] ^ (e == flip)) << (7 * j + e);
+      }
+      q[8 * s + 4] = (uint8_t)(v & 0xFF);
+      q[8 * s + 5] = (uint8_t)((v >> 8) & 0xFF);
+      q[8 * s + 6] = (uint8_t)((v >> 16) & 0xFF);
+      q[8 * s + 7] = (uint8_t)(v >> 24);
+    }
+  }
+}
