@@ -40,7 +40,7 @@ HBM_FALLBACK_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="decode1", choices=["decode1", "decode32", "prefill", "stack"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -52,6 +52,11 @@ def parse():
                     help="override the routed expert count (small cases for profiling; not a bench workload)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the tokens per step (small cases for profiling; not a bench workload)")
+    ap.add_argument("--workloads", default="auto",
+                    help="other workloads measured in the same run and reported under 'workloads': 'all' "
+                         "(decode32, prefill, stack, decode1_cached, quantize), 'none', or a comma list; "
+                         "'auto' = all on one GPU")
+    ap.add_argument("--workload-steps", type=int, default=20, help="timed steps of each extra workload")
     return ap.parse_args()
 
 
@@ -117,14 +122,15 @@ def expert_bytes(cfg) -> dict:
             "router": cfg.E * cfg.H * 2}
 
 
-def traffic_record(kernel: str):
-    """dram bytes per launch from a committed ncu summary, if its source hash
-    matches the current kernel source; else None."""
+def traffic_record(workload: str, kernel: str):
+    """dram bytes per launch of `kernel` in `workload` from a committed ncu
+    summary (key "workload:kernel"), if its source hash matches the current
+    kernel source; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     try:
-        rec = json.load(open(p)).get(kernel)
+        rec = json.load(open(p)).get(f"{workload}:{kernel}")
         if not rec:
             return None
         src = os.path.join(ROOT, rec["source"])
@@ -158,7 +164,34 @@ def rank_seed(cfg_seed, rank):
 
 
 # --------------------------------------------------------------- reference
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_tokens(cfg, x, budget_s, tokens_per_call):
+    """Oracle throughput on a bounded sample: calls of `tokens_per_call` tokens
+    until `budget_s` seconds have passed (at least one call)."""
+    import oracle
+
+    lw = synth.make_layer(cfg)
+    n, t0 = 0, time.perf_counter()
+    while n + tokens_per_call <= x.shape[0]:
+        oracle.layer_forward(lw, np.ascontiguousarray(x[n:n + tokens_per_call]))
+        n += tokens_per_call
+        if time.perf_counter() - t0 > budget_s:
+            break
+    return n, time.perf_counter() - t0
+
+
 def run_reference(args, cfg):
+    """The reference arm: the CPU oracle as it stands (OpenMP build, every host
+    core), one bounded sample of the workload per step."""
     import oracle
 
     rank = int(os.environ.get("RANK", "0"))
@@ -166,67 +199,73 @@ def run_reference(args, cfg):
         return
     oracle.build()
     lw = synth.make_layer(cfg)
-    # per step: one token through the whole layer (router, k experts, shared)
-    x = synth.make_x_fast(cfg, max(args.steps + args.warmup, 1))
-    per_step_tokens = 1
+    per_step_tokens = 1 if cfg.T < 64 else 16
+    x = synth.make_x_fast(cfg, max(args.steps + args.warmup, 1) * per_step_tokens)
     for i in range(args.warmup):
-        oracle.layer_forward(lw, np.ascontiguousarray(x[i:i + 1]))
+        oracle.layer_forward(lw, np.ascontiguousarray(x[i * per_step_tokens:(i + 1) * per_step_tokens]))
     t0 = time.perf_counter()
     for i in range(args.steps):
         j = args.warmup + i
-        oracle.layer_forward(lw, np.ascontiguousarray(x[j:j + 1]))
+        oracle.layer_forward(lw, np.ascontiguousarray(x[j * per_step_tokens:(j + 1) * per_step_tokens]))
     dt = time.perf_counter() - t0
     value = per_step_tokens * args.steps / dt
-    sample = f"{per_step_tokens} token per step through the full {cfg.name} layer (router, {cfg.k} experts, shared)"
+    cores = oracle.threads()
+    sample = (f"{per_step_tokens} token(s) per step through the full {cfg.name} layer (router, {cfg.k} experts, "
+              f"shared), C oracle on {cores} threads")
     line = {
         "impl": "reference", "metric": "moe_layer_tokens_per_s", "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": cfg.name, "tokens_per_step": per_step_tokens, "H": cfg.H, "I": cfg.I, "E": cfg.E,
                    "k": cfg.k, "I_s": cfg.Is},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
+                         "cpu_model": cpu_model(), "nproc": os.cpu_count()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(cfg, budget_s=15.0):
+def cpu_baseline(cfg, budget_s=12.0):
+    """The oracle timed on the host cores: the OpenMP build on every core (the
+    reported value) and the single-threaded build (context), each on a bounded
+    sample of the workload's tokens."""
+    import subprocess as sp
+
+    x = synth.make_x_fast(cfg, 64)
     import oracle
 
     oracle.build()
-    lw = synth.make_layer(cfg)
-    x = synth.make_x_fast(cfg, 64)
-    n, t0 = 0, time.perf_counter()
-    while n < 64:
-        oracle.layer_forward(lw, np.ascontiguousarray(x[n:n + 1]))
-        n += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": n / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} tokens of the {cfg.name} layer one at a time, single-threaded C oracle ({dt:.1f} s)"}
+    n, dt = oracle_tokens(cfg, x, budget_s, 1)
+    out = {"value": n / dt, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+           "sample": f"{n} tokens of the {cfg.name} layer one at a time, C oracle (OpenMP) on {oracle.threads()} "
+                     f"threads ({dt:.1f} s)",
+           "cpu_model": cpu_model(), "nproc": os.cpu_count()}
+    # the single-threaded build, in a child process (the OpenMP build is loaded here)
+    code = ("import sys, json; sys.path.insert(0, sys.argv[1]); import bench, synth; "
+            "cfg = synth.CONFIGS[sys.argv[2]]; x = synth.make_x_fast(cfg, 64); "
+            "n, dt = bench.oracle_tokens(cfg, x, float(sys.argv[3]), 1); print(json.dumps([n, dt]))")
+    try:
+        r = sp.run([sys.executable, "-c", code, ROOT, cfg.name, str(budget_s / 2)], capture_output=True, text=True,
+                   env=dict(os.environ, MOEREF_OPENMP="0"), timeout=600)
+        n1, dt1 = json.loads(r.stdout.strip().splitlines()[-1])
+        out["single_thread"] = {"value": n1 / dt1, "unit": "tokens/s", "cores": 1,
+                                "sample": f"{n1} tokens one at a time ({dt1:.1f} s)"}
+    except Exception as exc:  # the figure is context only
+        out["single_thread"] = {"unavailable": str(exc)[:200]}
+    return out
 
 
 # -------------------------------------------------------------------- ours
-def run_ours(args, cfg):
+def measure(args, cfg, world, rank, local, steps):
+    """Time `steps` steps of one workload (CUDA-graph replay, device events, max
+    over ranks), then the same steps with per-kernel events, then end to end
+    with host buffers. Returns the JSON fields of that workload."""
     import torch
-    import torch.distributed as dist
 
-    from bit_quantized_routed_iq2_b200 import build as moebuild
     from bit_quantized_routed_iq2_b200 import moe2bit
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        from datetime import timedelta
-
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
-    moebuild.build()
-    moe2bit.load()
-
     n_layers = args.layers or {"decode1": 4, "decode32": 4, "prefill": 2, "stack": cfg.layers}.get(cfg.name, 1)
+    is_stack = cfg.name.startswith("stack")
     T = cfg.T
     layers = []
     for l in range(n_layers):
@@ -235,7 +274,6 @@ def run_ours(args, cfg):
         del lw
     n_slots = 4
     xs_host = [synth.make_x_fast(cfg, T, layer=100 + s, cfg_seed=rank_seed(cfg.seed, rank)) for s in range(n_slots)]
-    xdt = torch.bfloat16 if cfg.x_dtype == "bf16" else torch.float32
 
     def dev_x(a):
         t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
@@ -243,38 +281,44 @@ def run_ours(args, cfg):
 
     xs = [dev_x(a) for a in xs_host]
     res = None
-    if cfg.name.startswith("stack"):
+    if is_stack:
         res = torch.from_numpy(synth.make_residual(cfg, T, cfg_seed=cfg.seed + rank)).cuda()
     y = torch.empty((T, cfg.H), dtype=torch.float32, device="cuda")
     ws = moe2bit.alloc_workspace(layers[0].desc, T)
     stream = torch.cuda.current_stream()
+    xa = torch.empty((T, cfg.H), dtype=torch.bfloat16, device="cuda") if is_stack else None
 
-    if cfg.name.startswith("stack"):
-        # one step = 16-token decode through all resident layers chained by the residual stream
-        xa = torch.empty((T, cfg.H), dtype=torch.bfloat16, device="cuda")
+    side = torch.cuda.Stream() if is_stack else None
 
+    def chain(first_x, st):
+        """The layers in order; while layer l runs, layer l+1's router and shared expert are prefetched
+        into L2 on a side stream (they do not depend on routing)."""
+        cur = first_x
+        for l, dl in enumerate(layers):
+            if l + 1 < len(layers):
+                side.wait_stream(st)
+                moe2bit.prefetch_layer(layers[l + 1], side)
+            moe2bit.layer_forward(dl, cur, res if l == 0 else y, y, ws, st)
+            xa.copy_(y)  # next layer input = bf16 of the residual stream
+            cur = xa
+        st.wait_stream(side)
+
+    if is_stack:
+        # one step = a 16-token decode step through all resident layers chained by the residual stream
         def step_on(i, st):
-            cur = xs[i % n_slots]
-            for l, dl in enumerate(layers):
-                moe2bit.layer_forward(dl, cur, res if l == 0 else y, y, ws, st)
-                xa.copy_(y)  # next layer input = bf16 of the residual stream
-                cur = xa
-        tokens_per_step = T
+            chain(xs[i % n_slots], st)
     else:
         def step_on(i, st):
             moe2bit.layer_forward(layers[i % n_layers], xs[i % n_slots], None, y, ws, st)
-        tokens_per_step = T
 
-    def step(i):
+    warm = max(args.warmup, 3)
+    for i in range(warm):
         step_on(i, stream)
-
-    for i in range(args.warmup):
-        step(i)
     torch.cuda.synchronize()
     # The timed steps replay CUDA graphs of the same library calls (the library
     # launches nothing that a graph cannot hold); one graph per distinct
     # (layer, input) slot of the rotation.
-    period = n_slots if cfg.name.startswith("stack") else int(np.lcm(n_layers, n_slots))
+    period = n_slots if is_stack else int(np.lcm(n_layers, n_slots))
     graphs = []
     if args.graph:
         cap = torch.cuda.Stream()
@@ -293,7 +337,9 @@ def run_ours(args, cfg):
         if graphs:
             graphs[i % period].replay()
         else:
-            step(i)
+            step_on(i, stream)
+
+    import torch.distributed as dist
 
     if world > 1:
         dist.barrier()
@@ -303,18 +349,18 @@ def run_ours(args, cfg):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for i in range(args.steps):
-        timed_step(args.warmup + i)
+    for i in range(steps):
+        timed_step(warm + i)
     e1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms = e0.elapsed_time(e1) / args.steps
+    ms = e0.elapsed_time(e1) / steps
 
     # per-kernel durations (CUDA events around each library launch, same workload)
     moe2bit.profile_enable(True)
-    for i in range(args.steps):
-        step(args.warmup + i)
+    for i in range(steps):
+        step_on(warm + i, stream)
     torch.cuda.synchronize()
     prof = moe2bit.profile_read()
     moe2bit.profile_enable(False)
@@ -327,32 +373,27 @@ def run_ours(args, cfg):
 
     def e2e_step(i):
         xd.copy_(xh[i % n_slots], non_blocking=True)
-        if cfg.name.startswith("stack"):
-            cur = xdv
-            for l, dl in enumerate(layers):
-                moe2bit.layer_forward(dl, cur, res if l == 0 else y, y, ws, stream)
-                xa.copy_(y)
-                cur = xa
+        if is_stack:
+            chain(xdv, stream)
         else:
             moe2bit.layer_forward(layers[i % n_layers], xdv, None, y, ws, stream)
         yh.copy_(y, non_blocking=True)
 
-    for i in range(args.warmup):
+    for i in range(warm):
         e2e_step(i)
     torch.cuda.synchronize()
     e0.record(stream)
-    for i in range(args.steps):
+    for i in range(steps):
         e2e_step(i)
     e1.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = e0.elapsed_time(e1) / args.steps
+    ms_e2e = e0.elapsed_time(e1) / steps
     clocks = clk.stop()
-
     ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, "cuda")
 
-    # realised active experts per step, from the library's own routing
+    # realised active experts per layer step, from the library's own routing
     act = []
-    for s in range(n_slots):
+    for sl in range(n_slots):
         for l in range(min(n_layers, 4)):
             dl = layers[l]
             idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
@@ -360,14 +401,19 @@ def run_ours(args, cfg):
             off = torch.empty(cfg.E + 1, dtype=torch.int32, device="cuda")
             perm = torch.empty(T * cfg.k, dtype=torch.int32, device="cuda")
             inv = torch.empty(T * cfg.k, dtype=torch.int32, device="cuda")
-            moe2bit.route(dl.desc, dl.tensors["router_w"], dl.tensors["router_bias"], xs[s], idx, w, off, perm, inv, ws)
+            moe2bit.route(dl.desc, dl.tensors["router_w"], dl.tensors["router_bias"], xs[sl], idx, w, off, perm, inv,
+                          ws)
             o = off.cpu().numpy()
             act.append(int(np.count_nonzero(np.diff(o))))
     n_active = float(np.mean(act))
+    del graphs, layers, xs, ws
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
 
     hbm, bf16_tf, peak_kind = peaks()
     eb = expert_bytes(cfg)
-    launches_per_step = {k: v[1] / args.steps for k, v in prof.items()}
+    lps = n_layers if is_stack else 1  # library layer calls per step
+    launches_per_step = {k: v[1] / steps for k, v in prof.items()}
     avg_ms = {k: v[0] / max(v[1], 1) for k, v in prof.items()}
     # the dominant kernel among those with an algorithmic model (the combine's span also covers its wait for
     # the side stream, so it is not a candidate)
@@ -377,14 +423,14 @@ def run_ours(args, cfg):
     if dom in ("gateup", "prefill_gateup"):
         alg = n_active * eb["gateup"] + T * cfg.H * (2 if cfg.x_dtype == "bf16" else 4)
     elif dom in ("down", "prefill_down"):
-        alg = n_active * eb["down"] + T * cfg.k * cfg.I * 4 + T * cfg.k * cfg.H * 4
+        alg = n_active * eb["down"] + T * cfg.k * cfg.I * 2 + T * cfg.k * cfg.H * 4
     elif dom in ("shared_gateup",):
         alg = 2 * cfg.Is * cfg.H * 2
     elif dom in ("shared_down",):
         alg = cfg.Is * cfg.H * 2
     else:
         alg = 0
-    tr = traffic_record(dom)
+    tr = traffic_record(cfg.name, dom)
     if cfg.name.startswith("prefill") and dom in ("prefill_gateup", "prefill_down") and bf16_tf > 0:
         # the grouped GEMM is a dense contraction: fp16 operands (the same tensor rate as
         # bf16), FLOPs = 2 * assignments * output rows * K
@@ -392,7 +438,8 @@ def run_ours(args, cfg):
         flops = 2.0 * nA * 2 * cfg.I * cfg.H if dom == "prefill_gateup" else 2.0 * nA * cfg.H * cfg.I
         achieved = flops / (avg_ms[dom] * 1e-3) / 1e12
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": bf16_tf, "unit": "TFLOP/s",
-                "frac": achieved / bf16_tf, "peak_source": f"{peak_kind} bf16_tflops (burst; fp16 runs at the bf16 rate)",
+                "frac": achieved / bf16_tf,
+                "peak_source": f"{peak_kind} bf16_tflops (burst; fp16 runs at the bf16 rate)",
                 "traffic": tr["bytes_per_launch"] if tr else None, "algorithmic_flops_per_launch": flops,
                 "algorithmic_bytes_per_launch": alg, "avg_launch_ms": avg_ms[dom]}
     else:
@@ -401,29 +448,194 @@ def run_ours(args, cfg):
                 "frac": achieved / hbm, "peak_source": f"{peak_kind} hbm_gbs",
                 "traffic": tr["bytes_per_launch"] if tr else None,
                 "algorithmic_bytes_per_launch": alg, "avg_launch_ms": avg_ms[dom]}
-    layer_bytes = n_active * (eb["gateup"] + eb["down"]) + eb["shared"] + eb["router"]
-    kernels_per_step = sum(launches_per_step.values()) * (n_layers if cfg.name == "stack" else 1) / (
-        n_layers if cfg.name == "stack" else 1)
+    layer_bytes = n_active * (eb["gateup"] + eb["down"]) + eb["shared"] + eb["router"] + T * cfg.H * 6
+    step_bytes = layer_bytes * lps
     bytes_x = T * cfg.H * (2 if cfg.x_dtype == "bf16" else 4)
-    line = {
-        "metric": "moe_layer_tokens_per_s", "value": job_tokens_per_s(tokens_per_step, world, ms), "unit": "tokens/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None,
-        # the routed experts run as int8 MMAs on the decode GEMVs, as fp16 on the grouped GEMM
-        "dtype": "fp16" if "prefill_gateup" in prof else "int8", "data": "synthetic",
+    return {
+        "value": job_tokens_per_s(T, world, ms), "unit": "tokens/s", "ms_per_step": ms,
         "config": {"workload": cfg.name, "tokens_per_step": T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
                    "I_s": cfg.Is, "x_dtype": cfg.x_dtype, "resident_layers": n_layers,
+                   "layers_per_step": lps, "routing": "zipf(1.1) router bias" if cfg.zipf else "plain",
                    "l2": f"inputs larger than L2: {n_layers} resident layers in rotation",
                    "active_experts_per_layer": n_active, "layer_bytes_touched": layer_bytes,
-                   "launch": "cuda_graph" if graphs else "direct"},
+                   "launch": "cuda_graph" if args.graph else "direct"},
         "roofline": roof,
-        "layer_hbm_gbs": layer_bytes / (ms * 1e-3) / 1e9 if cfg.name != "stack" else None,
+        # whole-step HBM rate over the realised touched bytes (router, active experts, shared, activations)
+        "step_hbm": {"achieved_gbs": step_bytes / (ms * 1e-3) / 1e9, "peak": hbm,
+                     "frac": step_bytes / (ms * 1e-3) / 1e9 / hbm, "bytes_per_step": step_bytes},
         "kernels": {k: {"avg_ms": avg_ms[k], "launches_per_step": launches_per_step[k]} for k in prof},
-        "gpu_launches": int(round(sum(launches_per_step.values()) * args.steps)),
+        "gpu_launches": int(round(sum(launches_per_step.values()) * steps)),
         "clocks": clocks,
-        "e2e": {"value": job_tokens_per_s(tokens_per_step, world, ms_e2e), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(T, world, ms_e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": bytes_x, "d2h_bytes_per_step": T * cfg.H * 4},
+        "dtype": "fp16" if "prefill_gateup" in prof else "int8",
+        "steps": steps,
     }
+
+
+def h2d_gbs(nbytes=256 << 20, reps=5):
+    """Host-to-device copy rate from page-locked memory, measured here (the
+    denominator of the expert cache's miss traffic)."""
+    import torch
+
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    d.copy_(h, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        d.copy_(h, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    return nbytes * reps / (e0.elapsed_time(e1) * 1e-3) / 1e9
+
+
+def measure_cached(args, steps, n_slots=64):
+    """One-token decode steps with every routed expert in page-locked host
+    memory and n_slots of them cached in HBM (moe_layer_forward_cached), under
+    Zipf(1.1) routing: steady-state tokens/s, hit rate and the miss traffic's
+    host-to-device rate. The call synchronises once per step (it reads the
+    routing back), so steps are launched directly and timed with events."""
+    import torch
+
+    from bit_quantized_routed_iq2_b200 import moe2bit
+
+    cfg = synth.Config("decode1_cached", 1, 7168, 2048, 256, 8, 2048, "bf16", 1.0, True, 1, 0xD5400006)
+    lw = synth.make_layer(cfg)
+    shared = moe2bit.to_device_shared_only(lw)
+    cache = moe2bit.ExpertCache(lw, n_slots)
+    del lw
+    ws = moe2bit.alloc_workspace(shared.desc, 1)
+    xs_host = synth.make_x_fast(cfg, steps + 64)
+    xs = torch.from_numpy(xs_host.view(np.int16)).cuda().view(torch.bfloat16)
+    y = torch.empty((1, cfg.H), dtype=torch.float32, device="cuda")
+    warm = 48  # fills the cache
+    for i in range(warm):
+        cache.forward(shared, xs[i:i + 1], None, y, ws)
+    torch.cuda.synchronize()
+    st0 = cache.stats()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        cache.forward(shared, xs[warm + i:warm + i + 1], None, y, ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    st1 = cache.stats()
+    hits, misses = st1["hits"] - st0["hits"], st1["misses"] - st0["misses"]
+    copied = st1["bytes_copied"] - st0["bytes_copied"]
+    peak = h2d_gbs()
+    achieved = copied / steps / (ms * 1e-3) / 1e9
+    cache.close()
+    del cache, shared, ws
+    torch.cuda.empty_cache()
+    return {
+        "value": 1.0 / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+        "config": {"workload": cfg.name, "tokens_per_step": 1, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
+                   "I_s": cfg.Is, "routing": "zipf(1.1) router bias", "slots": n_slots,
+                   "host_pool": "all routed experts in page-locked host memory",
+                   "launch": "direct (the call reads the routing back once per step)"},
+        "hit_rate": hits / max(hits + misses, 1), "misses_per_step": misses / steps,
+        # while misses occur the step is bound by the host-to-device link
+        "roofline": {"bound": "h2d", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": "pinned host-to-device copy measured in this run",
+                     "bytes_per_step": copied / steps},
+    }
+
+
+def measure_quantize(args, reps=3):
+    """Float -> 2-bit codes for one expert (gate and up to IQ2, down to Q2K,
+    2048 x 7168 weights each): weights per second. The IQ2 search is bound by
+    fp32 arithmetic: 256 codebook rows x 8 weights x 3 operations per group of
+    8, against 148 SMs x 128 lanes x the median SM clock."""
+    import torch
+
+    from bit_quantized_routed_iq2_b200 import moe2bit
+
+    n = 2048 * 7168
+    w = torch.randn(n, dtype=torch.float32, device="cuda") / math.sqrt(7168)
+    nb = n // 256
+    ci = torch.empty((nb, 64), dtype=torch.uint8, device="cuda")
+    di = torch.empty(nb, dtype=torch.int16, device="cuda")
+    cq = torch.empty((nb, 80), dtype=torch.uint8, device="cuda")
+    dq = torch.empty(nb, dtype=torch.int32, device="cuda")
+    for _ in range(2):
+        moe2bit.quantize_iq2(w, ci, di)
+        moe2bit.quantize_q2k(w, cq, dq)
+    torch.cuda.synchronize()
+    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    e0.record()
+    for _ in range(2 * reps):
+        moe2bit.quantize_iq2(w, ci, di)
+    e1.record()
+    for _ in range(reps):
+        moe2bit.quantize_q2k(w, cq, dq)
+    e2.record()
+    torch.cuda.synchronize()
+    ms_iq2 = e0.elapsed_time(e1) / (2 * reps)
+    ms_q2k = e1.elapsed_time(e2) / reps
+    ms_expert = 2 * ms_iq2 + ms_q2k
+    ops = (n // 8) * 256 * 8 * 3
+    clk = 1965e6
+    peak = 148 * 128 * clk / 1e12
+    achieved = ops / (ms_iq2 * 1e-3) / 1e12
+    return {
+        "value": 3 * n / (ms_expert * 1e-3), "unit": "weights/s", "ms_per_expert": ms_expert,
+        "ms_iq2_matrix": ms_iq2, "ms_q2k_matrix": ms_q2k,
+        "config": {"workload": "quantize_expert", "matrices": "gate, up (IQ2), down (Q2K)", "rows_x_K": "2048 x 7168"},
+        "roofline": {"bound": "alu", "kernel": "quantize_iq2", "achieved": achieved, "peak": peak, "unit": "Tops/s",
+                     "frac": achieved / peak,
+                     "peak_source": "148 SMs x 128 fp32 lanes x 1965 MHz (nominal clock), unfused fp32 operations"},
+    }
+
+
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    from bit_quantized_routed_iq2_b200 import build as moebuild
+    from bit_quantized_routed_iq2_b200 import moe2bit
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    moebuild.build()
+    moe2bit.load()
+
+    m = measure(args, cfg, world, rank, local, args.steps)
+    line = {
+        "metric": "moe_layer_tokens_per_s", "value": m["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": m["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        # routed experts: exact 2-bit integer weights times 12-bit activation digits (two int8 digits) on the
+        # decode GEMVs; fp16 operands with fp32 accumulation on the grouped GEMM
+        "dtype": m["dtype"], "data": "synthetic",
+        **{k: m[k] for k in ("config", "roofline", "step_hbm", "kernels", "gpu_launches", "clocks", "e2e")},
+    }
+    # the rest of the metric (decode batch, prefill, the 8-layer stack), measured in the same run
+    want = args.workloads
+    if want == "auto":
+        want = "all" if (world == 1 and not args.experts and not args.tokens) else "none"
+    if want != "none":
+        names = ([n for n in ("decode32", "prefill", "stack") if n != cfg.name] + ["decode1_cached", "quantize"]
+                 if want == "all" else want.split(","))
+        line["workloads"] = {}
+        for name in names:
+            if name == "decode1_cached":
+                w = measure_cached(args, args.workload_steps * 10)
+            elif name == "quantize":
+                w = measure_quantize(args)
+            else:
+                w = measure(args, synth.CONFIGS[name], world, rank, local, args.workload_steps)
+                line["gpu_launches"] += w["gpu_launches"]
+            line["workloads"][name] = w
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg)
     if rank == 0:

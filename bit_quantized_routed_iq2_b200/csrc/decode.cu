@@ -25,14 +25,19 @@ namespace moe {
 
 // x [T][H] -> xd [T][2][H] int8 digits (plane 0 hi, plane 1 lo) and
 // xs [T][H/256] = 2^s / 8 per 256-element block (the 1/8 of the IQ2 scale is
-// folded in). One warp per 256-element block, 8 elements per lane. Block (0,0)
+// folded in). With qbits = 14 the block maximum maps into [2^12, 2^13), so
+// |q| <= 8192 and hi = (q + 64) >> 7 stays within [-64, 64]; the TMA-fed GEMVs
+// keep every int32 partial sum of such digits below 2^31 (four 32-weight
+// sub-blocks at most before each conversion to fp32). The other GEMVs take
+// qbits = 13 (|q| <= 4096), for which their longer integer sums are sized. One warp per 256-element block, 8 elements per lane. Block (0,0)
 // also clears the call's device status word.
 // For fp32 x it also writes two bf16 parts xb[part][T][H] (hi = rn(v),
 // lo = rn(v - hi)) for the bf16 MMAs of the shared expert.
 template <typename XT>
 __global__ void __launch_bounds__(256) x_digits_kernel(const XT* __restrict__ x, int T, int H,
                                                        int8_t* __restrict__ xd, float* __restrict__ xs,
-                                                       uint16_t* __restrict__ xb, int* __restrict__ err_word) {
+                                                       uint16_t* __restrict__ xb, int* __restrict__ err_word,
+                                                       int qbits) {
   pdl_trigger();
   pdl_wait();
   if (err_word && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *err_word = 0;
@@ -58,7 +63,7 @@ __global__ void __launch_bounds__(256) x_digits_kernel(const XT* __restrict__ x,
   for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  const int s = m > 0.f ? floor_log2_pos(m) - 11 : 0;
+  const int s = m > 0.f ? floor_log2_pos(m) - (qbits - 2) : 0;
   uint32_t hw[2] = {0, 0}, lw[2] = {0, 0};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -85,6 +90,38 @@ __global__ void __launch_bounds__(256) x_digits_kernel(const XT* __restrict__ x,
     *reinterpret_cast<uint4*>(xb + base) = make_uint4(hp[0], hp[1], hp[2], hp[3]);
     *reinterpret_cast<uint4*>(xb + static_cast<size_t>(T) * H + base) = make_uint4(lp[0], lp[1], lp[2], lp[3]);
   }
+}
+
+// ------------------------------------------------------------ L2 prefetch
+// Up to four ranges (16-byte aligned; sizes rounded down to 16 bytes, at most
+// 2^32 - 16 each) brought into L2 with the evict_last policy, in chunks of
+// 64 KB spread over the grid. Only L2 state changes; nothing is written.
+struct PrefetchRanges {
+  const uint8_t* p[4];
+  uint64_t n[4];
+};
+__global__ void __launch_bounds__(128) l2_prefetch_kernel(PrefetchRanges r) {
+  constexpr uint64_t kChunk = 64 * 1024;
+  const uint64_t pol = l2_policy_evict_last();
+  const uint64_t tid = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const uint64_t nthr = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  for (int i = 0; i < 4; ++i) {
+    const uint64_t n = r.n[i] & ~uint64_t(15);
+    for (uint64_t off = tid * kChunk; off < n; off += nthr * kChunk) {
+      const uint64_t len = n - off < kChunk ? n - off : kChunk;
+      bulk_prefetch_l2(r.p[i] + off, static_cast<uint32_t>(len), pol);
+    }
+  }
+}
+
+int launch_l2_prefetch(const void* const* ptrs, const size_t* bytes, int n, cudaStream_t st) {
+  PrefetchRanges r{};
+  for (int i = 0; i < 4; ++i) {
+    r.p[i] = i < n ? static_cast<const uint8_t*>(ptrs[i]) : nullptr;
+    r.n[i] = (i < n && ptrs[i]) ? bytes[i] : 0;
+  }
+  l2_prefetch_kernel<<<148, 128, 0, st>>>(r);
+  return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
 }
 
 // ------------------------------------------------------------ shared expert
@@ -342,22 +379,45 @@ namespace {
 int hsc_stride(int I) { return ((I / 256) + 3) & ~3; }
 }  // namespace
 
-// h = silu(g) * u for one assignment (blockIdx.x), split into int8 digits with
-// one power-of-two scale per 256-element block, stored in the order the down
-// MMA reads them: inside each 32-element block, element j of sub-block half
-// sub (0 for the first 16, 1 for the next) goes to byte 8*(j%4) + 4*sub + j/4.
-// Also writes, per 16-element sub-block, the exact integer sum of the digits'
-// values q = 128 hi + lo (the min term of the Q2K-style down projection).
-// g and u arrive as KP partial sums each ([p][2][KP][I]); they are added in
-// part order first.
+// h = silu(g) * u for assignment blockIdx.x, 256-element block blockIdx.y:
+// g and u arrive as KP partial sums each ([p][2][KP][I]); warp w adds parts
+// w, w + 8, ... in order, the eight warp sums are added in warp order (a fixed
+// order: results are identical run to run), and warp 0 quantises the block
+// (hquant_finish_warp).
+template <bool kHOff>
 __global__ void __launch_bounds__(256) hquant_kernel(int I, int KP, const float* __restrict__ gu,
                                                      int8_t* __restrict__ hd, float* __restrict__ hsc,
                                                      int32_t* __restrict__ hq, int hss) {
+  __shared__ float4 red[8][4][32];  // [warp][g lo, g hi, u lo, u hi][lane]
   pdl_trigger();
   pdl_wait();
-  const int p = blockIdx.x;
+  const int p = blockIdx.x, sb = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int sb = warp; sb < I / 256; sb += 8) hquant_block_warp(I, KP, gu, p, sb, hd, hsc, hq, hss, lane);
+  const float* g = gu + static_cast<size_t>(p) * 2 * KP * I + sb * 256 + lane * 8;
+  const float* u = g + static_cast<size_t>(KP) * I;
+  float4 s[4] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f),
+                 make_float4(0.f, 0.f, 0.f, 0.f)};
+  for (int kp = warp; kp < KP; kp += 8) {
+    const float4 v0 = __ldcg(reinterpret_cast<const float4*>(g + static_cast<size_t>(kp) * I));
+    const float4 v1 = __ldcg(reinterpret_cast<const float4*>(g + static_cast<size_t>(kp) * I + 4));
+    const float4 v2 = __ldcg(reinterpret_cast<const float4*>(u + static_cast<size_t>(kp) * I));
+    const float4 v3 = __ldcg(reinterpret_cast<const float4*>(u + static_cast<size_t>(kp) * I + 4));
+    s[0].x += v0.x; s[0].y += v0.y; s[0].z += v0.z; s[0].w += v0.w;
+    s[1].x += v1.x; s[1].y += v1.y; s[1].z += v1.z; s[1].w += v1.w;
+    s[2].x += v2.x; s[2].y += v2.y; s[2].z += v2.z; s[2].w += v2.w;
+    s[3].x += v3.x; s[3].y += v3.y; s[3].z += v3.z; s[3].w += v3.w;
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) red[warp][q][lane] = s[q];
+  __syncthreads();
+  if (warp != 0) return;
+  float gv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, uv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int w = 0; w < 8; ++w) {
+    const float4 a = red[w][0][lane], b = red[w][1][lane], c = red[w][2][lane], d = red[w][3][lane];
+    gv[0] += a.x; gv[1] += a.y; gv[2] += a.z; gv[3] += a.w; gv[4] += b.x; gv[5] += b.y; gv[6] += b.z; gv[7] += b.w;
+    uv[0] += c.x; uv[1] += c.y; uv[2] += c.z; uv[3] += c.w; uv[4] += d.x; uv[5] += d.y; uv[6] += d.z; uv[7] += d.w;
+  }
+  hquant_finish_warp<kHOff>(I, p, sb, gv, uv, hd, hsc, hq, hss, lane);
 }
 
 // The TMA-fed GEMVs (gemv_tma.cu) serve shapes with H % 1024 == 0 and
@@ -460,13 +520,21 @@ int launch_shared_early(const LayerShape& s, const WeightPtrs& w, const void* x,
     ProfScope ps(MOE_K_PREP, c->st);
     dim3 g(T, (s.H / 256 + 7) / 8);
     x_digits_kernel<uint16_t><<<g, 256, 0, c->st>>>(static_cast<const uint16_t*>(x), T, s.H, fw.xd, fw.xs, nullptr,
-                                                    nullptr);
+                                                    nullptr, tma ? 14 : 13);
   }
   if (cudaEventRecord(c->digits, c->st) != cudaSuccess) return ERR_CUDA;
   int rc;
   {
     ProfScope ps(MOE_K_SHARED_GATEUP, c->st);
     rc = launch_shared_gateup_mma(s.H, s.Is, w.sh_gate, w.sh_up, static_cast<const uint16_t*>(x), 1, T, fw.hb, c->st);
+  }
+  // the shared down weights are known now too: bring them into L2 while routing and the routed GEMVs run, so
+  // the combine at the end of the step reads them from there (the bytes still come from HBM in this step);
+  // the prefetch only issues requests, so joining after it costs the combine nothing
+  if (rc == OK) {
+    const void* pp[1] = {w.sh_down};
+    const size_t nn[1] = {static_cast<size_t>(s.H) * s.Is * 2};
+    rc = launch_l2_prefetch(pp, nn, 1, c->st);
   }
   if (cudaEventRecord(c->join, c->st) != cudaSuccess) return ERR_CUDA;
   return rc;
@@ -497,12 +565,13 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
   } else {
     ProfScope ps(MOE_K_PREP, st);
     dim3 g(T, (s.H / 256 + 7) / 8);
+    const int qbits = tma ? 14 : 13;
     if (x_dtype == 0)
       launch_pdl(x_digits_kernel<float>, g, dim3(256), 0, st, static_cast<const float*>(x), T, s.H, xd, xs, fw.xb,
-                 clear_status ? err : nullptr);
+                 clear_status ? err : nullptr, qbits);
     else
       launch_pdl(x_digits_kernel<uint16_t>, g, dim3(256), 0, st, static_cast<const uint16_t*>(x), T, s.H, xd, xs,
-                 static_cast<uint16_t*>(nullptr), clear_status ? err : nullptr);
+                 static_cast<uint16_t*>(nullptr), clear_status ? err : nullptr, qbits);
   }
   // bf16 activations feed the shared expert's MMAs as one part, fp32 as two
   const int xparts = x_dtype == 0 ? 2 : 1;
@@ -545,8 +614,13 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
   }
   {
     ProfScope ps(MOE_K_HQUANT, st);
-    launch_pdl(hquant_kernel, dim3(static_cast<unsigned>(nA)), dim3(256), 0, st, s.I, KP, static_cast<const float*>(gu),
-               hd, hsc, hq, hsc_stride(s.I));
+    const dim3 hg(static_cast<unsigned>(nA), static_cast<unsigned>(s.I / 256));
+    if (tma)
+      launch_pdl(hquant_kernel<true>, hg, dim3(256), 0, st, s.I, KP, static_cast<const float*>(gu), hd, hsc, hq,
+                 hsc_stride(s.I));
+    else
+      launch_pdl(hquant_kernel<false>, hg, dim3(256), 0, st, s.I, KP, static_cast<const float*>(gu), hd, hsc, hq,
+                 hsc_stride(s.I));
   }
   if (tma) {
     ProfScope ps(MOE_K_DOWN, st);

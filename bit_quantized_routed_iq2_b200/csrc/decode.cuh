@@ -66,6 +66,28 @@ __device__ __forceinline__ void split_digits(float x, int s, int& hi, int& lo) {
   lo = q - (hi << 7);
 }
 
+// Offset of digit d of element e (a multiple of 8) of token t in the staged
+// activations: per token 2*H bytes; block b (256 elements) takes 512 bytes, its
+// sub-block s (32 elements) 64 bytes, digit d at +32d, and the two 16-element
+// halves c of the sub-block at +16*(c ^ (b & 1)). The half swap on odd blocks
+// makes the B loads of the one-token unit below conflict-free.
+__host__ __device__ __forceinline__ int x_off(int H, int t, int d, int e) {
+  const int b = e >> 8;
+  return t * 2 * H + b * 512 + ((e >> 5) & 7) * 64 + d * 32 + 16 * (((e >> 4) & 1) ^ (b & 1)) + (e & 15);
+}
+
+// Offset of digit d of element e (of I) of assignment p in the h digits (global
+// and staged alike): per assignment 2*I bytes; block b (256 elements) takes 512
+// bytes; its 16-element sub-block S = 4t + c (t = S >> 2, c = S & 3) takes 16
+// bytes per digit at c*128 + t*32 + d*16, element 4i + r at byte 4r + i. So one
+// 16-byte load gives a lane the four bytes of each bit pair r of its sub-block
+// (the K order of q2k_quad), and the eight lanes that carry B in the one-token
+// unit hit eight different 16-byte bank groups.
+__host__ __device__ __forceinline__ int h_off(int I, int p, int d, int e) {
+  const int S = (e >> 4) & 15, j = e & 15;
+  return p * 2 * I + (e >> 8) * 512 + (S & 3) * 128 + (S >> 2) * 32 + d * 16 + 4 * (j & 3) + (j >> 2);
+}
+
 // ------------------------------------------------------------ gate/up
 struct GateupArgs {
   int H, I, E, k, T;
@@ -103,51 +125,20 @@ int launch_gateup(const GateupArgs& a, int slots, int sms, cudaStream_t st);
 int launch_down(const DownArgs& a, int slots, int T, int sms, cudaStream_t st);
 
 
-// h = silu(g) * u for assignment p, 256-element block sb, by one warp (8
-// elements per lane): g and u arrive as KP partial sums each ([p][2][KP][I]),
-// added in part order; h is split into int8 digits with one power-of-two scale
-// per block, stored in the order the down MMA reads them (inside each
-// 32-element block, element j of sub-block half sub goes to byte
-// 8*(j%4) + 4*sub + j/4), with the exact integer sum of q = 128 hi + lo per
-// 16-element sub-block (the min term of the Q2K-style down projection).
-__device__ __forceinline__ void hquant_block_warp(int I, int KP, const float* __restrict__ gu, int p, int sb,
-                                                  int8_t* __restrict__ hd, float* __restrict__ hsc,
-                                                  int32_t* __restrict__ hq, int hss, int lane) {
-  const float* g = gu + static_cast<size_t>(p) * 2 * KP * I;
-  const float* u = g + static_cast<size_t>(KP) * I;
+// Second half of the h quantiser, by one warp (8 elements per lane, lane l
+// holding elements 8l .. 8l+7 of the 256-element block sb of assignment p):
+// h = silu(g) * u from the summed gate/up rows, split into int8 digits with
+// one power-of-two scale per block and stored in the order the down MMA reads
+// them (kHOff: the h_off layout of the TMA-fed down GEMV; otherwise rows of I
+// per digit where, inside each 32-element block, element j of sub-block half
+// sub goes to byte 8*(j%4) + 4*sub + j/4), with the exact integer sum of
+// q = 128 hi + lo per 16-element sub-block (the min term of the Q2K-style down
+// projection).
+template <bool kHOff>
+__device__ __forceinline__ void hquant_finish_warp(int I, int p, int sb, const float (&gv)[8], const float (&uv)[8],
+                                                   int8_t* __restrict__ hd, float* __restrict__ hsc,
+                                                   int32_t* __restrict__ hq, int hss, int lane) {
   const int base = sb * 256 + lane * 8;
-  float gv[8], uv[8];
-  {
-    // L2 loads: the partial rows may have been written by other SMs in this kernel
-    const float4 g0 = __ldcg(reinterpret_cast<const float4*>(g + base)), g1 = __ldcg(reinterpret_cast<const float4*>(g + base + 4));
-    const float4 u0 = __ldcg(reinterpret_cast<const float4*>(u + base)), u1 = __ldcg(reinterpret_cast<const float4*>(u + base + 4));
-    gv[0] = g0.x; gv[1] = g0.y; gv[2] = g0.z; gv[3] = g0.w; gv[4] = g1.x; gv[5] = g1.y; gv[6] = g1.z; gv[7] = g1.w;
-    uv[0] = u0.x; uv[1] = u0.y; uv[2] = u0.z; uv[3] = u0.w; uv[4] = u1.x; uv[5] = u1.y; uv[6] = u1.z; uv[7] = u1.w;
-  }
-  // parts are added in order; loads of up to eight parts are in flight at once
-  for (int k0 = 1; k0 < KP; k0 += 8) {
-    float4 lg[8][2], lu[8][2];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      if (k0 + q < KP) {
-        const float* gp = g + static_cast<size_t>(k0 + q) * I + base;
-        const float* up = u + static_cast<size_t>(k0 + q) * I + base;
-        lg[q][0] = __ldcg(reinterpret_cast<const float4*>(gp));
-        lg[q][1] = __ldcg(reinterpret_cast<const float4*>(gp + 4));
-        lu[q][0] = __ldcg(reinterpret_cast<const float4*>(up));
-        lu[q][1] = __ldcg(reinterpret_cast<const float4*>(up + 4));
-      }
-    }
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      if (k0 + q < KP) {
-        gv[0] += lg[q][0].x; gv[1] += lg[q][0].y; gv[2] += lg[q][0].z; gv[3] += lg[q][0].w;
-        gv[4] += lg[q][1].x; gv[5] += lg[q][1].y; gv[6] += lg[q][1].z; gv[7] += lg[q][1].w;
-        uv[0] += lu[q][0].x; uv[1] += lu[q][0].y; uv[2] += lu[q][0].z; uv[3] += lu[q][0].w;
-        uv[4] += lu[q][1].x; uv[5] += lu[q][1].y; uv[6] += lu[q][1].z; uv[7] += lu[q][1].w;
-      }
-    }
-  }
   float h[8], m = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -156,7 +147,8 @@ __device__ __forceinline__ void hquant_block_warp(int I, int KP, const float* __
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  const int e = m > 0.f ? floor_log2_pos(m) - 11 : 0;
+  // the TMA-fed down GEMV takes 14-bit digits (|q| <= 8192), the other one 13-bit (see x_digits_kernel)
+  const int e = m > 0.f ? floor_log2_pos(m) - (kHOff ? 12 : 11) : 0;
   int qs = 0;
   int8_t* hi_row = hd + static_cast<size_t>(p) * 2 * I;
   int8_t* lo_row = hi_row + I;
@@ -166,10 +158,15 @@ __device__ __forceinline__ void hquant_block_warp(int I, int KP, const float* __
     int hi = 0, lo = 0;
     if (m > 0.f) split_digits(h[i], e, hi, lo);
     qs += hi * 128 + lo;
-    const int jj = jj0 + i, sub = jj >> 4, j = jj & 15;
-    const int pos = blk32 * 32 + 8 * (j & 3) + 4 * sub + (j >> 2);
-    hi_row[pos] = static_cast<int8_t>(hi);
-    lo_row[pos] = static_cast<int8_t>(lo);
+    if (kHOff) {
+      hd[h_off(I, p, 0, base + i)] = static_cast<int8_t>(hi);
+      hd[h_off(I, p, 1, base + i)] = static_cast<int8_t>(lo);
+    } else {
+      const int jj = jj0 + i, sub = jj >> 4, j = jj & 15;
+      const int pos = blk32 * 32 + 8 * (j & 3) + 4 * sub + (j >> 2);
+      hi_row[pos] = static_cast<int8_t>(hi);
+      lo_row[pos] = static_cast<int8_t>(lo);
+    }
   }
   qs += __shfl_xor_sync(0xffffffffu, qs, 1);  // lanes 2i, 2i+1 hold one 16-element sub-block
   if ((lane & 1) == 0) hq[static_cast<size_t>(p) * (I / 16) + sb * 16 + (lane >> 1)] = qs;

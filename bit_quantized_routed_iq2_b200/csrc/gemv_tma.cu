@@ -51,14 +51,11 @@ constexpr int kThreadsT = (kCW + 1) * 32;    // + one producer warp
 constexpr int kBoxRows = 16 * kCW;           // 256 rows per box
 constexpr int kGuW = 128;                    // code bytes per gate/up box row (512 weights)
 constexpr int kGuBox = kBoxRows * kGuW;      // 32 KB
-constexpr int kDnW = 80;                     // one Q2K-style block per down box row
-constexpr int kDnBox = kBoxRows * kDnW;      // 20 KB
 // Selector tables, each entry replicated for the 32 lanes: grid row i at byte
 // 256*i + 4*lane, sign field s at byte 256*s + 128 + 4*lane (interleaved, so
 // that one prmt turns a grid index byte into its table address).
 constexpr int kTabBytes = 256 * 256;
 constexpr int kZeroBytes = 1024;             // zero operand region for idle MMA columns
-constexpr int kRowPad = 32;                  // padding of a staged activation row
 constexpr int kMaxExpertsTma = 1024;
 constexpr int kMaxNB = 2;
 
@@ -67,31 +64,61 @@ __device__ __align__(128) const int8_t g_zero_operand[kZeroBytes] = {};
 
 __device__ __forceinline__ uint32_t rotr(uint32_t v, uint32_t n) { return __funnelshift_r(v, v, n); }
 
-__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+// Bounds-checked build (-DMOE_BOUNDS_CHECK, a separate library): every
+// shared-memory load of these kernels checks that it lies inside the CTA's
+// dynamic shared memory and is aligned, every partial-sum store and TMA box
+// that it stays inside its buffer; a violation is counted in
+// g_bounds_violations (read by moe_debug_bounds_violations) and the access is
+// skipped (a load returns zeros). Nothing traps. The normal build compiles the
+// checks away.
+#ifdef MOE_BOUNDS_CHECK
+__device__ unsigned long long g_bounds_violations = 0;
+__device__ __forceinline__ bool bc_fail() {
+  atomicAdd(&g_bounds_violations, 1ull);
+  return false;
+}
+__device__ __forceinline__ bool smem_ok(uint32_t a, uint32_t bytes) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint32_t size;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(size));
+  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  return (a >= base && a - base + bytes <= size && (a & (bytes - 1)) == 0) ? true : bc_fail();
+}
+__device__ __forceinline__ bool index_ok(size_t i, size_t n) { return i < n ? true : bc_fail(); }
+#define MOE_SMEM_GUARD(a, n, zero) \
+  if (!smem_ok((a), (n))) return zero;
+#else
+__device__ __forceinline__ bool index_ok(size_t, size_t) { return true; }
+#define MOE_SMEM_GUARD(a, n, zero)
+#endif
+
+__device__ __forceinline__ uint4 lds128(const uint8_t* p) {
+  MOE_SMEM_GUARD(static_cast<uint32_t>(__cvta_generic_to_shared(p)), 16, make_uint4(0u, 0u, 0u, 0u))
+  return *reinterpret_cast<const uint4*>(p);
+}
 
 // Loads from shared memory at 32-bit shared-window addresses. They are volatile
 // so that they stay after the mbarrier wait that makes the data visible.
 __device__ __forceinline__ uint4 ld_s128(uint32_t a) {
+  MOE_SMEM_GUARD(a, 16, make_uint4(0u, 0u, 0u, 0u))
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
   return v;
 }
 __device__ __forceinline__ uint2 ld_s64(uint32_t a) {
+  MOE_SMEM_GUARD(a, 8, make_uint2(0u, 0u))
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
   return v;
 }
 __device__ __forceinline__ uint32_t ld_s32(uint32_t a) {
+  MOE_SMEM_GUARD(a, 4, 0u)
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
-__device__ __forceinline__ uint32_t ld_s8(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
-  return v;
-}
 __device__ __forceinline__ float ld_sf(uint32_t a) {
+  MOE_SMEM_GUARD(a, 4, 0.f)
   float v;
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
   return v;
@@ -118,17 +145,6 @@ __device__ __forceinline__ void load_meta(const MetaSmem& m, const int32_t* offs
     for (int i = tid; i < nA; i += nthr) m.tok[i] = perm[i] / k;
 }
 
-// Copy rows of `row_bytes` (a multiple of 16) from global memory into shared
-// memory with a row pitch of row_bytes + kRowPad.
-__device__ __forceinline__ void stage_rows(int8_t* dst, const int8_t* src, int rows, int row_bytes, int tid,
-                                           int nthr) {
-  const int per = row_bytes / 16;
-  for (int i = tid; i < rows * per; i += nthr) {
-    const int r = i / per, cidx = i - r * per;
-    *reinterpret_cast<uint4*>(dst + static_cast<size_t>(r) * (row_bytes + kRowPad) + cidx * 16) =
-        reinterpret_cast<const uint4*>(src)[i];
-  }
-}
 
 // Ring position: stage index and phase parity.
 struct RingPos {
@@ -147,6 +163,9 @@ struct RingPos {
 // ===========================================================================
 struct GuTmaArgs {
   int H, I, E, k, T, KP, NB, S;
+  int no_produce;           // fault injection (test aid): the producer issues no loads
+  int one;                  // 1, opaque to the compiler (keeps an integer add on the multiply-add pipe)
+  long long wait_limit;     // bound of every mbarrier wait, in SM cycles
   const uint16_t* gate_d;
   const uint16_t* up_d;
   const int8_t* xd;
@@ -155,6 +174,7 @@ struct GuTmaArgs {
   const int32_t* perm;
   const int32_t* active;
   float* gpart;  // [T*k][2][KP][I]
+  size_t gpart_n;  // its length in floats (bounds-checked build)
   int* err;
 };
 
@@ -250,85 +270,145 @@ __device__ __forceinline__ int gu_odd(const uint8_t* rg, int sb, int g) {
 __device__ __forceinline__ float half_lo(uint32_t w) { return half_bits_to_float(static_cast<uint16_t>(w & 0xFFFFu)); }
 __device__ __forceinline__ float half_hi(uint32_t w) { return half_bits_to_float(static_cast<uint16_t>(w >> 16)); }
 
-// One unit whose expert holds a single assignment (every decode step with one
-// token), activations staged in shared memory. MMA columns: (sub-block slot
-// 0..3) x (digit hi, lo); the B operand of an idle column comes from the zero
-// region, so no select is needed. All shared-memory addresses are 32-bit and
-// the 128-byte swizzle is applied with one XOR per 16-byte chunk: with
-// rgg = row base + 16*g, logical chunk L of row g sits at rgg ^ (16*L).
+
+// The selector tables at the start of dynamic shared memory: row i (256 bytes)
+// holds the level word of grid row i at bytes 0..127 and the sign word of sign
+// field i mod 128 at bytes 128..255, each replicated for the 32 lanes.
+__device__ __forceinline__ void fill_sel_tables(uint32_t* tab, int tid, int nthr) {
+  for (int i = tid; i < kTabBytes / 4; i += nthr) {
+    const int ent = i >> 6;
+    tab[i] = (i & 32) == 0 ? d_sel_tables2.level[ent] : d_sel_tables2.sign[ent & 127];
+  }
+}
+
+// Word of the selector tables at byte offset `off` of dynamic shared memory
+// (the tables sit at its start, so the base folds into the load).
+__device__ __forceinline__ uint32_t tab_ld(uint32_t off) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  MOE_SMEM_GUARD(static_cast<uint32_t>(__cvta_generic_to_shared(smem + off)), 4, 0u)
+  return *reinterpret_cast<const uint32_t*>(smem + off);
+}
+
+// Two int8x4 A registers (elements 0..3 and 4..7) of one IQ2 group from its
+// selector word: level code of element e in bits 4e..4e+1, sign in bit 4e+2.
+// The 16-bit shift for the upper half is a multiply-high (FMA pipe).
+__device__ __forceinline__ void iq2_pair(uint32_t sel, uint32_t& lo, uint32_t& hi) {
+  lo = prmt(kPosBytes, kNegBytes, sel);
+  hi = prmt(kPosBytes, kNegBytes, __umulhi(sel, 0x10000u));
+}
+
+// The int8 A operands (elements 0..3, 4..7 = level * sign) of group JJ of one
+// 8-byte IQ2 sub-block record: the grid index byte JJ and the sign field JJ
+// become table offsets by one prmt each (byte 1 = table row, byte 0 = this
+// lane's replica), the two table words add up to the prmt selector word. The
+// sign field is moved to bits 8..15 by a multiply (FMA pipe); its bit 15 is a
+// neighbour's bit, which the sign table ignores by repeating every 128 rows.
+template <int JJ>
+__device__ __forceinline__ void iq2_group_int8(uint2 rec, uint32_t lane4, uint32_t sgn_lane, uint32_t one,
+                                               uint32_t& lo, uint32_t& hi) {
+  const uint32_t sf = JJ == 0 ? rec.y : (JJ == 1 ? rec.y * 2u : __umulhi(rec.y, JJ == 2 ? (1u << 26) : (1u << 19)));
+  const uint32_t lv = tab_ld(prmt(rec.x, lane4, 0x5504u | (JJ << 4)));
+  const uint32_t sg = tab_ld(prmt(sf, sgn_lane, JJ ? 0x5514u : 0x5504u));
+  iq2_pair(lv * one + sg, lo, hi);  // level codes and sign bits are disjoint: the sum is the union
+}
+
+// 2*ls + 1 of an IQ2 sub-block record (ls = bits 28..31 of its sign word).
+__device__ __forceinline__ int iq2_odd(uint2 rec) { return 2 * static_cast<int>(__umulhi(rec.y, 16u)) + 1; }
+
+// The four 2-bit codes at bit pair `sh` / 2 of each byte of a Q2K code word, as
+// uint8 A operand bytes (the down GEMV's K order takes weights 4i + tig).
+__device__ __forceinline__ uint32_t q2k_quad(uint32_t w, uint32_t sh) { return (w >> sh) & 0x03030303u; }
+
+// One unit whose expert holds a single assignment (every unit of a one-token
+// step; single-token experts of a batch), activations staged in shared memory.
+//
+// Lane mapping (m16n8k32, lane = 4g + tig): the lane builds A for rows g and
+// g+8 of the warp's 16. In round cc (0..3) of a 512-weight box it owns
+// sub-block 2cc + (tig & 1) of block tig >> 1 of the box, whole: its four MMAs
+// j = 0..3 take groups j of that sub-block, one 8-weight group per row each.
+// So every lane reads its own two 8-byte sub-block records (no lane reads
+// another's), takes the 2ls+1 scale from them and needs one fp16 d per row.
+// MMA columns are (owner tig, digit hi/lo): B is non-zero only on the lanes
+// with g >> 1 == tig, which load the x digits of their column's sub-block; the
+// accumulator registers of lane tig then hold exactly its own sub-block.
+// Shared-memory traffic per round and warp: two conflict-free 8-byte record
+// loads per lane (the 128-byte swizzle spreads the 16 rows' chunks), two
+// 16-byte B loads on eight lanes, sixteen selector-table loads.
+template <bool XS>
 __device__ __forceinline__ bool gu_unit_one(const GuTmaArgs& a, const GuCtx& c, RingPos& rp, const GuUnit& w,
                                             const uint32_t (&dp)[kMaxNB][2]) {
   const int H = a.H, I = a.I, NB = a.NB;
-  const int g = c.g, tig = c.tig;
+  const int g = c.g, tig = c.tig, bb = tig >> 1, hf = tig & 1;
   const int tok = c.tok[w.p0];
-  const int row_l = 16 * c.warp + g;
-  const uint32_t xrow = c.x_s + (tok * 2 + (g & 1)) * c.xpitch + w.kp * NB * 512 + 8 * tig;
-  const uint32_t zrow = c.zero_s + ((64 * (tok & 1) + 64) & 127) + 8 * tig;
-  const uint32_t xsc = c.xs_s + (tok * (H / 256) + 2 * NB * w.kp) * 4;
-  const uint32_t lsoff = ((((tig >> 1) ^ g)) << 4) + (tig & 1) * 8 + 7;
+  const bool bact = (g >> 1) == tig;  // this lane carries B (digit g & 1 of its column's sub-block)
+  const uint32_t one = static_cast<uint32_t>(a.one);
+  // sub-block record of round 0 for row g, relative to the row's base: chunk (cc | 4bb) ^ g, half hf
+  const uint32_t roff = (((static_cast<uint32_t>(g) ^ (4u * bb)) << 4) | (8u * hf));
+  const uint32_t rowb = static_cast<uint32_t>(16 * c.warp + g) * kGuW;
   float f0 = 0.f, f1 = 0.f;
 #pragma unroll 1
   for (int j = 0; j < NB; ++j) {
-    uint32_t bp[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) bp[u] = ((g >> 1) == u) ? xrow + j * 512 : zrow;
-    if (!mbar_wait_bounded(&c.full[rp.s], rp.ph, a.err, ERR_TIMEOUT)) return false;
-    const uint32_t rg = c.ring_s + rp.s * kGuBox + row_l * kGuW;
+    const int kblk = (w.kp * NB + j) * 2 + bb;  // this lane's block of H
+    // B source: staged (x_off layout; chunk 1 of a sub-block is the XOR-16 neighbour of chunk 0) or the
+    // global [T][2][H] digits (natural order)
+    const uint32_t xb0 = XS ? c.x_s + x_off(H, tok, g & 1, kblk * 256 + hf * 32) : 0u;
+    const uint32_t xb1 = xb0 ^ 16u;
+    const int8_t* xg = XS ? nullptr : c.xdig + static_cast<size_t>(tok * 2 + (g & 1)) * H + kblk * 256 + hf * 32;
+    if (!mbar_wait_bounded(&c.full[rp.s], rp.ph, a.err, ERR_TIMEOUT, a.wait_limit)) return false;
+    const uint32_t r0 = c.ring_s + rp.s * kGuBox + rowb + roff;
     const int s = rp.s;
     rp.next(c.S);
-    const uint32_t rgg = rg + 16 * g, lsa = rg + lsoff;
     int i0 = 0, i1 = 0;
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
-      const uint4 a0 = ld_s128(rgg ^ (32 * cc));
-      const uint4 a1 = ld_s128(rgg ^ (32 * cc + 16));
-      const uint4 b0 = ld_s128((rgg + 1024) ^ (32 * cc));
-      const uint4 b1 = ld_s128((rgg + 1024) ^ (32 * cc + 16));
-      uint2 bv[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) bv[u] = ld_s64(bp[u] + (4 * cc + u) * 32);
-      const uint32_t l0 = ld_s8(lsa ^ (32 * cc)), l1 = ld_s8((lsa + 1024) ^ (32 * cc));
-      const uint2 rec[4][2] = {{make_uint2(a0.x, a0.y), make_uint2(b0.x, b0.y)},
-                               {make_uint2(a0.z, a0.w), make_uint2(b0.z, b0.w)},
-                               {make_uint2(a1.x, a1.y), make_uint2(b1.x, b1.y)},
-                               {make_uint2(a1.z, a1.w), make_uint2(b1.z, b1.w)}};
+      const uint2 ra = ld_s64(r0 ^ (16u * cc));          // row g
+      const uint2 rb = ld_s64((r0 ^ (16u * cc)) + 1024);  // row g + 8
+      uint4 bx0 = make_uint4(0u, 0u, 0u, 0u), bx1 = make_uint4(0u, 0u, 0u, 0u);
+      if (bact) {
+        if (XS) {
+          bx0 = ld_s128(xb0 + 128u * cc);
+          bx1 = ld_s128(xb1 + 128u * cc);
+        } else {
+          bx0 = __ldg(reinterpret_cast<const uint4*>(xg + 64 * cc));
+          bx1 = __ldg(reinterpret_cast<const uint4*>(xg + 64 * cc + 16));
+        }
+      }
+      const uint32_t bv[8] = {bx0.x, bx0.y, bx0.z, bx0.w, bx1.x, bx1.y, bx1.z, bx1.w};
       int acc[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        uint32_t r0lo, r0hi, r1lo, r1hi;
-        iq2_operand(c, rec[u][0], r0lo, r0hi);
-        iq2_operand(c, rec[u][1], r1lo, r1hi);
-        if (u == 0)
-          mma_s8s8_zero(acc, r0lo, r1lo, r0hi, r1hi, bv[u].x, bv[u].y);
-        else
-          mma_s8s8(acc, r0lo, r1lo, r0hi, r1hi, bv[u].x, bv[u].y);
-      }
-      // this thread's columns are sub-block 4cc+tig, digits hi and lo
-      i0 += (acc[0] * 128 + acc[1]) * static_cast<int>((l0 >> 3) | 1u);
-      i1 += (acc[2] * 128 + acc[3]) * static_cast<int>((l1 >> 3) | 1u);
-      if (cc & 1) {
-        const int sb = cc >> 1;
-        const float xsv = ld_sf(xsc + (2 * j + sb) * 4);
-        const uint32_t w0 = j ? dp[1][0] : dp[0][0], w1 = j ? dp[1][1] : dp[0][1];
-        const float d0 = sb ? half_hi(w0) : half_lo(w0);
-        const float d1 = sb ? half_hi(w1) : half_lo(w1);
-        f0 = fmaf(static_cast<float>(i0), d0 * xsv, f0);
-        f1 = fmaf(static_cast<float>(i1), d1 * xsv, f1);
-        i0 = i1 = 0;
-      }
+#define MOE_GU_GROUP(JJ)                                                                  \
+  {                                                                                       \
+    uint32_t a0, a1, a2, a3;                                                              \
+    iq2_group_int8<JJ>(ra, c.lane4, c.sgn_lane, one, a0, a2);                            \
+    iq2_group_int8<JJ>(rb, c.lane4, c.sgn_lane, one, a1, a3);                            \
+    if (JJ == 0) mma_s8s8_zero(acc, a0, a1, a2, a3, bv[2 * JJ], bv[2 * JJ + 1]);          \
+    else mma_s8s8(acc, a0, a1, a2, a3, bv[2 * JJ], bv[2 * JJ + 1]);                       \
+  }
+      MOE_GU_GROUP(0) MOE_GU_GROUP(1) MOE_GU_GROUP(2) MOE_GU_GROUP(3)
+#undef MOE_GU_GROUP
+      // this lane's columns: its own sub-block, digits hi and lo, rows g and g + 8
+      i0 += (acc[0] * 128 + acc[1]) * iq2_odd(ra);
+      i1 += (acc[2] * 128 + acc[3]) * iq2_odd(rb);
     }
     __syncwarp();
     if (c.lane == 0) mbar_arrive(&c.empty[s]);
+    const float xsv = XS ? ld_sf(c.xs_s + (tok * (H / 256) + kblk) * 4) : __ldg(c.xscl + tok * (H / 256) + kblk);
+    const uint32_t w0 = j ? dp[1][0] : dp[0][0], w1 = j ? dp[1][1] : dp[0][1];
+    const float d0 = bb ? half_hi(w0) : half_lo(w0);
+    const float d1 = bb ? half_hi(w1) : half_lo(w1);
+    f0 = fmaf(static_cast<float>(i0), d0 * xsv, f0);
+    f1 = fmaf(static_cast<float>(i1), d1 * xsv, f1);
   }
-  // the four lanes of a quad hold four different sub-blocks of the same rows
+  // the four lanes of a quad hold the four sub-block columns of rows g, g + 8
   f0 += __shfl_xor_sync(0xffffffffu, f0, 1);
   f0 += __shfl_xor_sync(0xffffffffu, f0, 2);
   f1 += __shfl_xor_sync(0xffffffffu, f1, 1);
   f1 += __shfl_xor_sync(0xffffffffu, f1, 2);
   if (tig == 0) {
-    float* out = a.gpart + ((static_cast<size_t>(w.p0) * 2 + w.m) * a.KP + w.kp) * I + w.rb * kBoxRows + row_l;
-    out[0] = f0;
-    out[8] = f1;
+    const size_t o = ((static_cast<size_t>(w.p0) * 2 + w.m) * a.KP + w.kp) * I + w.rb * kBoxRows + 16 * c.warp + g;
+    if (index_ok(o + 8, a.gpart_n)) {
+      a.gpart[o] = f0;
+      a.gpart[o + 8] = f1;
+    }
   }
   return true;
 }
@@ -336,7 +416,7 @@ __device__ __forceinline__ bool gu_unit_one(const GuTmaArgs& a, const GuCtx& c, 
 // One unit whose expert holds 2..4*MAXQ assignments. TPG tokens share one set
 // of MMA columns (TPG tokens x 4/TPG sub-block slots x 2 digits); MAXQ column
 // sets reuse the same A operands.
-template <int TPG, int MAXQ>
+template <int TPG, int MAXQ, bool XS>
 __device__ __forceinline__ bool gu_unit_multi(const GuTmaArgs& a, const GuCtx& c, RingPos& rp, const GuUnit& w,
                                               const uint32_t (&dp)[kMaxNB][2]) {
   constexpr int SPS = 4 / TPG;
@@ -346,15 +426,15 @@ __device__ __forceinline__ bool gu_unit_multi(const GuTmaArgs& a, const GuCtx& c
   const int tslot_b = (g >> 1) % TPG, sslot_b = (g >> 1) / TPG, dig_b = g & 1;
   const int tslot_c = tig % TPG, sslot_c = tig / TPG;
   const int row_l = 16 * c.warp + g;
-  const int8_t* xb[MAXQ];
+  // B of column set q: digit dig_b of token tb = q*TPG + tslot_b, elements e0 + 32*(sub-block) of the box
+  int xtok[MAXQ];
   const float* xsc[MAXQ];
   bool bon[MAXQ];
 #pragma unroll
   for (int q = 0; q < MAXQ; ++q) {
     const int tb = q * TPG + tslot_b, tc = q * TPG + tslot_c;
     bon[q] = q < ngroups && tb < ne;
-    xb[q] = bon[q] ? c.xdig + (c.tok[p0 + tb] * 2 + dig_b) * c.xpitch + 8 * tig + (w.kp * a.NB * 16 + sslot_b) * 32
-                   : c.zero + 8 * tig;
+    xtok[q] = bon[q] ? c.tok[p0 + tb] : 0;
     xsc[q] = (q < ngroups && tc < ne) ? c.xscl + c.tok[p0 + tc] * (H / 256) + 2 * a.NB * w.kp : nullptr;
   }
   int acc[MAXQ][4];
@@ -367,7 +447,7 @@ __device__ __forceinline__ bool gu_unit_multi(const GuTmaArgs& a, const GuCtx& c
   }
 #pragma unroll 1
   for (int j = 0; j < a.NB; ++j) {
-    if (!mbar_wait_bounded(&c.full[rp.s], rp.ph, a.err, ERR_TIMEOUT)) return false;
+    if (!mbar_wait_bounded(&c.full[rp.s], rp.ph, a.err, ERR_TIMEOUT, a.wait_limit)) return false;
     const int s = rp.s;
     rp.next(c.S);
     const uint8_t* rg = c.ring + s * kGuBox + row_l * kGuW;
@@ -388,8 +468,11 @@ __device__ __forceinline__ bool gu_unit_multi(const GuTmaArgs& a, const GuCtx& c
 #pragma unroll
         for (int jj = 0; jj < TPG; ++jj) {
           // column set jj covers sub-blocks 4cc + jj*SPS .. +SPS-1
-          const int8_t* xp = bon[q] ? xb[q] + j * 512 : xb[q];
-          const uint2 bl = *reinterpret_cast<const uint2*>(xp + (4 * cc + jj * SPS) * 32);
+          const int e = (w.kp * a.NB + j) * 512 + (4 * cc + jj * SPS + sslot_b) * 32 + 8 * tig;
+          const int8_t* xp = !bon[q] ? c.zero + 8 * tig
+                             : XS    ? c.xdig + x_off(H, xtok[q], dig_b, e)
+                                     : c.xdig + (xtok[q] * 2 + dig_b) * H + e;
+          const uint2 bl = *reinterpret_cast<const uint2*>(xp);
 #pragma unroll
           for (int sl = 0; sl < SPS; ++sl) {
             const int u = jj * SPS + sl;
@@ -406,7 +489,7 @@ __device__ __forceinline__ bool gu_unit_multi(const GuTmaArgs& a, const GuCtx& c
           iacc[q][1] += (acc[q][2] * 128 + acc[q][3]) * odd1;
         }
       }
-      if (cc & 1) {
+      {  // every four sub-blocks: with 14-bit activation digits a longer int32 sum could overflow
         const int sb = cc >> 1;
         const float d0 = sb ? half_hi(dj0) : half_lo(dj0);
         const float d1 = sb ? half_hi(dj1) : half_lo(dj1);
@@ -436,9 +519,11 @@ __device__ __forceinline__ bool gu_unit_multi(const GuTmaArgs& a, const GuCtx& c
   for (int q = 0; q < MAXQ; ++q) {
     const int t = q * TPG + tslot_c;
     if (q < ngroups && owner && t < ne) {
-      float* out = a.gpart + ((static_cast<size_t>(p0 + t) * 2 + w.m) * a.KP + w.kp) * I + w.rb * kBoxRows + row_l;
-      out[0] = facc[q][0];
-      out[8] = facc[q][1];
+      const size_t o = ((static_cast<size_t>(p0 + t) * 2 + w.m) * a.KP + w.kp) * I + w.rb * kBoxRows + row_l;
+      if (index_ok(o + 8, a.gpart_n)) {
+        a.gpart[o] = facc[q][0];
+        a.gpart[o + 8] = facc[q][1];
+      }
     }
   }
   return true;
@@ -457,7 +542,7 @@ __host__ __device__ inline GuPlan gu_plan(int E, int T, int k, int H, bool xs_in
   p.meta = kTabBytes;
   p.zero = p.meta + meta_bytes(E, T * k, true);
   p.x = p.zero + kZeroBytes;
-  p.xs = p.x + (xs_in ? align_up(static_cast<size_t>(T) * 2 * (H + kRowPad), 128) : 0);
+  p.xs = p.x + (xs_in ? align_up(static_cast<size_t>(T) * 2 * H, 128) : 0);
   const size_t end = p.xs + (xs_in ? align_up(static_cast<size_t>(T) * (H / 256) * 4, 128) : 0);
   p.ring = align_up(end, 1024);
   p.bars = p.ring + static_cast<size_t>(S) * kGuBox;
@@ -498,35 +583,38 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
     }
     fence_barrier_init();
   }
-  for (int i = tid; i < kTabBytes / 4; i += kThreadsT) {
-    const int ent = i >> 6;
-    reinterpret_cast<uint32_t*>(smem + pl.tab)[i] =
-        (i & 32) == 0 ? d_sel_tables2.level[ent] : (ent < 128 ? d_sel_tables2.sign[ent] : 0u);
-  }
+  fill_sel_tables(reinterpret_cast<uint32_t*>(smem + pl.tab), tid, kThreadsT);
   for (int i = tid; i < kZeroBytes / 16; i += kThreadsT) reinterpret_cast<uint4*>(zero)[i] = make_uint4(0, 0, 0, 0);
   pdl_wait();  // routing and activations come from the kernels before this one
   load_meta(ms, a.offsets, a.active, a.perm, a.E, nA, a.k, tid, kThreadsT);
-  if (XS) {
-    stage_rows(xsm, a.xd, T * 2, H, tid, kThreadsT);
+  if (XS) {  // [T][2][H] digits -> the staged layout of x_off, 16 bytes at a time
+    const int per = H / 16;
+    for (int i = tid; i < T * 2 * per; i += kThreadsT) {
+      const int row = i / per, e = (i - row * per) * 16;
+      *reinterpret_cast<uint4*>(xsm + x_off(H, row >> 1, row & 1, e)) = reinterpret_cast<const uint4*>(a.xd)[i];
+    }
     for (int i = tid; i < T * (H / 256); i += kThreadsT) xssm[i] = a.xs[i];
   }
   __syncthreads();
   const int nact = ms.act[a.E];
 
   if (warp == kCW) {  // producer
-    if (lane == 0) {
+    if (lane == 0 && !a.no_produce) {
       prefetch_tmap(&tm_gate);
       prefetch_tmap(&tm_up);
+      const uint64_t pol = l2_policy_evict_first();  // expert codes are read once per step
       RingPos rp{0, 0u};
       GuIter t;
       t.init(blockIdx.x, gridDim.x, a.KP, rbs);
       for (; t.slot < nact; t.next(a.KP, rbs)) {
         const int e = ms.act[t.slot];
         for (int j = 0; j < NB; ++j) {
-          if (!mbar_wait_bounded(&empty[rp.s], rp.ph ^ 1u, a.err, ERR_TIMEOUT)) return;
+          if (!mbar_wait_bounded(&empty[rp.s], rp.ph ^ 1u, a.err, ERR_TIMEOUT, a.wait_limit)) return;
           mbar_arrive_expect_tx(&full[rp.s], kGuBox);
-          tma_load_2d(ring + rp.s * kGuBox, t.m ? &tm_up : &tm_gate, (t.kp * NB + j) * kGuW, e * I + t.rb * kBoxRows,
-                      &full[rp.s]);
+          index_ok(static_cast<size_t>(e) * I + t.rb * kBoxRows + kBoxRows - 1, static_cast<size_t>(a.E) * I);
+          index_ok(static_cast<size_t>(t.kp * NB + j) * kGuW + kGuW - 1, static_cast<size_t>(H) / 4);
+          tma_load_2d_hint(ring + rp.s * kGuBox, t.m ? &tm_up : &tm_gate, (t.kp * NB + j) * kGuW,
+                           e * I + t.rb * kBoxRows, &full[rp.s], pol);
           rp.next(S);
         }
       }
@@ -543,7 +631,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
     c.xdig = xsm;
     c.xscl = xssm;
     c.zero = zero;
-    c.xpitch = H + kRowPad;
+    c.xpitch = 0;  // staged layout: x_off
   } else {
     c.xdig = a.xd;
     c.xscl = a.xs;
@@ -598,10 +686,9 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
       dload(nw, nd);
     }
     bool ok;
-    if (XS && (MAXQ == 1 || w.ne == 1)) ok = gu_unit_one(a, c, rp, w, d);
-    else if (w.ne == 1) ok = gu_unit_multi<4, 1>(a, c, rp, w, d);
-    else if (w.ne == 2) ok = gu_unit_multi<2, 1>(a, c, rp, w, d);
-    else ok = gu_unit_multi<4, (MAXQ > 1 ? MAXQ : 1)>(a, c, rp, w, d);
+    if (MAXQ == 1 || w.ne == 1) ok = gu_unit_one<XS>(a, c, rp, w, d);
+    else if (w.ne == 2) ok = gu_unit_multi<2, 1, XS>(a, c, rp, w, d);
+    else ok = gu_unit_multi<4, (MAXQ > 1 ? MAXQ : 1), XS>(a, c, rp, w, d);
     if (!ok) return;
   }
 }
@@ -609,6 +696,14 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
 // ===========================================================================
 // down
 // ===========================================================================
+// A down box is one Q2K block of 256 rows, brought in as two TMA boxes of the
+// same rows: the 64 q bytes with the 64-byte swizzle (rows 64 bytes apart,
+// 16-byte chunk c of row R at c ^ ((R >> 1) & 3)) and the 16 scale bytes dense.
+constexpr int kDnQBytes = kBoxRows * 64;             // 16 KB
+constexpr int kDnSBytes = kBoxRows * 16;             // 4 KB
+constexpr int kDnStage = kDnQBytes + kDnSBytes;      // 20 KB, a multiple of 1024
+
+
 struct DnTmaArgs {
   int H, I, E, k, T, DP, NB, S;
   const uint32_t* dd;
@@ -618,6 +713,7 @@ struct DnTmaArgs {
   const int32_t* offsets;
   const int32_t* active;
   float* opart;  // [T*k][DP][H]
+  size_t opart_n;  // its length in floats (bounds-checked build)
   int* err;
   int hss;
 };
@@ -664,99 +760,114 @@ struct DnCtx {
   const uint8_t* ring;
   uint64_t* full;
   uint64_t* empty;
-  const int8_t* hd;    // rows (assignment, digit) of I digits in MMA k order, pitch hpitch
+  const int8_t* hd;    // h digits (h_off layout), staged or global
   const float* hsc;    // [T*k][hss]
   const int32_t* hq;   // [T*k][I/16]
   const int8_t* zero;  // 128-byte aligned zero region
-  uint32_t ring_s, hd_s, hsc_s, hq_s, zero_s;  // shared-window addresses (staged variant)
-  int hpitch, warp, lane, g, tig, S;
+  uint32_t ring_s, hd_s, hsc_s, hq_s;  // shared-window addresses (staged variant)
+  int warp, lane, g, tig, S;
 };
 
 __device__ __forceinline__ float dn_block(uint32_t dd, float e2, int iA, int iM) {
   return e2 * fmaf(half_lo(dd), static_cast<float>(iA), -half_hi(dd) * static_cast<float>(iM));
 }
 
-// One down unit for an expert with one assignment. MMA columns:
-// (pair slot 0..1) x (half 0..1) x (digit hi, lo); idle column halves read the
-// zero region.
-// One down unit for an expert with one assignment, h staged in shared memory.
-// MMA columns: (pair slot 0..1) x (half 0..1) x (digit hi, lo); idle column
-// halves read the zero region. All shared-memory addresses are 32-bit with
-// compile-time offsets.
+// Q2K A operands of one 16-weight sub-block word for one row: bit pair r of
+// its four bytes (weights 4i + r) -> uint8 bytes. The shifts are multiplies
+// (FMA pipe), the masks LOP3s.
+__device__ __forceinline__ void q2k_sub4(uint32_t w, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  r0 = w & 0x03030303u;
+  r1 = __umulhi(w, 1u << 30) & 0x03030303u;
+  r2 = __umulhi(w, 1u << 28) & 0x03030303u;
+  r3 = __umulhi(w, 1u << 26) & 0x03030303u;
+}
+
+// One down unit whose expert holds a single assignment.
+//
+// Lane mapping (m16n8k32, lane = 4g + tig): rows g and g+8 of the warp's 16; in
+// round cc (0..3) the lane owns sub-block 4*tig + cc of the block, whole: two
+// MMAs take its bit pairs (0, 1) and (2, 3). Its four q words are one 16-byte
+// chunk per row and its four scale bytes one word per row, loaded once per
+// box, after which the stage is released. MMA columns are (owner tig, digit
+// hi/lo); B is non-zero on the lanes with g >> 1 == tig (one 16-byte load of
+// h digits per round), so the accumulators of lane tig hold its own sub-block.
+template <bool HS>
 __device__ __forceinline__ bool dn_unit_one(const DnTmaArgs& a, const DnCtx& c, RingPos& rp, const DnUnit& w,
                                             const uint32_t (&dd)[kMaxNB][2]) {
   const int H = a.H, I = a.I, NB = a.NB;
   const int g = c.g, tig = c.tig;
-  const int row_l = 16 * c.warp + g;
-  const uint32_t sh = 2 * tig;
-  const int sl_b = g >> 2, hb = (g >> 1) & 1, dig_b = g & 1;
-  const uint32_t hrow = c.hd_s + (w.p0 * 2 + dig_b) * c.hpitch + w.dp * NB * 256 + 8 * tig;
-  const uint32_t zrow = c.zero_s + ((64 * (w.p0 & 1) + 64) & 127) + 8 * tig;
-  const uint32_t hqr = c.hq_s + (w.p0 * (I / 16) + w.dp * NB * 16 + tig) * 4;
-  const uint32_t e2p = c.hsc_s + (w.p0 * a.hss + w.dp * NB) * 4;
+  const bool bact = (g >> 1) == tig;
+  const int row = 16 * c.warp + g;
+  const uint32_t qoff = static_cast<uint32_t>(row) * 64 + 16u * (static_cast<uint32_t>(tig) ^ ((g >> 1) & 3));
+  const uint32_t soff = kDnQBytes + static_cast<uint32_t>(row) * 16 + 4u * tig;
   float f0 = 0.f, f1 = 0.f;
 #pragma unroll 1
   for (int j = 0; j < NB; ++j) {
-    uint32_t bp0[2], bp1[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      bp0[u] = (sl_b == u && hb == 0) ? hrow + j * 256 : zrow;
-      bp1[u] = (sl_b == u && hb == 1) ? hrow + j * 256 + 4 : zrow + 4;
+    const int blk = w.dp * NB + j;  // block of I
+    const int hb = h_off(I, w.p0, g & 1, blk * 256 + 64 * tig);  // sub-block 4 tig, round 0
+    const int hqi = w.p0 * (I / 16) + blk * 16 + 4 * tig;
+    int4 hq4;
+    float e2;
+    if (HS) {
+      const uint4 v = ld_s128(c.hq_s + hqi * 4);
+      hq4 = make_int4(static_cast<int>(v.x), static_cast<int>(v.y), static_cast<int>(v.z), static_cast<int>(v.w));
+      e2 = ld_sf(c.hsc_s + (w.p0 * a.hss + blk) * 4);
+    } else {
+      hq4 = __ldcg(reinterpret_cast<const int4*>(c.hq + hqi));
+      e2 = __ldcg(c.hsc + w.p0 * a.hss + blk);
     }
     if (!mbar_wait_bounded(&c.full[rp.s], rp.ph, a.err, ERR_TIMEOUT)) return false;
-    const uint32_t rA = c.ring_s + rp.s * kDnBox + row_l * kDnW, rB = rA + 8 * kDnW;
-    const int s = rp.s;
+    const uint32_t st = c.ring_s + rp.s * kDnStage;
+    const uint4 qa = ld_s128(st + qoff), qb = ld_s128(st + qoff + 8 * 64);
+    const uint32_t sa = ld_s32(st + soff), sb = ld_s32(st + soff + 8 * 16);
+    __syncwarp();
+    if (c.lane == 0) mbar_arrive(&c.empty[rp.s]);  // the codes are in registers: the stage is free
     rp.next(c.S);
+    const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w}, wb[4] = {qb.x, qb.y, qb.z, qb.w};
+    const int hqv[4] = {hq4.x, hq4.y, hq4.z, hq4.w};
     int iA0 = 0, iA1 = 0, iM0 = 0, iM1 = 0;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {  // 16 q bytes = four sub-blocks = two MMAs
-      const uint4 qa = ld_s128(rA + 16 + 16 * cc);
-      const uint4 qb = ld_s128(rB + 16 + 16 * cc);
-      uint32_t bv0[2], bv1[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        bv0[u] = ld_s32(bp0[u] + (2 * cc + u) * 32);
-        bv1[u] = ld_s32(bp1[u] + (2 * cc + u) * 32);
+    for (int cc = 0; cc < 4; ++cc) {
+      uint4 bh = make_uint4(0u, 0u, 0u, 0u);
+      if (bact) {
+        if (HS) bh = ld_s128(c.hd_s + hb + 128 * cc);
+        else bh = __ldcg(reinterpret_cast<const uint4*>(c.hd + hb + 128 * cc));
       }
-      // this thread's columns: sub-block 4cc + tig (pair 2cc + tig/2, half tig&1)
-      const uint32_t scA = ld_s8(rA + 4 * cc + tig), scB = ld_s8(rB + 4 * cc + tig);
-      const int hqv = static_cast<int>(ld_s32(hqr + (j * 16 + 4 * cc) * 4));
+      uint32_t x0, x1, x2, x3, y0, y1, y2, y3;
+      q2k_sub4(wa[cc], x0, x1, x2, x3);
+      q2k_sub4(wb[cc], y0, y1, y2, y3);
       int acc[4];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const uint32_t wa0 = u ? qa.z : qa.x, wa1 = u ? qa.w : qa.y;
-        const uint32_t wb0 = u ? qb.z : qb.x, wb1 = u ? qb.w : qb.y;
-        const uint32_t a0 = (wa0 >> sh) & 0x03030303u, a1 = (wb0 >> sh) & 0x03030303u;
-        const uint32_t a2 = (wa1 >> sh) & 0x03030303u, a3 = (wb1 >> sh) & 0x03030303u;
-        if (u == 0) mma_u8s8_zero(acc, a0, a1, a2, a3, bv0[u], bv1[u]);
-        else mma_u8s8(acc, a0, a1, a2, a3, bv0[u], bv1[u]);
-      }
-      iA0 += (acc[0] * 128 + acc[1]) * static_cast<int>(scA & 15u);
-      iA1 += (acc[2] * 128 + acc[3]) * static_cast<int>(scB & 15u);
-      iM0 += static_cast<int>(scA >> 4) * hqv;
-      iM1 += static_cast<int>(scB >> 4) * hqv;
+      mma_u8s8_zero(acc, x0, y0, x1, y1, bh.x, bh.y);
+      mma_u8s8(acc, x2, y2, x3, y3, bh.z, bh.w);
+      const uint32_t ba = cc ? __umulhi(sa, 1u << (32 - 8 * cc)) : sa;  // scale byte cc at bits 0..7
+      const uint32_t bb = cc ? __umulhi(sb, 1u << (32 - 8 * cc)) : sb;
+      iA0 += (acc[0] * 128 + acc[1]) * static_cast<int>(ba & 15u);
+      iA1 += (acc[2] * 128 + acc[3]) * static_cast<int>(bb & 15u);
+      iM0 += static_cast<int>((ba >> 4) & 15u) * hqv[cc];
+      iM1 += static_cast<int>((bb >> 4) & 15u) * hqv[cc];
     }
-    const float e2 = ld_sf(e2p + j * 4);
-    __syncwarp();
-    if (c.lane == 0) mbar_arrive(&c.empty[s]);
     const uint32_t dA = j ? dd[1][0] : dd[0][0], dB = j ? dd[1][1] : dd[0][1];
     f0 += dn_block(dA, e2, iA0, iM0);
     f1 += dn_block(dB, e2, iA1, iM1);
   }
+  // the four lanes of a quad hold the four quarters of the block of rows g, g + 8
   f0 += __shfl_xor_sync(0xffffffffu, f0, 1);
   f0 += __shfl_xor_sync(0xffffffffu, f0, 2);
   f1 += __shfl_xor_sync(0xffffffffu, f1, 1);
   f1 += __shfl_xor_sync(0xffffffffu, f1, 2);
   if (tig == 0) {
-    float* out = a.opart + (static_cast<size_t>(w.p0) * a.DP + w.dp) * H + w.rb * kBoxRows + row_l;
-    out[0] = f0;
-    out[8] = f1;
+    const size_t o = (static_cast<size_t>(w.p0) * a.DP + w.dp) * H + w.rb * kBoxRows + row;
+    if (index_ok(o + 8, a.opart_n)) {
+      a.opart[o] = f0;
+      a.opart[o + 8] = f1;
+    }
   }
   return true;
 }
 
-// One down unit for an expert with 2..2*MAXQ assignments. MMA columns:
-// (token slot 0..1) x (half 0..1) x (digit hi, lo).
+// One down unit for an expert with 2..2*MAXQ assignments. Each MMA takes a pair
+// of sub-blocks (2pr, 2pr + 1), lane tig bit pair tig of their bytes; MMA
+// columns: (token slot 0..1) x (half 0..1) x (digit hi, lo).
 template <int MAXQ>
 __device__ __forceinline__ bool dn_unit_multi(const DnTmaArgs& a, const DnCtx& c, RingPos& rp, const DnUnit& w,
                                               const uint32_t (&dd)[kMaxNB][2]) {
@@ -766,26 +877,23 @@ __device__ __forceinline__ bool dn_unit_multi(const DnTmaArgs& a, const DnCtx& c
   const int dig_b = g & 1, hb = (g >> 1) & 1, sl_b = g >> 2;
   const int hc = tig & 1, sl_c = tig >> 1;
   const uint32_t sh = 2 * tig;
-  const int row_l = 16 * c.warp + g;
-  const int8_t* hrow[MAXQ];
-  bool b0on[MAXQ], b1on[MAXQ];
+  const int row = 16 * c.warp + g;
+  int pb[MAXQ];  // assignment of this lane's B column per group (-1: zero column)
   const int32_t* hq_ptr[MAXQ];
   const float* e2p[MAXQ];
 #pragma unroll
   for (int q = 0; q < MAXQ; ++q) {
     const int tb = 2 * q + sl_b, tc = 2 * q + sl_c;
-    const bool on = q < ngroups && tb < ne;
-    hrow[q] = c.hd + ((p0 + (on ? tb : 0)) * 2 + dig_b) * c.hpitch + w.dp * a.NB * 256 + 8 * tig;
-    b0on[q] = on && hb == 0;
-    b1on[q] = on && hb == 1;
+    pb[q] = (q < ngroups && tb < ne) ? p0 + tb : -1;
     const bool cv = q < ngroups && tc < ne;
     hq_ptr[q] = c.hq + (p0 + (cv ? tc : 0)) * (I / 16) + w.dp * a.NB * 16 + hc;
     e2p[q] = cv ? c.hsc + (p0 + tc) * a.hss + w.dp * a.NB : nullptr;
   }
-  const int8_t* zrow = c.zero + 8 * tig;
   float facc[MAXQ][2];
 #pragma unroll
   for (int q = 0; q < MAXQ; ++q) facc[q][0] = facc[q][1] = 0.f;
+  const uint32_t qoff = static_cast<uint32_t>(row) * 64;
+  const uint32_t qsw = static_cast<uint32_t>((g >> 1) & 3);
 #pragma unroll 1
   for (int j = 0; j < a.NB; ++j) {
     int acc[4];
@@ -795,30 +903,35 @@ __device__ __forceinline__ bool dn_unit_multi(const DnTmaArgs& a, const DnCtx& c
     if (!mbar_wait_bounded(&c.full[rp.s], rp.ph, a.err, ERR_TIMEOUT)) return false;
     const int s = rp.s;
     rp.next(c.S);
-    const uint8_t* rA = c.ring + s * kDnBox + row_l * kDnW;
-    const uint8_t* rB = rA + 8 * kDnW;
+    const uint8_t* st = c.ring + s * kDnStage;
+    const uint8_t* sA = st + kDnQBytes + row * 16;
+    const uint8_t* sB = sA + 8 * 16;
+    const int blk = w.dp * a.NB + j;
 #pragma unroll 1
-    for (int cc = 0; cc < 4; ++cc) {
-      const uint4 qa = lds128(rA + 16 + 16 * cc);
-      const uint4 qb = lds128(rB + 16 + 16 * cc);
+    for (int cc = 0; cc < 4; ++cc) {  // logical 16-byte chunk cc of the q bytes: sub-blocks 4cc .. 4cc + 3
+      const uint4 qa = lds128(st + qoff + 16 * (cc ^ qsw));
+      const uint4 qb = lds128(st + qoff + 8 * 64 + 16 * (cc ^ qsw));
       uint32_t af[2][4];
-      af[0][0] = (qa.x >> sh) & 0x03030303u; af[0][1] = (qb.x >> sh) & 0x03030303u;
-      af[0][2] = (qa.y >> sh) & 0x03030303u; af[0][3] = (qb.y >> sh) & 0x03030303u;
-      af[1][0] = (qa.z >> sh) & 0x03030303u; af[1][1] = (qb.z >> sh) & 0x03030303u;
-      af[1][2] = (qa.w >> sh) & 0x03030303u; af[1][3] = (qb.w >> sh) & 0x03030303u;
+      af[0][0] = q2k_quad(qa.x, sh); af[0][1] = q2k_quad(qb.x, sh);
+      af[0][2] = q2k_quad(qa.y, sh); af[0][3] = q2k_quad(qb.y, sh);
+      af[1][0] = q2k_quad(qa.z, sh); af[1][1] = q2k_quad(qb.z, sh);
+      af[1][2] = q2k_quad(qa.w, sh); af[1][3] = q2k_quad(qb.w, sh);
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int pr = 2 * cc + u;
         // this thread's columns: sub-block 2*pr + hc of token 2q + sl_c
         const int sub = 2 * pr + hc;
-        const uint32_t scA = rA[sub], scB = rB[sub];
+        const uint32_t scA = sA[sub], scB = sB[sub];
 #pragma unroll
         for (int q = 0; q < MAXQ; ++q) {
           if (q >= ngroups) break;
-          const int8_t* p0b = b0on[q] ? hrow[q] + j * 256 : zrow;
-          const int8_t* p1b = b1on[q] ? hrow[q] + j * 256 + 4 : zrow + 4;
-          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(p0b + pr * 32);
-          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(p1b + pr * 32);
+          uint32_t b0 = 0u, b1 = 0u;
+          if (pb[q] >= 0) {  // bit pair tig of sub-block 2pr + hb: bytes 4 tig .. 4 tig + 3 (elements tig + 4i)
+            const int8_t* hp = c.hd + h_off(I, pb[q], dig_b, blk * 256 + (2 * pr + hb) * 16 + tig);
+            const uint32_t v = *reinterpret_cast<const uint32_t*>(hp);
+            if (hb == 0) b0 = v;
+            else b1 = v;
+          }
           mma_u8s8_zero(acc, af[u][0], af[u][1], af[u][2], af[u][3], b0, b1);
           const int hqv = hq_ptr[q][j * 16 + 2 * pr];
           iA[q][0] += (acc[0] * 128 + acc[1]) * static_cast<int>(scA & 15u);
@@ -846,9 +959,11 @@ __device__ __forceinline__ bool dn_unit_multi(const DnTmaArgs& a, const DnCtx& c
     f1 += __shfl_xor_sync(0xffffffffu, f1, 1);
     const int t = 2 * q + sl_c;
     if (hc == 0 && t < ne) {
-      float* out = a.opart + (static_cast<size_t>(p0 + t) * a.DP + w.dp) * H + w.rb * kBoxRows + row_l;
-      out[0] = f0;
-      out[8] = f1;
+      const size_t o = (static_cast<size_t>(p0 + t) * a.DP + w.dp) * H + w.rb * kBoxRows + row;
+      if (index_ok(o + 8, a.opart_n)) {
+        a.opart[o] = f0;
+        a.opart[o + 8] = f1;
+      }
     }
   }
   return true;
@@ -863,17 +978,18 @@ __host__ __device__ inline DnPlan dn_plan(int E, int nA, int I, int hss, bool hs
   p.meta = 0;
   p.zero = meta_bytes(E, nA, false);
   p.hd = p.zero + kZeroBytes;
-  p.hsc = p.hd + (hs_in ? align_up(static_cast<size_t>(nA) * 2 * (I + kRowPad), 128) : 0);
+  p.hsc = p.hd + (hs_in ? align_up(static_cast<size_t>(nA) * 2 * I, 128) : 0);
   p.hq = p.hsc + (hs_in ? align_up(static_cast<size_t>(nA) * hss * 4, 128) : 0);
   const size_t end = p.hq + (hs_in ? align_up(static_cast<size_t>(nA) * (I / 16) * 4, 128) : 0);
   p.ring = align_up(end, 1024);
-  p.bars = p.ring + static_cast<size_t>(S) * kDnBox;
+  p.bars = p.ring + static_cast<size_t>(S) * kDnStage;
   p.total = p.bars + 2 * static_cast<size_t>(S) * 8;
   return p;
 }
 
 template <int MAXQ, bool HS>
-__global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_constant__ CUtensorMap tm_down,
+__global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                                const __grid_constant__ CUtensorMap tm_s,
                                                                 DnTmaArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   pdl_trigger();
@@ -894,6 +1010,10 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
   uint64_t* empty = full + S;
   const int rbs = H / kBoxRows;
 
+  if ((smem_addr(ring) & 1023u) != 0) {  // the swizzled q boxes assume 1024-byte aligned stages
+    if (tid == 0) atomicCAS(a.err, 0, ERR_CUDA);
+    return;
+  }
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
@@ -904,8 +1024,9 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
   for (int i = tid; i < kZeroBytes / 16; i += kThreadsT) reinterpret_cast<uint4*>(zero)[i] = make_uint4(0, 0, 0, 0);
   pdl_wait();  // routing and h come from the kernels before this one
   load_meta(ms, a.offsets, a.active, nullptr, a.E, nA, a.k, tid, kThreadsT);
-  if (HS) {
-    stage_rows(hd_s, a.hd, nA * 2, I, tid, kThreadsT);
+  if (HS) {  // the h_off layout is the same in global and shared memory
+    for (int i = tid; i < nA * 2 * I / 16; i += kThreadsT)
+      reinterpret_cast<uint4*>(hd_s)[i] = reinterpret_cast<const uint4*>(a.hd)[i];
     for (int i = tid; i < nA * a.hss; i += kThreadsT) hsc_s[i] = a.hsc[i];
     for (int i = tid; i < nA * (I / 16); i += kThreadsT) hq_s[i] = a.hq[i];
   }
@@ -914,7 +1035,9 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
 
   if (warp == kCW) {  // producer
     if (lane == 0) {
-      prefetch_tmap(&tm_down);
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_s);
+      const uint64_t pol = l2_policy_evict_first();  // expert codes are read once per step
       RingPos rp{0, 0u};
       DnIter t;
       t.init(blockIdx.x, gridDim.x, a.DP, rbs);
@@ -922,8 +1045,13 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
         const int e = ms.act[t.slot];
         for (int j = 0; j < NB; ++j) {
           if (!mbar_wait_bounded(&empty[rp.s], rp.ph ^ 1u, a.err, ERR_TIMEOUT)) return;
-          mbar_arrive_expect_tx(&full[rp.s], kDnBox);
-          tma_load_2d(ring + rp.s * kDnBox, &tm_down, (t.dp * NB + j) * kDnW, e * H + t.rb * kBoxRows, &full[rp.s]);
+          mbar_arrive_expect_tx(&full[rp.s], kDnStage);
+          const int x0 = (t.dp * NB + j) * 80, y0 = e * H + t.rb * kBoxRows;
+          index_ok(static_cast<size_t>(y0) + kBoxRows - 1, static_cast<size_t>(a.E) * H);
+          index_ok(static_cast<size_t>(x0) + 79, static_cast<size_t>(I / 256) * 80);
+          uint8_t* st = ring + rp.s * kDnStage;
+          tma_load_2d_hint(st, &tm_q, x0 + 16, y0, &full[rp.s], pol);
+          tma_load_2d_hint(st + kDnQBytes, &tm_s, x0, y0, &full[rp.s], pol);
           rp.next(S);
         }
       }
@@ -939,19 +1067,15 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
     c.hd = hd_s;
     c.hsc = hsc_s;
     c.hq = hq_s;
-    c.zero = zero;
-    c.hpitch = I + kRowPad;
     c.hd_s = smem_addr(hd_s);
     c.hsc_s = smem_addr(hsc_s);
     c.hq_s = smem_addr(hq_s);
-    c.zero_s = smem_addr(zero);
   } else {
     c.hd = a.hd;
     c.hsc = a.hsc;
     c.hq = a.hq;
-    c.zero = g_zero_operand;
-    c.hpitch = I;
   }
+  c.zero = zero;
   c.warp = warp;
   c.lane = lane;
   c.g = lane >> 2;
@@ -989,9 +1113,53 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
       ddload(nw, nd);
     }
     bool ok;
-    if (HS && (MAXQ == 1 || w.ne == 1)) ok = dn_unit_one(a, c, rp, w, d);
+    if (MAXQ == 1 || w.ne == 1) ok = dn_unit_one<HS>(a, c, rp, w, d);
     else ok = dn_unit_multi<(MAXQ > 1 ? MAXQ : 1)>(a, c, rp, w, d);
     if (!ok) return;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The decode GEMVs' operand builders run on their own, for exact checks: per
+// IQ2 sub-block record the int8 A bytes (level * sign) of its four groups and
+// 2ls + 1; per Q2K sub-block sc * q of its 16 weights (from the uint8 q bytes of
+// q2k_quad) and m. Every lane uses its own table replica, as in the GEMV.
+__global__ void __launch_bounds__(256) debug_gemv_iq2_kernel(const uint8_t* __restrict__ codes, int64_t nsub,
+                                                             int8_t* __restrict__ w, uint8_t* __restrict__ odd,
+                                                             uint32_t one) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  fill_sel_tables(reinterpret_cast<uint32_t*>(smem), threadIdx.x, blockDim.x);
+  __syncthreads();
+  const uint32_t lane = threadIdx.x & 31, lane4 = 4u * lane, sgn_lane = 128u + 4u * lane;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nsub;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint2 rec = *reinterpret_cast<const uint2*>(codes + 8 * i);
+    uint32_t o[8];
+    iq2_group_int8<0>(rec, lane4, sgn_lane, one, o[0], o[1]);
+    iq2_group_int8<1>(rec, lane4, sgn_lane, one, o[2], o[3]);
+    iq2_group_int8<2>(rec, lane4, sgn_lane, one, o[4], o[5]);
+    iq2_group_int8<3>(rec, lane4, sgn_lane, one, o[6], o[7]);
+    uint4* dst = reinterpret_cast<uint4*>(w + 32 * i);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    odd[i] = static_cast<uint8_t>(iq2_odd(rec));
+  }
+}
+
+__global__ void __launch_bounds__(256) debug_gemv_q2k_kernel(const uint8_t* __restrict__ codes, int64_t nsub,
+                                                             int16_t* __restrict__ scq, uint8_t* __restrict__ m) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nsub;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint8_t* blk = codes + (i / 16) * 80;
+    const int sb = static_cast<int>(i % 16);
+    const uint32_t word = *reinterpret_cast<const uint32_t*>(blk + 16 + 4 * sb);
+    const uint32_t scb = blk[sb];
+    for (int r = 0; r < 4; ++r) {
+      const uint32_t quad = q2k_quad(word, 2u * r);  // weights 4i + r of the sub-block, i = 0..3
+      for (int b = 0; b < 4; ++b)
+        scq[16 * i + 4 * b + r] = static_cast<int16_t>(static_cast<int>((quad >> (8 * b)) & 0xFFu) * (scb & 15u));
+    }
+    m[i] = static_cast<uint8_t>(scb >> 4);
   }
 }
 
@@ -1011,7 +1179,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 2-D byte tensor [rows][row_bytes] with a box of box_rows x box_bytes.
 bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_bytes,
-              uint32_t box_rows, bool swizzle128) {
+              uint32_t box_rows, CUtensorMapSwizzle swizzle) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {row_bytes, rows};
@@ -1019,13 +1187,16 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t row
   const cuuint32_t box[2] = {box_bytes, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 constexpr size_t kBudget = 227 * 1024;
+
+// Fault injection (moe_debug_inject): read at each gate/up launch.
+int g_inject_mode = 0;
+long long g_inject_limit = 0;
 
 int nb_for(int T) { return T == 1 ? 1 : 2; }
 
@@ -1037,12 +1208,46 @@ void launch_k(K kern, int grid, size_t smem, cudaStream_t st, const CUtensorMap&
 }
 
 template <typename K>
-void launch_k(K kern, int grid, size_t smem, cudaStream_t st, const CUtensorMap& m0, const DnTmaArgs& a) {
+void launch_k(K kern, int grid, size_t smem, cudaStream_t st, const CUtensorMap& m0, const CUtensorMap& m1,
+              const DnTmaArgs& a) {
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  launch_pdl(kern, dim3(grid), dim3(kThreadsT), smem, st, m0, a);
+  launch_pdl(kern, dim3(grid), dim3(kThreadsT), smem, st, m0, m1, a);
 }
 
 }  // namespace
+
+int launch_debug_gemv_iq2(const uint8_t* codes, int64_t nblocks, int8_t* w, uint8_t* odd, cudaStream_t st) {
+  const int64_t nsub = nblocks * 8;
+  const int grid = static_cast<int>(std::min<int64_t>((nsub + 255) / 256, 4096));
+  cudaFuncSetAttribute(debug_gemv_iq2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTabBytes);
+  debug_gemv_iq2_kernel<<<grid, 256, kTabBytes, st>>>(codes, nsub, w, odd, 1u);
+  return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
+}
+
+int launch_debug_gemv_q2k(const uint8_t* codes, int64_t nblocks, int16_t* scq, uint8_t* m, cudaStream_t st) {
+  const int64_t nsub = nblocks * 16;
+  const int grid = static_cast<int>(std::min<int64_t>((nsub + 255) / 256, 4096));
+  debug_gemv_q2k_kernel<<<grid, 256, 0, st>>>(codes, nsub, scq, m);
+  return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
+}
+
+int read_bounds_violations(unsigned long long* out) {
+#ifdef MOE_BOUNDS_CHECK
+  const unsigned long long zero = 0;
+  if (cudaMemcpyFromSymbol(out, g_bounds_violations, sizeof(*out)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_bounds_violations, &zero, sizeof(zero)) != cudaSuccess)
+    return ERR_CUDA;
+  return OK;
+#else
+  *out = 0;
+  return ERR_SHAPE;  // not a bounds-checked build
+#endif
+}
+
+void set_debug_inject(int mode, long long wait_limit) {
+  g_inject_mode = mode;
+  g_inject_limit = wait_limit;
+}
 
 bool tma_path_supported(const LayerShape& s, int T) {
   return s.H % 1024 == 0 && s.I % 512 == 0 && T >= 1 && T <= 16 && s.E <= kMaxExpertsTma &&
@@ -1058,14 +1263,18 @@ int launch_gateup_tma(const LayerShape& sh, const uint8_t* gate_codes, const uin
                       const Routing& r, float* gpart, int* err, int sms, cudaStream_t st) {
   CUtensorMap tg, tu;
   const uint64_t rb = sh.H / 4, rows = static_cast<uint64_t>(sh.E) * sh.I;
-  if (!make_map(&tg, gate_codes, rb, rows, kGuW, kBoxRows, true) ||
-      !make_map(&tu, up_codes, rb, rows, kGuW, kBoxRows, true))
+  if (!make_map(&tg, gate_codes, rb, rows, kGuW, kBoxRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tu, up_codes, rb, rows, kGuW, kBoxRows, CU_TENSOR_MAP_SWIZZLE_128B))
     return ERR_CUDA;
   GuTmaArgs a{};
   a.H = sh.H; a.I = sh.I; a.E = sh.E; a.k = sh.k; a.T = T;
   a.NB = nb_for(T); a.KP = tma_gu_parts(sh, T);
   a.gate_d = gate_d; a.up_d = up_d; a.xd = xd; a.xs = xs;
   a.offsets = r.offsets; a.perm = r.perm; a.active = r.active; a.gpart = gpart; a.err = err;
+  a.gpart_n = static_cast<size_t>(T) * sh.k * 2 * a.KP * sh.I;
+  a.no_produce = g_inject_mode == 1;
+  a.one = 1;
+  a.wait_limit = g_inject_mode ? g_inject_limit : kDefaultWaitCycles;
   // stage the activations when that still leaves three ring stages
   const size_t budget = kBudget;
   const bool xs_in = gu_plan(sh.E, T, sh.k, sh.H, true, 3).total <= budget;
@@ -1092,15 +1301,18 @@ int launch_gateup_tma(const LayerShape& sh, const uint8_t* gate_codes, const uin
 int launch_down_tma(const LayerShape& sh, const uint8_t* down_codes, const uint32_t* down_dd, const int8_t* hd,
                     const float* hsc, const int32_t* hq, int hss, int T, const Routing& r, float* opart, int* err,
                     int sms, cudaStream_t st) {
-  CUtensorMap td;
-  const uint64_t rb = static_cast<uint64_t>(sh.I / 256) * kDnW, rows = static_cast<uint64_t>(sh.E) * sh.H;
-  if (!make_map(&td, down_codes, rb, rows, kDnW, kBoxRows, false)) return ERR_CUDA;
+  CUtensorMap tq, ts;
+  const uint64_t rb = static_cast<uint64_t>(sh.I / 256) * 80, rows = static_cast<uint64_t>(sh.E) * sh.H;
+  if (!make_map(&tq, down_codes, rb, rows, 64, kBoxRows, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map(&ts, down_codes, rb, rows, 16, kBoxRows, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return ERR_CUDA;
   DnTmaArgs a{};
   a.H = sh.H; a.I = sh.I; a.E = sh.E; a.k = sh.k; a.T = T; a.hss = hss;
   a.NB = nb_for(T); a.DP = tma_dn_parts(sh, T);
   a.dd = down_dd; a.hd = hd; a.hsc = hsc; a.hq = hq;
   a.offsets = r.offsets; a.active = r.active; a.opart = opart; a.err = err;
   const int nA = T * sh.k;
+  a.opart_n = static_cast<size_t>(nA) * a.DP * sh.H;
   const bool hs_in = dn_plan(sh.E, nA, sh.I, hss, true, 4).total <= kBudget;
   int S = 2;
   while (S < 8 && dn_plan(sh.E, nA, sh.I, hss, hs_in, S + 1).total <= kBudget) ++S;
@@ -1112,11 +1324,11 @@ int launch_down_tma(const LayerShape& sh, const uint8_t* down_codes, const uint3
   const int grid = std::max(1, std::min(units, sms));
   if (T == 1) {  // one token: the single-assignment variant with h staged
     if (!hs_in) return ERR_SHAPE;
-    launch_k(down_tma_kernel<1, true>, grid, smem, st, td, a);
+    launch_k(down_tma_kernel<1, true>, grid, smem, st, tq, ts, a);
   } else if (hs_in) {  // at most 16 tokens per expert: eight groups of two
-    launch_k(down_tma_kernel<8, true>, grid, smem, st, td, a);
+    launch_k(down_tma_kernel<8, true>, grid, smem, st, tq, ts, a);
   } else {
-    launch_k(down_tma_kernel<8, false>, grid, smem, st, td, a);
+    launch_k(down_tma_kernel<8, false>, grid, smem, st, tq, ts, a);
   }
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
 }

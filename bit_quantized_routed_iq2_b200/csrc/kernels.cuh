@@ -37,6 +37,9 @@ int launch_route(const uint16_t* Wr, const float* bias, const void* x, int x_dty
                  int32_t* active, int* err, cudaStream_t st,
                  bool clear_status = false);
 int launch_active_from_offsets(const int32_t* offsets, int E, int32_t* active, cudaStream_t st);
+// ids <- map[ids] (n entries), then the stable permutation of the n ids over E values.
+int launch_remap_permute(int32_t* ids, int n, const int32_t* map, int E, int32_t* offsets, int32_t* perm,
+                         int32_t* inv, int32_t* active, cudaStream_t st);
 
 // Workspace needed by the FFN stage for T tokens (bytes) and the launcher.
 size_t ffn_workspace_bytes(const LayerShape& s, int T);
@@ -45,6 +48,9 @@ size_t ffn_workspace_bytes(const LayerShape& s, int T);
 int launch_ffn(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
                const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st,
                bool shared_early = false);
+
+// L2 prefetch (evict_last) of up to four device ranges (decode.cu).
+int launch_l2_prefetch(const void* const* ptrs, const size_t* bytes, int n, cudaStream_t st);
 
 // Tensor-core dequant-GEMV path (decode.cu): shapes with H % 256 == 0 and I % 256 == 0.
 bool fast_path_supported(const LayerShape& s);
@@ -96,6 +102,27 @@ size_t prefill_workspace_bytes(const LayerShape& s, int T);
 int launch_ffn_prefill(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
                        const float* residual, float* y, void* ws, int* err, bool clear_status, int sms,
                        cudaStream_t st);
+
+// Copies the device status word at `word` to *out after the work enqueued on `st` (synchronises `st`).
+int read_status_word(const int* word, int32_t* out, cudaStream_t st);
+
+// Test aid: fault injection into the decode gate/up GEMV (mode 1: its producer issues no loads, so its
+// consumers' bounded waits run out after `wait_limit` cycles). Mode 0 restores normal operation.
+void set_debug_inject(int mode, long long wait_limit);
+
+// Violations counted by the bounds-checked build of the decode GEMVs since the
+// last read (then reset); ERR_SHAPE from a normal build.
+int read_bounds_violations(unsigned long long* out);
+
+// Float weights -> block formats (quant.cu).
+int launch_quantize_q2k(const float* w, int64_t nblocks, uint8_t* codes, uint32_t* dd, cudaStream_t st);
+int launch_quantize_iq2(const float* w, int64_t nblocks, uint8_t* codes, uint16_t* d, cudaStream_t st);
+
+// The hot paths' own operand builders, run on their own (gemv_tma.cu, prefill.cu).
+int launch_debug_gemv_iq2(const uint8_t* codes, int64_t nblocks, int8_t* w, uint8_t* odd, cudaStream_t st);
+int launch_debug_gemv_q2k(const uint8_t* codes, int64_t nblocks, int16_t* scq, uint8_t* m, cudaStream_t st);
+int launch_debug_tc_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, uint16_t* out, cudaStream_t st);
+int launch_debug_tc_q2k(const uint8_t* codes, const uint32_t* dd, int64_t nblocks, uint16_t* out, cudaStream_t st);
 
 int launch_debug_dequant_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, float* out, cudaStream_t st);
 int launch_debug_dequant_q2k(const uint8_t* codes, const uint32_t* dd, int64_t nblocks, float* out,

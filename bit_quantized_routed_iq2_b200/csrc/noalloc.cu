@@ -64,4 +64,12 @@ moe_status moe_layer_forward_noalloc(const moe_layer_desc* desc, const moe_layer
   return moe_layer_forward(desc, w, x, x_dtype, T, residual, y, scratch, kNoallocScratchBytes, stream);
 }
 
+moe_status moe_read_status_noalloc(int32_t* status, void* stream) {
+  if (!status) return MOE_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  moe_status st = scratch_address(&scratch);
+  if (st != MOE_OK) return st;
+  return moe_read_status(scratch, status, stream);
+}
+
 }  // extern "C"

@@ -235,13 +235,58 @@ __device__ __forceinline__ void dq_iq2_sub(uint2 rec, float dsc, uint32_t tabL, 
 __device__ __forceinline__ void dq_q2k_sub(uint32_t w, uint32_t scb, float d, float dmin, uint32_t tabQ,
                                            uint32_t (&o)[8]) {
   const float A = d * static_cast<float>(scb & 15u), B = dmin * static_cast<float>(scb >> 4);
-  const uint32_t tlo = f2_to_h2(-B, A - B), thi = f2_to_h2(2.f * A - B, 3.f * A - B);
+  // q = 0 gives 0 - B (not -B): +0 when dmin * m is 0, as the fp32 weight d*sc*0 - dmin*0 is
+  const uint32_t tlo = f2_to_h2(__fsub_rn(0.f, B), A - B), thi = f2_to_h2(2.f * A - B, 3.f * A - B);
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     const uint32_t ent = b == 0 ? w * 128u : __umulhi(w, 1u << (39 - 8 * b));  // byte b at bits 7..14
     const uint32_t sel = lds32s(tabQ + (ent & 0x7F80u));                       // tabQ includes lane * 4
     o[2 * b] = prmt(tlo, thi, sel);
     o[2 * b + 1] = prmt(tlo, thi, __umulhi(sel, 0x10000u));
+  }
+}
+
+// The dequantisation tables of the dequantising kinds, at `tabs` (see
+// TcLayout): IQ2 level selectors (16 copies of 8 bytes per grid row), IQ2 signs
+// as fp16 +-1 pairs (8 copies of 16 bytes per sign field), Q2K selectors (32
+// copies of 4 bytes per code byte).
+template <int KIND>
+__device__ __forceinline__ void fill_dq_tables(uint8_t* tabs, int tid, int nthr) {
+  if (KIND == TC_IQ2_PAIR) {
+    for (int i = tid; i < 256 * 16 * 2; i += nthr) {  // (row, copy, word): two prmt selectors per word
+      const int ent = i >> 5, w = i & 1;
+      uint32_t word = 0;
+      for (int h = 0; h < 2; ++h) {
+        const int e0 = 4 * w + 2 * h;
+        uint32_t lv[2];
+        for (int q = 0; q < 2; ++q) {
+          const uint32_t v = d_codebook_tc.val[ent][e0 + q];
+          lv[q] = v == 8 ? 0u : (v == 25 ? 1u : 2u);
+        }
+        const uint32_t sel = lv[0] | ((3 + lv[0]) << 4) | (lv[1] << 8) | ((3 + lv[1]) << 12);
+        word |= sel << (16 * h);
+      }
+      reinterpret_cast<uint32_t*>(tabs)[i] = word;
+    }
+    for (int i = tid; i < 128 * 8 * 4; i += nthr) {  // (sign field, copy, word)
+      const int ent = i >> 5, w = i & 3;
+      uint32_t par = 0;
+      for (int b = 0; b < 7; ++b) par ^= (ent >> b) & 1;
+      const uint32_t s0 = (2 * w < 7) ? ((ent >> (2 * w)) & 1) : par;
+      const uint32_t s1 = (2 * w + 1 < 7) ? ((ent >> (2 * w + 1)) & 1) : par;
+      // fp16 pair of +-1 (0x3C00 / 0xBC00)
+      reinterpret_cast<uint32_t*>(tabs + 256 * 128)[i] = 0x3C003C00u | (s0 << 15) | (s1 << 31);
+    }
+  } else if (KIND == TC_Q2K) {
+    for (int i = tid; i < 256 * 32; i += nthr) {  // (byte of four 2-bit codes, copy) -> two selectors
+      const int byte = i >> 5;
+      uint32_t sel = 0;
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t c = (byte >> (2 * q)) & 3u;
+        sel |= ((2 * c) | ((2 * c + 1) << 4)) << (8 * q);
+      }
+      reinterpret_cast<uint32_t*>(tabs)[i] = sel;
+    }
   }
 }
 
@@ -340,42 +385,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
   // replica of this lane is folded into the table bases (entries 128 bytes apart)
   const uint32_t tabL = sbase + L::tabs + (lane & 15) * 8, tabS = sbase + L::tabs + 256 * 128 + (lane & 7) * 16,
                  tabQ = sbase + L::tabs + lane * 4;
-  if (KIND == TC_IQ2_PAIR) {
-    for (int i = tid; i < 256 * 16 * 2; i += kTcThreads) {  // (row, copy, word): two prmt selectors per word
-      const int ent = i >> 5, w = i & 1;
-      uint32_t word = 0;
-      for (int h = 0; h < 2; ++h) {
-        const int e0 = 4 * w + 2 * h;
-        uint32_t lv[2];
-        for (int q = 0; q < 2; ++q) {
-          const uint32_t v = d_codebook_tc.val[ent][e0 + q];
-          lv[q] = v == 8 ? 0u : (v == 25 ? 1u : 2u);
-        }
-        const uint32_t sel = lv[0] | ((3 + lv[0]) << 4) | (lv[1] << 8) | ((3 + lv[1]) << 12);
-        word |= sel << (16 * h);
-      }
-      reinterpret_cast<uint32_t*>(smem + L::tabs)[i] = word;
-    }
-    for (int i = tid; i < 128 * 8 * 4; i += kTcThreads) {  // (sign field, copy, word)
-      const int ent = i >> 5, w = i & 3;
-      uint32_t par = 0;
-      for (int b = 0; b < 7; ++b) par ^= (ent >> b) & 1;
-      const uint32_t s0 = (2 * w < 7) ? ((ent >> (2 * w)) & 1) : par;
-      const uint32_t s1 = (2 * w + 1 < 7) ? ((ent >> (2 * w + 1)) & 1) : par;
-      // fp16 pair of +-1 (0x3C00 / 0xBC00)
-      reinterpret_cast<uint32_t*>(smem + L::tabs + 256 * 128)[i] = 0x3C003C00u | (s0 << 15) | (s1 << 31);
-    }
-  } else if (KIND == TC_Q2K) {
-    for (int i = tid; i < 256 * 32; i += kTcThreads) {  // (byte of four 2-bit codes, copy) -> two selectors
-      const int byte = i >> 5;
-      uint32_t sel = 0;
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t c = (byte >> (2 * q)) & 3u;
-        sel |= ((2 * c) | ((2 * c + 1) << 4)) << (8 * q);
-      }
-      reinterpret_cast<uint32_t*>(smem + L::tabs)[i] = sel;
-    }
-  }
+  fill_dq_tables<KIND>(smem + L::tabs, tid, kTcThreads);
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -922,6 +932,53 @@ PrefillWs carve_prefill(const LayerShape& sh, int T, char* base) {
   return w;
 }
 
+// The grouped GEMM's dequantisers run on their own, for exact checks: every
+// 32-weight IQ2 sub-block (dq_iq2_sub, scale d / 8 * 2^10) and every 16-weight
+// Q2K sub-block (dq_q2k_sub) to the fp16 words the kernel stores into TMEM,
+// weights in K order. Each lane reads its own replica of the tables.
+__global__ void __launch_bounds__(256) debug_tc_iq2_kernel(const uint8_t* __restrict__ codes,
+                                                           const uint16_t* __restrict__ d, int64_t nsub,
+                                                           uint32_t* __restrict__ out) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  fill_dq_tables<TC_IQ2_PAIR>(smem, threadIdx.x, blockDim.x);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t tabL = sbase + (lane & 15) * 8, tabS = sbase + 256 * 128 + (lane & 7) * 16;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nsub;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint2 rec = *reinterpret_cast<const uint2*>(codes + 8 * i);
+    const float dsc = half_bits_to_float(d[i / 8]) * 128.0f;  // d / 8 * 2^10, as the GEMM's dequantisers
+    uint32_t o[16];
+    dq_iq2_sub(rec, dsc, tabL, tabS, o);
+    uint4* dst = reinterpret_cast<uint4*>(out + 16 * i);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+  }
+}
+
+__global__ void __launch_bounds__(256) debug_tc_q2k_kernel(const uint8_t* __restrict__ codes,
+                                                           const uint32_t* __restrict__ dd, int64_t nsub,
+                                                           uint32_t* __restrict__ out) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  fill_dq_tables<TC_Q2K>(smem, threadIdx.x, blockDim.x);
+  __syncthreads();
+  const uint32_t tabQ = smem_addr(smem) + (threadIdx.x & 31) * 4;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nsub;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint8_t* blk = codes + (i / 16) * 80;
+    const int sb = static_cast<int>(i % 16);
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(blk + 16 + 4 * sb);
+    const uint32_t ddv = dd[i / 16];
+    uint32_t o[8];
+    dq_q2k_sub(w, blk[sb], half_bits_to_float(static_cast<uint16_t>(ddv & 0xFFFFu)),
+               half_bits_to_float(static_cast<uint16_t>(ddv >> 16)), tabQ, o);
+    uint4* dst = reinterpret_cast<uint4*>(out + 8 * i);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
 }  // namespace
 
 // Router logits for many bf16 tokens on the same tensor-core GEMM: weights
@@ -1041,4 +1098,23 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
 }
 
+}  // namespace moe
+
+namespace moe {
+int launch_debug_tc_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, uint16_t* out, cudaStream_t st) {
+  const int64_t nsub = nblocks * 8;
+  const int grid = static_cast<int>(std::min<int64_t>((nsub + 255) / 256, 4096));
+  constexpr int smem = 256 * 128 + 128 * 128;
+  cudaFuncSetAttribute(debug_tc_iq2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  debug_tc_iq2_kernel<<<grid, 256, smem, st>>>(codes, d, nsub, reinterpret_cast<uint32_t*>(out));
+  return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
+}
+
+int launch_debug_tc_q2k(const uint8_t* codes, const uint32_t* dd, int64_t nblocks, uint16_t* out, cudaStream_t st) {
+  const int64_t nsub = nblocks * 16;
+  const int grid = static_cast<int>(std::min<int64_t>((nsub + 255) / 256, 4096));
+  constexpr int smem = 256 * 128;
+  debug_tc_q2k_kernel<<<grid, 256, smem, st>>>(codes, dd, nsub, reinterpret_cast<uint32_t*>(out));
+  return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
+}
 }  // namespace moe

@@ -96,6 +96,53 @@ __device__ __forceinline__ void skinny_mainloop(const uint16_t* const (&W)[NM], 
   }
 }
 
+// The same for a warp whose K slice is exactly one step of 32 * U columns, in
+// two halves: skinny_load_a fetches the weight slice (constants of the layer),
+// skinny_finish loads the B columns and multiplies. A kernel can issue the
+// first half before it waits for the kernels that produce B.
+template <int NM, int U>
+__device__ __forceinline__ void skinny_load_a(const uint16_t* const (&W)[NM], int K, int r0, int kbeg,
+                                              uint4 (&av)[U][NM][2]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
+#pragma unroll
+  for (int m = 0; m < NM; ++m) {
+    const uint16_t* a0 = W[m] + static_cast<size_t>(r0 + g) * K + 8 * tig + kbeg;
+    const uint16_t* a1 = W[m] + static_cast<size_t>(r0 + g + 8) * K + 8 * tig + kbeg;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      av[u][m][0] = ldg16(a0 + 32 * u);
+      av[u][m][1] = ldg16(a1 + 32 * u);
+    }
+  }
+}
+
+template <int NM, int NG, int U>
+__device__ __forceinline__ void skinny_finish(const uint4 (&av)[U][NM][2], int K, const uint16_t* xb, int P, int T,
+                                              int kbeg, float (&acc)[NM][NG][4]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
+  uint4 bv[U][NG];
+#pragma unroll
+  for (int q = 0; q < NG; ++q) {
+    const int col = 8 * q + g, tok = col / P, part = col - tok * P;
+    const uint16_t* brow = xb + (static_cast<size_t>(part) * T + (tok < T ? tok : 0)) * K + 8 * tig + kbeg;
+#pragma unroll
+    for (int u = 0; u < U; ++u) bv[u][q] = tok < T ? ldg16(brow + 32 * u) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int m = 0; m < NM; ++m)
+#pragma unroll
+    for (int q = 0; q < NG; ++q) acc[m][q][0] = acc[m][q][1] = acc[m][q][2] = acc[m][q][3] = 0.f;
+#pragma unroll
+  for (int u = 0; u < U; ++u)
+#pragma unroll
+    for (int m = 0; m < NM; ++m)
+#pragma unroll
+      for (int q = 0; q < NG; ++q) {
+        mma_bf16(acc[m][q], av[u][m][0].x, av[u][m][1].x, av[u][m][0].y, av[u][m][1].y, bv[u][q].x, bv[u][q].y);
+        mma_bf16(acc[m][q], av[u][m][0].z, av[u][m][1].z, av[u][m][0].w, av[u][m][1].w, bv[u][q].z, bv[u][q].w);
+      }
+}
+
 // Store a warp's partial tiles: red[warp][m][col][row].
 template <int NM, int NG>
 __device__ __forceinline__ void skinny_store(float* red, const float (&acc)[NM][NG][4]) {
@@ -171,17 +218,26 @@ __global__ void __launch_bounds__(512) shared_down_combine_mma_kernel(
     const float* residual, float* y) {
   __shared__ __align__(16) float red[ks_max<NG>() * NG * 8 * kRows];
   extern __shared__ float osum[];  // [T*k][kRows]
+  constexpr int U = NG == 1 ? 4 : 2;
   pdl_trigger();
-  pdl_wait();  // h, the routed partials and the routing come from the kernels before this one
   const int warp = threadIdx.x >> 5;
   const int r0 = blockIdx.x * kRows;
-  // the assignment rows of this thread's first gather item, loaded before the weight stream
   const int nitems = kRows * T * k;
-  const int a0 = threadIdx.x < nitems ? inv[threadIdx.x / kRows] : 0;
   const int span = Is / KS;
   float acc[1][NG][4];
   const uint16_t* const W[1] = {wd};
-  skinny_mainloop<1, NG>(W, Is, r0, hb, 2, T, warp * span, (warp + 1) * span, acc);
+  if (span == 32 * U) {
+    // the weight slice is a constant of the layer: it streams in while the kernels before this one finish
+    uint4 av[U][1][2];
+    skinny_load_a<1, U>(W, Is, r0, warp * span, av);
+    pdl_wait();  // h, the routed partials and the routing come from the kernels before this one
+    skinny_finish<1, NG, U>(av, Is, hb, 2, T, warp * span, acc);
+  } else {
+    pdl_wait();
+    skinny_mainloop<1, NG>(W, Is, r0, hb, 2, T, warp * span, (warp + 1) * span, acc);
+  }
+  // the assignment rows of this thread's first gather item
+  const int a0 = threadIdx.x < nitems ? inv[threadIdx.x / kRows] : 0;
   skinny_store<1, NG>(red, acc);
   for (int i = threadIdx.x; i < nitems; i += blockDim.x) {
     const int r = i % kRows, a = i / kRows;

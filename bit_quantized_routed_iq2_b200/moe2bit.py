@@ -12,7 +12,8 @@ import os
 from dataclasses import dataclass
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-SO_PATH = os.path.join(_HERE, "libmoe2bit.so")
+# MOE2BIT_SO may name another build of the same library (the bounds-checked libmoe2bit_bc.so in its tests)
+SO_PATH = os.environ.get("MOE2BIT_SO") or os.path.join(_HERE, "libmoe2bit.so")
 
 MOE_F32, MOE_BF16 = 0, 1
 STATUS = {
@@ -28,7 +29,11 @@ STATUS = {
 EXPORTS = (
     "moe_workspace_size", "moe_route", "moe_expert_ffn", "moe_layer_forward", "moe_status_string",
     "moe_debug_dequant_iq2", "moe_debug_dequant_q2k", "moe_debug_grid", "moe_profile_enable", "moe_profile_read",
-    "moe_layer_forward_noalloc",
+    "moe_layer_forward_noalloc", "moe_read_status", "moe_read_status_noalloc", "moe_debug_inject",
+    "moe_debug_gemv_operands_iq2", "moe_debug_gemv_operands_q2k", "moe_debug_tc_operands_iq2",
+    "moe_debug_tc_operands_q2k", "moe_quantize_q2k", "moe_quantize_iq2",
+    "moe_prefetch_layer", "moe_debug_bounds_check_build", "moe_debug_bounds_violations",
+    "moe_cache_bytes", "moe_cache_create", "moe_cache_destroy", "moe_cache_read_stats", "moe_layer_forward_cached",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 KERNEL_NAMES = ("router_logits", "topk", "permute", "active", "gateup", "down", "shared_gateup", "shared_down",
@@ -44,6 +49,10 @@ class MoeError(RuntimeError):
 
 class Desc(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("hidden", "inter", "n_experts", "top_k", "shared_inter")]
+
+
+class CacheStats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("calls", "hits", "misses", "bytes_copied")]
 
 
 class Weights(ctypes.Structure):
@@ -78,9 +87,26 @@ def load() -> ctypes.CDLL:
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_debug_dequant_iq2.argtypes = [vp, vp, i64, vp, vp]
     L.moe_debug_dequant_q2k.argtypes = [vp, vp, i64, vp, vp]
+    L.moe_debug_gemv_operands_iq2.argtypes = [vp, i64, vp, vp, vp]
+    L.moe_debug_gemv_operands_q2k.argtypes = [vp, i64, vp, vp, vp]
+    L.moe_debug_tc_operands_iq2.argtypes = [vp, vp, i64, vp, vp]
+    L.moe_debug_tc_operands_q2k.argtypes = [vp, vp, i64, vp, vp]
+    L.moe_prefetch_layer.argtypes = [pd, pw, vp]
+    L.moe_debug_bounds_check_build.argtypes = []
+    L.moe_debug_bounds_violations.argtypes = [ctypes.POINTER(ctypes.c_uint64)]
+    L.moe_cache_bytes.argtypes = [pd, i32, ctypes.POINTER(sz)]
+    L.moe_cache_create.argtypes = [pd, pw, i32, vp, sz, ctypes.POINTER(vp)]
+    L.moe_cache_destroy.argtypes = [vp]
+    L.moe_cache_read_stats.argtypes = [vp, ctypes.POINTER(CacheStats)]
+    L.moe_layer_forward_cached.argtypes = [vp, pw, vp, i32, i32, vp, vp, vp, sz, vp]
+    L.moe_quantize_q2k.argtypes = [vp, i64, vp, vp, vp]
+    L.moe_quantize_iq2.argtypes = [vp, i64, vp, vp, vp]
     L.moe_debug_grid.argtypes = [vp]
     L.moe_debug_grid.restype = None
     L.moe_layer_forward_noalloc.argtypes = [pd, pw, vp, i32, i32, vp, vp, vp]
+    L.moe_read_status.argtypes = [vp, ctypes.POINTER(i32), vp]
+    L.moe_read_status_noalloc.argtypes = [ctypes.POINTER(i32), vp]
+    L.moe_debug_inject.argtypes = [i32, i64]
     L.moe_profile_enable.argtypes = [i32]
     L.moe_profile_read.argtypes = [vp, vp]
     for name in EXPORTS:
@@ -161,6 +187,52 @@ def debug_dequant_q2k(codes, dd, out, stream=None):
     _check(load().moe_debug_dequant_q2k(_ptr(codes), _ptr(dd), nb, _ptr(out), _stream(stream)), "moe_debug_dequant_q2k")
 
 
+def quantize_q2k(w, codes, dd, stream=None):
+    """fp32 device weights (numel % 256 == 0) -> Q2K codes [nb][80] u8 and dd [nb] (int32 view)."""
+    nb = w.numel() // 256
+    _check(load().moe_quantize_q2k(_ptr(w), nb, _ptr(codes), _ptr(dd), _stream(stream)), "moe_quantize_q2k")
+
+
+def quantize_iq2(w, codes, d, stream=None):
+    """fp32 device weights -> IQ2 codes [nb][64] u8 and d [nb] (int16 view of fp16 bits)."""
+    nb = w.numel() // 256
+    _check(load().moe_quantize_iq2(_ptr(w), nb, _ptr(codes), _ptr(d), _stream(stream)), "moe_quantize_iq2")
+
+
+def bounds_violations() -> int:
+    """Violations counted by the bounds-checked build since the last read (-1 from a normal build)."""
+    L = load()
+    if not L.moe_debug_bounds_check_build():
+        return -1
+    v = ctypes.c_uint64(0)
+    _check(L.moe_debug_bounds_violations(ctypes.byref(v)), "moe_debug_bounds_violations")
+    return int(v.value)
+
+
+def debug_gemv_operands_iq2(codes, w, odd, stream=None):
+    nb = codes.numel() // 64
+    _check(load().moe_debug_gemv_operands_iq2(_ptr(codes), nb, _ptr(w), _ptr(odd), _stream(stream)),
+           "moe_debug_gemv_operands_iq2")
+
+
+def debug_gemv_operands_q2k(codes, scq, m, stream=None):
+    nb = codes.numel() // 80
+    _check(load().moe_debug_gemv_operands_q2k(_ptr(codes), nb, _ptr(scq), _ptr(m), _stream(stream)),
+           "moe_debug_gemv_operands_q2k")
+
+
+def debug_tc_operands_iq2(codes, d, out, stream=None):
+    nb = codes.numel() // 64
+    _check(load().moe_debug_tc_operands_iq2(_ptr(codes), _ptr(d), nb, _ptr(out), _stream(stream)),
+           "moe_debug_tc_operands_iq2")
+
+
+def debug_tc_operands_q2k(codes, dd, out, stream=None):
+    nb = codes.numel() // 80
+    _check(load().moe_debug_tc_operands_q2k(_ptr(codes), _ptr(dd), nb, _ptr(out), _stream(stream)),
+           "moe_debug_tc_operands_q2k")
+
+
 @dataclass
 class DeviceLayer:
     """Device-resident planes of one layer (torch tensors) plus the ABI structs."""
@@ -225,6 +297,12 @@ def layer_forward(layer: DeviceLayer, x, residual, y, ws, stream=None):
                                     _stream(stream)), "moe_layer_forward")
 
 
+def prefetch_layer(layer: DeviceLayer, stream=None):
+    """L2 prefetch of the layer's router and shared expert (moe_prefetch_layer)."""
+    w = layer.weights
+    _check(load().moe_prefetch_layer(ctypes.byref(layer.desc), ctypes.byref(w), _stream(stream)), "moe_prefetch_layer")
+
+
 def layer_forward_noalloc(layer: DeviceLayer, x, residual, y, stream=None):
     """The whole layer with the library's own fixed scratch array (no workspace
     argument); see moe_layer_forward_noalloc in include/moe2bit.h."""
@@ -232,6 +310,98 @@ def layer_forward_noalloc(layer: DeviceLayer, x, residual, y, stream=None):
     w = layer.weights
     _check(load().moe_layer_forward_noalloc(ctypes.byref(layer.desc), ctypes.byref(w), _ptr(x), _dtype_of(x), T,
                                             _ptr(residual), _ptr(y), _stream(stream)), "moe_layer_forward_noalloc")
+
+
+def read_status(ws, stream=None) -> int:
+    """Device status word of the last call that used workspace `ws` (0 = MOE_OK);
+    synchronises `stream`."""
+    v = ctypes.c_int32(-1)
+    _check(load().moe_read_status(_ptr(ws), ctypes.byref(v), _stream(stream)), "moe_read_status")
+    return int(v.value)
+
+
+def read_status_noalloc(stream=None) -> int:
+    """Device status word of the last moe_layer_forward_noalloc on this device."""
+    v = ctypes.c_int32(-1)
+    _check(load().moe_read_status_noalloc(ctypes.byref(v), _stream(stream)), "moe_read_status_noalloc")
+    return int(v.value)
+
+
+def debug_inject(mode: int, wait_limit_cycles: int = 0):
+    """Fault injection for tests (see moe_debug_inject in include/moe2bit.h)."""
+    _check(load().moe_debug_inject(mode, wait_limit_cycles), "moe_debug_inject")
+
+
+class ExpertCache:
+    """Host-resident routed experts with `n_slots` of them cached on the GPU
+    (moe_cache_create in include/moe2bit.h). The host planes are copied once
+    into page-locked memory owned by this object; the slot memory is a device
+    tensor owned by this object."""
+
+    ROUTED = ("gate_codes", "gate_d", "up_codes", "up_d", "down_codes", "down_dd")
+
+    def __init__(self, lw, n_slots: int, device="cuda"):
+        import numpy as np
+        import torch
+
+        self.desc = desc_of(lw.H, lw.I, lw.E, lw.k, lw.Is)
+        self.host = {}
+        for name in self.ROUTED:
+            a = np.ascontiguousarray(getattr(lw, name))
+            self.host[name] = torch.from_numpy(a.view(np.uint8).reshape(-1)).pin_memory()
+        n = ctypes.c_size_t(0)
+        _check(load().moe_cache_bytes(ctypes.byref(self.desc), n_slots, ctypes.byref(n)), "moe_cache_bytes")
+        self.slot_mem = torch.empty(int(n.value), dtype=torch.uint8, device=device)
+        pool = Weights()
+        for name in self.ROUTED:
+            setattr(pool, name, self.host[name].data_ptr())
+        h = ctypes.c_void_p()
+        _check(load().moe_cache_create(ctypes.byref(self.desc), ctypes.byref(pool), n_slots, _ptr(self.slot_mem),
+                                       int(n.value), ctypes.byref(h)), "moe_cache_create")
+        self.handle = h
+        self.n_slots = n_slots
+
+    def forward(self, layer: "DeviceLayer", x, residual, y, ws, stream=None):
+        """The layer with the routed planes from the cache; `layer` supplies the
+        device router and shared expert."""
+        T = x.shape[0]
+        w = layer.weights
+        _check(load().moe_layer_forward_cached(self.handle, ctypes.byref(w), _ptr(x), _dtype_of(x), T, _ptr(residual),
+                                               _ptr(y), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+               "moe_layer_forward_cached")
+
+    def stats(self) -> dict:
+        st = CacheStats()
+        _check(load().moe_cache_read_stats(self.handle, ctypes.byref(st)), "moe_cache_read_stats")
+        return {n: int(getattr(st, n)) for n, _ in CacheStats._fields_}
+
+    def close(self):
+        if getattr(self, "handle", None):
+            load().moe_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def to_device_shared_only(lw, device="cuda") -> "DeviceLayer":
+    """Device copies of the router and shared expert only (the routed planes
+    stay on the host, for ExpertCache)."""
+    import numpy as np
+    import torch
+
+    def up(a, dt):
+        return None if a is None else torch.from_numpy(np.ascontiguousarray(a).view(dt)).to(device)
+
+    t = {"router_w": up(lw.router_w, np.int16),
+         "router_bias": None if lw.router_bias is None else up(lw.router_bias, np.float32),
+         "sh_gate": up(lw.sh_gate, np.int16) if lw.Is else None,
+         "sh_up": up(lw.sh_up, np.int16) if lw.Is else None,
+         "sh_down": up(lw.sh_down, np.int16) if lw.Is else None}
+    return DeviceLayer(desc_of(lw.H, lw.I, lw.E, lw.k, lw.Is), t)
 
 
 def alloc_workspace(desc: Desc, max_tokens: int, device="cuda"):

@@ -26,7 +26,8 @@
  *   - Pointers marked "device" must be device-accessible memory of the current
  *     CUDA device; "host" pointers are ordinary host memory. All buffers are
  *     owned by the caller. The library never allocates or frees device memory
- *     and never synchronises. Work is ordered on `stream`: it starts after the
+ *     and never synchronises (moe_read_status, a host query, is the one
+ *     exception). Work is ordered on `stream`: it starts after the
  *     work already enqueued there and finishes before anything enqueued later.
  *     moe_layer_forward may run part of it on a side stream that it forks from
  *     `stream` and joins back with events (created once per device and caller
@@ -197,17 +198,133 @@ MOE_API moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer
  *     MOE_ERR_WORKSPACE_TOO_SMALL before anything is enqueued; the size covers
  *     a 32-token decode batch at H=7168, I=2048, E=256, k=8, I_s=2048.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture. It allocates nothing, ever.
+ *     (cudaGetSymbolAddress, with that device current). Under lazy module
+ *     loading (the CUDA default) that first lookup is also when the driver
+ *     loads the library's module and commits the array's memory. The first
+ *     decode-path call (bf16 x, T <= 16) for each device and caller stream
+ *     also creates the side stream and three events described under
+ *     moe_layer_forward; they are kept, one set per distinct caller stream,
+ *     until the process exits. So make the first call for each device and
+ *     each caller stream during start-up, outside any stream capture; later
+ *     calls create nothing and allocate nothing.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind; the library clears whatever must start at zero itself. Calls
  *     that overlap on the GPU (other streams, other host threads) race on the
  *     array: serialise them.
+ *   - The device status of the last call is read with
+ *     moe_read_status_noalloc.
  */
 #define MOE_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 MOE_API moe_status moe_layer_forward_noalloc(const moe_layer_desc* desc, const moe_layer_weights* w,
                                              const void* x, moe_dtype x_dtype, int32_t T, const float* residual,
                                              float* y, void* stream);
+
+/*
+ * Prefetch of the weights a layer reads before (and regardless of) routing:
+ * the router and the shared expert ([Q]: both unquantized) are brought into
+ * L2 with an evict-last policy, so that a moe_layer_forward of this layer
+ * issued later finds them there. Meant for a chain of layers: while layer l
+ * runs, prefetch layer l+1 on another stream (the routed experts of l+1 are
+ * unknown until its router has run; they stream with an evict-first policy
+ * and do not displace the prefetched lines). Changes only cache state; reads
+ * E*H*2 + 3*I_s*H*2 bytes from HBM. Asynchronous on `stream`; capturable.
+ * MOE_ERR_INVALID_ARG for a null router or (I_s > 0) null shared weights.
+ */
+MOE_API moe_status moe_prefetch_layer(const moe_layer_desc* desc, const moe_layer_weights* weights, void* stream);
+
+/*
+ * Device-side status of the last call that used workspace `ws` (moe_route,
+ * moe_expert_ffn or moe_layer_forward). Every call's first kernel clears a
+ * status word at the head of its workspace; a kernel that gives up a bounded
+ * wait (about two seconds, or the limit set by moe_debug_inject) records
+ * MOE_ERR_TIMEOUT there and returns, and a kernel that finds an inconsistent
+ * launch (a misaligned shared-memory window, a tile outside its operand)
+ * records MOE_ERR_CUDA or MOE_ERR_INVALID_ARG. The first code recorded wins;
+ * the outputs of a call with a non-zero status are undefined.
+ * This call enqueues a 4-byte device-to-host copy on `stream` and waits for
+ * `stream` (it is the one call of this interface that synchronises); it
+ * writes the word to *status (host pointer). Returns MOE_ERR_INVALID_ARG for
+ * a null or misaligned `ws` or a null `status`, MOE_ERR_CUDA if the copy fails.
+ */
+MOE_API moe_status moe_read_status(const void* ws, int32_t* status, void* stream);
+
+/* The same for moe_layer_forward_noalloc: reads the status word at the head
+ * of the library's scratch array on the current device. */
+MOE_API moe_status moe_read_status_noalloc(int32_t* status, void* stream);
+
+/*
+ * Fault injection, a test aid (process-wide, not thread-safe; mode 0 = off).
+ * Mode 1: the decode gate/up GEMV's producer warp issues no weight loads, so
+ * its consumer warps wait on shared-memory barriers that never complete; with
+ * `wait_limit_cycles` as their bound they give up, record MOE_ERR_TIMEOUT in
+ * the call's status word and return. Nothing faults, traps or hangs; later
+ * kernels of the call run on undefined partial sums. The following call with
+ * mode 0 behaves normally again.
+ * Returns MOE_ERR_INVALID_ARG for an unknown mode or a negative limit.
+ */
+MOE_API moe_status moe_debug_inject(int32_t mode, int64_t wait_limit_cycles);
+
+/*
+ * Expert cache: the routed experts of one layer live in host memory and the
+ * GPU keeps `n_slots` of them ("ds4 : analyse pratique pour un usage
+ * documenté", section « Exécuter des modèles plus grands que la RAM avec le
+ * streaming SSD »: non-routed weights stay resident while routed experts are
+ * kept in a cache and loaded on a miss; here host memory plays the SSD's part
+ * and HBM the cache's).
+ *   moe_cache_bytes: device bytes of the slot memory for n_slots
+ *     (1 <= n_slots <= n_experts): the six routed planes of n_slots experts
+ *     plus an expert -> slot map.
+ *   moe_cache_create: `host_pool` names the routed planes of all E experts in
+ *     the layout of moe_layer_weights, in page-locked host memory
+ *     (cudaHostAlloc / cudaHostRegister) that stays valid and unchanged for the
+ *     life of the cache; its router and shared fields are ignored. `slot_mem`
+ *     is caller-owned device memory of slot_mem_bytes >= moe_cache_bytes on the
+ *     current device. Creates a host object (the one host allocation of this
+ *     interface); destroy it with moe_cache_destroy. inter % 256 == 0 required.
+ *   moe_layer_forward_cached: the whole layer (same meaning and results as
+ *     moe_layer_forward, bit for bit) with the routed planes taken from the
+ *     cache: it routes, waits for the routing (this call synchronises `stream`
+ *     once and cannot be captured in a CUDA graph), keeps the experts already
+ *     in a slot (hits), copies each missing expert from the host pool into an
+ *     empty slot or the least recently used slot that this call does not need
+ *     (cudaMemcpyAsync on `stream`), maps the routing to slot ids and runs the
+ *     expert FFN over the slots. `weights` supplies the device router and
+ *     shared expert (its routed fields are ignored). Returns
+ *     MOE_ERR_WORKSPACE_TOO_SMALL, after the routing only, when one call needs
+ *     more distinct experts than there are slots (at most min(E, T * k)).
+ *     Not thread-safe per cache; calls on one cache must use one device.
+ *   moe_cache_read_stats: calls, hits and misses (experts), bytes copied.
+ */
+typedef struct moe_expert_cache moe_expert_cache;
+typedef struct {
+  int64_t calls;
+  int64_t hits;
+  int64_t misses;
+  int64_t bytes_copied;
+} moe_cache_stats;
+MOE_API moe_status moe_cache_bytes(const moe_layer_desc* desc, int32_t n_slots, size_t* bytes);
+MOE_API moe_status moe_cache_create(const moe_layer_desc* desc, const moe_layer_weights* host_pool, int32_t n_slots,
+                                    void* slot_mem, size_t slot_mem_bytes, moe_expert_cache** out);
+MOE_API moe_status moe_cache_destroy(moe_expert_cache* cache);
+MOE_API moe_status moe_cache_read_stats(const moe_expert_cache* cache, moe_cache_stats* stats);
+MOE_API moe_status moe_layer_forward_cached(moe_expert_cache* cache, const moe_layer_weights* weights, const void* x,
+                                            moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws,
+                                            size_t ws_bytes, void* stream);
+
+/*
+ * Bounds-checked build, a test aid standing in for a memory checker: the
+ * library can be built a second time with -DMOE_BOUNDS_CHECK
+ * (libmoe2bit_bc.so). In that build every shared-memory load of the decode
+ * GEMVs checks its address against the CTA's dynamic shared memory and its
+ * alignment, and every partial-sum store and TMA box its buffer; a violation
+ * is counted and the access skipped (loads return zeros), nothing traps.
+ *   moe_debug_bounds_check_build: 1 in that build, 0 otherwise.
+ *   moe_debug_bounds_violations: the count since the last read (then reset to
+ *     0), after the caller's synchronisation; MOE_ERR_UNSUPPORTED_SHAPE with
+ *     *count = 0 from a normal build.
+ */
+MOE_API int32_t moe_debug_bounds_check_build(void);
+MOE_API moe_status moe_debug_bounds_violations(uint64_t* count);
 
 /* Static, NUL-terminated name of a status code. */
 MOE_API const char* moe_status_string(moe_status s);
@@ -222,6 +339,65 @@ MOE_API moe_status moe_debug_dequant_iq2(const uint8_t* codes, const uint16_t* d
                                  void* stream);
 MOE_API moe_status moe_debug_dequant_q2k(const uint8_t* codes, const uint32_t* dd, int64_t nblocks, float* out,
                                  void* stream);
+
+/*
+ * Quantisers: float weights -> the block formats above, without an importance
+ * matrix ([Q]: the routed experts are quantized, up/gate IQ2_XXS-style, down
+ * Q2_K-style; the pages give no algorithm, these plain rules are the
+ * library's). `w` holds nblocks * 256 fp32 weights (device, 16-byte aligned),
+ * blocks along the flattened array exactly as the planes above (for a
+ * [rows][K] matrix with K % 256 == 0, block i is row i / (K/256)). Outputs are
+ * device planes of nblocks entries. Decisions are taken in fp32 with
+ * round-to-nearest-even operations, never fused, in the order written, so the
+ * bytes are reproducible by any correct implementation of the rule.
+ *   moe_quantize_q2k: per 16-weight sub-block lo = min(0, min w), hi = max w,
+ *     step = (hi - lo) / 3, off = -lo; d = fp16(max step / 15),
+ *     dmin = fp16(max off / 15); sc = clamp(rint(step / d), 0, 15),
+ *     m = clamp(rint(off / dmin), 0, 15) (0 when the divisor is 0);
+ *     q = clamp(rint((w + dmin * m) / (d * sc)), 0, 3) (0 when d * sc is 0).
+ *   moe_quantize_iq2: d = fp16(max |w| * 8 / 1333); per 32-weight sub-block
+ *     ls = clamp(rint((max |w| * 8 / (d * 43) - 1) / 2), 0, 15),
+ *     c = d * (2 ls + 1) / 8; per group of 8 the signs of w, with the element
+ *     of smallest |w| (lowest index on ties) flipped when the count of negatives
+ *     is odd; the codebook row minimising sum_e (|w_e| -+ c * grid[row][e])^2
+ *     (e ascending; + for the flipped element), the lower row on ties. A block
+ *     whose d rounds to 0 gets all-zero codes.
+ * Weights must be finite with every scale below 65504 (fp16). Asynchronous on
+ * `stream`; MOE_ERR_INVALID_ARG for null or misaligned pointers or a negative
+ * count.
+ */
+MOE_API moe_status moe_quantize_q2k(const float* w, int64_t nblocks, uint8_t* codes, uint32_t* dd, void* stream);
+MOE_API moe_status moe_quantize_iq2(const float* w, int64_t nblocks, uint8_t* codes, uint16_t* d, void* stream);
+
+/*
+ * The layer's own operand builders exposed for exact tests (same device
+ * functions and lookup tables as the hot kernels; every lane of a warp uses
+ * its own table replica, as in the kernels). `nblocks` 256-weight blocks.
+ *
+ * Decode GEMVs (int8 MMA operands):
+ *   moe_debug_gemv_operands_iq2: w[256 b + 32 s + 8 j + e] = level * sign of
+ *     weight e of group j of sub-block s (int8, device out [nblocks*256]) and
+ *     odd[8 b + s] = 2 ls + 1 (u8, device out [nblocks*8]); the weight is then
+ *     d * odd * w / 8.
+ *   moe_debug_gemv_operands_q2k: scq[256 b + i] = sc * q of weight i (int16,
+ *     device out [nblocks*256]) and m[16 b + s] (u8, [nblocks*16]); the weight
+ *     is then d * scq - dmin * m.
+ * Grouped GEMM (fp16 operands stored into tensor memory, weights in K order):
+ *   moe_debug_tc_operands_iq2: out[256 b + i] = fp16 bits of
+ *     sign * fp16(fp16(d * (2 ls + 1) * 2^10 / 8) * level), i.e. the weight
+ *     times 2^10 with one rounding of the scale and one of the product.
+ *   moe_debug_tc_operands_q2k: out[256 b + i] = fp16 bits of the weight's fp32
+ *     value d * sc * q - dmin * m rounded to fp16.
+ * codes: device, 16-byte aligned (IQ2) / any (Q2K); d, dd: device planes.
+ */
+MOE_API moe_status moe_debug_gemv_operands_iq2(const uint8_t* codes, int64_t nblocks, int8_t* w, uint8_t* odd,
+                                               void* stream);
+MOE_API moe_status moe_debug_gemv_operands_q2k(const uint8_t* codes, int64_t nblocks, int16_t* scq, uint8_t* m,
+                                               void* stream);
+MOE_API moe_status moe_debug_tc_operands_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, uint16_t* out,
+                                             void* stream);
+MOE_API moe_status moe_debug_tc_operands_q2k(const uint8_t* codes, const uint32_t* dd, int64_t nblocks,
+                                             uint16_t* out, void* stream);
 
 /*
  * Kernel timing, a profiling aid (off by default; not thread-safe). While

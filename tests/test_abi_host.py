@@ -93,3 +93,33 @@ def test_misaligned_and_small_workspace_rejected(lib):
     assert lib.moe_layer_forward(ctypes.byref(d), ctypes.byref(w), fake + 2, 1, 1, None, fake, fake, need, None) == 1
     # workspace too small
     assert lib.moe_layer_forward(ctypes.byref(d), ctypes.byref(w), fake, 1, 1, None, fake, fake, need - 1, None) == 3
+
+
+def test_status_query_and_injection_validate_on_host(lib):
+    """The status query and the fault-injection switch reject bad arguments
+    without touching a device; injection mode 0 is plain host state."""
+    v = ctypes.c_int32(0)
+    assert lib.moe_read_status(None, ctypes.byref(v), None) == 1
+    assert lib.moe_read_status((1 << 40) + 4, ctypes.byref(v), None) == 1  # misaligned workspace
+    assert lib.moe_read_status(1 << 40, None, None) == 1
+    assert lib.moe_read_status_noalloc(None, None) == 1
+    assert lib.moe_debug_inject(2, 0) == 1
+    assert lib.moe_debug_inject(1, -1) == 1
+    assert lib.moe_debug_inject(0, 0) == 0
+
+
+def test_cache_arguments_validate_on_host(lib):
+    d = moe2bit.desc_of(**DECODE)
+    n = ctypes.c_size_t(0)
+    assert lib.moe_cache_bytes(ctypes.byref(d), 0, ctypes.byref(n)) == 1
+    assert lib.moe_cache_bytes(ctypes.byref(d), 257, ctypes.byref(n)) == 1
+    assert lib.moe_cache_bytes(ctypes.byref(d), 8, ctypes.byref(n)) == 0
+    per_expert = 2 * 2048 * 7168 // 256 * (64 + 2) + 7168 * 2048 // 256 * (80 + 4)
+    assert n.value >= 8 * per_expert
+    h = ctypes.c_void_p()
+    w = moe2bit.Weights()
+    assert lib.moe_cache_create(ctypes.byref(d), ctypes.byref(w), 8, None, n.value, ctypes.byref(h)) == 1
+    assert lib.moe_cache_create(ctypes.byref(d), None, 8, 1 << 40, n.value, ctypes.byref(h)) == 1
+    assert lib.moe_cache_create(ctypes.byref(d), ctypes.byref(w), 8, 1 << 40, n.value - 1, ctypes.byref(h)) == 3
+    assert lib.moe_layer_forward_cached(None, ctypes.byref(w), None, 1, 1, None, None, None, 0, None) == 1
+    assert lib.moe_cache_read_stats(None, None) == 1

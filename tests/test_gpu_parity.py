@@ -10,7 +10,7 @@ import oracle
 import synth
 from bit_quantized_routed_iq2_b200 import build as moebuild
 from bit_quantized_routed_iq2_b200 import moe2bit
-from helpers import FFN_TOL, TOPK_W_TOL, normwise, screened_x
+from helpers import FFN_TOL, TOPK_W_TOL, elementwise, normwise, screened_x
 
 pytestmark = pytest.mark.gpu
 
@@ -158,14 +158,14 @@ SMALL_CASES = {
     "flat_blocks_k1": _small(H=256, I=64, E=4, k=1, Is=32, T=9, seed=0x5A14),
     "single_expert": _small(E=1, k=1, Is=0, T=5, seed=0x5A15),
     "k_eq_E": _small(E=4, k=4, T=7, seed=0x5A16),
-    # shapes served by the TMA-fed GEMVs (H % 1024 == 0, I % 512 == 0; T <= 4 unless the
-    # tensor-core path cannot take the shape)
+    # shapes served by the TMA-fed GEMVs (H % 1024 == 0, I % 512 == 0, T <= 16; above 16 tokens the
+    # tensor-core grouped GEMM takes over)
     "tma_t1": _small(H=1024, I=512, E=16, k=4, Is=64, T=1, seed=0x5A17),
     "tma_t5": _small(H=2048, I=1024, E=8, k=4, Is=128, T=5, seed=0x5A18),
     "tma_t16": _small(H=1024, I=512, E=8, k=4, Is=64, T=16, seed=0x5A19),
     "tma_t16_zipf_f32": _small(H=1024, I=1024, E=12, k=3, Is=0, T=16, x_dtype="f32", zipf=True, seed=0x5A1A),
     "tma_t3_shared_experts": _small(H=1024, I=512, E=4, k=4, Is=128, T=3, seed=0x5A20),
-    # shapes served by the tensor-core grouped GEMM (T > 4, H, I multiples of 256, I_s of 128)
+    # shapes served by the tensor-core grouped GEMM (T > 16, H, I multiples of 256, I_s of 128)
     "tc_t17": _small(H=512, I=256, E=4, k=2, Is=128, T=17, seed=0x5A1B),
     "tc_t64_f32": _small(H=1024, I=512, E=8, k=2, Is=256, T=64, x_dtype="f32", seed=0x5A1C),
     "tc_t200_zipf": _small(H=768, I=512, E=16, k=4, Is=0, T=200, zipf=True, seed=0x5A1D),
@@ -190,6 +190,17 @@ def test_route_small(torch_cuda, name):
     _check_route(torch_cuda, cfg, lw, moe2bit.to_device(lw), x)
 
 
+# Normwise and element-wise errors of every layer comparison, written out as a
+# JSON report when MOE_PARITY_REPORT names a file (the element-wise figure uses a
+# floor of 1e-3 * max |y_ref|; the bound asserted is the normwise one).
+REPORT = {}
+
+
+def _record(name, y, ref):
+    REPORT[name] = {"normwise": normwise(y, ref), "elementwise_floor_1e-3": elementwise(y, ref)}
+    return REPORT[name]["normwise"]
+
+
 @pytest.mark.parametrize("name", list(SMALL_CASES))
 def test_layer_forward_small(torch_cuda, name):
     cfg = SMALL_CASES[name]
@@ -199,7 +210,7 @@ def test_layer_forward_small(torch_cuda, name):
     dl = moe2bit.to_device(lw)
     y = _forward_gpu(torch_cuda, dl, x, res)
     ref, _, _ = oracle.layer_forward(lw, x, res)
-    assert normwise(y, ref) <= FFN_TOL
+    assert _record(name, y, ref) <= FFN_TOL
     # residual may alias the output
     y2 = _forward_gpu(torch_cuda, dl, x, res, alias=True)
     assert np.array_equal(y2, y)
@@ -247,33 +258,92 @@ def test_zero_tokens_is_noop(torch_cuda):
     torch.cuda.synchronize()
 
 
+# ------------------------------------------------------- outlier activations
+# One large element (+-64) per 256-element block among N(0,1) values: the
+# decode GEMVs quantise x in 256-element blocks (the outlier sets the block's
+# scale) and the grouped GEMM scales each token by one power of two.
+OUTLIER_CASES = {
+    "outlier_gemv_t1": _small(H=1024, I=512, E=16, k=4, Is=64, T=1, seed=0x5A40),
+    "outlier_gemv_t6": _small(H=2048, I=1024, E=8, k=4, Is=128, T=6, seed=0x5A41),
+    "outlier_gemm_t40": _small(H=1024, I=512, E=8, k=2, Is=128, T=40, seed=0x5A42),
+    "outlier_gemm_t40_f32": _small(H=1024, I=512, E=8, k=2, Is=128, T=40, x_dtype="f32", seed=0x5A43),
+}
+
+
+@pytest.mark.parametrize("name", list(OUTLIER_CASES))
+def test_layer_forward_outliers(torch_cuda, name):
+    cfg = OUTLIER_CASES[name]
+    lw = synth.make_layer(cfg)
+    x = screened_x(cfg, lw, outliers=True)
+    _check_route(torch_cuda, cfg, lw, moe2bit.to_device(lw), x)
+    y = _forward_gpu(torch_cuda, moe2bit.to_device(lw), x)
+    ref, _, _ = oracle.layer_forward(lw, x)
+    assert _record(name, y, ref) <= FFN_TOL
+
+
 # ------------------------------------------------------- full-size configs
-def _full_case(torch, name, sample_tokens):
+def _full_case(torch, name):
+    """The whole workload against the oracle: routing bit-exact for every token,
+    every token's output within the normwise bound (the oracle runs on all host
+    cores; each output is still one sequential double loop)."""
     cfg = synth.CONFIGS[name]
     lw = synth.make_layer(cfg)
     x = screened_x(cfg, lw)
     dl = moe2bit.to_device(lw)
     _check_route(torch, cfg, lw, dl, x)
     y = _forward_gpu(torch, dl, x)
-    for t in sample_tokens:
-        ref, _, _ = oracle.layer_forward(lw, np.ascontiguousarray(x[t:t + 1]))
-        assert normwise(y[t:t + 1], ref) <= FFN_TOL, (name, t)
+    ref, _, _ = oracle.layer_forward(lw, x)
+    _record(name, y, ref)
+    per_token = [normwise(y[t:t + 1], ref[t:t + 1]) for t in range(cfg.T)]
+    assert max(per_token) <= FFN_TOL, (name, int(np.argmax(per_token)), max(per_token))
     return y
 
 
 @pytest.mark.slow
 def test_full_decode1(torch_cuda):
-    _full_case(torch_cuda, "decode1", [0])
+    _full_case(torch_cuda, "decode1")
 
 
 @pytest.mark.slow
 def test_full_decode32(torch_cuda):
-    _full_case(torch_cuda, "decode32", [0, 17, 31])
+    _full_case(torch_cuda, "decode32")
 
 
 @pytest.mark.slow
-def test_full_prefill_sampled(torch_cuda):
-    _full_case(torch_cuda, "prefill", [0, 1023, 2047])
+def test_full_prefill_every_token(torch_cuda):
+    _full_case(torch_cuda, "prefill")
+
+
+@pytest.mark.slow
+def test_full_stack_two_layers_teacher_forced(torch_cuda):
+    """The 8-layer stack's shapes (16 tokens, H=7168, E=256, Zipf routing): two
+    chained layers, each checked against the oracle on the exact bf16 input and
+    fp32 residual the GPU saw (teacher-forced), output written over the
+    residual in place, as the stack step runs."""
+    torch = torch_cuda
+    cfg = synth.CONFIGS["stack"]
+    layers = [synth.make_layer(cfg, layer=l) for l in range(2)]
+    x = screened_x(cfg, layers[0])
+    res = synth.make_residual(cfg, cfg.T)
+    y = torch.from_numpy(np.ascontiguousarray(res)).cuda()
+    ws = moe2bit.alloc_workspace(moe2bit.to_device(layers[0]).desc, cfg.T)
+    for l, lw in enumerate(layers):
+        dl = moe2bit.to_device(lw)
+        res_in = y.cpu().numpy().copy()
+        _, _, logits = oracle.route(lw.router_w, lw.router_bias, x, cfg.k, want_logits=True)
+        srt = -np.sort(-logits, axis=1)
+        keep = (srt[:, cfg.k - 1] - srt[:, cfg.k]) >= 1e-4  # tokens whose routing fp32 cannot flip
+        idx, _, off, _, _ = _route_gpu(torch, dl, x, cfg.T, cfg.E, cfg.k)
+        ridx, _ = oracle.route(lw.router_w, lw.router_bias, x, cfg.k)
+        assert np.array_equal(idx[keep], ridx[keep]), l
+        moe2bit.layer_forward(dl, _x_dev(torch, x), y, y, ws)
+        torch.cuda.synchronize()
+        out = y.cpu().numpy()
+        ref, _, _ = oracle.layer_forward(lw, x, res_in)
+        assert keep.sum() >= cfg.T // 2, l
+        assert _record(f"stack_layer{l}", out[keep], ref[keep]) <= FFN_TOL, l
+        b = out.view(np.uint32)
+        x = ((b + 0x7FFF + ((b >> 16) & 1)) >> 16).astype(np.uint16)  # next input: bf16 (RNE) of the stream
 
 
 def test_layer_chain_teacher_forced(torch_cuda):
@@ -306,3 +376,14 @@ def test_layer_chain_teacher_forced(torch_cuda):
         # the next layer's input: the residual stream rounded to bf16 (round to nearest even)
         b = out.view(np.uint32)
         x = ((b + 0x7FFF + ((b >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def test_zz_write_parity_report():
+    """Writes the collected error figures (only when MOE_PARITY_REPORT is set)."""
+    import json
+    import os
+
+    path = os.environ.get("MOE_PARITY_REPORT")
+    if path:
+        with open(path, "w") as f:
+            json.dump(REPORT, f, indent=1, sort_keys=True)

@@ -41,6 +41,10 @@ CASES = {
     "tiny": synth.CONFIGS["tiny"],
     "small": synth.Config("small", 37, 512, 256, 16, 4, 64, "bf16", 1.0, False, 1, 0x5A11),
     "decode32": synth.CONFIGS["decode32"],
+    # the decode path (bf16, T <= 16): TMA-fed GEMVs and the shared expert on the side stream, which
+    # writes its part of the scratch while routing runs on the caller's stream
+    "decode_t1": synth.Config("decode_t1", 1, 7168, 2048, 16, 8, 2048, "bf16", 1.0, False, 1, 0x5A31),
+    "decode_t8": synth.Config("decode_t8", 8, 7168, 2048, 16, 8, 2048, "bf16", 1.0, True, 1, 0x5A32),
 }
 
 
@@ -61,6 +65,7 @@ def test_noalloc_matches_workspace_entry_point(torch_cuda, name):
         y = torch.full((cfg.T, cfg.H), float("nan"), dtype=torch.float32, device="cuda")
         moe2bit.layer_forward_noalloc(dl, xd, res, y)
         torch.cuda.synchronize()
+        assert moe2bit.read_status_noalloc() == 0
         outs.append(y.cpu().numpy())
     ref = y_ref.cpu().numpy()
     for got in outs:
