@@ -477,6 +477,7 @@ size_t fast_ffn_workspace_bytes(const LayerShape& s, int T) {
 // Side stream and fork/join events per (device, caller stream), created on first use.
 struct SideCtx {
   cudaStream_t st = nullptr;
+  // fork: caller -> side; digits: x digits ready; join: shared h ready
   cudaEvent_t fork = nullptr, digits = nullptr, join = nullptr;
 };
 static SideCtx* side_ctx(cudaStream_t st) {
@@ -527,14 +528,6 @@ int launch_shared_early(const LayerShape& s, const WeightPtrs& w, const void* x,
   {
     ProfScope ps(MOE_K_SHARED_GATEUP, c->st);
     rc = launch_shared_gateup_mma(s.H, s.Is, w.sh_gate, w.sh_up, static_cast<const uint16_t*>(x), 1, T, fw.hb, c->st);
-  }
-  // the shared down weights are known now too: bring them into L2 while routing and the routed GEMVs run, so
-  // the combine at the end of the step reads them from there (the bytes still come from HBM in this step);
-  // the prefetch only issues requests, so joining after it costs the combine nothing
-  if (rc == OK) {
-    const void* pp[1] = {w.sh_down};
-    const size_t nn[1] = {static_cast<size_t>(s.H) * s.Is * 2};
-    rc = launch_l2_prefetch(pp, nn, 1, c->st);
   }
   if (cudaEventRecord(c->join, c->st) != cudaSuccess) return ERR_CUDA;
   return rc;
@@ -638,9 +631,11 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
       SideCtx* c = side_ctx(st);
       if (!c || cudaStreamWaitEvent(st, c->join, 0) != cudaSuccess) return ERR_CUDA;
     }
-    ProfScope ps(MOE_K_COMBINE, st);
-    rc |= launch_shared_down_combine_mma(s.H, s.Is, w.sh_down, fw.hb, T, s.k, r.topk_w, r.inv, obuf, DP, residual,
-                                         y, st);
+    {
+      ProfScope ps(MOE_K_COMBINE, st);
+      rc |= launch_shared_down_combine_mma(s.H, s.Is, w.sh_down, fw.hb, T, s.k, r.topk_w, r.inv, obuf, DP,
+                                           residual, y, st);
+    }
   } else {
     ProfScope ps(MOE_K_COMBINE, st);
     const int grid = (s.H + 7) / 8;

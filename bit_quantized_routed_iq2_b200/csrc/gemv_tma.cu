@@ -44,7 +44,6 @@
 namespace moe {
 namespace {
 
-__device__ const Iq2SelTables d_sel_tables2 = make_sel_tables();
 
 constexpr int kCW = 16;                      // consumer warps (16 rows each)
 constexpr int kThreadsT = (kCW + 1) * 32;    // + one producer warp
@@ -271,14 +270,29 @@ __device__ __forceinline__ float half_lo(uint32_t w) { return half_bits_to_float
 __device__ __forceinline__ float half_hi(uint32_t w) { return half_bits_to_float(static_cast<uint16_t>(w >> 16)); }
 
 
-// The selector tables at the start of dynamic shared memory: row i (256 bytes)
-// holds the level word of grid row i at bytes 0..127 and the sign word of sign
-// field i mod 128 at bytes 128..255, each replicated for the 32 lanes.
-__device__ __forceinline__ void fill_sel_tables(uint32_t* tab, int tid, int nthr) {
-  for (int i = tid; i < kTabBytes / 4; i += nthr) {
+// The selector tables as they sit at the start of dynamic shared memory: row
+// i (256 bytes) holds the level word of grid row i at bytes 0..127 and the
+// sign word of sign field i mod 128 at bytes 128..255, each replicated for the
+// 32 lanes. Built at compile time; a kernel brings the 64 KB in with one bulk
+// asynchronous copy instead of thousands of dependent loads.
+struct SelRep {
+  uint32_t w[kTabBytes / 4];
+};
+constexpr SelRep make_sel_rep() {
+  const Iq2SelTables t = make_sel_tables();
+  SelRep r{};
+  for (int i = 0; i < kTabBytes / 4; ++i) {
     const int ent = i >> 6;
-    tab[i] = (i & 32) == 0 ? d_sel_tables2.level[ent] : d_sel_tables2.sign[ent & 127];
+    r.w[i] = (i & 32) == 0 ? t.level[ent] : t.sign[ent & 127];
   }
+  return r;
+}
+// (not const: it must live in global memory, the source of a bulk copy)
+__device__ __align__(128) SelRep g_sel_rep = make_sel_rep();
+
+// Word-by-word copy of the same tables (the debug kernel's path).
+__device__ __forceinline__ void fill_sel_tables(uint32_t* tab, int tid, int nthr) {
+  for (int i = tid; i < kTabBytes / 4; i += nthr) tab[i] = g_sel_rep.w[i];
 }
 
 // Word of the selector tables at byte offset `off` of dynamic shared memory
@@ -546,7 +560,7 @@ __host__ __device__ inline GuPlan gu_plan(int E, int T, int k, int H, bool xs_in
   const size_t end = p.xs + (xs_in ? align_up(static_cast<size_t>(T) * (H / 256) * 4, 128) : 0);
   p.ring = align_up(end, 1024);
   p.bars = p.ring + static_cast<size_t>(S) * kGuBox;
-  p.total = p.bars + 2 * static_cast<size_t>(S) * 8;
+  p.total = p.bars + (2 * static_cast<size_t>(S) + 1) * 8;  // full[S], empty[S], the table copy
   return p;
 }
 
@@ -576,14 +590,18 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
     if (tid == 0) atomicCAS(a.err, 0, ERR_CUDA);
     return;
   }
+  uint64_t* tabbar = empty + S;
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kCW);
     }
+    mbar_init(tabbar, 1);
     fence_barrier_init();
+    // the selector tables: one 64 KB bulk copy, in flight while the rest of the prologue runs
+    mbar_arrive_expect_tx(tabbar, kTabBytes);
+    bulk_copy_g2s(smem + pl.tab, &g_sel_rep, kTabBytes, tabbar);
   }
-  fill_sel_tables(reinterpret_cast<uint32_t*>(smem + pl.tab), tid, kThreadsT);
   for (int i = tid; i < kZeroBytes / 16; i += kThreadsT) reinterpret_cast<uint4*>(zero)[i] = make_uint4(0, 0, 0, 0);
   pdl_wait();  // routing and activations come from the kernels before this one
   load_meta(ms, a.offsets, a.active, a.perm, a.E, nA, a.k, tid, kThreadsT);
@@ -622,6 +640,8 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
     return;
   }
 
+  // the table copy must have landed before the first lookup (the producer never reads it)
+  if (!mbar_wait_bounded(tabbar, 0, a.err, ERR_TIMEOUT, a.wait_limit)) return;
   GuCtx c;
   c.tab = reinterpret_cast<const char*>(smem + pl.tab);
   c.ring = ring;

@@ -235,8 +235,9 @@ __device__ __forceinline__ void dq_iq2_sub(uint2 rec, float dsc, uint32_t tabL, 
 __device__ __forceinline__ void dq_q2k_sub(uint32_t w, uint32_t scb, float d, float dmin, uint32_t tabQ,
                                            uint32_t (&o)[8]) {
   const float A = d * static_cast<float>(scb & 15u), B = dmin * static_cast<float>(scb >> 4);
-  // q = 0 gives 0 - B (not -B): +0 when dmin * m is 0, as the fp32 weight d*sc*0 - dmin*0 is
-  const uint32_t tlo = f2_to_h2(__fsub_rn(0.f, B), A - B), thi = f2_to_h2(2.f * A - B, 3.f * A - B);
+  // q = 0 is evaluated as (d*sc)*0 - dmin*m, not -dmin*m: a zero weight then has the sign IEEE
+  // arithmetic gives the rule's expression (it follows the signs of d and dmin)
+  const uint32_t tlo = f2_to_h2(__fsub_rn(__fmul_rn(A, 0.f), B), A - B), thi = f2_to_h2(2.f * A - B, 3.f * A - B);
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     const uint32_t ent = b == 0 ? w * 128u : __umulhi(w, 1u << (39 - 8 * b));  // byte b at bits 7..14

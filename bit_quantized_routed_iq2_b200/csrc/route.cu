@@ -380,20 +380,10 @@ __global__ void __launch_bounds__(1024) topk_permute_small_kernel(const float* _
 }
 
 // Decode routing for at most 32 assignments (T*k <= 32, E <= 32*EPL) in one
-// warp. Top-k of each token: lane l holds the logits of experts l, l+32, ...;
-// each of the k rounds takes the warp maximum of an order-preserving integer
-// image of the logits with one redux.sync, then the lowest expert index
-// holding it with a second one (expert 32 i + l of the lane's smallest such
-// slot i is itself the key, so ties go to the lower index). Then, with the n
-// chosen experts broadcast once into every lane's registers: the offsets as
-// counts of smaller expert indices, each assignment's stable rank among equal
-// experts, and the active list by ballot prefix sums. Same outputs as
-// topk_permute_small_kernel, without block barriers or shared atomics.
-__device__ __forceinline__ uint32_t ordered_bits(float v) {
-  const uint32_t b = __float_as_uint(v);
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-
+// warp: the top-k of each token in turn, then (lane j = assignment j) the
+// offsets as counts of smaller expert indices, the stable rank among equal
+// experts by match, and the active list by ballot prefix sums. Same outputs
+// as topk_permute_small_kernel, without block barriers or shared atomics.
 template <int EPL>
 __global__ void __launch_bounds__(32) topk_permute_warp_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                                int32_t* __restrict__ topk_idx,
@@ -401,52 +391,21 @@ __global__ void __launch_bounds__(32) topk_permute_warp_kernel(const float* __re
                                                                int32_t* __restrict__ offsets,
                                                                int32_t* __restrict__ perm, int32_t* __restrict__ inv,
                                                                int32_t* __restrict__ active) {
+  __shared__ int idx_s[32];
   pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x;
   const int n = T * k;
-  int my_e = 0x7fffffff;  // expert of assignment `lane` (above every expert index when lane >= n)
-  for (int t = 0; t < T; ++t) {
-    const float* lrow = logits + static_cast<size_t>(t) * E;
-    uint32_t key[EPL];
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      const float v = e < E ? lrow[e] : -INFINITY;
-      key[i] = e < E ? (v == v ? ordered_bits(v) : ordered_bits(-INFINITY)) : 0u;  // NaN ranks with -inf
-    }
-    float chosen0 = 0.f, z = 0.f, wv = 0.f;
-    for (int j = 0; j < k; ++j) {
-      uint32_t m = 0;
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) m = max(m, key[i]);
-      m = __reduce_max_sync(0xffffffffu, m);
-      uint32_t cand = 0xffffffffu;
-#pragma unroll
-      for (int i = EPL - 1; i >= 0; --i)
-        if (key[i] == m && lane + 32 * i < E) cand = static_cast<uint32_t>(lane + 32 * i);
-      const int win = static_cast<int>(__reduce_min_sync(0xffffffffu, cand));
-      if ((win & 31) == lane) key[win >> 5] = 0u;  // taken
-      // the winner's logit, decoded from its key (exact: the map is a bijection)
-      const uint32_t vb = (m & 0x80000000u) ? (m & 0x7fffffffu) : ~m;
-      const float v = __uint_as_float(vb);
-      if (j == 0) chosen0 = v;
-      const float ex = expf(v - chosen0);
-      z += ex;
-      if (lane == j) wv = ex;
-      if (lane == t * k + j) my_e = win;
-      if (lane == 0) topk_idx[static_cast<size_t>(t) * k + j] = win;
-    }
-    if (lane < k) topk_w[static_cast<size_t>(t) * k + lane] = wv / z;
-  }
-  // every lane gets all n chosen experts
-  int es[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) es[j] = __shfl_sync(0xffffffffu, my_e, j);
-  // assignment `lane`: position = (assignments with a smaller expert) + (earlier ones with the same expert)
-  int p = 0;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) p += (j < n && (es[j] < my_e || (es[j] == my_e && j < lane))) ? 1 : 0;
+  for (int t = 0; t < T; ++t)
+    topk_warp<EPL>(logits + static_cast<size_t>(t) * E, E, k, topk_idx + static_cast<size_t>(t) * k,
+                   topk_w + static_cast<size_t>(t) * k, idx_s + t * k);
+  __syncwarp();
+  const int e = lane < n ? idx_s[lane] : 0x7fffffff;  // above every expert index
+  // assignment j: position = (assignments with a smaller expert) + (earlier ones with the same expert)
+  int below = 0;
+  for (int j = 0; j < n; ++j) below += __shfl_sync(0xffffffffu, e, j) < e ? 1 : 0;
+  const unsigned same = __match_any_sync(0xffffffffu, e);
+  const int p = below + __popc(same & ((1u << lane) - 1u));
   if (lane < n) {
     perm[p] = lane;
     inv[lane] = p;
@@ -456,16 +415,16 @@ __global__ void __launch_bounds__(32) topk_permute_warp_kernel(const float* __re
   for (int base = 0; base <= E; base += 32) {
     const int x = base + lane;
     int lt = 0, eq = 0;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      lt += (j < n && es[j] < x) ? 1 : 0;
-      eq += (j < n && es[j] == x) ? 1 : 0;
+    for (int j = 0; j < n; ++j) {
+      const int ej = __shfl_sync(0xffffffffu, e, j);
+      lt += ej < x ? 1 : 0;
+      eq += ej == x ? 1 : 0;
     }
     if (x <= E) offsets[x] = x == E ? n : lt;
     const bool has = x < E && eq > 0;
-    const unsigned mk = __ballot_sync(0xffffffffu, has);
-    if (has) active[nact + __popc(mk & ((1u << lane) - 1u))] = x;
-    nact += __popc(mk);
+    const unsigned m = __ballot_sync(0xffffffffu, has);
+    if (has) active[nact + __popc(m & ((1u << lane) - 1u))] = x;
+    nact += __popc(m);
   }
   if (lane == 0) active[E] = nact;
 }
