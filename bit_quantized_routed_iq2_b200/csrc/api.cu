@@ -445,9 +445,12 @@ moe_status moe_layer_forward_cached(moe_expert_cache* cache, const moe_layer_wei
   if (cudaGetDevice(&dev) != cudaSuccess || dev != cache->device) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int E = desc->n_experts, k = desc->top_k, S = cache->n_slots;
+  // the shared expert runs as in moe_layer_forward (side stream, step 5), so the outputs agree bit for bit;
+  // then the router is the first kernel on the caller's stream and clears the status word
+  const bool early = shared_early_ok(shape_of(desc), x_dtype, T);
   // 1. routing by expert
   int rc = launch_route(weights->router_w, weights->router_bias, x, x_dtype, T, desc->hidden, E, k, w.logits,
-                        w.topk_idx, w.topk_w, w.offsets, w.perm, w.inv, w.active, w.status, s, false);
+                        w.topk_idx, w.topk_w, w.offsets, w.perm, w.inv, w.active, w.status, s, early);
   if (rc != OK) return to_status(rc);
   // 2. the experts this call needs (a copy to pageable host memory returns once the routing is done)
   if (cudaMemcpyAsync(cache->h_active.data(), w.active, (E + 1) * sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
@@ -513,8 +516,13 @@ moe_status moe_layer_forward_cached(moe_expert_cache* cache, const moe_layer_wei
   wp.down_dd = reinterpret_cast<const uint32_t*>(cache->slot[5]);
   Routing r{w.topk_w, w.offsets, w.perm, w.inv, w.active};
   const bool routed_clears = x_dtype == MOE_BF16 && router_tc_supported(T, desc->hidden, E);
-  // the FFN's workspace part is sized for E experts, which covers S <= E slots
-  return to_status(launch_ffn(shape_of(&sd), wp, x, x_dtype, T, r, residual, y, w.ffn, w.status, !routed_clears, s));
+  // the FFN's workspace part is sized for E experts, which covers S <= E slots (its layout does not depend on E)
+  if (early) rc = launch_shared_early(shape_of(desc), wp, x, T, w.ffn, s);
+  if (rc == OK)
+    rc = launch_ffn(shape_of(&sd), wp, x, x_dtype, T, r, residual, y, w.ffn, w.status, !routed_clears && !early, s,
+                    early);
+  if (rc != OK && early) join_shared_early(s);
+  return to_status(rc);
 }
 
 }  // extern "C"

@@ -216,14 +216,16 @@ __global__ void __launch_bounds__(256) shared_gateup_kernel(int H, int Is, const
 
 // Same for few tokens (T <= TMAX): no shared-memory staging and no block-wide
 // barrier; activations come from global memory (L1-resident, the same for every
-// warp), four 16-byte weight loads of each matrix per lane are in flight.
+// warp), four 16-byte weight loads of each matrix per lane are in flight. One
+// warp per row, any number of warps per CTA: launched with small CTAs and no
+// shared memory, it fits beside the routed GEMVs on the same SMs.
 template <typename XT, int TMAX>
 __global__ void __launch_bounds__(256) shared_gateup_direct_kernel(int H, int Is, const uint16_t* __restrict__ sg,
                                                                    const uint16_t* __restrict__ su,
                                                                    const XT* __restrict__ x, int T,
                                                                    float* __restrict__ hs) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + warp;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= Is) return;
   float ag[TMAX], au[TMAX];
 #pragma unroll
@@ -279,6 +281,7 @@ __global__ void __launch_bounds__(256) shared_gateup_direct_kernel(int H, int Is
 // y[t][r] = sum_j w[t][j] o[inv[t*k+j]][r] (j ascending) + (Wsd hs_t)[r] + residual[t][r],
 // where o of an assignment is the sum of its DP partial rows (parts in order).
 // One warp per output row r, all tokens; the row's weights are loaded up front.
+// With k = 0 it is the shared expert's down projection alone.
 template <int TMAX>
 __global__ void __launch_bounds__(256) shared_down_combine_kernel(int H, int Is, int k, const uint16_t* __restrict__ sd,
                                                                   const float* __restrict__ hs, int T,
@@ -288,7 +291,7 @@ __global__ void __launch_bounds__(256) shared_down_combine_kernel(int H, int Is,
                                                                   const float* residual, float* y) {
   constexpr int WMAX = 8;  // 16-byte weight loads per lane kept in registers (Is <= 2048)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + warp;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= H) return;
   const int nw = (Is + 255) / 256;
   uint4 wv[WMAX];
@@ -357,6 +360,59 @@ __global__ void __launch_bounds__(256) shared_down_combine_kernel(int H, int Is,
       }
     }
   }
+}
+
+// y[t][r] = sum_j w[t][j] o[inv[t*k+j]][r] (j ascending) + ys[t][r] + residual[t][r],
+// where o of an assignment is the sum of its DP partial rows (parts in order)
+// and ys the shared expert's output computed beforehand. One thread per (t, r);
+// the assignments are taken eight at a time with all their routing words, then
+// all their partial rows, requested before any is added, so a thread waits for
+// memory once per eight assignments rather than twice per assignment.
+__global__ void __launch_bounds__(256) combine_routed_kernel(int H, int k, const float* __restrict__ topk_w,
+                                                             const int32_t* __restrict__ inv,
+                                                             const float* __restrict__ obuf, int DP,
+                                                             const float* __restrict__ ys, const float* residual,
+                                                             float* y) {
+  constexpr int JC = 8, DC = 8;
+  pdl_trigger();
+  pdl_wait();  // the routed partials come from the kernel before this one
+  const int r = blockIdx.x * blockDim.x + threadIdx.x, t = blockIdx.y;
+  if (r >= H) return;
+  float v = 0.f;
+  for (int j0 = 0; j0 < k; j0 += JC) {
+    const float* o[JC];
+    float wj[JC];
+#pragma unroll
+    for (int j = 0; j < JC; ++j) {
+      const int a = t * k + j0 + j;
+      const bool in = j0 + j < k;
+      o[j] = in ? obuf + static_cast<size_t>(inv[a]) * DP * H + r : nullptr;
+      wj[j] = in ? topk_w[a] : 0.f;
+    }
+    float sacc[JC];
+#pragma unroll
+    for (int j = 0; j < JC; ++j) sacc[j] = 0.f;
+    for (int d0 = 0; d0 < DP; d0 += DC) {
+      float pv[JC][DC];
+#pragma unroll
+      for (int j = 0; j < JC; ++j)
+#pragma unroll
+        for (int d = 0; d < DC; ++d)
+          pv[j][d] = (o[j] && d0 + d < DP) ? o[j][static_cast<size_t>(d0 + d) * H] : 0.f;
+#pragma unroll
+      for (int j = 0; j < JC; ++j)
+#pragma unroll
+        for (int d = 0; d < DC; ++d)
+          if (d0 + d < DP) sacc[j] += pv[j][d];
+    }
+#pragma unroll
+    for (int j = 0; j < JC; ++j)
+      if (j0 + j < k) v = fmaf(wj[j], sacc[j], v);
+  }
+  const size_t i = static_cast<size_t>(t) * H + r;
+  v += ys[i];
+  if (residual) v += residual[i];
+  y[i] = v;
 }
 
 // ------------------------------------------------------------ launcher
@@ -436,6 +492,7 @@ struct FastWs {
   int32_t* hq;
   float* obuf;
   float* hsh;
+  float* ysh;    // the shared expert's output [T][H] (computed on the side stream)
   uint16_t* xb;  // bf16 parts of fp32 x [2][T][H]
   uint16_t* hb;  // bf16 parts of the shared intermediate [2][T][Is]
   size_t bytes;
@@ -458,6 +515,7 @@ FastWs carve_fast(const LayerShape& s, int T, int KP, int DP, char* base) {
   w.hq = reinterpret_cast<int32_t*>(take(nA * (s.I / 16) * 4));
   w.obuf = reinterpret_cast<float*>(take(nA * DP * s.H * 4));
   w.hsh = reinterpret_cast<float*>(take(static_cast<size_t>(T) * (s.Is > 0 ? s.Is : 1) * 4));
+  w.ysh = reinterpret_cast<float*>(take(static_cast<size_t>(T) * s.H * 4));
   w.xb = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(T) * 2 * s.H * 2));
   w.hb = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(T) * 2 * (s.Is > 0 ? s.Is : 1) * 2));
   w.bytes = off;
@@ -473,6 +531,9 @@ size_t fast_ffn_workspace_bytes(const LayerShape& s, int T) {
   }
   return b;
 }
+
+// Token counts up to which the side stream runs the shared expert as warp-per-row GEMVs.
+constexpr int kSharedDirectMaxT = 4;
 
 // Side stream and fork/join events per (device, caller stream), created on first use.
 struct SideCtx {
@@ -524,13 +585,43 @@ int launch_shared_early(const LayerShape& s, const WeightPtrs& w, const void* x,
                                                     nullptr, tma ? 14 : 13);
   }
   if (cudaEventRecord(c->digits, c->st) != cudaSuccess) return ERR_CUDA;
-  int rc;
-  {
-    ProfScope ps(MOE_K_SHARED_GATEUP, c->st);
-    rc = launch_shared_gateup_mma(s.H, s.Is, w.sh_gate, w.sh_up, static_cast<const uint16_t*>(x), 1, T, fw.hb, c->st);
+  // the whole shared expert follows on the side stream, into ysh. For a few tokens its GEMVs run in CTAs of
+  // four warps without shared memory, which fit on the SMs beside the routed GEMVs (compute-bound at these
+  // sizes) and use the HBM bandwidth those leave; for more tokens the tensor-core kernels.
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  int rc = OK;
+  if (T <= kSharedDirectMaxT) {
+    {
+      ProfScope ps(MOE_K_SHARED_GATEUP, c->st);
+      const int grid = (s.Is + 3) / 4;
+      if (T == 1)
+        shared_gateup_direct_kernel<uint16_t, 1><<<grid, 128, 0, c->st>>>(s.H, s.Is, w.sh_gate, w.sh_up, xb, T, fw.hsh);
+      else
+        shared_gateup_direct_kernel<uint16_t, 4><<<grid, 128, 0, c->st>>>(s.H, s.Is, w.sh_gate, w.sh_up, xb, T, fw.hsh);
+    }
+    {
+      ProfScope ps(MOE_K_SHARED_DOWN, c->st);
+      const int grid = (s.H + 3) / 4;
+      if (T == 1)
+        shared_down_combine_kernel<1><<<grid, 128, 0, c->st>>>(s.H, s.Is, 0, w.sh_down, fw.hsh, T, nullptr, nullptr,
+                                                               nullptr, 1, nullptr, fw.ysh);
+      else
+        shared_down_combine_kernel<4><<<grid, 128, 0, c->st>>>(s.H, s.Is, 0, w.sh_down, fw.hsh, T, nullptr, nullptr,
+                                                               nullptr, 1, nullptr, fw.ysh);
+    }
+  } else {
+    {
+      ProfScope ps(MOE_K_SHARED_GATEUP, c->st);
+      rc = launch_shared_gateup_mma(s.H, s.Is, w.sh_gate, w.sh_up, xb, 1, T, fw.hb, c->st);
+    }
+    {
+      ProfScope ps(MOE_K_SHARED_DOWN, c->st);
+      rc |= launch_shared_down_combine_mma(s.H, s.Is, w.sh_down, fw.hb, T, 0, nullptr, nullptr, nullptr, 1, nullptr,
+                                           fw.ysh, c->st);
+    }
   }
   if (cudaEventRecord(c->join, c->st) != cudaSuccess) return ERR_CUDA;
-  return rc;
+  return rc != OK ? ERR_CUDA : (cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA);
 }
 
 int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
@@ -626,16 +717,17 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
     ProfScope ps(MOE_K_DOWN, st);
     rc |= launch_down(da, slots, T, sms, st);
   }
-  if (sh_mma) {
-    if (shared_early) {
-      SideCtx* c = side_ctx(st);
-      if (!c || cudaStreamWaitEvent(st, c->join, 0) != cudaSuccess) return ERR_CUDA;
-    }
-    {
-      ProfScope ps(MOE_K_COMBINE, st);
-      rc |= launch_shared_down_combine_mma(s.H, s.Is, w.sh_down, fw.hb, T, s.k, r.topk_w, r.inv, obuf, DP,
-                                           residual, y, st);
-    }
+  if (shared_early) {  // the shared output is ready in ysh once the side stream joins
+    SideCtx* c = side_ctx(st);
+    if (!c || cudaStreamWaitEvent(st, c->join, 0) != cudaSuccess) return ERR_CUDA;
+    ProfScope ps(MOE_K_COMBINE, st);
+    launch_pdl(combine_routed_kernel, dim3((s.H + 255) / 256, T), dim3(256), 0, st, s.H, s.k,
+               static_cast<const float*>(r.topk_w), static_cast<const int32_t*>(r.inv),
+               static_cast<const float*>(obuf), DP, static_cast<const float*>(fw.ysh), residual, y);
+  } else if (sh_mma) {
+    ProfScope ps(MOE_K_COMBINE, st);
+    rc |= launch_shared_down_combine_mma(s.H, s.Is, w.sh_down, fw.hb, T, s.k, r.topk_w, r.inv, obuf, DP, residual, y,
+                                         st);
   } else {
     ProfScope ps(MOE_K_COMBINE, st);
     const int grid = (s.H + 7) / 8;

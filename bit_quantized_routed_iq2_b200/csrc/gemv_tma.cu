@@ -544,6 +544,89 @@ __device__ __forceinline__ bool gu_unit_multi(const GuTmaArgs& a, const GuCtx& c
 }
 
 
+// The consumer loop of the one-token kernel (every expert holds one
+// assignment, the activations are staged). The lane mapping and the operand
+// construction are those of gu_unit_one; everything that depends only on the
+// lane is computed once, the B operand is loaded unconditionally (lanes that
+// carry no activations read the zero region, so no register is zeroed and no
+// branch is taken per round), and the two fp16 row scales of a unit are
+// loaded before its data wait and first used after its MMAs, so their latency
+// never stalls the warp.
+__device__ __forceinline__ void gu_consume_t1(const GuTmaArgs& a, const MetaSmem& ms, uint64_t* full, uint64_t* empty,
+                                              uint32_t ring_s, uint32_t x_s, uint32_t xs_s, uint32_t zero_s, int warp,
+                                              int lane) {
+  const int H = a.H, I = a.I, KP = a.KP, S = a.S, rbs = I / kBoxRows;
+  const int nact = ms.act[a.E];
+  const int g = lane >> 2, tig = lane & 3, bb = tig >> 1, hf = tig & 1;
+  const uint32_t lane4 = static_cast<uint32_t>(lane) << 2, sgn_lane = 128u + lane4;
+  const uint32_t one = static_cast<uint32_t>(a.one);
+  // this lane's round-0 record of row g (chunk (4bb) ^ g, half hf) inside stage 0
+  const uint32_t ring_lane = ring_s + static_cast<uint32_t>(16 * warp + g) * kGuW +
+                             (((static_cast<uint32_t>(g) ^ (4u * bb)) << 4) | (8u * hf));
+  // B: the x digits of this lane's column (block 2kp + bb of the x_off layout: kp steps 1024 bytes), or zeros
+  const bool bact = (g >> 1) == tig;
+  const uint32_t xb_base = bact ? x_s + static_cast<uint32_t>(x_off(H, 0, g & 1, bb * 256 + hf * 32)) : zero_s;
+  const uint32_t xb_step = bact ? 1024u : 0u;
+  const uint32_t xs_lane = xs_s + 4u * bb;  // + 8 kp: the 2^s / 8 of block 2kp + bb
+  const int row_l = 16 * warp + g;
+  const int dstride = H / 256;
+  RingPos rp{0, 0u};
+  GuIter t;
+  t.init(blockIdx.x, gridDim.x, KP, rbs);
+  for (; t.slot < nact; t.next(KP, rbs)) {
+    const int e = ms.act[t.slot];
+    const uint16_t* dr = (t.m ? a.up_d : a.gate_d) +
+                         (static_cast<size_t>(e) * I + t.rb * kBoxRows + row_l) * dstride + 2 * t.kp;
+    const uint32_t dw0 = __ldg(reinterpret_cast<const uint32_t*>(dr));                 // row g: blocks 2kp, 2kp+1
+    const uint32_t dw1 = __ldg(reinterpret_cast<const uint32_t*>(dr + 8 * dstride));  // row g + 8
+    const uint32_t xb0 = xb_base + static_cast<uint32_t>(t.kp) * xb_step, xb1 = xb0 ^ 16u;
+    if (!mbar_wait_bounded(&full[rp.s], rp.ph, a.err, ERR_TIMEOUT, a.wait_limit)) return;
+    const uint32_t r0 = ring_lane + static_cast<uint32_t>(rp.s) * kGuBox;
+    const int s = rp.s;
+    rp.next(S);
+    int i0 = 0, i1 = 0;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      const uint2 ra = ld_s64(r0 ^ (16u * cc));          // row g
+      const uint2 rb = ld_s64((r0 ^ (16u * cc)) + 1024);  // row g + 8
+      const uint4 bx0 = ld_s128(xb0 + 128u * cc);
+      const uint4 bx1 = ld_s128(xb1 + 128u * cc);
+      const uint32_t bv[8] = {bx0.x, bx0.y, bx0.z, bx0.w, bx1.x, bx1.y, bx1.z, bx1.w};
+      int acc[4];
+#define MOE_GU_GROUP(JJ)                                                                  \
+  {                                                                                       \
+    uint32_t a0, a1, a2, a3;                                                              \
+    iq2_group_int8<JJ>(ra, lane4, sgn_lane, one, a0, a2);                                \
+    iq2_group_int8<JJ>(rb, lane4, sgn_lane, one, a1, a3);                                \
+    if (JJ == 0) mma_s8s8_zero(acc, a0, a1, a2, a3, bv[2 * JJ], bv[2 * JJ + 1]);          \
+    else mma_s8s8(acc, a0, a1, a2, a3, bv[2 * JJ], bv[2 * JJ + 1]);                       \
+  }
+      MOE_GU_GROUP(0) MOE_GU_GROUP(1) MOE_GU_GROUP(2) MOE_GU_GROUP(3)
+#undef MOE_GU_GROUP
+      i0 += (acc[0] * 128 + acc[1]) * iq2_odd(ra);
+      i1 += (acc[2] * 128 + acc[3]) * iq2_odd(rb);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    const float xsv = ld_sf(xs_lane + 8u * static_cast<uint32_t>(t.kp));
+    const float d0 = bb ? half_hi(dw0) : half_lo(dw0);
+    const float d1 = bb ? half_hi(dw1) : half_lo(dw1);
+    float f0 = static_cast<float>(i0) * (d0 * xsv);
+    float f1 = static_cast<float>(i1) * (d1 * xsv);
+    f0 += __shfl_xor_sync(0xffffffffu, f0, 1);
+    f0 += __shfl_xor_sync(0xffffffffu, f0, 2);
+    f1 += __shfl_xor_sync(0xffffffffu, f1, 1);
+    f1 += __shfl_xor_sync(0xffffffffu, f1, 2);
+    if (tig == 0) {
+      const size_t o = ((static_cast<size_t>(ms.off[e]) * 2 + t.m) * KP + t.kp) * I + t.rb * kBoxRows + row_l;
+      if (index_ok(o + 8, a.gpart_n)) {
+        a.gpart[o] = f0;
+        a.gpart[o + 8] = f1;
+      }
+    }
+  }
+}
+
 // Shared-memory plan of the gate/up kernel (host and device agree on it); the
 // selector tables come first, at a fixed shared address, so lookups need no
 // base add.
@@ -605,15 +688,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
   for (int i = tid; i < kZeroBytes / 16; i += kThreadsT) reinterpret_cast<uint4*>(zero)[i] = make_uint4(0, 0, 0, 0);
   pdl_wait();  // routing and activations come from the kernels before this one
   load_meta(ms, a.offsets, a.active, a.perm, a.E, nA, a.k, tid, kThreadsT);
-  if (XS) {  // [T][2][H] digits -> the staged layout of x_off, 16 bytes at a time
-    const int per = H / 16;
-    for (int i = tid; i < T * 2 * per; i += kThreadsT) {
-      const int row = i / per, e = (i - row * per) * 16;
-      *reinterpret_cast<uint4*>(xsm + x_off(H, row >> 1, row & 1, e)) = reinterpret_cast<const uint4*>(a.xd)[i];
-    }
-    for (int i = tid; i < T * (H / 256); i += kThreadsT) xssm[i] = a.xs[i];
-  }
-  __syncthreads();
+  __syncthreads();  // barriers, zero region and routing metadata are in place: the producer may start
   const int nact = ms.act[a.E];
 
   if (warp == kCW) {  // producer
@@ -640,8 +715,23 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
     return;
   }
 
+  // consumers: stage the activations while the first boxes are in flight
+  if (XS) {  // [T][2][H] digits -> the staged layout of x_off, 16 bytes at a time, asynchronously
+    const int per = H / 16;
+    for (int i = tid; i < T * 2 * per; i += kCW * 32) {
+      const int row = i / per, e = (i - row * per) * 16;
+      cp_async16(smem_addr(xsm + x_off(H, row >> 1, row & 1, e)), a.xd + static_cast<size_t>(i) * 16);
+    }
+    for (int i = tid; i < T * (H / 256); i += kCW * 32) xssm[i] = a.xs[i];
+    cp_async_wait_all();
+  }
+  named_barrier(1, kCW * 32);
   // the table copy must have landed before the first lookup (the producer never reads it)
   if (!mbar_wait_bounded(tabbar, 0, a.err, ERR_TIMEOUT, a.wait_limit)) return;
+  if (MAXQ == 1) {  // one token
+    gu_consume_t1(a, ms, full, empty, smem_addr(ring), smem_addr(xsm), smem_addr(xssm), smem_addr(zero), warp, lane);
+    return;
+  }
   GuCtx c;
   c.tab = reinterpret_cast<const char*>(smem + pl.tab);
   c.ring = ring;
@@ -989,6 +1079,77 @@ __device__ __forceinline__ bool dn_unit_multi(const DnTmaArgs& a, const DnCtx& c
   return true;
 }
 
+// The consumer loop of the one-token down kernel (every expert holds one
+// assignment, h staged). Lane mapping and operands are those of dn_unit_one;
+// lane-only addresses are computed once, B is loaded unconditionally (lanes
+// without h read the zero region), and the two Q2K block scale words of a unit
+// are loaded before its data wait and first used after its MMAs.
+__device__ __forceinline__ void dn_consume_t1(const DnTmaArgs& a, const MetaSmem& ms, uint64_t* full, uint64_t* empty,
+                                              uint32_t ring_s, uint32_t hd_s, uint32_t hsc_s, uint32_t hq_s,
+                                              uint32_t zero_s, int warp, int lane) {
+  const int H = a.H, I = a.I, DP = a.DP, S = a.S, rbs = H / kBoxRows, nblk = I / 256;
+  const int nact = ms.act[a.E];
+  const int g = lane >> 2, tig = lane & 3;
+  const bool bact = (g >> 1) == tig;
+  const int row = 16 * warp + g;
+  const uint32_t qoff = static_cast<uint32_t>(row) * 64 + 16u * (static_cast<uint32_t>(tig) ^ ((g >> 1) & 3));
+  const uint32_t soff = kDnQBytes + static_cast<uint32_t>(row) * 16 + 4u * tig;
+  RingPos rp{0, 0u};
+  DnIter t;
+  t.init(blockIdx.x, gridDim.x, DP, rbs);
+  for (; t.slot < nact; t.next(DP, rbs)) {
+    const int e = ms.act[t.slot];
+    const int p0 = ms.off[e];
+    const int blk = t.dp;
+    const uint32_t* dr = a.dd + (static_cast<size_t>(e) * H + t.rb * kBoxRows + row) * nblk + blk;
+    const uint32_t dA = __ldg(dr), dB = __ldg(dr + 8 * nblk);
+    // sub-block 4 tig of block blk, round 0 (rounds step 128 bytes; the zero region covers them too)
+    const uint32_t hb = bact ? hd_s + static_cast<uint32_t>(h_off(I, p0, g & 1, blk * 256 + 64 * tig)) : zero_s;
+    const uint4 hqv = ld_s128(hq_s + 4u * static_cast<uint32_t>(p0 * (I / 16) + blk * 16 + 4 * tig));
+    const float e2 = ld_sf(hsc_s + 4u * static_cast<uint32_t>(p0 * a.hss + blk));
+    if (!mbar_wait_bounded(&full[rp.s], rp.ph, a.err, ERR_TIMEOUT)) return;
+    const uint32_t st = ring_s + static_cast<uint32_t>(rp.s) * kDnStage;
+    const uint4 qa = ld_s128(st + qoff), qb = ld_s128(st + qoff + 8 * 64);
+    const uint32_t sa = ld_s32(st + soff), sb = ld_s32(st + soff + 8 * 16);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[rp.s]);  // the codes are in registers: the stage is free
+    rp.next(S);
+    const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w}, wb[4] = {qb.x, qb.y, qb.z, qb.w};
+    const int hq[4] = {static_cast<int>(hqv.x), static_cast<int>(hqv.y), static_cast<int>(hqv.z),
+                       static_cast<int>(hqv.w)};
+    int iA0 = 0, iA1 = 0, iM0 = 0, iM1 = 0;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      const uint4 bh = ld_s128(hb + 128u * cc);
+      uint32_t x0, x1, x2, x3, y0, y1, y2, y3;
+      q2k_sub4(wa[cc], x0, x1, x2, x3);
+      q2k_sub4(wb[cc], y0, y1, y2, y3);
+      int acc[4];
+      mma_u8s8_zero(acc, x0, y0, x1, y1, bh.x, bh.y);
+      mma_u8s8(acc, x2, y2, x3, y3, bh.z, bh.w);
+      const uint32_t ba = cc ? __umulhi(sa, 1u << (32 - 8 * cc)) : sa;  // scale byte cc at bits 0..7
+      const uint32_t bs = cc ? __umulhi(sb, 1u << (32 - 8 * cc)) : sb;
+      iA0 += (acc[0] * 128 + acc[1]) * static_cast<int>(ba & 15u);
+      iA1 += (acc[2] * 128 + acc[3]) * static_cast<int>(bs & 15u);
+      iM0 += static_cast<int>((ba >> 4) & 15u) * hq[cc];
+      iM1 += static_cast<int>((bs >> 4) & 15u) * hq[cc];
+    }
+    float f0 = dn_block(dA, e2, iA0, iM0);
+    float f1 = dn_block(dB, e2, iA1, iM1);
+    f0 += __shfl_xor_sync(0xffffffffu, f0, 1);
+    f0 += __shfl_xor_sync(0xffffffffu, f0, 2);
+    f1 += __shfl_xor_sync(0xffffffffu, f1, 1);
+    f1 += __shfl_xor_sync(0xffffffffu, f1, 2);
+    if (tig == 0) {
+      const size_t o = (static_cast<size_t>(p0) * DP + blk) * H + t.rb * kBoxRows + row;
+      if (index_ok(o + 8, a.opart_n)) {
+        a.opart[o] = f0;
+        a.opart[o + 8] = f1;
+      }
+    }
+  }
+}
+
 // Shared-memory plan of the down kernel.
 struct DnPlan {
   size_t meta, zero, hd, hsc, hq, ring, bars, total;
@@ -1044,13 +1205,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
   for (int i = tid; i < kZeroBytes / 16; i += kThreadsT) reinterpret_cast<uint4*>(zero)[i] = make_uint4(0, 0, 0, 0);
   pdl_wait();  // routing and h come from the kernels before this one
   load_meta(ms, a.offsets, a.active, nullptr, a.E, nA, a.k, tid, kThreadsT);
-  if (HS) {  // the h_off layout is the same in global and shared memory
-    for (int i = tid; i < nA * 2 * I / 16; i += kThreadsT)
-      reinterpret_cast<uint4*>(hd_s)[i] = reinterpret_cast<const uint4*>(a.hd)[i];
-    for (int i = tid; i < nA * a.hss; i += kThreadsT) hsc_s[i] = a.hsc[i];
-    for (int i = tid; i < nA * (I / 16); i += kThreadsT) hq_s[i] = a.hq[i];
-  }
-  __syncthreads();
+  __syncthreads();  // barriers, zero region and routing metadata are in place: the producer may start
   const int nact = ms.act[a.E];
 
   if (warp == kCW) {  // producer
@@ -1076,6 +1231,20 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
         }
       }
     }
+    return;
+  }
+  // consumers: stage h while the first boxes are in flight (the h_off layout is the same in global and
+  // shared memory; I % 256 == 0 makes both byte counts multiples of 16)
+  if (HS) {
+    for (int i = tid; i < nA * 2 * I / 16; i += kCW * 32) cp_async16(smem_addr(hd_s) + 16u * i, a.hd + 16 * static_cast<size_t>(i));
+    for (int i = tid; i < nA * (I / 64); i += kCW * 32) cp_async16(smem_addr(hq_s) + 16u * i, a.hq + 4 * static_cast<size_t>(i));
+    for (int i = tid; i < nA * a.hss; i += kCW * 32) hsc_s[i] = a.hsc[i];
+    cp_async_wait_all();
+  }
+  named_barrier(1, kCW * 32);
+  if (MAXQ == 1) {  // one token
+    dn_consume_t1(a, ms, full, empty, smem_addr(ring), smem_addr(hd_s), smem_addr(hsc_s), smem_addr(hq_s),
+                  smem_addr(zero), warp, lane);
     return;
   }
   DnCtx c;

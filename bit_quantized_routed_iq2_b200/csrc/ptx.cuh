@@ -86,6 +86,18 @@ __device__ __forceinline__ bool mbar_wait_bounded_sleepy(uint64_t* bar, uint32_t
   }
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only), and the wait for all of
+// this thread's outstanding ones.
+__device__ __forceinline__ void cp_async16(uint32_t dst_s, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_s), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Barrier `id` (1..15) among the first `nthreads` threads of the CTA (whole warps).
+__device__ __forceinline__ void named_barrier(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Bulk copy global -> this CTA's shared memory, completion counted on `bar`.
 // dst, src and bytes must be multiples of 16.
 __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

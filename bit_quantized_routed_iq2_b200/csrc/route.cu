@@ -62,6 +62,28 @@ __global__ void __launch_bounds__(128) router_logits_small_kernel(const uint16_t
   float acc[TT];
 #pragma unroll
   for (int t = 0; t < TT; ++t) acc[t] = 0.f;
+  if constexpr (TT == 1 && sizeof(XT) == 2) {  // one bf16 token: all activation slices in flight at once
+    uint4 xv[MAXJ];
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+      const int c = tid * 8 + j * 1024;
+      xv[j] = (j < nj && c < H && t0 < T)
+                  ? *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(x) + static_cast<size_t>(t0) * H + c)
+                  : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float a = 0.f;
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+      const int c = tid * 8 + j * 1024;
+      if (j >= nj || c >= H) break;
+      float w8[8], x8[8];
+      bf16x8(wv[j], w8);
+      bf16x8(xv[j], x8);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a = fmaf(w8[i], x8[i], a);
+    }
+    acc[0] = a;
+  } else {
 #pragma unroll
   for (int j = 0; j < MAXJ; ++j) {
     const int c = tid * 8 + j * 1024;
@@ -78,6 +100,7 @@ __global__ void __launch_bounds__(128) router_logits_small_kernel(const uint16_t
       for (int i = 0; i < 8; ++i) a = fmaf(w8[i], x8[i], a);
       acc[t] = a;
     }
+  }
   }
 #pragma unroll
   for (int t = 0; t < TT; ++t) {
@@ -429,6 +452,101 @@ __global__ void __launch_bounds__(32) topk_permute_warp_kernel(const float* __re
   if (lane == 0) active[E] = nact;
 }
 
+// The same outputs for T * k <= 32 and T * E <= kRankMaxLogits by one CTA,
+// without serial rounds: every logit counts the logits of its token that rank
+// above it (greater, or equal with a lower expert index; NaN ranks as -inf),
+// and the k with a count below k write themselves into their slot. The weights
+// are summed in slot order by one thread per token, as in topk_warp. The
+// permutation is computed in parallel from the chosen experts in shared
+// memory: assignment j goes to (assignments with a smaller expert) + (earlier
+// ones with the same expert), offsets[x] counts the assignments below x, and
+// the first assignment of each distinct expert writes it into the active list
+// at the number of distinct experts below it.
+constexpr int kRankMaxLogits = 4096;
+__global__ void __launch_bounds__(256) topk_permute_rank_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                                int32_t* __restrict__ topk_idx,
+                                                                float* __restrict__ topk_w,
+                                                                int32_t* __restrict__ offsets,
+                                                                int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                                int32_t* __restrict__ active) {
+  __shared__ __align__(16) float ls[kRankMaxLogits];
+  __shared__ int sel[32];
+  __shared__ float chosen[32];
+  __shared__ int first[32];
+  pdl_trigger();
+  pdl_wait();
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const int n = T * k;
+  for (int i = tid; i < T * E; i += nthr) {
+    const float v = logits[i];
+    ls[i] = v == v ? v : -INFINITY;
+  }
+  __syncthreads();
+  for (int i = tid; i < T * E; i += nthr) {
+    const int t = i / E, e = i - t * E;
+    const float v = ls[i];
+    const float* row = ls + t * E;
+    int rank = 0;
+    if ((E & 3) == 0) {  // rows start 16-byte aligned: four logits per load
+      for (int j = 0; j < E; j += 4) {
+        const float4 u = *reinterpret_cast<const float4*>(row + j);
+        rank += (u.x > v || (u.x == v && j < e)) ? 1 : 0;
+        rank += (u.y > v || (u.y == v && j + 1 < e)) ? 1 : 0;
+        rank += (u.z > v || (u.z == v && j + 2 < e)) ? 1 : 0;
+        rank += (u.w > v || (u.w == v && j + 3 < e)) ? 1 : 0;
+      }
+    } else {
+      for (int j = 0; j < E; ++j) {
+        const float u = row[j];
+        rank += (u > v || (u == v && j < e)) ? 1 : 0;
+      }
+    }
+    if (rank < k) {
+      sel[t * k + rank] = e;
+      chosen[t * k + rank] = v;
+    }
+  }
+  __syncthreads();
+  if (tid < T) {
+    const float* c = chosen + tid * k;
+    float z = 0.f;
+    for (int j = 0; j < k; ++j) z += expf(c[j] - c[0]);
+    for (int j = 0; j < k; ++j) {
+      topk_idx[tid * k + j] = sel[tid * k + j];
+      topk_w[tid * k + j] = expf(c[j] - c[0]) / z;
+    }
+  }
+  if (tid < n) {
+    const int e = sel[tid];
+    int below = 0, fst = 1;
+    for (int j = 0; j < n; ++j) {
+      const int ej = sel[j];
+      below += (ej < e || (ej == e && j < tid)) ? 1 : 0;
+      if (ej == e && j < tid) fst = 0;
+    }
+    perm[below] = tid;
+    inv[tid] = below;
+    first[tid] = fst;
+  }
+  __syncthreads();
+  for (int x = tid; x <= E; x += nthr) {
+    int lt = 0;
+    for (int j = 0; j < n; ++j) lt += sel[j] < x ? 1 : 0;
+    offsets[x] = x == E ? n : lt;
+  }
+  if (tid < n && first[tid]) {
+    const int e = sel[tid];
+    int pos = 0;
+    for (int j = 0; j < n; ++j) pos += (first[j] && sel[j] < e) ? 1 : 0;
+    active[pos] = e;
+  }
+  if (tid == 0) {
+    int nact = 0;
+    for (int j = 0; j < n; ++j) nact += first[j];
+    active[E] = nact;
+  }
+}
+
 // Active-expert list from caller-provided offsets (used by moe_expert_ffn).
 __global__ void __launch_bounds__(1024) active_from_offsets_kernel(const int32_t* __restrict__ offsets, int E,
                                                                    int32_t* __restrict__ active) {
@@ -459,6 +577,9 @@ int launch_route(const uint16_t* Wr, const float* bias, const void* x, int x_dty
       const int rc = launch_router_tc(Wr, bias, static_cast<const uint16_t*>(x), T, H, E, logits, err,
                                       sms > 0 ? sms : 148, st);
       if (rc != OK) return rc;
+    } else if (T == 1 && x_dtype == 1) {
+      launch_pdl(router_logits_small_kernel<uint16_t, 1>, dim3(1, E), dim3(128), 0, st, Wr, bias,
+                 static_cast<const uint16_t*>(x), T, H, E, logits, clear_status ? err : nullptr);
     } else if (T <= 64) {
       constexpr int TT = 4;
       dim3 g((T + TT - 1) / TT, E);
@@ -479,7 +600,11 @@ int launch_route(const uint16_t* Wr, const float* bias, const void* x, int x_dty
     }
   }
   const size_t psmem = 32 * E * sizeof(uint16_t) + 3 * E * sizeof(int);
-  if (T * k <= 32 && E <= 256) {
+  if (T * k <= 32 && T * E <= kRankMaxLogits) {
+    ProfScope ps(MOE_K_PERMUTE, st);
+    launch_pdl(topk_permute_rank_kernel, dim3(1), dim3(256), 0, st, logits, T, E, k, topk_idx, topk_w, offsets, perm,
+               inv, active);
+  } else if (T * k <= 32 && E <= 256) {
     ProfScope ps(MOE_K_PERMUTE, st);
     launch_pdl(topk_permute_warp_kernel<8>, dim3(1), dim3(32), 0, st, logits, T, E, k, topk_idx, topk_w, offsets,
                perm, inv, active);

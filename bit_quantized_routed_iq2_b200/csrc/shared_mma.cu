@@ -258,108 +258,6 @@ __global__ void __launch_bounds__(512) shared_down_combine_mma_kernel(
   }
 }
 
-// The same output for one or two tokens as a GEMV on a persistent grid whose
-// CTA b owns the contiguous rows [b R, b R + R) of W_sd: one bulk copy brings
-// those rows (R x Is bf16, up to ~200 KB) into shared memory before the
-// kernel waits for its predecessors (the weights are constants of the layer),
-// so the only exposed latency after the wait is h and the routed partials.
-// h is rebuilt in shared memory as fp32 (hi + lo parts). Warp w takes rows
-// w, w + 16, ... of the CTA; each lane holds 8 columns of every 256-column
-// stripe. Per row: lane partial dot products in column order, a fixed
-// xor-shuffle tree, then the routed part (lane i takes slot i / DP, part
-// i % DP; these loads are issued before the dot products), the shared part and
-// the residual.
-template <int TT>
-__global__ void __launch_bounds__(512) shared_down_combine_gemv_kernel(
-    int H, int Is, int R, const uint16_t* __restrict__ wd, const uint16_t* __restrict__ hb, int T, int k,
-    const float* __restrict__ topk_w, const int32_t* __restrict__ inv, const float* __restrict__ obuf, int DP,
-    const float* residual, float* y) {
-  extern __shared__ __align__(128) uint8_t sm[];
-  float* hs = reinterpret_cast<float*>(sm);                                         // [T][Is]
-  const uint16_t* ws = reinterpret_cast<const uint16_t*>(sm + static_cast<size_t>(TT) * Is * 4);  // [R][Is]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + static_cast<size_t>(TT) * Is * 4 + static_cast<size_t>(R) * Is * 2);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const int r0 = blockIdx.x * R, nr = min(R, H - r0);
-  pdl_trigger();
-  if (nr <= 0) return;
-  if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
-    fence_barrier_init();
-    const uint32_t bytes = static_cast<uint32_t>(nr) * Is * 2;  // a multiple of 16: Is % 256 == 0
-    mbar_arrive_expect_tx(bar, bytes);
-    bulk_copy_g2s(const_cast<uint16_t*>(ws), wd + static_cast<size_t>(r0) * Is, bytes, bar);
-  }
-  pdl_wait();  // h, the routed partials and the routing come from the kernels before this one
-  // routed partials of this warp's rows, requested before anything waits on them
-  constexpr int kMaxRows = 4;
-  float ov[kMaxRows][TT][2];
-#pragma unroll
-  for (int q = 0; q < kMaxRows; ++q) {
-    const int rr = warp + nw * q;
-#pragma unroll
-    for (int t = 0; t < TT; ++t)
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        const int i = lane + 32 * h2;
-        float v = 0.f;
-        if (rr < nr && t < T && i < k * DP) {
-          const int aidx = t * k + i / DP;
-          v = __ldg(topk_w + aidx) *
-              __ldcg(obuf + (static_cast<size_t>(__ldg(inv + aidx)) * DP + i % DP) * H + r0 + rr);
-        }
-        ov[q][t][h2] = v;
-      }
-  }
-  for (int i = threadIdx.x; i < T * Is; i += blockDim.x)
-    hs[i] = bf16_bits_f(hb[i]) + bf16_bits_f(hb[static_cast<size_t>(T) * Is + i]);
-  __syncthreads();
-  if (!mbar_wait_bounded(bar, 0, nullptr, 0)) return;
-  const int nj = Is / 256;
-#pragma unroll
-  for (int q = 0; q < kMaxRows; ++q) {
-    const int rr = warp + nw * q;
-    if (rr >= nr) continue;
-    const uint16_t* wrow = ws + static_cast<size_t>(rr) * Is;
-    float acc[TT];
-#pragma unroll
-    for (int t = 0; t < TT; ++t) acc[t] = 0.f;
-    for (int j = 0; j < nj; ++j) {
-      const uint4 wv = *reinterpret_cast<const uint4*>(wrow + 256 * j + 8 * lane);
-      const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-      for (int t = 0; t < TT; ++t) {
-        if (t >= T) break;
-        const float4 ha = *reinterpret_cast<const float4*>(hs + t * Is + 256 * j + 8 * lane);
-        const float4 hb4 = *reinterpret_cast<const float4*>(hs + t * Is + 256 * j + 8 * lane + 4);
-        const float hv[8] = {ha.x, ha.y, ha.z, ha.w, hb4.x, hb4.y, hb4.z, hb4.w};
-        float a = acc[t];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          a = fmaf(__uint_as_float(ww[e] << 16), hv[2 * e], a);
-          a = fmaf(__uint_as_float(ww[e] & 0xFFFF0000u), hv[2 * e + 1], a);
-        }
-        acc[t] = a;
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < TT; ++t) {
-      if (t >= T) break;
-      float sv = acc[t];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sv += __shfl_xor_sync(0xffffffffu, sv, o);
-      float v = ov[q][t][0] + ov[q][t][1];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) {
-        v += sv;
-        const int r = r0 + rr;
-        if (residual) v += residual[static_cast<size_t>(t) * H + r];
-        y[static_cast<size_t>(t) * H + r] = v;
-      }
-    }
-  }
-}
-
 int pick_ks(int K, int ksmax) {
   for (int ks = ksmax; ks >= 1; ks >>= 1)
     if (K % (32 * ks) == 0) return ks;
@@ -398,30 +296,6 @@ int launch_shared_gateup_mma(int H, int Is, const uint16_t* wg, const uint16_t* 
 int launch_shared_down_combine_mma(int H, int Is, const uint16_t* wd, const uint16_t* hb, int T, int k,
                                    const float* topk_w, const int32_t* inv, const float* obuf, int DP,
                                    const float* residual, float* y, cudaStream_t st) {
-  if (T <= 2 && Is % 256 == 0 && Is <= 2048 && k * DP <= 64) {
-    // one or two tokens: the persistent GEMV with the weights staged in shared memory, when a CTA's rows fit
-    int dev = 0, sms = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-    const int R = (H + sms - 1) / sms;
-    const size_t dyn = static_cast<size_t>(2) * Is * 4 + static_cast<size_t>(R) * Is * 2 + 16;
-    if (R <= 4 * 16 && dyn <= 227 * 1024) {
-      const int grid = (H + R - 1) / R;
-      if (T == 1) {
-        cudaFuncSetAttribute(shared_down_combine_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(dyn));
-        launch_pdl(shared_down_combine_gemv_kernel<1>, dim3(grid), dim3(512), dyn, st, H, Is, R, wd, hb, T, k,
-                   topk_w, inv, obuf, DP, residual, y);
-      } else {
-        cudaFuncSetAttribute(shared_down_combine_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(dyn));
-        launch_pdl(shared_down_combine_gemv_kernel<2>, dim3(grid), dim3(512), dyn, st, H, Is, R, wd, hb, T, k,
-                   topk_w, inv, obuf, DP, residual, y);
-      }
-      return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
-    }
-  }
   const int ng = groups_for(2 * T);
   const int ks = pick_ks(Is, ksmax_for(ng));
   if (ks == 0) return ERR_SHAPE;
