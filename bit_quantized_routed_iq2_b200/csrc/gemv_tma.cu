@@ -351,7 +351,7 @@ __device__ __forceinline__ uint32_t q2k_quad(uint32_t w, uint32_t sh) { return (
 template <bool XS>
 __device__ __forceinline__ bool gu_unit_one(const GuTmaArgs& a, const GuCtx& c, RingPos& rp, const GuUnit& w,
                                             const uint32_t (&dp)[kMaxNB][2]) {
-  const int H = a.H, I = a.I, NB = a.NB;
+  const int I = a.I, NB = a.NB;
   const int g = c.g, tig = c.tig, bb = tig >> 1, hf = tig & 1;
   const int tok = c.tok[w.p0];
   const bool bact = (g >> 1) == tig;  // this lane carries B (digit g & 1 of its column's sub-block)
@@ -362,12 +362,10 @@ __device__ __forceinline__ bool gu_unit_one(const GuTmaArgs& a, const GuCtx& c, 
   float f0 = 0.f, f1 = 0.f;
 #pragma unroll 1
   for (int j = 0; j < NB; ++j) {
-    const int kblk = (w.kp * NB + j) * 2 + bb;  // this lane's block of H
-    // B source: staged (x_off layout; chunk 1 of a sub-block is the XOR-16 neighbour of chunk 0) or the
-    // global [T][2][H] digits (natural order)
-    const uint32_t xb0 = XS ? c.x_s + x_off(H, tok, g & 1, kblk * 256 + hf * 32) : 0u;
+    const int kblk = j * 2 + bb;  // this lane's block of the staged slice
+    // B source: the staged slice (x_off layout; chunk 1 of a sub-block is the XOR-16 neighbour of chunk 0)
+    const uint32_t xb0 = c.x_s + x_off(c.xpitch, tok, g & 1, kblk * 256 + hf * 32);
     const uint32_t xb1 = xb0 ^ 16u;
-    const int8_t* xg = XS ? nullptr : c.xdig + static_cast<size_t>(tok * 2 + (g & 1)) * H + kblk * 256 + hf * 32;
     if (!mbar_wait_bounded(&c.full[rp.s], rp.ph, a.err, ERR_TIMEOUT, a.wait_limit)) return false;
     const uint32_t r0 = c.ring_s + rp.s * kGuBox + rowb + roff;
     const int s = rp.s;
@@ -379,13 +377,8 @@ __device__ __forceinline__ bool gu_unit_one(const GuTmaArgs& a, const GuCtx& c, 
       const uint2 rb = ld_s64((r0 ^ (16u * cc)) + 1024);  // row g + 8
       uint4 bx0 = make_uint4(0u, 0u, 0u, 0u), bx1 = make_uint4(0u, 0u, 0u, 0u);
       if (bact) {
-        if (XS) {
-          bx0 = ld_s128(xb0 + 128u * cc);
-          bx1 = ld_s128(xb1 + 128u * cc);
-        } else {
-          bx0 = __ldg(reinterpret_cast<const uint4*>(xg + 64 * cc));
-          bx1 = __ldg(reinterpret_cast<const uint4*>(xg + 64 * cc + 16));
-        }
+        bx0 = ld_s128(xb0 + 128u * cc);
+        bx1 = ld_s128(xb1 + 128u * cc);
       }
       const uint32_t bv[8] = {bx0.x, bx0.y, bx0.z, bx0.w, bx1.x, bx1.y, bx1.z, bx1.w};
       int acc[4];
@@ -405,7 +398,7 @@ __device__ __forceinline__ bool gu_unit_one(const GuTmaArgs& a, const GuCtx& c, 
     }
     __syncwarp();
     if (c.lane == 0) mbar_arrive(&c.empty[s]);
-    const float xsv = XS ? ld_sf(c.xs_s + (tok * (H / 256) + kblk) * 4) : __ldg(c.xscl + tok * (H / 256) + kblk);
+    const float xsv = ld_sf(c.xs_s + (tok * (c.xpitch / 256) + kblk) * 4);
     const uint32_t w0 = j ? dp[1][0] : dp[0][0], w1 = j ? dp[1][1] : dp[0][1];
     const float d0 = bb ? half_hi(w0) : half_lo(w0);
     const float d1 = bb ? half_hi(w1) : half_lo(w1);
@@ -434,7 +427,7 @@ template <int TPG, int MAXQ, bool XS>
 __device__ __forceinline__ bool gu_unit_multi(const GuTmaArgs& a, const GuCtx& c, RingPos& rp, const GuUnit& w,
                                               const uint32_t (&dp)[kMaxNB][2]) {
   constexpr int SPS = 4 / TPG;
-  const int H = a.H, I = a.I, ne = w.ne, p0 = w.p0;
+  const int I = a.I, ne = w.ne, p0 = w.p0;
   const int ngroups = (ne + TPG - 1) / TPG;
   const int g = c.g, tig = c.tig;
   const int tslot_b = (g >> 1) % TPG, sslot_b = (g >> 1) / TPG, dig_b = g & 1;
@@ -449,7 +442,7 @@ __device__ __forceinline__ bool gu_unit_multi(const GuTmaArgs& a, const GuCtx& c
     const int tb = q * TPG + tslot_b, tc = q * TPG + tslot_c;
     bon[q] = q < ngroups && tb < ne;
     xtok[q] = bon[q] ? c.tok[p0 + tb] : 0;
-    xsc[q] = (q < ngroups && tc < ne) ? c.xscl + c.tok[p0 + tc] * (H / 256) + 2 * a.NB * w.kp : nullptr;
+    xsc[q] = (q < ngroups && tc < ne) ? c.xscl + c.tok[p0 + tc] * (c.xpitch / 256) : nullptr;
   }
   int acc[MAXQ][4];
   int iacc[MAXQ][2];
@@ -476,16 +469,22 @@ __device__ __forceinline__ bool gu_unit_multi(const GuTmaArgs& a, const GuCtx& c
         iq2_operand(c, rec[u][0], af[u][0][0], af[u][0][1]);
         iq2_operand(c, rec[u][1], af[u][1][0], af[u][1][1]);
       }
+      // 2 ls + 1 of the sub-block of each column set, rows g and g + 8 (the same for every token group)
+      int odd0[TPG], odd1[TPG];
+#pragma unroll
+      for (int jj = 0; jj < TPG; ++jj) {
+        const int sbi = 4 * cc + jj * SPS + sslot_c;
+        odd0[jj] = gu_odd(rg, sbi, g);
+        odd1[jj] = gu_odd(rg + 1024, sbi, g);
+      }
 #pragma unroll
       for (int q = 0; q < MAXQ; ++q) {
         if (q >= ngroups) break;
 #pragma unroll
         for (int jj = 0; jj < TPG; ++jj) {
-          // column set jj covers sub-blocks 4cc + jj*SPS .. +SPS-1
-          const int e = (w.kp * a.NB + j) * 512 + (4 * cc + jj * SPS + sslot_b) * 32 + 8 * tig;
-          const int8_t* xp = !bon[q] ? c.zero + 8 * tig
-                             : XS    ? c.xdig + x_off(H, xtok[q], dig_b, e)
-                                     : c.xdig + (xtok[q] * 2 + dig_b) * H + e;
+          // column set jj covers sub-blocks 4cc + jj*SPS .. +SPS-1 of box j of the staged slice
+          const int e = j * 512 + (4 * cc + jj * SPS + sslot_b) * 32 + 8 * tig;
+          const int8_t* xp = bon[q] ? c.xdig + x_off(c.xpitch, xtok[q], dig_b, e) : c.zero + 8 * tig;
           const uint2 bl = *reinterpret_cast<const uint2*>(xp);
 #pragma unroll
           for (int sl = 0; sl < SPS; ++sl) {
@@ -497,10 +496,8 @@ __device__ __forceinline__ bool gu_unit_multi(const GuTmaArgs& a, const GuCtx& c
             else
               mma_s8s8(acc[q], af[u][0][0], af[u][1][0], af[u][0][1], af[u][1][1], b0, b1);
           }
-          const int sbi = 4 * cc + jj * SPS + sslot_c;
-          const int odd0 = gu_odd(rg, sbi, g), odd1 = gu_odd(rg + 1024, sbi, g);
-          iacc[q][0] += (acc[q][0] * 128 + acc[q][1]) * odd0;
-          iacc[q][1] += (acc[q][2] * 128 + acc[q][3]) * odd1;
+          iacc[q][0] += (acc[q][0] * 128 + acc[q][1]) * odd0[jj];
+          iacc[q][1] += (acc[q][2] * 128 + acc[q][3]) * odd1[jj];
         }
       }
       {  // every four sub-blocks: with 14-bit activation digits a longer int32 sum could overflow
@@ -633,14 +630,16 @@ __device__ __forceinline__ void gu_consume_t1(const GuTmaArgs& a, const MetaSmem
 struct GuPlan {
   size_t tab, meta, zero, x, xs, ring, bars, total;
 };
-__host__ __device__ inline GuPlan gu_plan(int E, int T, int k, int H, bool xs_in, int S) {
+// Hx: the activation columns staged per CTA (all of H for one token; for more
+// tokens the CTA's fixed NB*512-column slice).
+__host__ __device__ inline GuPlan gu_plan(int E, int T, int k, int Hx, bool xs_in, int S) {
   GuPlan p;
   p.tab = 0;
   p.meta = kTabBytes;
   p.zero = p.meta + meta_bytes(E, T * k, true);
   p.x = p.zero + kZeroBytes;
-  p.xs = p.x + (xs_in ? align_up(static_cast<size_t>(T) * 2 * H, 128) : 0);
-  const size_t end = p.xs + (xs_in ? align_up(static_cast<size_t>(T) * (H / 256) * 4, 128) : 0);
+  p.xs = p.x + (xs_in ? align_up(static_cast<size_t>(T) * 2 * Hx, 128) : 0);
+  const size_t end = p.xs + (xs_in ? align_up(static_cast<size_t>(T) * (Hx / 256) * 4, 128) : 0);
   p.ring = align_up(end, 1024);
   p.bars = p.ring + static_cast<size_t>(S) * kGuBox;
   p.total = p.bars + (2 * static_cast<size_t>(S) + 1) * 8;  // full[S], empty[S], the table copy
@@ -656,7 +655,13 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H, I = a.I, T = a.T, S = a.S, NB = a.NB;
   const int nA = T * a.k;
-  const GuPlan pl = gu_plan(a.E, T, a.k, H, XS, S);
+  // staged activation columns: all of H for one token; otherwise the CTA serves one fixed part kpc of H
+  // (units walked over (slot, m, rb) by the CTAs of that part) and stages that NB*512-column slice only
+  const int Hx = MAXQ == 1 ? H : NB * 512;
+  const int kpc = MAXQ == 1 ? 0 : static_cast<int>(blockIdx.x % a.KP);
+  const int kib = MAXQ == 1 ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x / a.KP);
+  const int kG = MAXQ == 1 ? static_cast<int>(gridDim.x) : static_cast<int>((gridDim.x - kpc + a.KP - 1) / a.KP);
+  const GuPlan pl = gu_plan(a.E, T, a.k, Hx, XS, S);
   MetaSmem ms;
   ms.off = reinterpret_cast<int32_t*>(smem + pl.meta);
   ms.act = ms.off + (a.E + 1);
@@ -698,15 +703,16 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
       const uint64_t pol = l2_policy_evict_first();  // expert codes are read once per step
       RingPos rp{0, 0u};
       GuIter t;
-      t.init(blockIdx.x, gridDim.x, a.KP, rbs);
-      for (; t.slot < nact; t.next(a.KP, rbs)) {
+      t.init(kib, kG, MAXQ == 1 ? a.KP : 1, rbs);
+      for (; t.slot < nact; t.next(MAXQ == 1 ? a.KP : 1, rbs)) {
         const int e = ms.act[t.slot];
+        const int kp = MAXQ == 1 ? t.kp : kpc;
         for (int j = 0; j < NB; ++j) {
           if (!mbar_wait_bounded(&empty[rp.s], rp.ph ^ 1u, a.err, ERR_TIMEOUT, a.wait_limit)) return;
           mbar_arrive_expect_tx(&full[rp.s], kGuBox);
           index_ok(static_cast<size_t>(e) * I + t.rb * kBoxRows + kBoxRows - 1, static_cast<size_t>(a.E) * I);
-          index_ok(static_cast<size_t>(t.kp * NB + j) * kGuW + kGuW - 1, static_cast<size_t>(H) / 4);
-          tma_load_2d_hint(ring + rp.s * kGuBox, t.m ? &tm_up : &tm_gate, (t.kp * NB + j) * kGuW,
+          index_ok(static_cast<size_t>(kp * NB + j) * kGuW + kGuW - 1, static_cast<size_t>(H) / 4);
+          tma_load_2d_hint(ring + rp.s * kGuBox, t.m ? &tm_up : &tm_gate, (kp * NB + j) * kGuW,
                            e * I + t.rb * kBoxRows, &full[rp.s], pol);
           rp.next(S);
         }
@@ -716,13 +722,19 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
   }
 
   // consumers: stage the activations while the first boxes are in flight
-  if (XS) {  // [T][2][H] digits -> the staged layout of x_off, 16 bytes at a time, asynchronously
-    const int per = H / 16;
+  if (XS) {  // columns [kpc Hx, kpc Hx + Hx) of the [T][2][H] digits -> the x_off layout of an Hx-column
+             // matrix, 16 bytes at a time, asynchronously; their 2^s/8 scales likewise
+    const int per = Hx / 16;
     for (int i = tid; i < T * 2 * per; i += kCW * 32) {
       const int row = i / per, e = (i - row * per) * 16;
-      cp_async16(smem_addr(xsm + x_off(H, row >> 1, row & 1, e)), a.xd + static_cast<size_t>(i) * 16);
+      cp_async16(smem_addr(xsm + x_off(Hx, row >> 1, row & 1, e)),
+                 a.xd + static_cast<size_t>(row) * H + static_cast<size_t>(kpc) * Hx + e);
     }
-    for (int i = tid; i < T * (H / 256); i += kCW * 32) xssm[i] = a.xs[i];
+    const int bpr = Hx / 256;
+    for (int i = tid; i < T * bpr; i += kCW * 32) {
+      const int tt = i / bpr;
+      xssm[i] = a.xs[tt * (H / 256) + kpc * bpr + (i - tt * bpr)];
+    }
     cp_async_wait_all();
   }
   named_barrier(1, kCW * 32);
@@ -737,17 +749,10 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
   c.ring = ring;
   c.full = full;
   c.empty = empty;
-  if (XS) {
-    c.xdig = xsm;
-    c.xscl = xssm;
-    c.zero = zero;
-    c.xpitch = 0;  // staged layout: x_off
-  } else {
-    c.xdig = a.xd;
-    c.xscl = a.xs;
-    c.zero = g_zero_operand;
-    c.xpitch = H;
-  }
+  c.xdig = xsm;  // the staged slice (x_off layout of an Hx-column matrix)
+  c.xscl = xssm;
+  c.zero = zero;
+  c.xpitch = Hx;
   c.ring_s = smem_addr(ring);
   c.x_s = smem_addr(xsm);
   c.xs_s = smem_addr(xssm);
@@ -778,11 +783,12 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
   };
   RingPos rp{0, 0u};
   GuIter t;
-  t.init(blockIdx.x, gridDim.x, a.KP, rbs);
+  t.init(kib, kG, 1, rbs);
   uint32_t nd[kMaxNB][2] = {};
   GuUnit nw{};
   if (t.slot < nact) {
     nw = gu_unit_of(t, ms);
+    nw.kp = kpc;
     dload(nw, nd);
   }
   while (t.slot < nact) {
@@ -790,9 +796,10 @@ __global__ void __launch_bounds__(kThreadsT, 1) gateup_tma_kernel(const __grid_c
     uint32_t d[kMaxNB][2];
 #pragma unroll
     for (int j = 0; j < kMaxNB; ++j) d[j][0] = nd[j][0], d[j][1] = nd[j][1];
-    t.next(a.KP, rbs);
+    t.next(1, rbs);
     if (t.slot < nact) {
       nw = gu_unit_of(t, ms);
+      nw.kp = kpc;
       dload(nw, nd);
     }
     bool ok;
@@ -876,6 +883,7 @@ struct DnCtx {
   const int8_t* zero;  // 128-byte aligned zero region
   uint32_t ring_s, hd_s, hsc_s, hq_s;  // shared-window addresses (staged variant)
   int warp, lane, g, tig, S;
+  int hI, hqp, hsp;  // h_off pitch, hq and hsc entries per assignment (staged slice or global)
 };
 
 __device__ __forceinline__ float dn_block(uint32_t dd, float e2, int iA, int iM) {
@@ -904,7 +912,7 @@ __device__ __forceinline__ void q2k_sub4(uint32_t w, uint32_t& r0, uint32_t& r1,
 template <bool HS>
 __device__ __forceinline__ bool dn_unit_one(const DnTmaArgs& a, const DnCtx& c, RingPos& rp, const DnUnit& w,
                                             const uint32_t (&dd)[kMaxNB][2]) {
-  const int H = a.H, I = a.I, NB = a.NB;
+  const int H = a.H, NB = a.NB;
   const int g = c.g, tig = c.tig;
   const bool bact = (g >> 1) == tig;
   const int row = 16 * c.warp + g;
@@ -913,18 +921,18 @@ __device__ __forceinline__ bool dn_unit_one(const DnTmaArgs& a, const DnCtx& c, 
   float f0 = 0.f, f1 = 0.f;
 #pragma unroll 1
   for (int j = 0; j < NB; ++j) {
-    const int blk = w.dp * NB + j;  // block of I
-    const int hb = h_off(I, w.p0, g & 1, blk * 256 + 64 * tig);  // sub-block 4 tig, round 0
-    const int hqi = w.p0 * (I / 16) + blk * 16 + 4 * tig;
+    const int blk = (HS ? 0 : w.dp * NB) + j;  // block of the staged slice, or of I
+    const int hb = h_off(c.hI, w.p0, g & 1, blk * 256 + 64 * tig);  // sub-block 4 tig, round 0
+    const int hqi = w.p0 * c.hqp + blk * 16 + 4 * tig;
     int4 hq4;
     float e2;
     if (HS) {
       const uint4 v = ld_s128(c.hq_s + hqi * 4);
       hq4 = make_int4(static_cast<int>(v.x), static_cast<int>(v.y), static_cast<int>(v.z), static_cast<int>(v.w));
-      e2 = ld_sf(c.hsc_s + (w.p0 * a.hss + blk) * 4);
+      e2 = ld_sf(c.hsc_s + (w.p0 * c.hsp + blk) * 4);
     } else {
       hq4 = __ldcg(reinterpret_cast<const int4*>(c.hq + hqi));
-      e2 = __ldcg(c.hsc + w.p0 * a.hss + blk);
+      e2 = __ldcg(c.hsc + w.p0 * c.hsp + blk);
     }
     if (!mbar_wait_bounded(&c.full[rp.s], rp.ph, a.err, ERR_TIMEOUT)) return false;
     const uint32_t st = c.ring_s + rp.s * kDnStage;
@@ -978,10 +986,11 @@ __device__ __forceinline__ bool dn_unit_one(const DnTmaArgs& a, const DnCtx& c, 
 // One down unit for an expert with 2..2*MAXQ assignments. Each MMA takes a pair
 // of sub-blocks (2pr, 2pr + 1), lane tig bit pair tig of their bytes; MMA
 // columns: (token slot 0..1) x (half 0..1) x (digit hi, lo).
-template <int MAXQ>
+template <int MAXQ, bool HS>
 __device__ __forceinline__ bool dn_unit_multi(const DnTmaArgs& a, const DnCtx& c, RingPos& rp, const DnUnit& w,
                                               const uint32_t (&dd)[kMaxNB][2]) {
-  const int H = a.H, I = a.I, ne = w.ne, p0 = w.p0;
+  const int H = a.H, ne = w.ne, p0 = w.p0;
+  const int bb0 = HS ? 0 : w.dp * a.NB;  // first block of the unit in the staged slice, or in I
   const int g = c.g, tig = c.tig;
   const int ngroups = (ne + 1) / 2;
   const int dig_b = g & 1, hb = (g >> 1) & 1, sl_b = g >> 2;
@@ -996,8 +1005,8 @@ __device__ __forceinline__ bool dn_unit_multi(const DnTmaArgs& a, const DnCtx& c
     const int tb = 2 * q + sl_b, tc = 2 * q + sl_c;
     pb[q] = (q < ngroups && tb < ne) ? p0 + tb : -1;
     const bool cv = q < ngroups && tc < ne;
-    hq_ptr[q] = c.hq + (p0 + (cv ? tc : 0)) * (I / 16) + w.dp * a.NB * 16 + hc;
-    e2p[q] = cv ? c.hsc + (p0 + tc) * a.hss + w.dp * a.NB : nullptr;
+    hq_ptr[q] = c.hq + (p0 + (cv ? tc : 0)) * c.hqp + bb0 * 16 + hc;
+    e2p[q] = cv ? c.hsc + (p0 + tc) * c.hsp + bb0 : nullptr;
   }
   float facc[MAXQ][2];
 #pragma unroll
@@ -1016,7 +1025,7 @@ __device__ __forceinline__ bool dn_unit_multi(const DnTmaArgs& a, const DnCtx& c
     const uint8_t* st = c.ring + s * kDnStage;
     const uint8_t* sA = st + kDnQBytes + row * 16;
     const uint8_t* sB = sA + 8 * 16;
-    const int blk = w.dp * a.NB + j;
+    const int blk = bb0 + j;
 #pragma unroll 1
     for (int cc = 0; cc < 4; ++cc) {  // logical 16-byte chunk cc of the q bytes: sub-blocks 4cc .. 4cc + 3
       const uint4 qa = lds128(st + qoff + 16 * (cc ^ qsw));
@@ -1037,7 +1046,7 @@ __device__ __forceinline__ bool dn_unit_multi(const DnTmaArgs& a, const DnCtx& c
           if (q >= ngroups) break;
           uint32_t b0 = 0u, b1 = 0u;
           if (pb[q] >= 0) {  // bit pair tig of sub-block 2pr + hb: bytes 4 tig .. 4 tig + 3 (elements tig + 4i)
-            const int8_t* hp = c.hd + h_off(I, pb[q], dig_b, blk * 256 + (2 * pr + hb) * 16 + tig);
+            const int8_t* hp = c.hd + h_off(c.hI, pb[q], dig_b, blk * 256 + (2 * pr + hb) * 16 + tig);
             const uint32_t v = *reinterpret_cast<const uint32_t*>(hp);
             if (hb == 0) b0 = v;
             else b1 = v;
@@ -1154,14 +1163,16 @@ __device__ __forceinline__ void dn_consume_t1(const DnTmaArgs& a, const MetaSmem
 struct DnPlan {
   size_t meta, zero, hd, hsc, hq, ring, bars, total;
 };
-__host__ __device__ inline DnPlan dn_plan(int E, int nA, int I, int hss, bool hs_in, int S) {
+// Ix, hssx: the h columns and scale entries staged per assignment (all of I for
+// one token; for more tokens the CTA's fixed NB*256-column slice, NB scales).
+__host__ __device__ inline DnPlan dn_plan(int E, int nA, int Ix, int hssx, bool hs_in, int S) {
   DnPlan p;
   p.meta = 0;
   p.zero = meta_bytes(E, nA, false);
   p.hd = p.zero + kZeroBytes;
-  p.hsc = p.hd + (hs_in ? align_up(static_cast<size_t>(nA) * 2 * I, 128) : 0);
-  p.hq = p.hsc + (hs_in ? align_up(static_cast<size_t>(nA) * hss * 4, 128) : 0);
-  const size_t end = p.hq + (hs_in ? align_up(static_cast<size_t>(nA) * (I / 16) * 4, 128) : 0);
+  p.hsc = p.hd + (hs_in ? align_up(static_cast<size_t>(nA) * 2 * Ix, 128) : 0);
+  p.hq = p.hsc + (hs_in ? align_up(static_cast<size_t>(nA) * hssx * 4, 128) : 0);
+  const size_t end = p.hq + (hs_in ? align_up(static_cast<size_t>(nA) * (Ix / 16) * 4, 128) : 0);
   p.ring = align_up(end, 1024);
   p.bars = p.ring + static_cast<size_t>(S) * kDnStage;
   p.total = p.bars + 2 * static_cast<size_t>(S) * 8;
@@ -1177,7 +1188,14 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H, I = a.I, S = a.S, NB = a.NB;
   const int nA = a.T * a.k;
-  const DnPlan pl = dn_plan(a.E, nA, I, a.hss, HS, S);
+  // staged h: all of I for one token; for more tokens (HS) the CTA serves one fixed part dpc of I (units
+  // walked over (slot, rb) by the CTAs of that part) and stages that NB*256-column slice of every assignment
+  const bool slice = MAXQ > 1 && HS;
+  const int Ix = slice ? NB * 256 : I, hssx = slice ? NB : a.hss;
+  const int dpc = slice ? static_cast<int>(blockIdx.x % a.DP) : 0;
+  const int dib = slice ? static_cast<int>(blockIdx.x / a.DP) : static_cast<int>(blockIdx.x);
+  const int dG = slice ? static_cast<int>((gridDim.x - dpc + a.DP - 1) / a.DP) : static_cast<int>(gridDim.x);
+  const DnPlan pl = dn_plan(a.E, nA, Ix, hssx, HS, S);
   MetaSmem ms;
   ms.off = reinterpret_cast<int32_t*>(smem + pl.meta);
   ms.act = ms.off + (a.E + 1);
@@ -1215,13 +1233,14 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
       const uint64_t pol = l2_policy_evict_first();  // expert codes are read once per step
       RingPos rp{0, 0u};
       DnIter t;
-      t.init(blockIdx.x, gridDim.x, a.DP, rbs);
-      for (; t.slot < nact; t.next(a.DP, rbs)) {
+      t.init(dib, dG, slice ? 1 : a.DP, rbs);
+      for (; t.slot < nact; t.next(slice ? 1 : a.DP, rbs)) {
         const int e = ms.act[t.slot];
+        const int dp = slice ? dpc : t.dp;
         for (int j = 0; j < NB; ++j) {
           if (!mbar_wait_bounded(&empty[rp.s], rp.ph ^ 1u, a.err, ERR_TIMEOUT)) return;
           mbar_arrive_expect_tx(&full[rp.s], kDnStage);
-          const int x0 = (t.dp * NB + j) * 80, y0 = e * H + t.rb * kBoxRows;
+          const int x0 = (dp * NB + j) * 80, y0 = e * H + t.rb * kBoxRows;
           index_ok(static_cast<size_t>(y0) + kBoxRows - 1, static_cast<size_t>(a.E) * H);
           index_ok(static_cast<size_t>(x0) + 79, static_cast<size_t>(I / 256) * 80);
           uint8_t* st = ring + rp.s * kDnStage;
@@ -1235,10 +1254,22 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
   }
   // consumers: stage h while the first boxes are in flight (the h_off layout is the same in global and
   // shared memory; I % 256 == 0 makes both byte counts multiples of 16)
-  if (HS) {
-    for (int i = tid; i < nA * 2 * I / 16; i += kCW * 32) cp_async16(smem_addr(hd_s) + 16u * i, a.hd + 16 * static_cast<size_t>(i));
-    for (int i = tid; i < nA * (I / 64); i += kCW * 32) cp_async16(smem_addr(hq_s) + 16u * i, a.hq + 4 * static_cast<size_t>(i));
-    for (int i = tid; i < nA * a.hss; i += kCW * 32) hsc_s[i] = a.hsc[i];
+  if (HS) {  // per assignment: h digits of blocks [dpc NB, dpc NB + NB) (contiguous in the h_off layout, here
+             // and in the slice), their per-16 sums and their scales; with slice == false all of them
+    const int hc = Ix / 8, qc = Ix / 64;  // 16-byte chunks per assignment: h digits, per-16 sums
+    for (int i = tid; i < nA * hc; i += kCW * 32) {
+      const int pp = i / hc, cidx = i - pp * hc;
+      cp_async16(smem_addr(hd_s) + 16u * i,
+                 a.hd + static_cast<size_t>(pp) * 2 * I + static_cast<size_t>(dpc) * NB * 512 + 16 * cidx);
+    }
+    for (int i = tid; i < nA * qc; i += kCW * 32) {
+      const int pp = i / qc, cidx = i - pp * qc;
+      cp_async16(smem_addr(hq_s) + 16u * i, a.hq + static_cast<size_t>(pp) * (I / 16) + dpc * NB * 16 + 4 * cidx);
+    }
+    for (int i = tid; i < nA * hssx; i += kCW * 32) {
+      const int pp = i / hssx;
+      hsc_s[i] = a.hsc[static_cast<size_t>(pp) * a.hss + dpc * NB + (i - pp * hssx)];
+    }
     cp_async_wait_all();
   }
   named_barrier(1, kCW * 32);
@@ -1270,6 +1301,9 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
   c.g = lane >> 2;
   c.tig = lane & 3;
   c.S = S;
+  c.hI = HS ? Ix : I;
+  c.hqp = (HS ? Ix : I) / 16;
+  c.hsp = HS ? hssx : a.hss;
   const int row_l = 16 * warp + c.g;
   const int nblk = I / 256;
   auto ddload = [&](const DnUnit& w, uint32_t (&d)[kMaxNB][2]) {
@@ -1284,11 +1318,12 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
   };
   RingPos rp{0, 0u};
   DnIter t;
-  t.init(blockIdx.x, gridDim.x, a.DP, rbs);
+  t.init(dib, dG, slice ? 1 : a.DP, rbs);
   uint32_t nd[kMaxNB][2] = {};
   DnUnit nw{};
   if (t.slot < nact) {
     nw = dn_unit_of(t, ms);
+    if (slice) nw.dp = dpc;
     ddload(nw, nd);
   }
   while (t.slot < nact) {
@@ -1296,14 +1331,15 @@ __global__ void __launch_bounds__(kThreadsT, 1) down_tma_kernel(const __grid_con
     uint32_t d[kMaxNB][2];
 #pragma unroll
     for (int j = 0; j < kMaxNB; ++j) d[j][0] = nd[j][0], d[j][1] = nd[j][1];
-    t.next(a.DP, rbs);
+    t.next(slice ? 1 : a.DP, rbs);
     if (t.slot < nact) {
       nw = dn_unit_of(t, ms);
+      if (slice) nw.dp = dpc;
       ddload(nw, nd);
     }
     bool ok;
     if (MAXQ == 1 || w.ne == 1) ok = dn_unit_one<HS>(a, c, rp, w, d);
-    else ok = dn_unit_multi<(MAXQ > 1 ? MAXQ : 1)>(a, c, rp, w, d);
+    else ok = dn_unit_multi<(MAXQ > 1 ? MAXQ : 1), HS>(a, c, rp, w, d);
     if (!ok) return;
   }
 }
@@ -1466,24 +1502,21 @@ int launch_gateup_tma(const LayerShape& sh, const uint8_t* gate_codes, const uin
   a.wait_limit = g_inject_mode ? g_inject_limit : kDefaultWaitCycles;
   // stage the activations when that still leaves three ring stages
   const size_t budget = kBudget;
-  const bool xs_in = gu_plan(sh.E, T, sh.k, sh.H, true, 3).total <= budget;
+  const int Hx = T == 1 ? sh.H : a.NB * 512;  // staged activation columns per CTA (see the kernel)
+  const bool xs_in = gu_plan(sh.E, T, sh.k, Hx, true, 3).total <= budget;
   int S = 2;
-  while (S < 6 && gu_plan(sh.E, T, sh.k, sh.H, xs_in, S + 1).total <= budget) ++S;
-  if (gu_plan(sh.E, T, sh.k, sh.H, xs_in, S).total > budget) return ERR_SHAPE;
+  while (S < 6 && gu_plan(sh.E, T, sh.k, Hx, xs_in, S + 1).total <= budget) ++S;
+  if (!xs_in || gu_plan(sh.E, T, sh.k, Hx, xs_in, S).total > budget) return ERR_SHAPE;
   a.S = S;
-  const size_t smem = gu_plan(sh.E, T, sh.k, sh.H, xs_in, S).total;
+  const size_t smem = gu_plan(sh.E, T, sh.k, Hx, xs_in, S).total;
   const size_t nA = static_cast<size_t>(T) * sh.k;
   const int slots = static_cast<int>(std::min<size_t>(nA, static_cast<size_t>(sh.E)));
   const int units = slots * 2 * (sh.I / kBoxRows) * a.KP;
   const int grid = std::max(1, std::min(units, sms));
-  if (T == 1) {  // one token: the single-assignment variant with staged activations
-    if (!xs_in) return ERR_SHAPE;
+  if (T == 1)  // one token: the single-assignment variant with staged activations
     launch_k(gateup_tma_kernel<1, true>, grid, smem, st, tg, tu, a);
-  } else if (xs_in) {  // at most 16 tokens per expert: four groups of four
+  else  // at most 16 tokens per expert: four groups of four, each CTA on one part of H
     launch_k(gateup_tma_kernel<4, true>, grid, smem, st, tg, tu, a);
-  } else {
-    launch_k(gateup_tma_kernel<4, false>, grid, smem, st, tg, tu, a);
-  }
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
 }
 
@@ -1502,12 +1535,14 @@ int launch_down_tma(const LayerShape& sh, const uint8_t* down_codes, const uint3
   a.offsets = r.offsets; a.active = r.active; a.opart = opart; a.err = err;
   const int nA = T * sh.k;
   a.opart_n = static_cast<size_t>(nA) * a.DP * sh.H;
-  const bool hs_in = dn_plan(sh.E, nA, sh.I, hss, true, 4).total <= kBudget;
+  // staged h per assignment: all of I for one token, a slice of NB*256 columns for more (see the kernel)
+  const int Ix = T == 1 ? sh.I : a.NB * 256, hssx = T == 1 ? hss : a.NB;
+  const bool hs_in = dn_plan(sh.E, nA, Ix, hssx, true, 3).total <= kBudget;
   int S = 2;
-  while (S < 8 && dn_plan(sh.E, nA, sh.I, hss, hs_in, S + 1).total <= kBudget) ++S;
-  if (dn_plan(sh.E, nA, sh.I, hss, hs_in, S).total > kBudget) return ERR_SHAPE;
+  while (S < 8 && dn_plan(sh.E, nA, Ix, hssx, hs_in, S + 1).total <= kBudget) ++S;
+  if (dn_plan(sh.E, nA, Ix, hssx, hs_in, S).total > kBudget) return ERR_SHAPE;
   a.S = S;
-  const size_t smem = dn_plan(sh.E, nA, sh.I, hss, hs_in, S).total;
+  const size_t smem = dn_plan(sh.E, nA, Ix, hssx, hs_in, S).total;
   const int slots = std::min(nA, sh.E);
   const int units = slots * (sh.H / kBoxRows) * a.DP;
   const int grid = std::max(1, std::min(units, sms));

@@ -452,58 +452,83 @@ __global__ void __launch_bounds__(32) topk_permute_warp_kernel(const float* __re
   if (lane == 0) active[E] = nact;
 }
 
-// The same outputs for T * k <= 32 and T * E <= kRankMaxLogits by one CTA,
-// without serial rounds: every logit counts the logits of its token that rank
-// above it (greater, or equal with a lower expert index; NaN ranks as -inf),
-// and the k with a count below k write themselves into their slot. The weights
-// are summed in slot order by one thread per token, as in topk_warp. The
-// permutation is computed in parallel from the chosen experts in shared
-// memory: assignment j goes to (assignments with a smaller expert) + (earlier
-// ones with the same expert), offsets[x] counts the assignments below x, and
-// the first assignment of each distinct expert writes it into the active list
-// at the number of distinct experts below it.
-constexpr int kRankMaxLogits = 4096;
-__global__ void __launch_bounds__(256) topk_permute_rank_kernel(const float* __restrict__ logits, int T, int E, int k,
-                                                                int32_t* __restrict__ topk_idx,
-                                                                float* __restrict__ topk_w,
-                                                                int32_t* __restrict__ offsets,
-                                                                int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-                                                                int32_t* __restrict__ active) {
-  __shared__ __align__(16) float ls[kRankMaxLogits];
+// The same outputs for T * k <= 32, k <= 32 and T * ceil(E / 32) <= 32 by one
+// CTA of T * ceil(E / 32) warps. Order: larger logit first, equal logits by
+// lower expert index (NaN ranks as -inf, padding after every expert). Warp w of
+// token t sorts experts 32w..32w+31 with a bitonic network of shuffles; its
+// first min(k, 32) are the only ones that can be among the token's k, and
+// among those candidates each counts the ones ranked above it: the k with a
+// count below k write themselves into their slot. The weights are summed in
+// slot order by one thread per token, as in topk_warp. The permutation is
+// computed in parallel from the chosen experts in shared memory: assignment j
+// goes to (assignments with a smaller expert) + (earlier ones with the same
+// expert), offsets[x] counts the assignments below x, and the first assignment
+// of each distinct expert writes it into the active list at the number of
+// distinct experts below it.
+__device__ __forceinline__ bool ranks_before(float av, int ai, float bv, int bi) {
+  return av > bv || (av == bv && ai < bi);
+}
+
+__global__ void __launch_bounds__(1024) topk_permute_sort_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                                 int32_t* __restrict__ topk_idx,
+                                                                 float* __restrict__ topk_w,
+                                                                 int32_t* __restrict__ offsets,
+                                                                 int32_t* __restrict__ perm,
+                                                                 int32_t* __restrict__ inv,
+                                                                 int32_t* __restrict__ active) {
+  __shared__ float cand_v[1024];
+  __shared__ int cand_i[1024];
   __shared__ int sel[32];
   __shared__ float chosen[32];
   __shared__ int first[32];
   pdl_trigger();
   pdl_wait();
-  const int tid = threadIdx.x, nthr = blockDim.x;
-  const int n = T * k;
-  for (int i = tid; i < T * E; i += nthr) {
-    const float v = logits[i];
-    ls[i] = v == v ? v : -INFINITY;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int W = (E + 31) / 32, kc = k < 32 ? k : 32, n = T * k;
+  const int t = warp / W, e = (warp - t * W) * 32 + lane;
+  float v = -INFINITY;
+  int idx = E + lane;  // padding ranks after every expert
+  if (e < E) {
+    const float l = logits[static_cast<size_t>(t) * E + e];
+    v = l == l ? l : -INFINITY;
+    idx = e;
   }
-  __syncthreads();
-  for (int i = tid; i < T * E; i += nthr) {
-    const int t = i / E, e = i - t * E;
-    const float v = ls[i];
-    const float* row = ls + t * E;
-    int rank = 0;
-    if ((E & 3) == 0) {  // rows start 16-byte aligned: four logits per load
-      for (int j = 0; j < E; j += 4) {
-        const float4 u = *reinterpret_cast<const float4*>(row + j);
-        rank += (u.x > v || (u.x == v && j < e)) ? 1 : 0;
-        rank += (u.y > v || (u.y == v && j + 1 < e)) ? 1 : 0;
-        rank += (u.z > v || (u.z == v && j + 2 < e)) ? 1 : 0;
-        rank += (u.w > v || (u.w == v && j + 3 < e)) ? 1 : 0;
-      }
-    } else {
-      for (int j = 0; j < E; ++j) {
-        const float u = row[j];
-        rank += (u > v || (u == v && j < e)) ? 1 : 0;
+  // bitonic sort of the warp's 32 keys into rank order
+#pragma unroll
+  for (int kk = 2; kk <= 32; kk <<= 1) {
+#pragma unroll
+    for (int j = kk >> 1; j > 0; j >>= 1) {
+      const float pv = __shfl_xor_sync(0xffffffffu, v, j);
+      const int pi = __shfl_xor_sync(0xffffffffu, idx, j);
+      const bool p_first = ranks_before(pv, pi, v, idx);
+      const bool lower = (lane & j) == 0, fwd = (lane & kk) == 0;
+      // in a forward block the lower lane keeps the key that ranks first
+      if (lower == fwd ? p_first : !p_first) {
+        v = pv;
+        idx = pi;
       }
     }
-    if (rank < k) {
-      sel[t * k + rank] = e;
-      chosen[t * k + rank] = v;
+  }
+  const int wt = warp - t * W;  // warp within the token
+  if (lane < kc) {
+    cand_v[t * W * kc + wt * kc + lane] = v;
+    cand_i[t * W * kc + wt * kc + lane] = idx;
+  }
+  __syncthreads();
+  {
+    const int nc = W * kc;  // candidates of a token
+    const int ct = tid / nc, c = tid - ct * nc;
+    if (ct < T) {
+      const float* cv = cand_v + ct * nc;
+      const int* ci = cand_i + ct * nc;
+      const float mv = cv[c];
+      const int mi = ci[c];
+      int rank = 0;
+      for (int j = 0; j < nc; ++j) rank += ranks_before(cv[j], ci[j], mv, mi) ? 1 : 0;
+      if (rank < k) {
+        sel[ct * k + rank] = mi;
+        chosen[ct * k + rank] = mv;
+      }
     }
   }
   __syncthreads();
@@ -517,28 +542,28 @@ __global__ void __launch_bounds__(256) topk_permute_rank_kernel(const float* __r
     }
   }
   if (tid < n) {
-    const int e = sel[tid];
+    const int ej = sel[tid];
     int below = 0, fst = 1;
     for (int j = 0; j < n; ++j) {
-      const int ej = sel[j];
-      below += (ej < e || (ej == e && j < tid)) ? 1 : 0;
-      if (ej == e && j < tid) fst = 0;
+      const int ei = sel[j];
+      below += (ei < ej || (ei == ej && j < tid)) ? 1 : 0;
+      if (ei == ej && j < tid) fst = 0;
     }
     perm[below] = tid;
     inv[tid] = below;
     first[tid] = fst;
   }
   __syncthreads();
-  for (int x = tid; x <= E; x += nthr) {
+  for (int x = tid; x <= E; x += blockDim.x) {
     int lt = 0;
     for (int j = 0; j < n; ++j) lt += sel[j] < x ? 1 : 0;
     offsets[x] = x == E ? n : lt;
   }
   if (tid < n && first[tid]) {
-    const int e = sel[tid];
+    const int ej = sel[tid];
     int pos = 0;
-    for (int j = 0; j < n; ++j) pos += (first[j] && sel[j] < e) ? 1 : 0;
-    active[pos] = e;
+    for (int j = 0; j < n; ++j) pos += (first[j] && sel[j] < ej) ? 1 : 0;
+    active[pos] = ej;
   }
   if (tid == 0) {
     int nact = 0;
@@ -600,10 +625,10 @@ int launch_route(const uint16_t* Wr, const float* bias, const void* x, int x_dty
     }
   }
   const size_t psmem = 32 * E * sizeof(uint16_t) + 3 * E * sizeof(int);
-  if (T * k <= 32 && T * E <= kRankMaxLogits) {
+  if (T * k <= 32 && k <= 32 && T * ((E + 31) / 32) <= 32) {
     ProfScope ps(MOE_K_PERMUTE, st);
-    launch_pdl(topk_permute_rank_kernel, dim3(1), dim3(256), 0, st, logits, T, E, k, topk_idx, topk_w, offsets, perm,
-               inv, active);
+    launch_pdl(topk_permute_sort_kernel, dim3(1), dim3(32 * T * ((E + 31) / 32)), 0, st, logits, T, E, k, topk_idx,
+               topk_w, offsets, perm, inv, active);
   } else if (T * k <= 32 && E <= 256) {
     ProfScope ps(MOE_K_PERMUTE, st);
     launch_pdl(topk_permute_warp_kernel<8>, dim3(1), dim3(32), 0, st, logits, T, E, k, topk_idx, topk_w, offsets,
