@@ -33,7 +33,12 @@ class Weights(ctypes.Structure):
             "router_w", "router_bias", "gate_codes", "gate_d", "up_codes", "up_d",
             "down_codes", "down_dd", "sh_gate", "sh_up", "sh_down",
         )
+    ] + [("expert_format", ctypes.c_int32)] + [
+        (n, ctypes.c_void_p) for n in ("gate_scales", "up_scales", "down_scales")
     ]
+
+
+FMT_IQ2_Q2K, FMT_MXFP4 = 0, 1
 
 
 def build(force: bool = False, openmp: bool | None = None) -> str:
@@ -86,6 +91,9 @@ def lib():
         L.moeref_grid.argtypes = [vp]
         L.moeref_dequant_iq2.argtypes = [vp, vp, i64, vp]
         L.moeref_dequant_q2k.argtypes = [vp, vp, i64, vp]
+        L.moeref_e2m1.restype = ctypes.c_double
+        L.moeref_e2m1.argtypes = [ctypes.c_uint]
+        L.moeref_dequant_mxfp4.argtypes = [vp, vp, i64, vp]
         L.moeref_route.argtypes = [i32, i32, i32, vp, vp, vp, i32, i32, vp, vp, vp]
         L.moeref_permute.argtypes = [i32, i32, i32, vp, vp, vp, vp]
         L.moeref_f32_to_f16.restype = ctypes.c_uint16
@@ -151,6 +159,21 @@ def dequant_q2k(codes: np.ndarray, dd: np.ndarray) -> np.ndarray:
     return out
 
 
+def e2m1(c: int) -> float:
+    """The value of one FP4 E2M1 element code (OCP MX v1.0)."""
+    return float(lib().moeref_e2m1(int(c)))
+
+
+def dequant_mxfp4(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """MXFP4 blocks (codes [nb][16] u8, E8M0 scales [nb] u8) -> fp32 [nb * 32]."""
+    codes = np.ascontiguousarray(codes, np.uint8).reshape(-1, 16)
+    scales = np.ascontiguousarray(scales, np.uint8).reshape(-1)
+    assert codes.shape[0] == scales.shape[0]
+    out = np.zeros(codes.shape[0] * 32, np.float32)
+    lib().moeref_dequant_mxfp4(_p(codes), _p(scales), codes.shape[0], _p(out))
+    return out
+
+
 def f32_to_f16(v: float) -> int:
     return int(lib().moeref_f32_to_f16(float(v)))
 
@@ -202,11 +225,17 @@ def permute(idx: np.ndarray, E: int):
 
 
 def _structs(lw):
+    """Oracle structs of a layer; a layer with ``fmt == "mxfp4"`` carries MXFP4
+    code planes and E8M0 scale planes instead of the IQ2 / Q2K planes."""
     desc = Desc(lw.H, lw.I, lw.E, lw.k, lw.Is)
-    keep = [np.ascontiguousarray(a) if a is not None else None for a in (
-        lw.router_w, lw.router_bias, lw.gate_codes, lw.gate_d, lw.up_codes, lw.up_d,
-        lw.down_codes, lw.down_dd, lw.sh_gate, lw.sh_up, lw.sh_down)]
-    W = Weights(*[_p(a) for a in keep])
+    mx = getattr(lw, "fmt", "iq2") == "mxfp4"
+    arrs = (lw.router_w, lw.router_bias, lw.gate_codes, None if mx else lw.gate_d, lw.up_codes,
+            None if mx else lw.up_d, lw.down_codes, None if mx else lw.down_dd, lw.sh_gate, lw.sh_up, lw.sh_down)
+    keep = [np.ascontiguousarray(a) if a is not None else None for a in arrs]
+    sc = [np.ascontiguousarray(getattr(lw, n)) for n in ("gate_scales", "up_scales", "down_scales")] if mx else []
+    keep += sc
+    W = Weights(*[_p(a) for a in keep[:11]], FMT_MXFP4 if mx else FMT_IQ2_Q2K,
+                *([_p(a) for a in sc] if mx else [None, None, None]))
     return desc, W, keep
 
 

@@ -54,7 +54,16 @@ typedef struct {
   const uint16_t* sh_gate;   /* bf16 [Is][H] */
   const uint16_t* sh_up;     /* bf16 [Is][H] */
   const uint16_t* sh_down;   /* bf16 [H][Is] */
+  /* second expert format: REF_FMT_MXFP4 takes the routed matrices from the
+     code planes above read as MXFP4 codes [rows][K/2] with these E8M0 planes
+     [rows][K/32]; the d / dd planes are then unused */
+  int32_t expert_format;
+  const uint8_t* gate_scales;
+  const uint8_t* up_scales;
+  const uint8_t* down_scales;
 } moeref_weights;
+
+enum { REF_FMT_IQ2_Q2K = 0, REF_FMT_MXFP4 = 1 };
 
 /* ---------------------------------------------------------------- scalars */
 
@@ -178,6 +187,41 @@ void moeref_dequant_q2k(const uint8_t* codes, const uint32_t* dd, int64_t nblock
 /* Dequantise expert e's [rows][K] matrix into dense floats. Blocks run over the
  * row-major flattened index of the matrix, so when K < 256 one block spans
  * 256/K consecutive rows. */
+/* ------------------------------------------------------------------ MXFP4
+ * OCP Microscaling Formats (MX) v1.0: an MXFP4 block is 32 FP4 E2M1 elements
+ * and one E8M0 scale. E2M1: bit 3 sign, bits 2..1 exponent (bias 1), bit 0
+ * mantissa; exponent 0 is subnormal (value = mantissa * 2^(1-1) * 0.5), else
+ * (1 + mantissa / 2) * 2^(exponent - 1); no infinities or NaN. E8M0: the value
+ * 2^(E - 127) (E = 255 is NaN and is not used here). The library's packing:
+ * element 2i of a block in the low nibble of byte i, element 2i+1 in the high
+ * nibble ("ds4 : analyse pratique pour un usage documenté", « Support de
+ * modèles et choix de quantification », names the MXFP4 variant of the routed
+ * experts; the bits are the MX specification's).
+ * Parity: pinned by the specification's table of E2M1 values, E8M0 powers of
+ * two, a hand-decoded block and a dense float64 FFN over independently decoded
+ * weights. */
+double moeref_e2m1(unsigned c) {
+  const unsigned ex = (c >> 1) & 3u, man = c & 1u;
+  const double mag = ex == 0 ? 0.5 * man : (1.0 + 0.5 * man) * ldexp(1.0, (int)ex - 1);
+  return (c & 8u) ? -mag : mag;
+}
+
+void moeref_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t nblocks, float* out) {
+  for (int64_t b = 0; b < nblocks; ++b) {
+    const double sc = ldexp(1.0, (int)scales[b] - 127);
+    for (int i = 0; i < 32; ++i) {
+      const unsigned byte = codes[b * 16 + i / 2];
+      const unsigned c = (i & 1) ? (byte >> 4) : (byte & 15u);
+      out[b * 32 + i] = (float)(moeref_e2m1(c) * sc);
+    }
+  }
+}
+
+static void dequant_matrix_mxfp4(const uint8_t* codes, const uint8_t* scales, int e, int rows, int K, float* out) {
+  const int64_t nb = (int64_t)rows * K / 32;
+  moeref_dequant_mxfp4(codes + (int64_t)e * nb * 16, scales + (int64_t)e * nb, nb, out);
+}
+
 static void dequant_matrix_iq2(const uint8_t* codes, const uint16_t* d, int e, int rows, int K, float* out) {
   int64_t nb = (int64_t)rows * K / QK;
   moeref_dequant_iq2(codes + (int64_t)e * nb * IQ2_BYTES, d + (int64_t)e * nb, nb, out);
@@ -285,10 +329,13 @@ int moeref_expert_ffn(const moeref_desc* desc, const moeref_weights* W, const vo
   if (!desc || !W || T < 0) return REF_ERR_ARG;
   const int H = desc->hidden, I = desc->inter, E = desc->n_experts, k = desc->top_k, Is = desc->shared_inter;
   if (H <= 0 || I <= 0 || E <= 0 || k <= 0 || k > E || Is < 0) return REF_ERR_ARG;
-  if (((int64_t)H * I) % QK) return REF_ERR_SHAPE;
+  const int mx = W->expert_format == REF_FMT_MXFP4;
+  if (W->expert_format != REF_FMT_IQ2_Q2K && !mx) return REF_ERR_ARG;
+  if (((int64_t)H * I) % QK || (mx && (H % 32 || I % 32))) return REF_ERR_SHAPE;
   if (T == 0) return REF_OK;
-  if (!x || !topk_idx || !topk_w || !y || !W->gate_codes || !W->gate_d || !W->up_codes || !W->up_d ||
-      !W->down_codes || !W->down_dd)
+  if (!x || !topk_idx || !topk_w || !y || !W->gate_codes || !W->up_codes || !W->down_codes)
+    return REF_ERR_ARG;
+  if (mx ? (!W->gate_scales || !W->up_scales || !W->down_scales) : (!W->gate_d || !W->up_d || !W->down_dd))
     return REF_ERR_ARG;
   if (Is > 0 && (!W->sh_gate || !W->sh_up || !W->sh_down)) return REF_ERR_ARG;
 
@@ -306,9 +353,15 @@ int moeref_expert_ffn(const moeref_desc* desc, const moeref_weights* W, const vo
     for (int64_t a = 0; a < nA; ++a)
       if (topk_idx[a] == e) mine[na++] = a;
     if (!na) continue;
-    dequant_matrix_iq2(W->gate_codes, W->gate_d, e, I, H, wg);
-    dequant_matrix_iq2(W->up_codes, W->up_d, e, I, H, wu);
-    dequant_matrix_q2k(W->down_codes, W->down_dd, e, H, I, wd);
+    if (mx) {
+      dequant_matrix_mxfp4(W->gate_codes, W->gate_scales, e, I, H, wg);
+      dequant_matrix_mxfp4(W->up_codes, W->up_scales, e, I, H, wu);
+      dequant_matrix_mxfp4(W->down_codes, W->down_scales, e, H, I, wd);
+    } else {
+      dequant_matrix_iq2(W->gate_codes, W->gate_d, e, I, H, wg);
+      dequant_matrix_iq2(W->up_codes, W->up_d, e, I, H, wu);
+      dequant_matrix_q2k(W->down_codes, W->down_dd, e, H, I, wd);
+    }
     /* the assignments of expert e (and, with OpenMP, their rows) are
        independent; each dot product is the same sequential loop */
     double* hh = (double*)malloc(sizeof(double) * (size_t)na * I);

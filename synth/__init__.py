@@ -29,6 +29,8 @@ _lib = None
 T_ROUTER_W, T_ROUTER_B, T_GATE_CODES, T_GATE_D, T_UP_CODES, T_UP_D = 0, 1, 2, 3, 4, 5
 T_DOWN_CODES, T_DOWN_DD, T_SH_GATE, T_SH_UP, T_SH_DOWN, T_X, T_RESID = 6, 7, 8, 9, 10, 11, 12
 
+T_MX_GATE_CODES, T_MX_GATE_E, T_MX_UP_CODES, T_MX_UP_E, T_MX_DOWN_CODES, T_MX_DOWN_E = 13, 14, 15, 16, 17, 18
+
 IQ2_BLOCK_BYTES = 64  # code bytes per 256-weight block (plus one fp16 d)
 Q2K_BLOCK_BYTES = 80  # code bytes per 256-weight block (plus one u32 d|dmin)
 QK = 256
@@ -204,6 +206,78 @@ def make_layer(cfg: Config | dict, layer: int = 0, cfg_seed: int | None = None, 
     su = normal_bf16(seed(cs, layer, T_SH_UP), (Is, H), 1.0 / math.sqrt(H))
     sd = normal_bf16(seed(cs, layer, T_SH_DOWN), (H, Is), 1.0 / math.sqrt(max(Is, 1)))
     return LayerWeights(H, I, E, cfg.k, Is, rw, rb, gate_codes, gate_d, up_codes, up_d, down_codes, down_dd, sg, su, sd)
+
+
+@dataclass
+class MxLayerWeights:
+    """Host planes of one layer with MXFP4 routed experts (library layout).
+
+    gate/up: codes [E][I][H/2] u8 (two E2M1 elements per byte, low nibble first),
+             scales [E][I][H/32] u8 (E8M0)
+    down:    codes [E][H][I/2] u8, scales [E][H][I/32] u8
+    router and shared expert: as LayerWeights (the same streams as make_layer)
+    """
+
+    H: int
+    I: int
+    E: int
+    k: int
+    Is: int
+    router_w: np.ndarray
+    router_bias: np.ndarray | None
+    gate_codes: np.ndarray
+    gate_scales: np.ndarray
+    up_codes: np.ndarray
+    up_scales: np.ndarray
+    down_codes: np.ndarray
+    down_scales: np.ndarray
+    sh_gate: np.ndarray
+    sh_up: np.ndarray
+    sh_down: np.ndarray
+    fmt: str = "mxfp4"
+
+
+# mean square of the 16 E2M1 values (uniform codes): (0 + .25 + 1 + 2.25 + 4 + 9 + 16 + 36) / 8
+MX_ELEM_MS = 8.5625
+
+
+def mx_scale_exponent(K: int) -> int:
+    """E8M0 exponent that puts the weight RMS near 1/sqrt(K) for uniform codes."""
+    return 127 + int(round(math.log2(1.0 / (math.sqrt(MX_ELEM_MS) * math.sqrt(K)))))
+
+
+def mx_scales(s: int, shape, K: int) -> np.ndarray:
+    """E8M0 scale bytes: the exponent of mx_scale_exponent(K) plus a uniform jitter of -1, 0 or +1."""
+    return (mx_scale_exponent(K) - 1 + rand_bytes(s, shape) % 3).astype(np.uint8)
+
+
+def make_layer_mxfp4(cfg: Config | dict, layer: int = 0, cfg_seed: int | None = None, experts=None) -> MxLayerWeights:
+    """One layer with MXFP4 routed experts: uniform random code bytes, scales from
+    mx_scales; router and shared expert from the streams of make_layer."""
+    if isinstance(cfg, dict):
+        cfg = Config(**cfg)
+    cs = cfg.seed if cfg_seed is None else cfg_seed
+    H, I, E, Is = cfg.H, cfg.I, cfg.E, cfg.Is
+    assert H % 32 == 0 and I % 32 == 0
+    rw = normal_bf16(seed(cs, layer, T_ROUTER_W), (E, H), 1.28 / math.sqrt(H))
+    rb = zipf_bias(seed(cs, layer, T_ROUTER_B), E, 1.1) if cfg.zipf else None
+    gc = np.zeros((E, I, H // 2), np.uint8)
+    uc = np.zeros((E, I, H // 2), np.uint8)
+    dc = np.zeros((E, H, I // 2), np.uint8)
+    gs = np.zeros((E, I, H // 32), np.uint8)
+    us = np.zeros((E, I, H // 32), np.uint8)
+    ds = np.zeros((E, H, I // 32), np.uint8)
+    for e in range(E) if experts is None else sorted(set(int(v) for v in experts)):
+        lib().moegen_bytes(seed(cs, layer, T_MX_GATE_CODES, e), _p(gc[e]), gc[e].size)
+        lib().moegen_bytes(seed(cs, layer, T_MX_UP_CODES, e), _p(uc[e]), uc[e].size)
+        lib().moegen_bytes(seed(cs, layer, T_MX_DOWN_CODES, e), _p(dc[e]), dc[e].size)
+        gs[e] = mx_scales(seed(cs, layer, T_MX_GATE_E, e), gs[e].shape, H)
+        us[e] = mx_scales(seed(cs, layer, T_MX_UP_E, e), us[e].shape, H)
+        ds[e] = mx_scales(seed(cs, layer, T_MX_DOWN_E, e), ds[e].shape, I)
+    sg = normal_bf16(seed(cs, layer, T_SH_GATE), (Is, H), 1.0 / math.sqrt(H))
+    su = normal_bf16(seed(cs, layer, T_SH_UP), (Is, H), 1.0 / math.sqrt(H))
+    sd = normal_bf16(seed(cs, layer, T_SH_DOWN), (H, Is), 1.0 / math.sqrt(max(Is, 1)))
+    return MxLayerWeights(H, I, E, cfg.k, Is, rw, rb, gc, gs, uc, us, dc, ds, sg, su, sd)
 
 
 def make_token(cfg: Config, t: int, attempt: int = 0, layer: int = 0, cfg_seed: int | None = None) -> np.ndarray:
