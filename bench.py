@@ -545,6 +545,84 @@ def measure_cached(args, steps, n_slots=64):
     }
 
 
+def measure_mxfp4(args, steps):
+    """One-token decode with MXFP4 routed experts (moe_layer_forward_mxfp4), the
+    decode1 shapes (H=7168, I=2048, E=256, k=8, I_s=2048), 2 resident layers of
+    all 256 experts (12 GB) and 4 inputs in rotation (inputs larger than L2),
+    CUDA-graph replay; roofline of the gate/up GEMV over the bytes of the 8
+    active experts' gate and up planes (4.25 bits per weight)."""
+    import torch
+
+    from bit_quantized_routed_iq2_b200 import moe2bit
+
+    cfg = synth.Config("decode1_mxfp4", 1, 7168, 2048, 256, 8, 2048, "bf16", 1.0, False, 1, 0xD5400007)
+    layers = []
+    for l in range(2):
+        lw = synth.make_layer_mxfp4(cfg, layer=l)
+        layers.append(moe2bit.to_device_mxfp4(lw))
+        del lw
+    n_slots = 4
+    xs = [torch.from_numpy(synth.make_x_fast(cfg, 1, layer=100 + s).view(np.int16)).cuda().view(torch.bfloat16)
+          for s in range(n_slots)]
+    y = torch.empty((1, cfg.H), dtype=torch.float32, device="cuda")
+    ws = moe2bit.alloc_workspace_mxfp4(layers[0].desc, 1)
+    stream = torch.cuda.current_stream()
+
+    def step_on(i, st):
+        moe2bit.layer_forward_mxfp4(layers[i % 2], xs[i % n_slots], None, y, ws, st)
+
+    for i in range(max(args.warmup, 3)):
+        step_on(i, stream)
+    torch.cuda.synchronize()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    graphs = []
+    for j in range(n_slots):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            step_on(j, cap)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    for g in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        graphs[i % n_slots].replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    moe2bit.profile_enable(True)
+    for i in range(steps):
+        step_on(i, stream)
+    torch.cuda.synchronize()
+    prof = moe2bit.profile_read()
+    moe2bit.profile_enable(False)
+    assert moe2bit.read_status(ws) == 0
+    del graphs, layers, xs, ws
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    hbm, _, peak_kind = peaks()
+    avg_ms = {k: v[0] / max(v[1], 1) for k, v in prof.items()}
+    # gate + up codes and scales of the 8 active experts, plus the activations
+    alg = cfg.k * 2 * cfg.I * cfg.H * (0.5 + 1.0 / 32) + cfg.H * 2
+    achieved = alg / (avg_ms["gateup"] * 1e-3) / 1e9
+    dn_alg = cfg.k * cfg.H * cfg.I * (0.5 + 1.0 / 32)
+    return {
+        "value": 1.0 / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+        "config": {"workload": cfg.name, "tokens_per_step": 1, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
+                   "I_s": cfg.Is, "experts": "MXFP4 (OCP MX: E2M1 x 32 + E8M0), all three routed matrices",
+                   "resident_layers": 2, "l2": "inputs larger than L2: 2 resident layers of 6 GB",
+                   "launch": "cuda_graph"},
+        "kernels": {k: {"avg_ms": v, "launches_per_step": prof[k][1] / steps} for k, v in avg_ms.items()},
+        "roofline": {"bound": "hbm", "kernel": "gateup", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg,
+                     "avg_launch_ms": avg_ms["gateup"],
+                     "down_frac": dn_alg / (avg_ms["down"] * 1e-3) / 1e9 / hbm},
+    }
+
+
 def measure_quantize(args, reps=3):
     """Float -> 2-bit codes for one expert (gate and up to IQ2, down to Q2K,
     2048 x 7168 weights each): weights per second. The IQ2 search is bound by
@@ -624,14 +702,16 @@ def run_ours(args, cfg):
     if want == "auto":
         want = "all" if (world == 1 and not args.experts and not args.tokens) else "none"
     if want != "none":
-        names = ([n for n in ("decode32", "prefill", "stack") if n != cfg.name] + ["decode1_cached", "quantize"]
-                 if want == "all" else want.split(","))
+        names = ([n for n in ("decode32", "prefill", "stack") if n != cfg.name] +
+                 ["decode1_mxfp4", "decode1_cached", "quantize"] if want == "all" else want.split(","))
         line["workloads"] = {}
         for name in names:
             if name == "decode1_cached":
                 w = measure_cached(args, args.workload_steps * 10)
             elif name == "quantize":
                 w = measure_quantize(args)
+            elif name == "decode1_mxfp4":
+                w = measure_mxfp4(args, args.workload_steps)
             else:
                 w = measure(args, synth.CONFIGS[name], world, rank, local, args.workload_steps)
                 line["gpu_launches"] += w["gpu_launches"]

@@ -48,7 +48,8 @@ struct RouteWs {
   size_t bytes;
 };
 
-RouteWs carve(const moe_layer_desc* d, int32_t T, void* base) {
+// ffn_bytes: the FFN part of the workspace (default: that of the IQ2 / Q2K layer forward).
+RouteWs carve(const moe_layer_desc* d, int32_t T, void* base, size_t ffn_bytes = SIZE_MAX) {
   const size_t nA = static_cast<size_t>(T) * d->top_k, E = d->n_experts;
   char* p = static_cast<char*>(base);
   RouteWs w{};
@@ -66,7 +67,7 @@ RouteWs carve(const moe_layer_desc* d, int32_t T, void* base) {
   w.perm = reinterpret_cast<int32_t*>(take(nA * 4));
   w.inv = reinterpret_cast<int32_t*>(take(nA * 4));
   w.active = reinterpret_cast<int32_t*>(take((E + 1) * 4));
-  w.ffn = take(ffn_workspace_bytes(shape_of(d), T));
+  w.ffn = take(ffn_bytes == SIZE_MAX ? ffn_workspace_bytes(shape_of(d), T) : ffn_bytes);
   w.bytes = off;
   return w;
 }
@@ -523,6 +524,85 @@ moe_status moe_layer_forward_cached(moe_expert_cache* cache, const moe_layer_wei
                     early);
   if (rc != OK && early) join_shared_early(s);
   return to_status(rc);
+}
+
+
+// ------------------------------------------------------------ MXFP4 experts
+namespace {
+moe_status check_mx(const moe_layer_desc* desc, int32_t T) {
+  moe_status st = check_desc(desc);
+  if (st != MOE_OK) return st;
+  if ((st = check_tokens(desc, T)) != MOE_OK) return st;
+  if (T > 0 && !mx_path_supported(shape_of(desc), T)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+}  // namespace
+
+moe_status moe_workspace_size_mxfp4(const moe_layer_desc* desc, int32_t max_tokens, size_t* bytes) {
+  moe_status st = check_mx(desc, max_tokens);
+  if (st != MOE_OK) return st;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = carve(desc, max_tokens, nullptr, mx_ffn_workspace_bytes(shape_of(desc), max_tokens)).bytes;
+  return MOE_OK;
+}
+
+moe_status moe_layer_forward_mxfp4(const moe_layer_desc* desc, const moe_mxfp4_weights* weights, const void* x,
+                                   moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  moe_status st = check_mx(desc, T);
+  if (st != MOE_OK) return st;
+  if (x_dtype != MOE_F32 && x_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!weights) return MOE_ERR_INVALID_ARG;
+  const void* planes[] = {weights->router_w,  weights->gate_codes, weights->gate_scales, weights->up_codes,
+                          weights->up_scales, weights->down_codes, weights->down_scales};
+  for (const void* p : planes)
+    if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (weights->router_bias && !aligned16(weights->router_bias)) return MOE_ERR_INVALID_ARG;
+  if (desc->shared_inter > 0) {
+    const void* sh[] = {weights->sh_gate, weights->sh_up, weights->sh_down};
+    for (const void* p : sh)
+      if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  }
+  const void* req[] = {x, y, ws};
+  for (const void* p : req)
+    if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (residual && !aligned16(residual)) return MOE_ERR_INVALID_ARG;
+  const LayerShape sh = shape_of(desc);
+  RouteWs w = carve(desc, T, ws, mx_ffn_workspace_bytes(sh, T));
+  if (ws_bytes < w.bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  WeightPtrs shw{};  // router and shared expert (the routed fields are unused here)
+  shw.router_w = weights->router_w;
+  shw.router_bias = weights->router_bias;
+  shw.sh_gate = weights->sh_gate;
+  shw.sh_up = weights->sh_up;
+  shw.sh_down = weights->sh_down;
+  const MxPlanes mp{weights->gate_codes, weights->gate_scales, weights->up_codes,
+                    weights->up_scales,  weights->down_codes, weights->down_scales};
+  // as moe_layer_forward: the shared expert and the digits start first on the side stream (with this
+  // path's workspace layout); every return after the fork joins it back
+  const bool early = shared_early_ok(sh, x_dtype, T);
+  int rc = OK;
+  if (early) rc = launch_shared_early(sh, shw, x, T, w.ffn, s, mx_parts(sh.H), mx_parts(sh.I));
+  if (rc == OK)
+    rc = launch_route(weights->router_w, weights->router_bias, x, x_dtype, T, desc->hidden, desc->n_experts,
+                      desc->top_k, w.logits, w.topk_idx, w.topk_w, w.offsets, w.perm, w.inv, w.active, w.status, s,
+                      early);
+  if (rc == OK) {
+    Routing r{w.topk_w, w.offsets, w.perm, w.inv, w.active};
+    const bool routed_clears = x_dtype == MOE_BF16 && router_tc_supported(T, desc->hidden, desc->n_experts);
+    rc = launch_ffn_mxfp4(sh, shw, mp, x, x_dtype, T, r, residual, y, w.ffn, w.status, !routed_clears && !early, s,
+                          early);
+  }
+  if (rc != OK && early) join_shared_early(s);
+  return to_status(rc);
+}
+
+moe_status moe_debug_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t n_blocks, float* out,
+                                   void* stream) {
+  if (!codes || !scales || !out || n_blocks < 0) return MOE_ERR_INVALID_ARG;
+  return to_status(launch_mx_dequant(codes, scales, n_blocks, out, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

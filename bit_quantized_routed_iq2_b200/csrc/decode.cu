@@ -569,11 +569,15 @@ void join_shared_early(cudaStream_t st) {
   if (SideCtx* c = side_ctx(st)) cudaStreamWaitEvent(st, c->join, 0);
 }
 
-int launch_shared_early(const LayerShape& s, const WeightPtrs& w, const void* x, int T, void* ws, cudaStream_t st) {
+int launch_shared_early(const LayerShape& s, const WeightPtrs& w, const void* x, int T, void* ws, cudaStream_t st,
+                        int KP, int DP) {
   SideCtx* c = side_ctx(st);
   if (!c) return ERR_CUDA;
   const bool tma = tma_shape(s, T) && tma_path_supported(s, T);
-  const int KP = tma ? tma_gu_parts(s, T) : 1, DP = tma ? tma_dn_parts(s, T) : 1;
+  if (KP <= 0) {  // the layout of launch_ffn_fast
+    KP = tma ? tma_gu_parts(s, T) : 1;
+    DP = tma ? tma_dn_parts(s, T) : 1;
+  }
   const FastWs fw = carve_fast(s, T, KP, DP, static_cast<char*>(ws));
   if (cudaEventRecord(c->fork, st) != cudaSuccess || cudaStreamWaitEvent(c->st, c->fork, 0) != cudaSuccess)
     return ERR_CUDA;
@@ -733,6 +737,90 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
     const int grid = (s.H + 7) / 8;
     shared_down_combine_kernel<8><<<grid, 256, 0, st>>>(s.H, s.Is, s.k, s.Is > 0 ? w.sh_down : nullptr, hsh, T,
                                                         r.topk_w, r.inv, obuf, DP, residual, y);
+  }
+  if (rc != OK) return ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
+}
+
+
+// ------------------------------------------------------------ MXFP4 experts
+// The same step as launch_ffn_fast (digits, gate/up, h, down, shared expert,
+// combine) with the MXFP4 GEMVs of mxfp4.cu: gate/up and down in 256-element
+// parts of their reduction axes, h re-quantised as activation digits.
+size_t mx_ffn_workspace_bytes(const LayerShape& s, int T) {
+  return carve_fast(s, T, mx_parts(s.H), mx_parts(s.I), nullptr).bytes;
+}
+
+int launch_ffn_mxfp4(const LayerShape& s, const WeightPtrs& shw, const MxPlanes& w, const void* x, int x_dtype,
+                     int T, const Routing& r, const float* residual, float* y, void* ws, int* err, bool clear_status,
+                     cudaStream_t st, bool shared_early) {
+  const int nA = T * s.k;
+  const int KP = mx_parts(s.H), DP = mx_parts(s.I);
+  const FastWs fw = carve_fast(s, T, KP, DP, static_cast<char*>(ws));
+  const int sms = num_sms();
+  int rc = OK;
+  if (shared_early) {  // the digits come from the side stream (launch_shared_early with this layout)
+    SideCtx* c = side_ctx(st);
+    if (!c || cudaStreamWaitEvent(st, c->digits, 0) != cudaSuccess) return ERR_CUDA;
+  } else {
+    ProfScope ps(MOE_K_PREP, st);
+    dim3 g(T, (s.H / 256 + 7) / 8);
+    if (x_dtype == 0)
+      launch_pdl(x_digits_kernel<float>, g, dim3(256), 0, st, static_cast<const float*>(x), T, s.H, fw.xd, fw.xs,
+                 fw.xb, clear_status ? err : nullptr, 14);
+    else
+      launch_pdl(x_digits_kernel<uint16_t>, g, dim3(256), 0, st, static_cast<const uint16_t*>(x), T, s.H, fw.xd,
+                 fw.xs, static_cast<uint16_t*>(nullptr), clear_status ? err : nullptr, 14);
+  }
+  {
+    ProfScope ps(MOE_K_GATEUP, st);
+    rc |= launch_mx_gemv(true, s.H, s.I, s.E, s.k, T, w.gate_codes, w.gate_scales, w.up_codes, w.up_scales, fw.xd,
+                         fw.xs, r, fw.gu, err, sms, st);
+  }
+  {
+    ProfScope ps(MOE_K_HQUANT, st);
+    rc |= launch_mx_hquant(s.I, KP, nA, fw.gu, fw.hd, fw.hsc, st);
+  }
+  {
+    ProfScope ps(MOE_K_DOWN, st);
+    rc |= launch_mx_gemv(false, s.I, s.H, s.E, s.k, T, w.down_codes, w.down_scales, nullptr, nullptr, fw.hd, fw.hsc,
+                         r, fw.obuf, err, sms, st);
+  }
+  if (shared_early) {  // the shared output is ready in ysh once the side stream joins
+    SideCtx* c = side_ctx(st);
+    if (!c || cudaStreamWaitEvent(st, c->join, 0) != cudaSuccess) return ERR_CUDA;
+    ProfScope ps(MOE_K_COMBINE, st);
+    launch_pdl(combine_routed_kernel, dim3((s.H + 255) / 256, T), dim3(256), 0, st, s.H, s.k,
+               static_cast<const float*>(r.topk_w), static_cast<const int32_t*>(r.inv),
+               static_cast<const float*>(fw.obuf), DP, static_cast<const float*>(fw.ysh), residual, y);
+  } else {
+    // the shared expert here, then its down projection fused with the combine
+    const int xparts = x_dtype == 0 ? 2 : 1;
+    const uint16_t* xbp = x_dtype == 0 ? fw.xb : static_cast<const uint16_t*>(x);
+    if (s.Is > 0 && shared_mma_supported(s.H, s.Is, T, xparts, s.k)) {
+      {
+        ProfScope ps(MOE_K_SHARED_GATEUP, st);
+        rc |= launch_shared_gateup_mma(s.H, s.Is, shw.sh_gate, shw.sh_up, xbp, xparts, T, fw.hb, st);
+      }
+      ProfScope ps(MOE_K_COMBINE, st);
+      rc |= launch_shared_down_combine_mma(s.H, s.Is, shw.sh_down, fw.hb, T, s.k, r.topk_w, r.inv, fw.obuf, DP,
+                                           residual, y, st);
+    } else {
+      if (s.Is > 0) {
+        ProfScope ps(MOE_K_SHARED_GATEUP, st);
+        const int grid = (s.Is + 7) / 8;
+        if (x_dtype == 0)
+          shared_gateup_direct_kernel<float, 4><<<grid, 256, 0, st>>>(s.H, s.Is, shw.sh_gate, shw.sh_up,
+                                                                      static_cast<const float*>(x), T, fw.hsh);
+        else
+          shared_gateup_direct_kernel<uint16_t, 4><<<grid, 256, 0, st>>>(s.H, s.Is, shw.sh_gate, shw.sh_up,
+                                                                         static_cast<const uint16_t*>(x), T, fw.hsh);
+      }
+      ProfScope ps(MOE_K_COMBINE, st);
+      shared_down_combine_kernel<8><<<(s.H + 7) / 8, 256, 0, st>>>(s.H, s.Is, s.k, s.Is > 0 ? shw.sh_down : nullptr,
+                                                                   fw.hsh, T, r.topk_w, r.inv, fw.obuf, DP,
+                                                                   residual, y);
+    }
   }
   if (rc != OK) return ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;

@@ -68,6 +68,22 @@ int tma_dn_parts(const LayerShape& s, int T);
 int launch_gateup_tma(const LayerShape& sh, const uint8_t* gate_codes, const uint16_t* gate_d,
                       const uint8_t* up_codes, const uint16_t* up_d, const int8_t* xd, const float* xs, int T,
                       const Routing& r, float* gpart, int* err, int sms, cudaStream_t st);
+// MXFP4 routed experts (mxfp4.cu; the step in decode.cu).
+struct MxPlanes {
+  const uint8_t *gate_codes, *gate_scales, *up_codes, *up_scales, *down_codes, *down_scales;
+};
+size_t mx_ffn_workspace_bytes(const LayerShape& s, int T);
+int launch_ffn_mxfp4(const LayerShape& s, const WeightPtrs& shw, const MxPlanes& w, const void* x, int x_dtype,
+                     int T, const Routing& r, const float* residual, float* y, void* ws, int* err, bool clear_status,
+                     cudaStream_t st, bool shared_early);
+bool mx_path_supported(const LayerShape& s, int T);
+int mx_parts(int K);
+int launch_mx_gemv(bool pair, int K, int R, int E, int k, int T, const uint8_t* codes0, const uint8_t* sc0,
+                   const uint8_t* codes1, const uint8_t* sc1, const int8_t* ad, const float* as, const Routing& r,
+                   float* part, int* err, int sms, cudaStream_t st);
+int launch_mx_hquant(int I, int KP, int nA, const float* gu, int8_t* hd, float* hs, cudaStream_t st);
+int launch_mx_dequant(const uint8_t* codes, const uint8_t* scales, int64_t nb, float* out, cudaStream_t st);
+
 int launch_down_tma(const LayerShape& sh, const uint8_t* down_codes, const uint32_t* down_dd, const int8_t* hd,
                     const float* hsc, const int32_t* hq, int hss, int T, const Routing& r, float* opart, int* err,
                     int sms, cudaStream_t st);
@@ -79,7 +95,9 @@ bool shared_mma_supported(int H, int Is, int T, int x_parts, int k);
 // shared gate/up runs on a side stream forked from `st` before the router, and
 // the decode path's combine waits for it. Returns true when it was launched.
 bool shared_early_ok(const LayerShape& s, int x_dtype, int T);
-int launch_shared_early(const LayerShape& s, const WeightPtrs& w, const void* x, int T, void* ffn_ws, cudaStream_t st);
+// KP, DP: the part counts of the caller's workspace layout (<= 0: those of launch_ffn_fast).
+int launch_shared_early(const LayerShape& s, const WeightPtrs& w, const void* x, int T, void* ffn_ws, cudaStream_t st,
+                        int KP = -1, int DP = -1);
 // Joins the side stream back into `st` (the error path of a call that forked it).
 void join_shared_early(cudaStream_t st);
 int launch_shared_gateup_mma(int H, int Is, const uint16_t* wg, const uint16_t* wu, const uint16_t* xb, int P,

@@ -34,6 +34,7 @@ EXPORTS = (
     "moe_debug_tc_operands_q2k", "moe_quantize_q2k", "moe_quantize_iq2",
     "moe_prefetch_layer", "moe_debug_bounds_check_build", "moe_debug_bounds_violations",
     "moe_cache_bytes", "moe_cache_create", "moe_cache_destroy", "moe_cache_read_stats", "moe_layer_forward_cached",
+    "moe_workspace_size_mxfp4", "moe_layer_forward_mxfp4", "moe_debug_dequant_mxfp4",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 KERNEL_NAMES = ("router_logits", "topk", "permute", "active", "gateup", "down", "shared_gateup", "shared_down",
@@ -63,6 +64,14 @@ class Weights(ctypes.Structure):
     ]
 
 
+class MxWeights(ctypes.Structure):
+    """moe_mxfp4_weights: router, MXFP4 code and E8M0 scale planes, shared expert."""
+
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "router_w", "router_bias", "gate_codes", "gate_scales", "up_codes", "up_scales",
+        "down_codes", "down_scales", "sh_gate", "sh_up", "sh_down")]
+
+
 _lib = None
 
 
@@ -87,6 +96,9 @@ def load() -> ctypes.CDLL:
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_debug_dequant_iq2.argtypes = [vp, vp, i64, vp, vp]
     L.moe_debug_dequant_q2k.argtypes = [vp, vp, i64, vp, vp]
+    L.moe_workspace_size_mxfp4.argtypes = [pd, i32, ctypes.POINTER(sz)]
+    L.moe_layer_forward_mxfp4.argtypes = [pd, ctypes.POINTER(MxWeights), vp, i32, i32, vp, vp, vp, sz, vp]
+    L.moe_debug_dequant_mxfp4.argtypes = [vp, vp, i64, vp, vp]
     L.moe_debug_gemv_operands_iq2.argtypes = [vp, i64, vp, vp, vp]
     L.moe_debug_gemv_operands_q2k.argtypes = [vp, i64, vp, vp, vp]
     L.moe_debug_tc_operands_iq2.argtypes = [vp, vp, i64, vp, vp]
@@ -310,6 +322,70 @@ def layer_forward_noalloc(layer: DeviceLayer, x, residual, y, stream=None):
     w = layer.weights
     _check(load().moe_layer_forward_noalloc(ctypes.byref(layer.desc), ctypes.byref(w), _ptr(x), _dtype_of(x), T,
                                             _ptr(residual), _ptr(y), _stream(stream)), "moe_layer_forward_noalloc")
+
+
+@dataclass
+class MxDeviceLayer:
+    """Device planes of a layer with MXFP4 routed experts."""
+
+    desc: Desc
+    tensors: dict
+
+    @property
+    def weights(self) -> "MxWeights":
+        t = self.tensors
+        return MxWeights(*[_ptr(t.get(n)) for n in (
+            "router_w", "router_bias", "gate_codes", "gate_scales", "up_codes", "up_scales",
+            "down_codes", "down_scales", "sh_gate", "sh_up", "sh_down")])
+
+
+def to_device_mxfp4(lw, device="cuda") -> MxDeviceLayer:
+    """Upload the host planes of an MXFP4 layer (synth.MxLayerWeights layout)."""
+    import numpy as np
+    import torch
+
+    def up(a, dt):
+        if a is None:
+            return None
+        return torch.from_numpy(np.ascontiguousarray(a).view(dt)).to(device)
+
+    t = {
+        "router_w": up(lw.router_w, np.int16),
+        "router_bias": None if lw.router_bias is None else up(lw.router_bias, np.float32),
+        "gate_codes": up(lw.gate_codes, np.uint8), "gate_scales": up(lw.gate_scales, np.uint8),
+        "up_codes": up(lw.up_codes, np.uint8), "up_scales": up(lw.up_scales, np.uint8),
+        "down_codes": up(lw.down_codes, np.uint8), "down_scales": up(lw.down_scales, np.uint8),
+        "sh_gate": up(lw.sh_gate, np.int16) if lw.Is else None,
+        "sh_up": up(lw.sh_up, np.int16) if lw.Is else None,
+        "sh_down": up(lw.sh_down, np.int16) if lw.Is else None,
+    }
+    return MxDeviceLayer(desc_of(lw.H, lw.I, lw.E, lw.k, lw.Is), t)
+
+
+def workspace_size_mxfp4(desc: Desc, max_tokens: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().moe_workspace_size_mxfp4(ctypes.byref(desc), max_tokens, ctypes.byref(n)), "moe_workspace_size_mxfp4")
+    return int(n.value)
+
+
+def alloc_workspace_mxfp4(desc: Desc, max_tokens: int, device="cuda"):
+    import torch
+
+    return torch.empty(max(workspace_size_mxfp4(desc, max_tokens), 16), dtype=torch.uint8, device=device)
+
+
+def layer_forward_mxfp4(layer: MxDeviceLayer, x, residual, y, ws, stream=None):
+    T = x.shape[0]
+    w = layer.weights
+    _check(load().moe_layer_forward_mxfp4(ctypes.byref(layer.desc), ctypes.byref(w), _ptr(x), _dtype_of(x), T,
+                                          _ptr(residual), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
+                                          _stream(stream)), "moe_layer_forward_mxfp4")
+
+
+def debug_dequant_mxfp4(codes, scales, out, stream=None):
+    nb = codes.numel() // 16
+    _check(load().moe_debug_dequant_mxfp4(_ptr(codes), _ptr(scales), nb, _ptr(out), _stream(stream)),
+           "moe_debug_dequant_mxfp4")
 
 
 def read_status(ws, stream=None) -> int:

@@ -426,6 +426,77 @@ typedef enum {
 MOE_API moe_status moe_profile_enable(int32_t on);
 MOE_API moe_status moe_profile_read(float* total_ms, int32_t* launches);
 
+/*
+ * MXFP4 routed experts (second expert format).
+ *
+ * [Q] names an MXFP4 file that keeps the routed expert weights as published
+ * (no requantisation), running on CUDA with native FP4 matrix instructions on
+ * Blackwell for batched expert work. The pages give no bit layout; the element
+ * and scale encodings below are those of the OCP Microscaling Formats (MX) v1.0
+ * specification (MXFP4: blocks of 32 FP4 E2M1 elements sharing one E8M0 scale),
+ * and the packing into planes is this library's.
+ *
+ * All three routed matrices of a layer are MXFP4. A matrix [rows][K] (K = H for
+ * gate and up, K = I for down; K % 32 == 0) is two planes:
+ *   codes  [rows][K/2] bytes: element 2i of a row in bits 0..3 of byte i,
+ *          element 2i+1 in bits 4..7;
+ *   scales [rows][K/32] bytes: E8M0 exponent E of block b (elements 32b..32b+31).
+ * Element code c: sign = bit 3, magnitude m(c & 7) = 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+ * Weight: w = (-1)^sign * m * 2^(E - 127), exact in fp32 for E in [1, 254].
+ * E = 255 (the format's NaN) and E = 0 are outside what this library supports
+ * (the results for them are unspecified; nothing checks the scale bytes).
+ * The router and the shared expert are the bf16 ones of moe_layer_weights.
+ */
+typedef struct {
+  const uint16_t* router_w;     /* bf16 [E][H] */
+  const float* router_bias;     /* fp32 [E], or NULL */
+  const uint8_t* gate_codes;    /* [E][I][H/2] */
+  const uint8_t* gate_scales;   /* [E][I][H/32] */
+  const uint8_t* up_codes;      /* [E][I][H/2] */
+  const uint8_t* up_scales;     /* [E][I][H/32] */
+  const uint8_t* down_codes;    /* [E][H][I/2] */
+  const uint8_t* down_scales;   /* [E][H][I/32] */
+  const uint16_t* sh_gate;      /* bf16 [I_s][H] (unused when I_s == 0) */
+  const uint16_t* sh_up;        /* bf16 [I_s][H] */
+  const uint16_t* sh_down;      /* bf16 [H][I_s] */
+} moe_mxfp4_weights;
+
+/*
+ * moe_workspace_size_mxfp4: workspace bytes of moe_layer_forward_mxfp4 for any
+ * T <= max_tokens (host only); MOE_ERR_UNSUPPORTED_SHAPE for shapes the MXFP4
+ * path does not serve (see below).
+ *
+ * The layer forward of moe_layer_forward with MXFP4 routed experts: the same
+ * routing, shared expert, combine, residual and output, with the gate, up and
+ * down projections of each assignment taken over the decoded MXFP4 weights.
+ * Decode only: 1 <= T <= 16 tokens (T == 0 enqueues nothing). Shapes, in
+ * addition to those of the common conventions: hidden % 512 == 0,
+ * inter % 512 == 0, n_experts <= 1024; otherwise MOE_ERR_UNSUPPORTED_SHAPE.
+ * Every pointer of `w` (the shared-expert ones when I_s > 0) is a 16-byte
+ * aligned device pointer, else MOE_ERR_INVALID_ARG. Workspace: ws_bytes >=
+ * moe_workspace_size_mxfp4(desc, T) (its gate/up partial sums are finer than
+ * those of moe_layer_forward), else MOE_ERR_WORKSPACE_TOO_SMALL. Stream, side
+ * stream, status word (moe_read_status) and errors as moe_layer_forward.
+ * Numerics: activations enter the integer products as two signed digits of a
+ * 14-bit fixed-point code per 256-element block (as in moe_layer_forward's
+ * decode path), the decoded elements times 2 are exact int8 values, every block
+ * of 32 is scaled exactly by its power of two; accumulation in fp32 per block
+ * and across blocks.
+ */
+MOE_API moe_status moe_workspace_size_mxfp4(const moe_layer_desc* desc, int32_t max_tokens, size_t* bytes);
+MOE_API moe_status moe_layer_forward_mxfp4(const moe_layer_desc* desc, const moe_mxfp4_weights* w, const void* x,
+                                           moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws,
+                                           size_t ws_bytes, void* stream);
+
+/*
+ * Decode n_blocks consecutive MXFP4 blocks (codes: device [n_blocks][16] bytes,
+ * scales: device [n_blocks] E8M0 bytes) into out: device fp32 [n_blocks][32],
+ * with the GPU path's element decoding (2 * element as int8, times 2^(E - 128)).
+ * Stream-ordered; MOE_ERR_INVALID_ARG for null pointers or n_blocks < 0.
+ */
+MOE_API moe_status moe_debug_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t n_blocks, float* out,
+                                           void* stream);
+
 /* Host copy of the library's compiled-in 256 x 8 IQ2 codebook (row-major,
  * values in {8, 25, 43}). `out` is a host pointer to 2048 bytes. */
 MOE_API void moe_debug_grid(uint8_t* out);

@@ -1,0 +1,105 @@
+"""MXFP4 routed experts on the GPU (moe_layer_forward_mxfp4) against the oracle.
+
+Element decoding bit-for-bit (as values) through moe_debug_dequant_mxfp4; the
+layer within the normwise bound of the 2-bit path (FFN_TOL) at small shapes
+(one and several tokens, fp32 and bf16 activations, with and without a shared
+expert, uneven routing) and at the one-token decode shape (H=7168, I=2048,
+E=256, k=8, I_s=2048).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from bit_quantized_routed_iq2_b200 import moe2bit
+from helpers import FFN_TOL, normwise, screened_x
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch_cuda():
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    moe2bit.load()
+    return torch
+
+
+def _x_dev(torch, x):
+    t = torch.from_numpy(np.ascontiguousarray(x).view(np.int16) if x.dtype == np.uint16 else x).cuda()
+    return t.view(torch.bfloat16) if x.dtype == np.uint16 else t
+
+
+def test_dequant_matches_oracle(torch_cuda):
+    torch = torch_cuda
+    nb = 4096
+    codes = synth.rand_bytes(0x4D5801, (nb, 16))
+    scales = (1 + synth.rand_bytes(0x4D5802, (nb,)) % 254).astype(np.uint8)  # every E in [1, 254]
+    # every element code at least once per byte position
+    codes[:256] = np.arange(256, dtype=np.uint8)[:, None]
+    out = torch.empty(nb * 32, dtype=torch.float32, device="cuda")
+    moe2bit.debug_dequant_mxfp4(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(), out)
+    torch.cuda.synchronize()
+    ref = oracle.dequant_mxfp4(codes, scales)
+    # equal as values (the GPU's integer operands give +0 where the format's code 8 means -0)
+    assert np.array_equal(out.cpu().numpy(), ref)
+
+
+def _mx_forward(torch, dl, x, residual=None):
+    T = x.shape[0]
+    y = torch.full((T, dl.desc.hidden), float("nan"), dtype=torch.float32, device="cuda")
+    res = None if residual is None else torch.from_numpy(np.ascontiguousarray(residual)).cuda()
+    ws = moe2bit.alloc_workspace_mxfp4(dl.desc, T)
+    moe2bit.layer_forward_mxfp4(dl, _x_dev(torch, x), res, y, ws)
+    torch.cuda.synchronize()
+    assert moe2bit.read_status(ws) == 0
+    return y.cpu().numpy()
+
+
+CASES = {
+    "t1_bf16": dict(T=1, x_dtype="bf16", Is=128, zipf=False),
+    "t2_f32_noshared": dict(T=2, x_dtype="f32", Is=0, zipf=False),
+    "t5_bf16_zipf": dict(T=5, x_dtype="bf16", Is=128, zipf=True),
+    "t16_bf16_zipf": dict(T=16, x_dtype="bf16", Is=128, zipf=True),
+    "t16_f32": dict(T=16, x_dtype="f32", Is=64, zipf=False),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_mxfp4_layer_small(torch_cuda, name):
+    c = CASES[name]
+    cfg = synth.Config("mx_" + name, c["T"], 1024, 512, 16, 4, c["Is"], c["x_dtype"], 1.0, c["zipf"], 1,
+                       0x4D58A0 + len(name))
+    lw = synth.make_layer_mxfp4(cfg)
+    x = screened_x(cfg, lw)
+    res = synth.make_residual(cfg, cfg.T)
+    y = _mx_forward(torch_cuda, moe2bit.to_device_mxfp4(lw), x, res)
+    ref, _, _ = oracle.layer_forward(lw, x, res)
+    assert normwise(y, ref) <= FFN_TOL, (name, normwise(y, ref))
+
+
+def test_mxfp4_rejects_unsupported_shapes(torch_cuda):
+    desc = moe2bit.desc_of(1280, 512, 16, 4, 0)  # hidden not a multiple of 512
+    with pytest.raises(RuntimeError):
+        moe2bit.workspace_size_mxfp4(desc, 1)
+    desc = moe2bit.desc_of(1024, 512, 16, 4, 0)
+    with pytest.raises(RuntimeError):
+        moe2bit.workspace_size_mxfp4(desc, 17)  # decode only
+    assert moe2bit.workspace_size_mxfp4(desc, 16) > 0
+
+
+@pytest.mark.slow
+def test_mxfp4_decode1_shape(torch_cuda):
+    """H=7168, I=2048, E=256, k=8, I_s=2048, one bf16 token: the routed experts'
+    planes are generated (the others stay zero and are never read)."""
+    cfg = synth.CONFIGS["decode1"]
+    base = synth.make_layer(cfg, experts=[])
+    x = screened_x(cfg, base)
+    idx, _ = oracle.route(base.router_w, base.router_bias, x, cfg.k)
+    lw = synth.make_layer_mxfp4(cfg, experts=np.unique(idx))
+    y = _mx_forward(torch_cuda, moe2bit.to_device_mxfp4(lw), x)
+    ref, ridx, _ = oracle.layer_forward(lw, x)
+    assert np.array_equal(np.sort(ridx, axis=1), np.sort(idx, axis=1))
+    assert normwise(y, ref) <= FFN_TOL, normwise(y, ref)
