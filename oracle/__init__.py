@@ -38,7 +38,7 @@ class Weights(ctypes.Structure):
     ]
 
 
-FMT_IQ2_Q2K, FMT_MXFP4 = 0, 1
+FMT_IQ2_Q2K, FMT_MXFP4, FMT_Q4 = 0, 1, 2
 
 
 def build(force: bool = False, openmp: bool | None = None) -> str:
@@ -94,6 +94,7 @@ def lib():
         L.moeref_e2m1.restype = ctypes.c_double
         L.moeref_e2m1.argtypes = [ctypes.c_uint]
         L.moeref_dequant_mxfp4.argtypes = [vp, vp, i64, vp]
+        L.moeref_dequant_q4.argtypes = [vp, vp, i64, vp]
         L.moeref_route.argtypes = [i32, i32, i32, vp, vp, vp, i32, i32, vp, vp, vp]
         L.moeref_permute.argtypes = [i32, i32, i32, vp, vp, vp, vp]
         L.moeref_f32_to_f16.restype = ctypes.c_uint16
@@ -174,6 +175,16 @@ def dequant_mxfp4(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     return out
 
 
+def dequant_q4(codes: np.ndarray, d: np.ndarray) -> np.ndarray:
+    """Q4-style blocks (codes [nb][16] u8, fp16 d [nb]) -> fp32 [nb * 32]."""
+    codes = np.ascontiguousarray(codes, np.uint8).reshape(-1, 16)
+    d = np.ascontiguousarray(d, np.uint16).reshape(-1)
+    assert codes.shape[0] == d.shape[0]
+    out = np.zeros(codes.shape[0] * 32, np.float32)
+    lib().moeref_dequant_q4(_p(codes), _p(d), codes.shape[0], _p(out))
+    return out
+
+
 def f32_to_f16(v: float) -> int:
     return int(lib().moeref_f32_to_f16(float(v)))
 
@@ -228,13 +239,14 @@ def _structs(lw):
     """Oracle structs of a layer; a layer with ``fmt == "mxfp4"`` carries MXFP4
     code planes and E8M0 scale planes instead of the IQ2 / Q2K planes."""
     desc = Desc(lw.H, lw.I, lw.E, lw.k, lw.Is)
-    mx = getattr(lw, "fmt", "iq2") == "mxfp4"
+    fmt = getattr(lw, "fmt", "iq2")
+    mx = fmt in ("mxfp4", "q4")
     arrs = (lw.router_w, lw.router_bias, lw.gate_codes, None if mx else lw.gate_d, lw.up_codes,
             None if mx else lw.up_d, lw.down_codes, None if mx else lw.down_dd, lw.sh_gate, lw.sh_up, lw.sh_down)
     keep = [np.ascontiguousarray(a) if a is not None else None for a in arrs]
     sc = [np.ascontiguousarray(getattr(lw, n)) for n in ("gate_scales", "up_scales", "down_scales")] if mx else []
     keep += sc
-    W = Weights(*[_p(a) for a in keep[:11]], FMT_MXFP4 if mx else FMT_IQ2_Q2K,
+    W = Weights(*[_p(a) for a in keep[:11]], {"mxfp4": FMT_MXFP4, "q4": FMT_Q4}.get(fmt, FMT_IQ2_Q2K),
                 *([_p(a) for a in sc] if mx else [None, None, None]))
     return desc, W, keep
 

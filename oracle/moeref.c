@@ -63,7 +63,8 @@ typedef struct {
   const uint8_t* down_scales;
 } moeref_weights;
 
-enum { REF_FMT_IQ2_Q2K = 0, REF_FMT_MXFP4 = 1 };
+enum { REF_FMT_IQ2_Q2K = 0, REF_FMT_MXFP4 = 1, REF_FMT_Q4 = 2 };
+/* With REF_FMT_Q4 the three scale pointers hold fp16 d per block, [rows][K/32] uint16. */
 
 /* ---------------------------------------------------------------- scalars */
 
@@ -222,6 +223,32 @@ static void dequant_matrix_mxfp4(const uint8_t* codes, const uint8_t* scales, in
   moeref_dequant_mxfp4(codes + (int64_t)e * nb * 16, scales + (int64_t)e * nb, nb, out);
 }
 
+/* -------------------------------------------------------------------- Q4
+ * The 4-bit routed-expert variant the pages mention ("Un modèle de 284
+ * milliards ...", « Comment un 284B tient »: Q4 models; "antirez/ds4 ...":
+ * checkpoints shared between the 2-bit and 4-bit routed-expert variants) has
+ * no published layout. This project's Q4-style block: 32 weights along the
+ * reduction axis, one fp16 scale d and 32 unsigned 4-bit codes q (element 2i
+ * in the low nibble of code byte i, 2i+1 in the high nibble):
+ * w = d * (q - 8), exact in fp32.
+ * Parity: pinned by a hand-decoded block, the affine law in q and the scaling
+ * law in d, and a dense float64 MoE over the decoded weights. */
+void moeref_dequant_q4(const uint8_t* codes, const uint16_t* d, int64_t nblocks, float* out) {
+  for (int64_t b = 0; b < nblocks; ++b) {
+    const double s = moeref_f16_to_f64(d[b]);
+    for (int i = 0; i < 32; ++i) {
+      const unsigned byte = codes[b * 16 + i / 2];
+      const int q = (int)((i & 1) ? (byte >> 4) : (byte & 15u));
+      out[b * 32 + i] = (float)(s * (double)(q - 8));
+    }
+  }
+}
+
+static void dequant_matrix_q4(const uint8_t* codes, const uint16_t* d, int e, int rows, int K, float* out) {
+  const int64_t nb = (int64_t)rows * K / 32;
+  moeref_dequant_q4(codes + (int64_t)e * nb * 16, d + (int64_t)e * nb, nb, out);
+}
+
 static void dequant_matrix_iq2(const uint8_t* codes, const uint16_t* d, int e, int rows, int K, float* out) {
   int64_t nb = (int64_t)rows * K / QK;
   moeref_dequant_iq2(codes + (int64_t)e * nb * IQ2_BYTES, d + (int64_t)e * nb, nb, out);
@@ -329,7 +356,8 @@ int moeref_expert_ffn(const moeref_desc* desc, const moeref_weights* W, const vo
   if (!desc || !W || T < 0) return REF_ERR_ARG;
   const int H = desc->hidden, I = desc->inter, E = desc->n_experts, k = desc->top_k, Is = desc->shared_inter;
   if (H <= 0 || I <= 0 || E <= 0 || k <= 0 || k > E || Is < 0) return REF_ERR_ARG;
-  const int mx = W->expert_format == REF_FMT_MXFP4;
+  const int q4 = W->expert_format == REF_FMT_Q4;
+  const int mx = W->expert_format == REF_FMT_MXFP4 || q4; /* block-32 formats with scale planes */
   if (W->expert_format != REF_FMT_IQ2_Q2K && !mx) return REF_ERR_ARG;
   if (((int64_t)H * I) % QK || (mx && (H % 32 || I % 32))) return REF_ERR_SHAPE;
   if (T == 0) return REF_OK;
@@ -353,7 +381,11 @@ int moeref_expert_ffn(const moeref_desc* desc, const moeref_weights* W, const vo
     for (int64_t a = 0; a < nA; ++a)
       if (topk_idx[a] == e) mine[na++] = a;
     if (!na) continue;
-    if (mx) {
+    if (q4) {
+      dequant_matrix_q4(W->gate_codes, (const uint16_t*)W->gate_scales, e, I, H, wg);
+      dequant_matrix_q4(W->up_codes, (const uint16_t*)W->up_scales, e, I, H, wu);
+      dequant_matrix_q4(W->down_codes, (const uint16_t*)W->down_scales, e, H, I, wd);
+    } else if (mx) {
       dequant_matrix_mxfp4(W->gate_codes, W->gate_scales, e, I, H, wg);
       dequant_matrix_mxfp4(W->up_codes, W->up_scales, e, I, H, wu);
       dequant_matrix_mxfp4(W->down_codes, W->down_scales, e, H, I, wd);

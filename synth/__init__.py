@@ -280,6 +280,70 @@ def make_layer_mxfp4(cfg: Config | dict, layer: int = 0, cfg_seed: int | None = 
     return MxLayerWeights(H, I, E, cfg.k, Is, rw, rb, gc, gs, uc, us, dc, ds, sg, su, sd)
 
 
+T_Q4_GATE_CODES, T_Q4_GATE_D, T_Q4_UP_CODES, T_Q4_UP_D, T_Q4_DOWN_CODES, T_Q4_DOWN_D = 19, 20, 21, 22, 23, 24
+# mean square of q - 8 for uniform 4-bit codes: (sum of (q-8)^2, q = 0..15) / 16
+Q4_ELEM_MS = 21.5
+
+
+@dataclass
+class Q4LayerWeights:
+    """Host planes of one layer with Q4-style routed experts (library layout).
+
+    gate/up: codes [E][I][H/2] u8 (two 4-bit codes per byte, low nibble first), d [E][I][H/32] fp16 bits
+    down:    codes [E][H][I/2] u8, d [E][H][I/32] fp16 bits
+    router and shared expert: as LayerWeights (the same streams as make_layer)
+    """
+
+    H: int
+    I: int
+    E: int
+    k: int
+    Is: int
+    router_w: np.ndarray
+    router_bias: np.ndarray | None
+    gate_codes: np.ndarray
+    gate_scales: np.ndarray
+    up_codes: np.ndarray
+    up_scales: np.ndarray
+    down_codes: np.ndarray
+    down_scales: np.ndarray
+    sh_gate: np.ndarray
+    sh_up: np.ndarray
+    sh_down: np.ndarray
+    fmt: str = "q4"
+
+
+def make_layer_q4(cfg: Config | dict, layer: int = 0, cfg_seed: int | None = None, experts=None) -> Q4LayerWeights:
+    """One layer with Q4-style routed experts: uniform random code bytes, fp16 scales from the
+    f16_scale recipe with base 1 / (sqrt(Q4_ELEM_MS) sqrt(K)); router and shared expert from the
+    streams of make_layer."""
+    if isinstance(cfg, dict):
+        cfg = Config(**cfg)
+    cs = cfg.seed if cfg_seed is None else cfg_seed
+    H, I, E, Is = cfg.H, cfg.I, cfg.E, cfg.Is
+    assert H % 32 == 0 and I % 32 == 0
+    rw = normal_bf16(seed(cs, layer, T_ROUTER_W), (E, H), 1.28 / math.sqrt(H))
+    rb = zipf_bias(seed(cs, layer, T_ROUTER_B), E, 1.1) if cfg.zipf else None
+    gc = np.zeros((E, I, H // 2), np.uint8)
+    uc = np.zeros((E, I, H // 2), np.uint8)
+    dc = np.zeros((E, H, I // 2), np.uint8)
+    gd = np.zeros((E, I, H // 32), np.uint16)
+    ud = np.zeros((E, I, H // 32), np.uint16)
+    dd = np.zeros((E, H, I // 32), np.uint16)
+    bh, bi = 1.0 / math.sqrt(Q4_ELEM_MS * H), 1.0 / math.sqrt(Q4_ELEM_MS * I)
+    for e in range(E) if experts is None else sorted(set(int(v) for v in experts)):
+        lib().moegen_bytes(seed(cs, layer, T_Q4_GATE_CODES, e), _p(gc[e]), gc[e].size)
+        lib().moegen_bytes(seed(cs, layer, T_Q4_UP_CODES, e), _p(uc[e]), uc[e].size)
+        lib().moegen_bytes(seed(cs, layer, T_Q4_DOWN_CODES, e), _p(dc[e]), dc[e].size)
+        lib().moegen_f16_scale(seed(cs, layer, T_Q4_GATE_D, e), _p(gd[e]), gd[e].size, bh)
+        lib().moegen_f16_scale(seed(cs, layer, T_Q4_UP_D, e), _p(ud[e]), ud[e].size, bh)
+        lib().moegen_f16_scale(seed(cs, layer, T_Q4_DOWN_D, e), _p(dd[e]), dd[e].size, bi)
+    sg = normal_bf16(seed(cs, layer, T_SH_GATE), (Is, H), 1.0 / math.sqrt(H))
+    su = normal_bf16(seed(cs, layer, T_SH_UP), (Is, H), 1.0 / math.sqrt(H))
+    sd = normal_bf16(seed(cs, layer, T_SH_DOWN), (H, Is), 1.0 / math.sqrt(max(Is, 1)))
+    return Q4LayerWeights(H, I, E, cfg.k, Is, rw, rb, gc, gd, uc, ud, dc, dd, sg, su, sd)
+
+
 def make_token(cfg: Config, t: int, attempt: int = 0, layer: int = 0, cfg_seed: int | None = None) -> np.ndarray:
     """One token's activations (H,), fp32 or bf16 bits; ``attempt`` selects the
     redraw stream used when a token is rejected for a near-tie in the router."""
