@@ -545,31 +545,38 @@ def measure_cached(args, steps, n_slots=64):
     }
 
 
-def measure_mxfp4(args, steps):
-    """One-token decode with MXFP4 routed experts (moe_layer_forward_mxfp4), the
-    decode1 shapes (H=7168, I=2048, E=256, k=8, I_s=2048), 2 resident layers of
-    all 256 experts (12 GB) and 4 inputs in rotation (inputs larger than L2),
+def measure_mxfp4(args, steps, fmt="mxfp4"):
+    """One-token decode with block-32 routed experts: MXFP4 (moe_layer_forward_mxfp4,
+    4.25 bits per weight) or Q4-style (moe_layer_forward_q4, 4.5 bits per weight);
+    the decode1 shapes (H=7168, I=2048, E=256, k=8, I_s=2048), 2 resident layers
+    of all 256 experts and 4 inputs in rotation (inputs larger than L2),
     CUDA-graph replay; roofline of the gate/up GEMV over the bytes of the 8
-    active experts' gate and up planes (4.25 bits per weight)."""
+    active experts' gate and up planes."""
     import torch
 
     from bit_quantized_routed_iq2_b200 import moe2bit
 
-    cfg = synth.Config("decode1_mxfp4", 1, 7168, 2048, 256, 8, 2048, "bf16", 1.0, False, 1, 0xD5400007)
+    q4 = fmt == "q4"
+    cfg = synth.Config("decode1_" + fmt, 1, 7168, 2048, 256, 8, 2048, "bf16", 1.0, False, 1,
+                       0xD5400008 if q4 else 0xD5400007)
+    make = synth.make_layer_q4 if q4 else synth.make_layer_mxfp4
+    upload = moe2bit.to_device_q4 if q4 else moe2bit.to_device_mxfp4
+    forward = moe2bit.layer_forward_q4 if q4 else moe2bit.layer_forward_mxfp4
+    scale_bytes = 2.0 if q4 else 1.0  # per 32-weight block
     layers = []
     for l in range(2):
-        lw = synth.make_layer_mxfp4(cfg, layer=l)
-        layers.append(moe2bit.to_device_mxfp4(lw))
+        lw = make(cfg, layer=l)
+        layers.append(upload(lw))
         del lw
     n_slots = 4
     xs = [torch.from_numpy(synth.make_x_fast(cfg, 1, layer=100 + s).view(np.int16)).cuda().view(torch.bfloat16)
           for s in range(n_slots)]
     y = torch.empty((1, cfg.H), dtype=torch.float32, device="cuda")
-    ws = moe2bit.alloc_workspace_mxfp4(layers[0].desc, 1)
+    ws = moe2bit.alloc_workspace_mxfp4(layers[0].desc, 1)  # moe_workspace_size_q4 is the same size
     stream = torch.cuda.current_stream()
 
     def step_on(i, st):
-        moe2bit.layer_forward_mxfp4(layers[i % 2], xs[i % n_slots], None, y, ws, st)
+        forward(layers[i % 2], xs[i % n_slots], None, y, ws, st)
 
     for i in range(max(args.warmup, 3)):
         step_on(i, stream)
@@ -606,13 +613,14 @@ def measure_mxfp4(args, steps):
     hbm, _, peak_kind = peaks()
     avg_ms = {k: v[0] / max(v[1], 1) for k, v in prof.items()}
     # gate + up codes and scales of the 8 active experts, plus the activations
-    alg = cfg.k * 2 * cfg.I * cfg.H * (0.5 + 1.0 / 32) + cfg.H * 2
+    alg = cfg.k * 2 * cfg.I * cfg.H * (0.5 + scale_bytes / 32) + cfg.H * 2
     achieved = alg / (avg_ms["gateup"] * 1e-3) / 1e9
-    dn_alg = cfg.k * cfg.H * cfg.I * (0.5 + 1.0 / 32)
+    dn_alg = cfg.k * cfg.H * cfg.I * (0.5 + scale_bytes / 32)
     return {
         "value": 1.0 / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
         "config": {"workload": cfg.name, "tokens_per_step": 1, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
-                   "I_s": cfg.Is, "experts": "MXFP4 (OCP MX: E2M1 x 32 + E8M0), all three routed matrices",
+                   "I_s": cfg.Is, "experts": ("Q4-style (32 x 4-bit codes + fp16 d, w = d (q - 8))" if q4 else
+                                              "MXFP4 (OCP MX: E2M1 x 32 + E8M0)") + ", all three routed matrices",
                    "resident_layers": 2, "l2": "inputs larger than L2: 2 resident layers of 6 GB",
                    "launch": "cuda_graph"},
         "kernels": {k: {"avg_ms": v, "launches_per_step": prof[k][1] / steps} for k, v in avg_ms.items()},
@@ -703,15 +711,15 @@ def run_ours(args, cfg):
         want = "all" if (world == 1 and not args.experts and not args.tokens) else "none"
     if want != "none":
         names = ([n for n in ("decode32", "prefill", "stack") if n != cfg.name] +
-                 ["decode1_mxfp4", "decode1_cached", "quantize"] if want == "all" else want.split(","))
+                 ["decode1_mxfp4", "decode1_q4", "decode1_cached", "quantize"] if want == "all" else want.split(","))
         line["workloads"] = {}
         for name in names:
             if name == "decode1_cached":
                 w = measure_cached(args, args.workload_steps * 10)
             elif name == "quantize":
                 w = measure_quantize(args)
-            elif name == "decode1_mxfp4":
-                w = measure_mxfp4(args, args.workload_steps)
+            elif name in ("decode1_mxfp4", "decode1_q4"):
+                w = measure_mxfp4(args, args.workload_steps, name.split("_")[1])
             else:
                 w = measure(args, synth.CONFIGS[name], world, rank, local, args.workload_steps)
                 line["gpu_launches"] += w["gpu_launches"]

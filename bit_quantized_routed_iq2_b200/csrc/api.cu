@@ -546,21 +546,23 @@ moe_status moe_workspace_size_mxfp4(const moe_layer_desc* desc, int32_t max_toke
   return MOE_OK;
 }
 
-moe_status moe_layer_forward_mxfp4(const moe_layer_desc* desc, const moe_mxfp4_weights* weights, const void* x,
-                                   moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws,
-                                   size_t ws_bytes, void* stream) {
+namespace {
+// The layer forward over block-32 routed experts (MXFP4 or Q4-style): `planes` holds the three code planes
+// and the three scale planes (their element type per `mp.fmt`), `shw` the router and the shared expert.
+moe_status blk32_forward(const moe_layer_desc* desc, const WeightPtrs& shw, const MxPlanes& mp, const void* x,
+                         moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws, size_t ws_bytes,
+                         void* stream) {
   moe_status st = check_mx(desc, T);
   if (st != MOE_OK) return st;
   if (x_dtype != MOE_F32 && x_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
-  if (!weights) return MOE_ERR_INVALID_ARG;
-  const void* planes[] = {weights->router_w,  weights->gate_codes, weights->gate_scales, weights->up_codes,
-                          weights->up_scales, weights->down_codes, weights->down_scales};
+  const void* planes[] = {shw.router_w, mp.gate_codes, mp.gate_scales, mp.up_codes,
+                          mp.up_scales, mp.down_codes, mp.down_scales};
   for (const void* p : planes)
     if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
-  if (weights->router_bias && !aligned16(weights->router_bias)) return MOE_ERR_INVALID_ARG;
+  if (shw.router_bias && !aligned16(shw.router_bias)) return MOE_ERR_INVALID_ARG;
   if (desc->shared_inter > 0) {
-    const void* sh[] = {weights->sh_gate, weights->sh_up, weights->sh_down};
+    const void* sh[] = {shw.sh_gate, shw.sh_up, shw.sh_down};
     for (const void* p : sh)
       if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
   }
@@ -572,23 +574,14 @@ moe_status moe_layer_forward_mxfp4(const moe_layer_desc* desc, const moe_mxfp4_w
   RouteWs w = carve(desc, T, ws, mx_ffn_workspace_bytes(sh, T));
   if (ws_bytes < w.bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  WeightPtrs shw{};  // router and shared expert (the routed fields are unused here)
-  shw.router_w = weights->router_w;
-  shw.router_bias = weights->router_bias;
-  shw.sh_gate = weights->sh_gate;
-  shw.sh_up = weights->sh_up;
-  shw.sh_down = weights->sh_down;
-  const MxPlanes mp{weights->gate_codes, weights->gate_scales, weights->up_codes,
-                    weights->up_scales,  weights->down_codes, weights->down_scales};
   // as moe_layer_forward: the shared expert and the digits start first on the side stream (with this
   // path's workspace layout); every return after the fork joins it back
   const bool early = shared_early_ok(sh, x_dtype, T);
   int rc = OK;
   if (early) rc = launch_shared_early(sh, shw, x, T, w.ffn, s, mx_parts(sh.H), mx_parts(sh.I));
   if (rc == OK)
-    rc = launch_route(weights->router_w, weights->router_bias, x, x_dtype, T, desc->hidden, desc->n_experts,
-                      desc->top_k, w.logits, w.topk_idx, w.topk_w, w.offsets, w.perm, w.inv, w.active, w.status, s,
-                      early);
+    rc = launch_route(shw.router_w, shw.router_bias, x, x_dtype, T, desc->hidden, desc->n_experts, desc->top_k,
+                      w.logits, w.topk_idx, w.topk_w, w.offsets, w.perm, w.inv, w.active, w.status, s, early);
   if (rc == OK) {
     Routing r{w.topk_w, w.offsets, w.perm, w.inv, w.active};
     const bool routed_clears = x_dtype == MOE_BF16 && router_tc_supported(T, desc->hidden, desc->n_experts);
@@ -599,10 +592,56 @@ moe_status moe_layer_forward_mxfp4(const moe_layer_desc* desc, const moe_mxfp4_w
   return to_status(rc);
 }
 
+WeightPtrs blk32_shared(const uint16_t* router_w, const float* router_bias, const uint16_t* sh_gate,
+                        const uint16_t* sh_up, const uint16_t* sh_down) {
+  WeightPtrs shw{};  // router and shared expert (the routed fields are unused on this path)
+  shw.router_w = router_w;
+  shw.router_bias = router_bias;
+  shw.sh_gate = sh_gate;
+  shw.sh_up = sh_up;
+  shw.sh_down = sh_down;
+  return shw;
+}
+}  // namespace
+
+moe_status moe_layer_forward_mxfp4(const moe_layer_desc* desc, const moe_mxfp4_weights* weights, const void* x,
+                                   moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  if (!weights) return T == 0 && check_mx(desc, T) == MOE_OK ? MOE_OK : MOE_ERR_INVALID_ARG;
+  const MxPlanes mp{0, weights->gate_codes, weights->gate_scales, weights->up_codes,
+                    weights->up_scales, weights->down_codes, weights->down_scales};
+  return blk32_forward(desc,
+                       blk32_shared(weights->router_w, weights->router_bias, weights->sh_gate, weights->sh_up,
+                                    weights->sh_down),
+                       mp, x, x_dtype, T, residual, y, ws, ws_bytes, stream);
+}
+
+moe_status moe_workspace_size_q4(const moe_layer_desc* desc, int32_t max_tokens, size_t* bytes) {
+  return moe_workspace_size_mxfp4(desc, max_tokens, bytes);
+}
+
+moe_status moe_layer_forward_q4(const moe_layer_desc* desc, const moe_q4_weights* weights, const void* x,
+                                moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws,
+                                size_t ws_bytes, void* stream) {
+  if (!weights) return T == 0 && check_mx(desc, T) == MOE_OK ? MOE_OK : MOE_ERR_INVALID_ARG;
+  const MxPlanes mp{1, weights->gate_codes, weights->gate_d, weights->up_codes,
+                    weights->up_d, weights->down_codes, weights->down_d};
+  return blk32_forward(desc,
+                       blk32_shared(weights->router_w, weights->router_bias, weights->sh_gate, weights->sh_up,
+                                    weights->sh_down),
+                       mp, x, x_dtype, T, residual, y, ws, ws_bytes, stream);
+}
+
+moe_status moe_debug_dequant_q4(const uint8_t* codes, const uint16_t* d, int64_t n_blocks, float* out,
+                                void* stream) {
+  if (!codes || !d || !out || n_blocks < 0) return MOE_ERR_INVALID_ARG;
+  return to_status(launch_mx_dequant(1, codes, d, n_blocks, out, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_debug_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t n_blocks, float* out,
                                    void* stream) {
   if (!codes || !scales || !out || n_blocks < 0) return MOE_ERR_INVALID_ARG;
-  return to_status(launch_mx_dequant(codes, scales, n_blocks, out, static_cast<cudaStream_t>(stream)));
+  return to_status(launch_mx_dequant(0, codes, scales, n_blocks, out, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -743,10 +743,11 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
 }
 
 
-// ------------------------------------------------------------ MXFP4 experts
+// ------------------------------------------------------------ block-32 experts
 // The same step as launch_ffn_fast (digits, gate/up, h, down, shared expert,
-// combine) with the MXFP4 GEMVs of mxfp4.cu: gate/up and down in 256-element
-// parts of their reduction axes, h re-quantised as activation digits.
+// combine) with the block-32 GEMVs of mxfp4.cu (MXFP4 or Q4-style): gate/up and
+// down in 256-element parts of their reduction axes, h re-quantised as
+// activation digits.
 size_t mx_ffn_workspace_bytes(const LayerShape& s, int T) {
   return carve_fast(s, T, mx_parts(s.H), mx_parts(s.I), nullptr).bytes;
 }
@@ -774,8 +775,8 @@ int launch_ffn_mxfp4(const LayerShape& s, const WeightPtrs& shw, const MxPlanes&
   }
   {
     ProfScope ps(MOE_K_GATEUP, st);
-    rc |= launch_mx_gemv(true, s.H, s.I, s.E, s.k, T, w.gate_codes, w.gate_scales, w.up_codes, w.up_scales, fw.xd,
-                         fw.xs, r, fw.gu, err, sms, st);
+    rc |= launch_mx_gemv(w.fmt, true, s.H, s.I, s.E, s.k, T, w.gate_codes, w.gate_scales, w.up_codes, w.up_scales,
+                         fw.xd, fw.xs, r, fw.gu, err, sms, st);
   }
   {
     ProfScope ps(MOE_K_HQUANT, st);
@@ -783,8 +784,8 @@ int launch_ffn_mxfp4(const LayerShape& s, const WeightPtrs& shw, const MxPlanes&
   }
   {
     ProfScope ps(MOE_K_DOWN, st);
-    rc |= launch_mx_gemv(false, s.I, s.H, s.E, s.k, T, w.down_codes, w.down_scales, nullptr, nullptr, fw.hd, fw.hsc,
-                         r, fw.obuf, err, sms, st);
+    rc |= launch_mx_gemv(w.fmt, false, s.I, s.H, s.E, s.k, T, w.down_codes, w.down_scales, nullptr, nullptr, fw.hd,
+                         fw.hsc, r, fw.obuf, err, sms, st);
   }
   if (shared_early) {  // the shared output is ready in ysh once the side stream joins
     SideCtx* c = side_ctx(st);

@@ -70,7 +70,13 @@ int launch_gateup_tma(const LayerShape& sh, const uint8_t* gate_codes, const uin
                       const Routing& r, float* gpart, int* err, int sms, cudaStream_t st);
 // MXFP4 routed experts (mxfp4.cu; the step in decode.cu).
 struct MxPlanes {
-  const uint8_t *gate_codes, *gate_scales, *up_codes, *up_scales, *down_codes, *down_scales;
+  int fmt;  // 0 = MXFP4, 1 = Q4-style
+  const uint8_t* gate_codes;
+  const void* gate_scales;
+  const uint8_t* up_codes;
+  const void* up_scales;
+  const uint8_t* down_codes;
+  const void* down_scales;
 };
 size_t mx_ffn_workspace_bytes(const LayerShape& s, int T);
 int launch_ffn_mxfp4(const LayerShape& s, const WeightPtrs& shw, const MxPlanes& w, const void* x, int x_dtype,
@@ -78,11 +84,12 @@ int launch_ffn_mxfp4(const LayerShape& s, const WeightPtrs& shw, const MxPlanes&
                      cudaStream_t st, bool shared_early);
 bool mx_path_supported(const LayerShape& s, int T);
 int mx_parts(int K);
-int launch_mx_gemv(bool pair, int K, int R, int E, int k, int T, const uint8_t* codes0, const uint8_t* sc0,
-                   const uint8_t* codes1, const uint8_t* sc1, const int8_t* ad, const float* as, const Routing& r,
+// fmt: 0 = MXFP4 (E8M0 byte scales), 1 = Q4-style (fp16 scales)
+int launch_mx_gemv(int fmt, bool pair, int K, int R, int E, int k, int T, const uint8_t* codes0, const void* sc0,
+                   const uint8_t* codes1, const void* sc1, const int8_t* ad, const float* as, const Routing& r,
                    float* part, int* err, int sms, cudaStream_t st);
 int launch_mx_hquant(int I, int KP, int nA, const float* gu, int8_t* hd, float* hs, cudaStream_t st);
-int launch_mx_dequant(const uint8_t* codes, const uint8_t* scales, int64_t nb, float* out, cudaStream_t st);
+int launch_mx_dequant(int fmt, const uint8_t* codes, const void* scales, int64_t nb, float* out, cudaStream_t st);
 
 int launch_down_tma(const LayerShape& sh, const uint8_t* down_codes, const uint32_t* down_dd, const int8_t* hd,
                     const float* hsc, const int32_t* hq, int hss, int T, const Routing& r, float* opart, int* err,

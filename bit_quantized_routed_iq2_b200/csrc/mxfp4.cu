@@ -1,6 +1,6 @@
-// mxfp4.cu - decode GEMVs for MXFP4 routed experts (the second expert format
-// of moe_layer_forward_mxfp4), the h quantiser that feeds their down
-// projection, and the debug decoder.
+// mxfp4.cu - decode GEMVs for the block-32 routed-expert formats: MXFP4
+// (moe_layer_forward_mxfp4) and the Q4-style format (moe_layer_forward_q4);
+// the h quantiser that feeds their down projections; the debug decoders.
 //
 // Source: "ds4 : analyse pratique pour un usage documenté", section « Support
 // de modèles et choix de quantification » (an MXFP4 file keeps the routed
@@ -76,19 +76,34 @@ __device__ __forceinline__ float ld_sf_mx(uint32_t addr) {
   return v;
 }
 
-// positive and negative magnitudes of the 8 E2M1 magnitude codes, times 2, as int8 bytes
-constexpr uint32_t kMxPos0 = 0x03020100u, kMxPos1 = 0x0C080604u;  // 0 1 2 3 | 4 6 8 12
-constexpr uint32_t kMxNeg0 = 0xFDFEFF00u, kMxNeg1 = 0xF4F8FAFCu;  // 0 -1 -2 -3 | -4 -6 -8 -12
+// The two block-32 formats of this file: MXFP4 (E2M1 elements, E8M0 scale
+// byte per block) and the Q4-style format (unsigned 4-bit codes q, fp16 scale
+// d per block, w = d (q - 8)). Both decode a 4-bit code c by its low three bits
+// from one of two 8-entry byte tables, chosen by bit 3:
+//   MXFP4: bit 3 = sign; int8 = 2 * E2M1 value (0 1 2 3 4 6 8 12, negated)
+//   Q4:    bit 3 = q >= 8; int8 = q - 8 (-8 .. -1, 0 .. 7)
+enum BlkFmt : int { FMT_MXFP4 = 0, FMT_Q4 = 1 };
+template <int FMT> struct BlkTab;
+template <> struct BlkTab<FMT_MXFP4> {
+  static constexpr uint32_t t0 = 0x03020100u, t1 = 0x0C080604u;  // bit 3 clear: 0 1 2 3 | 4 6 8 12
+  static constexpr uint32_t u0 = 0xFDFEFF00u, u1 = 0xF4F8FAFCu;  // bit 3 set:  0 -1 -2 -3 | -4 -6 -8 -12
+};
+template <> struct BlkTab<FMT_Q4> {
+  static constexpr uint32_t t0 = 0xFBFAF9F8u, t1 = 0xFFFEFDFCu;  // q 0..7:  -8 .. -1
+  static constexpr uint32_t u0 = 0x03020100u, u1 = 0x07060504u;  // q 8..15:  0 .. 7
+};
 
-// Eight element codes (one 32-bit word, element i in nibble i) -> two int8x4
-// operand registers: elements 0..3 and 4..7, each 2 * E2M1 value.
-__device__ __forceinline__ void mx_decode8(uint32_t w, uint32_t& lo, uint32_t& hi) {
+// Eight codes (one 32-bit word, element i in nibble i) -> two int8x4 operand
+// registers: elements 0..3 and 4..7.
+template <int FMT>
+__device__ __forceinline__ void blk_decode8(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  using TB = BlkTab<FMT>;
   const uint32_t mag = w & 0x77777777u;
-  // byte i of the result comes from byte i of the positive pick (selector i) or of the negative pick (i + 4)
+  // byte i of the result comes from byte i of the first pick (selector i) or of the second (i + 4)
   const uint32_t sel = ((w >> 1) & 0x44444444u) | 0x32103210u;
   const uint32_t maghi = __umulhi(mag, 0x10000u), selhi = __umulhi(sel, 0x10000u);
-  lo = prmt(prmt(kMxPos0, kMxPos1, mag), prmt(kMxNeg0, kMxNeg1, mag), sel);
-  hi = prmt(prmt(kMxPos0, kMxPos1, maghi), prmt(kMxNeg0, kMxNeg1, maghi), selhi);
+  lo = prmt(prmt(TB::t0, TB::t1, mag), prmt(TB::u0, TB::u1, mag), sel);
+  hi = prmt(prmt(TB::t0, TB::t1, maghi), prmt(TB::u0, TB::u1, maghi), selhi);
 }
 
 // 2^(E - 128) exactly, for every byte E (subnormal for E < 2).
@@ -96,10 +111,34 @@ __device__ __forceinline__ float mx_pow2(uint32_t E) {
   return E >= 2u ? __uint_as_float((E - 1u) << 23) : __uint_as_float(0x00200000u << E);
 }
 
+// Mixed-radix walk over units v = v0, v0 + dv, ...: v = (slot * M + m) * rbs + rb.
+struct UnitIt {
+  int rb, m, slot, drb, dm, dslot;
+  __device__ __forceinline__ void init(int v0, int dv, int rbs, int M) {
+    rb = v0 % rbs;
+    int q = v0 / rbs;
+    m = q % M;
+    slot = q / M;
+    drb = dv % rbs;
+    q = dv / rbs;
+    dm = q % M;
+    dslot = q / M;
+  }
+  __device__ __forceinline__ void next(int rbs, int M) {
+    rb += drb;
+    int c = rb >= rbs ? 1 : 0;
+    rb -= c * rbs;
+    m += dm + c;
+    c = m >= M ? 1 : 0;
+    m -= c * M;
+    slot += dslot + c;
+  }
+};
+
 struct MxArgs {
   int K, R, E, k, KP, S, pair, nrows, nA;
-  const uint8_t* sc0;   // E8M0 planes [E][R][K/32] (gate or the single matrix; up)
-  const uint8_t* sc1;
+  const void* sc0;      // scale planes [E][R][K/32]: E8M0 bytes (MXFP4) or fp16 (Q4); gate or the single
+  const void* sc1;      // matrix, and up
   const int8_t* ad;     // activation digits [nrows][2][K], natural order
   const float* as;      // their scales [nrows][K/256] (2^s / 8)
   const int32_t* offsets;
@@ -125,6 +164,7 @@ __host__ __device__ inline MxPlan mx_plan(int E, int nA, int nrows, int S) {
   return p;
 }
 
+template <int FMT>
 __global__ void __launch_bounds__(kMxThreads, 1) mx_gemv_kernel(const __grid_constant__ CUtensorMap tm0,
                                                                const __grid_constant__ CUtensorMap tm1, MxArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -165,7 +205,6 @@ __global__ void __launch_bounds__(kMxThreads, 1) mx_gemv_kernel(const __grid_con
   for (int i = tid; i < a.nA; i += kMxThreads) arow[i] = a.pair ? a.perm[i] / a.k : i;
   __syncthreads();
   const int nact = act[a.E];
-  const int nunits = nact * M * rbs;
 
   if (warp == kMxCW) {  // producer
     if (lane == 0) {
@@ -173,13 +212,14 @@ __global__ void __launch_bounds__(kMxThreads, 1) mx_gemv_kernel(const __grid_con
       if (a.pair) prefetch_tmap(&tm1);
       const uint64_t pol = l2_policy_evict_first();  // expert codes are read once per step
       RingPos rp{0, 0u};
-      for (int v = kib; v < nunits; v += kG) {
-        const int rb = v % rbs, q = v / rbs, m = q % M, slot = q / M;
-        const int e = act[slot];
+      UnitIt it;
+      it.init(kib, kG, rbs, M);
+      for (; it.slot < nact; it.next(rbs, M)) {
+        const int e = act[it.slot];
         if (!mbar_wait_bounded(&empty[rp.s], rp.ph ^ 1u, a.err, ERR_TIMEOUT)) return;
         mbar_arrive_expect_tx(&full[rp.s], kMxBox);
-        tma_load_2d_hint(ring + rp.s * kMxBox, m ? &tm1 : &tm0, kpc * kMxBoxW, e * R + rb * kMxRows, &full[rp.s],
-                         pol);
+        tma_load_2d_hint(ring + rp.s * kMxBox, it.m ? &tm1 : &tm0, kpc * kMxBoxW, e * R + it.rb * kMxRows,
+                         &full[rp.s], pol);
         rp.next(S);
       }
     }
@@ -208,14 +248,35 @@ __global__ void __launch_bounds__(kMxThreads, 1) mx_gemv_kernel(const __grid_con
   const uint32_t ass_s = smem_addr(ass);
   const int spr = K / 32;  // scale bytes per row
   RingPos rp{0, 0u};
-  for (int v = kib; v < nunits; v += kG) {
-    const int rb = v % rbs, q = v / rbs, m = q % M, slot = q / M;
-    const int e = act[slot];
+  // this CTA's units v = kib, kib + kG, ... as a mixed-radix counter (rb fastest, then m, then slot)
+  UnitIt it;
+  it.init(kib, kG, rbs, M);
+  // the scales of a unit, rows g and g + 8 (MXFP4: 8 bytes per row; Q4: 8 fp16 per row), loaded one unit
+  // ahead so that their latency is hidden behind the previous unit
+  auto ldsc = [&](const UnitIt& u, uint4& s0v, uint4& s8v) {
+    const int eu = act[u.slot];
+    const size_t sidx = (static_cast<size_t>(eu) * R + u.rb * kMxRows + row_l) * spr + kpc * 8;
+    if (FMT == FMT_MXFP4) {
+      const uint8_t* scp = static_cast<const uint8_t*>(u.m ? a.sc1 : a.sc0) + sidx;
+      const uint2 v0 = __ldg(reinterpret_cast<const uint2*>(scp));
+      const uint2 v8 = __ldg(reinterpret_cast<const uint2*>(scp + 8 * static_cast<size_t>(spr)));
+      s0v = make_uint4(v0.x, v0.y, 0u, 0u);
+      s8v = make_uint4(v8.x, v8.y, 0u, 0u);
+    } else {
+      const uint16_t* scp = static_cast<const uint16_t*>(u.m ? a.sc1 : a.sc0) + sidx;
+      s0v = __ldg(reinterpret_cast<const uint4*>(scp));
+      s8v = __ldg(reinterpret_cast<const uint4*>(scp + 8 * static_cast<size_t>(spr)));
+    }
+  };
+  uint4 nsg0 = make_uint4(0u, 0u, 0u, 0u), nsg8 = nsg0;
+  if (it.slot < nact) ldsc(it, nsg0, nsg8);
+  while (it.slot < nact) {
+    const int rb = it.rb, m = it.m;
+    const int e = act[it.slot];
     const int p0 = off[e], ne = off[e + 1] - p0;
-    // the scales of the unit's 8 blocks, rows g and g + 8: loaded before the data wait, used after the MMAs
-    const uint8_t* scp = (m ? a.sc1 : a.sc0) + (static_cast<size_t>(e) * R + rb * kMxRows + row_l) * spr + kpc * 8;
-    const uint2 sg0 = __ldg(reinterpret_cast<const uint2*>(scp));
-    const uint2 sg8 = __ldg(reinterpret_cast<const uint2*>(scp + 8 * static_cast<size_t>(spr)));
+    const uint4 sg0 = nsg0, sg8 = nsg8;
+    it.next(rbs, M);
+    if (it.slot < nact) ldsc(it, nsg0, nsg8);
     if (!mbar_wait_bounded(&full[rp.s], rp.ph, a.err, ERR_TIMEOUT)) return;
     const uint32_t st = rec0 + static_cast<uint32_t>(rp.s) * kMxBox;
     const uint4 ra0 = ld_s128_mx(st + 16u * ch0), rb0 = ld_s128_mx(st + 8u * kMxBoxW + 16u * ch0);
@@ -225,9 +286,23 @@ __global__ void __launch_bounds__(kMxThreads, 1) mx_gemv_kernel(const __grid_con
     rp.next(S);
     const uint32_t wa[2][4] = {{ra0.x, ra0.y, ra0.z, ra0.w}, {ra1.x, ra1.y, ra1.z, ra1.w}};
     const uint32_t wb[2][4] = {{rb0.x, rb0.y, rb0.z, rb0.w}, {rb1.x, rb1.y, rb1.z, rb1.w}};
-    // 2^(E - 128) of this lane's blocks (tig and 4 + tig), rows g and g + 8
-    const float s0[2] = {mx_pow2((sg0.x >> (8 * tig)) & 0xFFu), mx_pow2((sg0.y >> (8 * tig)) & 0xFFu)};
-    const float s8[2] = {mx_pow2((sg8.x >> (8 * tig)) & 0xFFu), mx_pow2((sg8.y >> (8 * tig)) & 0xFFu)};
+    // the scale factors of this lane's blocks (tig and 4 + tig), rows g and g + 8: MXFP4 2^(E - 128)
+    // (the elements enter doubled), Q4 d
+    float s0[2], s8[2];
+    if (FMT == FMT_MXFP4) {
+      s0[0] = mx_pow2((sg0.x >> (8 * tig)) & 0xFFu);
+      s0[1] = mx_pow2((sg0.y >> (8 * tig)) & 0xFFu);
+      s8[0] = mx_pow2((sg8.x >> (8 * tig)) & 0xFFu);
+      s8[1] = mx_pow2((sg8.y >> (8 * tig)) & 0xFFu);
+    } else {
+      // fp16 of block b is half b & 1 of word b >> 1: blocks tig (words 0, 1) and 4 + tig (words 2, 3)
+      const bool hw = (tig >> 1) != 0;
+      const uint32_t sh = 16u * (tig & 1);
+      s0[0] = half_bits_to_float(static_cast<uint16_t>((hw ? sg0.y : sg0.x) >> sh));
+      s0[1] = half_bits_to_float(static_cast<uint16_t>((hw ? sg0.w : sg0.z) >> sh));
+      s8[0] = half_bits_to_float(static_cast<uint16_t>((hw ? sg8.y : sg8.x) >> sh));
+      s8[1] = half_bits_to_float(static_cast<uint16_t>((hw ? sg8.w : sg8.z) >> sh));
+    }
     for (int t0 = 0; t0 < ne; t0 += kMxTok) {
       float f0[kMxTok], f1[kMxTok];
       int ar[kMxTok];
@@ -241,8 +316,8 @@ __global__ void __launch_bounds__(kMxThreads, 1) mx_gemv_kernel(const __grid_con
         uint32_t A[4][4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          mx_decode8(wa[cc][j], A[j][0], A[j][2]);  // row g: elements 8j..8j+3, 8j+4..8j+7
-          mx_decode8(wb[cc][j], A[j][1], A[j][3]);  // row g + 8
+          blk_decode8<FMT>(wa[cc][j], A[j][0], A[j][2]);  // row g: elements 8j..8j+3, 8j+4..8j+7
+          blk_decode8<FMT>(wb[cc][j], A[j][1], A[j][3]);  // row g + 8
         }
 #pragma unroll
         for (int t = 0; t < kMxTok; ++t) {
@@ -345,15 +420,17 @@ __global__ void __launch_bounds__(256) mx_hquant_kernel(int I, int KP, const flo
 }
 
 // Debug decoder: one thread per block, the kernels' element decoding.
-__global__ void mx_dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales, int64_t nb,
+template <int FMT>
+__global__ void mx_dequant_kernel(const uint8_t* __restrict__ codes, const void* __restrict__ scales, int64_t nb,
                                   float* __restrict__ out) {
   for (int64_t b = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; b < nb;
        b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const float sc = mx_pow2(scales[b]);
+    const float sc = FMT == FMT_MXFP4 ? mx_pow2(static_cast<const uint8_t*>(scales)[b])
+                                      : half_bits_to_float(static_cast<const uint16_t*>(scales)[b]);
     for (int w = 0; w < 4; ++w) {
       const uint32_t word = *reinterpret_cast<const uint32_t*>(codes + b * 16 + 4 * w);
       uint32_t lo, hi;
-      mx_decode8(word, lo, hi);
+      blk_decode8<FMT>(word, lo, hi);
       for (int i = 0; i < 8; ++i) {
         const int8_t v = static_cast<int8_t>(((i < 4 ? lo : hi) >> (8 * (i & 3))) & 0xFFu);
         out[b * 32 + 8 * w + i] = static_cast<float>(v) * sc;
@@ -402,8 +479,8 @@ int mx_parts(int K) { return K / kMxPart; }
 
 // One MXFP4 GEMV launch: pair = gate + up over the token rows of x digits (partials [nA][2][KP][R]),
 // else the single (down) matrix over the assignment rows of h digits (partials [nA][KP][R]).
-int launch_mx_gemv(bool pair, int K, int R, int E, int k, int T, const uint8_t* codes0, const uint8_t* sc0,
-                   const uint8_t* codes1, const uint8_t* sc1, const int8_t* ad, const float* as,
+int launch_mx_gemv(int fmt, bool pair, int K, int R, int E, int k, int T, const uint8_t* codes0, const void* sc0,
+                   const uint8_t* codes1, const void* sc1, const int8_t* ad, const float* as,
                    const Routing& r, float* part, int* err, int sms, cudaStream_t st) {
   const int nA = T * k, nrows = pair ? T : nA;
   CUtensorMap t0, t1;
@@ -424,8 +501,15 @@ int launch_mx_gemv(bool pair, int K, int R, int E, int k, int T, const uint8_t* 
   const int slots = std::min(nA, E);
   const int units = slots * (pair ? 2 : 1) * (R / kMxRows) * a.KP;
   const int grid = std::max(a.KP, std::min(units, sms));
-  cudaFuncSetAttribute(mx_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  launch_pdl(mx_gemv_kernel, dim3(grid), dim3(kMxThreads), smem, st, t0, t1, a);
+  if (fmt == FMT_MXFP4) {
+    cudaFuncSetAttribute(mx_gemv_kernel<FMT_MXFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    launch_pdl(mx_gemv_kernel<FMT_MXFP4>, dim3(grid), dim3(kMxThreads), smem, st, t0, t1, a);
+  } else if (fmt == FMT_Q4) {
+    cudaFuncSetAttribute(mx_gemv_kernel<FMT_Q4>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    launch_pdl(mx_gemv_kernel<FMT_Q4>, dim3(grid), dim3(kMxThreads), smem, st, t0, t1, a);
+  } else {
+    return ERR_ARG;
+  }
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
 }
 
@@ -434,10 +518,15 @@ int launch_mx_hquant(int I, int KP, int nA, const float* gu, int8_t* hd, float* 
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
 }
 
-int launch_mx_dequant(const uint8_t* codes, const uint8_t* scales, int64_t nb, float* out, cudaStream_t st) {
+int launch_mx_dequant(int fmt, const uint8_t* codes, const void* scales, int64_t nb, float* out, cudaStream_t st) {
   if (nb <= 0) return OK;
   const int grid = static_cast<int>(std::min<int64_t>((nb + 255) / 256, 4096));
-  mx_dequant_kernel<<<grid, 256, 0, st>>>(codes, scales, nb, out);
+  if (fmt == FMT_MXFP4)
+    mx_dequant_kernel<FMT_MXFP4><<<grid, 256, 0, st>>>(codes, scales, nb, out);
+  else if (fmt == FMT_Q4)
+    mx_dequant_kernel<FMT_Q4><<<grid, 256, 0, st>>>(codes, scales, nb, out);
+  else
+    return ERR_ARG;
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
 }
 

@@ -35,6 +35,7 @@ EXPORTS = (
     "moe_prefetch_layer", "moe_debug_bounds_check_build", "moe_debug_bounds_violations",
     "moe_cache_bytes", "moe_cache_create", "moe_cache_destroy", "moe_cache_read_stats", "moe_layer_forward_cached",
     "moe_workspace_size_mxfp4", "moe_layer_forward_mxfp4", "moe_debug_dequant_mxfp4",
+    "moe_workspace_size_q4", "moe_layer_forward_q4", "moe_debug_dequant_q4",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 KERNEL_NAMES = ("router_logits", "topk", "permute", "active", "gateup", "down", "shared_gateup", "shared_down",
@@ -65,7 +66,8 @@ class Weights(ctypes.Structure):
 
 
 class MxWeights(ctypes.Structure):
-    """moe_mxfp4_weights: router, MXFP4 code and E8M0 scale planes, shared expert."""
+    """moe_mxfp4_weights (router, MXFP4 code and E8M0 scale planes, shared expert); the same
+    pointer layout serves moe_q4_weights (code planes and fp16 d planes)."""
 
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "router_w", "router_bias", "gate_codes", "gate_scales", "up_codes", "up_scales",
@@ -99,6 +101,9 @@ def load() -> ctypes.CDLL:
     L.moe_workspace_size_mxfp4.argtypes = [pd, i32, ctypes.POINTER(sz)]
     L.moe_layer_forward_mxfp4.argtypes = [pd, ctypes.POINTER(MxWeights), vp, i32, i32, vp, vp, vp, sz, vp]
     L.moe_debug_dequant_mxfp4.argtypes = [vp, vp, i64, vp, vp]
+    L.moe_workspace_size_q4.argtypes = [pd, i32, ctypes.POINTER(sz)]
+    L.moe_layer_forward_q4.argtypes = [pd, ctypes.POINTER(MxWeights), vp, i32, i32, vp, vp, vp, sz, vp]
+    L.moe_debug_dequant_q4.argtypes = [vp, vp, i64, vp, vp]
     L.moe_debug_gemv_operands_iq2.argtypes = [vp, i64, vp, vp, vp]
     L.moe_debug_gemv_operands_q2k.argtypes = [vp, i64, vp, vp, vp]
     L.moe_debug_tc_operands_iq2.argtypes = [vp, vp, i64, vp, vp]
@@ -360,6 +365,25 @@ def to_device_mxfp4(lw, device="cuda") -> MxDeviceLayer:
         "sh_down": up(lw.sh_down, np.int16) if lw.Is else None,
     }
     return MxDeviceLayer(desc_of(lw.H, lw.I, lw.E, lw.k, lw.Is), t)
+
+
+def to_device_q4(lw, device="cuda") -> MxDeviceLayer:
+    """Upload the host planes of a Q4-style layer (synth.Q4LayerWeights layout). The fp16 d planes
+    travel as their bytes (the upload of to_device_mxfp4 views every scale plane as bytes)."""
+    return to_device_mxfp4(lw, device)
+
+
+def layer_forward_q4(layer: MxDeviceLayer, x, residual, y, ws, stream=None):
+    T = x.shape[0]
+    w = layer.weights
+    _check(load().moe_layer_forward_q4(ctypes.byref(layer.desc), ctypes.byref(w), _ptr(x), _dtype_of(x), T,
+                                       _ptr(residual), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
+                                       _stream(stream)), "moe_layer_forward_q4")
+
+
+def debug_dequant_q4(codes, d, out, stream=None):
+    nb = codes.numel() // 16
+    _check(load().moe_debug_dequant_q4(_ptr(codes), _ptr(d), nb, _ptr(out), _stream(stream)), "moe_debug_dequant_q4")
 
 
 def workspace_size_mxfp4(desc: Desc, max_tokens: int) -> int:

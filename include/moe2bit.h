@@ -497,6 +497,51 @@ MOE_API moe_status moe_layer_forward_mxfp4(const moe_layer_desc* desc, const moe
 MOE_API moe_status moe_debug_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t n_blocks, float* out,
                                            void* stream);
 
+/*
+ * Q4-style routed experts (third expert format).
+ *
+ * The pages name 4-bit routed-expert variants ([R]: Q4 models; [W]: routed
+ * expert checkpoints shared between the 2-bit and 4-bit variants) without a
+ * layout. This library's Q4-style block: 32 weights along the reduction axis,
+ * one fp16 scale d and 32 unsigned 4-bit codes q; w = d * (q - 8). A matrix
+ * [rows][K] (K % 32 == 0) is two planes:
+ *   codes [rows][K/2] bytes: element 2i in bits 0..3 of byte i, 2i+1 in bits 4..7;
+ *   d     [rows][K/32] fp16.
+ * moe_layer_forward_q4 is moe_layer_forward_mxfp4 with these planes: the same
+ * routing, shared expert, combine, shapes (hidden % 512 == 0, inter % 512 ==
+ * 0, 1 <= T <= 16, n_experts <= 1024), alignment, workspace
+ * (moe_workspace_size_q4, equal to moe_workspace_size_mxfp4), status and
+ * errors; the elements enter the integer products as the exact int8 q - 8 and
+ * every block is scaled by its d in fp32.
+ */
+typedef struct {
+  const uint16_t* router_w;     /* bf16 [E][H] */
+  const float* router_bias;     /* fp32 [E], or NULL */
+  const uint8_t* gate_codes;    /* [E][I][H/2] */
+  const uint16_t* gate_d;       /* fp16 [E][I][H/32] */
+  const uint8_t* up_codes;      /* [E][I][H/2] */
+  const uint16_t* up_d;         /* fp16 [E][I][H/32] */
+  const uint8_t* down_codes;    /* [E][H][I/2] */
+  const uint16_t* down_d;       /* fp16 [E][H][I/32] */
+  const uint16_t* sh_gate;      /* bf16 [I_s][H] (unused when I_s == 0) */
+  const uint16_t* sh_up;        /* bf16 [I_s][H] */
+  const uint16_t* sh_down;      /* bf16 [H][I_s] */
+} moe_q4_weights;
+
+MOE_API moe_status moe_workspace_size_q4(const moe_layer_desc* desc, int32_t max_tokens, size_t* bytes);
+MOE_API moe_status moe_layer_forward_q4(const moe_layer_desc* desc, const moe_q4_weights* w, const void* x,
+                                        moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws,
+                                        size_t ws_bytes, void* stream);
+
+/*
+ * Decode n_blocks consecutive Q4-style blocks (codes: device [n_blocks][16]
+ * bytes, d: device fp16 [n_blocks]) into out: device fp32 [n_blocks][32], with
+ * the GPU path's decoding (int8 q - 8 times d). Stream-ordered;
+ * MOE_ERR_INVALID_ARG for null pointers or n_blocks < 0.
+ */
+MOE_API moe_status moe_debug_dequant_q4(const uint8_t* codes, const uint16_t* d, int64_t n_blocks, float* out,
+                                        void* stream);
+
 /* Host copy of the library's compiled-in 256 x 8 IQ2 codebook (row-major,
  * values in {8, 25, 43}). `out` is a host pointer to 2048 bytes. */
 MOE_API void moe_debug_grid(uint8_t* out);

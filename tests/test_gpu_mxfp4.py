@@ -1,4 +1,5 @@
-"""MXFP4 routed experts on the GPU (moe_layer_forward_mxfp4) against the oracle.
+"""Block-32 routed experts on the GPU against the oracle: MXFP4
+(moe_layer_forward_mxfp4) and the Q4-style format (moe_layer_forward_q4).
 
 Element decoding bit-for-bit (as values) through moe_debug_dequant_mxfp4; the
 layer within the normwise bound of the 2-bit path (FFN_TOL) at small shapes
@@ -102,4 +103,63 @@ def test_mxfp4_decode1_shape(torch_cuda):
     y = _mx_forward(torch_cuda, moe2bit.to_device_mxfp4(lw), x)
     ref, ridx, _ = oracle.layer_forward(lw, x)
     assert np.array_equal(np.sort(ridx, axis=1), np.sort(idx, axis=1))
+    assert normwise(y, ref) <= FFN_TOL, normwise(y, ref)
+
+
+# ------------------------------------------------------------------ Q4-style
+def test_q4_dequant_matches_oracle(torch_cuda):
+    torch = torch_cuda
+    nb = 4096
+    codes = synth.rand_bytes(0x513401, (nb, 16))
+    codes[:256] = np.arange(256, dtype=np.uint8)[:, None]
+    d = synth.f16_scale(0x513402, (nb,), 0.01)
+    d[:4] = [0x3C00, 0xBC00, 0x0001, 0x7BFF]  # 1, -1, the smallest subnormal, the largest finite
+    out = torch.empty(nb * 32, dtype=torch.float32, device="cuda")
+    moe2bit.debug_dequant_q4(torch.from_numpy(codes).cuda(), torch.from_numpy(d.view(np.int16)).cuda(), out)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy(), oracle.dequant_q4(codes, d))
+
+
+def _q4_forward(torch, dl, x, residual=None):
+    T = x.shape[0]
+    y = torch.full((T, dl.desc.hidden), float("nan"), dtype=torch.float32, device="cuda")
+    res = None if residual is None else torch.from_numpy(np.ascontiguousarray(residual)).cuda()
+    n = ctypes_size_q4(dl.desc, T)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    moe2bit.layer_forward_q4(dl, _x_dev(torch, x), res, y, ws)
+    torch.cuda.synchronize()
+    assert moe2bit.read_status(ws) == 0
+    return y.cpu().numpy()
+
+
+def ctypes_size_q4(desc, T):
+    import ctypes
+
+    n = ctypes.c_size_t(0)
+    assert moe2bit.load().moe_workspace_size_q4(ctypes.byref(desc), T, ctypes.byref(n)) == 0
+    return max(int(n.value), 16)
+
+
+@pytest.mark.parametrize("name", ["t1_bf16", "t5_bf16_zipf", "t16_f32"])
+def test_q4_layer_small(torch_cuda, name):
+    c = CASES[name]
+    cfg = synth.Config("q4_" + name, c["T"], 1024, 512, 16, 4, c["Is"], c["x_dtype"], 1.0, c["zipf"], 1,
+                       0x5134A0 + len(name))
+    lw = synth.make_layer_q4(cfg)
+    x = screened_x(cfg, lw)
+    res = synth.make_residual(cfg, cfg.T)
+    y = _q4_forward(torch_cuda, moe2bit.to_device_q4(lw), x, res)
+    ref, _, _ = oracle.layer_forward(lw, x, res)
+    assert normwise(y, ref) <= FFN_TOL, (name, normwise(y, ref))
+
+
+@pytest.mark.slow
+def test_q4_decode1_shape(torch_cuda):
+    cfg = synth.CONFIGS["decode1"]
+    base = synth.make_layer(cfg, experts=[])
+    x = screened_x(cfg, base)
+    idx, _ = oracle.route(base.router_w, base.router_bias, x, cfg.k)
+    lw = synth.make_layer_q4(cfg, experts=np.unique(idx))
+    y = _q4_forward(torch_cuda, moe2bit.to_device_q4(lw), x)
+    ref, _, _ = oracle.layer_forward(lw, x)
     assert normwise(y, ref) <= FFN_TOL, normwise(y, ref)
