@@ -480,6 +480,7 @@ __global__ void __launch_bounds__(1024) topk_permute_sort_kernel(const float* __
   __shared__ int cand_i[1024];
   __shared__ int sel[32];
   __shared__ float chosen[32];
+  __shared__ float ex[32];
   __shared__ int first[32];
   pdl_trigger();
   pdl_wait();
@@ -532,13 +533,15 @@ __global__ void __launch_bounds__(1024) topk_permute_sort_kernel(const float* __
     }
   }
   __syncthreads();
+  // exp(l_j - l_0) of every chosen slot at once, then the sum in slot order by one thread per token
+  if (tid < n) ex[tid] = expf(chosen[tid] - chosen[(tid / k) * k]);
+  __syncthreads();
   if (tid < T) {
-    const float* c = chosen + tid * k;
     float z = 0.f;
-    for (int j = 0; j < k; ++j) z += expf(c[j] - c[0]);
+    for (int j = 0; j < k; ++j) z += ex[tid * k + j];
     for (int j = 0; j < k; ++j) {
       topk_idx[tid * k + j] = sel[tid * k + j];
-      topk_w[tid * k + j] = expf(c[j] - c[0]) / z;
+      topk_w[tid * k + j] = ex[tid * k + j] / z;
     }
   }
   if (tid < n) {
