@@ -38,7 +38,7 @@ class Weights(ctypes.Structure):
     ]
 
 
-FMT_IQ2_Q2K, FMT_MXFP4, FMT_Q4 = 0, 1, 2
+FMT_IQ2_Q2K, FMT_MXFP4, FMT_Q4, FMT_MXFP4_A8 = 0, 1, 2, 3
 
 
 def build(force: bool = False, openmp: bool | None = None) -> str:
@@ -95,6 +95,11 @@ def lib():
         L.moeref_e2m1.argtypes = [ctypes.c_uint]
         L.moeref_dequant_mxfp4.argtypes = [vp, vp, i64, vp]
         L.moeref_dequant_q4.argtypes = [vp, vp, i64, vp]
+        L.moeref_e4m3_decode.restype = ctypes.c_double
+        L.moeref_e4m3_decode.argtypes = [ctypes.c_uint]
+        L.moeref_e4m3_encode.restype = ctypes.c_uint
+        L.moeref_e4m3_encode.argtypes = [ctypes.c_double]
+        L.moeref_quant_mxfp8.argtypes = [vp, i64, vp, vp]
         L.moeref_route.argtypes = [i32, i32, i32, vp, vp, vp, i32, i32, vp, vp, vp]
         L.moeref_permute.argtypes = [i32, i32, i32, vp, vp, vp, vp]
         L.moeref_f32_to_f16.restype = ctypes.c_uint16
@@ -175,6 +180,28 @@ def dequant_mxfp4(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     return out
 
 
+def e4m3_decode(c: int) -> float:
+    """The value of one FP8 E4M3 code (OCP MX v1.0 element type; NaN for S.1111.111)."""
+    return float(lib().moeref_e4m3_decode(int(c)))
+
+
+def e4m3_encode(v: float) -> int:
+    """Nearest finite E4M3 code to ``v`` (ties to the even code, saturating at 448)."""
+    return int(lib().moeref_e4m3_encode(float(v)))
+
+
+def quant_mxfp8(v: np.ndarray):
+    """Values (a multiple of 32, blocks along the flattened array, float64) ->
+    (E4M3 codes [nb][32] u8, E8M0 scale bytes [nb] u8) by the MX block rule."""
+    v = np.ascontiguousarray(v, np.float64).reshape(-1)
+    assert v.size % 32 == 0
+    nb = v.size // 32
+    el = np.zeros((nb, 32), np.uint8)
+    sc = np.zeros(nb, np.uint8)
+    lib().moeref_quant_mxfp8(_p(v), nb, _p(el), _p(sc))
+    return el, sc
+
+
 def dequant_q4(codes: np.ndarray, d: np.ndarray) -> np.ndarray:
     """Q4-style blocks (codes [nb][16] u8, fp16 d [nb]) -> fp32 [nb * 32]."""
     codes = np.ascontiguousarray(codes, np.uint8).reshape(-1, 16)
@@ -235,26 +262,30 @@ def permute(idx: np.ndarray, E: int):
     return offsets, perm, inv
 
 
-def _structs(lw):
+def _structs(lw, act_mxfp8: bool = False):
     """Oracle structs of a layer; a layer with ``fmt == "mxfp4"`` carries MXFP4
-    code planes and E8M0 scale planes instead of the IQ2 / Q2K planes."""
+    code planes and E8M0 scale planes instead of the IQ2 / Q2K planes.
+    ``act_mxfp8`` (MXFP4 layers only) quantises the routed experts' activations
+    to MXFP8 before each contraction (the block-scaled FP4 x FP8 reading)."""
     desc = Desc(lw.H, lw.I, lw.E, lw.k, lw.Is)
     fmt = getattr(lw, "fmt", "iq2")
+    assert not act_mxfp8 or fmt == "mxfp4", "MXFP8 activations go with MXFP4 weights"
     mx = fmt in ("mxfp4", "q4")
     arrs = (lw.router_w, lw.router_bias, lw.gate_codes, None if mx else lw.gate_d, lw.up_codes,
             None if mx else lw.up_d, lw.down_codes, None if mx else lw.down_dd, lw.sh_gate, lw.sh_up, lw.sh_down)
     keep = [np.ascontiguousarray(a) if a is not None else None for a in arrs]
     sc = [np.ascontiguousarray(getattr(lw, n)) for n in ("gate_scales", "up_scales", "down_scales")] if mx else []
     keep += sc
-    W = Weights(*[_p(a) for a in keep[:11]], {"mxfp4": FMT_MXFP4, "q4": FMT_Q4}.get(fmt, FMT_IQ2_Q2K),
+    code = FMT_MXFP4_A8 if act_mxfp8 else {"mxfp4": FMT_MXFP4, "q4": FMT_Q4}.get(fmt, FMT_IQ2_Q2K)
+    W = Weights(*[_p(a) for a in keep[:11]], code,
                 *([_p(a) for a in sc] if mx else [None, None, None]))
     return desc, W, keep
 
 
-def expert_ffn(lw, x, idx, w, residual=None) -> np.ndarray:
+def expert_ffn(lw, x, idx, w, residual=None, act_mxfp8: bool = False) -> np.ndarray:
     x = np.ascontiguousarray(x)
     T = x.shape[0]
-    desc, W, keep = _structs(lw)
+    desc, W, keep = _structs(lw, act_mxfp8)
     y = np.zeros((T, lw.H), np.float32)
     res = None if residual is None else np.ascontiguousarray(residual, np.float32)
     _check(lib().moeref_expert_ffn(ctypes.byref(desc), ctypes.byref(W), _p(x), _dtype_code(x), T,
@@ -263,10 +294,10 @@ def expert_ffn(lw, x, idx, w, residual=None) -> np.ndarray:
     return y
 
 
-def layer_forward(lw, x, residual=None):
+def layer_forward(lw, x, residual=None, act_mxfp8: bool = False):
     x = np.ascontiguousarray(x)
     T = x.shape[0]
-    desc, W, keep = _structs(lw)
+    desc, W, keep = _structs(lw, act_mxfp8)
     y = np.zeros((T, lw.H), np.float32)
     idx = np.zeros((T, lw.k), np.int32)
     w = np.zeros((T, lw.k), np.float32)

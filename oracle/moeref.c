@@ -63,8 +63,11 @@ typedef struct {
   const uint8_t* down_scales;
 } moeref_weights;
 
-enum { REF_FMT_IQ2_Q2K = 0, REF_FMT_MXFP4 = 1, REF_FMT_Q4 = 2 };
-/* With REF_FMT_Q4 the three scale pointers hold fp16 d per block, [rows][K/32] uint16. */
+enum { REF_FMT_IQ2_Q2K = 0, REF_FMT_MXFP4 = 1, REF_FMT_Q4 = 2, REF_FMT_MXFP4_A8 = 3 };
+/* With REF_FMT_Q4 the three scale pointers hold fp16 d per block, [rows][K/32] uint16.
+   REF_FMT_MXFP4_A8: the MXFP4 weights of REF_FMT_MXFP4, and the two routed
+   contractions take their activations (x, then h) quantised to MXFP8 first
+   (moeref_quant_mxfp8 below); the shared expert is unaffected. */
 
 /* ---------------------------------------------------------------- scalars */
 
@@ -223,6 +226,77 @@ static void dequant_matrix_mxfp4(const uint8_t* codes, const uint8_t* scales, in
   moeref_dequant_mxfp4(codes + (int64_t)e * nb * 16, scales + (int64_t)e * nb, nb, out);
 }
 
+/* ------------------------------------------------------------------ MXFP8
+ * Activations for a block-scaled FP4 x FP8 contraction: OCP Microscaling
+ * Formats (MX) v1.0, the FP8 E4M3 element type with one E8M0 scale per block
+ * of 32 (the MXFP8 format of that specification). E4M3: sign bit 7, exponent
+ * bits 6..3 with bias 7, mantissa bits 2..0; exponent field 0 holds the
+ * subnormals m * 2^-9; S.1111.111 is NaN and there is no infinity, so the
+ * largest finite magnitude is 1.75 * 2^8 = 448.
+ * Conversion of a block (the specification's rule): the shared exponent is
+ * X = floor(log2(max |v_i|)) - emax, emax = 8 for E4M3 (the exponent of the
+ * largest normal), clamped to the E8M0 range [-127, 127]; each element is
+ * v_i / 2^X rounded to the nearest E4M3 value, ties to the even code, and
+ * magnitudes beyond 448 saturate to 448 (the specification leaves overflow of
+ * FP8 to the implementation; saturation is the reading taken here). A block of
+ * zeros gets X = -127. The scale byte is X + 127.
+ * Parity: pinned by the E4M3 value table of the specification, a library
+ * float8_e4m3fn conversion on in-range values, hand-computed blocks and a
+ * dense float64 MoE with an independent implementation of the block rule. */
+double moeref_e4m3_decode(unsigned c) {
+  const unsigned ex = (c >> 3) & 15u, man = c & 7u;
+  if (ex == 15u && man == 7u) return NAN;
+  const double mag = ex == 0 ? ldexp((double)man, -9) : ldexp(1.0 + man / 8.0, (int)ex - 7);
+  return (c & 0x80u) ? -mag : mag;
+}
+
+/* nearest finite E4M3 code to v (ties to the even code), saturating at 448;
+   a binary search over the increasing magnitudes of codes 0x00..0x7E */
+unsigned moeref_e4m3_encode(double v) {
+  const unsigned sign = (v < 0.0 || (v == 0.0 && signbit(v))) ? 0x80u : 0u;
+  const double a = fabs(v);
+  unsigned lo = 0, hi = 0x7Eu; /* invariant: value(lo) <= a (or lo = 0), answer in [lo, hi] */
+  if (a >= moeref_e4m3_decode(0x7Eu)) return sign | 0x7Eu;
+  while (hi - lo > 1u) {
+    const unsigned mid = (lo + hi) / 2u;
+    if (moeref_e4m3_decode(mid) <= a) lo = mid; else hi = mid;
+  }
+  /* a lies in [value(lo), value(hi)) */
+  const double dl = a - moeref_e4m3_decode(lo), dh = moeref_e4m3_decode(hi) - a;
+  unsigned c;
+  if (dl < dh) c = lo;
+  else if (dh < dl) c = hi;
+  else c = (lo & 1u) ? hi : lo;
+  return sign | c;
+}
+
+/* n blocks of 32 values -> E4M3 codes [n][32] and E8M0 scale bytes [n] */
+void moeref_quant_mxfp8(const double* v, int64_t nblocks, uint8_t* elem, uint8_t* scale) {
+  for (int64_t b = 0; b < nblocks; ++b) {
+    double amax = 0.0;
+    for (int i = 0; i < 32; ++i) amax = fmax(amax, fabs(v[b * 32 + i]));
+    int X = -127;
+    if (amax > 0.0) {
+      int e2;
+      frexp(amax, &e2); /* amax = f * 2^e2, f in [0.5, 1): floor(log2 amax) = e2 - 1 */
+      X = (e2 - 1) - 8;
+      if (X < -127) X = -127;
+      if (X > 127) X = 127;
+    }
+    scale[b] = (uint8_t)(X + 127);
+    for (int i = 0; i < 32; ++i) elem[b * 32 + i] = (uint8_t)moeref_e4m3_encode(ldexp(v[b * 32 + i], -X));
+  }
+}
+
+/* the values an MXFP8 block represents: element * 2^(scale - 127), in place */
+static void mxfp8_round_trip(double* v, int64_t nblocks) {
+  uint8_t el[32], sc;
+  for (int64_t b = 0; b < nblocks; ++b) {
+    moeref_quant_mxfp8(v + b * 32, 1, el, &sc);
+    for (int i = 0; i < 32; ++i) v[b * 32 + i] = ldexp(moeref_e4m3_decode(el[i]), (int)sc - 127);
+  }
+}
+
 /* -------------------------------------------------------------------- Q4
  * The 4-bit routed-expert variant the pages mention ("Un modèle de 284
  * milliards ...", « Comment un 284B tient »: Q4 models; "antirez/ds4 ...":
@@ -357,7 +431,8 @@ int moeref_expert_ffn(const moeref_desc* desc, const moeref_weights* W, const vo
   const int H = desc->hidden, I = desc->inter, E = desc->n_experts, k = desc->top_k, Is = desc->shared_inter;
   if (H <= 0 || I <= 0 || E <= 0 || k <= 0 || k > E || Is < 0) return REF_ERR_ARG;
   const int q4 = W->expert_format == REF_FMT_Q4;
-  const int mx = W->expert_format == REF_FMT_MXFP4 || q4; /* block-32 formats with scale planes */
+  const int a8 = W->expert_format == REF_FMT_MXFP4_A8;
+  const int mx = W->expert_format == REF_FMT_MXFP4 || q4 || a8; /* block-32 formats with scale planes */
   if (W->expert_format != REF_FMT_IQ2_Q2K && !mx) return REF_ERR_ARG;
   if (((int64_t)H * I) % QK || (mx && (H % 32 || I % 32))) return REF_ERR_SHAPE;
   if (T == 0) return REF_OK;
@@ -401,6 +476,7 @@ int moeref_expert_ffn(const moeref_desc* desc, const moeref_weights* W, const vo
     if (!hh || !xa) { free(hh); free(xa); free(mine); free(o); free(wg); free(wu); free(wd); return REF_ERR_NOMEM; }
     for (int64_t i = 0; i < na; ++i)
       for (int c = 0; c < H; ++c) xa[i * H + c] = act_in(x, x_dtype, (mine[i] / k) * H + c);
+    if (a8) mxfp8_round_trip(xa, na * H / 32); /* rows of H, blocks of 32 along H */
 #pragma omp parallel for collapse(2) schedule(static)
     for (int64_t i = 0; i < na; ++i)
       for (int r = 0; r < I; ++r) {
@@ -412,6 +488,7 @@ int moeref_expert_ffn(const moeref_desc* desc, const moeref_weights* W, const vo
         }
         hh[i * I + r] = silu(g) * u;
       }
+    if (a8) mxfp8_round_trip(hh, na * I / 32); /* rows of I, blocks of 32 along I */
 #pragma omp parallel for collapse(2) schedule(static)
     for (int64_t i = 0; i < na; ++i)
       for (int r = 0; r < H; ++r) {
