@@ -529,21 +529,28 @@ moe_status moe_layer_forward_cached(moe_expert_cache* cache, const moe_layer_wei
 
 // ------------------------------------------------------------ MXFP4 experts
 namespace {
-moe_status check_mx(const moe_layer_desc* desc, int32_t T) {
+// fmt 0 = MXFP4 (GEMVs up to 16 tokens, the block-scaled grouped GEMM above), 1 = Q4-style (up to 16 tokens)
+moe_status check_mx(const moe_layer_desc* desc, int32_t T, int fmt) {
   moe_status st = check_desc(desc);
   if (st != MOE_OK) return st;
   if ((st = check_tokens(desc, T)) != MOE_OK) return st;
-  if (T > 0 && !mx_path_supported(shape_of(desc), T)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const LayerShape sh = shape_of(desc);
+  const bool ok = T <= kPrefillMinT ? mx_path_supported(sh, T) : (fmt == 0 && mx_prefill_supported(sh, T));
+  if (T > 0 && !ok) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+moe_status blk32_workspace_size(const moe_layer_desc* desc, int32_t max_tokens, int fmt, size_t* bytes) {
+  moe_status st = check_mx(desc, max_tokens, fmt);
+  if (st != MOE_OK) return st;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = carve(desc, max_tokens, nullptr, mx_ffn_workspace_bytes(shape_of(desc), max_tokens)).bytes;
   return MOE_OK;
 }
 }  // namespace
 
 moe_status moe_workspace_size_mxfp4(const moe_layer_desc* desc, int32_t max_tokens, size_t* bytes) {
-  moe_status st = check_mx(desc, max_tokens);
-  if (st != MOE_OK) return st;
-  if (!bytes) return MOE_ERR_INVALID_ARG;
-  *bytes = carve(desc, max_tokens, nullptr, mx_ffn_workspace_bytes(shape_of(desc), max_tokens)).bytes;
-  return MOE_OK;
+  return blk32_workspace_size(desc, max_tokens, 0, bytes);
 }
 
 namespace {
@@ -552,7 +559,7 @@ namespace {
 moe_status blk32_forward(const moe_layer_desc* desc, const WeightPtrs& shw, const MxPlanes& mp, const void* x,
                          moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws, size_t ws_bytes,
                          void* stream) {
-  moe_status st = check_mx(desc, T);
+  moe_status st = check_mx(desc, T, mp.fmt);
   if (st != MOE_OK) return st;
   if (x_dtype != MOE_F32 && x_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
@@ -576,7 +583,7 @@ moe_status blk32_forward(const moe_layer_desc* desc, const WeightPtrs& shw, cons
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // as moe_layer_forward: the shared expert and the digits start first on the side stream (with this
   // path's workspace layout); every return after the fork joins it back
-  const bool early = shared_early_ok(sh, x_dtype, T);
+  const bool early = T <= kPrefillMinT && shared_early_ok(sh, x_dtype, T);
   int rc = OK;
   if (early) rc = launch_shared_early(sh, shw, x, T, w.ffn, s, mx_parts(sh.H), mx_parts(sh.I));
   if (rc == OK)
@@ -607,7 +614,7 @@ WeightPtrs blk32_shared(const uint16_t* router_w, const float* router_bias, cons
 moe_status moe_layer_forward_mxfp4(const moe_layer_desc* desc, const moe_mxfp4_weights* weights, const void* x,
                                    moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws,
                                    size_t ws_bytes, void* stream) {
-  if (!weights) return T == 0 && check_mx(desc, T) == MOE_OK ? MOE_OK : MOE_ERR_INVALID_ARG;
+  if (!weights) return T == 0 && check_mx(desc, T, 0) == MOE_OK ? MOE_OK : MOE_ERR_INVALID_ARG;
   const MxPlanes mp{0, weights->gate_codes, weights->gate_scales, weights->up_codes,
                     weights->up_scales, weights->down_codes, weights->down_scales};
   return blk32_forward(desc,
@@ -617,13 +624,13 @@ moe_status moe_layer_forward_mxfp4(const moe_layer_desc* desc, const moe_mxfp4_w
 }
 
 moe_status moe_workspace_size_q4(const moe_layer_desc* desc, int32_t max_tokens, size_t* bytes) {
-  return moe_workspace_size_mxfp4(desc, max_tokens, bytes);
+  return blk32_workspace_size(desc, max_tokens, 1, bytes);
 }
 
 moe_status moe_layer_forward_q4(const moe_layer_desc* desc, const moe_q4_weights* weights, const void* x,
                                 moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws,
                                 size_t ws_bytes, void* stream) {
-  if (!weights) return T == 0 && check_mx(desc, T) == MOE_OK ? MOE_OK : MOE_ERR_INVALID_ARG;
+  if (!weights) return T == 0 && check_mx(desc, T, 1) == MOE_OK ? MOE_OK : MOE_ERR_INVALID_ARG;
   const MxPlanes mp{1, weights->gate_codes, weights->gate_d, weights->up_codes,
                     weights->up_d, weights->down_codes, weights->down_d};
   return blk32_forward(desc,

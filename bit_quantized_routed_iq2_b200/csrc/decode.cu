@@ -749,12 +749,18 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
 // down in 256-element parts of their reduction axes, h re-quantised as
 // activation digits.
 size_t mx_ffn_workspace_bytes(const LayerShape& s, int T) {
-  return carve_fast(s, T, mx_parts(s.H), mx_parts(s.I), nullptr).bytes;
+  // one workspace serves every T up to the given one: the GEMV step up to 16 tokens, the grouped GEMM above
+  const size_t dec = carve_fast(s, std::min(T, kPrefillMinT), mx_parts(s.H), mx_parts(s.I), nullptr).bytes;
+  return T > kPrefillMinT && mx_prefill_supported(s, T) ? std::max(dec, mx_prefill_workspace_bytes(s, T)) : dec;
 }
 
 int launch_ffn_mxfp4(const LayerShape& s, const WeightPtrs& shw, const MxPlanes& w, const void* x, int x_dtype,
                      int T, const Routing& r, const float* residual, float* y, void* ws, int* err, bool clear_status,
                      cudaStream_t st, bool shared_early) {
+  if (T > kPrefillMinT) {  // many tokens: the block-scaled grouped GEMM (MXFP4 only)
+    if (shared_early) return ERR_ARG;
+    return launch_ffn_mx_prefill(s, shw, w, x, x_dtype, T, r, residual, y, ws, err, clear_status, num_sms(), st);
+  }
   const int nA = T * s.k;
   const int KP = mx_parts(s.H), DP = mx_parts(s.I);
   const FastWs fw = carve_fast(s, T, KP, DP, static_cast<char*>(ws));

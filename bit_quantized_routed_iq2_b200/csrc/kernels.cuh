@@ -128,6 +128,20 @@ int launch_ffn_prefill(const LayerShape& s, const WeightPtrs& w, const void* x, 
                        const float* residual, float* y, void* ws, int* err, bool clear_status, int sms,
                        cudaStream_t st);
 
+// The shared expert alone on the tensor-core GEMM (prefill.cu): s_out = fp32 [T][H].
+size_t prefill_shared_workspace_bytes(const LayerShape& s, int T);
+int launch_prefill_shared(const LayerShape& s, const uint16_t* wg, const uint16_t* wu, const uint16_t* wd,
+                          const void* x, int x_dtype, int T, void* ws, float* s_out, int* err, int sms,
+                          cudaStream_t st);
+
+// MXFP4 routed experts for more than 16 tokens (mx_gemm.cu): a grouped GEMM on the block-scaled
+// tensor cores, FP4 weights x MXFP8 activations.
+bool mx_prefill_supported(const LayerShape& s, int T);
+size_t mx_prefill_workspace_bytes(const LayerShape& s, int T);
+int launch_ffn_mx_prefill(const LayerShape& s, const WeightPtrs& shw, const MxPlanes& w, const void* x, int x_dtype,
+                          int T, const Routing& r, const float* residual, float* y, void* ws, int* err,
+                          bool clear_status, int sms, cudaStream_t st);
+
 // Copies the device status word at `word` to *out after the work enqueued on `st` (synchronises `st`).
 int read_status_word(const int* word, int32_t* out, cudaStream_t st);
 

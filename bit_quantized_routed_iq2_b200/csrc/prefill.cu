@@ -1099,6 +1099,53 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
 }
 
+// The shared expert alone on the tensor-core GEMM for T tokens: s = Wsd (silu(Wsg x) * (Wsu x)), fp32 [T][H].
+// Workspace: bf16 parts of x (fp32 inputs) and of h.
+size_t prefill_shared_workspace_bytes(const LayerShape& sh, int T) {
+  return align_up(static_cast<size_t>(T) * sh.H * 2 * 2, 1024) +
+         align_up(static_cast<size_t>(T) * (sh.Is > 0 ? sh.Is : 1) * 2 * 2, 1024);
+}
+
+int launch_prefill_shared(const LayerShape& sh, const uint16_t* wg, const uint16_t* wu, const uint16_t* wd,
+                          const void* x, int x_dtype, int T, void* ws, float* s_out, int* err, int sms,
+                          cudaStream_t st) {
+  __nv_bfloat16* xb = static_cast<__nv_bfloat16*>(ws);
+  __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) +
+                                                       align_up(static_cast<size_t>(T) * sh.H * 2 * 2, 1024));
+  int rc = OK;
+  if (x_dtype == 0) {
+    ProfScope ps(MOE_K_PREP, st);
+    bf16_parts_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const float*>(x), static_cast<size_t>(T) * sh.H, xb);
+  }
+  CUtensorMap mb, ma0, ma1;
+  {
+    ProfScope ps(MOE_K_SHARED_GATEUP, st);
+    const int planes = x_dtype == 0 ? 2 : 1;
+    const void* xsrc = x_dtype == 0 ? static_cast<const void*>(xb) : x;
+    if (!tc_map(&mb, xsrc, true, sh.H, T, planes) || !tc_map(&ma0, wg, true, sh.H, sh.Is, 1) ||
+        !tc_map(&ma1, wu, true, sh.H, sh.Is, 1))
+      return ERR_CUDA;
+    TcArgs a{};
+    a.n_experts = 1; a.b_rows = T;
+    a.rows_e = sh.Is; a.K = sh.H; a.mt = sh.Is / kMT; a.planes = planes;
+    a.dense_rows = T; a.out = hs; a.ldo = sh.Is; a.out_rows = T;
+    a.oscale = 1.0f; a.err = err;
+    rc |= launch_tc<TC_BF16_PAIR>(mb, ma0, ma1, a, sms, st);
+  }
+  {
+    ProfScope ps(MOE_K_SHARED_DOWN, st);
+    if (!tc_map(&mb, hs, true, sh.Is, T, 2) || !tc_map(&ma0, wd, true, sh.Is, sh.H, 1)) return ERR_CUDA;
+    TcArgs a{};
+    a.n_experts = 1; a.b_rows = T;
+    a.rows_e = sh.H; a.K = sh.Is; a.mt = sh.H / kMT; a.planes = 2;
+    a.dense_rows = T; a.out = s_out; a.ldo = sh.H; a.out_rows = T;
+    a.oscale = 1.0f; a.err = err;
+    rc |= launch_tc<TC_BF16>(mb, ma0, ma0, a, sms, st);
+  }
+  if (rc != OK) return ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
+}
+
 }  // namespace moe
 
 namespace moe {

@@ -70,6 +70,46 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// Instruction descriptor for kind::mxf8f6f4 with block scaling: A FP4 E2M1,
+// B FP8 E4M3, both K-major, E8M0 scale factors, fp32 accumulator, M x N,
+// K = 32 per instruction. The scale-factor byte ids (which byte of the 32-bit
+// TMEM words holds this instruction's scales) are set per instruction.
+__host__ __device__ constexpr uint32_t umma_idesc_mx_e2m1_e4m3(int M, int N) {
+  return (5u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t umma_idesc_sf_ids(uint32_t idesc, uint32_t a_id, uint32_t b_id) {
+  return (idesc & ~((3u << 29) | (3u << 4))) | (a_id << 29) | (b_id << 4);
+}
+
+// D[tmem] (+)= (A[smem] * 2^SFA) * (B[smem] * 2^SFB)^T per 32-element block of
+// K, issued by one thread; sfa / sfb are the TMEM addresses of the scale
+// factors (byte id in bits 31..30).
+__device__ __forceinline__ void umma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Shared-memory descriptor of 32 rows of 16 bytes stored one after another
+// (no swizzle, 8-row groups 128 bytes apart): the source of a 32x128b copy.
+__device__ __forceinline__ uint64_t umma_desc_rows16(uint32_t saddr) {
+  uint64_t d = static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// Copy 32 rows x 128 bits from shared memory into TMEM lanes 0..31 (row i to
+// lane i, four 32-bit columns from `taddr`), repeated in the lanes of all four
+// warp quarters; ordered before later tcgen05 operations of the same thread.
+__device__ __forceinline__ void tmem_cp_32x128_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrive once on `bar` when all MMAs issued so far by this thread have completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))

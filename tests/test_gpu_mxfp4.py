@@ -5,7 +5,9 @@ Element decoding bit-for-bit (as values) through moe_debug_dequant_mxfp4; the
 layer within the normwise bound of the 2-bit path (FFN_TOL) at small shapes
 (one and several tokens, fp32 and bf16 activations, with and without a shared
 expert, uneven routing) and at the one-token decode shape (H=7168, I=2048,
-E=256, k=8, I_s=2048).
+E=256, k=8, I_s=2048). Above 16 tokens (the block-scaled grouped GEMM) against
+the oracle with MXFP8 activations, at small shapes with ragged and multi-tile
+experts and on sampled tokens of the 2048-token prefill shape.
 """
 import numpy as np
 import pytest
@@ -13,7 +15,7 @@ import pytest
 import oracle
 import synth
 from bit_quantized_routed_iq2_b200 import moe2bit
-from helpers import FFN_TOL, normwise, screened_x
+from helpers import FFN_TOL, near_tie_tokens, normwise, screened_x
 
 pytestmark = pytest.mark.gpu
 
@@ -82,13 +84,64 @@ def test_mxfp4_layer_small(torch_cuda, name):
 
 
 def test_mxfp4_rejects_unsupported_shapes(torch_cuda):
+    import ctypes
+
     desc = moe2bit.desc_of(1280, 512, 16, 4, 0)  # hidden not a multiple of 512
     with pytest.raises(RuntimeError):
         moe2bit.workspace_size_mxfp4(desc, 1)
     desc = moe2bit.desc_of(1024, 512, 16, 4, 0)
-    with pytest.raises(RuntimeError):
-        moe2bit.workspace_size_mxfp4(desc, 17)  # decode only
     assert moe2bit.workspace_size_mxfp4(desc, 16) > 0
+    # above 16 tokens MXFP4 takes the block-scaled grouped GEMM; its workspace covers the GEMV step too
+    assert moe2bit.workspace_size_mxfp4(desc, 300) >= moe2bit.workspace_size_mxfp4(desc, 16)
+    # the Q4-style format has no many-token path
+    n = ctypes.c_size_t(0)
+    assert moe2bit.load().moe_workspace_size_q4(ctypes.byref(desc), 17, ctypes.byref(n)) != 0
+    assert moe2bit.load().moe_workspace_size_q4(ctypes.byref(desc), 16, ctypes.byref(n)) == 0
+
+
+# More than 16 tokens: FP4 weights x MXFP8 activations on the block-scaled tensor cores; the oracle takes
+# the same activation quantisation (act_mxfp8). Tiles hold up to 112 tokens of one expert.
+MANY = {
+    "t17_bf16": dict(T=17, x_dtype="bf16", Is=128, zipf=False, E=16, k=4),
+    "t40_bf16_zipf": dict(T=40, x_dtype="bf16", Is=128, zipf=True, E=16, k=4),
+    "t200_f32_zipf_noshared": dict(T=200, x_dtype="f32", Is=0, zipf=True, E=8, k=2),
+    "t300_bf16": dict(T=300, x_dtype="bf16", Is=256, zipf=False, E=4, k=2),
+}
+
+
+@pytest.mark.parametrize("name", list(MANY))
+def test_mxfp4_layer_many_tokens(torch_cuda, name):
+    c = MANY[name]
+    cfg = synth.Config("mxg_" + name, c["T"], 1024, 512, c["E"], c["k"], c["Is"], c["x_dtype"], 1.0, c["zipf"], 1,
+                       0x4D47A0 + len(name))
+    lw = synth.make_layer_mxfp4(cfg)
+    x = screened_x(cfg, lw)
+    res = synth.make_residual(cfg, cfg.T)
+    y = _mx_forward(torch_cuda, moe2bit.to_device_mxfp4(lw), x, res)
+    ref, idx, _ = oracle.layer_forward(lw, x, res, act_mxfp8=True)
+    if name.startswith("t300") or name.startswith("t200"):  # an expert spans several tiles (ragged last one)
+        assert np.bincount(idx.reshape(-1), minlength=cfg.E).max() > 112
+    assert normwise(y, ref) <= FFN_TOL, (name, normwise(y, ref))
+    # against the exact-activation oracle the FP8 rounding of x and h shows (a few 1e-2 normwise at most)
+    exact, _, _ = oracle.layer_forward(lw, x, res)
+    assert normwise(y, exact) < 0.1
+
+
+@pytest.mark.slow
+def test_mxfp4_prefill_shape_sampled(torch_cuda):
+    """H=7168, I=2048, E=256, k=8, I_s=2048, 2048 bf16 tokens (every expert active): the GPU runs the whole
+    batch in the launch configuration the benchmark times; the oracle checks a sample of tokens (a token's
+    output depends on that token alone)."""
+    cfg = synth.CONFIGS["prefill"]
+    lw = synth.make_layer_mxfp4(cfg)
+    x = synth.make_x_fast(cfg, cfg.T)
+    y = _mx_forward(torch_cuda, moe2bit.to_device_mxfp4(lw), x)
+    cand = np.array([0, 1, 2, 3, 777, 778, 1500, 1501, cfg.T - 2, cfg.T - 1])
+    _, _, logits = oracle.route(lw.router_w, lw.router_bias, x[cand], cfg.k, want_logits=True)
+    rows = np.setdiff1d(cand, cand[near_tie_tokens(logits, cfg.k)])[:5]  # routing decided in any precision
+    assert rows.size == 5
+    ref, _, _ = oracle.layer_forward(lw, x[rows], act_mxfp8=True)
+    assert normwise(y[rows], ref) <= FFN_TOL, normwise(y[rows], ref)
 
 
 @pytest.mark.slow
