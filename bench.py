@@ -54,7 +54,8 @@ def parse():
                     help="override the tokens per step (small cases for profiling; not a bench workload)")
     ap.add_argument("--workloads", default="auto",
                     help="other workloads measured in the same run and reported under 'workloads': 'all' "
-                         "(decode32, prefill, stack, decode1_cached, quantize), 'none', or a comma list; "
+                         "(decode32, prefill, stack, decode1_mxfp4, decode1_q4, prefill_mxfp4, decode1_cached, "
+                         "quantize), 'none', or a comma list; "
                          "'auto' = all on one GPU")
     ap.add_argument("--workload-steps", type=int, default=20, help="timed steps of each extra workload")
     return ap.parse_args()
@@ -631,6 +632,70 @@ def measure_mxfp4(args, steps, fmt="mxfp4"):
     }
 
 
+def measure_mxfp4_prefill(args, steps):
+    """2048 bf16 tokens with MXFP4 routed experts (the prefill shapes H=7168, I=2048, E=256, k=8,
+    I_s=2048; every expert active): FP4 weights x MXFP8 activations on the block-scaled tensor cores
+    (moe_layer_forward_mxfp4 above 16 tokens). One resident layer of 6 GB (weights larger than L2).
+    Roofline of the gate/up grouped GEMM against HBM: every active expert's gate and up codes and
+    scales, the MXFP8 activations it reads and the MXFP8 h it writes; the tensor-pipe fraction (FP8 x FP4
+    flops over twice the bf16 peak, the nominal fp8 : bf16 ratio) beside it."""
+    import torch
+
+    from bit_quantized_routed_iq2_b200 import moe2bit
+
+    cfg = synth.Config("prefill_mxfp4", 2048, 7168, 2048, 256, 8, 2048, "bf16", math.sqrt(0.5), False, 1,
+                       0xD540000A)
+    lw = synth.make_layer_mxfp4(cfg)
+    dl = moe2bit.to_device_mxfp4(lw)
+    del lw
+    x = torch.from_numpy(synth.make_x_fast(cfg, cfg.T).view(np.int16)).cuda().view(torch.bfloat16)
+    y = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
+    ws = moe2bit.alloc_workspace_mxfp4(dl.desc, cfg.T)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(args.warmup, 3)):
+        moe2bit.layer_forward_mxfp4(dl, x, None, y, ws, stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        moe2bit.layer_forward_mxfp4(dl, x, None, y, ws, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    moe2bit.profile_enable(True)
+    for _ in range(steps):
+        moe2bit.layer_forward_mxfp4(dl, x, None, y, ws, stream)
+    torch.cuda.synchronize()
+    prof = moe2bit.profile_read()
+    moe2bit.profile_enable(False)
+    assert moe2bit.read_status(ws) == 0
+    del dl, ws, x, y
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    hbm, bf16_tf, peak_kind = peaks()
+    avg_ms = {k: v[0] / max(v[1], 1) for k, v in prof.items()}
+    nA = cfg.T * cfg.k
+    alg = (cfg.E * 2 * cfg.I * cfg.H * (0.5 + 1 / 32) + nA * cfg.H * (1 + 1 / 32) + nA * cfg.I * (1 + 1 / 32))
+    achieved = alg / (avg_ms["prefill_gateup"] * 1e-3) / 1e9
+    dn_alg = cfg.E * cfg.H * cfg.I * (0.5 + 1 / 32) + nA * cfg.I * (1 + 1 / 32) + nA * cfg.H * 4
+    flops = 2.0 * nA * 2 * cfg.I * cfg.H
+    fp8_tf = 2.0 * bf16_tf
+    return {
+        "value": cfg.T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+        "config": {"workload": cfg.name, "tokens_per_step": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
+                   "I_s": cfg.Is, "experts": "MXFP4 (OCP MX: E2M1 x 32 + E8M0), all three routed matrices",
+                   "activations": "routed: MXFP8 (E4M3 x 32 + E8M0); shared expert: bf16",
+                   "l2": "inputs larger than L2: one resident layer of 6 GB", "launch": "stream"},
+        "kernels": {k: {"avg_ms": v, "launches_per_step": prof[k][1] / steps} for k, v in avg_ms.items()},
+        "roofline": {"bound": "hbm", "kernel": "prefill_gateup", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg,
+                     "avg_launch_ms": avg_ms["prefill_gateup"],
+                     "tensor_frac": flops / (avg_ms["prefill_gateup"] * 1e-3) / 1e12 / fp8_tf,
+                     "tensor_peak_tflops": fp8_tf,
+                     "down_frac": dn_alg / (avg_ms["prefill_down"] * 1e-3) / 1e9 / hbm},
+    }
+
+
 def measure_quantize(args, reps=3):
     """Float -> 2-bit codes for one expert (gate and up to IQ2, down to Q2K,
     2048 x 7168 weights each): weights per second. The IQ2 search is bound by
@@ -711,7 +776,8 @@ def run_ours(args, cfg):
         want = "all" if (world == 1 and not args.experts and not args.tokens) else "none"
     if want != "none":
         names = ([n for n in ("decode32", "prefill", "stack") if n != cfg.name] +
-                 ["decode1_mxfp4", "decode1_q4", "decode1_cached", "quantize"] if want == "all" else want.split(","))
+                 ["decode1_mxfp4", "decode1_q4", "prefill_mxfp4", "decode1_cached", "quantize"] if want == "all"
+                 else want.split(","))
         line["workloads"] = {}
         for name in names:
             if name == "decode1_cached":
@@ -720,6 +786,8 @@ def run_ours(args, cfg):
                 w = measure_quantize(args)
             elif name in ("decode1_mxfp4", "decode1_q4"):
                 w = measure_mxfp4(args, args.workload_steps, name.split("_")[1])
+            elif name == "prefill_mxfp4":
+                w = measure_mxfp4_prefill(args, max(3, args.workload_steps // 4))
             else:
                 w = measure(args, synth.CONFIGS[name], world, rank, local, args.workload_steps)
                 line["gpu_launches"] += w["gpu_launches"]
