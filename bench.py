@@ -58,6 +58,8 @@ def parse():
                          "quantize), 'none', or a comma list; "
                          "'auto' = all on one GPU")
     ap.add_argument("--workload-steps", type=int, default=20, help="timed steps of each extra workload")
+    ap.add_argument("--workloads-only", action="store_true",
+                    help="profiling aid: skip the main configuration and print only the 'workloads' object")
     return ap.parse_args()
 
 
@@ -643,8 +645,9 @@ def measure_mxfp4_prefill(args, steps):
 
     from bit_quantized_routed_iq2_b200 import moe2bit
 
-    cfg = synth.Config("prefill_mxfp4", 2048, 7168, 2048, 256, 8, 2048, "bf16", math.sqrt(0.5), False, 1,
-                       0xD540000A)
+    E = args.experts or 256
+    cfg = synth.Config("prefill_mxfp4" if E == 256 else f"prefill_mxfp4_E{E}", 2048 * E // 256, 7168, 2048, E, 8,
+                       2048, "bf16", math.sqrt(0.5), False, 1, 0xD540000A)
     lw = synth.make_layer_mxfp4(cfg)
     dl = moe2bit.to_device_mxfp4(lw)
     del lw
@@ -760,7 +763,12 @@ def run_ours(args, cfg):
     moebuild.build()
     moe2bit.load()
 
-    m = measure(args, cfg, world, rank, local, args.steps)
+    if args.workloads_only:  # profiling aid: the listed workloads alone, no main line
+        assert world == 1 and args.workloads not in ("auto", "all", "none")
+        m = {"value": None, "ms_per_step": None, "dtype": None, "gpu_launches": 0,
+             **{k: None for k in ("config", "roofline", "step_hbm", "kernels", "clocks", "e2e")}}
+    else:
+        m = measure(args, cfg, world, rank, local, args.steps)
     line = {
         "metric": "moe_layer_tokens_per_s", "value": m["value"], "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": m["ms_per_step"],

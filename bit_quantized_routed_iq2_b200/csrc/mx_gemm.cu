@@ -231,42 +231,63 @@ __global__ void __launch_bounds__(kMgThreads, 1) mx_gemm_kernel(const __grid_con
     }
   } else if (warp == kMgSfWarp) {
     // per 512 elements of K, 16 scale bytes of each row: rows r0 + 32 r1 of the weight tile (and of the
-    // token tile) for this lane r0, then per stage q of the four the 32-bit word q of each
+    // token tile) for this lane r0, then per stage q of the four the 32-bit word q of each. The next
+    // 512 elements' bytes (of this tile or of the CTA's next one) are loaded before this one's are written.
     const size_t ldk = static_cast<size_t>(a.K / 32);
     const int nsup = a.K / (4 * kMgKS);
+    auto next_unit = [&](int uu) {
+      while (uu < nunits && mg_tile(a, uu / a.mt).n == 0) uu += gridDim.x;
+      return uu;
+    };
+    auto load_sup = [&](int uu, int j, uint4 (&ga)[4], uint4 (&ua)[4], uint4 (&gb)[4]) {
+      const MgTile t = a.tiles[uu / a.mt];  // validated by next_unit
+      const size_t wrow = static_cast<size_t>(t.e) * a.rows_e + (uu % a.mt) * kMgMT + lane;
+#pragma unroll
+      for (int r1 = 0; r1 < 4; ++r1) {
+        ga[r1] = __ldg(reinterpret_cast<const uint4*>(a.sa0 + (wrow + 32 * r1) * ldk) + j);
+        if (PAIR) ua[r1] = __ldg(reinterpret_cast<const uint4*>(a.sa1 + (wrow + 32 * r1) * ldk) + j);
+        const int brow = min(t.p0 + lane + 32 * r1, a.b_rows - 1);  // rows past the tile: any valid row
+        gb[r1] = __ldg(reinterpret_cast<const uint4*>(a.sb + static_cast<size_t>(brow) * ldk) + j);
+      }
+    };
     int s = 0;
     uint32_t ph = 0;
+    int u = next_unit(blockIdx.x), j = 0;
+    uint4 ga[4], ua[4], gb[4];
+    if (u < nunits) load_sup(u, 0, ga, ua, gb);
     bool ok = true;
-    for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
-      const MgTile t = mg_tile(a, u / a.mt);
-      if (t.n == 0) continue;
-      const size_t wrow = static_cast<size_t>(t.e) * a.rows_e + (u % a.mt) * kMgMT + lane;
-      for (int j = 0; j < nsup && ok; ++j) {
-        uint4 ga[4], ua[4], gb[4];
-#pragma unroll
-        for (int r1 = 0; r1 < 4; ++r1) {
-          ga[r1] = __ldg(reinterpret_cast<const uint4*>(a.sa0 + (wrow + 32 * r1) * ldk) + j);
-          if (PAIR) ua[r1] = __ldg(reinterpret_cast<const uint4*>(a.sa1 + (wrow + 32 * r1) * ldk) + j);
-          const int brow = min(t.p0 + lane + 32 * r1, a.b_rows - 1);  // rows past the tile: any valid row
-          gb[r1] = __ldg(reinterpret_cast<const uint4*>(a.sb + static_cast<size_t>(brow) * ldk) + j);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (!mg_wait_warp(&emptyB[s], ph ^ 1u, a.err, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const uint32_t ch = sbase + L::sf_off + s * L::sf_slot + 16 * lane;
-          sts128(ch, word_of(ga[0], q), word_of(ga[1], q), word_of(ga[2], q), word_of(ga[3], q));
-          if (PAIR) sts128(ch + 512, word_of(ua[0], q), word_of(ua[1], q), word_of(ua[2], q), word_of(ua[3], q));
-          sts128(ch + (PAIR ? 1024 : 512), word_of(gb[0], q), word_of(gb[1], q), word_of(gb[2], q),
-                 word_of(gb[3], q));
-          fence_proxy_async_smem();  // the chunks are read by the tensor core's copy
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sfF[s]);
-          if (++s == kStages) { s = 0; ph ^= 1u; }
-        }
+    while (u < nunits && ok) {
+      int un = u, jn = j + 1;
+      if (jn == nsup) {
+        jn = 0;
+        un = next_unit(u + gridDim.x);
       }
+      uint4 na[4], nu[4], nb[4];
+      if (un < nunits) load_sup(un, jn, na, nu, nb);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (!mg_wait_warp(&emptyB[s], ph ^ 1u, a.err, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint32_t ch = sbase + L::sf_off + s * L::sf_slot + 16 * lane;
+        sts128(ch, word_of(ga[0], q), word_of(ga[1], q), word_of(ga[2], q), word_of(ga[3], q));
+        if (PAIR) sts128(ch + 512, word_of(ua[0], q), word_of(ua[1], q), word_of(ua[2], q), word_of(ua[3], q));
+        sts128(ch + (PAIR ? 1024 : 512), word_of(gb[0], q), word_of(gb[1], q), word_of(gb[2], q),
+               word_of(gb[3], q));
+        fence_proxy_async_smem();  // the chunks are read by the tensor core's copy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sfF[s]);
+        if (++s == kStages) { s = 0; ph ^= 1u; }
+      }
+#pragma unroll
+      for (int r1 = 0; r1 < 4; ++r1) {
+        ga[r1] = na[r1];
+        if (PAIR) ua[r1] = nu[r1];
+        gb[r1] = nb[r1];
+      }
+      u = un;
+      j = jn;
     }
   } else if (warp == kMgMmaWarp) {
     // the whole warp runs the loop (waits stay warp-uniform); one elected lane copies and issues
