@@ -693,6 +693,7 @@ def measure_mxfp4_prefill(args, steps):
         "roofline": {"bound": "hbm", "kernel": "prefill_gateup", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg,
                      "avg_launch_ms": avg_ms["prefill_gateup"],
+                     "traffic": (traffic_record(cfg.name, "prefill_gateup") or {}).get("bytes_per_launch"),
                      "tensor_frac": flops / (avg_ms["prefill_gateup"] * 1e-3) / 1e12 / fp8_tf,
                      "tensor_peak_tflops": fp8_tf,
                      "down_frac": dn_alg / (avg_ms["prefill_down"] * 1e-3) / 1e9 / hbm},

@@ -1,6 +1,7 @@
 // api.cu - the C ABI declared in include/moe2bit.h: argument validation,
 // workspace carving and the launch sequence of each entry point.
 #include <cstring>
+#include <initializer_list>
 #include <vector>
 
 #include "../../include/moe2bit.h"
@@ -567,6 +568,10 @@ moe_status blk32_forward(const moe_layer_desc* desc, const WeightPtrs& shw, cons
                           mp.up_scales, mp.down_codes, mp.down_scales};
   for (const void* p : planes)
     if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (T > kPrefillMinT)  // the grouped GEMM's unpacking copy of the FP4 codes needs 32-byte bases
+    for (const void* p : {static_cast<const void*>(mp.gate_codes), static_cast<const void*>(mp.up_codes),
+                          static_cast<const void*>(mp.down_codes)})
+      if (reinterpret_cast<uintptr_t>(p) % 32 != 0) return MOE_ERR_INVALID_ARG;
   if (shw.router_bias && !aligned16(shw.router_bias)) return MOE_ERR_INVALID_ARG;
   if (desc->shared_inter > 0) {
     const void* sh[] = {shw.sh_gate, shw.sh_up, shw.sh_down};

@@ -469,19 +469,30 @@ typedef struct {
  * The layer forward of moe_layer_forward with MXFP4 routed experts: the same
  * routing, shared expert, combine, residual and output, with the gate, up and
  * down projections of each assignment taken over the decoded MXFP4 weights.
- * Decode only: 1 <= T <= 16 tokens (T == 0 enqueues nothing). Shapes, in
- * addition to those of the common conventions: hidden % 512 == 0,
- * inter % 512 == 0, n_experts <= 1024; otherwise MOE_ERR_UNSUPPORTED_SHAPE.
- * Every pointer of `w` (the shared-expert ones when I_s > 0) is a 16-byte
- * aligned device pointer, else MOE_ERR_INVALID_ARG. Workspace: ws_bytes >=
- * moe_workspace_size_mxfp4(desc, T) (its gate/up partial sums are finer than
- * those of moe_layer_forward), else MOE_ERR_WORKSPACE_TOO_SMALL. Stream, side
- * stream, status word (moe_read_status) and errors as moe_layer_forward.
- * Numerics: activations enter the integer products as two signed digits of a
- * 14-bit fixed-point code per 256-element block (as in moe_layer_forward's
- * decode path), the decoded elements times 2 are exact int8 values, every block
- * of 32 is scaled exactly by its power of two; accumulation in fp32 per block
- * and across blocks.
+ * T == 0 enqueues nothing. Shapes, in addition to those of the common
+ * conventions: hidden % 512 == 0, inter % 512 == 0; for 1 <= T <= 16 also
+ * n_experts <= 1024; above 16 tokens I_s % 128 == 0 (or I_s == 0); otherwise
+ * MOE_ERR_UNSUPPORTED_SHAPE. Every pointer of `w` (the shared-expert ones when
+ * I_s > 0) is a 16-byte aligned device pointer, else MOE_ERR_INVALID_ARG; above
+ * 16 tokens the three code planes are 32-byte aligned (the copy that unpacks
+ * them requires it), else MOE_ERR_INVALID_ARG. Workspace:
+ * ws_bytes >= moe_workspace_size_mxfp4(desc, T), else
+ * MOE_ERR_WORKSPACE_TOO_SMALL. Stream, side stream, status word
+ * (moe_read_status) and errors as moe_layer_forward.
+ * Numerics, 1 <= T <= 16 (dequant-GEMVs): activations enter the integer
+ * products as two signed digits of a 14-bit fixed-point code per 256-element
+ * block (as in moe_layer_forward's decode path), the decoded elements times 2
+ * are exact int8 values, every block of 32 is scaled exactly by its power of
+ * two; accumulation in fp32 per block and across blocks.
+ * Numerics, T > 16 (grouped GEMM on the block-scaled tensor cores, FP4 x FP8):
+ * the routed experts' activations x, and h = silu(g) * u, are quantised to
+ * MXFP8 before their contraction: per block of 32 consecutive elements along
+ * the reduction axis the E8M0 exponent X = floor(log2 max|v|) - 8 (clamped to
+ * [-127, 127], -127 for a zero block) and elements v / 2^X rounded to FP8 E4M3
+ * (nearest even, saturating at 448). Products of the FP4 and FP8 elements and
+ * both block scales are exact; accumulation is fp32 in the tensor core. The
+ * shared expert runs in bf16 (two bf16 parts for fp32 activations) as in
+ * moe_layer_forward's many-token path.
  */
 MOE_API moe_status moe_workspace_size_mxfp4(const moe_layer_desc* desc, int32_t max_tokens, size_t* bytes);
 MOE_API moe_status moe_layer_forward_mxfp4(const moe_layer_desc* desc, const moe_mxfp4_weights* w, const void* x,
