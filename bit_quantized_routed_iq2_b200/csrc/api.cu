@@ -530,13 +530,15 @@ moe_status moe_layer_forward_cached(moe_expert_cache* cache, const moe_layer_wei
 
 // ------------------------------------------------------------ MXFP4 experts
 namespace {
-// fmt 0 = MXFP4 (GEMVs up to 16 tokens, the block-scaled grouped GEMM above), 1 = Q4-style (up to 16 tokens)
+// fmt 0 = MXFP4 (GEMVs up to 16 tokens, the block-scaled grouped GEMM above), 1 = Q4-style (GEMVs up to 16
+// tokens, the dequantising grouped GEMM above)
 moe_status check_mx(const moe_layer_desc* desc, int32_t T, int fmt) {
   moe_status st = check_desc(desc);
   if (st != MOE_OK) return st;
   if ((st = check_tokens(desc, T)) != MOE_OK) return st;
   const LayerShape sh = shape_of(desc);
-  const bool ok = T <= kPrefillMinT ? mx_path_supported(sh, T) : (fmt == 0 && mx_prefill_supported(sh, T));
+  const bool ok = T <= kPrefillMinT ? mx_path_supported(sh, T)
+                                     : (fmt == 0 ? mx_prefill_supported(sh, T) : prefill_path_supported(sh, T));
   if (T > 0 && !ok) return MOE_ERR_UNSUPPORTED_SHAPE;
   return MOE_OK;
 }
@@ -545,7 +547,7 @@ moe_status blk32_workspace_size(const moe_layer_desc* desc, int32_t max_tokens, 
   moe_status st = check_mx(desc, max_tokens, fmt);
   if (st != MOE_OK) return st;
   if (!bytes) return MOE_ERR_INVALID_ARG;
-  *bytes = carve(desc, max_tokens, nullptr, mx_ffn_workspace_bytes(shape_of(desc), max_tokens)).bytes;
+  *bytes = carve(desc, max_tokens, nullptr, mx_ffn_workspace_bytes(shape_of(desc), max_tokens, fmt)).bytes;
   return MOE_OK;
 }
 }  // namespace
@@ -568,7 +570,7 @@ moe_status blk32_forward(const moe_layer_desc* desc, const WeightPtrs& shw, cons
                           mp.up_scales, mp.down_codes, mp.down_scales};
   for (const void* p : planes)
     if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
-  if (T > kPrefillMinT)  // the grouped GEMM's unpacking copy of the FP4 codes needs 32-byte bases
+  if (T > kPrefillMinT && mp.fmt == 0)  // the block-scaled GEMM's unpacking copy of the FP4 codes needs 32-byte bases
     for (const void* p : {static_cast<const void*>(mp.gate_codes), static_cast<const void*>(mp.up_codes),
                           static_cast<const void*>(mp.down_codes)})
       if (reinterpret_cast<uintptr_t>(p) % 32 != 0) return MOE_ERR_INVALID_ARG;
@@ -583,7 +585,7 @@ moe_status blk32_forward(const moe_layer_desc* desc, const WeightPtrs& shw, cons
     if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
   if (residual && !aligned16(residual)) return MOE_ERR_INVALID_ARG;
   const LayerShape sh = shape_of(desc);
-  RouteWs w = carve(desc, T, ws, mx_ffn_workspace_bytes(sh, T));
+  RouteWs w = carve(desc, T, ws, mx_ffn_workspace_bytes(sh, T, mp.fmt));
   if (ws_bytes < w.bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // as moe_layer_forward: the shared expert and the digits start first on the side stream (with this

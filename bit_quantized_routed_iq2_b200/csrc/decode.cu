@@ -748,18 +748,22 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
 // combine) with the block-32 GEMVs of mxfp4.cu (MXFP4 or Q4-style): gate/up and
 // down in 256-element parts of their reduction axes, h re-quantised as
 // activation digits.
-size_t mx_ffn_workspace_bytes(const LayerShape& s, int T) {
+size_t mx_ffn_workspace_bytes(const LayerShape& s, int T, int fmt) {
   // one workspace serves every T up to the given one: the GEMV step up to 16 tokens, the grouped GEMM above
   const size_t dec = carve_fast(s, std::min(T, kPrefillMinT), mx_parts(s.H), mx_parts(s.I), nullptr).bytes;
-  return T > kPrefillMinT && mx_prefill_supported(s, T) ? std::max(dec, mx_prefill_workspace_bytes(s, T)) : dec;
+  if (T <= kPrefillMinT) return dec;
+  if (fmt == 0) return mx_prefill_supported(s, T) ? std::max(dec, mx_prefill_workspace_bytes(s, T)) : dec;
+  return prefill_path_supported(s, T) ? std::max(dec, prefill_workspace_bytes(s, T)) : dec;
 }
 
 int launch_ffn_mxfp4(const LayerShape& s, const WeightPtrs& shw, const MxPlanes& w, const void* x, int x_dtype,
                      int T, const Routing& r, const float* residual, float* y, void* ws, int* err, bool clear_status,
                      cudaStream_t st, bool shared_early) {
-  if (T > kPrefillMinT) {  // many tokens: the block-scaled grouped GEMM (MXFP4 only)
+  if (T > kPrefillMinT) {  // many tokens: MXFP4 on the block-scaled grouped GEMM, Q4-style on the dequantising one
     if (shared_early) return ERR_ARG;
-    return launch_ffn_mx_prefill(s, shw, w, x, x_dtype, T, r, residual, y, ws, err, clear_status, num_sms(), st);
+    if (w.fmt == 0)
+      return launch_ffn_mx_prefill(s, shw, w, x, x_dtype, T, r, residual, y, ws, err, clear_status, num_sms(), st);
+    return launch_ffn_prefill(s, shw, x, x_dtype, T, r, residual, y, ws, err, clear_status, num_sms(), st, &w);
   }
   const int nA = T * s.k;
   const int KP = mx_parts(s.H), DP = mx_parts(s.I);

@@ -78,7 +78,8 @@ struct MxPlanes {
   const uint8_t* down_codes;
   const void* down_scales;
 };
-size_t mx_ffn_workspace_bytes(const LayerShape& s, int T);
+// fmt: 0 = MXFP4, 1 = Q4-style (the many-token step differs: block-scaled GEMM or the dequantising one)
+size_t mx_ffn_workspace_bytes(const LayerShape& s, int T, int fmt);
 int launch_ffn_mxfp4(const LayerShape& s, const WeightPtrs& shw, const MxPlanes& w, const void* x, int x_dtype,
                      int T, const Routing& r, const float* residual, float* y, void* ws, int* err, bool clear_status,
                      cudaStream_t st, bool shared_early);
@@ -124,9 +125,10 @@ int launch_router_tc(const uint16_t* Wr, const float* bias, const uint16_t* x, i
 constexpr int kPrefillMinT = 16;
 bool prefill_path_supported(const LayerShape& s, int T);
 size_t prefill_workspace_bytes(const LayerShape& s, int T);
+// q4: Q4-style routed experts (codes and fp16 d planes) in place of the IQ2 / Q2K planes of `w`.
 int launch_ffn_prefill(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
                        const float* residual, float* y, void* ws, int* err, bool clear_status, int sms,
-                       cudaStream_t st);
+                       cudaStream_t st, const MxPlanes* q4 = nullptr);
 
 // The shared expert alone on the tensor-core GEMM (prefill.cu): s_out = fp32 [T][H].
 size_t prefill_shared_workspace_bytes(const LayerShape& s, int T);

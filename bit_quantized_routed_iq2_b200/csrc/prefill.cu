@@ -76,7 +76,15 @@ enum TcKind : int {
   TC_Q2K = 1,        // routed down: dequantised Q2K, fp32 out
   TC_BF16_PAIR = 2,  // shared gate+up: bf16 tiles by TMA, SwiGLU, bf16 hi/lo h out
   TC_BF16 = 3,       // shared down: bf16 tiles by TMA, fp32 out
+  TC_Q4_PAIR = 4,    // routed gate+up: dequantised Q4-style pair, SwiGLU, fp16 h out
+  TC_Q4 = 5,         // routed down: dequantised Q4-style blocks, fp16 out
 };
+// Kind predicates: weights dequantised by the SMs; two weight matrices (gate and up) per tile; the routed
+// gate/up epilogue (SwiGLU, fp16 h); the routed down epilogue (fp16 expert outputs).
+constexpr bool tc_dq(int K) { return K == TC_IQ2_PAIR || K == TC_Q2K || K == TC_Q4_PAIR || K == TC_Q4; }
+constexpr bool tc_two(int K) { return K == TC_IQ2_PAIR || K == TC_BF16_PAIR || K == TC_Q4_PAIR; }
+constexpr bool tc_hout(int K) { return K == TC_IQ2_PAIR || K == TC_Q4_PAIR; }
+constexpr bool tc_oout(int K) { return K == TC_Q2K || K == TC_Q4; }
 
 struct TcPair {
   int e, p0, n, pad;  // expert (weight block), first B row, rows of B used
@@ -122,20 +130,24 @@ struct TcArgs {
 // all 512 columns.
 template <int KIND>
 struct TcLayout {
-  static constexpr bool dq = (KIND == TC_IQ2_PAIR || KIND == TC_Q2K);
-  static constexpr bool pair = (KIND == TC_IQ2_PAIR || KIND == TC_BF16_PAIR);
-  static constexpr int stages = dq ? 8 : (pair ? 4 : 6);                 // shared-memory ring
+  static constexpr bool dq = tc_dq(KIND);
+  static constexpr bool pair = tc_two(KIND);
+  static constexpr int stages = dq ? (KIND == TC_Q4_PAIR ? 7 : 8) : (pair ? 4 : 6);  // shared-memory ring
   static constexpr size_t stage_bytes = dq ? kTile : (pair ? 3 : 2) * kTile;
   // code bytes of one 256-weight block for the tile's 128 rows: IQ2 64 bytes per row of gate and of up,
-  // Q2K the whole 80-byte block
-  static constexpr size_t code_bytes = KIND == TC_IQ2_PAIR ? 2 * 128 * 64 : (KIND == TC_Q2K ? 128 * 80 : 0);
+  // Q2K the whole 80-byte block, Q4-style 128 code bytes per row (of gate and of up)
+  static constexpr size_t code_bytes = KIND == TC_IQ2_PAIR ? 2 * 128 * 64
+                                       : KIND == TC_Q2K    ? 128 * 80
+                                       : KIND == TC_Q4_PAIR ? 2 * 128 * 128
+                                       : KIND == TC_Q4      ? 128 * 128
+                                                            : 0;
   static constexpr size_t code_off = stages * stage_bytes;
   static constexpr size_t b_off = dq ? 0 : (pair ? 2 : 1) * kTile;      // B tile inside a stage
-  static constexpr int a_stages = KIND == TC_IQ2_PAIR ? 4 : 8;           // TMEM A ring (dq kinds)
+  static constexpr int a_stages = tc_hout(KIND) ? 4 : 8;                 // TMEM A ring (dq kinds)
   static constexpr uint32_t a_cols = pair ? 64 : 32;                     // TMEM columns per A stage
-  static constexpr int acc_bufs = KIND == TC_IQ2_PAIR ? 1 : 2;
+  static constexpr int acc_bufs = tc_hout(KIND) ? 1 : 2;
   static constexpr uint32_t acc_base = dq ? 256 : 0;
-  static constexpr uint32_t acc_stride = KIND == TC_Q2K ? 128 : 256;    // columns per accumulator buffer
+  static constexpr uint32_t acc_stride = tc_oout(KIND) ? 128 : 256;     // columns per accumulator buffer
   static constexpr size_t tabs = code_off + (dq ? kCStages * code_bytes : 0);
   static constexpr size_t tab_bytes =
       KIND == TC_IQ2_PAIR ? (256 * 128 + 128 * 128) : (KIND == TC_Q2K ? 256 * 128 : 0);
@@ -247,6 +259,33 @@ __device__ __forceinline__ void dq_q2k_sub(uint32_t w, uint32_t scb, float d, fl
   }
 }
 
+__device__ __forceinline__ uint32_t hsub2_u(uint32_t a, uint32_t b) {
+  __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// One Q4-style block of a row (32 weights: element 2i in the low nibble of
+// code byte i, 2i+1 in the high nibble; w = d * (q - 8)) with s2 = the fp16
+// pair (s, s), s = fp16(d * 2^10) -> 16 words of fp16 pairs in K order. The
+// pair (1024 + q0, 1024 + q1) is built from its bits (0x6400 | q), so
+// q - 8 = (1024 + q) - 1032 is exact in fp16; each weight is then the fp16
+// rounding of s * (q - 8). The 2^10 keeps small scales clear of fp16
+// subnormals and is taken out in the fp32 epilogue.
+__device__ __forceinline__ void dq_q4_block(uint4 c, uint32_t s2, uint32_t (&o)[16]) {
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+  constexpr uint32_t kHalf1032Twice = 0x64086408u;  // fp16 pair (1032, 1032)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t lo = w[i] & 0x0F0F0F0Fu, hi = (w[i] >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      // bytes: low nibble of byte b (element 2b) at byte 0, its high nibble (element 2b + 1) at byte 2
+      const uint32_t pr = (prmt(lo, hi, static_cast<uint32_t>(b | ((4 + b) << 8))) & 0x00FF00FFu) | 0x64006400u;
+      o[4 * i + b] = hmul2_u(hsub2_u(pr, kHalf1032Twice), s2);
+    }
+  }
+}
+
 // The dequantisation tables of the dequantising kinds, at `tabs` (see
 // TcLayout): IQ2 level selectors (16 copies of 8 bytes per grid row), IQ2 signs
 // as fp16 +-1 pairs (8 copies of 16 bytes per sign field), Q2K selectors (32
@@ -334,8 +373,9 @@ template <int KIND>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_b,
                                                                 const __grid_constant__ CUtensorMap tm_a0,
                                                                 const __grid_constant__ CUtensorMap tm_a1, TcArgs a) {
-  constexpr bool PAIR = (KIND == TC_IQ2_PAIR || KIND == TC_BF16_PAIR);
-  constexpr bool DQ = (KIND == TC_IQ2_PAIR || KIND == TC_Q2K);
+  constexpr bool PAIR = tc_two(KIND);
+  constexpr bool DQ = tc_dq(KIND);
+  constexpr bool Q4K = (KIND == TC_Q4_PAIR || KIND == TC_Q4);
   constexpr bool BF16 = (KIND == TC_BF16_PAIR || KIND == TC_BF16);
   using L = TcLayout<KIND>;
   constexpr int kStages = L::stages;
@@ -420,6 +460,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             if (KIND == TC_IQ2_PAIR) {
               tma_load_2d(ce, &tm_a0, 64 * (ks >> 2), wrow, &fullC[c]);
               tma_load_2d(ce + 128 * 64, &tm_a1, 64 * (ks >> 2), wrow, &fullC[c]);
+            } else if (KIND == TC_Q4_PAIR) {
+              tma_load_2d(ce, &tm_a0, 128 * (ks >> 2), wrow, &fullC[c]);
+              tma_load_2d(ce + 128 * 128, &tm_a1, 128 * (ks >> 2), wrow, &fullC[c]);
+            } else if (KIND == TC_Q4) {
+              tma_load_2d(ce, &tm_a0, 128 * (ks >> 2), wrow, &fullC[c]);
             } else {
               tma_load_2d(ce, &tm_a0, 80 * (ks >> 2), wrow, &fullC[c]);
             }
@@ -545,8 +590,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       if (KIND == TC_IQ2_PAIR) return static_cast<uint32_t>(__ldg((part ? a.d1 : a.d0) + grow * nblk + b));
       return __ldg(a.dd + grow * nblk + b);
     };
+    // Q4-style kinds: the fp16 d of the stage's two 32-weight blocks of this row (one word), loaded one
+    // stage of this group ahead
+    auto ldq4 = [&](size_t grow, int ks_) -> uint32_t {
+      const uint16_t* dp = (KIND == TC_Q4_PAIR && part) ? a.d1 : a.d0;
+      return __ldg(reinterpret_cast<const uint32_t*>(dp + grow * (a.K / 32)) + ks_);
+    };
     int u = next_tile(blockIdx.x);
-    uint32_t dq1 = u < nunits ? ldscale(row_of(u), 0) : 0u;
+    uint32_t dq1 = (!Q4K && u < nunits) ? ldscale(row_of(u), 0) : 0u;
+    uint32_t q4n = (Q4K && u < nunits) ? ldq4(row_of(u), grp) : 0u;
     while (u < nunits) {
       const int un = next_tile(u + gridDim.x);
       const size_t grow = row_of(u);
@@ -559,10 +611,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           ok = false;
           break;
         }
-        if ((ks & 3) == grp) {  // the group's first stage of a block
+        if (!Q4K && (ks & 3) == grp) {  // the group's first stage of a block
           const int b = ks >> 2;
           dq0 = dq1;
           dq1 = b + 1 < nblk ? ldscale(grow, b + 1) : (un < nunits ? ldscale(grow_n, 0) : 0u);
+        }
+        uint32_t q4d = 0;
+        if (Q4K) {
+          q4d = q4n;
+          q4n = ks + 2 < nks ? ldq4(grow, ks + 2) : (un < nunits ? ldq4(grow_n, grp) : 0u);
         }
         const int sa = static_cast<int>(gs % kAStages);
         const uint32_t pha = static_cast<uint32_t>((gs / kAStages) & 1);
@@ -582,6 +639,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           const uint32_t tc = tmem + tlane + part * 32 + sa * L::a_cols;
           tmem_st16(tc, o0);
           tmem_st16(tc + 16, o1);
+        } else if (KIND == TC_Q4_PAIR) {
+          // part = matrix; the row's 64 weights of this stage: two 32-weight blocks, 32 code bytes
+          const uint32_t cq = ce + part * (128 * 128) + r * 128 + 32 * q;
+          const uint4 c0 = lds128s(cq), c1 = lds128s(cq + 16);
+          const float s0 = half_bits_to_float(static_cast<uint16_t>(q4d & 0xFFFFu)) * 1024.0f;
+          const float s1 = half_bits_to_float(static_cast<uint16_t>(q4d >> 16)) * 1024.0f;
+          uint32_t o0[16], o1[16];
+          dq_q4_block(c0, f2_to_h2(s0, s0), o0);
+          dq_q4_block(c1, f2_to_h2(s1, s1), o1);
+          const uint32_t tc = tmem + tlane + part * 32 + sa * L::a_cols;
+          tmem_st16(tc, o0);
+          tmem_st16(tc + 16, o1);
+        } else if (KIND == TC_Q4) {
+          // part = half of the stage's 64 weights = block 2 * ks + part (16 code bytes)
+          const uint4 c0 = lds128s(ce + r * 128 + 32 * q + 16 * part);
+          const float s0 = half_bits_to_float(static_cast<uint16_t>(part ? q4d >> 16 : q4d & 0xFFFFu)) * 1024.0f;
+          uint32_t o0[16];
+          dq_q4_block(c0, f2_to_h2(s0, s0), o0);
+          tmem_st16(tmem + tlane + part * 16 + sa * L::a_cols, o0);
         } else {
           // part = half of the stage's 64 weights = sub-blocks 4 * (ks % 4) + 2 * part, +1 of the block
           const uint2 w = lds64s(ce + r * 80 + 16 + 16 * q + 8 * part);
@@ -617,7 +693,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       const int buf = t % kAccBufs;
       // the tile's per-row exponents (lane n % 32 of word n / 32), loaded before the wait
       int ex4[4] = {0, 0, 0, 0};
-      if (KIND == TC_IQ2_PAIR) {
+      if (tc_hout(KIND)) {
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           if (32 * i + lane < pr.n) ex4[i] = __ldg(a.row_exp + pr.p0 + 32 * i + lane);
@@ -639,7 +715,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           const int n = c0 + j;
           if (n >= pr.n) break;
           const size_t orow = static_cast<size_t>(pr.p0 + n);
-          if (KIND == TC_IQ2_PAIR) {
+          if (tc_hout(KIND)) {
             // B row = x * 2^-e: g, u come back as exact fp32 rescalings; h leaves as
             // fp16(h * 2^(-2e-12)), the scale that keeps it inside the fp16 range
             const int ex = __shfl_sync(0xffffffffu, exw, (c0 & 31) + j);
@@ -658,7 +734,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
             reinterpret_cast<__nv_bfloat16*>(a.out)[orow * a.ldo + row] = hi;
             reinterpret_cast<__nv_bfloat16*>(a.out)[(static_cast<size_t>(a.out_rows) + orow) * a.ldo + row] = lo;
-          } else if (KIND == TC_Q2K) {  // routed expert outputs, combined later in slot order
+          } else if (tc_oout(KIND)) {  // routed expert outputs, combined later in slot order
             // B row = h * 2^(-2e-12), so the accumulator is o * 2^(-2e-12) (h and o are
             // quadratic in x); it is stored as is and the combine applies 2^(2e+12)
             reinterpret_cast<__half*>(a.out)[orow * a.ldo + row] = __float2half_rn(__uint_as_float(g[j]) * a.oscale);
@@ -1011,7 +1087,7 @@ size_t prefill_workspace_bytes(const LayerShape& s, int T) { return carve_prefil
 
 int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x, int x_dtype, int T,
                        const Routing& r, const float* residual, float* y, void* ws, int* err, bool clear_status,
-                       int sms, cudaStream_t st) {
+                       int sms, cudaStream_t st, const MxPlanes* q4) {
   const PrefillWs pw = carve_prefill(sh, T, static_cast<char*>(ws));
   const int nA = T * sh.k;
   int rc = OK;
@@ -1041,16 +1117,22 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
   {
     ProfScope ps(MOE_K_PREFILL_GATEUP, st);
     const uint64_t wrows = static_cast<uint64_t>(sh.E) * sh.I;
-    if (!tc_map(&mb, pw.xp, false, sh.H, nA, 1) || !code_map(&ma0, w.gate_codes, sh.H / 4, wrows, 64) ||
-        !code_map(&ma1, w.up_codes, sh.H / 4, wrows, 64))
+    // IQ2: 64 code bytes per 256 weights; Q4-style: 128
+    const uint8_t* gc = q4 ? q4->gate_codes : w.gate_codes;
+    const uint8_t* uc = q4 ? q4->up_codes : w.up_codes;
+    const uint32_t cb = q4 ? 128 : 64;
+    if (!tc_map(&mb, pw.xp, false, sh.H, nA, 1) || !code_map(&ma0, gc, sh.H / 256 * cb, wrows, cb) ||
+        !code_map(&ma1, uc, sh.H / 256 * cb, wrows, cb))
       return ERR_CUDA;
     TcArgs a{};
     a.n_experts = sh.E; a.b_rows = nA;
     a.rows_e = sh.I; a.K = sh.H; a.mt = sh.I / kMT; a.planes = 1;
-    a.c0 = w.gate_codes; a.d0 = w.gate_d; a.c1 = w.up_codes; a.d1 = w.up_d;
+    a.c0 = gc; a.c1 = uc;
+    a.d0 = q4 ? static_cast<const uint16_t*>(q4->gate_scales) : w.gate_d;
+    a.d1 = q4 ? static_cast<const uint16_t*>(q4->up_scales) : w.up_d;
     a.pairs = pw.pairs; a.npairs = pw.counts; a.out = pw.hh; a.ldo = sh.I; a.out_rows = nA;
     a.oscale = 1.0f / 1024.0f; a.err = err; a.row_exp = pw.aexp;
-    rc |= launch_tc<TC_IQ2_PAIR>(mb, ma0, ma1, a, sms, st);
+    rc |= q4 ? launch_tc<TC_Q4_PAIR>(mb, ma0, ma1, a, sms, st) : launch_tc<TC_IQ2_PAIR>(mb, ma0, ma1, a, sms, st);
   }
   if (sh.Is > 0) {
     ProfScope ps(MOE_K_SHARED_GATEUP, st);
@@ -1068,16 +1150,20 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
   }
   {
     ProfScope ps(MOE_K_PREFILL_DOWN, st);
+    // Q2K: 80 code bytes per 256 weights; Q4-style: 128
+    const uint8_t* dc = q4 ? q4->down_codes : w.down_codes;
+    const uint32_t cb = q4 ? 128 : 80;
     if (!tc_map(&mb, pw.hh, false, sh.I, nA, 1) ||
-        !code_map(&ma0, w.down_codes, static_cast<uint64_t>(sh.I / 256) * 80, static_cast<uint64_t>(sh.E) * sh.H, 80))
+        !code_map(&ma0, dc, static_cast<uint64_t>(sh.I / 256) * cb, static_cast<uint64_t>(sh.E) * sh.H, cb))
       return ERR_CUDA;
     TcArgs a{};
     a.n_experts = sh.E; a.b_rows = nA;
     a.rows_e = sh.H; a.K = sh.I; a.mt = sh.H / kMT; a.planes = 1;
-    a.c0 = w.down_codes; a.dd = w.down_dd;
+    a.c0 = dc; a.dd = w.down_dd;
+    if (q4) a.d0 = static_cast<const uint16_t*>(q4->down_scales);
     a.pairs = pw.pairs; a.npairs = pw.counts; a.out = pw.o; a.ldo = sh.H; a.out_rows = nA;
-    a.oscale = 1.0f; a.err = err; a.row_exp = pw.aexp;
-    rc |= launch_tc<TC_Q2K>(mb, ma0, ma0, a, sms, st);
+    a.oscale = q4 ? 1.0f / 1024.0f : 1.0f; a.err = err; a.row_exp = pw.aexp;
+    rc |= q4 ? launch_tc<TC_Q4>(mb, ma0, ma0, a, sms, st) : launch_tc<TC_Q2K>(mb, ma0, ma0, a, sms, st);
   }
   if (sh.Is > 0) {
     ProfScope ps(MOE_K_SHARED_DOWN, st);

@@ -7,7 +7,8 @@ layer within the normwise bound of the 2-bit path (FFN_TOL) at small shapes
 expert, uneven routing) and at the one-token decode shape (H=7168, I=2048,
 E=256, k=8, I_s=2048). Above 16 tokens (the block-scaled grouped GEMM) against
 the oracle with MXFP8 activations, at small shapes with ragged and multi-tile
-experts and on sampled tokens of the 2048-token prefill shape.
+experts and on sampled tokens of the 2048-token prefill shape; the Q4-style
+format above 16 tokens (the dequantising grouped GEMM) against the exact oracle.
 """
 import numpy as np
 import pytest
@@ -93,10 +94,16 @@ def test_mxfp4_rejects_unsupported_shapes(torch_cuda):
     assert moe2bit.workspace_size_mxfp4(desc, 16) > 0
     # above 16 tokens MXFP4 takes the block-scaled grouped GEMM; its workspace covers the GEMV step too
     assert moe2bit.workspace_size_mxfp4(desc, 300) >= moe2bit.workspace_size_mxfp4(desc, 16)
-    # the Q4-style format has no many-token path
+    # the Q4-style format takes the dequantising grouped GEMM above 16 tokens; its shared-expert GEMMs need
+    # I_s % 128 == 0 there
     n = ctypes.c_size_t(0)
-    assert moe2bit.load().moe_workspace_size_q4(ctypes.byref(desc), 17, ctypes.byref(n)) != 0
     assert moe2bit.load().moe_workspace_size_q4(ctypes.byref(desc), 16, ctypes.byref(n)) == 0
+    assert moe2bit.load().moe_workspace_size_q4(ctypes.byref(desc), 300, ctypes.byref(n)) == 0
+    odd = moe2bit.desc_of(1024, 512, 16, 4, 64)
+    assert moe2bit.load().moe_workspace_size_q4(ctypes.byref(odd), 16, ctypes.byref(n)) == 0
+    assert moe2bit.load().moe_workspace_size_q4(ctypes.byref(odd), 17, ctypes.byref(n)) != 0
+    with pytest.raises(RuntimeError):
+        moe2bit.workspace_size_mxfp4(odd, 17)
 
 
 # More than 16 tokens: FP4 weights x MXFP8 activations on the block-scaled tensor cores; the oracle takes
@@ -216,3 +223,34 @@ def test_q4_decode1_shape(torch_cuda):
     y = _q4_forward(torch_cuda, moe2bit.to_device_q4(lw), x)
     ref, _, _ = oracle.layer_forward(lw, x)
     assert normwise(y, ref) <= FFN_TOL, normwise(y, ref)
+
+
+# More than 16 tokens with Q4-style experts: the dequantising grouped GEMM (fp16 weight tiles in TMEM,
+# tcgen05.mma kind::f16) against the exact oracle.
+@pytest.mark.parametrize("name", ["t17_bf16", "t40_bf16_zipf", "t200_f32_zipf_noshared", "t300_bf16"])
+def test_q4_layer_many_tokens(torch_cuda, name):
+    c = MANY[name]
+    cfg = synth.Config("q4g_" + name, c["T"], 1024, 512, c["E"], c["k"], c["Is"], c["x_dtype"], 1.0, c["zipf"], 1,
+                       0x5147A0 + len(name))
+    lw = synth.make_layer_q4(cfg)
+    x = screened_x(cfg, lw)
+    res = synth.make_residual(cfg, cfg.T)
+    y = _q4_forward(torch_cuda, moe2bit.to_device_q4(lw), x, res)
+    ref, _, _ = oracle.layer_forward(lw, x, res)
+    assert normwise(y, ref) <= FFN_TOL, (name, normwise(y, ref))
+
+
+@pytest.mark.slow
+def test_q4_prefill_shape_sampled(torch_cuda):
+    """The 2048-token prefill shape with Q4-style experts (every expert active); sampled tokens against the
+    oracle as in test_mxfp4_prefill_shape_sampled."""
+    cfg = synth.CONFIGS["prefill"]
+    lw = synth.make_layer_q4(cfg)
+    x = synth.make_x_fast(cfg, cfg.T)
+    y = _q4_forward(torch_cuda, moe2bit.to_device_q4(lw), x)
+    cand = np.array([0, 1, 2, 3, 777, 778, 1500, 1501, cfg.T - 2, cfg.T - 1])
+    _, _, logits = oracle.route(lw.router_w, lw.router_bias, x[cand], cfg.k, want_logits=True)
+    rows = np.setdiff1d(cand, cand[near_tie_tokens(logits, cfg.k)])[:5]
+    assert rows.size == 5
+    ref, _, _ = oracle.layer_forward(lw, x[rows])
+    assert normwise(y[rows], ref) <= FFN_TOL, normwise(y[rows], ref)
