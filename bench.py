@@ -54,7 +54,7 @@ def parse():
                     help="override the tokens per step (small cases for profiling; not a bench workload)")
     ap.add_argument("--workloads", default="auto",
                     help="other workloads measured in the same run and reported under 'workloads': 'all' "
-                         "(decode32, prefill, stack, decode1_mxfp4, decode1_q4, prefill_mxfp4, decode1_cached, "
+                         "(decode32, prefill, stack, decode1_mxfp4, decode1_q4, prefill_mxfp4, prefill_q4, decode1_cached, "
                          "quantize), 'none', or a comma list; "
                          "'auto' = all on one GPU")
     ap.add_argument("--workload-steps", type=int, default=20, help="timed steps of each extra workload")
@@ -634,40 +634,52 @@ def measure_mxfp4(args, steps, fmt="mxfp4"):
     }
 
 
-def measure_mxfp4_prefill(args, steps):
-    """2048 bf16 tokens with MXFP4 routed experts (the prefill shapes H=7168, I=2048, E=256, k=8,
-    I_s=2048; every expert active): FP4 weights x MXFP8 activations on the block-scaled tensor cores
-    (moe_layer_forward_mxfp4 above 16 tokens). One resident layer of 6 GB (weights larger than L2).
-    Roofline of the gate/up grouped GEMM against HBM: every active expert's gate and up codes and
-    scales, the MXFP8 activations it reads and the MXFP8 h it writes; the tensor-pipe fraction (FP8 x FP4
-    flops over twice the bf16 peak, the nominal fp8 : bf16 ratio) beside it."""
+def measure_blk32_prefill(args, steps, fmt="mxfp4"):
+    """2048 bf16 tokens with block-32 routed experts (the prefill shapes H=7168, I=2048, E=256, k=8,
+    I_s=2048; every expert active), one resident layer of 6-6.6 GB (weights larger than L2).
+    MXFP4: FP4 weights x MXFP8 activations on the block-scaled tensor cores; roofline of the gate/up
+    grouped GEMM against HBM (every active expert's gate and up codes and scales, the MXFP8 activations it
+    reads and the MXFP8 h it writes), the tensor-pipe fraction (FP8 x FP4 flops over twice the bf16 peak,
+    the nominal fp8 : bf16 ratio) beside it.
+    Q4-style: the dequantising grouped GEMM (fp16 weight tiles, tcgen05 kind::f16); roofline of its gate/up
+    launch against the bf16 tensor peak, the HBM fraction of its weight bytes beside it."""
     import torch
 
     from bit_quantized_routed_iq2_b200 import moe2bit
 
+    q4 = fmt == "q4"
     E = args.experts or 256
-    cfg = synth.Config("prefill_mxfp4" if E == 256 else f"prefill_mxfp4_E{E}", 2048 * E // 256, 7168, 2048, E, 8,
-                       2048, "bf16", math.sqrt(0.5), False, 1, 0xD540000A)
-    lw = synth.make_layer_mxfp4(cfg)
-    dl = moe2bit.to_device_mxfp4(lw)
+    name = "prefill_" + fmt + ("" if E == 256 else f"_E{E}")
+    cfg = synth.Config(name, 2048 * E // 256, 7168, 2048, E, 8, 2048, "bf16", math.sqrt(0.5), False, 1,
+                       0xD540000B if q4 else 0xD540000A)
+    lw = (synth.make_layer_q4 if q4 else synth.make_layer_mxfp4)(cfg)
+    dl = (moe2bit.to_device_q4 if q4 else moe2bit.to_device_mxfp4)(lw)
     del lw
+    forward = moe2bit.layer_forward_q4 if q4 else moe2bit.layer_forward_mxfp4
     x = torch.from_numpy(synth.make_x_fast(cfg, cfg.T).view(np.int16)).cuda().view(torch.bfloat16)
     y = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
-    ws = moe2bit.alloc_workspace_mxfp4(dl.desc, cfg.T)
+    if q4:
+        import ctypes
+
+        n = ctypes.c_size_t(0)
+        assert moe2bit.load().moe_workspace_size_q4(ctypes.byref(dl.desc), cfg.T, ctypes.byref(n)) == 0
+        ws = torch.empty(max(int(n.value), 16), dtype=torch.uint8, device="cuda")
+    else:
+        ws = moe2bit.alloc_workspace_mxfp4(dl.desc, cfg.T)
     stream = torch.cuda.current_stream()
     for _ in range(max(args.warmup, 3)):
-        moe2bit.layer_forward_mxfp4(dl, x, None, y, ws, stream)
+        forward(dl, x, None, y, ws, stream)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(steps):
-        moe2bit.layer_forward_mxfp4(dl, x, None, y, ws, stream)
+        forward(dl, x, None, y, ws, stream)
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     moe2bit.profile_enable(True)
     for _ in range(steps):
-        moe2bit.layer_forward_mxfp4(dl, x, None, y, ws, stream)
+        forward(dl, x, None, y, ws, stream)
     torch.cuda.synchronize()
     prof = moe2bit.profile_read()
     moe2bit.profile_enable(False)
@@ -678,25 +690,40 @@ def measure_mxfp4_prefill(args, steps):
     hbm, bf16_tf, peak_kind = peaks()
     avg_ms = {k: v[0] / max(v[1], 1) for k, v in prof.items()}
     nA = cfg.T * cfg.k
-    alg = (cfg.E * 2 * cfg.I * cfg.H * (0.5 + 1 / 32) + nA * cfg.H * (1 + 1 / 32) + nA * cfg.I * (1 + 1 / 32))
-    achieved = alg / (avg_ms["prefill_gateup"] * 1e-3) / 1e9
-    dn_alg = cfg.E * cfg.H * cfg.I * (0.5 + 1 / 32) + nA * cfg.I * (1 + 1 / 32) + nA * cfg.H * 4
+    wb = 0.5 + (2.0 if q4 else 1.0) / 32  # bytes per weight: codes + scales
     flops = 2.0 * nA * 2 * cfg.I * cfg.H
+    gu_s = avg_ms["prefill_gateup"] * 1e-3
+    if q4:
+        alg = cfg.E * 2 * cfg.I * cfg.H * wb + nA * cfg.H * 2 + nA * cfg.I * 2  # weights, fp16 x in, fp16 h out
+        dn_alg = cfg.E * cfg.H * cfg.I * wb + nA * cfg.I * 2 + nA * cfg.H * 2
+    else:
+        alg = cfg.E * 2 * cfg.I * cfg.H * wb + nA * cfg.H * (1 + 1 / 32) + nA * cfg.I * (1 + 1 / 32)
+        dn_alg = cfg.E * cfg.H * cfg.I * wb + nA * cfg.I * (1 + 1 / 32) + nA * cfg.H * 4
     fp8_tf = 2.0 * bf16_tf
+    hbm_ach = alg / gu_s / 1e9
+    if q4:
+        tf = flops / gu_s / 1e12
+        roof = {"bound": "tensor", "kernel": "prefill_gateup", "achieved": tf, "peak": bf16_tf, "unit": "TFLOP/s",
+                "frac": tf / bf16_tf, "peak_source": peak_kind, "algorithmic_flops_per_launch": flops,
+                "hbm_frac": hbm_ach / hbm}
+    else:
+        roof = {"bound": "hbm", "kernel": "prefill_gateup", "achieved": hbm_ach, "peak": hbm, "unit": "GB/s",
+                "frac": hbm_ach / hbm, "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg,
+                "tensor_frac": flops / gu_s / 1e12 / fp8_tf, "tensor_peak_tflops": fp8_tf}
+    roof.update({"avg_launch_ms": avg_ms["prefill_gateup"],
+                 "traffic": (traffic_record(cfg.name, "prefill_gateup") or {}).get("bytes_per_launch"),
+                 "down_hbm_frac": dn_alg / (avg_ms["prefill_down"] * 1e-3) / 1e9 / hbm})
     return {
         "value": cfg.T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
         "config": {"workload": cfg.name, "tokens_per_step": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
-                   "I_s": cfg.Is, "experts": "MXFP4 (OCP MX: E2M1 x 32 + E8M0), all three routed matrices",
-                   "activations": "routed: MXFP8 (E4M3 x 32 + E8M0); shared expert: bf16",
-                   "l2": "inputs larger than L2: one resident layer of 6 GB", "launch": "stream"},
+                   "I_s": cfg.Is,
+                   "experts": ("Q4-style (32 x 4-bit codes + fp16 d, w = d (q - 8))" if q4 else
+                               "MXFP4 (OCP MX: E2M1 x 32 + E8M0)") + ", all three routed matrices",
+                   "activations": ("routed: fp16 with a power-of-2 scale per token" if q4 else
+                                   "routed: MXFP8 (E4M3 x 32 + E8M0)") + "; shared expert: bf16",
+                   "l2": "inputs larger than L2: one resident layer of 6 GB or more", "launch": "stream"},
         "kernels": {k: {"avg_ms": v, "launches_per_step": prof[k][1] / steps} for k, v in avg_ms.items()},
-        "roofline": {"bound": "hbm", "kernel": "prefill_gateup", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg,
-                     "avg_launch_ms": avg_ms["prefill_gateup"],
-                     "traffic": (traffic_record(cfg.name, "prefill_gateup") or {}).get("bytes_per_launch"),
-                     "tensor_frac": flops / (avg_ms["prefill_gateup"] * 1e-3) / 1e12 / fp8_tf,
-                     "tensor_peak_tflops": fp8_tf,
-                     "down_frac": dn_alg / (avg_ms["prefill_down"] * 1e-3) / 1e9 / hbm},
+        "roofline": roof,
     }
 
 
@@ -785,7 +812,8 @@ def run_ours(args, cfg):
         want = "all" if (world == 1 and not args.experts and not args.tokens) else "none"
     if want != "none":
         names = ([n for n in ("decode32", "prefill", "stack") if n != cfg.name] +
-                 ["decode1_mxfp4", "decode1_q4", "prefill_mxfp4", "decode1_cached", "quantize"] if want == "all"
+                 ["decode1_mxfp4", "decode1_q4", "prefill_mxfp4", "prefill_q4", "decode1_cached", "quantize"]
+                 if want == "all"
                  else want.split(","))
         line["workloads"] = {}
         for name in names:
@@ -795,8 +823,8 @@ def run_ours(args, cfg):
                 w = measure_quantize(args)
             elif name in ("decode1_mxfp4", "decode1_q4"):
                 w = measure_mxfp4(args, args.workload_steps, name.split("_")[1])
-            elif name == "prefill_mxfp4":
-                w = measure_mxfp4_prefill(args, max(3, args.workload_steps // 4))
+            elif name in ("prefill_mxfp4", "prefill_q4"):
+                w = measure_blk32_prefill(args, max(3, args.workload_steps // 4), name.split("_")[1])
             else:
                 w = measure(args, synth.CONFIGS[name], world, rank, local, args.workload_steps)
                 line["gpu_launches"] += w["gpu_launches"]
