@@ -560,8 +560,9 @@ def measure_mxfp4(args, steps, fmt="mxfp4"):
     from bit_quantized_routed_iq2_b200 import moe2bit
 
     q4 = fmt == "q4"
-    cfg = synth.Config("decode1_" + fmt, 1, 7168, 2048, 256, 8, 2048, "bf16", 1.0, False, 1,
-                       0xD5400008 if q4 else 0xD5400007)
+    E = args.experts or 256  # a smaller E (profiling captures) keeps the 8 active experts per step
+    cfg = synth.Config("decode1_" + fmt + ("" if E == 256 else f"_E{E}"), 1, 7168, 2048, E, 8, 2048, "bf16", 1.0,
+                       False, 1, 0xD5400008 if q4 else 0xD5400007)
     make = synth.make_layer_q4 if q4 else synth.make_layer_mxfp4
     upload = moe2bit.to_device_q4 if q4 else moe2bit.to_device_mxfp4
     forward = moe2bit.layer_forward_q4 if q4 else moe2bit.layer_forward_mxfp4
@@ -619,17 +620,18 @@ def measure_mxfp4(args, steps, fmt="mxfp4"):
     alg = cfg.k * 2 * cfg.I * cfg.H * (0.5 + scale_bytes / 32) + cfg.H * 2
     achieved = alg / (avg_ms["gateup"] * 1e-3) / 1e9
     dn_alg = cfg.k * cfg.H * cfg.I * (0.5 + scale_bytes / 32)
+    tr = traffic_record("decode1_" + fmt, "gateup")
     return {
         "value": 1.0 / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
         "config": {"workload": cfg.name, "tokens_per_step": 1, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
                    "I_s": cfg.Is, "experts": ("Q4-style (32 x 4-bit codes + fp16 d, w = d (q - 8))" if q4 else
                                               "MXFP4 (OCP MX: E2M1 x 32 + E8M0)") + ", all three routed matrices",
-                   "resident_layers": 2, "l2": "inputs larger than L2: 2 resident layers of 6 GB",
+                   "resident_layers": 2, "l2": "inputs larger than L2: 2 resident layers of all experts",
                    "launch": "cuda_graph"},
         "kernels": {k: {"avg_ms": v, "launches_per_step": prof[k][1] / steps} for k, v in avg_ms.items()},
         "roofline": {"bound": "hbm", "kernel": "gateup", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg,
-                     "avg_launch_ms": avg_ms["gateup"],
+                     "avg_launch_ms": avg_ms["gateup"], "traffic": tr["bytes_per_launch"] if tr else None,
                      "down_frac": dn_alg / (avg_ms["down"] * 1e-3) / 1e9 / hbm},
     }
 
