@@ -293,16 +293,18 @@ def measure(args, cfg, world, rank, local, steps):
 
     side = torch.cuda.Stream() if is_stack else None
 
-    def chain(first_x, st):
+    def chain(first_x, st, out=None):
         """The layers in order; while layer l runs, layer l+1's router and shared expert are prefetched
-        into L2 on a side stream (they do not depend on routing)."""
+        into L2 on a side stream (they do not depend on routing). The residual stream is `out` (default y)."""
+        yo = y if out is None else out
         cur = first_x
         for l, dl in enumerate(layers):
             if l + 1 < len(layers):
                 side.wait_stream(st)
                 moe2bit.prefetch_layer(layers[l + 1], side)
-            moe2bit.layer_forward(dl, cur, res if l == 0 else y, y, ws, st)
-            xa.copy_(y)  # next layer input = bf16 of the residual stream
+            moe2bit.layer_forward(dl, cur, res if l == 0 else yo, yo, ws, st)
+            with torch.cuda.stream(st):
+                xa.copy_(yo)  # next layer input = bf16 of the residual stream
             cur = xa
         st.wait_stream(side)
 
@@ -374,23 +376,68 @@ def measure(args, cfg, world, rank, local, steps):
     xd = torch.empty((T, cfg.H), dtype=torch.int16 if cfg.x_dtype == "bf16" else torch.float32, device="cuda")
     xdv = xd.view(torch.bfloat16) if cfg.x_dtype == "bf16" else xd
 
-    def e2e_step(i):
-        xd.copy_(xh[i % n_slots], non_blocking=True)
-        if is_stack:
-            chain(xdv, stream)
-        else:
-            moe2bit.layer_forward(layers[i % n_layers], xdv, None, y, ws, stream)
-        yh.copy_(y, non_blocking=True)
+    # Every step copies its own x from pinned host memory and reads its own y back into pinned host memory.
+    # Step i's graph holds three independent branches: the input copy of step i + 1, the layer of step i and the
+    # read-back of step i - 1 (x and y double-buffered), so the copies overlap the neighbouring steps' layers as
+    # a serving loop would run; an input copy before the first step and a read-back after the last complete the
+    # timed region (one copy of each kind more than the steps need).
+    xdb = [xd, torch.empty_like(xd)]
+    yb = [y, torch.empty_like(y)]
+    yhb = [yh, torch.empty_like(yh).pin_memory()]
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    eperiod = int(np.lcm(2, period))
 
+    def xview(b):
+        return xdb[b].view(torch.bfloat16) if cfg.x_dtype == "bf16" else xdb[b]
+
+    def e2e_step(i, st):
+        h2d.wait_stream(st)
+        d2h.wait_stream(st)
+        with torch.cuda.stream(h2d):
+            xdb[(i + 1) % 2].copy_(xh[(i + 1) % n_slots], non_blocking=True)
+        with torch.cuda.stream(d2h):
+            yhb[(i + 1) % 2].copy_(yb[(i + 1) % 2], non_blocking=True)  # the read-back of step i - 1
+        if is_stack:
+            chain(xview(i % 2), st, out=yb[i % 2])
+        else:
+            moe2bit.layer_forward(layers[i % n_layers], xview(i % 2), None, yb[i % 2], ws, st)
+        st.wait_stream(h2d)
+        st.wait_stream(d2h)
+
+    def e2e_first(st):
+        with torch.cuda.stream(st):
+            xdb[0].copy_(xh[0], non_blocking=True)
+
+    def e2e_last(i, st):
+        with torch.cuda.stream(st):
+            yhb[i % 2].copy_(yb[i % 2], non_blocking=True)
+
+    e2e_first(stream)
     for i in range(warm):
-        e2e_step(i)
+        e2e_step(i, stream)
     torch.cuda.synchronize()
+    e2e_graphs = []
+    if args.graph:
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        for j in range(eperiod):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                e2e_step(j, cap)
+            e2e_graphs.append(g)
+        torch.cuda.synchronize()
     e0.record(stream)
+    e2e_first(stream)
     for i in range(steps):
-        e2e_step(i)
+        if e2e_graphs:
+            e2e_graphs[i % eperiod].replay()
+        else:
+            e2e_step(i, stream)
+    e2e_last(steps - 1, stream)
     e1.record(stream)
     torch.cuda.synchronize()
     ms_e2e = e0.elapsed_time(e1) / steps
+    del e2e_graphs
     clocks = clk.stop()
     ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, "cuda")
 
@@ -470,7 +517,9 @@ def measure(args, cfg, world, rank, local, steps):
         "gpu_launches": int(round(sum(launches_per_step.values()) * steps)),
         "clocks": clocks,
         "e2e": {"value": job_tokens_per_s(T, world, ms_e2e), "unit": "tokens/s",
-                "h2d_bytes_per_step": bytes_x, "d2h_bytes_per_step": T * cfg.H * 4},
+                "h2d_bytes_per_step": bytes_x, "d2h_bytes_per_step": T * cfg.H * 4,
+                "copies": "every step: x from pinned host, y to pinned host; in step i's graph the input copy of "
+                          "step i+1 and the read-back of step i-1 run beside the layer (double-buffered)"},
         "dtype": "fp16" if "prefill_gateup" in prof else "int8",
         "steps": steps,
     }
