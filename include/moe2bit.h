@@ -520,10 +520,16 @@ MOE_API moe_status moe_debug_dequant_mxfp4(const uint8_t* codes, const uint8_t* 
  *   d     [rows][K/32] fp16.
  * moe_layer_forward_q4 is moe_layer_forward_mxfp4 with these planes: the same
  * routing, shared expert, combine, shapes (hidden % 512 == 0, inter % 512 ==
- * 0, 1 <= T <= 16, n_experts <= 1024), alignment, workspace
- * (moe_workspace_size_q4, equal to moe_workspace_size_mxfp4), status and
- * errors; the elements enter the integer products as the exact int8 q - 8 and
- * every block is scaled by its d in fp32.
+ * 0; n_experts <= 1024 up to 16 tokens; I_s % 128 == 0 or I_s == 0 above),
+ * 16-byte alignment (no 32-byte rule), status and errors; its workspace is
+ * moe_workspace_size_q4 (it differs from the MXFP4 one above 16 tokens).
+ * Numerics, 1 <= T <= 16: the elements enter the integer products as the exact
+ * int8 q - 8 and every block is scaled by its d in fp32 (activations as in
+ * moe_layer_forward_mxfp4's GEMVs). T > 16: the many-token path of
+ * moe_layer_forward (fp16 weight tiles on the tensor cores, fp32
+ * accumulation), each weight entering as fp16(fp16(d * 2^10) * (q - 8)), the
+ * 2^10 removed in fp32; activations and h as in moe_layer_forward's many-token
+ * path.
  */
 typedef struct {
   const uint16_t* router_w;     /* bf16 [E][H] */
