@@ -621,55 +621,62 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           q4d = q4n;
           q4n = ks + 2 < nks ? ldq4(grow, ks + 2) : (un < nunits ? ldq4(grow_n, grp) : 0u);
         }
+        // A free TMEM A slot is needed only for the stores. The Q4-style kinds decode into registers first,
+        // so their longer decode overlaps the MMAs still reading the slot (6 % faster gate/up); the 2-bit kinds
+        // wait first (decoding first was no faster for them, within the run-to-run spread of ~2 %).
         const int sa = static_cast<int>(gs % kAStages);
         const uint32_t pha = static_cast<uint32_t>((gs / kAStages) & 1);
-        if (!tc_wait_warp(&emptyA[sa], pha ^ 1u, a.err, abort_flag)) {
+        if (!Q4K && !tc_wait_warp(&emptyA[sa], pha ^ 1u, a.err, abort_flag)) {
           ok = false;
           break;
         }
-        tc_fence_after();
         const uint32_t ce = sbase + L::code_off + cb * L::code_bytes;
+        uint32_t o0[16], o1[16];
         if (KIND == TC_IQ2_PAIR) {
           // part = matrix; the row's two 8-byte records of this stage (32 weights each)
           const uint4 rec = lds128s(ce + part * (128 * 64) + r * 64 + 16 * q);
           const float dsc = half_bits_to_float(static_cast<uint16_t>(dq0)) * 128.0f;  // d / 8 * 2^10
-          uint32_t o0[16], o1[16];
           dq_iq2_sub(make_uint2(rec.x, rec.y), dsc, tabL, tabS, o0);
           dq_iq2_sub(make_uint2(rec.z, rec.w), dsc, tabL, tabS, o1);
-          const uint32_t tc = tmem + tlane + part * 32 + sa * L::a_cols;
-          tmem_st16(tc, o0);
-          tmem_st16(tc + 16, o1);
         } else if (KIND == TC_Q4_PAIR) {
           // part = matrix; the row's 64 weights of this stage: two 32-weight blocks, 32 code bytes
           const uint32_t cq = ce + part * (128 * 128) + r * 128 + 32 * q;
           const uint4 c0 = lds128s(cq), c1 = lds128s(cq + 16);
           const float s0 = half_bits_to_float(static_cast<uint16_t>(q4d & 0xFFFFu)) * 1024.0f;
           const float s1 = half_bits_to_float(static_cast<uint16_t>(q4d >> 16)) * 1024.0f;
-          uint32_t o0[16], o1[16];
           dq_q4_block(c0, f2_to_h2(s0, s0), o0);
           dq_q4_block(c1, f2_to_h2(s1, s1), o1);
-          const uint32_t tc = tmem + tlane + part * 32 + sa * L::a_cols;
-          tmem_st16(tc, o0);
-          tmem_st16(tc + 16, o1);
         } else if (KIND == TC_Q4) {
           // part = half of the stage's 64 weights = block 2 * ks + part (16 code bytes)
           const uint4 c0 = lds128s(ce + r * 128 + 32 * q + 16 * part);
           const float s0 = half_bits_to_float(static_cast<uint16_t>(part ? q4d >> 16 : q4d & 0xFFFFu)) * 1024.0f;
-          uint32_t o0[16];
           dq_q4_block(c0, f2_to_h2(s0, s0), o0);
-          tmem_st16(tmem + tlane + part * 16 + sa * L::a_cols, o0);
         } else {
           // part = half of the stage's 64 weights = sub-blocks 4 * (ks % 4) + 2 * part, +1 of the block
           const uint2 w = lds64s(ce + r * 80 + 16 + 16 * q + 8 * part);
           const uint32_t scb = lds16s(ce + r * 80 + 4 * q + 2 * part);
           const float d = half_bits_to_float(static_cast<uint16_t>(dq0 & 0xFFFFu));
           const float dmin = half_bits_to_float(static_cast<uint16_t>(dq0 >> 16));
-          uint32_t o0[8], o1[8];
-          dq_q2k_sub(w.x, scb & 0xFFu, d, dmin, tabQ, o0);
-          dq_q2k_sub(w.y, scb >> 8, d, dmin, tabQ, o1);
-          const uint32_t tc = tmem + tlane + part * 16 + sa * L::a_cols;
-          tmem_st8(tc, o0);
-          tmem_st8(tc + 8, o1);
+          uint32_t q0[8], q1[8];
+          dq_q2k_sub(w.x, scb & 0xFFu, d, dmin, tabQ, q0);
+          dq_q2k_sub(w.y, scb >> 8, d, dmin, tabQ, q1);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            o0[i] = q0[i];
+            o0[8 + i] = q1[i];
+          }
+        }
+        if (Q4K && !tc_wait_warp(&emptyA[sa], pha ^ 1u, a.err, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (tc_two(KIND)) {  // gate (or up) stage of the pair: 32 columns
+          const uint32_t tc = tmem + tlane + part * 32 + sa * L::a_cols;
+          tmem_st16(tc, o0);
+          tmem_st16(tc + 16, o1);
+        } else {  // half of a single matrix's stage: 16 columns
+          tmem_st16(tmem + tlane + part * 16 + sa * L::a_cols, o0);
         }
         tmem_st_wait();
         tc_fence_before();
