@@ -17,6 +17,7 @@
 //   warps 0-3   epilogue: TMEM -> registers -> SwiGLU / scaling -> global
 //   warp 4      producer: TMA loads of the token tiles (and bf16 weight tiles)
 //   warp 5      TMEM allocation; one lane issues the MMAs and commits
+//   warp 6      dequantising kinds: TMA loads of the code blocks (their own ring)
 //   warps 8-23  dequantisers: 2-bit codes -> fp16 weight tiles (128-byte swizzle),
 //               each thread one sub-block of one row per stage
 // Stages of (A tiles, B tile) circulate through full/empty mbarriers; the MMA
@@ -59,6 +60,7 @@ constexpr int kTcThreads = 768;
 constexpr int kEpiWarps = 4;     // warps 0-3
 constexpr int kProdWarp = 4;
 constexpr int kMmaWarp = 5;
+constexpr int kCodeWarp = 6;    // dequantising kinds: issues the code-block ring
 constexpr int kDqWarp0 = 8;      // warps 8-23
 constexpr int kDqWarps = 16;
 constexpr int kMT = 128;         // weight rows per tile (MMA M)
@@ -445,32 +447,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       prefetch_tmap(&tm_b);
       int s = 0;
       uint32_t ph = 0;
-      int issued = 0, c = 0, issued_c = 0;
-      uint32_t pc = 0;
+      int issued = 0;
       for (int u = blockIdx.x; u < nunits && !*abort_flag; u += gridDim.x) {
         const TcPair pr = tc_pair(a, u / a.mt);
         const int m0 = (u % a.mt) * kMT;
         if (pr.n == 0) continue;
         for (int ks = 0; ks < nks; ++ks) {
-          if (DQ && (ks & 3) == 0) {  // a new 256-weight block: its code bytes for all four stages
-            if (!tc_wait_sleepy(&emptyC[c], pc ^ 1u, a.err, abort_flag, 256)) break;
-            uint8_t* ce = smem + L::code_off + c * L::code_bytes;
-            const int wrow = pr.e * a.rows_e + m0;
-            mbar_arrive_expect_tx(&fullC[c], L::code_bytes);
-            if (KIND == TC_IQ2_PAIR) {
-              tma_load_2d(ce, &tm_a0, 64 * (ks >> 2), wrow, &fullC[c]);
-              tma_load_2d(ce + 128 * 64, &tm_a1, 64 * (ks >> 2), wrow, &fullC[c]);
-            } else if (KIND == TC_Q4_PAIR) {
-              tma_load_2d(ce, &tm_a0, 128 * (ks >> 2), wrow, &fullC[c]);
-              tma_load_2d(ce + 128 * 128, &tm_a1, 128 * (ks >> 2), wrow, &fullC[c]);
-            } else if (KIND == TC_Q4) {
-              tma_load_2d(ce, &tm_a0, 128 * (ks >> 2), wrow, &fullC[c]);
-            } else {
-              tma_load_2d(ce, &tm_a0, 80 * (ks >> 2), wrow, &fullC[c]);
-            }
-            ++issued_c;
-            if (++c == kCStages) { c = 0; pc ^= 1u; }
-          }
           if (!tc_wait_sleepy(&emptyB[s], ph ^ 1u, a.err, abort_flag, 256)) break;  // the ring runs ahead
           uint8_t* st = smem + s * L::stage_bytes;
           const int kx = (ks % ks_plane) * kKS, pl = ks / ks_plane;
@@ -492,6 +474,40 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           if (--s < 0) { s = kStages - 1; ph ^= 1u; }
           mbar_wait_bounded(&fullB[s], ph, nullptr, 0);
         }
+      }
+    }
+  } else if (DQ && warp == kCodeWarp) {
+    // the code-block ring has its own issuing lane, so a code entry that the dequantising warps release
+    // late never holds back the token tiles, which then run the whole B ring ahead of the MMAs
+    if (lane == 0) {
+      prefetch_tmap(&tm_a0);
+      int c = 0, issued_c = 0;
+      uint32_t pc = 0;
+      for (int u = blockIdx.x; u < nunits && !*abort_flag; u += gridDim.x) {
+        const TcPair pr = tc_pair(a, u / a.mt);
+        const int m0 = (u % a.mt) * kMT;
+        if (pr.n == 0) continue;
+        const int wrow = pr.e * a.rows_e + m0;
+        for (int b = 0; b < nks / 4; ++b) {  // one entry per 256-weight block: its code bytes for four stages
+          if (!tc_wait_sleepy(&emptyC[c], pc ^ 1u, a.err, abort_flag, 256)) break;
+          uint8_t* ce = smem + L::code_off + c * L::code_bytes;
+          mbar_arrive_expect_tx(&fullC[c], L::code_bytes);
+          if (KIND == TC_IQ2_PAIR) {
+            tma_load_2d(ce, &tm_a0, 64 * b, wrow, &fullC[c]);
+            tma_load_2d(ce + 128 * 64, &tm_a1, 64 * b, wrow, &fullC[c]);
+          } else if (KIND == TC_Q4_PAIR) {
+            tma_load_2d(ce, &tm_a0, 128 * b, wrow, &fullC[c]);
+            tma_load_2d(ce + 128 * 128, &tm_a1, 128 * b, wrow, &fullC[c]);
+          } else if (KIND == TC_Q4) {
+            tma_load_2d(ce, &tm_a0, 128 * b, wrow, &fullC[c]);
+          } else {
+            tma_load_2d(ce, &tm_a0, 80 * b, wrow, &fullC[c]);
+          }
+          ++issued_c;
+          if (++c == kCStages) { c = 0; pc ^= 1u; }
+        }
+      }
+      if (*abort_flag) {  // let every issued code copy land before the CTA can exit
         for (int i = 0; i < kCStages && i < issued_c; ++i) {
           if (--c < 0) { c = kCStages - 1; pc ^= 1u; }
           mbar_wait_bounded(&fullC[c], pc, nullptr, 0);
