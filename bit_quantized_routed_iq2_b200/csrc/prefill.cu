@@ -371,10 +371,15 @@ __device__ __forceinline__ TcPair tc_pair(const TcArgs& a, int i) {
   return p;
 }
 
+// Tensor maps of one launch: the B operand in boxes of 32, 64, 96 and 128 rows (a tile loads the smallest box
+// that covers its rows, so the TMA moves no rows of other tiles), and the A weight or code planes.
+struct alignas(64) TcMaps {
+  CUtensorMap b[4];
+  CUtensorMap a0, a1;
+};
+
 template <int KIND>
-__global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_b,
-                                                                const __grid_constant__ CUtensorMap tm_a0,
-                                                                const __grid_constant__ CUtensorMap tm_a1, TcArgs a) {
+__global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ TcMaps tm, TcArgs a) {
   constexpr bool PAIR = tc_two(KIND);
   constexpr bool DQ = tc_dq(KIND);
   constexpr bool Q4K = (KIND == TC_Q4_PAIR || KIND == TC_Q4);
@@ -444,7 +449,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
 
   if (warp == kProdWarp) {
     if (lane == 0) {
-      prefetch_tmap(&tm_b);
+      for (int i = 0; i < 4; ++i) prefetch_tmap(&tm.b[i]);
       int s = 0;
       uint32_t ph = 0;
       int issued = 0;
@@ -452,19 +457,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         const TcPair pr = tc_pair(a, u / a.mt);
         const int m0 = (u % a.mt) * kMT;
         if (pr.n == 0) continue;
+        const int bi = (pr.n - 1) >> 5;                                    // B box of 32 (bi + 1) rows
+        const uint32_t btx = 32u * 128u * static_cast<uint32_t>(bi + 1);  // its bytes (rows of 64 x 2 bytes)
         for (int ks = 0; ks < nks; ++ks) {
           if (!tc_wait_sleepy(&emptyB[s], ph ^ 1u, a.err, abort_flag, 256)) break;  // the ring runs ahead
           uint8_t* st = smem + s * L::stage_bytes;
           const int kx = (ks % ks_plane) * kKS, pl = ks / ks_plane;
           if (BF16) {
-            mbar_arrive_expect_tx(&fullB[s], L::stage_bytes);
+            mbar_arrive_expect_tx(&fullB[s], static_cast<uint32_t>(L::b_off) + btx);
             // the weight maps are 3-D like every map of this file (one plane)
-            tma_load_3d(st, &tm_a0, kx, pr.e * a.rows_e + m0, 0, &fullB[s]);
-            if (PAIR) tma_load_3d(st + kTile, &tm_a1, kx, pr.e * a.rows_e + m0, 0, &fullB[s]);
+            tma_load_3d(st, &tm.a0, kx, pr.e * a.rows_e + m0, 0, &fullB[s]);
+            if (PAIR) tma_load_3d(st + kTile, &tm.a1, kx, pr.e * a.rows_e + m0, 0, &fullB[s]);
           } else {
-            mbar_arrive_expect_tx(&fullB[s], L::stage_bytes);
+            mbar_arrive_expect_tx(&fullB[s], btx);
           }
-          tma_load_3d(st + L::b_off, &tm_b, kx, pr.p0, pl, &fullB[s]);
+          tma_load_3d(st + L::b_off, &tm.b[bi], kx, pr.p0, pl, &fullB[s]);
           ++issued;
           if (++s == kStages) { s = 0; ph ^= 1u; }
         }
@@ -480,7 +487,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     // the code-block ring has its own issuing lane, so a code entry that the dequantising warps release
     // late never holds back the token tiles, which then run the whole B ring ahead of the MMAs
     if (lane == 0) {
-      prefetch_tmap(&tm_a0);
+      prefetch_tmap(&tm.a0);
       int c = 0, issued_c = 0;
       uint32_t pc = 0;
       for (int u = blockIdx.x; u < nunits && !*abort_flag; u += gridDim.x) {
@@ -493,15 +500,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           uint8_t* ce = smem + L::code_off + c * L::code_bytes;
           mbar_arrive_expect_tx(&fullC[c], L::code_bytes);
           if (KIND == TC_IQ2_PAIR) {
-            tma_load_2d(ce, &tm_a0, 64 * b, wrow, &fullC[c]);
-            tma_load_2d(ce + 128 * 64, &tm_a1, 64 * b, wrow, &fullC[c]);
+            tma_load_2d(ce, &tm.a0, 64 * b, wrow, &fullC[c]);
+            tma_load_2d(ce + 128 * 64, &tm.a1, 64 * b, wrow, &fullC[c]);
           } else if (KIND == TC_Q4_PAIR) {
-            tma_load_2d(ce, &tm_a0, 128 * b, wrow, &fullC[c]);
-            tma_load_2d(ce + 128 * 128, &tm_a1, 128 * b, wrow, &fullC[c]);
+            tma_load_2d(ce, &tm.a0, 128 * b, wrow, &fullC[c]);
+            tma_load_2d(ce + 128 * 128, &tm.a1, 128 * b, wrow, &fullC[c]);
           } else if (KIND == TC_Q4) {
-            tma_load_2d(ce, &tm_a0, 128 * b, wrow, &fullC[c]);
+            tma_load_2d(ce, &tm.a0, 128 * b, wrow, &fullC[c]);
           } else {
-            tma_load_2d(ce, &tm_a0, 80 * b, wrow, &fullC[c]);
+            tma_load_2d(ce, &tm.a0, 80 * b, wrow, &fullC[c]);
           }
           ++issued_c;
           if (++c == kCStages) { c = 0; pc ^= 1u; }
@@ -955,13 +962,14 @@ PFN_cuTensorMapEncodeTiled_v12000 tc_encode_fn() {
   return fn;
 }
 
-// [planes][rows][K] 16-bit elements, box 64 (K) x 128 rows x 1 plane, 128-byte swizzle.
-bool tc_map(CUtensorMap* m, const void* base, bool bf16, uint64_t K, uint64_t rows, uint64_t planes) {
+// [planes][rows][K] 16-bit elements, box 64 (K) x box_rows rows x 1 plane, 128-byte swizzle.
+bool tc_map(CUtensorMap* m, const void* base, bool bf16, uint64_t K, uint64_t rows, uint64_t planes,
+            uint32_t box_rows = 128) {
   auto fn = tc_encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {K, rows, planes};
   const cuuint64_t strides[2] = {K * 2, K * 2 * rows};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -984,12 +992,18 @@ bool code_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t row
   return r == CUDA_SUCCESS;
 }
 
+// The four B maps (boxes of 32, 64, 96, 128 rows) over one B plane set.
+bool tc_bmaps(TcMaps* m, const void* base, bool bf16, uint64_t K, uint64_t rows, uint64_t planes) {
+  for (int i = 0; i < 4; ++i)
+    if (!tc_map(&m->b[i], base, bf16, K, rows, planes, 32u * (i + 1))) return false;
+  return true;
+}
+
 template <int KIND>
-int launch_tc(const CUtensorMap& mb, const CUtensorMap& ma0, const CUtensorMap& ma1, const TcArgs& a, int sms,
-              cudaStream_t st) {
+int launch_tc(const TcMaps& tm, const TcArgs& a, int sms, cudaStream_t st) {
   const size_t smem = TcLayout<KIND>::total;
   cudaFuncSetAttribute(tc_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  tc_gemm_kernel<KIND><<<sms, kTcThreads, smem, st>>>(mb, ma0, ma1, a);
+  tc_gemm_kernel<KIND><<<sms, kTcThreads, smem, st>>>(tm, a);
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
 }
 
@@ -1090,14 +1104,15 @@ bool router_tc_supported(int T, int H, int E) {
 
 int launch_router_tc(const uint16_t* Wr, const float* bias, const uint16_t* x, int T, int H, int E, float* logits,
                      int* err, int sms, cudaStream_t st) {
-  CUtensorMap mb, ma;
-  if (!tc_map(&mb, x, true, H, T, 1) || !tc_map(&ma, Wr, true, H, E, 1)) return ERR_CUDA;
+  TcMaps tm;
+  if (!tc_bmaps(&tm, x, true, H, T, 1) || !tc_map(&tm.a0, Wr, true, H, E, 1)) return ERR_CUDA;
+  tm.a1 = tm.a0;
   TcArgs a{};
   a.n_experts = 1; a.b_rows = T;
   a.rows_e = E; a.K = H; a.mt = E / kMT; a.planes = 1;
   a.dense_rows = T; a.bias = bias; a.out = logits; a.ldo = E; a.out_rows = T;
   a.oscale = 1.0f; a.err = err; a.clear_err = 1;
-  return launch_tc<TC_BF16>(mb, ma, ma, a, sms, st);
+  return launch_tc<TC_BF16>(tm, a, sms, st);
 }
 
 bool prefill_path_supported(const LayerShape& s, int T) {
@@ -1135,7 +1150,7 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
       bf16_parts_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const float*>(x), n, pw.xb);
     }
   }
-  CUtensorMap mb, ma0, ma1;
+  TcMaps tm;
   // routed gate/up: A = IQ2 gate/up rows (dequantised), B = expert-sorted fp16 activations
   {
     ProfScope ps(MOE_K_PREFILL_GATEUP, st);
@@ -1144,8 +1159,8 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
     const uint8_t* gc = q4 ? q4->gate_codes : w.gate_codes;
     const uint8_t* uc = q4 ? q4->up_codes : w.up_codes;
     const uint32_t cb = q4 ? 128 : 64;
-    if (!tc_map(&mb, pw.xp, false, sh.H, nA, 1) || !code_map(&ma0, gc, sh.H / 256 * cb, wrows, cb) ||
-        !code_map(&ma1, uc, sh.H / 256 * cb, wrows, cb))
+    if (!tc_bmaps(&tm, pw.xp, false, sh.H, nA, 1) || !code_map(&tm.a0, gc, sh.H / 256 * cb, wrows, cb) ||
+        !code_map(&tm.a1, uc, sh.H / 256 * cb, wrows, cb))
       return ERR_CUDA;
     TcArgs a{};
     a.n_experts = sh.E; a.b_rows = nA;
@@ -1155,30 +1170,31 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
     a.d1 = q4 ? static_cast<const uint16_t*>(q4->up_scales) : w.up_d;
     a.pairs = pw.pairs; a.npairs = pw.counts; a.out = pw.hh; a.ldo = sh.I; a.out_rows = nA;
     a.oscale = 1.0f / 1024.0f; a.err = err; a.row_exp = pw.aexp;
-    rc |= q4 ? launch_tc<TC_Q4_PAIR>(mb, ma0, ma1, a, sms, st) : launch_tc<TC_IQ2_PAIR>(mb, ma0, ma1, a, sms, st);
+    rc |= q4 ? launch_tc<TC_Q4_PAIR>(tm, a, sms, st) : launch_tc<TC_IQ2_PAIR>(tm, a, sms, st);
   }
   if (sh.Is > 0) {
     ProfScope ps(MOE_K_SHARED_GATEUP, st);
     const int planes = x_dtype == 0 ? 2 : 1;
     const void* xsrc = x_dtype == 0 ? static_cast<const void*>(pw.xb) : x;
-    if (!tc_map(&mb, xsrc, true, sh.H, T, planes) || !tc_map(&ma0, w.sh_gate, true, sh.H, sh.Is, 1) ||
-        !tc_map(&ma1, w.sh_up, true, sh.H, sh.Is, 1))
+    if (!tc_bmaps(&tm, xsrc, true, sh.H, T, planes) || !tc_map(&tm.a0, w.sh_gate, true, sh.H, sh.Is, 1) ||
+        !tc_map(&tm.a1, w.sh_up, true, sh.H, sh.Is, 1))
       return ERR_CUDA;
     TcArgs a{};
     a.n_experts = 1; a.b_rows = T;
     a.rows_e = sh.Is; a.K = sh.H; a.mt = sh.Is / kMT; a.planes = planes;
     a.dense_rows = T; a.out = pw.hs; a.ldo = sh.Is; a.out_rows = T;
     a.oscale = 1.0f; a.err = err;
-    rc |= launch_tc<TC_BF16_PAIR>(mb, ma0, ma1, a, sms, st);
+    rc |= launch_tc<TC_BF16_PAIR>(tm, a, sms, st);
   }
   {
     ProfScope ps(MOE_K_PREFILL_DOWN, st);
     // Q2K: 80 code bytes per 256 weights; Q4-style: 128
     const uint8_t* dc = q4 ? q4->down_codes : w.down_codes;
     const uint32_t cb = q4 ? 128 : 80;
-    if (!tc_map(&mb, pw.hh, false, sh.I, nA, 1) ||
-        !code_map(&ma0, dc, static_cast<uint64_t>(sh.I / 256) * cb, static_cast<uint64_t>(sh.E) * sh.H, cb))
+    if (!tc_bmaps(&tm, pw.hh, false, sh.I, nA, 1) ||
+        !code_map(&tm.a0, dc, static_cast<uint64_t>(sh.I / 256) * cb, static_cast<uint64_t>(sh.E) * sh.H, cb))
       return ERR_CUDA;
+    tm.a1 = tm.a0;
     TcArgs a{};
     a.n_experts = sh.E; a.b_rows = nA;
     a.rows_e = sh.H; a.K = sh.I; a.mt = sh.H / kMT; a.planes = 1;
@@ -1186,17 +1202,18 @@ int launch_ffn_prefill(const LayerShape& sh, const WeightPtrs& w, const void* x,
     if (q4) a.d0 = static_cast<const uint16_t*>(q4->down_scales);
     a.pairs = pw.pairs; a.npairs = pw.counts; a.out = pw.o; a.ldo = sh.H; a.out_rows = nA;
     a.oscale = q4 ? 1.0f / 1024.0f : 1.0f; a.err = err; a.row_exp = pw.aexp;
-    rc |= q4 ? launch_tc<TC_Q4>(mb, ma0, ma0, a, sms, st) : launch_tc<TC_Q2K>(mb, ma0, ma0, a, sms, st);
+    rc |= q4 ? launch_tc<TC_Q4>(tm, a, sms, st) : launch_tc<TC_Q2K>(tm, a, sms, st);
   }
   if (sh.Is > 0) {
     ProfScope ps(MOE_K_SHARED_DOWN, st);
-    if (!tc_map(&mb, pw.hs, true, sh.Is, T, 2) || !tc_map(&ma0, w.sh_down, true, sh.Is, sh.H, 1)) return ERR_CUDA;
+    if (!tc_bmaps(&tm, pw.hs, true, sh.Is, T, 2) || !tc_map(&tm.a0, w.sh_down, true, sh.Is, sh.H, 1)) return ERR_CUDA;
+    tm.a1 = tm.a0;
     TcArgs a{};
     a.n_experts = 1; a.b_rows = T;
     a.rows_e = sh.H; a.K = sh.Is; a.mt = sh.H / kMT; a.planes = 2;
     a.dense_rows = T; a.out = pw.s; a.ldo = sh.H; a.out_rows = T;
     a.oscale = 1.0f; a.err = err;
-    rc |= launch_tc<TC_BF16>(mb, ma0, ma0, a, sms, st);
+    rc |= launch_tc<TC_BF16>(tm, a, sms, st);
   }
   {
     ProfScope ps(MOE_K_COMBINE, st);
@@ -1226,30 +1243,31 @@ int launch_prefill_shared(const LayerShape& sh, const uint16_t* wg, const uint16
     ProfScope ps(MOE_K_PREP, st);
     bf16_parts_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const float*>(x), static_cast<size_t>(T) * sh.H, xb);
   }
-  CUtensorMap mb, ma0, ma1;
+  TcMaps tm;
   {
     ProfScope ps(MOE_K_SHARED_GATEUP, st);
     const int planes = x_dtype == 0 ? 2 : 1;
     const void* xsrc = x_dtype == 0 ? static_cast<const void*>(xb) : x;
-    if (!tc_map(&mb, xsrc, true, sh.H, T, planes) || !tc_map(&ma0, wg, true, sh.H, sh.Is, 1) ||
-        !tc_map(&ma1, wu, true, sh.H, sh.Is, 1))
+    if (!tc_bmaps(&tm, xsrc, true, sh.H, T, planes) || !tc_map(&tm.a0, wg, true, sh.H, sh.Is, 1) ||
+        !tc_map(&tm.a1, wu, true, sh.H, sh.Is, 1))
       return ERR_CUDA;
     TcArgs a{};
     a.n_experts = 1; a.b_rows = T;
     a.rows_e = sh.Is; a.K = sh.H; a.mt = sh.Is / kMT; a.planes = planes;
     a.dense_rows = T; a.out = hs; a.ldo = sh.Is; a.out_rows = T;
     a.oscale = 1.0f; a.err = err;
-    rc |= launch_tc<TC_BF16_PAIR>(mb, ma0, ma1, a, sms, st);
+    rc |= launch_tc<TC_BF16_PAIR>(tm, a, sms, st);
   }
   {
     ProfScope ps(MOE_K_SHARED_DOWN, st);
-    if (!tc_map(&mb, hs, true, sh.Is, T, 2) || !tc_map(&ma0, wd, true, sh.Is, sh.H, 1)) return ERR_CUDA;
+    if (!tc_bmaps(&tm, hs, true, sh.Is, T, 2) || !tc_map(&tm.a0, wd, true, sh.Is, sh.H, 1)) return ERR_CUDA;
+    tm.a1 = tm.a0;
     TcArgs a{};
     a.n_experts = 1; a.b_rows = T;
     a.rows_e = sh.H; a.K = sh.Is; a.mt = sh.H / kMT; a.planes = 2;
     a.dense_rows = T; a.out = s_out; a.ldo = sh.H; a.out_rows = T;
     a.oscale = 1.0f; a.err = err;
-    rc |= launch_tc<TC_BF16>(mb, ma0, ma0, a, sms, st);
+    rc |= launch_tc<TC_BF16>(tm, a, sms, st);
   }
   if (rc != OK) return ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
