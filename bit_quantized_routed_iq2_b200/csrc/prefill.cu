@@ -889,8 +889,14 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(const XT* __restrict_
       v[4] = __uint_as_float(w.z << 16); v[5] = __uint_as_float(w.z & 0xFFFF0000u);
       v[6] = __uint_as_float(w.w << 16); v[7] = __uint_as_float(w.w & 0xFFFF0000u);
     }
+    if (ex >= -127 && ex <= 126) {  // 2^-ex is a normal float: one rounding, the value ldexpf gives
+      const float sc = __int_as_float((127 - ex) << 23);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) v[q] = ldexpf(v[q], -ex);
+      for (int q = 0; q < 8; ++q) v[q] *= sc;
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = ldexpf(v[q], -ex);
+    }
     uint4 o;
     o.x = f2_to_h2(v[0], v[1]);
     o.y = f2_to_h2(v[2], v[3]);

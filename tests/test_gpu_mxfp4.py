@@ -254,3 +254,39 @@ def test_q4_prefill_shape_sampled(torch_cuda):
     assert rows.size == 5
     ref, _, _ = oracle.layer_forward(lw, x[rows])
     assert normwise(y[rows], ref) <= FFN_TOL, normwise(y[rows], ref)
+
+
+def test_mxfp4_many_tokens_need_32_byte_code_planes(torch_cuda):
+    """Above 16 tokens the unpacking copy of the FP4 codes needs 32-byte plane bases: a plane that is 16-byte
+    but not 32-byte aligned is rejected on the host (MOE_ERR_INVALID_ARG) before anything is enqueued, while
+    the one-token GEMVs accept it and give the same result as the aligned plane."""
+    torch = torch_cuda
+    import ctypes
+
+    cfg = synth.Config("mx_align", 40, 1024, 512, 8, 2, 0, "bf16", 1.0, False, 1, 0x4D4131)
+    lw = synth.make_layer_mxfp4(cfg)
+    dl = moe2bit.to_device_mxfp4(lw)
+    g = dl.tensors["gate_codes"]
+    buf = torch.empty(g.numel() + 64, dtype=torch.uint8, device="cuda")
+    off = (32 - buf.data_ptr() % 32) % 32 + 16  # 16 (mod 32)
+    shifted = buf[off:off + g.numel()]
+    shifted.copy_(g.reshape(-1))
+    assert shifted.data_ptr() % 32 == 16
+    x = screened_x(cfg, lw)
+    xd = _x_dev(torch, x)
+    y = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
+    ws = moe2bit.alloc_workspace_mxfp4(dl.desc, cfg.T)
+    w = dl.weights
+    w.gate_codes = shifted.data_ptr()
+    L = moe2bit.load()
+    rc = L.moe_layer_forward_mxfp4(ctypes.byref(dl.desc), ctypes.byref(w), xd.data_ptr(), 1, cfg.T, None,
+                                   y.data_ptr(), ws.data_ptr(), ws.numel(), None)
+    assert rc == 1  # MOE_ERR_INVALID_ARG
+    # one token: the GEMVs take the 16-byte aligned plane
+    y1 = torch.empty((1, cfg.H), dtype=torch.float32, device="cuda")
+    y2 = torch.empty((1, cfg.H), dtype=torch.float32, device="cuda")
+    assert L.moe_layer_forward_mxfp4(ctypes.byref(dl.desc), ctypes.byref(w), xd.data_ptr(), 1, 1, None,
+                                     y1.data_ptr(), ws.data_ptr(), ws.numel(), None) == 0
+    moe2bit.layer_forward_mxfp4(dl, xd[:1], None, y2, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
