@@ -525,6 +525,7 @@ __global__ void __launch_bounds__(1024) topk_permute_sort_kernel(const float* __
       const float mv = cv[c];
       const int mi = ci[c];
       int rank = 0;
+#pragma unroll 8
       for (int j = 0; j < nc; ++j) rank += ranks_before(cv[j], ci[j], mv, mi) ? 1 : 0;
       if (rank < k) {
         sel[ct * k + rank] = mi;
@@ -533,20 +534,21 @@ __global__ void __launch_bounds__(1024) topk_permute_sort_kernel(const float* __
     }
   }
   __syncthreads();
-  // exp(l_j - l_0) of every chosen slot at once, then the sum in slot order by one thread per token
+  // exp(l_j - l_0) of every chosen slot at once; then each slot's thread forms its token's sum in slot
+  // order (the same sum in every thread of the token) and writes its own weight
   if (tid < n) ex[tid] = expf(chosen[tid] - chosen[(tid / k) * k]);
   __syncthreads();
-  if (tid < T) {
+  if (tid < n) {
+    const int t0 = (tid / k) * k;
     float z = 0.f;
-    for (int j = 0; j < k; ++j) z += ex[tid * k + j];
-    for (int j = 0; j < k; ++j) {
-      topk_idx[tid * k + j] = sel[tid * k + j];
-      topk_w[tid * k + j] = ex[tid * k + j] / z;
-    }
+    for (int j = 0; j < k; ++j) z += ex[t0 + j];
+    topk_idx[tid] = sel[tid];
+    topk_w[tid] = ex[tid] / z;
   }
   if (tid < n) {
     const int ej = sel[tid];
     int below = 0, fst = 1;
+#pragma unroll 8
     for (int j = 0; j < n; ++j) {
       const int ei = sel[j];
       below += (ei < ej || (ei == ej && j < tid)) ? 1 : 0;
@@ -559,17 +561,20 @@ __global__ void __launch_bounds__(1024) topk_permute_sort_kernel(const float* __
   __syncthreads();
   for (int x = tid; x <= E; x += blockDim.x) {
     int lt = 0;
+#pragma unroll 8
     for (int j = 0; j < n; ++j) lt += sel[j] < x ? 1 : 0;
     offsets[x] = x == E ? n : lt;
   }
   if (tid < n && first[tid]) {
     const int ej = sel[tid];
     int pos = 0;
+#pragma unroll 8
     for (int j = 0; j < n; ++j) pos += (first[j] && sel[j] < ej) ? 1 : 0;
     active[pos] = ej;
   }
   if (tid == 0) {
     int nact = 0;
+#pragma unroll 8
     for (int j = 0; j < n; ++j) nact += first[j];
     active[E] = nact;
   }
