@@ -289,7 +289,9 @@ def measure(args, cfg, world, rank, local, steps):
     y = torch.empty((T, cfg.H), dtype=torch.float32, device="cuda")
     ws = moe2bit.alloc_workspace(layers[0].desc, T)
     stream = torch.cuda.current_stream()
-    xa = torch.empty((T, cfg.H), dtype=torch.bfloat16, device="cuda") if is_stack else None
+    # the next layer's bf16 input, written by the library beside y (two buffers: a layer's output may not
+    # overlap its own input)
+    xa = [torch.empty((T, cfg.H), dtype=torch.bfloat16, device="cuda") for _ in range(2)] if is_stack else None
 
     side = torch.cuda.Stream() if is_stack else None
 
@@ -302,10 +304,9 @@ def measure(args, cfg, world, rank, local, steps):
             if l + 1 < len(layers):
                 side.wait_stream(st)
                 moe2bit.prefetch_layer(layers[l + 1], side)
-            moe2bit.layer_forward(dl, cur, res if l == 0 else yo, yo, ws, st)
-            with torch.cuda.stream(st):
-                xa.copy_(yo)  # next layer input = bf16 of the residual stream
-            cur = xa
+            nxt = xa[l % 2] if l + 1 < len(layers) else None  # bf16 of the residual stream, for layer l + 1
+            moe2bit.layer_forward(dl, cur, res if l == 0 else yo, yo, ws, st, y_next=nxt)
+            cur = nxt
         st.wait_stream(side)
 
     if is_stack:

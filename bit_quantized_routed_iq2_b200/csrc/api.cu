@@ -214,9 +214,17 @@ moe_status moe_expert_ffn(const moe_layer_desc* desc, const moe_layer_weights* w
       launch_ffn(shape_of(desc), weights_of(weights), x, x_dtype, T, r, residual, y, w.ffn, w.status, true, s));
 }
 
-moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights* weights, const void* x,
-                             moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws,
-                             size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+  return pa < pb + nb && pb < pa + na;
+}
+
+moe_status layer_forward_impl(const moe_layer_desc* desc, const moe_layer_weights* weights, const void* x,
+                              moe_dtype x_dtype, int32_t T, const float* residual, float* y, uint16_t* y_next,
+                              void* ws, size_t ws_bytes, void* stream) {
   moe_status st = check_desc(desc);
   if (st != MOE_OK) return st;
   if ((st = check_tokens(desc, T)) != MOE_OK) return st;
@@ -229,8 +237,16 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights
   for (const void* p : req)
     if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
   if (residual && !aligned16(residual)) return MOE_ERR_INVALID_ARG;
+  if (y_next) {  // written while x, y and the residual are still read: no overlap with any of them
+    const size_t n = static_cast<size_t>(T) * desc->hidden;
+    const size_t xb = n * (x_dtype == MOE_F32 ? 4 : 2);
+    if (!aligned16(y_next) || overlaps(y_next, 2 * n, x, xb) || overlaps(y_next, 2 * n, y, 4 * n) ||
+        (residual && overlaps(y_next, 2 * n, residual, 4 * n)))
+      return MOE_ERR_INVALID_ARG;
+  }
   RouteWs w = carve(desc, T, ws);
   if (ws_bytes < w.bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (y_next && overlaps(y_next, static_cast<size_t>(T) * desc->hidden * 2, ws, w.bytes)) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the shared expert does not depend on routing: its gate/up starts first, on a side stream. Once the
   // fork may have been recorded, every return joins the side stream back (a capture in progress needs
@@ -248,10 +264,26 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights
     // expert and the digits run ahead on the side stream, the tensor-core router for many bf16 tokens
     const bool routed_clears = x_dtype == MOE_BF16 && router_tc_supported(T, desc->hidden, desc->n_experts);
     rc = launch_ffn(shape_of(desc), weights_of(weights), x, x_dtype, T, r, residual, y, w.ffn, w.status,
-                    !routed_clears && !early, s, early);
+                    !routed_clears && !early, s, early, y_next);
   }
   if (rc != OK && early) join_shared_early(s);
   return to_status(rc);
+}
+}  // namespace
+
+extern "C" {
+
+moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights* weights, const void* x,
+                             moe_dtype x_dtype, int32_t T, const float* residual, float* y, void* ws,
+                             size_t ws_bytes, void* stream) {
+  return layer_forward_impl(desc, weights, x, x_dtype, T, residual, y, nullptr, ws, ws_bytes, stream);
+}
+
+moe_status moe_layer_forward_next(const moe_layer_desc* desc, const moe_layer_weights* weights, const void* x,
+                                  moe_dtype x_dtype, int32_t T, const float* residual, float* y, uint16_t* y_next,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  if (!y_next && T > 0) return MOE_ERR_INVALID_ARG;
+  return layer_forward_impl(desc, weights, x, x_dtype, T, residual, y, y_next, ws, ws_bytes, stream);
 }
 
 moe_status moe_prefetch_layer(const moe_layer_desc* desc, const moe_layer_weights* weights, void* stream) {

@@ -367,12 +367,14 @@ __global__ void __launch_bounds__(256) shared_down_combine_kernel(int H, int Is,
 // and ys the shared expert's output computed beforehand. One thread per (t, r);
 // the assignments are taken eight at a time with all their routing words, then
 // all their partial rows, requested before any is added, so a thread waits for
-// memory once per eight assignments rather than twice per assignment.
+// memory once per eight assignments rather than twice per assignment. With yb,
+// the same value rounded to bf16 (nearest, ties to even) is stored there too:
+// the next layer's input.
 __global__ void __launch_bounds__(256) combine_routed_kernel(int H, int k, const float* __restrict__ topk_w,
                                                              const int32_t* __restrict__ inv,
                                                              const float* __restrict__ obuf, int DP,
                                                              const float* __restrict__ ys, const float* residual,
-                                                             float* y) {
+                                                             float* y, uint16_t* __restrict__ yb) {
   constexpr int JC = 8, DC = 8;
   pdl_trigger();
   pdl_wait();  // the routed partials come from the kernel before this one
@@ -413,6 +415,22 @@ __global__ void __launch_bounds__(256) combine_routed_kernel(int H, int k, const
   v += ys[i];
   if (residual) v += residual[i];
   y[i] = v;
+  if (yb) yb[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+// yb[i] = bf16(y[i]) (nearest, ties to even) for the paths whose last kernel
+// does not write the bf16 copy itself; n a multiple of 4, both 16-byte aligned.
+__global__ void __launch_bounds__(256) y_to_bf16_kernel(const float* __restrict__ y, uint16_t* __restrict__ yb,
+                                                        size_t n4) {
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 v = reinterpret_cast<const float4*>(y)[i];
+    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(v.x)) |
+                        (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
+    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(v.z)) |
+                        (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.w))) << 16);
+    reinterpret_cast<uint2*>(yb)[i] = make_uint2(lo, hi);
+  }
 }
 
 // ------------------------------------------------------------ launcher
@@ -630,7 +648,7 @@ int launch_shared_early(const LayerShape& s, const WeightPtrs& w, const void* x,
 
 int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
                     const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st,
-                    bool shared_early) {
+                    bool shared_early, uint16_t* y_bf16) {
   const size_t nA = static_cast<size_t>(T) * s.k;
   const bool tma = tma_shape(s, T) && tma_path_supported(s, T);
   const int KP = tma ? tma_gu_parts(s, T) : 1, DP = tma ? tma_dn_parts(s, T) : 1;
@@ -727,7 +745,7 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
     ProfScope ps(MOE_K_COMBINE, st);
     launch_pdl(combine_routed_kernel, dim3((s.H + 255) / 256, T), dim3(256), 0, st, s.H, s.k,
                static_cast<const float*>(r.topk_w), static_cast<const int32_t*>(r.inv),
-               static_cast<const float*>(obuf), DP, static_cast<const float*>(fw.ysh), residual, y);
+               static_cast<const float*>(obuf), DP, static_cast<const float*>(fw.ysh), residual, y, y_bf16);
   } else if (sh_mma) {
     ProfScope ps(MOE_K_COMBINE, st);
     rc |= launch_shared_down_combine_mma(s.H, s.Is, w.sh_down, fw.hb, T, s.k, r.topk_w, r.inv, obuf, DP, residual, y,
@@ -738,7 +756,17 @@ int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int
     shared_down_combine_kernel<8><<<grid, 256, 0, st>>>(s.H, s.Is, s.k, s.Is > 0 ? w.sh_down : nullptr, hsh, T,
                                                         r.topk_w, r.inv, obuf, DP, residual, y);
   }
+  if (y_bf16 && !shared_early) rc |= launch_y_to_bf16(y, y_bf16, static_cast<size_t>(T) * s.H, st);
   if (rc != OK) return ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
+}
+
+int launch_y_to_bf16(const float* y, uint16_t* yb, size_t n, cudaStream_t st) {
+  const size_t n4 = n / 4;
+  if (n4 == 0) return OK;
+  ProfScope ps(MOE_K_COMBINE, st);
+  const int grid = static_cast<int>(std::min<size_t>((n4 + 255) / 256, static_cast<size_t>(num_sms()) * 8));
+  y_to_bf16_kernel<<<grid, 256, 0, st>>>(y, yb, n4);
   return cudaGetLastError() == cudaSuccess ? OK : ERR_CUDA;
 }
 
@@ -803,7 +831,8 @@ int launch_ffn_mxfp4(const LayerShape& s, const WeightPtrs& shw, const MxPlanes&
     ProfScope ps(MOE_K_COMBINE, st);
     launch_pdl(combine_routed_kernel, dim3((s.H + 255) / 256, T), dim3(256), 0, st, s.H, s.k,
                static_cast<const float*>(r.topk_w), static_cast<const int32_t*>(r.inv),
-               static_cast<const float*>(fw.obuf), DP, static_cast<const float*>(fw.ysh), residual, y);
+               static_cast<const float*>(fw.obuf), DP, static_cast<const float*>(fw.ysh), residual, y,
+               static_cast<uint16_t*>(nullptr));
   } else {
     // the shared expert here, then its down projection fused with the combine
     const int xparts = x_dtype == 0 ? 2 : 1;

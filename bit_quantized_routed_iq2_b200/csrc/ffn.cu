@@ -296,16 +296,20 @@ static int launch_ffn_simple(const LayerShape& s, const WeightPtrs& w, const voi
 
 int launch_ffn(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
                const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st,
-               bool shared_early) {
+               bool shared_early, uint16_t* y_bf16) {
+  if (fast_path_supported(s) && !use_prefill(s, T))
+    return launch_ffn_fast(s, w, x, x_dtype, T, r, residual, y, ws, err, clear_status, st, shared_early, y_bf16);
+  int rc;
   if (use_prefill(s, T)) {
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return launch_ffn_prefill(s, w, x, x_dtype, T, r, residual, y, ws, err, clear_status, sms > 0 ? sms : 148, st);
+    rc = launch_ffn_prefill(s, w, x, x_dtype, T, r, residual, y, ws, err, clear_status, sms > 0 ? sms : 148, st);
+  } else {
+    rc = launch_ffn_simple(s, w, x, x_dtype, T, r, residual, y, ws, st);
   }
-  if (fast_path_supported(s))
-    return launch_ffn_fast(s, w, x, x_dtype, T, r, residual, y, ws, err, clear_status, st, shared_early);
-  return launch_ffn_simple(s, w, x, x_dtype, T, r, residual, y, ws, st);
+  if (rc == OK && y_bf16) rc = launch_y_to_bf16(y, y_bf16, static_cast<size_t>(T) * s.H, st);
+  return rc;
 }
 
 int launch_debug_dequant_iq2(const uint8_t* codes, const uint16_t* d, int64_t nblocks, float* out, cudaStream_t st) {

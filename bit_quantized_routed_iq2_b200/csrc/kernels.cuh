@@ -44,10 +44,14 @@ int launch_remap_permute(int32_t* ids, int n, const int32_t* map, int E, int32_t
 // Workspace needed by the FFN stage for T tokens (bytes) and the launcher.
 size_t ffn_workspace_bytes(const LayerShape& s, int T);
 // clear_status: the FFN's first kernel clears *err (false when an earlier
-// kernel of the same call already did).
+// kernel of the same call already did). y_bf16 (optional, [T][H]): also store
+// bf16(y), rounded to nearest even, by the combine kernel where it can, else by
+// a cast kernel after it.
 int launch_ffn(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
                const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st,
-               bool shared_early = false);
+               bool shared_early = false, uint16_t* y_bf16 = nullptr);
+// yb = bf16(y) elementwise (nearest, ties to even); n a multiple of 4, both 16-byte aligned (decode.cu).
+int launch_y_to_bf16(const float* y, uint16_t* yb, size_t n, cudaStream_t st);
 
 // L2 prefetch (evict_last) of up to four device ranges (decode.cu).
 int launch_l2_prefetch(const void* const* ptrs, const size_t* bytes, int n, cudaStream_t st);
@@ -59,7 +63,7 @@ bool use_prefill(const LayerShape& s, int T);
 size_t fast_ffn_workspace_bytes(const LayerShape& s, int T);
 int launch_ffn_fast(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dtype, int T, const Routing& r,
                     const float* residual, float* y, void* ws, int* err, bool clear_status, cudaStream_t st,
-                    bool shared_early = false);
+                    bool shared_early = false, uint16_t* y_bf16 = nullptr);
 
 // TMA-fed GEMVs (gemv_tma.cu).
 bool tma_path_supported(const LayerShape& s, int T);

@@ -35,7 +35,7 @@ EXPORTS = (
     "moe_prefetch_layer", "moe_debug_bounds_check_build", "moe_debug_bounds_violations",
     "moe_cache_bytes", "moe_cache_create", "moe_cache_destroy", "moe_cache_read_stats", "moe_layer_forward_cached",
     "moe_workspace_size_mxfp4", "moe_layer_forward_mxfp4", "moe_debug_dequant_mxfp4",
-    "moe_workspace_size_q4", "moe_layer_forward_q4", "moe_debug_dequant_q4",
+    "moe_workspace_size_q4", "moe_layer_forward_q4", "moe_debug_dequant_q4", "moe_layer_forward_next",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 KERNEL_NAMES = ("router_logits", "topk", "permute", "active", "gateup", "down", "shared_gateup", "shared_down",
@@ -94,6 +94,7 @@ def load() -> ctypes.CDLL:
     L.moe_route.argtypes = [pd, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moe_expert_ffn.argtypes = [pd, pw, vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moe_layer_forward.argtypes = [pd, pw, vp, i32, i32, vp, vp, vp, sz, vp]
+    L.moe_layer_forward_next.argtypes = [pd, pw, vp, i32, i32, vp, vp, vp, vp, sz, vp]
     L.moe_status_string.argtypes = [i32]
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_debug_dequant_iq2.argtypes = [vp, vp, i64, vp, vp]
@@ -306,12 +307,19 @@ def expert_ffn(layer: DeviceLayer, x, topk_w, offsets, perm, inv, residual, y, w
                                  _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "moe_expert_ffn")
 
 
-def layer_forward(layer: DeviceLayer, x, residual, y, ws, stream=None):
+def layer_forward(layer: DeviceLayer, x, residual, y, ws, stream=None, y_next=None):
+    """moe_layer_forward; with y_next (bf16 [T][H]) moe_layer_forward_next, which also writes bf16(y) there."""
     T = x.shape[0]
     w = layer.weights
-    _check(load().moe_layer_forward(ctypes.byref(layer.desc), ctypes.byref(w), _ptr(x), _dtype_of(x), T,
-                                    _ptr(residual), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
-                                    _stream(stream)), "moe_layer_forward")
+    if y_next is None:
+        _check(load().moe_layer_forward(ctypes.byref(layer.desc), ctypes.byref(w), _ptr(x), _dtype_of(x), T,
+                                        _ptr(residual), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
+                                        _stream(stream)), "moe_layer_forward")
+    else:
+        _check(load().moe_layer_forward_next(ctypes.byref(layer.desc), ctypes.byref(w), _ptr(x), _dtype_of(x), T,
+                                             _ptr(residual), _ptr(y), _ptr(y_next), _ptr(ws),
+                                             ws.numel() * ws.element_size(), _stream(stream)),
+               "moe_layer_forward_next")
 
 
 def prefetch_layer(layer: DeviceLayer, stream=None):

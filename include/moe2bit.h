@@ -186,6 +186,25 @@ MOE_API moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer
                              size_t ws_bytes, void* stream);
 
 /*
+ * moe_layer_forward that also hands the next layer its input: besides the fp32
+ * y (the residual stream), y_next[t][h] = bf16(y[t][h]), rounded to nearest
+ * with ties to even. Chained layers keep the residual stream in fp32 and take
+ * its bf16 rounding as their input (the pages chain the MoE layers without
+ * naming the formats; this is the library's reading), and with this call that
+ * rounding is the library's own work rather than a cast by the caller.
+ * Same arguments, workspace and results as moe_layer_forward, plus
+ * y_next: device bf16 [T][H] (uint16 bit patterns), 16-byte aligned, required
+ * (MOE_ERR_INVALID_ARG when NULL and T > 0), overlapping none of x, y,
+ * residual or the workspace (MOE_ERR_INVALID_ARG otherwise; a chain of layers
+ * alternates two input buffers). On the decode path with bf16 x (T <= 16) the
+ * combine kernel stores both outputs; on the other paths a cast kernel runs
+ * after the combine.
+ */
+MOE_API moe_status moe_layer_forward_next(const moe_layer_desc* desc, const moe_layer_weights* w, const void* x,
+                                          moe_dtype x_dtype, int32_t T, const float* residual, float* y,
+                                          uint16_t* y_next, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * The whole layer without any caller-provided scratch: same arguments and
  * results as moe_layer_forward, minus `ws` / `ws_bytes`. (The ds4 pages have
  * no counterpart of this call; it exists for callers of this library that

@@ -85,3 +85,12 @@ def elementwise(a: np.ndarray, ref: np.ndarray, floor_frac: float = 1e-3) -> flo
         return 0.0
     fl = floor_frac * float(np.max(np.abs(ref)))
     return float(np.max(np.abs(a - ref) / (np.abs(ref) + fl))) if fl > 0 else float(np.max(np.abs(a - ref)))
+
+
+def bf16_rne_bits(y: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns of finite fp32 values, rounded to nearest with ties to even: add 0x7FFF plus the
+    lowest kept bit to the fp32 bits, then drop the low 16 bits (a carry into the exponent is the correct
+    rounding up to the next binade, or to infinity)."""
+    assert np.all(np.isfinite(y))
+    u = np.ascontiguousarray(y, np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)

@@ -95,6 +95,30 @@ def test_misaligned_and_small_workspace_rejected(lib):
     assert lib.moe_layer_forward(ctypes.byref(d), ctypes.byref(w), fake, 1, 1, None, fake, fake, need - 1, None) == 3
 
 
+def test_next_layer_output_validated_on_host(lib):
+    # moe_layer_forward_next: y_next is required, 16-byte aligned and disjoint from x, y, residual and the
+    # workspace; every case below fails validation before anything is enqueued
+    d = moe2bit.desc_of(**DECODE)
+    base = 1 << 40
+    w = moe2bit.Weights(*([base] * 11))
+    need = moe2bit.workspace_size(d, 1)
+    x, y, ws, res = base, base + (1 << 30), base + (1 << 31), base + (3 << 30)
+    f = lib.moe_layer_forward_next
+
+    def call(y_next, residual=None):
+        return f(ctypes.byref(d), ctypes.byref(w), x, 1, 1, residual, y, y_next, ws, need, None)
+
+    assert call(None) == 1
+    assert call(x) == 1                                   # the input itself
+    assert call(x + 2 * d.hidden - 16) == 1               # the input's last 16 bytes
+    assert call(y + 16) == 1                              # inside y
+    assert call(res, residual=res) == 1                   # the residual
+    assert call(ws + 4096) == 1                           # inside the workspace
+    assert call(base + (1 << 32) + 8) == 1                # misaligned
+    # T = 0 is a no-op for every entry point, y_next included
+    assert f(ctypes.byref(d), ctypes.byref(w), x, 1, 0, None, y, None, ws, need, None) == 0
+
+
 def test_status_query_and_injection_validate_on_host(lib):
     """The status query and the fault-injection switch reject bad arguments
     without touching a device; injection mode 0 is plain host state."""
