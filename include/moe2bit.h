@@ -196,9 +196,10 @@ MOE_API moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer
  * y_next: device bf16 [T][H] (uint16 bit patterns), 16-byte aligned, required
  * (MOE_ERR_INVALID_ARG when NULL and T > 0), overlapping none of x, y,
  * residual or the workspace (MOE_ERR_INVALID_ARG otherwise; a chain of layers
- * alternates two input buffers). On the decode path with bf16 x (T <= 16) the
- * combine kernel stores both outputs; on the other paths a cast kernel runs
- * after the combine.
+ * alternates two input buffers). On the decode path with bf16 x and a shared
+ * expert (T <= 16, the shared expert on the side stream) the routed combine
+ * kernel stores both outputs; on the other paths a cast kernel runs after the
+ * combine.
  */
 MOE_API moe_status moe_layer_forward_next(const moe_layer_desc* desc, const moe_layer_weights* w, const void* x,
                                           moe_dtype x_dtype, int32_t T, const float* residual, float* y,
