@@ -306,6 +306,9 @@ int launch_ffn(const LayerShape& s, const WeightPtrs& w, const void* x, int x_dt
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     rc = launch_ffn_prefill(s, w, x, x_dtype, T, r, residual, y, ws, err, clear_status, sms > 0 ? sms : 148, st);
   } else {
+    // the plain kernels have no bounded waits and never write the status word: clear it here, as the first
+    // kernel of every other path does
+    if (clear_status && err && cudaMemsetAsync(err, 0, sizeof(int), st) != cudaSuccess) return ERR_CUDA;
     rc = launch_ffn_simple(s, w, x, x_dtype, T, r, residual, y, ws, st);
   }
   if (rc == OK && y_bf16) rc = launch_y_to_bf16(y, y_bf16, static_cast<size_t>(T) * s.H, st);

@@ -70,3 +70,25 @@ def test_status_is_clear_after_normal_calls(torch_cuda):
         ws.fill_(0xA5)  # a stale word from an earlier user of the memory must not survive the call
         moe2bit.layer_forward(dl, _x_dev(torch, x), None, y, ws)
         assert moe2bit.read_status(ws) == 0, T
+
+
+def test_status_is_clear_after_the_plain_path(torch_cuda):
+    # shapes with I below 256 (the tiny configuration, fp32 x) run the plain kernels, which have no bounded
+    # waits; the call must still clear a stale status word, through both layer entry points
+    torch = torch_cuda
+    cfg = synth.CONFIGS["tiny"]
+    lw = synth.make_layer(cfg)
+    x = screened_x(cfg, lw)
+    dl = moe2bit.to_device(lw)
+    xd = torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    y = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
+    ws = moe2bit.alloc_workspace(dl.desc, cfg.T)
+    ws.fill_(0xA5)
+    moe2bit.layer_forward(dl, xd, None, y, ws)
+    assert moe2bit.read_status(ws) == 0
+    ws.fill_(0xA5)
+    yb = torch.empty((cfg.T, cfg.H), dtype=torch.int16, device="cuda")
+    moe2bit.layer_forward(dl, xd, None, y, ws, y_next=yb)
+    assert moe2bit.read_status(ws) == 0
+    ref, _, _ = oracle.layer_forward(lw, x)
+    assert normwise(y.cpu().numpy(), ref) <= FFN_TOL
