@@ -983,80 +983,91 @@ __device__ __forceinline__ bool dn_unit_one(const DnTmaArgs& a, const DnCtx& c, 
   return true;
 }
 
-// One down unit for an expert with 2..2*MAXQ assignments. Each MMA takes a pair
-// of sub-blocks (2pr, 2pr + 1), lane tig bit pair tig of their bytes; MMA
-// columns: (token slot 0..1) x (half 0..1) x (digit hi, lo).
+// One down unit for an expert with 2..2*MAXQ assignments, taken four at a time.
+// Each sub-block's 4-bit scale sc is folded into its uint8 A operand: sc * q is
+// at most 45, so the 32-bit product of the four q bytes with sc carries nothing
+// from byte to byte. An MMA then spans two whole sub-blocks (K 0..15: sub-block
+// 2pr, K 16..31: 2pr + 1, lane tig bit pair tig of their bytes) and its
+// accumulators sum sc * q * h over the whole block, with no scaling per MMA.
+// MMA columns: (assignment slot 0..3) x (digit hi, lo), so lane tig's
+// accumulators hold slot tig's two digits for rows g and g + 8. The min term
+// sums m * (per-16 sum of h) over the block's sub-blocks per row and slot.
 template <int MAXQ, bool HS>
 __device__ __forceinline__ bool dn_unit_multi(const DnTmaArgs& a, const DnCtx& c, RingPos& rp, const DnUnit& w,
                                               const uint32_t (&dd)[kMaxNB][2]) {
+  constexpr int G = (2 * MAXQ + 3) / 4;  // groups of four assignments
   const int H = a.H, ne = w.ne, p0 = w.p0;
   const int bb0 = HS ? 0 : w.dp * a.NB;  // first block of the unit in the staged slice, or in I
   const int g = c.g, tig = c.tig;
-  const int ngroups = (ne + 1) / 2;
-  const int dig_b = g & 1, hb = (g >> 1) & 1, sl_b = g >> 2;
-  const int hc = tig & 1, sl_c = tig >> 1;
+  const int ngroups = (ne + 3) / 4;
+  const int dig_b = g & 1, sl_b = g >> 1;  // this lane's B column: slot sl_b, digit dig_b
   const uint32_t sh = 2 * tig;
   const int row = 16 * c.warp + g;
-  int pb[MAXQ];  // assignment of this lane's B column per group (-1: zero column)
-  const int32_t* hq_ptr[MAXQ];
-  const float* e2p[MAXQ];
+  int pb[G];                // assignment of this lane's B column per group (-1: zero column)
+  const int32_t* hq_ptr[G]; // per-16 sums of the assignment in slot tig
+  const float* e2p[G];
 #pragma unroll
-  for (int q = 0; q < MAXQ; ++q) {
-    const int tb = 2 * q + sl_b, tc = 2 * q + sl_c;
+  for (int q = 0; q < G; ++q) {
+    const int tb = 4 * q + sl_b, tc = 4 * q + tig;
     pb[q] = (q < ngroups && tb < ne) ? p0 + tb : -1;
     const bool cv = q < ngroups && tc < ne;
-    hq_ptr[q] = c.hq + (p0 + (cv ? tc : 0)) * c.hqp + bb0 * 16 + hc;
+    hq_ptr[q] = c.hq + (p0 + (cv ? tc : 0)) * c.hqp + bb0 * 16;
     e2p[q] = cv ? c.hsc + (p0 + tc) * c.hsp + bb0 : nullptr;
   }
-  float facc[MAXQ][2];
+  float facc[G][2];
 #pragma unroll
-  for (int q = 0; q < MAXQ; ++q) facc[q][0] = facc[q][1] = 0.f;
+  for (int q = 0; q < G; ++q) facc[q][0] = facc[q][1] = 0.f;
   const uint32_t qoff = static_cast<uint32_t>(row) * 64;
   const uint32_t qsw = static_cast<uint32_t>((g >> 1) & 3);
 #pragma unroll 1
   for (int j = 0; j < a.NB; ++j) {
-    int acc[4];
-    int iA[MAXQ][2], iM[MAXQ][2];
+    int acc[G][4], iM[G][2];
 #pragma unroll
-    for (int q = 0; q < MAXQ; ++q) iA[q][0] = iA[q][1] = iM[q][0] = iM[q][1] = 0;
+    for (int q = 0; q < G; ++q) {
+      acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0;
+      iM[q][0] = iM[q][1] = 0;
+    }
     if (!mbar_wait_bounded(&c.full[rp.s], rp.ph, a.err, ERR_TIMEOUT)) return false;
     const int s = rp.s;
     rp.next(c.S);
     const uint8_t* st = c.ring + s * kDnStage;
-    const uint8_t* sA = st + kDnQBytes + row * 16;
-    const uint8_t* sB = sA + 8 * 16;
+    const uint8_t* sA = st + kDnQBytes + row * 16;  // scale bytes (sc | m << 4) of the 16 sub-blocks, row g
+    const uint8_t* sB = sA + 8 * 16;                // row g + 8
     const int blk = bb0 + j;
 #pragma unroll 1
     for (int cc = 0; cc < 4; ++cc) {  // logical 16-byte chunk cc of the q bytes: sub-blocks 4cc .. 4cc + 3
       const uint4 qa = lds128(st + qoff + 16 * (cc ^ qsw));
       const uint4 qb = lds128(st + qoff + 8 * 64 + 16 * (cc ^ qsw));
+      const uint32_t wa = *reinterpret_cast<const uint32_t*>(sA + 4 * cc);
+      const uint32_t wb = *reinterpret_cast<const uint32_t*>(sB + 4 * cc);
       uint32_t af[2][4];
-      af[0][0] = q2k_quad(qa.x, sh); af[0][1] = q2k_quad(qb.x, sh);
-      af[0][2] = q2k_quad(qa.y, sh); af[0][3] = q2k_quad(qb.y, sh);
-      af[1][0] = q2k_quad(qa.z, sh); af[1][1] = q2k_quad(qb.z, sh);
-      af[1][2] = q2k_quad(qa.w, sh); af[1][3] = q2k_quad(qb.w, sh);
+      af[0][0] = q2k_quad(qa.x, sh) * (wa & 15u);
+      af[0][1] = q2k_quad(qb.x, sh) * (wb & 15u);
+      af[0][2] = q2k_quad(qa.y, sh) * ((wa >> 8) & 15u);
+      af[0][3] = q2k_quad(qb.y, sh) * ((wb >> 8) & 15u);
+      af[1][0] = q2k_quad(qa.z, sh) * ((wa >> 16) & 15u);
+      af[1][1] = q2k_quad(qb.z, sh) * ((wb >> 16) & 15u);
+      af[1][2] = q2k_quad(qa.w, sh) * ((wa >> 24) & 15u);
+      af[1][3] = q2k_quad(qb.w, sh) * ((wb >> 24) & 15u);
+      const int ma[4] = {static_cast<int>((wa >> 4) & 15u), static_cast<int>((wa >> 12) & 15u),
+                         static_cast<int>((wa >> 20) & 15u), static_cast<int>(wa >> 28)};
+      const int mb[4] = {static_cast<int>((wb >> 4) & 15u), static_cast<int>((wb >> 12) & 15u),
+                         static_cast<int>((wb >> 20) & 15u), static_cast<int>(wb >> 28)};
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int pr = 2 * cc + u;
-        // this thread's columns: sub-block 2*pr + hc of token 2q + sl_c
-        const int sub = 2 * pr + hc;
-        const uint32_t scA = sA[sub], scB = sB[sub];
+      for (int q = 0; q < G; ++q) {
+        if (q >= ngroups) break;
+        const int4 hv = *reinterpret_cast<const int4*>(hq_ptr[q] + j * 16 + 4 * cc);
+        iM[q][0] += ma[0] * hv.x + ma[1] * hv.y + ma[2] * hv.z + ma[3] * hv.w;
+        iM[q][1] += mb[0] * hv.x + mb[1] * hv.y + mb[2] * hv.z + mb[3] * hv.w;
 #pragma unroll
-        for (int q = 0; q < MAXQ; ++q) {
-          if (q >= ngroups) break;
+        for (int u = 0; u < 2; ++u) {
           uint32_t b0 = 0u, b1 = 0u;
-          if (pb[q] >= 0) {  // bit pair tig of sub-block 2pr + hb: bytes 4 tig .. 4 tig + 3 (elements tig + 4i)
-            const int8_t* hp = c.hd + h_off(c.hI, pb[q], dig_b, blk * 256 + (2 * pr + hb) * 16 + tig);
-            const uint32_t v = *reinterpret_cast<const uint32_t*>(hp);
-            if (hb == 0) b0 = v;
-            else b1 = v;
+          if (pb[q] >= 0) {  // bit pair tig of sub-blocks 4cc + 2u and 4cc + 2u + 1 (elements tig + 4i)
+            const int e0 = blk * 256 + (4 * cc + 2 * u) * 16 + tig;
+            b0 = *reinterpret_cast<const uint32_t*>(c.hd + h_off(c.hI, pb[q], dig_b, e0));
+            b1 = *reinterpret_cast<const uint32_t*>(c.hd + h_off(c.hI, pb[q], dig_b, e0 + 16));
           }
-          mma_u8s8_zero(acc, af[u][0], af[u][1], af[u][2], af[u][3], b0, b1);
-          const int hqv = hq_ptr[q][j * 16 + 2 * pr];
-          iA[q][0] += (acc[0] * 128 + acc[1]) * static_cast<int>(scA & 15u);
-          iA[q][1] += (acc[2] * 128 + acc[3]) * static_cast<int>(scB & 15u);
-          iM[q][0] += static_cast<int>(scA >> 4) * hqv;
-          iM[q][1] += static_cast<int>(scB >> 4) * hqv;
+          mma_u8s8(acc[q], af[u][0], af[u][1], af[u][2], af[u][3], b0, b1);
         }
       }
     }
@@ -1064,24 +1075,20 @@ __device__ __forceinline__ bool dn_unit_multi(const DnTmaArgs& a, const DnCtx& c
     if (c.lane == 0) mbar_arrive(&c.empty[s]);
     const uint32_t dA = j ? dd[1][0] : dd[0][0], dB = j ? dd[1][1] : dd[0][1];
 #pragma unroll
-    for (int q = 0; q < MAXQ; ++q) {
+    for (int q = 0; q < G; ++q) {
       const float e2 = e2p[q] ? e2p[q][j] : 0.f;
-      facc[q][0] += dn_block(dA, e2, iA[q][0], iM[q][0]);
-      facc[q][1] += dn_block(dB, e2, iA[q][1], iM[q][1]);
+      facc[q][0] += dn_block(dA, e2, acc[q][0] * 128 + acc[q][1], iM[q][0]);
+      facc[q][1] += dn_block(dB, e2, acc[q][2] * 128 + acc[q][3], iM[q][1]);
     }
   }
 #pragma unroll
-  for (int q = 0; q < MAXQ; ++q) {
-    if (q >= ngroups) break;
-    float f0 = facc[q][0], f1 = facc[q][1];
-    f0 += __shfl_xor_sync(0xffffffffu, f0, 1);
-    f1 += __shfl_xor_sync(0xffffffffu, f1, 1);
-    const int t = 2 * q + sl_c;
-    if (hc == 0 && t < ne) {
+  for (int q = 0; q < G; ++q) {
+    const int t = 4 * q + tig;
+    if (q < ngroups && t < ne) {
       const size_t o = (static_cast<size_t>(p0 + t) * a.DP + w.dp) * H + w.rb * kBoxRows + row;
       if (index_ok(o + 8, a.opart_n)) {
-        a.opart[o] = f0;
-        a.opart[o + 8] = f1;
+        a.opart[o] = facc[q][0];
+        a.opart[o + 8] = facc[q][1];
       }
     }
   }
