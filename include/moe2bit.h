@@ -29,10 +29,10 @@
  *     and never synchronises (moe_read_status, a host query, is the one
  *     exception). Work is ordered on `stream`: it starts after the
  *     work already enqueued there and finishes before anything enqueued later.
- *     moe_layer_forward may run part of it on a side stream that it forks from
- *     `stream` and joins back with events (created once per device and caller
- *     stream, kept for the life of the process); this is safe inside CUDA graph
- *     capture.
+ *     The whole-layer calls (moe_layer_forward and its variants) may run part
+ *     of it on a side stream that they fork from `stream` and join back with
+ *     events (created once per device and caller stream, kept for the life of
+ *     the process); this is safe inside CUDA graph capture.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *   - Argument and shape errors are detected on the host before anything is
  *     enqueued and are returned as a status; nothing is launched in that case.
